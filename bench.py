@@ -1,0 +1,595 @@
+#!/usr/bin/env python
+"""Benchmark of the Dual-Flow decode step on B200.
+
+One step = one Dual-Flow decoder layer at one generated position for a batch
+of sequences, both flows: RMSNorm, grouped QKV projection (both flows' rows,
+one tcgen05 GEMM), primary-only KV append, dual shared-KV decode attention
+(split + combine), grouped W_o projection with residual, RMSNorm, grouped
+gate/up projection with fused SwiGLU + b coupling, grouped down projection
+with residual + c coupling. Default workload: d_model 4096, 32 query heads
+per flow on 8 KV heads, head_dim 128, SwiGLU width 14336, 64 sequences per
+flow (M = 128 rows), cache 4096 tokens + the appended one, bf16 weights
+~ N(0, 0.02), synthetic seeded data. Metric: decode tokens/s (one token per
+sequence per step, per layer) and the KV-read GB/s of the attention kernel.
+
+--impl reference times the fp64 CPU oracle on the machine's host cores on a
+bounded sample of the same workload (the reference arm for this method has no
+upstream code to run).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+sequences with its own cache and weight replica (weak scaling; sequences are
+independent, so there is no data-path collective); the timed region is
+bracketed by barriers and the slowest rank's time is reported.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dual-flow decode tokens/s and KV-read GB/s (% of B200 HBM peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+ATTN_SRC = os.path.join(ROOT, "dual_flow_transformer_b200", "csrc", "decode_attn.cu")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["layer", "mha", "gqa", "long", "tiny"], default="layer")
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0,
+                    help="target seconds of oracle work for the CPU baseline sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_from_profile(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when there is none or the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "decode_attn_%s.md" % workload)
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != sha:
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.strip().split(",") for r in self.file.read().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (IndexError, ValueError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device="cuda"):
+    """Slowest rank's value (timing plumbing, not a data-path collective)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base, rank):
+    """Weak scaling: every rank decodes its own batch of sequences."""
+    return base + 1000 * rank
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def attn_algorithmic_bytes(B, Hq, Hkv, D, seqlens_sum, esize, dual=True):
+    """Per decode-attention launch: K and V read once + Q1 (+ Q2raw, a) + O1 (+ O2)."""
+    kv = seqlens_sum * Hkv * D * 2 * esize
+    q = B * Hq * D * esize * (2 if dual else 1)
+    a = Hq * D * esize if dual else 0
+    o = B * Hq * D * esize * (2 if dual else 1)
+    return kv + q + a + o
+
+
+class LayerRun:
+    """The full layer step of the 'layer' workload on this GPU."""
+
+    def __init__(self, args, dev, seed):
+        import torch
+        from dual_flow_transformer_b200 import synth
+        from dual_flow_transformer_b200.layer import DualFlowLayer
+        w = synth.WORKLOADS["layer"]
+        self.w = w
+        self.host = synth.make_layer_inputs(w, seed=seed)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.host.items()}
+        self.d = d
+        W = {k: d[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
+        self.layer = DualFlowLayer(W, w.Hq, w.Hkv, w.D, w.F, w.B, w.cache_len + 1, device=dev,
+                                   num_splits=args.num_splits)
+        self.X = torch.cat([d["x1"], d["x2"]]).contiguous()
+        self.seqlens = (d["positions"] + 1).to(torch.int32)
+        # the step runs as CUDA-graph replays over fixed buffers (X lives in x_in)
+        self.layer.x_in.copy_(self.X)
+        self.layer.capture(self.layer.x_in, d["k_cache"], d["v_cache"], d["block_table"],
+                           d["positions"], self.seqlens)
+        self.tokens_per_step = w.B
+        self.launches_per_step = self.layer.launches_per_step
+        L = w.cache_len + 1
+        self.attn_bytes = attn_algorithmic_bytes(w.B, w.Hq, w.Hkv, w.D, w.B * L, 2)
+        self.kv_bytes = w.B * L * w.Hkv * w.D * 2 * 2
+        self.units = w.B * w.Hkv * L  # (sequence, KV head, token) units per attention launch
+        self.bytes_per_unit = w.D * 2 * 2
+        self.config = {"workload": "dual-flow decoder layer step: d_model %d, %d/%d heads, "
+                                   "head_dim %d, SwiGLU %d, batch %d per flow (M=%d), cache %d+1"
+                                   % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
+                       "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
+                       "attended": L, "attn_splits": self.layer.splits,
+                       "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
+                             % (self.kv_bytes / 1e9, 436207616 / 1e9)}
+        self.dominant = "dualflow_decode_attn (split + combine kernels)"
+
+    def step(self, timers=None):
+        self.layer.replay(timers)
+
+    def step_host(self, x_host, out_host):
+        d = self.d
+        self.layer.step_host(x_host, out_host, d["k_cache"], d["v_cache"], d["block_table"],
+                             d["positions"], self.seqlens)
+
+    def host_io(self):
+        import torch
+        xh = torch.cat([self.host["x1"], self.host["x2"]]).contiguous().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        return xh, oh
+
+    def check_err(self):
+        return int(self.layer.err.item())
+
+
+class AttnRun:
+    """Decode attention alone on one of the attention workloads."""
+
+    def __init__(self, args, dev, seed, name):
+        import torch
+        from dual_flow_transformer_b200 import api, synth
+        w = synth.WORKLOADS[name]
+        self.w = w
+        self.api = api
+        self.host = synth.make_attn_inputs(w, seed=seed)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.host.items()}
+        self.d = d
+        self.max_len = int(self.host["seqlens"].max())
+        self.ns = args.num_splits
+        nb = api.decode_attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, self.max_len, self.ns)
+        self.ws = torch.empty(max(256, nb), dtype=torch.uint8, device=dev)
+        self.o1 = torch.empty_like(d["q1"])
+        self.o2 = torch.empty_like(d["q1"])
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        S = api.decode_attn_num_splits(w.B, w.Hkv, self.max_len, self.ns)
+        self.tokens_per_step = w.B
+        self.launches_per_step = (1 if S == 1 else 2) + (1 if w.append else 0)
+        esize = 4 if w.dtype == "fp32" else 2
+        tot = int(self.host["seqlens"].sum())
+        self.attn_bytes = attn_algorithmic_bytes(w.B, w.Hq, w.Hkv, w.D, tot, esize)
+        self.kv_bytes = tot * w.Hkv * w.D * 2 * esize
+        self.units = tot * w.Hkv
+        self.bytes_per_unit = w.D * 2 * esize
+        self.config = {"workload": "dual-flow decode attention '%s': batch %d, %d/%d heads, "
+                                   "head_dim %d, %s, lengths %d..%d%s" % (
+                                       name, w.B, w.Hq, w.Hkv, w.D, w.dtype, w.len_lo, w.len_hi,
+                                       ", random block table" if w.random_table else ""),
+                       "attn_splits": S,
+                       "l2": "inputs larger than L2" if self.kv_bytes > 126e6
+                             else "inputs smaller than L2 (not flushed)"}
+        self.dominant = "dualflow_decode_attn (split + combine kernels)"
+        # CUDA graphs: [append] and [attention], replayed every step
+        self._append()
+        self._attn()
+        torch.cuda.synchronize()
+        self.g_append = None
+        if w.append:
+            self.g_append = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_append):
+                self._append()
+        self.g_attn = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_attn):
+            self._attn()
+        torch.cuda.synchronize()
+
+    def _append(self):
+        d = self.d
+        if self.w.append:
+            self.api.kv_append(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
+                               d["block_table"], d["positions"], err_flag=self.err)
+
+    def _attn(self):
+        d = self.d
+        self.api.decode_attn(d["q1"], d["q2raw"], d["a"], d["k_cache"], d["v_cache"],
+                             d["block_table"], d["seqlens"], self.max_len, o1=self.o1, o2=self.o2,
+                             num_splits=self.ns, workspace=self.ws, err_flag=self.err)
+
+    def step(self, timers=None):
+        if self.g_append is not None:
+            self.g_append.replay()
+        if timers is not None:
+            timers["attn"][0].record()
+        self.g_attn.replay()
+        if timers is not None:
+            timers["attn"][1].record()
+
+    def host_io(self):
+        import torch
+        q = torch.stack([self.host["q1"], self.host["q2raw"]]).pin_memory()
+        o = torch.empty_like(q).pin_memory()
+        return q, o
+
+    def step_host(self, q_host, o_host):
+        d = self.d
+        d["q1"].copy_(q_host[0], non_blocking=True)
+        d["q2raw"].copy_(q_host[1], non_blocking=True)
+        self.step()
+        o_host[0].copy_(self.o1, non_blocking=True)
+        o_host[1].copy_(self.o2, non_blocking=True)
+
+    def check_err(self):
+        return int(self.err.item())
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_layer_sample(host, n_seq):
+    """Inputs of the oracle for the first n_seq sequences of a layer workload
+    (input preparation: dtype widening and page selection, no arithmetic)."""
+    import numpy as np
+    import torch
+    sel = list(range(n_seq))
+    tbl = host["block_table"][sel]
+    pages = sorted(set(int(p) for p in tbl.flatten().tolist() if p >= 0))
+    remap = {p: i for i, p in enumerate(pages)}
+    new_tbl = np.array([[remap.get(int(p), -1) for p in row] for row in tbl.tolist()], np.int32)
+    f = lambda t: t.to(torch.float32).numpy().astype(np.float64)
+    kc = host["k_cache"][pages].to(torch.float32).numpy()
+    vc = host["v_cache"][pages].to(torch.float32).numpy()
+    return dict(x1=f(host["x1"][sel]), x2=f(host["x2"][sel]), w_qkv=f(host["w_qkv"]),
+                w_o=f(host["w_o"]), w_gu=f(host["w_gu"]), w_down=f(host["w_down"]),
+                a=f(host["a"]), b=f(host["b"]), c=f(host["c"]), k_cache=kc, v_cache=vc,
+                block_table=new_tbl, positions=host["positions"][sel].numpy(),
+                Hq=host["Hq"], Hkv=host["Hkv"], D=host["D"], F=host["F"])
+
+
+def oracle_attn_sample(host, sel):
+    import numpy as np
+    import torch
+    f = lambda t: t.to(torch.float32).numpy()
+    return dict(q1=f(host["q1"][sel]), q2raw=f(host["q2raw"][sel]), a=f(host["a"]),
+                k_cache=f(host["k_cache"]), v_cache=f(host["v_cache"]),
+                block_table=host["block_table"][sel].numpy(),
+                seqlens=host["seqlens"][sel].numpy())
+
+
+def time_oracle(run, workload, budget_s, max_steps=None):
+    """Time the oracle on a bounded sample. Returns (tokens/s, sample text,
+    seconds, steps). One oracle step = the sample, timed with perf_counter."""
+    import oracle
+    if workload == "layer":
+        n_seq = 1
+        inp = oracle_layer_sample(run.host, n_seq)
+        t0 = time.perf_counter()
+        oracle.layer_step(**inp)
+        t1 = time.perf_counter() - t0
+        steps = max(1, min(int(budget_s / max(t1, 1e-6)), max_steps or 10 ** 9))
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            oracle.layer_step(**inp)
+        el = time.perf_counter() - t0
+        sample = ("%d step(s) of the fp64 oracle layer step on %d of %d sequences (both flows), "
+                  "full weights, cache %d+1; weights pre-widened to fp64 outside the timing"
+                  % (steps, n_seq, run.w.B, run.w.cache_len))
+        return n_seq * steps / el, sample, el, steps
+    B = run.w.B
+    sel, el, k = [], 0.0, 0
+    inp_all = None
+    while k < B and el < budget_s:
+        sel = [k]
+        inp = oracle_attn_sample(run.host, sel)
+        t0 = time.perf_counter()
+        oracle.decode_attn(**inp)
+        el += time.perf_counter() - t0
+        k += 1
+    sample = "fp64 oracle decode attention (both flows) on %d of %d sequences" % (k, B)
+    del inp_all
+    return k / el, sample, el, k
+
+
+# ----------------------------------------------------------------------------- main
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from dual_flow_transformer_b200 import synth  # input generators only
+
+    class Host:
+        pass
+
+    h = Host()
+    if args.workload == "layer":
+        h.w = synth.WORKLOADS["layer"]
+        h.host = synth.make_layer_inputs(h.w)
+    else:
+        h.w = synth.WORKLOADS[args.workload]
+        h.host = synth.make_attn_inputs(h.w)
+    import oracle
+    budget = 150.0
+    if args.workload == "layer":
+        inp = oracle_layer_sample(h.host, 1)
+        t0 = time.perf_counter()
+        oracle.layer_step(**inp)
+        t1 = time.perf_counter() - t0
+        total = args.warmup + args.steps
+        steps = args.steps if t1 * total <= budget else max(1, int(budget / t1) - args.warmup)
+        warm = min(args.warmup, 1)
+        for _ in range(warm):
+            oracle.layer_step(**inp)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            oracle.layer_step(**inp)
+        el = time.perf_counter() - t0
+        tokens = steps
+        sample = ("fp64 oracle layer step on 1 of %d sequences (both flows) per step" % h.w.B)
+    else:
+        inp = oracle_attn_sample(h.host, [0])
+        t0 = time.perf_counter()
+        oracle.decode_attn(**inp)
+        t1 = time.perf_counter() - t0
+        total = args.warmup + args.steps
+        steps = args.steps if t1 * total <= budget else max(1, int(budget / t1) - args.warmup)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            oracle.decode_attn(**oracle_attn_sample(h.host, [i % h.w.B]))
+        el = time.perf_counter() - t0
+        tokens = steps
+        sample = "fp64 oracle decode attention on 1 sequence per step"
+    value = tokens / el
+    cores = _threads_used()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        print("warm-up must be at least 3 steps", file=sys.stderr)
+        return 2
+    import torch
+    world, rank, local = dist_setup(args)
+    if world != args.gpus:
+        print("--gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    seed_base = synth_seed(args.workload)
+    seed = rank_seed(seed_base, rank)
+    run = LayerRun(args, dev, seed) if args.workload == "layer" else \
+        AttnRun(args, dev, seed, args.workload)
+
+    for _ in range(args.warmup):
+        run.step()
+    torch.cuda.synchronize()
+    if run.check_err():
+        print("device error flag %d after warm-up" % run.check_err(), file=sys.stderr)
+        return 3
+
+    # ---------------------------------------------------------------- timed region
+    timers = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    if not args.no_clocks and rank == 0:
+        clocks.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(args.steps):
+        run.step(timers={"attn": timers[i]})
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if (not args.no_clocks and rank == 0) else None
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms, world)
+    attn_ms = sum(s.elapsed_time(e) for s, e in timers) / args.steps
+    attn_ms = max_over_ranks(attn_ms, world)
+    err = run.check_err()
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        xh, oh = run.host_io()
+        for _ in range(3):
+            run.step_host(xh, oh)
+        torch.cuda.synchronize()
+        barrier(world)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(args.steps):
+            run.step_host(xh, oh)
+        e2.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms2 = max_over_ranks(s2.elapsed_time(e2), world)
+        e2e = {"value": world * run.tokens_per_step * args.steps / (ms2 / 1e3),
+               "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+
+    # ---------------------------------------------------------------- CPU baseline (oracle)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, el, steps = time_oracle(run, args.workload, args.cpu_budget_s)
+        cpu = {"value": v, "unit": "tokens/s", "cores": _threads_used(), "kind": "oracle",
+               "sample": sample, "seconds": round(el, 2)}
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+    peak, peak_kind = measured_hbm_peak()
+    achieved = run.attn_bytes / (attn_ms / 1e3) / 1e9
+    value = world * run.tokens_per_step * args.steps / (ms_max / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations/cache, N(0,0.02) weights, N(0,0.1) couplings)",
+        "config": dict(run.config, parallelism="replicas" if world > 1 else "single GPU"),
+        "kv_read_gbs": run.kv_bytes / (attn_ms / 1e3) / 1e9,
+        "kv_frac_of_hbm_peak": run.kv_bytes / (attn_ms / 1e3) / 1e9 / peak,
+        "attn_ms_per_launch": attn_ms,
+        "roofline": {"kernel": run.dominant, "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind + " (STREAM-style copy, MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic_from_profile(args.workload),
+                     "algorithmic_bytes_per_launch": run.attn_bytes,
+                     "units_per_launch": run.units, "bytes_per_unit": run.bytes_per_unit},
+        "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": run.launches_per_step * args.steps,
+        "clocks": clk, "device_error_flag": err,
+    }
+    if clk is None and not args.no_clocks:
+        line["clocks"] = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def synth_seed(workload):
+    from dual_flow_transformer_b200 import synth
+    return synth.WORKLOADS[workload].seed
+
+
+if __name__ == "__main__":
+    sys.exit(main())

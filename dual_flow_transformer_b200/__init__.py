@@ -1,0 +1,16 @@
+"""Dual-Flow Transformer decode step on NVIDIA B200 (sm_100a).
+
+The compute lives in libdualflow.so (C ABI, include/dualflow.h); this
+package is its thin binding plus the layer-step composition.
+"""
+
+from .api import (  # noqa: F401
+    decode_attn,
+    decode_attn_num_splits,
+    decode_attn_workspace_size,
+    grouped_proj,
+    grouped_proj_workspace_size,
+    kv_append,
+    new_proj_workspace,
+    rmsnorm,
+)

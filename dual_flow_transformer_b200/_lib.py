@@ -1,0 +1,86 @@
+"""ctypes loader for libdualflow.so.
+
+Argument marshalling only. There is no fallback: if the shared library is
+missing or fails to load, importing the API raises, because every step of
+the decode path runs in the library's CUDA kernels.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+LIB_PATH = _build.LIB_PATH
+
+DF_OK, DF_ERR_NULL, DF_ERR_SHAPE, DF_ERR_UNSUPPORTED, DF_ERR_WORKSPACE, DF_ERR_ALIGN, DF_ERR_CUDA = range(7)
+DF_FP32, DF_BF16 = 0, 1
+DF_EPI_NONE, DF_EPI_SWIGLU, DF_EPI_RESIDUAL = 0, 1, 2
+DF_DEVERR_SEQLEN, DF_DEVERR_BLOCK, DF_DEVERR_POSITION, DF_DEVERR_TIMEOUT = 1, 2, 4, 8
+
+_c_int, _c_i64, _c_size, _c_float, _vp = (ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                                           ctypes.c_float, ctypes.c_void_p)
+
+# name -> (restype, argtypes); the order matches include/dualflow.h
+SIGNATURES = {
+    "dualflow_abi_version": (_c_int, []),
+    "dualflow_status_string": (ctypes.c_char_p, [_c_int]),
+    "dualflow_decode_attn_num_splits": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dualflow_decode_attn_workspace_size": (_c_size, [_c_int] * 7),
+    "dualflow_decode_attn": (_c_int, [
+        _vp, _vp, _vp, _c_i64,          # q1, q2raw, a, q_stride_b
+        _vp, _vp,                       # k_cache, v_cache
+        _vp, _c_int,                    # block_table, max_blocks_per_seq
+        _vp, _c_int,                    # seqlens, max_seqlen
+        _vp, _vp, _c_i64,               # o1, o2, o_stride_b
+        _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,  # B, Hq, Hkv, D, block_size, num_blocks
+        _c_float, _c_int, _c_int,       # scale, dtype, num_splits
+        _vp, _c_size, _vp, _vp]),       # workspace, bytes, err_flag, stream
+    "dualflow_kv_append": (_c_int, [
+        _vp, _vp, _c_i64, _vp, _vp, _vp, _c_int, _vp,
+        _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+    "dualflow_grouped_proj_workspace_size": (_c_size, [_c_int] * 4),
+    "dualflow_grouped_proj": (_c_int, [
+        _vp, _c_i64, _c_int, _c_int,    # x, ldx, m_primary, m_aux
+        _vp, _c_int, _c_int, _c_int,    # w, N, K, n_aux
+        _vp, _c_i64,                    # y, ldy
+        _c_int, _vp, _vp, _c_i64,       # epilogue, coupling, residual, ldr
+        _vp, _c_size, _vp, _vp]),       # workspace, bytes, err_flag, stream
+    "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
+}
+
+_lib = None
+
+
+class DualflowError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s -> %s" % (fn, status_string(status)))
+
+
+def load(build_if_missing: bool = True):
+    """Load (building first if needed) and return the ctypes handle."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_missing and not _build.up_to_date():
+        _build.build()
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libdualflow.so is not built (%s); run __graft_entry__.build()" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().dualflow_status_string(int(status)).decode()
+
+
+def check(fn_name: str, status: int):
+    if status != DF_OK:
+        raise DualflowError(fn_name, status)

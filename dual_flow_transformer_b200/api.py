@@ -1,0 +1,175 @@
+"""Thin Python binding over libdualflow.so (argument marshalling only).
+
+Tensors are torch CUDA tensors used as plain device buffers; every
+computation runs inside the library's kernels. Outputs and workspaces that
+the caller does not pass are allocated here with torch (device memory is
+plumbing), never computed here.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+
+def _lib():
+    return L.load()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return L.DF_BF16
+    if dt == torch.float32:
+        return L.DF_FP32
+    raise TypeError("unsupported dtype %s (bf16 or fp32)" % dt)
+
+
+def _heads_view_ok(t: torch.Tensor, Hq: int, D: int) -> bool:
+    return t.dim() == 3 and t.shape[1] == Hq and t.shape[2] == D and t.stride(2) == 1 \
+        and t.stride(1) == D
+
+
+# ----------------------------------------------------------------- attention
+
+def decode_attn_num_splits(B, Hkv, max_seqlen, num_splits=0, block_size=64) -> int:
+    return _lib().dualflow_decode_attn_num_splits(B, Hkv, max_seqlen, block_size, num_splits)
+
+
+def decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, num_splits=0, block_size=64) -> int:
+    return _lib().dualflow_decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size,
+                                                      num_splits)
+
+
+def decode_attn(q1, q2raw, a, k_cache, v_cache, block_table, seqlens, max_seqlen, *,
+                o1=None, o2=None, primary_out=True, scale=0.0, num_splits=0, workspace=None,
+                err_flag=None, stream=None):
+    """Dual-flow decode attention; returns (o1, o2).
+
+    q1, q2raw: [B, Hq, D] (heads contiguous; any batch stride, equal for
+    both); a: [Hq, D] or None; caches [num_blocks, Hkv, 64, D]; block_table
+    int32 [B, max_blocks]; seqlens int32 [B]; max_seqlen: host int.
+    primary_out=False makes an auxiliary-only call (o1 not written).
+    """
+    B, Hq, D = q1.shape
+    num_blocks, Hkv, bs, Dk = k_cache.shape
+    if Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("cache shape mismatch")
+    if not _heads_view_ok(q1, Hq, D):
+        raise ValueError("q1 must be [B, Hq, D] with contiguous heads")
+    if q2raw is not None and (not _heads_view_ok(q2raw, Hq, D) or q2raw.stride(0) != q1.stride(0)):
+        raise ValueError("q2raw must match q1's layout")
+    if not (k_cache.is_contiguous() and v_cache.is_contiguous() and block_table.is_contiguous()):
+        raise ValueError("caches and block table must be contiguous")
+    dev = q1.device
+    if primary_out and o1 is None:
+        o1 = torch.empty((B, Hq, D), dtype=q1.dtype, device=dev)
+    if not primary_out:
+        o1 = None
+    if q2raw is not None and o2 is None:
+        o2 = torch.empty((B, Hq, D), dtype=q1.dtype, device=dev)
+    if q2raw is None:
+        o2 = None
+    os_b = (o1 if o1 is not None else o2).stride(0)
+    for o in (o1, o2):
+        if o is not None and (not _heads_view_ok(o, Hq, D) or o.stride(0) != os_b):
+            raise ValueError("outputs must be [B, Hq, D] with contiguous heads and equal strides")
+    need = decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, num_splits, bs)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = _lib().dualflow_decode_attn(
+        _ptr(q1), _ptr(q2raw), _ptr(a), q1.stride(0), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_table), block_table.shape[1], _ptr(seqlens), int(max_seqlen),
+        _ptr(o1), _ptr(o2), os_b, B, Hq, Hkv, D, bs, num_blocks, float(scale),
+        dtype_code(q1.dtype), int(num_splits), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    L.check("dualflow_decode_attn", st)
+    return o1, o2
+
+
+# ----------------------------------------------------------------- append
+
+def kv_append(k_new, v_new, k_cache, v_cache, block_table, positions, *, err_flag=None,
+              stream=None):
+    """Primary-only append of k_new/v_new [B, Hkv, D] at positions[b]."""
+    B, Hkv, D = k_new.shape
+    num_blocks, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or v_new.shape != k_new.shape or v_new.stride() != k_new.stride():
+        raise ValueError("shape mismatch")
+    if k_new.stride(2) != 1 or k_new.stride(1) != D:
+        raise ValueError("k_new must have contiguous heads")
+    st = _lib().dualflow_kv_append(
+        _ptr(k_new), _ptr(v_new), k_new.stride(0), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_table), block_table.shape[1], _ptr(positions), B, Hkv, D, bs, num_blocks,
+        dtype_code(k_new.dtype), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_kv_append", st)
+
+
+# ----------------------------------------------------------------- projection
+
+EPILOGUES = {"none": L.DF_EPI_NONE, "swiglu": L.DF_EPI_SWIGLU, "residual": L.DF_EPI_RESIDUAL}
+
+
+def grouped_proj_workspace_size(M, N, K, epilogue="none") -> int:
+    return _lib().dualflow_grouped_proj_workspace_size(M, N, K, EPILOGUES[epilogue])
+
+
+def new_proj_workspace(M, N, K, epilogue="none", device="cuda"):
+    """Zero-initialised workspace (its tile counters must start at zero)."""
+    return torch.zeros(max(256, grouped_proj_workspace_size(M, N, K, epilogue)), dtype=torch.uint8,
+                       device=device)
+
+
+def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupling=None,
+                 residual=None, workspace=None, err_flag=None, stream=None):
+    """y = epilogue(x w^T) for both flows' rows in one GEMM.
+
+    x: bf16 [M, K] (row stride multiple of 8), rows [0, m_primary) primary,
+    the rest auxiliary; w: bf16 [N, K] contiguous. epilogue "swiglu": w is
+    [W_gate; W_up] and y is [M, N/2]; "residual": y = residual + x w^T.
+    coupling: b (swiglu) or c (residual) vector, bf16, or None.
+    """
+    M, K = x.shape
+    N, K2 = w.shape
+    if K2 != K or x.stride(1) != 1 or not w.is_contiguous():
+        raise ValueError("x [M, K] with unit column stride and w [N, K] contiguous required")
+    epi = EPILOGUES[epilogue]
+    n_out = N // 2 if epi == L.DF_EPI_SWIGLU else N
+    if y is None:
+        y = torch.empty((M, n_out), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        workspace = new_proj_workspace(M, N, K, epilogue, x.device)
+    st = _lib().dualflow_grouped_proj(
+        _ptr(x), x.stride(0), int(m_primary), int(M - m_primary), _ptr(w), N, K,
+        n_out if n_aux is None else int(n_aux), _ptr(y), y.stride(0), epi, _ptr(coupling),
+        _ptr(residual), 0 if residual is None else residual.stride(0), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_grouped_proj", st)
+    return y
+
+
+# ----------------------------------------------------------------- norm
+
+def rmsnorm(x, gain=None, y=None, eps=1e-5, stream=None):
+    rows, cols = x.shape
+    if y is None:
+        y = torch.empty_like(x)
+    st = _lib().dualflow_rmsnorm(_ptr(x), x.stride(0), _ptr(gain), _ptr(y), y.stride(0), rows, cols,
+                                 float(eps), _stream(stream))
+    L.check("dualflow_rmsnorm", st)
+    return y

@@ -1,0 +1,70 @@
+// ABI-wide host code: version, status strings, tensor-map encoding through the
+// driver entry point, device properties.
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "host_util.h"
+
+namespace df {
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess) {
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+}
+}  // namespace
+
+bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint64_t row_pitch_bytes, uint32_t box_rows, uint32_t box_cols) {
+  std::call_once(g_encode_once, load_encode);
+  if (!g_encode) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t elem_strides[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace df
+
+extern "C" int dualflow_abi_version(void) { return 1; }
+
+extern "C" const char* dualflow_status_string(int status) {
+  switch (status) {
+    case DF_OK: return "DF_OK";
+    case DF_ERR_NULL: return "DF_ERR_NULL: a required pointer is NULL";
+    case DF_ERR_SHAPE: return "DF_ERR_SHAPE: sizes inconsistent or out of range";
+    case DF_ERR_UNSUPPORTED: return "DF_ERR_UNSUPPORTED: request not implemented by this build";
+    case DF_ERR_WORKSPACE: return "DF_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    case DF_ERR_ALIGN: return "DF_ERR_ALIGN: pointer or stride misaligned";
+    case DF_ERR_CUDA: return "DF_ERR_CUDA: a CUDA call or kernel launch failed";
+    default: return "unknown dualflow status";
+  }
+}

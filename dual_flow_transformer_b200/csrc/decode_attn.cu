@@ -1,0 +1,762 @@
+// Dual-flow decode attention: asymmetric shared-KV attention of the primary
+// query Q1 and the coupled auxiliary query Q2 = Q2raw + a (.) Q1 over the single
+// primary cache (K1, V1), split over the sequence (flash-decoding), plus the
+// split-combine kernel.
+//
+// Method: "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi
+// Chiave" -- the auxiliary flow attends to the primary flow's keys and values
+// without writing its own, so each KV region can be loaded once for both flows.
+//
+// bf16 kernel design (sm_100a):
+//  * one CTA per (split, KV head g, sequence b); 4 consumer warps + 1 TMA
+//    producer warp; 64-token pages of K and V arrive by TMA (128-byte swizzle)
+//    into a STAGES-deep shared-memory ring guarded by mbarriers;
+//  * each page is read from HBM exactly once and serves all 2*G query rows of
+//    KV head g: rows 0..3 = primary heads, 4..7 = auxiliary heads (bf16 "hi"
+//    part of the fp32 coupled Q2), 12..15 = the auxiliary "lo" part
+//    (bf16(Q2 - hi)), 8..11 = the primary lo part (zero, Q1 is bf16-exact).
+//    The m16n8k16 fragment keeps row r and r+8 in the same thread, so hi + lo
+//    scores add in registers: Q2 enters the scores at ~16 significant bits;
+//  * QK^T and PV run on mma.sync (bf16 in, fp32 accumulate). The softmax
+//    weights P are split the same way (hi in rows r, lo in rows r+8) so PV
+//    also sees ~16-bit weights. Each warp owns 16 tokens of every page and
+//    keeps its own running max / sum per row (online softmax in the exp2
+//    domain, quad shuffles), merged across warps through shared memory;
+//  * every query row's arithmetic is independent of every other row's, and
+//    the split plan depends only on (B, Hkv, max_seqlen), so O1 is
+//    bit-identical whatever the auxiliary inputs are.
+#include <math.h>
+
+#include "common.cuh"
+#include "host_util.h"
+
+namespace df {
+namespace attn {
+
+constexpr int kPage = 64;                 // tokens per page (block_size)
+constexpr int kConsumerWarps = 4;         // each owns 16 tokens of a page
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStagesBf16 = 3;            // pipeline depth of the bf16 kernel
+constexpr int kTargetCtas = 148 * 2 * 8;  // ~8 waves of 2 resident CTAs per SM
+constexpr int kMinChunkPages = 8;         // >= 512 tokens per split
+
+struct Params {
+  const void* q1;
+  const void* q2raw;
+  const void* a;
+  int64_t q_stride_b;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  int max_blocks_per_seq;
+  const int32_t* seqlens;
+  int max_seqlen;
+  void* o1;
+  void* o2;
+  int64_t o_stride_b;
+  int B, Hq, Hkv, G, num_blocks;
+  float scale_log2;  // softmax scale * log2(e)
+  int chunk_pages;   // pages per split
+  int num_splits;
+  float* part_o;     // [B][2Hq][S][D]
+  float* part_ml;    // [B][2Hq][S][2] (running max in log2 units, sum)
+  int32_t* err;
+  int dual;          // auxiliary rows computed
+  int write1;        // store O1
+  int write2;        // store O2
+};
+
+struct Plan {
+  int splits;
+  int chunk_pages;
+};
+
+inline Plan make_plan(int B, int Hkv, int max_seqlen, int block_size, int requested) {
+  const int max_pages = static_cast<int>(ceil_div(max_seqlen, block_size));
+  int s0;
+  if (requested > 0) {
+    s0 = requested < max_pages ? requested : max_pages;
+  } else {
+    const int64_t units = static_cast<int64_t>(B) * Hkv;
+    int64_t want = ceil_div(kTargetCtas, units);
+    int64_t cap = max_pages / kMinChunkPages;
+    if (cap < 1) cap = 1;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    s0 = static_cast<int>(want);
+  }
+  Plan p;
+  p.chunk_pages = static_cast<int>(ceil_div(max_pages, s0));
+  p.splits = static_cast<int>(ceil_div(max_pages, p.chunk_pages));
+  return p;
+}
+
+// max that propagates NaN (fmaxf drops it), so NaN inputs give NaN outputs.
+__device__ __forceinline__ float max_nan(float a, float b) { return (a != a || a > b) ? a : b; }
+
+// Normalise; an empty row (no attended token) gives 0, a NaN row stays NaN.
+__device__ __forceinline__ float safe_div(float o, float l) { return (l == 0.f) ? 0.f : o / l; }
+
+__device__ __forceinline__ int attended_len(const Params& p, int b) {
+  const int L = p.seqlens[b];
+  if (L < 1) return 0;
+  return L < p.max_seqlen ? L : p.max_seqlen;
+}
+
+__device__ __forceinline__ void flag_len(const Params& p, int b) {
+  const int L = p.seqlens[b];
+  if (L < 1 || L > p.max_seqlen) set_err(p.err, DF_DEVERR_SEQLEN);
+}
+
+// Byte address of 16-byte chunk `ch` of token row `tok` inside a TMA-written
+// [64 tokens][D] bf16 tile stored as D/64 column halves of [64][128 B] with the
+// 128-byte swizzle (chunk index XOR row index within each 8-row group).
+__device__ __forceinline__ uint32_t swz(uint32_t base, int tok, int ch) {
+  return base + (ch >> 3) * (kPage * 128) + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4);
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_f(const T* p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+template <typename T>
+__device__ __forceinline__ void st_f(T* p, float v);
+template <>
+__device__ __forceinline__ void st_f<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void st_f<__nv_bfloat16>(__nv_bfloat16* p, float v) {
+  *p = __float2bfloat16_rn(v);
+}
+
+// Write zeros for every requested output row of (b, g): used when a sequence
+// has no attended token (seqlens[b] < 1) and there is a single split.
+template <typename T, int D>
+__device__ void write_zero_rows(const Params& p, int b, int g, int tid, int nthreads) {
+  for (int idx = tid; idx < 2 * p.G * D; idx += nthreads) {
+    const int r = idx / D, d = idx % D;
+    const int flow = r / p.G, h = g * p.G + (r % p.G);
+    if (flow == 0 && p.write1)
+      st_f(static_cast<T*>(p.o1) + b * p.o_stride_b + h * D + d, 0.f);
+    if (flow == 1 && p.write2)
+      st_f(static_cast<T*>(p.o2) + b * p.o_stride_b + h * D + d, 0.f);
+  }
+}
+
+// ------------------------------------------------------------------ bf16 split
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2)
+    split_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const Params p) {
+  constexpr int kTileBytes = kPage * D * 2;  // one K (or V) page
+  constexpr int kStageBytes = 2 * kTileBytes;
+  constexpr int KS = D / 16;  // k-steps of Q K^T
+  constexpr int NT = D / 8;   // n-tiles of P V
+  constexpr float kNegInf = -INFINITY;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
+  uint64_t* empty = full + STAGES;
+  int* stage_valid = reinterpret_cast<int*>(empty + STAGES);
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (split == 0 && g == 0 && threadIdx.x == 0) flag_len(p, b);
+  const int L = attended_len(p, b);
+  const int npages = (L + kPage - 1) / kPage;
+  const int pg0 = split * p.chunk_pages;
+  const int pg1 = min(npages, pg0 + p.chunk_pages);
+  if (pg0 >= pg1) {
+    if (p.num_splits == 1)
+      write_zero_rows<__nv_bfloat16, D>(p, b, g, threadIdx.x, blockDim.x);
+    return;
+  }
+  const int ntiles = pg1 - pg0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------------ producer warp
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      const uint64_t policy = l2_policy_evict_first();
+      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[st], ((i / STAGES) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        const int page = tbl[pg0 + i];
+        if (page < 0 || page >= p.num_blocks) {
+          set_err(p.err, DF_DEVERR_BLOCK);
+          stage_valid[st] = 0;
+          mbar_arrive(&full[st]);
+          ++issued;
+          continue;
+        }
+        stage_valid[st] = 1;
+        mbar_arrive_expect_tx(&full[st], kStageBytes);
+        const int row = (page * p.Hkv + g) * kPage;
+        uint8_t* sK = smem + st * kStageBytes;
+        uint8_t* sV = sK + kTileBytes;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d_hint(sK + h * kPage * 128, &tmK, &full[st], h * 64, row, policy);
+          tma_load_2d_hint(sV + h * kPage * 128, &tmV, &full[st], h * 64, row, policy);
+        }
+        ++issued;
+      }
+      // Do not leave the CTA with copies in flight: wait (bounded) for the last
+      // issued pages, whose completion the consumers may not have observed.
+      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumer warps
+  const int gid = lane >> 2, tq = lane & 3;
+  const int G = p.G;
+
+  // Q fragments (A operand of Q K^T): rows gid and gid + 8 of the 16-row tile.
+  uint32_t qa[KS][4];
+  {
+    const __nv_bfloat16* q1 = static_cast<const __nv_bfloat16*>(p.q1) + b * p.q_stride_b;
+    const __nv_bfloat16* q2 = static_cast<const __nv_bfloat16*>(p.q2raw) + b * p.q_stride_b;
+    const __nv_bfloat16* av = static_cast<const __nv_bfloat16*>(p.a);
+    const int j = gid & 3;
+    const bool aux = gid >= 4;
+    const bool valid = (j < G) && (!aux || p.dual);
+    const int h = g * G + j;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int d0 = ks * 16 + half * 8 + 2 * tq;
+        __nv_bfloat16 lo_row[2], hi_row[2];  // rows gid (hi part) and gid + 8 (lo part)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          __nv_bfloat16 top = __float2bfloat16_rn(0.f), bot = __float2bfloat16_rn(0.f);
+          if (valid) {
+            const __nv_bfloat16 x1 = q1[h * D + d0 + e];
+            if (!aux) {
+              top = x1;
+            } else {
+              float q = __bfloat162float(q2[h * D + d0 + e]);
+              if (av != nullptr) q = fmaf(__bfloat162float(av[h * D + d0 + e]), __bfloat162float(x1), q);
+              split_bf16(q, top, bot);
+            }
+          }
+          hi_row[e] = top;
+          lo_row[e] = bot;
+        }
+        qa[ks][half * 2 + 0] = pack_bf16x2(hi_row[0], hi_row[1]);
+        qa[ks][half * 2 + 1] = pack_bf16x2(lo_row[0], lo_row[1]);
+      }
+    }
+  }
+
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float m_run = kNegInf, l_run = 0.f;
+  const int tok0 = warp * 16;
+  bool timed_out = false;
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i % STAGES;
+    if (!mbar_wait_warp(&full[st], (i / STAGES) & 1)) {
+      timed_out = true;
+      break;
+    }
+    bool zeroed = false;
+    const int nvalid = L - (pg0 + i) * kPage - tok0;  // valid tokens among this warp's 16
+    if (stage_valid[st] && nvalid > 0) {
+      const uint32_t kb = smem_u32(smem + st * kStageBytes);
+      const uint32_t vb = kb + kTileBytes;
+
+      // S = Q K^T for the warp's 16 tokens (two n-tiles of 8).
+      float sc[2][4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+      {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tok = tok0 + (mi >> 1) * 8 + r;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(swz(kb, tok, 2 * ks + (mi & 1)), b0, b1, b2, b3);
+          mma_bf16_16816(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+          mma_bf16_16816(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+        }
+      }
+      // Scores of row gid: hi rows + lo rows, scaled to log2 units, masked.
+      float sv[2][2];
+      float mx = kNegInf;
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = n * 8 + 2 * tq + e;
+          const float v = (sc[n][e] + sc[n][e + 2]) * p.scale_log2;
+          sv[n][e] = (t < nvalid) ? v : kNegInf;
+          mx = max_nan(mx, sv[n][e]);
+        }
+      mx = max_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = max_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = max_nan(m_run, mx);
+      const float m_use = (m_new == kNegInf) ? 0.f : m_new;
+      const float alpha = exp2f(m_run - m_use);
+      float pv[2][2], psum = 0.f;
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          pv[n][e] = exp2f(sv[n][e] - m_use);
+          psum += pv[n][e];
+        }
+      l_run = l_run * alpha + psum;
+      m_run = m_new;
+      if (!__all_sync(0xffffffffu, alpha == 1.f)) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          acc[n][0] *= alpha;
+          acc[n][1] *= alpha;
+          acc[n][2] *= alpha;
+          acc[n][3] *= alpha;
+        }
+      }
+      // P as the A operand of P V: hi parts in row gid, lo parts in row gid + 8.
+      __nv_bfloat16 ph[2][2], pl[2][2];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) split_bf16(pv[n][e], ph[n][e], pl[n][e]);
+      const uint32_t pa0 = pack_bf16x2(ph[0][0], ph[0][1]);
+      const uint32_t pa1 = pack_bf16x2(pl[0][0], pl[0][1]);
+      const uint32_t pa2 = pack_bf16x2(ph[1][0], ph[1][1]);
+      const uint32_t pa3 = pack_bf16x2(pl[1][0], pl[1][1]);
+
+      // Rows past the sequence end hold stale bytes (possibly NaN patterns);
+      // a zero weight times NaN would still be NaN, so clear those V rows.
+      if (nvalid < 16) {
+        uint8_t* vrow = smem + st * kStageBytes + kTileBytes;
+        for (int idx = lane; idx < (16 - nvalid) * (D / 8); idx += 32) {
+          const int tok = tok0 + nvalid + idx / (D / 8);
+          const int ch = idx % (D / 8);
+          *reinterpret_cast<uint4*>(vrow + (ch >> 3) * (kPage * 128) + tok * 128 + (ch & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        zeroed = true;
+        __syncwarp();
+      }
+      {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tok = tok0 + (mi & 1) * 8 + r;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(swz(vb, tok, 2 * np + (mi >> 1)), v0, v1, v2, v3);
+          mma_bf16_16816(acc[2 * np], pa0, pa1, pa2, pa3, v0, v1);
+          mma_bf16_16816(acc[2 * np + 1], pa0, pa1, pa2, pa3, v2, v3);
+        }
+      }
+    }
+    // Release the stage to the producer. Generic-proxy writes (the zeroing)
+    // must be ordered before the next asynchronous (TMA) write of the buffer.
+    if (zeroed) fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // All consumer warps are done with the ring before it is reused as scratch.
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  if (__any_sync(0xffffffffu, timed_out)) timed_out = true;
+  __shared__ int any_timeout;
+  if (threadIdx.x == 0) any_timeout = 0;
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  if (timed_out && lane == 0) {
+    any_timeout = 1;
+    set_err(p.err, DF_DEVERR_TIMEOUT);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  if (any_timeout) return;
+
+  // Merge the 4 warps' (max, sum, O) per logical row through shared memory.
+  float* ms = reinterpret_cast<float*>(smem);      // [4 warps][8 rows]
+  float* ls = ms + kConsumerWarps * 8;             // [4][8]
+  float* os = ls + kConsumerWarps * 8;             // [4][8][D]
+  float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+  if (tq == 0) {
+    ms[warp * 8 + gid] = m_run;
+    ls[warp * 8 + gid] = l_tot;
+  }
+  float* orow = os + (warp * 8 + gid) * D;
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    *reinterpret_cast<float2*>(orow + n * 8 + 2 * tq) =
+        make_float2(acc[n][0] + acc[n][2], acc[n][1] + acc[n][3]);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+
+  for (int idx = threadIdx.x; idx < 8 * D; idx += kConsumerWarps * 32) {
+    const int row = idx / D, d = idx % D;
+    const int flow = row >> 2, j = row & 3;
+    if (j >= G || (flow == 1 && !p.dual)) continue;
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = max_nan(M, ms[w * 8 + row]);
+    float Ls = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = ms[w * 8 + row];
+      const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
+      Ls += wt * ls[w * 8 + row];
+      O += wt * os[(w * 8 + row) * D + d];
+    }
+    const int h = g * G + j;
+    if (p.num_splits == 1) {
+      const float out = safe_div(O, Ls);
+      if (flow == 0 && p.write1)
+        static_cast<__nv_bfloat16*>(p.o1)[b * p.o_stride_b + h * D + d] = __float2bfloat16_rn(out);
+      if (flow == 1 && p.write2)
+        static_cast<__nv_bfloat16*>(p.o2)[b * p.o_stride_b + h * D + d] = __float2bfloat16_rn(out);
+    } else {
+      const int64_t slot =
+          (static_cast<int64_t>(b) * 2 * p.Hq + flow * p.Hq + h) * p.num_splits + split;
+      p.part_o[slot * D + d] = O;
+      if (d == 0) {
+        p.part_ml[slot * 2] = M;
+        p.part_ml[slot * 2 + 1] = Ls;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ fp32 split
+// Plain CUDA-core kernel for fp32 inputs (exact fp32 arithmetic throughout).
+
+template <int D>
+__global__ void __launch_bounds__(128) split_f32_kernel(const Params p) {
+  constexpr float kNegInf = -INFINITY;
+  extern __shared__ float fsm[];
+  float* sq = fsm;             // [8][D] query rows (primary 0..G-1, aux G..2G-1)
+  float* sk = sq + 8 * D;      // [64][D]
+  float* sv = sk + kPage * D;  // [64][D]
+  float* sp = sv + kPage * D;  // [8][64] scores / weights
+  float* sm_ = sp + 8 * kPage; // [8] running max
+  float* sl = sm_ + 8;         // [8] running sum
+  float* sa = sl + 8;          // [8] rescale factor
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int t = threadIdx.x;
+  if (split == 0 && g == 0 && t == 0) flag_len(p, b);
+  const int L = attended_len(p, b);
+  const int npages = (L + kPage - 1) / kPage;
+  const int pg0 = split * p.chunk_pages;
+  const int pg1 = min(npages, pg0 + p.chunk_pages);
+  if (pg0 >= pg1) {
+    if (p.num_splits == 1) write_zero_rows<float, D>(p, b, g, t, blockDim.x);
+    return;
+  }
+  const int G = p.G;
+  const int R = p.dual ? 2 * G : G;
+  const float* q1 = static_cast<const float*>(p.q1) + b * p.q_stride_b;
+  const float* q2 = static_cast<const float*>(p.q2raw) + b * p.q_stride_b;
+  const float* av = static_cast<const float*>(p.a);
+  for (int idx = t; idx < R * D; idx += 128) {
+    const int r = idx / D, d = idx % D;
+    const int h = g * G + (r % G);
+    const float x1 = q1[h * D + d];
+    float q = x1;
+    if (r >= G) {
+      q = q2[h * D + d];
+      if (av) q = fmaf(av[h * D + d], x1, q);
+    }
+    sq[r * D + d] = q;
+  }
+  if (t < 8) {
+    sm_[t] = kNegInf;
+    sl[t] = 0.f;
+  }
+  constexpr int kPer = 8 * D / 128;
+  float o[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) o[k] = 0.f;
+
+  const float* kc = static_cast<const float*>(p.k_cache);
+  const float* vc = static_cast<const float*>(p.v_cache);
+  const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+  for (int pg = pg0; pg < pg1; ++pg) {
+    const int page = tbl[pg];
+    if (page < 0 || page >= p.num_blocks) {
+      if (t == 0) set_err(p.err, DF_DEVERR_BLOCK);
+      continue;
+    }
+    const int nval = min(kPage, L - pg * kPage);
+    __syncthreads();
+    const int64_t base = (static_cast<int64_t>(page) * p.Hkv + g) * kPage * D;
+    for (int idx = t; idx < nval * D; idx += 128) {
+      sk[idx] = kc[base + idx];
+      sv[idx] = vc[base + idx];
+    }
+    __syncthreads();
+    for (int idx = t; idx < R * nval; idx += 128) {
+      const int r = idx / nval, tok = idx % nval;
+      float s = 0.f;
+      for (int d = 0; d < D; ++d) s = fmaf(sq[r * D + d], sk[tok * D + d], s);
+      sp[r * kPage + tok] = s * p.scale_log2;
+    }
+    __syncthreads();
+    if (t < R) {
+      float mx = kNegInf;
+      for (int tok = 0; tok < nval; ++tok) mx = max_nan(mx, sp[t * kPage + tok]);
+      const float m_new = max_nan(sm_[t], mx);
+      const float m_use = (m_new == kNegInf) ? 0.f : m_new;
+      const float al = exp2f(sm_[t] - m_use);
+      float sum = 0.f;
+      for (int tok = 0; tok < nval; ++tok) {
+        const float e = exp2f(sp[t * kPage + tok] - m_use);
+        sp[t * kPage + tok] = e;
+        sum += e;
+      }
+      sl[t] = sl[t] * al + sum;
+      sm_[t] = m_new;
+      sa[t] = al;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int idx = t + 128 * k;
+      if (idx < R * D) {
+        const int r = idx / D, d = idx % D;
+        float acc = o[k] * sa[r];
+        for (int tok = 0; tok < nval; ++tok) acc = fmaf(sp[r * kPage + tok], sv[tok * D + d], acc);
+        o[k] = acc;
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = t + 128 * k;
+    if (idx >= R * D) continue;
+    const int r = idx / D, d = idx % D;
+    const int flow = r / G, h = g * G + (r % G);
+    const float M = sm_[r], Ls = sl[r];
+    if (p.num_splits == 1) {
+      const float out = safe_div(o[k], Ls);
+      if (flow == 0 && p.write1) static_cast<float*>(p.o1)[b * p.o_stride_b + h * D + d] = out;
+      if (flow == 1 && p.write2) static_cast<float*>(p.o2)[b * p.o_stride_b + h * D + d] = out;
+    } else {
+      const int64_t slot =
+          (static_cast<int64_t>(b) * 2 * p.Hq + flow * p.Hq + h) * p.num_splits + split;
+      p.part_o[slot * D + d] = o[k];
+      if (d == 0) {
+        p.part_ml[slot * 2] = M;
+        p.part_ml[slot * 2 + 1] = Ls;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ combine
+// O = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s, in split
+// order (deterministic), then one rounding to the output dtype.
+
+template <typename T, int D>
+__global__ void __launch_bounds__(D) combine_kernel(const Params p) {
+  constexpr float kNegInf = -INFINITY;
+  const int row = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int flow = row / p.Hq, h = row % p.Hq;
+  if ((flow == 0 && !p.write1) || (flow == 1 && !p.write2)) return;
+  const int L = attended_len(p, b);
+  const int npages = (L + kPage - 1) / kPage;
+  const int nsplit = (npages + p.chunk_pages - 1) / p.chunk_pages;
+  const int64_t slot0 = (static_cast<int64_t>(b) * 2 * p.Hq + row) * p.num_splits;
+  float M = kNegInf;
+  for (int s = 0; s < nsplit; ++s) M = max_nan(M, p.part_ml[(slot0 + s) * 2]);
+  float Ls = 0.f, O = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float ms = p.part_ml[(slot0 + s) * 2];
+    const float wt = (ms == kNegInf) ? 0.f : exp2f(ms - M);
+    Ls += wt * p.part_ml[(slot0 + s) * 2 + 1];
+    O += wt * p.part_o[(slot0 + s) * D + d];
+  }
+  const float out = safe_div(O, Ls);
+  T* dst = static_cast<T*>(flow == 0 ? p.o1 : p.o2);
+  st_f(dst + b * p.o_stride_b + h * D + d, out);
+}
+
+// ------------------------------------------------------------------ launch
+
+template <int D>
+size_t bf16_smem_bytes() {
+  return 1024 + static_cast<size_t>(kStagesBf16) * 2 * kPage * D * 2 + 2 * kStagesBf16 * 8 +
+         kStagesBf16 * 4 + 64;
+}
+
+template <int D>
+size_t f32_smem_bytes() {
+  return sizeof(float) * (8 * D + 2 * kPage * D + 8 * kPage + 24);
+}
+
+template <int D>
+cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                   cudaStream_t stream) {
+  const dim3 grid(p.num_splits, p.Hkv, p.B);
+  if (dtype == DF_BF16) {
+    const size_t smem = bf16_smem_bytes<D>();
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(split_bf16_kernel<D, kStagesBf16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    split_bf16_kernel<D, kStagesBf16><<<grid, kThreads, smem, stream>>>(*tmK, *tmV, p);
+    if (p.num_splits > 1)
+      combine_kernel<__nv_bfloat16, D><<<dim3(2 * p.Hq, p.B), D, 0, stream>>>(p);
+  } else {
+    const size_t smem = f32_smem_bytes<D>();
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(split_f32_kernel<D>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    split_f32_kernel<D><<<grid, 128, smem, stream>>>(p);
+    if (p.num_splits > 1) combine_kernel<float, D><<<dim3(2 * p.Hq, p.B), D, 0, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace attn
+}  // namespace df
+
+using df::attn::make_plan;
+using df::attn::Plan;
+
+extern "C" int dualflow_decode_attn_num_splits(int B, int Hkv, int max_seqlen, int block_size,
+                                               int num_splits) {
+  if (B < 1 || Hkv < 1 || max_seqlen < 1 || block_size < 1 || num_splits < 0) return 0;
+  return make_plan(B, Hkv, max_seqlen, block_size, num_splits).splits;
+}
+
+extern "C" size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, int D,
+                                                      int max_seqlen, int block_size,
+                                                      int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || max_seqlen < 1 || block_size < 1 || num_splits < 0)
+    return 0;
+  const Plan pl = make_plan(B, Hkv, max_seqlen, block_size, num_splits);
+  if (pl.splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * 2 * Hq * pl.splits;
+  return df::round_up(rows * D * sizeof(float), 256) + df::round_up(rows * 2 * sizeof(float), 256);
+}
+
+extern "C" df_status dualflow_decode_attn(
+    const void* q1, const void* q2raw, const void* a, int64_t q_stride_b, const void* k_cache,
+    const void* v_cache, const int32_t* block_table, int max_blocks_per_seq,
+    const int32_t* seqlens, int max_seqlen, void* o1, void* o2, int64_t o_stride_b, int B, int Hq,
+    int Hkv, int D, int block_size, int num_blocks, float scale, int dtype, int num_splits,
+    void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  using namespace df;
+  if (!q1 || !k_cache || !v_cache || !block_table || !seqlens) return DF_ERR_NULL;
+  const bool want2 = (o2 != nullptr) && (q2raw != nullptr);
+  if (!o1 && !want2) return DF_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || num_blocks < 1 || max_blocks_per_seq < 1 ||
+      max_seqlen < 1 || num_splits < 0)
+    return DF_ERR_SHAPE;
+  if (Hq % Hkv != 0) return DF_ERR_SHAPE;
+  if (B > 65535 || Hkv > 65535) return DF_ERR_SHAPE;
+  if (static_cast<int64_t>(max_seqlen) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return DF_ERR_SHAPE;
+  if (block_size != attn::kPage) return DF_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return DF_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 4) return DF_ERR_UNSUPPORTED;
+  if (dtype != DF_FP32 && dtype != DF_BF16) return DF_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(num_blocks) * Hkv * attn::kPage >= (int64_t(1) << 31))
+    return DF_ERR_UNSUPPORTED;
+  const int64_t qs = q_stride_b ? q_stride_b : static_cast<int64_t>(Hq) * D;
+  const int64_t os = o_stride_b ? o_stride_b : static_cast<int64_t>(Hq) * D;
+  if (qs < static_cast<int64_t>(Hq) * D || os < static_cast<int64_t>(Hq) * D) return DF_ERR_SHAPE;
+  const uintptr_t esize = dtype == DF_BF16 ? 2 : 4;
+  const uintptr_t qa_align = dtype == DF_BF16 ? 4 : 4;
+  if (!aligned(q1, qa_align) || (q2raw && !aligned(q2raw, qa_align)) || (a && !aligned(a, qa_align)) ||
+      (o1 && !aligned(o1, esize)) || (o2 && !aligned(o2, esize)))
+    return DF_ERR_ALIGN;
+  if (dtype == DF_BF16 && (qs % 2 != 0)) return DF_ERR_ALIGN;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return DF_ERR_ALIGN;
+
+  const Plan pl = make_plan(B, Hkv, max_seqlen, block_size, num_splits);
+  attn::Params p{};
+  p.q1 = q1;
+  p.q2raw = want2 ? q2raw : nullptr;
+  p.a = want2 ? a : nullptr;
+  p.q_stride_b = qs;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_table = block_table;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.seqlens = seqlens;
+  p.max_seqlen = max_seqlen;
+  p.o1 = o1;
+  p.o2 = want2 ? o2 : nullptr;
+  p.o_stride_b = os;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.num_blocks = num_blocks;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.chunk_pages = pl.chunk_pages;
+  p.num_splits = pl.splits;
+  p.err = err_flag;
+  p.dual = want2 ? 1 : 0;
+  p.write1 = o1 ? 1 : 0;
+  p.write2 = want2 ? 1 : 0;
+  if (pl.splits > 1) {
+    const size_t need = dualflow_decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size,
+                                                            num_splits);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DF_ERR_WORKSPACE;
+    const size_t rows = static_cast<size_t>(B) * 2 * Hq * pl.splits;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         round_up(rows * D * sizeof(float), 256));
+  }
+
+  CUtensorMap tmK, tmV;
+  if (dtype == DF_BF16) {
+    const uint64_t rows = static_cast<uint64_t>(num_blocks) * Hkv * attn::kPage;
+    if (!encode_tmap_bf16_2d(&tmK, k_cache, rows, D, D * 2, attn::kPage, 64) ||
+        !encode_tmap_bf16_2d(&tmV, v_cache, rows, D, D * 2, attn::kPage, 64))
+      return DF_ERR_CUDA;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (D == 64) ? attn::launch<64>(p, dtype, &tmK, &tmV, st)
+                            : attn::launch<128>(p, dtype, &tmK, &tmV, st);
+  return e == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}

@@ -1,0 +1,566 @@
+// Grouped shared-weight projection on the 5th-generation tensor cores.
+//
+// Method: both flows share every attention, MLP and output matrix ("Sintesi
+// Tecnica: Dual-Flow Transformers", section "Architettura Core"), so at a
+// decode step the primary rows and the auxiliary rows are multiplied by the
+// same weight in ONE GEMM and each weight byte is read from HBM once
+// ("Costi di Inferenza": no growth in the unique weights read).
+//
+// Design (sm_100a, one CTA per SM, persistent stream-K):
+//  * the whole M <= 128 rows form one UMMA M-tile; W tiles of 128 rows x 64 k
+//    (bf16, 128-byte swizzle) and the matching X tile arrive by TMA into a
+//    6-deep shared-memory ring;
+//  * one elected thread issues tcgen05.mma (kind::f16, M=128, N=128, K=16,
+//    fp32 accumulation in TMEM, two 128-column accumulators so the epilogue
+//    of one segment overlaps the MMAs of the next) and tcgen05.commit frees
+//    ring stages and publishes accumulators;
+//  * the k-iterations of all tiles are divided evenly over the CTAs (stream-K)
+//    so every SM streams the same number of weight bytes; a tile cut between
+//    CTAs is summed by whichever of its CTAs finishes last (fp32 partials in an
+//    L2-resident workspace, a per-tile arrival counter, no waiting on other
+//    CTAs, fixed summation order -> deterministic);
+//  * 4 epilogue warps read TMEM (tcgen05.ld 32x32b) and apply the fused
+//    epilogue: plain store, SwiGLU with the b_l coupling, or residual add with
+//    the c_l coupling. The coupling pairs auxiliary row m_primary + j with
+//    primary row j of the same tile through shared memory.
+// Every mbarrier wait is bounded; on a timeout the kernel flags it, drains its
+// own copies/MMAs (bounded) and frees TMEM before returning.
+#include <math.h>
+
+#include "common.cuh"
+#include "host_util.h"
+
+namespace df {
+namespace gemm {
+
+constexpr int kBM = 128;           // rows per tile (all rows of both flows)
+constexpr int kBN = 128;           // accumulator columns per tile
+constexpr int kBK = 64;            // k per stage (one 128-byte swizzle atom)
+constexpr int kStages = 6;
+constexpr int kTileA = kBM * kBK * 2;   // 16 KB
+constexpr int kTileB = kBN * kBK * 2;   // 16 KB
+constexpr int kStageBytes = kTileA + kTileB;
+constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA/TMEM, warps 2-5 epilogue
+constexpr int kEpiThreads = 128;
+constexpr int kMaxCtas = 148;      // one CTA per SM of a B200
+constexpr int kXPitch = 33;        // floats per row of the coupling exchange buffer
+constexpr int kTmemCols = 256;     // two fp32 accumulators of 128 columns
+// Tile counters live at the start of the workspace in a region of FIXED size,
+// so one workspace can be shared by projections of different shapes.
+constexpr size_t kCounterBytes = 65536;
+constexpr int kMaxTiles = static_cast<int>(kCounterBytes / sizeof(int));
+
+struct Params {
+  int M, m_primary, N, K, n_aux;
+  int epilogue;
+  int n_tiles, kblocks, ctas;
+  long long total_iters;
+  __nv_bfloat16* y;
+  int64_t ldy;
+  const __nv_bfloat16* coupling;
+  const __nv_bfloat16* residual;
+  int64_t ldr;
+  int* counters;     // [n_tiles]
+  float* partials;   // [2 * ctas][128][128]
+  int32_t* err;
+  int F;             // SWIGLU: rows of W_gate (= output columns)
+};
+
+__host__ __device__ inline long long iter_begin(const Params& p, int cta) {
+  return static_cast<long long>(cta) * p.total_iters / p.ctas;
+}
+__device__ inline int owner_of(const Params& p, long long it) {
+  return static_cast<int>(((it + 1) * p.ctas - 1) / p.total_iters);
+}
+
+// Descriptor of a K-major bf16 tile with 128-byte swizzle: 8-row core groups
+// 1024 bytes apart (stride byte offset), leading offset unused (1), version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// kind::f16 instruction descriptor: D fp32, A/B bf16, both K-major, N=128, M=128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kBM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  __syncwarp();
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = s[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[q * 8 + 2 * k] = bf16_bits_to_float(static_cast<uint16_t>(w[k] & 0xffffu));
+      v[q * 8 + 2 * k + 1] = bf16_bits_to_float(static_cast<uint16_t>(w[k] >> 16));
+    }
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = pack_bf16x2(__float2bfloat16_rn(v[q * 8 + 2 * k]),
+                         __float2bfloat16_rn(v[q * 8 + 2 * k + 1]));
+    d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Epilogue of one 32-column output chunk held by this thread (row `row`).
+// `val` = raw accumulator (NONE/RESIDUAL) or SiLU(gate)*up (SWIGLU).
+// Coupling: primary rows publish their values, auxiliary rows add
+// coupling[col] * value of their paired primary row.
+__device__ __forceinline__ void finish_chunk(const Params& p, int row, int col0, float (&val)[32],
+                                             float* xbuf) {
+  const bool coupled = p.coupling != nullptr;
+  if (coupled) {
+    if (row < p.m_primary) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) xbuf[row * kXPitch + i] = val[i];
+    }
+    epi_bar();
+    if (row >= p.m_primary && row < p.M) {
+      float cv[32];
+      load_bf16x32(p.coupling + col0, cv);
+      const float* src = xbuf + (row - p.m_primary) * kXPitch;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) val[i] = fmaf(cv[i], src[i], val[i]);
+    }
+    epi_bar();
+  }
+  if (row >= p.M) return;
+  if (row >= p.m_primary && col0 >= p.n_aux) return;
+  if (p.epilogue == DF_EPI_RESIDUAL) {
+    float rv[32];
+    load_bf16x32(p.residual + row * p.ldr + col0, rv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) val[i] += rv[i];
+  }
+  store_bf16x32(p.y + row * p.ldy + col0, val);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// Source of accumulator chunks: TMEM (a tile owned by one CTA) or the fp32
+// partials of all contributing CTAs q_a..q_b summed in CTA (= k) order.
+struct ChunkSrc {
+  bool from_tmem;
+  uint32_t taddr;  // this row's TMEM address of the accumulator (column 0)
+  int tile, row, q_a, q_b;
+};
+
+__device__ __forceinline__ const float* partial_row(const Params& p, int q, int tile, int row) {
+  const int first_tile = static_cast<int>(iter_begin(p, q) / p.kblocks);
+  const int slot = 2 * q + (first_tile == tile ? 0 : 1);
+  return p.partials + (static_cast<size_t>(slot) * kBM + row) * kBN;
+}
+
+__device__ __forceinline__ void read_chunk(const Params& p, const ChunkSrc& s, int col,
+                                           float (&v)[32]) {
+  if (s.from_tmem) {
+    tmem_ld32(s.taddr + col, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    for (int q = s.q_a; q <= s.q_b; ++q) {
+      const float4* src = reinterpret_cast<const float4*>(partial_row(p, q, s.tile, s.row) + col);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 f = __ldcg(src + k);
+        v[4 * k] += f.x;
+        v[4 * k + 1] += f.y;
+        v[4 * k + 2] += f.z;
+        v[4 * k + 3] += f.w;
+      }
+    }
+  }
+}
+
+// Full epilogue of a tile from the given source.
+__device__ void tile_epilogue(const Params& p, int tile, int row, const ChunkSrc& src,
+                              float* xbuf) {
+  if (p.epilogue == DF_EPI_SWIGLU) {
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float g[32], u[32];
+      read_chunk(p, src, 32 * c, g);
+      read_chunk(p, src, 64 + 32 * c, u);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+      finish_chunk(p, row, tile * 64 + 32 * c, g, xbuf);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      read_chunk(p, src, 32 * c, v);
+      finish_chunk(p, row, tile * kBN + 32 * c, v, xbuf);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_proj_kernel(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* xbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [128][33]
+  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kBM * kXPitch);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* flags = reinterpret_cast<int*>(tmem_slot + 1);  // [0] timeout, [1] fixup owner
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const long long it_begin = iter_begin(p, cta);
+  const long long it_end = iter_begin(p, cta + 1);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiThreads / 32);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "n"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int KB = p.kblocks;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmW);
+      const uint64_t pol_w = l2_policy_evict_first();  // weights: streamed once
+      const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read by every CTA
+      long long n = 0;  // stages issued
+      bool ok = true;
+      for (long long it = it_begin; it < it_end && ok; ++it, ++n) {
+        const int s = static_cast<int>(n % kStages);
+        if (n >= kStages && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / kStages) - 1) & 1))) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        const int tile = static_cast<int>(it / KB), kb = static_cast<int>(it % KB);
+        uint8_t* sa = smem + s * kStageBytes;
+        uint8_t* sb = sa + kTileA;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+        if (p.epilogue == DF_EPI_SWIGLU) {
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * 64, pol_w);
+          tma_load_2d_hint(sb + kTileB / 2, &tmW, &full[s], kb * kBK, p.F + tile * 64, pol_w);
+        } else {
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * kBN, pol_w);
+        }
+      }
+      // drain own copies still in flight
+      for (long long i = (n > kStages ? n - kStages : 0); i < n; ++i)
+        mbar_wait(&full[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      long long n = 0;  // stages consumed
+      int seg = 0;
+      bool ok = true;
+      long long it = it_begin;
+      while (it < it_end && ok) {
+        const int k0 = static_cast<int>(it % KB);
+        const long long seg_len = min(static_cast<long long>(KB - k0), it_end - it);
+        const int acc = seg & 1;
+        if (seg >= 2 && !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        for (long long j = 0; j < seg_len; ++j, ++n) {
+          const int s = static_cast<int>(n % kStages);
+          if (!mbar_wait(&full[s], static_cast<uint32_t>((n / kStages) & 1))) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+          const uint32_t b_addr = a_addr + kTileA;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            umma_bf16(d_tmem, smem_desc(a_addr + kk * 32), smem_desc(b_addr + kk * 32), kIdesc,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        it += seg_len;
+        ++seg;
+      }
+      // drain: wait until the last committed MMAs have completed
+      if (n > 0) mbar_wait(&empty[(n - 1) % kStages], static_cast<uint32_t>(((n - 1) / kStages) & 1));
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127
+    int seg = 0;
+    long long it = it_begin;
+    while (it < it_end) {
+      const int tile = static_cast<int>(it / KB);
+      const int k0 = static_cast<int>(it % KB);
+      const long long seg_len = min(static_cast<long long>(KB - k0), it_end - it);
+      const int acc = seg & 1;
+      // bounded wait; the give-up decision is made uniform over the 4 warps
+      const bool got = mbar_wait_warp(&acc_full[acc], static_cast<uint32_t>((seg >> 1) & 1));
+      if (!got && lane == 0) atomicOr(&flags[0], 1);
+      epi_bar();
+      if (flags[0]) {
+        if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const long long t_first = static_cast<long long>(tile) * KB;
+      const int q_a = owner_of(p, t_first);
+      const int q_b = owner_of(p, t_first + KB - 1);
+      ChunkSrc src;
+      src.from_tmem = true;
+      src.taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
+      src.tile = tile;
+      src.row = row;
+      src.q_a = q_a;
+      src.q_b = q_b;
+      if (q_a == q_b) {
+        tile_epilogue(p, tile, row, src, xbuf);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      } else {
+        // partial tile: publish this CTA's fp32 partial in its slot
+        const bool first_seg = (it == it_begin);
+        const int slot = 2 * cta + (first_seg ? 0 : 1);
+        float* part = p.partials + (static_cast<size_t>(slot) * kBM + row) * kBN;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(src.taddr + 32 * c, v);
+          float4* dst = reinterpret_cast<float4*>(part + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            __stcg(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        __threadfence();
+        epi_bar();
+        if (et == 0) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          const int last = (old == q_b - q_a);
+          if (last) atomicExch(&p.counters[tile], 0);
+          flags[1] = last;
+        }
+        epi_bar();
+        const int last = flags[1];
+        epi_bar();
+        if (last) {
+          __threadfence();
+          ChunkSrc fx;
+          fx.from_tmem = false;
+          fx.taddr = 0;
+          fx.tile = tile;
+          fx.row = row;
+          fx.q_a = q_a;
+          fx.q_b = q_b;
+          tile_epilogue(p, tile, row, fx, xbuf);
+        }
+      }
+      it += seg_len;
+      ++seg;
+    }
+  }
+
+  // teardown: everyone done with TMEM before it is freed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "n"(kTmemCols)
+                 : "memory");
+  }
+}
+
+struct Layout {
+  int n_tiles, kblocks, ctas;
+  long long total;
+  size_t counters_bytes, partial_bytes;
+};
+
+inline Layout make_layout(int N, int K, int epilogue) {
+  Layout l;
+  l.n_tiles = (epilogue == DF_EPI_SWIGLU) ? N / 128 : N / kBN;
+  l.kblocks = K / kBK;
+  l.total = static_cast<long long>(l.n_tiles) * l.kblocks;
+  l.ctas = static_cast<int>(l.total < kMaxCtas ? l.total : kMaxCtas);
+  l.counters_bytes = kCounterBytes;
+  l.partial_bytes = static_cast<size_t>(2) * l.ctas * kBM * kBN * sizeof(float);
+  return l;
+}
+
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kBM * kXPitch * 4 + 256;
+
+}  // namespace gemm
+}  // namespace df
+
+extern "C" size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int epilogue) {
+  using namespace df::gemm;
+  if (M < 1 || N < 1 || K < 1 || epilogue < 0 || epilogue > 2) return 0;
+  const Layout l = make_layout(N, K, epilogue);
+  if (l.total < 1) return 0;
+  return l.counters_bytes + l.partial_bytes;
+}
+
+extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
+                                           const void* w, int N, int K, int n_aux, void* y,
+                                           int64_t ldy, int epilogue, const void* coupling,
+                                           const void* residual, int64_t ldr, void* workspace,
+                                           size_t workspace_bytes, int32_t* err_flag,
+                                           void* stream) {
+  using namespace df;
+  using namespace df::gemm;
+  if (!x || !w || !y) return DF_ERR_NULL;
+  if (epilogue < DF_EPI_NONE || epilogue > DF_EPI_RESIDUAL) return DF_ERR_UNSUPPORTED;
+  if (epilogue == DF_EPI_RESIDUAL && !residual) return DF_ERR_NULL;
+  if (epilogue == DF_EPI_NONE && (coupling || residual)) return DF_ERR_SHAPE;
+  const int M = m_primary + m_aux;
+  if (m_primary < 0 || m_aux < 0 || M < 1 || N < 1 || K < 1) return DF_ERR_SHAPE;
+  if (coupling && m_aux != m_primary) return DF_ERR_SHAPE;
+  if (M > kBM) return DF_ERR_UNSUPPORTED;
+  if (K % kBK != 0) return DF_ERR_UNSUPPORTED;
+  if (epilogue == DF_EPI_SWIGLU ? (N % 128 != 0) : (N % kBN != 0)) return DF_ERR_UNSUPPORTED;
+  const int n_out = epilogue == DF_EPI_SWIGLU ? N / 2 : N;
+  if (n_aux < 0 || n_aux > n_out) return DF_ERR_SHAPE;
+  if (n_aux % 32 != 0 && n_aux != n_out) return DF_ERR_UNSUPPORTED;
+  const int64_t lx = ldx ? ldx : K, ly = ldy ? ldy : n_out, lr = ldr ? ldr : n_out;
+  if (lx < K || ly < n_out || (residual && lr < n_out)) return DF_ERR_SHAPE;
+  if (lx % 8 || ly % 8 || (residual && lr % 8)) return DF_ERR_ALIGN;
+  if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16) || (residual && !aligned(residual, 16)) ||
+      (coupling && !aligned(coupling, 16)))
+    return DF_ERR_ALIGN;
+  const Layout l = make_layout(N, K, epilogue);
+  if (l.n_tiles > kMaxTiles) return DF_ERR_UNSUPPORTED;
+  const size_t need = l.counters_bytes + l.partial_bytes;
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DF_ERR_WORKSPACE;
+
+  Params p{};
+  p.M = M;
+  p.m_primary = m_primary;
+  p.N = N;
+  p.K = K;
+  p.n_aux = n_aux;
+  p.epilogue = epilogue;
+  p.n_tiles = l.n_tiles;
+  p.kblocks = l.kblocks;
+  p.ctas = l.ctas;
+  p.total_iters = l.total;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ldy = ly;
+  p.coupling = static_cast<const __nv_bfloat16*>(coupling);
+  p.residual = static_cast<const __nv_bfloat16*>(residual);
+  p.ldr = lr;
+  p.counters = static_cast<int*>(workspace);
+  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + l.counters_bytes);
+  p.err = err_flag;
+  p.F = N / 2;
+
+  CUtensorMap tmX, tmW;
+  if (!encode_tmap_bf16_2d(&tmX, x, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                           static_cast<uint64_t>(lx) * 2, kBM, kBK) ||
+      !encode_tmap_bf16_2d(&tmW, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                           static_cast<uint64_t>(K) * 2,
+                           epilogue == DF_EPI_SWIGLU ? 64 : kBN, kBK))
+    return DF_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(grouped_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return DF_ERR_CUDA;
+    attr_set = true;
+  }
+  grouped_proj_kernel<<<l.ctas, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmX, tmW,
+                                                                                            p);
+  return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}

@@ -1,0 +1,27 @@
+// Host-side helpers shared by the ABI entry points: tensor-map encoding via the
+// driver entry point (no link-time dependency on libcuda, so the library loads
+// on machines without a GPU driver), and small arithmetic helpers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace df {
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t round_up(size_t a, size_t m) { return (a + m - 1) / m * m; }
+inline bool aligned(const void* p, uintptr_t n) {
+  return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0;
+}
+
+// Encode a 2-D row-major bf16 tensor map: `rows` rows of `cols` elements with a
+// row pitch of `row_pitch_bytes`, box = box_rows x box_cols, 128-byte swizzle.
+// Returns false if the driver entry point is unavailable or encoding fails.
+bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint64_t row_pitch_bytes, uint32_t box_rows, uint32_t box_cols);
+
+// Streaming-multiprocessor count of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace df

@@ -1,0 +1,160 @@
+"""One Dual-Flow decoder layer at one generated position, both flows.
+
+Composition of library calls only (each step is a libdualflow kernel):
+
+  1. RMSNorm of X = [x1 rows; x2 rows]                      dualflow_rmsnorm
+  2. QKV = Xn W_qkv^T, one GEMM for both flows; auxiliary
+     rows stored only for the Q columns                       dualflow_grouped_proj
+  3. append the primary rows' K/V at position L (the
+     auxiliary flow never writes the cache)                  dualflow_kv_append
+  4. dual decode attention over L + 1 tokens, Q2 coupled
+     to Q1 through a_l inside the kernel                     dualflow_decode_attn
+  5. X' = X + O W_o^T                                        dualflow_grouped_proj (residual)
+  6. RMSNorm of X'                                           dualflow_rmsnorm
+  7. H = SiLU(X'n W_gate^T) * (X'n W_up^T), aux += b_l H1    dualflow_grouped_proj (swiglu)
+  8. X'' = X' + H W_down^T, aux += c_l (H1 W_down^T)         dualflow_grouped_proj (residual)
+
+Pages: "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
+Core" (shared matrices, primary-only cache writes, auxiliary flow active at
+generated positions), "Meccanismi Chiave" (asymmetric shared-KV attention and
+the a/b/c coupling vectors) and "Costi di Inferenza" (grouped decode reads the
+weights and the cache once for both flows). The normalisation, SwiGLU MLP and
+the additive coupling forms are the readings taken where the pages are silent.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+# Launches of our kernels per layer step: rmsnorm, qkv GEMM, append, attention
+# split (+ combine when split), W_o GEMM, rmsnorm, gate/up GEMM, down GEMM.
+
+
+class DualFlowLayer:
+    def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
+                 num_splits=0):
+        self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
+        self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
+        self.d_model = weights["w_o"].shape[0]
+        self.max_seqlen = int(max_seqlen)
+        self.eps = eps
+        self.num_splits = num_splits
+        dev = torch.device(device)
+        bf = torch.bfloat16
+        M = 2 * B
+        qd, kvd = Hq * D, Hkv * D
+        self.xn = torch.empty(M, self.d_model, dtype=bf, device=dev)
+        self.qkv = torch.empty(M, qd + 2 * kvd, dtype=bf, device=dev)
+        self.attn = torch.empty(M, qd, dtype=bf, device=dev)
+        self.x_mid = torch.empty(M, self.d_model, dtype=bf, device=dev)
+        self.xn2 = torch.empty(M, self.d_model, dtype=bf, device=dev)
+        self.h = torch.empty(M, F, dtype=bf, device=dev)
+        self.x_out = torch.empty(M, self.d_model, dtype=bf, device=dev)
+        self.x_in = torch.empty(M, self.d_model, dtype=bf, device=dev)
+        ws = max(api.grouped_proj_workspace_size(M, *weights["w_qkv"].shape, "none"),
+                 api.grouped_proj_workspace_size(M, *weights["w_o"].shape, "residual"),
+                 api.grouped_proj_workspace_size(M, *weights["w_gu"].shape, "swiglu"),
+                 api.grouped_proj_workspace_size(M, *weights["w_down"].shape, "residual"))
+        self.proj_ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
+        aw = api.decode_attn_workspace_size(B, Hq, Hkv, D, self.max_seqlen, num_splits)
+        self.attn_ws = torch.empty(max(aw, 256), dtype=torch.uint8, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.splits = api.decode_attn_num_splits(B, Hkv, self.max_seqlen, num_splits)
+
+    @property
+    def launches_per_step(self) -> int:
+        return 8 + (1 if self.splits > 1 else 0)
+
+    # ------------------------------------------------------------ CUDA graphs
+    def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):
+        """Capture the step as three CUDA graphs (before attention, attention,
+        after attention) over fixed buffers, so a step costs three graph
+        launches instead of nine library calls from Python. The step runs once
+        eagerly first, so one-time host set-up happens outside the capture.
+        Events recorded between the graphs time the attention on the stream."""
+        args = (X, k_cache, v_cache, block_table, positions, seqlens)
+        self.step(*args)
+        torch.cuda.synchronize()
+        self._graph_args = args
+        self.graphs = []
+        for part in ("pre", "attn", "post"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._step_part(part, *args)
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def replay(self, timers=None):
+        """One captured step on the current stream. timers: optional
+        {"attn": (start_event, end_event)} recorded around the attention."""
+        self.graphs[0].replay()
+        if timers is not None:
+            timers["attn"][0].record()
+        self.graphs[1].replay()
+        if timers is not None:
+            timers["attn"][1].record()
+        self.graphs[2].replay()
+        return self.x_out
+
+    def step(self, X, k_cache, v_cache, block_table, positions, seqlens, stream=None,
+             timers=None):
+        """X: bf16 [2B, d_model] (primary rows then auxiliary rows). Returns the
+        layer output (a preallocated buffer, overwritten by the next step).
+        seqlens must equal positions + 1 (the attended length after the append).
+        timers: optional dict of (start, end) CUDA events around the attention."""
+        args = (X, k_cache, v_cache, block_table, positions, seqlens)
+        self._step_part("pre", *args, stream=stream)
+        if timers is not None:
+            timers["attn"][0].record()
+        self._step_part("attn", *args, stream=stream)
+        if timers is not None:
+            timers["attn"][1].record()
+        self._step_part("post", *args, stream=stream)
+        return self.x_out
+
+    def _step_part(self, part, X, k_cache, v_cache, block_table, positions, seqlens, stream=None):
+        """One third of the step: "pre" (norm, QKV, append), "attn", "post"."""
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        qd, kvd = Hq * D, Hkv * D
+        w = self.w
+        qkv = self.qkv
+        if part == "pre":
+            api.rmsnorm(X, y=self.xn, eps=self.eps, stream=stream)
+            api.grouped_proj(self.xn, B, w["w_qkv"], n_aux=qd, y=qkv, workspace=self.proj_ws,
+                             err_flag=self.err, stream=stream)
+            api.kv_append(qkv[:B, qd:qd + kvd].view(B, Hkv, D), qkv[:B, qd + kvd:].view(B, Hkv, D),
+                          k_cache, v_cache, block_table, positions, err_flag=self.err,
+                          stream=stream)
+        elif part == "attn":
+            api.decode_attn(qkv[:B, :qd].view(B, Hq, D), qkv[B:, :qd].view(B, Hq, D), w["a"],
+                            k_cache, v_cache, block_table, seqlens, self.max_seqlen,
+                            o1=self.attn[:B].view(B, Hq, D), o2=self.attn[B:].view(B, Hq, D),
+                            num_splits=self.num_splits, workspace=self.attn_ws,
+                            err_flag=self.err, stream=stream)
+        else:
+            api.grouped_proj(self.attn, B, w["w_o"], y=self.x_mid, epilogue="residual",
+                             residual=X, workspace=self.proj_ws, err_flag=self.err,
+                             stream=stream)
+            api.rmsnorm(self.x_mid, y=self.xn2, eps=self.eps, stream=stream)
+            api.grouped_proj(self.xn2, B, w["w_gu"], y=self.h, epilogue="swiglu",
+                             coupling=w["b"], workspace=self.proj_ws, err_flag=self.err,
+                             stream=stream)
+            api.grouped_proj(self.h, B, w["w_down"], y=self.x_out, epilogue="residual",
+                             coupling=w["c"], residual=self.x_mid, workspace=self.proj_ws,
+                             err_flag=self.err, stream=stream)
+
+
+    def step_host(self, x_host, out_host, k_cache, v_cache, block_table, positions, seqlens,
+                  stream=None):
+        """Host-buffer entry point: copies X from (pinned) host memory, runs the
+        step and copies the layer output back, all queued on the stream."""
+        self.x_in.copy_(x_host, non_blocking=True)
+        if getattr(self, "graphs", None) and self._graph_args[0] is self.x_in:
+            out = self.replay()
+        else:
+            out = self.step(self.x_in, k_cache, v_cache, block_table, positions, seqlens,
+                            stream=stream)
+        out_host.copy_(out, non_blocking=True)
+        return out_host

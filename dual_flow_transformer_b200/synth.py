@@ -132,19 +132,25 @@ def make_block_table(g, capacities, block_size=BLOCK_SIZE, random_table=False):
     return table, total
 
 
-def make_attn_inputs(w: AttnWorkload, seed: Optional[int] = None, B: Optional[int] = None):
+def make_attn_inputs(w: AttnWorkload, seed: Optional[int] = None, B: Optional[int] = None,
+                     lengths=None):
     """Host tensors for one decode-attention step of workload ``w``.
 
     Returns a dict with: q1, q2raw [B, Hq, D]; a [Hq, D]; k_cache, v_cache
     [num_blocks, Hkv, 64, D]; block_table [B, max_blocks] int32; seqlens [B]
     int32 (attended length after any append); positions [B] int32 (append
     slot = cache length before the step) and k_new, v_new [B, Hkv, D] when the
-    workload includes the append.
+    workload includes the append. ``lengths`` (optional) replaces the drawn
+    lengths (edge-case tests).
     """
     g = _gen(w.seed if seed is None else seed)
-    B = w.B if B is None else B
     dt = w.torch_dtype
-    lens = make_lengths(g, B, w.len_lo, w.len_hi)
+    if lengths is not None:
+        lens = torch.as_tensor(lengths, dtype=torch.int32)
+        B = lens.numel()
+    else:
+        B = w.B if B is None else B
+        lens = make_lengths(g, B, w.len_lo, w.len_hi)
     if w.append:
         positions = lens.clone()
         seqlens = lens + 1

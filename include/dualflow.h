@@ -1,0 +1,194 @@
+/*
+ * dualflow.h -- C ABI of the Dual-Flow Transformer decode-step library
+ * (libdualflow.so, NVIDIA B200 / sm_100a).
+ *
+ * The method (arXiv 2608.12385, "Dual-Flow Transformers"; technical summary
+ * page "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
+ * Core" and "Meccanismi Chiave") runs two residual flows through the same
+ * weights. The primary flow is an ordinary causal Transformer and is the only
+ * writer of the single persistent KV cache (K1, V1). The auxiliary flow, active
+ * at the last prompt position and at every generated position, builds its own
+ * query Q2, coupled one way to the primary query Q1 through a learned
+ * per-layer vector a_l, and attends to the primary K1/V1 without ever writing
+ * the cache or feeding back into the primary flow. Because both flows share
+ * the weights and the cache, one pass over each weight matrix and each KV page
+ * can serve both ("grouped execution"). This library is that decode step.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates nothing and keeps no state between calls; calls are reentrant.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream). Argument errors are detected on the host
+ *    and returned BEFORE any launch. A failed launch returns DF_ERR_CUDA.
+ *  - Errors that depend on device data (a length, a page index, a position)
+ *    never trap: the kernel skips the bad access and ORs a DF_DEVERR_* bit into
+ *    *err_flag (device int32, may be NULL). The caller reads it after syncing.
+ *  - Every wait inside a kernel is bounded (about 2 s); a wait that gives up
+ *    sets DF_DEVERR_TIMEOUT and the kernel returns.
+ *  - bf16 = IEEE bfloat16 (1-8-7), stored as 2-byte values. "Elements" strides
+ *    count elements of the tensor's dtype.
+ *  - Paged KV cache layout: cache[num_blocks][Hkv][block_size][D], token j of
+ *    sequence b in page block_table[b * max_blocks_per_seq + j / block_size],
+ *    slot j % block_size. block_size must be 64.
+ */
+#ifndef DUALFLOW_H
+#define DUALFLOW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DF_OK = 0,
+  DF_ERR_NULL = 1,        /* a required pointer is NULL                        */
+  DF_ERR_SHAPE = 2,       /* sizes inconsistent or out of range                */
+  DF_ERR_UNSUPPORTED = 3, /* valid request this build does not implement       */
+  DF_ERR_WORKSPACE = 4,   /* workspace missing, too small or misaligned        */
+  DF_ERR_ALIGN = 5,       /* pointer or stride not aligned as documented       */
+  DF_ERR_CUDA = 6         /* a CUDA runtime call or a launch failed            */
+} df_status;
+
+typedef enum { DF_FP32 = 0, DF_BF16 = 1 } df_dtype;
+
+typedef enum {
+  DF_EPI_NONE = 0,     /* y = x w^T                                             */
+  DF_EPI_SWIGLU = 1,   /* y = SiLU(gate) * up (+ b * y_primary on aux rows)     */
+  DF_EPI_RESIDUAL = 2  /* y = residual + x w^T (+ c * (x w^T)_primary on aux)   */
+} df_epilogue;
+
+/* Bits ORed into *err_flag by kernels (device-side data errors). */
+#define DF_DEVERR_SEQLEN   0x1 /* seqlens[b] < 1 (output 0) or above max_seqlen (clamped) */
+#define DF_DEVERR_BLOCK    0x2 /* a block_table entry outside [0, num_blocks): page skipped */
+#define DF_DEVERR_POSITION 0x4 /* an append position outside the sequence's table: skipped */
+#define DF_DEVERR_TIMEOUT  0x8 /* a bounded in-kernel wait gave up: outputs invalid         */
+
+/* Version of this ABI (incremented on any signature change). */
+int dualflow_abi_version(void);
+
+/* Human-readable name of a df_status value; never NULL. */
+const char* dualflow_status_string(int status);
+
+/* ------------------------------------------------------------------------ */
+/* Dual-flow decode attention (asymmetric shared-KV attention).              */
+/*                                                                           */
+/* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi       */
+/* Chiave": the primary query Q1 runs ordinary causal attention over K1/V1;  */
+/* the auxiliary query Q2 = Q2raw + a (.) Q1 (element-wise; the pages name   */
+/* the coupling vector but print no formula, this additive one-way form is   */
+/* the reading taken) attends over the SAME K1/V1. For sequence b, query     */
+/* head h, KV head g = h / (Hq / Hkv), flow f:                               */
+/*   O_f[b,h] = softmax(scale * q_f K1[b,g]^T) V1[b,g] over the first         */
+/*   seqlens[b] tokens of the cache.                                         */
+/* Each KV page is read from HBM once for all 2 * Hq/Hkv query rows of its    */
+/* KV head. Split over the sequence (flash-decoding) with per-split fp32     */
+/* partials in `workspace`, then a separate combine kernel.                  */
+/*                                                                           */
+/* q1, q2raw : [B][Hq][D] (dtype), sequence b at q + b*q_stride_b elements   */
+/*             (q_stride_b = 0 means Hq*D). 4-byte aligned; q_stride_b even. */
+/* a         : [Hq][D] (dtype) or NULL (q2raw is then used as Q2 as is).     */
+/* k_cache, v_cache : paged cache (dtype), 16-byte aligned. Read only: this  */
+/*             call never writes the cache.                                  */
+/* block_table : int32 [B][max_blocks_per_seq]; seqlens : int32 [B], the     */
+/*             attended length of each sequence (>= 1, <= max_seqlen).       */
+/* max_seqlen : host upper bound of seqlens; <= max_blocks_per_seq*block_size.*/
+/* o1, o2    : [B][Hq][D] (dtype) outputs at o + b*o_stride_b (0 = Hq*D).    */
+/*             o1 == NULL: aux-only call (q1 still needed for the coupling). */
+/*             o2 == NULL or q2raw == NULL: primary-only call.               */
+/*             O1 is bit-identical in primary-only, aux-only and dual calls  */
+/*             and independent of q2raw/a (even NaN/Inf): the split plan      */
+/*             depends only on (B, Hkv, max_seqlen, num_splits).              */
+/* scale     : softmax scale; <= 0 selects 1/sqrt(D).                         */
+/* dtype     : DF_BF16 (fp32 accumulation; Q2 and softmax weights kept to     */
+/*             ~16 mantissa bits through a bf16 hi/lo split) or DF_FP32.      */
+/* num_splits: 0 = automatic; otherwise the requested number of splits.      */
+/* workspace : device scratch, 256-byte aligned, at least                    */
+/*             dualflow_decode_attn_workspace_size(...) bytes (0 when the    */
+/*             plan has one split, then workspace may be NULL).               */
+/* Supported: D in {64, 128}, block_size 64, Hq/Hkv in {1,2,3,4}.            */
+/* ------------------------------------------------------------------------ */
+int dualflow_decode_attn_num_splits(int B, int Hkv, int max_seqlen, int block_size,
+                                    int num_splits);
+size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, int D, int max_seqlen,
+                                           int block_size, int num_splits);
+df_status dualflow_decode_attn(const void* q1, const void* q2raw, const void* a,
+                               int64_t q_stride_b, const void* k_cache, const void* v_cache,
+                               const int32_t* block_table, int max_blocks_per_seq,
+                               const int32_t* seqlens, int max_seqlen, void* o1, void* o2,
+                               int64_t o_stride_b, int B, int Hq, int Hkv, int D,
+                               int block_size, int num_blocks, float scale, int dtype,
+                               int num_splits, void* workspace, size_t workspace_bytes,
+                               int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Primary-only KV append.                                                  */
+/*                                                                           */
+/* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Architettura      */
+/* Core": only the primary flow writes the persistent KV cache. Copies       */
+/* k_new[b][g][:] and v_new[b][g][:] (every KV head g) into the page          */
+/* block_table[b][positions[b] / block_size], slot positions[b] % block_size.*/
+/* A bit-exact copy; no other cache byte changes.                            */
+/*                                                                           */
+/* k_new, v_new : [B][Hkv][D] (dtype) at + b*new_stride_b elements (0 means  */
+/*             Hkv*D); 16-byte aligned rows (D*size and stride*size % 16 == 0).*/
+/* positions : int32 [B], the slot to write (= cache length before the step).*/
+/*             Out-of-table positions or page numbers are skipped and flagged.*/
+/* ------------------------------------------------------------------------ */
+df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_stride_b,
+                             void* k_cache, void* v_cache, const int32_t* block_table,
+                             int max_blocks_per_seq, const int32_t* positions, int B, int Hkv,
+                             int D, int block_size, int num_blocks, int dtype,
+                             int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Grouped shared-weight projection (tcgen05 tensor cores, TMEM accumulator).*/
+/*                                                                           */
+/* Pages "Sintesi Tecnica" ("Architettura Core": both flows share every      */
+/* attention, MLP and output matrix; "Costi di Inferenza": grouped decode     */
+/* reads the unique weights once) and the jumtra.com summary ("提案手法の詳細").*/
+/* Both flows' rows multiply the same bf16 weight in ONE GEMM:               */
+/*   x = [m_primary primary rows ; m_aux auxiliary rows] (bf16 [M][K], row   */
+/*   stride ldx), w = bf16 [N][K] (row stride K), fp32 accumulation.          */
+/* Auxiliary rows are stored only for output columns < n_aux (n_aux = N:     */
+/* all); e.g. the aux flow needs only the Q part of a fused QKV projection.   */
+/* Epilogues (the coupling reads are one way, primary -> auxiliary; aux row  */
+/* m_primary + j is paired with primary row j, so m_aux must be m_primary    */
+/* when a coupling vector is given):                                          */
+/*  DF_EPI_NONE     : y[M][N] = x w^T; coupling and residual must be NULL.   */
+/*  DF_EPI_SWIGLU   : w = [W_gate (F rows) ; W_up (F rows)], N = 2F;          */
+/*                    y[M][F] = SiLU(x W_gate^T) * (x W_up^T), and aux rows   */
+/*                    add coupling[n] * y_primary[j][n] (b_l; NULL = none).    */
+/*  DF_EPI_RESIDUAL : y[M][N] = residual + x w^T, and aux rows add            */
+/*                    coupling[n] * (x w^T)[j][n] before the residual (c_l).   */
+/* y and residual may alias (in-place residual add). All bf16.               */
+/* Supported: M = m_primary + m_aux in [1, 128]; K % 64 == 0; N % 128 == 0    */
+/* (SWIGLU: F % 64 == 0); ldx, ldy, ldr multiples of 8 elements; x, w        */
+/* 16-byte aligned. workspace: >= dualflow_grouped_proj_workspace_size(...)  */
+/* bytes, 256-byte aligned, ZEROED before its first use (it holds tile       */
+/* counters that each call leaves at zero again).                            */
+/* ------------------------------------------------------------------------ */
+size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int epilogue);
+df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
+                                const void* w, int N, int K, int n_aux, void* y, int64_t ldy,
+                                int epilogue, const void* coupling, const void* residual,
+                                int64_t ldr, void* workspace, size_t workspace_bytes,
+                                int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Row RMS normalisation (layer step, pre-attention and pre-MLP).            */
+/*                                                                           */
+/* y[r][:] = x[r][:] / sqrt(mean(x[r][:]^2) + eps) * gain[:] (gain NULL = 1), */
+/* fp32 arithmetic, bf16 in and out. The pages name no normalisation; the    */
+/* layer step reads the "Dense LLaMA" family of the summary's "Contributi    */
+/* Chiave" as pre-norm RMSNorm. cols % 8 == 0; rows 16-byte aligned.          */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_rmsnorm(const void* x, int64_t ldx, const void* gain, void* y, int64_t ldy,
+                           int rows, int cols, float eps, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUALFLOW_H */

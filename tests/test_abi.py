@@ -1,0 +1,130 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every
+symbol the header declares, and rejects invalid arguments with the documented
+status BEFORE touching the device (no test here can launch a kernel: every
+call below carries at least one invalid argument)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from dual_flow_transformer_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dualflow.h")
+
+FAKE = 0x7f0000000000  # 4 KiB-aligned fake device address (never dereferenced)
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dualflow_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return L.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in L.SIGNATURES, "binding lacks a signature for " + n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dualflow_abi_version() == 1
+    for s in range(7):
+        assert lib.dualflow_status_string(s).decode().startswith("DF_")
+    assert lib.dualflow_status_string(99)
+
+
+def _attn(lib, **over):
+    a = dict(q1=FAKE, q2raw=FAKE, a=FAKE, qs=0, kc=FAKE, vc=FAKE, tbl=FAKE, mbps=4, sl=FAKE,
+             maxlen=200, o1=FAKE, o2=FAKE, os=0, B=2, Hq=8, Hkv=2, D=128, bs=64, nb=8,
+             scale=0.0, dtype=L.DF_BF16, ns=0, ws=FAKE, wsb=1 << 30, err=None, stream=None)
+    a.update(over)
+    return lib.dualflow_decode_attn(a["q1"], a["q2raw"], a["a"], a["qs"], a["kc"], a["vc"], a["tbl"],
+                                    a["mbps"], a["sl"], a["maxlen"], a["o1"], a["o2"], a["os"],
+                                    a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["nb"], a["scale"],
+                                    a["dtype"], a["ns"], a["ws"], a["wsb"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q1=None), L.DF_ERR_NULL),
+    (dict(kc=None), L.DF_ERR_NULL),
+    (dict(tbl=None), L.DF_ERR_NULL),
+    (dict(o1=None, o2=None), L.DF_ERR_NULL),
+    (dict(o1=None, q2raw=None), L.DF_ERR_NULL),
+    (dict(Hq=6, Hkv=4), L.DF_ERR_SHAPE),
+    (dict(B=0), L.DF_ERR_SHAPE),
+    (dict(maxlen=0), L.DF_ERR_SHAPE),
+    (dict(maxlen=257), L.DF_ERR_SHAPE),          # above max_blocks_per_seq * 64
+    (dict(qs=100), L.DF_ERR_SHAPE),              # smaller than Hq * D
+    (dict(ns=-1), L.DF_ERR_SHAPE),
+    (dict(D=96), L.DF_ERR_UNSUPPORTED),
+    (dict(bs=32, maxlen=100), L.DF_ERR_UNSUPPORTED),
+    (dict(Hq=16, Hkv=2), L.DF_ERR_UNSUPPORTED),  # 8 query rows per KV head and flow
+    (dict(dtype=7), L.DF_ERR_UNSUPPORTED),
+    (dict(q1=FAKE + 2), L.DF_ERR_ALIGN),
+    (dict(kc=FAKE + 8), L.DF_ERR_ALIGN),
+    (dict(qs=1025), L.DF_ERR_ALIGN),
+    (dict(ws=None, ns=4), L.DF_ERR_WORKSPACE),
+    (dict(wsb=16, ns=4), L.DF_ERR_WORKSPACE),
+    (dict(ws=FAKE + 16, ns=4), L.DF_ERR_WORKSPACE),
+])
+def test_decode_attn_rejects_invalid_arguments(lib, over, status):
+    assert _attn(lib, **over) == status
+
+
+def test_decode_attn_plan(lib):
+    ns = lib.dualflow_decode_attn_num_splits
+    ws = lib.dualflow_decode_attn_workspace_size
+    assert ns(1, 2, 129, 64, 0) >= 1
+    assert ns(1, 1, 64, 64, 5) == 1                # never more splits than pages
+    assert ns(64, 8, 4097, 64, 3) == 3
+    for B, Hkv, L_ in [(32, 32, 2048), (64, 8, 8192), (8, 8, 131072), (64, 8, 4097), (1, 2, 129)]:
+        s = ns(B, Hkv, L_, 64, 0)
+        pages = -(-L_ // 64)
+        chunk = -(-pages // s)
+        assert 1 <= s <= pages and -(-pages // chunk) == s
+        if s > 1:
+            assert ws(B, 2 * Hkv, Hkv, 128, L_, 64, 0) >= B * 2 * 2 * Hkv * s * 130 * 4
+        else:
+            assert ws(B, 2 * Hkv, Hkv, 128, L_, 64, 0) == 0
+    assert ns(0, 1, 10, 64, 0) == 0 and ws(0, 1, 1, 64, 10, 64, 0) == 0
+
+
+def _append(lib, **over):
+    a = dict(kn=FAKE, vn=FAKE, st=0, kc=FAKE, vc=FAKE, tbl=FAKE, mbps=4, pos=FAKE, B=2, Hkv=2,
+             D=128, bs=64, nb=8, dtype=L.DF_BF16, err=None, stream=None)
+    a.update(over)
+    return lib.dualflow_kv_append(a["kn"], a["vn"], a["st"], a["kc"], a["vc"], a["tbl"], a["mbps"],
+                                  a["pos"], a["B"], a["Hkv"], a["D"], a["bs"], a["nb"], a["dtype"],
+                                  a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(kn=None), L.DF_ERR_NULL),
+    (dict(pos=None), L.DF_ERR_NULL),
+    (dict(B=0), L.DF_ERR_SHAPE),
+    (dict(st=10), L.DF_ERR_SHAPE),
+    (dict(dtype=5), L.DF_ERR_UNSUPPORTED),
+    (dict(D=4), L.DF_ERR_ALIGN),               # 8-byte rows cannot use 16-byte copies
+    (dict(kc=FAKE + 4), L.DF_ERR_ALIGN),
+])
+def test_kv_append_rejects_invalid_arguments(lib, over, status):
+    assert _append(lib, **over) == status
+
+
+def test_rmsnorm_rejects_invalid_arguments(lib):
+    f = lib.dualflow_rmsnorm
+    assert f(None, 0, None, FAKE, 0, 4, 64, 1e-5, None) == L.DF_ERR_NULL
+    assert f(FAKE, 0, None, FAKE, 0, 0, 64, 1e-5, None) == L.DF_ERR_SHAPE
+    assert f(FAKE, 0, None, FAKE, 0, 4, 60, 1e-5, None) == L.DF_ERR_UNSUPPORTED
+    assert f(FAKE + 2, 0, None, FAKE, 0, 4, 64, 1e-5, None) == L.DF_ERR_ALIGN
+    assert f(FAKE, 0, None, FAKE, 0, 4, 64, -1.0, None) == L.DF_ERR_SHAPE
