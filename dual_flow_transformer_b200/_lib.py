@@ -18,6 +18,7 @@ DF_OK, DF_ERR_NULL, DF_ERR_SHAPE, DF_ERR_UNSUPPORTED, DF_ERR_WORKSPACE, DF_ERR_A
 DF_FP32, DF_BF16 = 0, 1
 DF_EPI_NONE, DF_EPI_SWIGLU, DF_EPI_RESIDUAL = 0, 1, 2
 DF_DEVERR_SEQLEN, DF_DEVERR_BLOCK, DF_DEVERR_POSITION, DF_DEVERR_TIMEOUT = 1, 2, 4, 8
+DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 _c_int, _c_i64, _c_size, _c_float, _vp = (ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
                                            ctypes.c_float, ctypes.c_void_p)
@@ -37,6 +38,10 @@ SIGNATURES = {
         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,  # B, Hq, Hkv, D, block_size, num_blocks
         _c_float, _c_int, _c_int,       # scale, dtype, num_splits
         _vp, _c_size, _vp, _vp]),       # workspace, bytes, err_flag, stream
+    "dualflow_decode_attn_noalloc": (_c_int, [
+        _vp, _vp, _vp, _c_i64, _vp, _vp, _vp, _c_int, _vp, _c_int, _vp, _vp, _c_i64,
+        _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int,
+        _vp, _vp]),                     # err_flag, stream (no workspace)
     "dualflow_kv_append": (_c_int, [
         _vp, _vp, _c_i64, _vp, _vp, _vp, _c_int, _vp,
         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),

@@ -27,6 +27,8 @@
 //    bit-identical whatever the auxiliary inputs are.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "host_util.h"
 
@@ -759,4 +761,62 @@ extern "C" df_status dualflow_decode_attn(
   cudaError_t e = (D == 64) ? attn::launch<64>(p, dtype, &tmK, &tmV, st)
                             : attn::launch<128>(p, dtype, &tmK, &tmV, st);
   return e == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ no-alloc variant
+// Some callers cannot give this library a workspace: a serving engine that has
+// handed all free device memory to its own KV-page pool before decoding
+// starts, or a plain C host program with no device allocator of its own. For
+// them the split partials live in a fixed array in the library's own device
+// memory (allocated when the module loads, held by every GPU that loads the
+// library until the process exits). Only host code needs the array's device
+// address; the name itself is a host-side stand-in.
+
+namespace df {
+namespace noalloc {
+
+static __device__ __align__(256) uint8_t g_scratch[DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_mu;
+void* g_addr[64] = {};  // device address of g_scratch, per device ordinal
+
+// Device address of the scratch array on the current device; looked up once
+// per device (with that device current) and cached.
+df_status scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return DF_ERR_CUDA;
+    g_addr[dev] = p;
+  }
+  *out = g_addr[dev];
+  return DF_OK;
+}
+
+}  // namespace noalloc
+}  // namespace df
+
+extern "C" df_status dualflow_decode_attn_noalloc(
+    const void* q1, const void* q2raw, const void* a, int64_t q_stride_b, const void* k_cache,
+    const void* v_cache, const int32_t* block_table, int max_blocks_per_seq,
+    const int32_t* seqlens, int max_seqlen, void* o1, void* o2, int64_t o_stride_b, int B, int Hq,
+    int Hkv, int D, int block_size, int num_blocks, float scale, int dtype, int num_splits,
+    int32_t* err_flag, void* stream) {
+  if (!q1 || !k_cache || !v_cache || !block_table || !seqlens) return DF_ERR_NULL;
+  if (!o1 && !(o2 && q2raw)) return DF_ERR_NULL;
+  const size_t need = dualflow_decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size,
+                                                          num_splits);
+  if (need > DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES) return DF_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const df_status st = df::noalloc::scratch_address(&scratch);
+    if (st != DF_OK) return st;
+  }
+  return dualflow_decode_attn(q1, q2raw, a, q_stride_b, k_cache, v_cache, block_table,
+                              max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq,
+                              Hkv, D, block_size, num_blocks, scale, dtype, num_splits, scratch,
+                              need > 0 ? DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES : 0, err_flag,
+                              stream);
 }

@@ -17,6 +17,8 @@
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller. The library
  *    allocates nothing and keeps no state between calls; calls are reentrant.
+ *    (One exception, dualflow_decode_attn_noalloc, uses a fixed scratch array
+ *    inside the library; its own comment below gives the rules.)
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = legacy default stream). Argument errors are detected on the host
  *    and returned BEFORE any launch. A failed launch returns DF_ERR_CUDA.
@@ -121,6 +123,40 @@ df_status dualflow_decode_attn(const void* q1, const void* q2raw, const void* a,
                                int block_size, int num_blocks, float scale, int dtype,
                                int num_splits, void* workspace, size_t workspace_bytes,
                                int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention without a caller workspace.                              */
+/*                                                                           */
+/* The paper has no counterpart: this is a deployment convenience.           */
+/* Some callers cannot allocate device memory for a workspace -- a serving    */
+/* engine that has given all free device memory to its own KV-page pool      */
+/* before decoding starts, or a plain C host program with no device          */
+/* allocator. This entry point computes exactly what dualflow_decode_attn    */
+/* computes (same arguments minus workspace/workspace_bytes, same results)   */
+/* but keeps the split partials in a fixed array inside the library's own    */
+/* device memory: DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES (16 MiB), reserved on  */
+/* every GPU that loads the library and held until the process exits. It     */
+/* never calls cudaMalloc/cudaFree or any allocating routine.                */
+/*  - A request whose workspace would exceed that size (see                  */
+/*    dualflow_decode_attn_workspace_size) returns DF_ERR_WORKSPACE before    */
+/*    any launch.                                                            */
+/*  - The first call on a device looks up the array's device address with    */
+/*    that device current (cudaGetSymbolAddress) and caches it; make that    */
+/*    first call before any stream capture. A failed lookup: DF_ERR_CUDA.    */
+/*  - All calls on a device share the one array, which keeps the last call's */
+/*    contents (nothing in it needs to start at zero: every partial that the */
+/*    combine reads is written first by the same call). Calls that overlap   */
+/*    on the GPU (different streams, no ordering) race on it: order them.    */
+/* ------------------------------------------------------------------------ */
+#define DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+df_status dualflow_decode_attn_noalloc(const void* q1, const void* q2raw, const void* a,
+                                       int64_t q_stride_b, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_table,
+                                       int max_blocks_per_seq, const int32_t* seqlens,
+                                       int max_seqlen, void* o1, void* o2, int64_t o_stride_b,
+                                       int B, int Hq, int Hkv, int D, int block_size,
+                                       int num_blocks, float scale, int dtype, int num_splits,
+                                       int32_t* err_flag, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Primary-only KV append.                                                  */
