@@ -46,6 +46,7 @@ SIGNATURES = {
         _vp, _vp, _c_i64, _vp, _vp, _vp, _c_int, _vp,
         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "dualflow_grouped_proj_workspace_size": (_c_size, [_c_int] * 4),
+    "dualflow_grouped_proj_num_launches": (_c_int, [_c_int] * 4),
     "dualflow_grouped_proj": (_c_int, [
         _vp, _c_i64, _c_int, _c_int,    # x, ldx, m_primary, m_aux
         _vp, _c_int, _c_int, _c_int,    # w, N, K, n_aux

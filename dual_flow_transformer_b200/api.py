@@ -129,8 +129,12 @@ def grouped_proj_workspace_size(M, N, K, epilogue="none") -> int:
     return _lib().dualflow_grouped_proj_workspace_size(M, N, K, EPILOGUES[epilogue])
 
 
+def grouped_proj_num_launches(M, N, K, epilogue="none") -> int:
+    return _lib().dualflow_grouped_proj_num_launches(M, N, K, EPILOGUES[epilogue])
+
+
 def new_proj_workspace(M, N, K, epilogue="none", device="cuda"):
-    """Zero-initialised workspace (its tile counters must start at zero)."""
+    """Workspace for grouped_proj (fp32 partials of split tiles)."""
     return torch.zeros(max(256, grouped_proj_workspace_size(M, N, K, epilogue)), dtype=torch.uint8,
                        device=device)
 

@@ -41,6 +41,11 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStagesBf16 = 3;            // pipeline depth of the bf16 kernel
 constexpr int kTargetCtas = 148 * 2 * 8;  // ~8 waves of 2 resident CTAs per SM
 constexpr int kMinChunkPages = 8;         // >= 512 tokens per split
+// KV pages prefetched into L2 this many pages ahead of the shared-memory ring.
+#ifndef DF_ATTN_PREFETCH_PAGES
+#define DF_ATTN_PREFETCH_PAGES 0
+#endif
+constexpr int kPrefetchPages = DF_ATTN_PREFETCH_PAGES;
 
 struct Params {
   const void* q1;
@@ -199,9 +204,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tensormap(&tmV);
       const uint64_t policy = l2_policy_evict_first();
       const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      auto prefetch_page = [&](int i) {
+        const int page = tbl[pg0 + i];
+        if (page < 0 || page >= p.num_blocks) return;
+        const int row = (page * p.Hkv + g) * kPage;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_prefetch_2d(&tmK, h * 64, row);
+          tma_prefetch_2d(&tmV, h * 64, row);
+        }
+      };
+      if (kPrefetchPages > 0)
+        for (int i = STAGES; i < ntiles && i < STAGES + kPrefetchPages; ++i) prefetch_page(i);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % STAGES;
+        if (kPrefetchPages > 0 && i + STAGES + kPrefetchPages < ntiles)
+          prefetch_page(i + STAGES + kPrefetchPages);
         if (i >= STAGES && !mbar_wait(&empty[st], ((i / STAGES) - 1) & 1)) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
           break;

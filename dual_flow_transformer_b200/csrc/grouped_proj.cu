@@ -7,18 +7,21 @@
 // ("Costi di Inferenza": no growth in the unique weights read).
 //
 // Design (sm_100a, one CTA per SM, persistent stream-K):
-//  * the whole M <= 128 rows form one UMMA M-tile; W tiles of 128 rows x 64 k
-//    (bf16, 128-byte swizzle) and the matching X tile arrive by TMA into a
-//    6-deep shared-memory ring;
-//  * one elected thread issues tcgen05.mma (kind::f16, M=128, N=128, K=16,
-//    fp32 accumulation in TMEM, two 128-column accumulators so the epilogue
+//  * the whole M <= 128 rows form one UMMA M-tile; each k-step stages a
+//    128 x 64 activation tile and a 256 x 64 weight tile (bf16, 128-byte
+//    swizzle) by TMA into a 4-deep shared-memory ring. N = 256 per MMA halves
+//    the activation bytes re-read from L2 per weight byte (with 128 columns
+//    the L2 -> SM traffic, not DRAM, capped the weight stream);
+//  * one elected thread issues tcgen05.mma (kind::f16, M=128, N=256, K=16,
+//    fp32 accumulation in TMEM, two 256-column accumulators so the epilogue
 //    of one segment overlaps the MMAs of the next) and tcgen05.commit frees
 //    ring stages and publishes accumulators;
 //  * the k-iterations of all tiles are divided evenly over the CTAs (stream-K)
-//    so every SM streams the same number of weight bytes; a tile cut between
-//    CTAs is summed by whichever of its CTAs finishes last (fp32 partials in an
-//    L2-resident workspace, a per-tile arrival counter, no waiting on other
-//    CTAs, fixed summation order -> deterministic);
+//    so every SM streams the same number of weight bytes. A tile whose
+//    k-range is cut between CTAs is published as fp32 partials (L2-resident
+//    workspace) and summed by a second, fully parallel kernel in fixed
+//    contributor order (deterministic); tiles owned by one CTA are finished
+//    straight from TMEM;
 //  * 4 epilogue warps read TMEM (tcgen05.ld 32x32b) and apply the fused
 //    epilogue: plain store, SwiGLU with the b_l coupling, or residual add with
 //    the c_l coupling. The coupling pairs auxiliary row m_primary + j with
@@ -34,24 +37,22 @@ namespace df {
 namespace gemm {
 
 constexpr int kBM = 128;           // rows per tile (all rows of both flows)
-constexpr int kBN = 128;           // accumulator columns per tile
+constexpr int kBN = 256;           // accumulator columns per tile (one N=256 MMA)
 constexpr int kBK = 64;            // k per stage (one 128-byte swizzle atom)
-constexpr int kStages = 6;
-constexpr int kTileA = kBM * kBK * 2;   // 16 KB
-constexpr int kTileB = kBN * kBK * 2;   // 16 KB
+constexpr int kStages = 4;
+constexpr int kTileA = kBM * kBK * 2;   // 16 KB of activations
+constexpr int kTileB = kBN * kBK * 2;   // 32 KB of weights
 constexpr int kStageBytes = kTileA + kTileB;
 constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA/TMEM, warps 2-5 epilogue
 constexpr int kEpiThreads = 128;
 constexpr int kMaxCtas = 148;      // one CTA per SM of a B200
+constexpr int kXRows = 64;         // coupled epilogues pair at most 64 primary rows
 constexpr int kXPitch = 33;        // floats per row of the coupling exchange buffer
-constexpr int kTmemCols = 256;     // two fp32 accumulators of 128 columns
-// Tile counters live at the start of the workspace in a region of FIXED size,
-// so one workspace can be shared by projections of different shapes.
-constexpr size_t kCounterBytes = 65536;
-constexpr int kMaxTiles = static_cast<int>(kCounterBytes / sizeof(int));
+constexpr int kTmemCols = 512;     // two fp32 accumulators of 256 columns
+constexpr int kRedThreads = 256;   // split-tile reduction: 16 rows x 16 column groups
 
 struct Params {
-  int M, m_primary, N, K, n_aux;
+  int M, m_primary, N, K, n_out, n_aux;
   int epilogue;
   int n_tiles, kblocks, ctas;
   long long total_iters;
@@ -60,8 +61,7 @@ struct Params {
   const __nv_bfloat16* coupling;
   const __nv_bfloat16* residual;
   int64_t ldr;
-  int* counters;     // [n_tiles]
-  float* partials;   // [2 * ctas][128][128]
+  float* partials;   // [2 * ctas][128][256] fp32
   int32_t* err;
   int F;             // SWIGLU: rows of W_gate (= output columns)
 };
@@ -69,8 +69,12 @@ struct Params {
 __host__ __device__ inline long long iter_begin(const Params& p, int cta) {
   return static_cast<long long>(cta) * p.total_iters / p.ctas;
 }
-__device__ inline int owner_of(const Params& p, long long it) {
+__host__ __device__ inline int owner_of(const Params& p, long long it) {
   return static_cast<int>(((it + 1) * p.ctas - 1) / p.total_iters);
+}
+// First output column of a tile and output columns per tile.
+__host__ __device__ inline int tile_col0(const Params& p, int tile) {
+  return p.epilogue == DF_EPI_SWIGLU ? tile * (kBN / 2) : tile * kBN;
 }
 
 // Descriptor of a K-major bf16 tile with 128-byte swizzle: 8-row core groups
@@ -81,7 +85,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
          (static_cast<uint64_t>(2) << 61);
 }
 
-// kind::f16 instruction descriptor: D fp32, A/B bf16, both K-major, N=128, M=128.
+// kind::f16 instruction descriptor: D fp32, A/B bf16, both K-major, N=256, M=128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                             (static_cast<uint32_t>(kBN >> 3) << 17) |
                             (static_cast<uint32_t>(kBM >> 4) << 24);
@@ -131,10 +135,11 @@ __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+template <int NV>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* src, float (&v)[NV]) {
   const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NV / 8; ++q) {
     const uint4 u = s[q];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -145,10 +150,11 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v
   }
 }
 
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+template <int NV>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NV]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NV / 8; ++q) {
     uint32_t w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -158,97 +164,74 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
   }
 }
 
-// Epilogue of one 32-column output chunk held by this thread (row `row`).
-// `val` = raw accumulator (NONE/RESIDUAL) or SiLU(gate)*up (SWIGLU).
-// Coupling: primary rows publish their values, auxiliary rows add
-// coupling[col] * value of their paired primary row.
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// Residual add (RESIDUAL epilogue) and store of NV output columns of one row,
+// honouring the output width and the auxiliary-row column limit.
+template <int NV>
+__device__ __forceinline__ void store_row(const Params& p, int row, int col0, float (&val)[NV]) {
+  if (row >= p.M || col0 >= p.n_out) return;
+  if (row >= p.m_primary && col0 >= p.n_aux) return;
+  if (p.epilogue == DF_EPI_RESIDUAL) {
+    float rv[NV];
+    load_bf16<NV>(p.residual + row * p.ldr + col0, rv);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) val[i] += rv[i];
+  }
+  store_bf16<NV>(p.y + row * p.ldy + col0, val);
+}
+
+// Epilogue of one 32-column output chunk held by this thread (row `row`) in the
+// GEMM kernel. Coupling: primary rows publish their values through shared
+// memory, auxiliary rows add coupling[col] * value of their paired primary row.
 __device__ __forceinline__ void finish_chunk(const Params& p, int row, int col0, float (&val)[32],
                                              float* xbuf) {
-  const bool coupled = p.coupling != nullptr;
-  if (coupled) {
+  if (p.coupling != nullptr) {
     if (row < p.m_primary) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) xbuf[row * kXPitch + i] = val[i];
     }
     epi_bar();
-    if (row >= p.m_primary && row < p.M) {
+    if (row >= p.m_primary && row < p.M && col0 < p.n_out) {
       float cv[32];
-      load_bf16x32(p.coupling + col0, cv);
+      load_bf16<32>(p.coupling + col0, cv);
       const float* src = xbuf + (row - p.m_primary) * kXPitch;
 #pragma unroll
       for (int i = 0; i < 32; ++i) val[i] = fmaf(cv[i], src[i], val[i]);
     }
     epi_bar();
   }
-  if (row >= p.M) return;
-  if (row >= p.m_primary && col0 >= p.n_aux) return;
-  if (p.epilogue == DF_EPI_RESIDUAL) {
-    float rv[32];
-    load_bf16x32(p.residual + row * p.ldr + col0, rv);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) val[i] += rv[i];
-  }
-  store_bf16x32(p.y + row * p.ldy + col0, val);
+  store_row<32>(p, row, col0, val);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
-
-// Source of accumulator chunks: TMEM (a tile owned by one CTA) or the fp32
-// partials of all contributing CTAs q_a..q_b summed in CTA (= k) order.
-struct ChunkSrc {
-  bool from_tmem;
-  uint32_t taddr;  // this row's TMEM address of the accumulator (column 0)
-  int tile, row, q_a, q_b;
-};
+// Epilogue of a tile whose whole k-range this CTA accumulated (TMEM source).
+__device__ void tile_epilogue_tmem(const Params& p, int tile, int row, uint32_t taddr,
+                                   float* xbuf) {
+  const int col0 = tile_col0(p, tile);
+  if (p.epilogue == DF_EPI_SWIGLU) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 64; ++c) {
+      float g[32], u[32];
+      tmem_ld32(taddr + 32 * c, g);
+      tmem_ld32(taddr + kBN / 2 + 32 * c, u);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+      finish_chunk(p, row, col0 + 32 * c, g, xbuf);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      float v[32];
+      tmem_ld32(taddr + 32 * c, v);
+      finish_chunk(p, row, col0 + 32 * c, v, xbuf);
+    }
+  }
+}
 
 __device__ __forceinline__ const float* partial_row(const Params& p, int q, int tile, int row) {
   const int first_tile = static_cast<int>(iter_begin(p, q) / p.kblocks);
   const int slot = 2 * q + (first_tile == tile ? 0 : 1);
   return p.partials + (static_cast<size_t>(slot) * kBM + row) * kBN;
-}
-
-__device__ __forceinline__ void read_chunk(const Params& p, const ChunkSrc& s, int col,
-                                           float (&v)[32]) {
-  if (s.from_tmem) {
-    tmem_ld32(s.taddr + col, v);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = 0.f;
-    for (int q = s.q_a; q <= s.q_b; ++q) {
-      const float4* src = reinterpret_cast<const float4*>(partial_row(p, q, s.tile, s.row) + col);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 f = __ldcg(src + k);
-        v[4 * k] += f.x;
-        v[4 * k + 1] += f.y;
-        v[4 * k + 2] += f.z;
-        v[4 * k + 3] += f.w;
-      }
-    }
-  }
-}
-
-// Full epilogue of a tile from the given source.
-__device__ void tile_epilogue(const Params& p, int tile, int row, const ChunkSrc& src,
-                              float* xbuf) {
-  if (p.epilogue == DF_EPI_SWIGLU) {
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      float g[32], u[32];
-      read_chunk(p, src, 32 * c, g);
-      read_chunk(p, src, 64 + 32 * c, u);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
-      finish_chunk(p, row, tile * 64 + 32 * c, g, xbuf);
-    }
-  } else {
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      read_chunk(p, src, 32 * c, v);
-      finish_chunk(p, row, tile * kBN + 32 * c, v, xbuf);
-    }
-  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -257,13 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* xbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [128][33]
-  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kBM * kXPitch);
+  float* xbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [64][33]
+  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kXRows * kXPitch);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  int* flags = reinterpret_cast<int*>(tmem_slot + 1);  // [0] timeout, [1] fixup owner
+  int* flags = reinterpret_cast<int*>(tmem_slot + 1);  // [0] timeout
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -280,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], kEpiThreads / 32);
     }
     flags[0] = 0;
-    flags[1] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -304,12 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_w = l2_policy_evict_first();  // weights: streamed once
       const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read by every CTA
       long long n = 0;  // stages issued
-      bool ok = true;
-      for (long long it = it_begin; it < it_end && ok; ++it, ++n) {
+      for (long long it = it_begin; it < it_end; ++it, ++n) {
         const int s = static_cast<int>(n % kStages);
         if (n >= kStages && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / kStages) - 1) & 1))) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
-          ok = false;
           break;
         }
         const int tile = static_cast<int>(it / KB), kb = static_cast<int>(it % KB);
@@ -318,8 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
         if (p.epilogue == DF_EPI_SWIGLU) {
-          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * 64, pol_w);
-          tma_load_2d_hint(sb + kTileB / 2, &tmW, &full[s], kb * kBK, p.F + tile * 64, pol_w);
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * (kBN / 2), pol_w);
+          tma_load_2d_hint(sb + kTileB / 2, &tmW, &full[s], kb * kBK, p.F + tile * (kBN / 2),
+                           pol_w);
         } else {
           tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * kBN, pol_w);
         }
@@ -341,7 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int acc = seg & 1;
         if (seg >= 2 && !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
-          ok = false;
           break;
         }
         tc_fence_after();
@@ -392,61 +372,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       const long long t_first = static_cast<long long>(tile) * KB;
-      const int q_a = owner_of(p, t_first);
-      const int q_b = owner_of(p, t_first + KB - 1);
-      ChunkSrc src;
-      src.from_tmem = true;
-      src.taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
-      src.tile = tile;
-      src.row = row;
-      src.q_a = q_a;
-      src.q_b = q_b;
-      if (q_a == q_b) {
-        tile_epilogue(p, tile, row, src, xbuf);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (owner_of(p, t_first) == owner_of(p, t_first + KB - 1)) {
+        tile_epilogue_tmem(p, tile, row, taddr, xbuf);
       } else {
-        // partial tile: publish this CTA's fp32 partial in its slot
-        const bool first_seg = (it == it_begin);
-        const int slot = 2 * cta + (first_seg ? 0 : 1);
-        float* part = p.partials + (static_cast<size_t>(slot) * kBM + row) * kBN;
+        // split tile: publish this CTA's fp32 partial; the reduce kernel sums them
+        float* part = p.partials + (static_cast<size_t>(2 * cta + (it == it_begin ? 0 : 1)) * kBM +
+                                    row) * kBN;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kBN / 32; ++c) {
           float v[32];
-          tmem_ld32(src.taddr + 32 * c, v);
+          tmem_ld32(taddr + 32 * c, v);
           float4* dst = reinterpret_cast<float4*>(part + 32 * c);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             __stcg(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        __threadfence();
-        epi_bar();
-        if (et == 0) {
-          const int old = atomicAdd(&p.counters[tile], 1);
-          const int last = (old == q_b - q_a);
-          if (last) atomicExch(&p.counters[tile], 0);
-          flags[1] = last;
-        }
-        epi_bar();
-        const int last = flags[1];
-        epi_bar();
-        if (last) {
-          __threadfence();
-          ChunkSrc fx;
-          fx.from_tmem = false;
-          fx.taddr = 0;
-          fx.tile = tile;
-          fx.row = row;
-          fx.q_a = q_a;
-          fx.q_b = q_b;
-          tile_epilogue(p, tile, row, fx, xbuf);
-        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
       it += seg_len;
       ++seg;
     }
@@ -463,24 +409,110 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Sum of the fp32 partials of a split tile (contributors in k order, so the
+// result is deterministic) followed by the same fused epilogue. One CTA per
+// (tile, group of 16 rows); a coupled group holds 8 primary rows and their 8
+// paired auxiliary rows so the coupling stays inside the CTA.
+__global__ void __launch_bounds__(kRedThreads) reduce_kernel(const Params p) {
+  const int tile = blockIdx.x, grp = blockIdx.y;
+  const long long t_first = static_cast<long long>(tile) * p.kblocks;
+  const int q_a = owner_of(p, t_first), q_b = owner_of(p, t_first + p.kblocks - 1);
+  if (q_a == q_b) return;  // handled by the GEMM kernel
+  __shared__ float share[8][kBN / 2 + 4];
+  const int slot16 = threadIdx.x >> 4;  // row slot 0..15
+  const int tc = threadIdx.x & 15;      // column group 0..15
+  const bool coupled = p.coupling != nullptr;
+  int row;
+  bool valid;
+  if (coupled) {
+    const int j = grp * 8 + (slot16 & 7);
+    row = slot16 < 8 ? j : p.m_primary + j;
+    valid = j < p.m_primary;
+  } else {
+    row = grp * 16 + slot16;
+    valid = row < p.M;
+  }
+  const bool swiglu = p.epilogue == DF_EPI_SWIGLU;
+  // accumulator columns read by this thread: 16 contiguous (plain) or 8 gate + 8 up (SwiGLU)
+  const int ca = swiglu ? 8 * tc : 16 * tc;
+  const int cb = swiglu ? kBN / 2 + 8 * tc : 16 * tc + 8;
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  if (valid) {
+    for (int q = q_a; q <= q_b; ++q) {
+      const float* pr = partial_row(p, q, tile, row);
+      const float4 a0 = __ldcg(reinterpret_cast<const float4*>(pr + ca));
+      const float4 a1 = __ldcg(reinterpret_cast<const float4*>(pr + ca + 4));
+      const float4 b0 = __ldcg(reinterpret_cast<const float4*>(pr + cb));
+      const float4 b1 = __ldcg(reinterpret_cast<const float4*>(pr + cb + 4));
+      acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
+      acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+      acc[8] += b0.x; acc[9] += b0.y; acc[10] += b0.z; acc[11] += b0.w;
+      acc[12] += b1.x; acc[13] += b1.y; acc[14] += b1.z; acc[15] += b1.w;
+    }
+  }
+  const int col0 = tile_col0(p, tile) + (swiglu ? 8 * tc : 16 * tc);
+  if (swiglu) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = silu_f(acc[i]) * acc[8 + i];
+    if (coupled) {
+      if (slot16 < 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) share[slot16][8 * tc + i] = v[i];
+      }
+      __syncthreads();
+      if (slot16 >= 8 && valid && col0 < p.n_out) {
+        float cv[8];
+        load_bf16<8>(p.coupling + col0, cv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = fmaf(cv[i], share[slot16 - 8][8 * tc + i], v[i]);
+      }
+    }
+    if (valid) store_row<8>(p, row, col0, v);
+  } else {
+    if (coupled) {
+      // two passes of 8 columns through the 8 x 128(+4) shared buffer
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (slot16 < 8) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) share[slot16][8 * tc + i] = acc[8 * h + i];
+        }
+        __syncthreads();
+        if (slot16 >= 8 && valid && col0 + 8 * h < p.n_out) {
+          float cv[8];
+          load_bf16<8>(p.coupling + col0 + 8 * h, cv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[8 * h + i] = fmaf(cv[i], share[slot16 - 8][8 * tc + i],
+                                                            acc[8 * h + i]);
+        }
+        __syncthreads();
+      }
+    }
+    if (valid) store_row<16>(p, row, col0, acc);
+  }
+}
+
 struct Layout {
   int n_tiles, kblocks, ctas;
   long long total;
-  size_t counters_bytes, partial_bytes;
+  size_t partial_bytes;
 };
 
 inline Layout make_layout(int N, int K, int epilogue) {
   Layout l;
-  l.n_tiles = (epilogue == DF_EPI_SWIGLU) ? N / 128 : N / kBN;
+  l.n_tiles = (epilogue == DF_EPI_SWIGLU) ? static_cast<int>(ceil_div(N / 2, kBN / 2))
+                                          : static_cast<int>(ceil_div(N, kBN));
   l.kblocks = K / kBK;
   l.total = static_cast<long long>(l.n_tiles) * l.kblocks;
   l.ctas = static_cast<int>(l.total < kMaxCtas ? l.total : kMaxCtas);
-  l.counters_bytes = kCounterBytes;
-  l.partial_bytes = static_cast<size_t>(2) * l.ctas * kBM * kBN * sizeof(float);
+  l.partial_bytes = static_cast<size_t>(2) * kMaxCtas * kBM * kBN * sizeof(float);
   return l;
 }
 
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kBM * kXPitch * 4 + 256;
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kXRows * kXPitch * 4 + 256;
 
 }  // namespace gemm
 }  // namespace df
@@ -490,7 +522,22 @@ extern "C" size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int 
   if (M < 1 || N < 1 || K < 1 || epilogue < 0 || epilogue > 2) return 0;
   const Layout l = make_layout(N, K, epilogue);
   if (l.total < 1) return 0;
-  return l.counters_bytes + l.partial_bytes;
+  return l.partial_bytes;
+}
+
+extern "C" int dualflow_grouped_proj_num_launches(int M, int N, int K, int epilogue) {
+  using namespace df::gemm;
+  if (M < 1 || N < 1 || K < 1 || epilogue < 0 || epilogue > 2) return 0;
+  const Layout l = make_layout(N, K, epilogue);
+  if (l.total < 1) return 0;
+  Params p{};
+  p.total_iters = l.total;
+  p.ctas = l.ctas;
+  for (int t = 0; t < l.n_tiles; ++t) {
+    const long long f = static_cast<long long>(t) * l.kblocks;
+    if (owner_of(p, f) != owner_of(p, f + l.kblocks - 1)) return 2;
+  }
+  return 1;
 }
 
 extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
@@ -510,7 +557,7 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   if (coupling && m_aux != m_primary) return DF_ERR_SHAPE;
   if (M > kBM) return DF_ERR_UNSUPPORTED;
   if (K % kBK != 0) return DF_ERR_UNSUPPORTED;
-  if (epilogue == DF_EPI_SWIGLU ? (N % 128 != 0) : (N % kBN != 0)) return DF_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return DF_ERR_UNSUPPORTED;  // SWIGLU: F = N / 2 must be a multiple of 64
   const int n_out = epilogue == DF_EPI_SWIGLU ? N / 2 : N;
   if (n_aux < 0 || n_aux > n_out) return DF_ERR_SHAPE;
   if (n_aux % 32 != 0 && n_aux != n_out) return DF_ERR_UNSUPPORTED;
@@ -521,8 +568,8 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
       (coupling && !aligned(coupling, 16)))
     return DF_ERR_ALIGN;
   const Layout l = make_layout(N, K, epilogue);
-  if (l.n_tiles > kMaxTiles) return DF_ERR_UNSUPPORTED;
-  const size_t need = l.counters_bytes + l.partial_bytes;
+  if (l.n_tiles > 65535) return DF_ERR_UNSUPPORTED;
+  const size_t need = l.partial_bytes;
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DF_ERR_WORKSPACE;
 
   Params p{};
@@ -531,6 +578,7 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   p.N = N;
   p.K = K;
   p.n_aux = n_aux;
+  p.n_out = n_out;
   p.epilogue = epilogue;
   p.n_tiles = l.n_tiles;
   p.kblocks = l.kblocks;
@@ -541,8 +589,7 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   p.coupling = static_cast<const __nv_bfloat16*>(coupling);
   p.residual = static_cast<const __nv_bfloat16*>(residual);
   p.ldr = lr;
-  p.counters = static_cast<int*>(workspace);
-  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + l.counters_bytes);
+  p.partials = static_cast<float*>(workspace);
   p.err = err_flag;
   p.F = N / 2;
 
@@ -551,7 +598,7 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
                            static_cast<uint64_t>(lx) * 2, kBM, kBK) ||
       !encode_tmap_bf16_2d(&tmW, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
                            static_cast<uint64_t>(K) * 2,
-                           epilogue == DF_EPI_SWIGLU ? 64 : kBN, kBK))
+                           epilogue == DF_EPI_SWIGLU ? kBN / 2 : kBN, kBK))
     return DF_ERR_CUDA;
   static bool attr_set = false;
   if (!attr_set) {
@@ -560,7 +607,18 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
       return DF_ERR_CUDA;
     attr_set = true;
   }
-  grouped_proj_kernel<<<l.ctas, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmX, tmW,
-                                                                                            p);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  grouped_proj_kernel<<<l.ctas, kThreads, kSmemBytes, st>>>(tmX, tmW, p);
+  // split tiles (a k-range shared by several CTAs) are summed by a second kernel
+  bool any_split = false;
+  for (int t = 0; t < l.n_tiles && !any_split; ++t) {
+    const long long f = static_cast<long long>(t) * l.kblocks;
+    any_split = owner_of(p, f) != owner_of(p, f + l.kblocks - 1);
+  }
+  if (any_split) {
+    const int groups = coupling ? static_cast<int>(ceil_div(m_primary, 8))
+                                : static_cast<int>(ceil_div(M, 16));
+    reduce_kernel<<<dim3(l.n_tiles, groups), kRedThreads, 0, st>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
 }

@@ -28,9 +28,6 @@ import torch
 
 from . import api
 
-# Launches of our kernels per layer step: rmsnorm, qkv GEMM, append, attention
-# split (+ combine when split), W_o GEMM, rmsnorm, gate/up GEMM, down GEMM.
-
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
@@ -62,10 +59,17 @@ class DualFlowLayer:
         self.attn_ws = torch.empty(max(aw, 256), dtype=torch.uint8, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.splits = api.decode_attn_num_splits(B, Hkv, self.max_seqlen, num_splits)
+        self._gemm_launches = (
+            api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
+            + api.grouped_proj_num_launches(M, *weights["w_o"].shape, "residual")
+            + api.grouped_proj_num_launches(M, *weights["w_gu"].shape, "swiglu")
+            + api.grouped_proj_num_launches(M, *weights["w_down"].shape, "residual"))
 
     @property
     def launches_per_step(self) -> int:
-        return 8 + (1 if self.splits > 1 else 0)
+        """Kernel launches of one step: 2 norms, append, attention split (+ combine),
+        and the grouped projections (1 or 2 launches each)."""
+        return 3 + (2 if self.splits > 1 else 1) + self._gemm_launches
 
     # ------------------------------------------------------------ CUDA graphs
     def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):

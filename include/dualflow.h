@@ -201,11 +201,16 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
 /* y and residual may alias (in-place residual add). All bf16.               */
 /* Supported: M = m_primary + m_aux in [1, 128]; K % 64 == 0; N % 128 == 0    */
 /* (SWIGLU: F % 64 == 0); ldx, ldy, ldr multiples of 8 elements; x, w        */
-/* 16-byte aligned. workspace: >= dualflow_grouped_proj_workspace_size(...)  */
-/* bytes, 256-byte aligned, ZEROED before its first use (it holds tile       */
-/* counters that each call leaves at zero again).                            */
+/* 16-byte aligned; n_aux a multiple of 32 or the full output width.          */
+/* workspace: >= dualflow_grouped_proj_workspace_size(...) bytes, 256-byte    */
+/* aligned, no initial contents required; one workspace may serve            */
+/* projections of any shape issued in order on one stream. Launches: the     */
+/* GEMM kernel plus, when a tile's k-range is split over CTAs, a reduction    */
+/* kernel that sums the fp32 partials in fixed order (deterministic).         */
 /* ------------------------------------------------------------------------ */
 size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int epilogue);
+/* Number of kernel launches one dualflow_grouped_proj call makes (1 or 2). */
+int dualflow_grouped_proj_num_launches(int M, int N, int K, int epilogue);
 df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
                                 const void* w, int N, int K, int n_aux, void* y, int64_t ldy,
                                 int epilogue, const void* coupling, const void* residual,
