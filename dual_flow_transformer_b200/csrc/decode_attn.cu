@@ -175,6 +175,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
 
   if (split == 0 && g == 0 && threadIdx.x == 0) flag_len(p, b);
   const int L = attended_len(p, b);
@@ -490,6 +492,8 @@ __global__ void __launch_bounds__(128) split_f32_kernel(const Params p) {
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int t = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (split == 0 && g == 0 && t == 0) flag_len(p, b);
   const int L = attended_len(p, b);
   const int npages = (L + kPage - 1) / kPage;
@@ -609,6 +613,8 @@ __global__ void __launch_bounds__(D) combine_kernel(const Params p) {
   constexpr float kNegInf = -INFINITY;
   const int row = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int flow = row / p.Hq, h = row % p.Hq;
+  pdl_wait();
+  pdl_trigger();
   if ((flow == 0 && !p.write1) || (flow == 1 && !p.write2)) return;
   const int L = attended_len(p, b);
   const int npages = (L + kPage - 1) / kPage;
@@ -655,9 +661,13 @@ cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUt
       if (e != cudaSuccess) return e;
       attr_set = true;
     }
-    split_bf16_kernel<D, kStagesBf16><<<grid, kThreads, smem, stream>>>(*tmK, *tmV, p);
-    if (p.num_splits > 1)
-      combine_kernel<__nv_bfloat16, D><<<dim3(2 * p.Hq, p.B), D, 0, stream>>>(p);
+    cudaError_t e = launch_pdl(split_bf16_kernel<D, kStagesBf16>, grid, dim3(kThreads), smem, stream,
+                               *tmK, *tmV, p);
+    if (e != cudaSuccess) return e;
+    if (p.num_splits > 1) {
+      e = launch_pdl(combine_kernel<__nv_bfloat16, D>, dim3(2 * p.Hq, p.B), dim3(D), 0, stream, p);
+      if (e != cudaSuccess) return e;
+    }
   } else {
     const size_t smem = f32_smem_bytes<D>();
     static bool attr_set = false;
@@ -668,8 +678,12 @@ cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUt
       if (e != cudaSuccess) return e;
       attr_set = true;
     }
-    split_f32_kernel<D><<<grid, 128, smem, stream>>>(p);
-    if (p.num_splits > 1) combine_kernel<float, D><<<dim3(2 * p.Hq, p.B), D, 0, stream>>>(p);
+    cudaError_t e = launch_pdl(split_f32_kernel<D>, grid, dim3(128), smem, stream, p);
+    if (e != cudaSuccess) return e;
+    if (p.num_splits > 1) {
+      e = launch_pdl(combine_kernel<float, D>, dim3(2 * p.Hq, p.B), dim3(D), 0, stream, p);
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaGetLastError();
 }

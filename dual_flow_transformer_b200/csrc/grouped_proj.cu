@@ -32,9 +32,13 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "grouped_proj_tiles.h"
+#include "umma.cuh"
 
 namespace df {
 namespace gemm {
+
+using namespace umma;
 
 constexpr int kBM = 128;           // rows per tile (all rows of both flows)
 constexpr int kBN = 256;           // accumulator columns per tile (one N=256 MMA)
@@ -49,7 +53,8 @@ constexpr int kMaxCtas = 148;      // one CTA per SM of a B200
 constexpr int kXRows = 64;         // coupled epilogues pair at most 64 primary rows
 constexpr int kXPitch = 33;        // floats per row of the coupling exchange buffer
 constexpr int kTmemCols = 512;     // two fp32 accumulators of 256 columns
-constexpr int kRedThreads = 256;   // split-tile reduction: 16 rows x 16 column groups
+constexpr int kRedThreads = 512;   // split-tile reduction: 16 rows x 32 column groups
+constexpr int kStgPitch = 36;      // floats per row of a warp's 32 x 32 staging tile
 
 struct Params {
   int M, m_primary, N, K, n_out, n_aux;
@@ -77,94 +82,12 @@ __host__ __device__ inline int tile_col0(const Params& p, int tile) {
   return p.epilogue == DF_EPI_SWIGLU ? tile * (kBN / 2) : tile * kBN;
 }
 
-// Descriptor of a K-major bf16 tile with 128-byte swizzle: 8-row core groups
-// 1024 bytes apart (stride byte offset), leading offset unused (1), version 1.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
-         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-         (static_cast<uint64_t>(2) << 61);
-}
-
 // kind::f16 instruction descriptor: D fp32, A/B bf16, both K-major, N=256, M=128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            (static_cast<uint32_t>(kBN >> 3) << 17) |
-                            (static_cast<uint32_t>(kBM >> 4) << 24);
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  __syncwarp();
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
+constexpr uint32_t kIdesc = umma::make_idesc(kBM, kBN);
 
 __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
 }
-
-template <int NV>
-__device__ __forceinline__ void load_bf16(const __nv_bfloat16* src, float (&v)[NV]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int q = 0; q < NV / 8; ++q) {
-    const uint4 u = s[q];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[q * 8 + 2 * k] = bf16_bits_to_float(static_cast<uint16_t>(w[k] & 0xffffu));
-      v[q * 8 + 2 * k + 1] = bf16_bits_to_float(static_cast<uint16_t>(w[k] >> 16));
-    }
-  }
-}
-
-template <int NV>
-__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NV]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < NV / 8; ++q) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      w[k] = pack_bf16x2(__float2bfloat16_rn(v[q * 8 + 2 * k]),
-                         __float2bfloat16_rn(v[q * 8 + 2 * k + 1]));
-    d[q] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
 // Residual add (RESIDUAL epilogue) and store of NV output columns of one row,
 // honouring the output width and the auxiliary-row column limit.
@@ -181,11 +104,37 @@ __device__ __forceinline__ void store_row(const Params& p, int row, int col0, fl
   store_bf16<NV>(p.y + row * p.ldy + col0, val);
 }
 
-// Epilogue of one 32-column output chunk held by this thread (row `row`) in the
-// GEMM kernel. Coupling: primary rows publish their values through shared
-// memory, auxiliary rows add coupling[col] * value of their paired primary row.
-__device__ __forceinline__ void finish_chunk(const Params& p, int row, int col0, float (&val)[32],
-                                             float* xbuf) {
+// A warp holds a 32 x 32 fp32 block: lane = row (32 rows of its TMEM quarter),
+// registers = 32 consecutive columns. Stage it through shared memory so that
+// global stores are row-contiguous: each store instruction then covers 4 rows
+// x 32 columns (8 lanes per row). Returns, per lane, 8 groups of 4 columns.
+__device__ __forceinline__ void stage_block(const float (&v)[32], float* stg, int lane) {
+  float4* srow = reinterpret_cast<float4*>(stg + lane * kStgPitch);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) srow[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  __syncwarp();
+}
+
+// fp32 partial of one 32-column chunk, coalesced (streamed to L2).
+__device__ __forceinline__ void write_partial_chunk(const float (&v)[32], float* stg, float* slot,
+                                                    int quarter, int c, int lane) {
+  stage_block(v, stg, lane);
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int rl = rr * 4 + (lane >> 3), cg = (lane & 7) * 4;
+    const float4 f = *reinterpret_cast<const float4*>(stg + rl * kStgPitch + cg);
+    __stcg(reinterpret_cast<float4*>(slot + (quarter * 32 + rl) * kBN + 32 * c + cg), f);
+  }
+  __syncwarp();
+}
+
+// Epilogue of one 32-column output chunk of this warp's 32 rows (lane = row in
+// `val`). Coupling: primary rows publish their values through shared memory,
+// auxiliary rows add coupling[col] * value of their paired primary row. Then
+// residual add and bf16 store, row-contiguous after the shared-memory transpose.
+__device__ __forceinline__ void finish_chunk(const Params& p, int quarter, int lane, int col0,
+                                             float (&val)[32], float* xbuf, float* stg) {
+  const int row = quarter * 32 + lane;
   if (p.coupling != nullptr) {
     if (row < p.m_primary) {
 #pragma unroll
@@ -201,29 +150,50 @@ __device__ __forceinline__ void finish_chunk(const Params& p, int row, int col0,
     }
     epi_bar();
   }
-  store_row<32>(p, row, col0, val);
+  stage_block(val, stg, lane);
+  if (col0 < p.n_out) {
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const int rl = rr * 4 + (lane >> 3), cg = (lane & 7) * 4;
+      const int r = quarter * 32 + rl;
+      if (r >= p.M || (r >= p.m_primary && col0 >= p.n_aux)) continue;
+      const float4 f = *reinterpret_cast<const float4*>(stg + rl * kStgPitch + cg);
+      float o[4] = {f.x, f.y, f.z, f.w};
+      if (p.epilogue == DF_EPI_RESIDUAL) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p.residual + r * p.ldr + col0 + cg);
+        o[0] += bf16_bits_to_float(static_cast<uint16_t>(u.x & 0xffffu));
+        o[1] += bf16_bits_to_float(static_cast<uint16_t>(u.x >> 16));
+        o[2] += bf16_bits_to_float(static_cast<uint16_t>(u.y & 0xffffu));
+        o[3] += bf16_bits_to_float(static_cast<uint16_t>(u.y >> 16));
+      }
+      *reinterpret_cast<uint2*>(p.y + r * p.ldy + col0 + cg) =
+          make_uint2(pack_bf16x2(__float2bfloat16_rn(o[0]), __float2bfloat16_rn(o[1])),
+                     pack_bf16x2(__float2bfloat16_rn(o[2]), __float2bfloat16_rn(o[3])));
+    }
+  }
+  __syncwarp();
 }
 
 // Epilogue of a tile whose whole k-range this CTA accumulated (TMEM source).
-__device__ void tile_epilogue_tmem(const Params& p, int tile, int row, uint32_t taddr,
-                                   float* xbuf) {
+__device__ void tile_epilogue_tmem(const Params& p, int tile, int quarter, int lane, uint32_t taddr,
+                                   float* xbuf, float* stg) {
   const int col0 = tile_col0(p, tile);
   if (p.epilogue == DF_EPI_SWIGLU) {
 #pragma unroll 1
     for (int c = 0; c < kBN / 64; ++c) {
       float g[32], u[32];
-      tmem_ld32(taddr + 32 * c, g);
-      tmem_ld32(taddr + kBN / 2 + 32 * c, u);
+      tmem_ld<32>(taddr + 32 * c, g);
+      tmem_ld<32>(taddr + kBN / 2 + 32 * c, u);
 #pragma unroll
       for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
-      finish_chunk(p, row, col0 + 32 * c, g, xbuf);
+      finish_chunk(p, quarter, lane, col0 + 32 * c, g, xbuf, stg);
     }
   } else {
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
-      tmem_ld32(taddr + 32 * c, v);
-      finish_chunk(p, row, col0 + 32 * c, v, xbuf);
+      tmem_ld<32>(taddr + 32 * c, v);
+      finish_chunk(p, quarter, lane, col0 + 32 * c, v, xbuf, stg);
     }
   }
 }
@@ -241,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   float* xbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [64][33]
-  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kXRows * kXPitch);
+  float* stg_all = xbuf + kXRows * kXPitch;  // 4 epilogue warps x [32][36] (16-byte aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg_all + 4 * 32 * kStgPitch);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
@@ -277,6 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int KB = p.kblocks;
+  // set-up above overlaps the previous kernel; global memory only from here on
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -354,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue warps
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-    const int row = quarter * 32 + lane;
     const int et = threadIdx.x - 64;  // 0..127
+    float* stg = stg_all + (warp - 2) * 32 * kStgPitch;
     int seg = 0;
     long long it = it_begin;
     while (it < it_end) {
@@ -375,19 +349,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       const long long t_first = static_cast<long long>(tile) * KB;
       if (owner_of(p, t_first) == owner_of(p, t_first + KB - 1)) {
-        tile_epilogue_tmem(p, tile, row, taddr, xbuf);
+        tile_epilogue_tmem(p, tile, quarter, lane, taddr, xbuf, stg);
       } else {
         // split tile: publish this CTA's fp32 partial; the reduce kernel sums them
-        float* part = p.partials + (static_cast<size_t>(2 * cta + (it == it_begin ? 0 : 1)) * kBM +
-                                    row) * kBN;
+        float* slot =
+            p.partials + static_cast<size_t>(2 * cta + (it == it_begin ? 0 : 1)) * kBM * kBN;
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
           float v[32];
-          tmem_ld32(taddr + 32 * c, v);
-          float4* dst = reinterpret_cast<float4*>(part + 32 * c);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            __stcg(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+          tmem_ld<32>(taddr + 32 * c, v);
+          write_partial_chunk(v, stg, slot, quarter, c, lane);
         }
       }
       tc_fence_before();
@@ -411,16 +382,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Sum of the fp32 partials of a split tile (contributors in k order, so the
 // result is deterministic) followed by the same fused epilogue. One CTA per
-// (tile, group of 16 rows); a coupled group holds 8 primary rows and their 8
-// paired auxiliary rows so the coupling stays inside the CTA.
-__global__ void __launch_bounds__(kRedThreads) reduce_kernel(const Params p) {
+// (tile, group of 16 rows), 512 threads = 16 rows x 32 column groups, two CTAs
+// per SM; each thread keeps up to 4 contributors' loads in flight. A coupled group holds 8
+// primary rows and their 8 paired auxiliary rows so the coupling stays inside
+// the CTA.
+__global__ void __launch_bounds__(kRedThreads, 2) reduce_kernel(const Params p) {
   const int tile = blockIdx.x, grp = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
   const long long t_first = static_cast<long long>(tile) * p.kblocks;
   const int q_a = owner_of(p, t_first), q_b = owner_of(p, t_first + p.kblocks - 1);
   if (q_a == q_b) return;  // handled by the GEMM kernel
-  __shared__ float share[8][kBN / 2 + 4];
-  const int slot16 = threadIdx.x >> 4;  // row slot 0..15
-  const int tc = threadIdx.x & 15;      // column group 0..15
+  __shared__ float share[8][kBN];
+  const int slot16 = threadIdx.x >> 5;  // row slot 0..15
+  const int c = threadIdx.x & 31;       // column group 0..31
   const bool coupled = p.coupling != nullptr;
   int row;
   bool valid;
@@ -433,65 +408,69 @@ __global__ void __launch_bounds__(kRedThreads) reduce_kernel(const Params p) {
     valid = row < p.M;
   }
   const bool swiglu = p.epilogue == DF_EPI_SWIGLU;
-  // accumulator columns read by this thread: 16 contiguous (plain) or 8 gate + 8 up (SwiGLU)
-  const int ca = swiglu ? 8 * tc : 16 * tc;
-  const int cb = swiglu ? kBN / 2 + 8 * tc : 16 * tc + 8;
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  // accumulator columns of this thread: 8 contiguous (plain) or 4 gate + 4 up (SwiGLU)
+  const int ca = swiglu ? 4 * c : 8 * c;
+  const int cb = swiglu ? kBN / 2 + 4 * c : 8 * c + 4;
+  float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
   if (valid) {
-    for (int q = q_a; q <= q_b; ++q) {
-      const float* pr = partial_row(p, q, tile, row);
-      const float4 a0 = __ldcg(reinterpret_cast<const float4*>(pr + ca));
-      const float4 a1 = __ldcg(reinterpret_cast<const float4*>(pr + ca + 4));
-      const float4 b0 = __ldcg(reinterpret_cast<const float4*>(pr + cb));
-      const float4 b1 = __ldcg(reinterpret_cast<const float4*>(pr + cb + 4));
-      acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
-      acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
-      acc[8] += b0.x; acc[9] += b0.y; acc[10] += b0.z; acc[11] += b0.w;
-      acc[12] += b1.x; acc[13] += b1.y; acc[14] += b1.z; acc[15] += b1.w;
+    for (int q0 = q_a; q0 <= q_b; q0 += 4) {
+      float4 va[4], vb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (q0 + i <= q_b) {
+          const float* pr = partial_row(p, q0 + i, tile, row);
+          va[i] = __ldcg(reinterpret_cast<const float4*>(pr + ca));
+          vb[i] = __ldcg(reinterpret_cast<const float4*>(pr + cb));
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (q0 + i <= q_b) {
+          sa.x += va[i].x; sa.y += va[i].y; sa.z += va[i].z; sa.w += va[i].w;
+          sb.x += vb[i].x; sb.y += vb[i].y; sb.z += vb[i].z; sb.w += vb[i].w;
+        }
+      }
     }
   }
-  const int col0 = tile_col0(p, tile) + (swiglu ? 8 * tc : 16 * tc);
   if (swiglu) {
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = silu_f(acc[i]) * acc[8 + i];
+    float v[4] = {silu_f(sa.x) * sb.x, silu_f(sa.y) * sb.y, silu_f(sa.z) * sb.z,
+                  silu_f(sa.w) * sb.w};
+    const int col0 = tile_col0(p, tile) + 4 * c;
     if (coupled) {
       if (slot16 < 8) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) share[slot16][8 * tc + i] = v[i];
+        for (int i = 0; i < 4; ++i) share[slot16][4 * c + i] = v[i];
+      }
+      __syncthreads();
+      if (slot16 >= 8 && valid && col0 < p.n_out) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p.coupling + col0);
+        const float cv[4] = {bf16_bits_to_float(u.x & 0xffffu), bf16_bits_to_float(u.x >> 16),
+                             bf16_bits_to_float(u.y & 0xffffu), bf16_bits_to_float(u.y >> 16)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = fmaf(cv[i], share[slot16 - 8][4 * c + i], v[i]);
+      }
+    }
+    if (!valid || row >= p.M || col0 >= p.n_out || (row >= p.m_primary && col0 >= p.n_aux)) return;
+    const uint2 out = make_uint2(pack_bf16x2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                                 pack_bf16x2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+    *reinterpret_cast<uint2*>(p.y + row * p.ldy + col0) = out;
+  } else {
+    float v[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+    const int col0 = tile_col0(p, tile) + 8 * c;
+    if (coupled) {
+      if (slot16 < 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) share[slot16][8 * c + i] = v[i];
       }
       __syncthreads();
       if (slot16 >= 8 && valid && col0 < p.n_out) {
         float cv[8];
         load_bf16<8>(p.coupling + col0, cv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = fmaf(cv[i], share[slot16 - 8][8 * tc + i], v[i]);
+        for (int i = 0; i < 8; ++i) v[i] = fmaf(cv[i], share[slot16 - 8][8 * c + i], v[i]);
       }
     }
     if (valid) store_row<8>(p, row, col0, v);
-  } else {
-    if (coupled) {
-      // two passes of 8 columns through the 8 x 128(+4) shared buffer
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (slot16 < 8) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) share[slot16][8 * tc + i] = acc[8 * h + i];
-        }
-        __syncthreads();
-        if (slot16 >= 8 && valid && col0 + 8 * h < p.n_out) {
-          float cv[8];
-          load_bf16<8>(p.coupling + col0 + 8 * h, cv);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[8 * h + i] = fmaf(cv[i], share[slot16 - 8][8 * tc + i],
-                                                            acc[8 * h + i]);
-        }
-        __syncthreads();
-      }
-    }
-    if (valid) store_row<16>(p, row, col0, acc);
   }
 }
 
@@ -512,7 +491,8 @@ inline Layout make_layout(int N, int K, int epilogue) {
   return l;
 }
 
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kXRows * kXPitch * 4 + 256;
+constexpr size_t kSmemBytes =
+    1024 + kStages * kStageBytes + kXRows * kXPitch * 4 + 4 * 32 * kStgPitch * 4 + 256;
 
 }  // namespace gemm
 }  // namespace df
@@ -528,6 +508,7 @@ extern "C" size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int 
 extern "C" int dualflow_grouped_proj_num_launches(int M, int N, int K, int epilogue) {
   using namespace df::gemm;
   if (M < 1 || N < 1 || K < 1 || epilogue < 0 || epilogue > 2) return 0;
+  if (df::tgemm::planned_launches(M, N, K, epilogue)) return 1;
   const Layout l = make_layout(N, K, epilogue);
   if (l.total < 1) return 0;
   Params p{};
@@ -593,6 +574,15 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   p.err = err_flag;
   p.F = N / 2;
 
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    // tile-parallel / cluster split-K plan when it is modelled to be faster
+    tgemm::Request rq{x, lx, m_primary, m_aux, w, N, K, n_aux, y, ly, epilogue, coupling,
+                      residual, lr, err_flag, st};
+    const int launched = tgemm::launch_if_better(rq);
+    if (launched < 0) return DF_ERR_CUDA;
+    if (launched > 0) return DF_OK;
+  }
   CUtensorMap tmX, tmW;
   if (!encode_tmap_bf16_2d(&tmX, x, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                            static_cast<uint64_t>(lx) * 2, kBM, kBK) ||
@@ -607,8 +597,9 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
       return DF_ERR_CUDA;
     attr_set = true;
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  grouped_proj_kernel<<<l.ctas, kThreads, kSmemBytes, st>>>(tmX, tmW, p);
+  if (launch_pdl(grouped_proj_kernel, dim3(l.ctas), dim3(kThreads), kSmemBytes, st, tmX, tmW, p) !=
+      cudaSuccess)
+    return DF_ERR_CUDA;
   // split tiles (a k-range shared by several CTAs) are summed by a second kernel
   bool any_split = false;
   for (int t = 0; t < l.n_tiles && !any_split; ++t) {
@@ -618,7 +609,9 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   if (any_split) {
     const int groups = coupling ? static_cast<int>(ceil_div(m_primary, 8))
                                 : static_cast<int>(ceil_div(M, 16));
-    reduce_kernel<<<dim3(l.n_tiles, groups), kRedThreads, 0, st>>>(p);
+    if (launch_pdl(reduce_kernel, dim3(l.n_tiles, groups), dim3(kRedThreads), 0, st, p) !=
+        cudaSuccess)
+      return DF_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
 }

@@ -1,0 +1,693 @@
+// Grouped shared-weight projection, tile-parallel / cluster split-K plan.
+//
+// Same product as the stream-K kernel (both flows' rows times one shared bf16
+// weight, fp32 accumulation in TMEM, fused SwiGLU/residual/coupling epilogues;
+// "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura Core" and
+// "Meccanismi Chiave"), but every output tile is finished without fp32
+// partials in global memory:
+//  * the tile width BN (the MMA's N, a multiple of 16 up to 256) is chosen per
+//    shape so that the tile count fills the 148 SMs; with C = 1 each CTA owns
+//    whole tiles (persistent over tiles, two TMEM accumulators);
+//  * when there are too few tiles, a thread-block cluster of C <= 8 CTAs
+//    splits one tile's k-range. Each CTA parks its fp32 accumulator in its own
+//    shared memory, and after a cluster barrier every CTA sums its share of the
+//    tile's rows across the cluster through distributed shared memory (in rank
+//    order, so the result is deterministic), applies the epilogue and stores.
+// The producer/MMA/epilogue warp roles, the TMA ring and the bounded waits are
+// as in the stream-K kernel.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "grouped_proj_tiles.h"
+#include "host_util.h"
+#include "umma.cuh"
+
+namespace df {
+namespace tgemm {
+
+using namespace umma;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kMaxStages = 8;
+constexpr int kXRows = 64;
+constexpr int kXPitch = 33;
+constexpr int kStgPitch = 36;
+constexpr int kTileX = kBM * kBK * 2;  // 16 KB activation tile per stage
+constexpr int kRingBytes = 196 * 1024;
+constexpr int kMaxCluster = 8;
+constexpr int kSms = 148;
+constexpr int kMaxOut = 256;  // output columns per tile (coupling prefetch buffer)
+constexpr size_t kSmemBytes =
+    1024 + kRingBytes + kXRows * kXPitch * 4 + 4 * 32 * kStgPitch * 4 + kMaxOut * 4 + 256;
+
+struct Params {
+  int M, m_primary, n_out, n_aux, epilogue;
+  int kblocks, BN, half, out_per_tile, n_tiles, C, stages, stage_bytes;
+  uint32_t idesc;
+  int F;
+  __nv_bfloat16* y;
+  int64_t ldy;
+  const __nv_bfloat16* coupling;
+  const __nv_bfloat16* residual;
+  int64_t ldr;
+  int32_t* err;
+};
+
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+// Distributed-shared-memory load. No memory clobber: ordering against the
+// cluster barrier comes from both being volatile asm, and leaving the clobber
+// out lets independent loads be issued back to back.
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ bool store_ok(const Params& p, int row, int col) {
+  return row < p.M && col < p.n_out && !(row >= p.m_primary && col >= p.n_aux);
+}
+
+// Epilogue of one chunk of W output columns held row-wise (lane = row of this
+// warp's TMEM quarter): coupling through shared memory, then residual add and
+// bf16 store. W = 32 goes through the warp's staging tile so that stores are
+// row-contiguous; W = 8 (tile tails) stores per row.
+template <int W>
+__device__ __forceinline__ void finish_chunk(const Params& p, int quarter, int lane, int col0,
+                                             float (&val)[W], float* xbuf, float* stg,
+                                             const float* cpl) {
+  const int row = quarter * 32 + lane;
+  if (p.coupling != nullptr) {
+    if (row < p.m_primary) {
+#pragma unroll
+      for (int i = 0; i < W; ++i) xbuf[row * kXPitch + i] = val[i];
+    }
+    epi_bar();
+    if (row >= p.m_primary && row < p.M) {
+      const float* src = xbuf + (row - p.m_primary) * kXPitch;
+#pragma unroll
+      for (int i = 0; i < W; ++i) val[i] = fmaf(cpl[i], src[i], val[i]);
+    }
+    epi_bar();
+  }
+  if constexpr (W == 32) {
+    float4* srow = reinterpret_cast<float4*>(stg + lane * kStgPitch);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      srow[i] = make_float4(val[4 * i], val[4 * i + 1], val[4 * i + 2], val[4 * i + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const int rl = rr * 4 + (lane >> 3), cg = (lane & 7) * 4;
+      const int r = quarter * 32 + rl;
+      if (!store_ok(p, r, col0 + cg)) continue;
+      const float4 f = *reinterpret_cast<const float4*>(stg + rl * kStgPitch + cg);
+      float o[4] = {f.x, f.y, f.z, f.w};
+      if (p.epilogue == DF_EPI_RESIDUAL) {
+        float rv[4];
+        load_bf16x4(p.residual + r * p.ldr + col0 + cg, rv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] += rv[i];
+      }
+      store_bf16x4(p.y + r * p.ldy + col0 + cg, o);
+    }
+    __syncwarp();
+  } else {
+    if (store_ok(p, row, col0)) {
+      if (p.epilogue == DF_EPI_RESIDUAL) {
+        float rv[W];
+        load_bf16<W>(p.residual + row * p.ldr + col0, rv);
+#pragma unroll
+        for (int i = 0; i < W; ++i) val[i] += rv[i];
+      }
+      store_bf16<W>(p.y + row * p.ldy + col0, val);
+    }
+  }
+}
+
+// Epilogue of a whole tile straight from TMEM (C = 1).
+__device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, uint32_t taddr,
+                              float* xbuf, float* stg, const float* cpl_s) {
+  const int col0 = tile * p.out_per_tile;
+  if (p.epilogue == DF_EPI_SWIGLU) {
+    const int H = p.half;
+    int c = 0;
+    for (; c + 32 <= H; c += 32) {
+      float g[32], u[32];
+      tmem_ld<32>(taddr + c, g);
+      tmem_ld<32>(taddr + H + c, u);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+      finish_chunk<32>(p, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
+    }
+    for (; c < H; c += 8) {
+      float g[8], u[8];
+      tmem_ld<8>(taddr + c, g);
+      tmem_ld<8>(taddr + H + c, u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) g[i] = silu_f(g[i]) * u[i];
+      finish_chunk<8>(p, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
+    }
+  } else {
+    int c = 0;
+    for (; c + 32 <= p.BN; c += 32) {
+      float v[32];
+      tmem_ld<32>(taddr + c, v);
+      finish_chunk<32>(p, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
+    }
+    for (; c < p.BN; c += 8) {
+      float v[8];
+      tmem_ld<8>(taddr + c, v);
+      finish_chunk<8>(p, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
+    }
+  }
+}
+
+// C > 1: this CTA's share of the tile's rows, summed over the cluster's
+// accumulators (parked in each CTA's shared memory) in rank order, then the
+// epilogue. All threads of the CTA take part, two items (4 output columns of
+// one row each) at a time with every remote load issued before any sum.
+__device__ void cluster_epilogue(const Params& p, int tile, int rank, uint32_t acc_local,
+                                 float* prim, int tid, int nthreads,
+                                 const __nv_bfloat16* res_s, const float* cpl_s) {
+  constexpr int kBatch = 2;
+  const int pitch = p.BN + 4;
+  const bool coupled = p.coupling != nullptr;
+  const bool swiglu = p.epilogue == DF_EPI_SWIGLU;
+  const bool resid = p.epilogue == DF_EPI_RESIDUAL;
+  const int opt = p.out_per_tile;
+  const int groups = opt / 4;  // 4-column groups per row
+  int r0, r1;                  // primary (or all) rows of this rank
+  if (coupled) {
+    r0 = rank * p.m_primary / p.C;
+    r1 = (rank + 1) * p.m_primary / p.C;
+  } else {
+    r0 = rank * p.M / p.C;
+    r1 = (rank + 1) * p.M / p.C;
+  }
+  const int col_base = tile * opt;
+  const int total = (r1 - r0) * groups;
+  for (int pass = 0; pass < (coupled ? 2 : 1); ++pass) {
+    const int row_off = (pass == 1 ? p.m_primary : 0) + r0;
+    for (int base = tid; base < total; base += nthreads * kBatch) {
+      float4 va[kBatch][kMaxCluster], vu[kBatch][kMaxCluster];
+      float rv[kBatch][4], cv[kBatch][4];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int item = base + b * nthreads;
+        if (item >= total) continue;
+        const int rl = item / groups, j = (item % groups) * 4;
+        const int row = row_off + rl, col = col_base + j;
+        const uint32_t off_a = acc_local + (row * pitch + j) * 4;
+        const uint32_t off_u = acc_local + (row * pitch + p.half + j) * 4;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) {
+          if (q < p.C) {
+            va[b][q] = ld_cluster_f4(map_to_rank(off_a, q));
+            if (swiglu) vu[b][q] = ld_cluster_f4(map_to_rank(off_u, q));
+          }
+        }
+        if (resid && store_ok(p, row, col)) {
+          if (res_s != nullptr) {
+            load_bf16x4(res_s + (pass * (r1 - r0) + rl) * opt + j, rv[b]);
+          } else {
+            load_bf16x4(p.residual + row * p.ldr + col, rv[b]);
+          }
+        } else {
+          rv[b][0] = rv[b][1] = rv[b][2] = rv[b][3] = 0.f;
+        }
+        if (coupled && pass == 1 && col < p.n_out) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cv[b][i] = cpl_s[j + i];
+        } else {
+          cv[b][0] = cv[b][1] = cv[b][2] = cv[b][3] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int item = base + b * nthreads;
+        if (item >= total) continue;
+        const int rl = item / groups, j = (item % groups) * 4;
+        const int row = row_off + rl, col = col_base + j;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), u = a;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) {
+          if (q < p.C) {
+            a.x += va[b][q].x; a.y += va[b][q].y; a.z += va[b][q].z; a.w += va[b][q].w;
+            if (swiglu) {
+              u.x += vu[b][q].x; u.y += vu[b][q].y; u.z += vu[b][q].z; u.w += vu[b][q].w;
+            }
+          }
+        }
+        float o[4] = {a.x, a.y, a.z, a.w};
+        if (swiglu) {
+          o[0] = silu_f(a.x) * u.x;
+          o[1] = silu_f(a.y) * u.y;
+          o[2] = silu_f(a.z) * u.z;
+          o[3] = silu_f(a.w) * u.w;
+        }
+        if (coupled && pass == 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) prim[rl * opt + j + i] = o[i];
+        }
+        if (coupled && pass == 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = fmaf(cv[b][i], prim[rl * opt + j + i], o[i]);
+        }
+        if (!store_ok(p, row, col)) continue;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] += rv[b][i];
+        store_bf16x4(p.y + row * p.ldy + col, o);
+      }
+    }
+    if (coupled && pass == 0) __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tile_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                     const __grid_constant__ CUtensorMap tmW, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* xbuf = reinterpret_cast<float*>(smem + kRingBytes);      // [64][33]
+  float* stg_all = xbuf + kXRows * kXPitch;                        // 4 x [32][36]
+  float* cpl_s = stg_all + 4 * 32 * kStgPitch;                     // [256] coupling of a tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(cpl_s + kMaxOut);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* acc_full = empty + kMaxStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* flags = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.stages;
+  const int KB = p.kblocks;
+  int tile_first, tile_stride, kb0, kb1, rank;
+  if (p.C > 1) {
+    tile_first = blockIdx.x / p.C;
+    rank = blockIdx.x % p.C;
+    tile_stride = p.n_tiles;  // one tile per cluster
+    kb0 = rank * KB / p.C;
+    kb1 = (rank + 1) * KB / p.C;
+  } else {
+    tile_first = blockIdx.x;
+    rank = 0;
+    tile_stride = gridDim.x;
+    kb0 = 0;
+    kb1 = KB;
+  }
+  const uint32_t tmem_cols = p.C > 1 ? 256u : 512u;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiThreads / 32);
+    }
+    flags[0] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmW);
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      long long n = 0;
+      bool ok = true;
+      for (int t = tile_first; t < p.n_tiles && ok; t += tile_stride) {
+        for (int kb = kb0; kb < kb1; ++kb, ++n) {
+          const int s = static_cast<int>(n % S);
+          if (n >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / S) - 1) & 1))) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * p.stage_bytes;
+          uint8_t* sb = sa + kTileX;
+          mbar_arrive_expect_tx(&full[s], p.stage_bytes);
+          tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+          if (p.epilogue == DF_EPI_SWIGLU) {
+            tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.half, pol_w);
+            tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + t * p.half, pol_w);
+          } else {
+            tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.BN, pol_w);
+          }
+        }
+      }
+      for (long long i = (n > S ? n - S : 0); i < n; ++i)
+        mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1));
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      long long n = 0;
+      int seg = 0;
+      bool ok = true;
+      for (int t = tile_first; t < p.n_tiles && ok; t += tile_stride, ++seg) {
+        const int acc = seg & 1;
+        if (seg >= 2 && !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * p.BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++n) {
+          const int s = static_cast<int>(n % S);
+          if (!mbar_wait(&full[s], static_cast<uint32_t>((n / S) & 1))) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * p.stage_bytes);
+          const uint32_t b_addr = a_addr + kTileX;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            umma_bf16(d_tmem, smem_desc(a_addr + kk * 32), smem_desc(b_addr + kk * 32), p.idesc,
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+      }
+      if (n > 0) mbar_wait(&empty[(n - 1) % S], static_cast<uint32_t>(((n - 1) / S) & 1));
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int quarter = warp & 3;
+    const int et = threadIdx.x - 64;
+    float* stg = stg_all + (warp - 2) * 32 * kStgPitch;
+    int seg = 0;
+    for (int t = tile_first; t < p.n_tiles; t += tile_stride, ++seg) {
+      const int acc = seg & 1;
+      if (p.C == 1 && p.coupling != nullptr) {
+        // this tile's coupling vector, fetched while the MMAs run
+        const int c0 = t * p.out_per_tile;
+        for (int i = et; i < p.out_per_tile; i += kEpiThreads)
+          cpl_s[i] = (c0 + i < p.n_out) ? __bfloat162float(p.coupling[c0 + i]) : 0.f;
+      }
+      const bool got = mbar_wait_warp(&acc_full[acc], static_cast<uint32_t>((seg >> 1) & 1));
+      if (!got && lane == 0) atomicOr(&flags[0], 1);
+      epi_bar();
+      if (flags[0]) {
+        if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * p.BN;
+      if (p.C == 1) {
+        tile_epilogue(p, t, quarter, lane, taddr, xbuf, stg, cpl_s);
+      } else {
+        // park the fp32 accumulator rows in this CTA's shared memory (the ring
+        // is idle: every stage has been consumed by the MMAs that completed)
+        float* arow = reinterpret_cast<float*>(smem) + (quarter * 32 + lane) * (p.BN + 4);
+        int c = 0;
+        for (; c + 32 <= p.BN; c += 32) {
+          float v[32];
+          tmem_ld<32>(taddr + c, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(arow + c)[i] =
+                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        for (; c < p.BN; c += 8) {
+          float v[8];
+          tmem_ld<8>(taddr + c, v);
+          reinterpret_cast<float4*>(arow + c)[0] = make_float4(v[0], v[1], v[2], v[3]);
+          reinterpret_cast<float4*>(arow + c)[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const __nv_bfloat16* res_s = nullptr;
+  if (p.C > 1 && !flags[0]) {
+    // Prefetch this rank's epilogue inputs into the (idle) staging area: the
+    // tile's coupling slice and, when they fit, the residual rows it will write.
+    const int opt = p.out_per_tile;
+    const int col0 = tile_first * opt;
+    const bool coupled = p.coupling != nullptr;
+    const int rows_base = coupled ? p.m_primary : p.M;
+    const int r0 = rank * rows_base / p.C, r1 = (rank + 1) * rows_base / p.C;
+    const int nrows = (r1 - r0) * (coupled ? 2 : 1);
+    if (coupled) {
+      for (int i = threadIdx.x; i < opt; i += kThreads)
+        cpl_s[i] = (col0 + i < p.n_out) ? __bfloat162float(p.coupling[col0 + i]) : 0.f;
+    }
+    if (p.epilogue == DF_EPI_RESIDUAL &&
+        nrows * opt * 2 <= 4 * 32 * kStgPitch * 4) {
+      __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(stg_all);
+      const int vec = opt / 8;  // 16-byte vectors per row
+      for (int i = threadIdx.x; i < nrows * vec; i += kThreads) {
+        const int rl = i / vec, v = i % vec;
+        const int pass = rl / (r1 - r0), rr = rl % (r1 - r0);
+        const int row = (pass == 1 ? p.m_primary : 0) + r0 + rr;
+        const int col = col0 + v * 8;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (row < p.M && col < p.n_out)
+          val = *reinterpret_cast<const uint4*>(p.residual + row * p.ldr + col);
+        reinterpret_cast<uint4*>(rs)[i] = val;
+      }
+      res_s = rs;
+    }
+  }
+  if (p.C > 1) {
+    cluster_sync_all();  // every accumulator of the cluster is parked
+    if (!flags[0]) {
+      float* prim = reinterpret_cast<float*>(smem) + kBM * (p.BN + 4);
+      cluster_epilogue(p, tile_first, rank, smem_u32(smem), prim, threadIdx.x, kThreads, res_s,
+                       cpl_s);
+    }
+    cluster_sync_all();  // no CTA leaves while others still read its shared memory
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(tmem_cols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ planning
+
+struct ClusterCaps {
+  int max_clusters[kMaxCluster + 1];  // resident clusters of size C (0 = unavailable)
+};
+
+std::mutex g_mu;
+bool g_attr_set[64] = {};
+bool g_caps_ok[64] = {};
+ClusterCaps g_caps[64];
+
+// Resident-cluster capacity of this kernel on the current device, per cluster
+// size (depends on the GPC layout); queried once per device.
+const ClusterCaps* caps_for_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_attr_set[dev]) {
+    if (cudaFuncSetAttribute(tile_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return nullptr;
+    g_attr_set[dev] = true;
+  }
+  if (!g_caps_ok[dev]) {
+    ClusterCaps c{};
+    for (int C = 1; C <= kMaxCluster; ++C) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(C * kSms);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = C;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, tile_gemm_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      c.max_clusters[C] = n;
+    }
+    g_caps[dev] = c;
+    g_caps_ok[dev] = true;
+  }
+  return &g_caps[dev];
+}
+
+struct Plan {
+  bool ok;
+  int BN, C, n_tiles, ctas, stages, stage_bytes;
+  double est_us;
+};
+
+// Pick the tile width and cluster size with the lowest modelled time. Rates:
+// ~46 GB/s of DRAM and ~77 GB/s of total TMA traffic per SM (measured with a
+// TMA streaming probe on B200), plus fixed costs for the cluster exchange and
+// per-tile epilogues.
+Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps) {
+  Plan best{};
+  best.ok = false;
+  best.est_us = 1e30;
+  const bool swiglu = epilogue == DF_EPI_SWIGLU;
+  const int n_out = swiglu ? N / 2 : N;
+  const int KB = K / kBK;
+  for (int BN = 256; BN >= 64; BN -= 16) {
+    const int opt = swiglu ? BN / 2 : BN;
+    const int n_tiles = static_cast<int>(ceil_div(n_out, opt));
+    const int stage_bytes = kTileX + BN * 128;
+    int stages = kRingBytes / stage_bytes;
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 3) continue;
+    for (int C = 1; C <= kMaxCluster && C <= KB; ++C) {
+      int ctas, tpc;
+      if (C == 1) {
+        ctas = n_tiles < kSms ? n_tiles : kSms;
+        tpc = static_cast<int>(ceil_div(n_tiles, ctas));
+      } else {
+        if (!caps || n_tiles > caps->max_clusters[C]) continue;
+        if (C > 1 && kBM * (BN + 4) * 4 + 32 * BN * 4 > kRingBytes) continue;
+        ctas = n_tiles * C;
+        tpc = 1;
+      }
+      if (C > 1 && ctas > kSms) continue;
+      const double kbpc = static_cast<double>(ceil_div(KB, C));
+      const double w = tpc * kbpc * BN * 128.0;
+      const double tot = tpc * kbpc * (BN * 128.0 + kTileX);
+      double t = w / 46e3;  // bytes / (46 GB/s) in microseconds
+      if (tot / 77e3 > t) t = tot / 77e3;
+      t += (C > 1 ? 2.5 : 0.0) + tpc * 1.5 + 2.5;
+      if (t < best.est_us) {
+        best = Plan{true, BN, C, n_tiles, ctas, stages, stage_bytes, t};
+      }
+    }
+  }
+  (void)M;
+  return best;
+}
+
+// Modelled time of the stream-K kernel for the same shape (same rates), used
+// to choose between the two plans.
+double stream_k_estimate(int N, int K, int epilogue) {
+  const bool swiglu = epilogue == DF_EPI_SWIGLU;
+  const int n_tiles = static_cast<int>(swiglu ? ceil_div(N / 2, 128) : ceil_div(N, 256));
+  const double units = static_cast<double>(n_tiles) * (K / kBK);
+  const double per_cta = units / kSms;
+  double t = per_cta * 32768.0 / 46e3;
+  const double tot = per_cta * 49152.0 / 77e3;
+  if (tot > t) t = tot;
+  const bool split = (static_cast<long long>(K / kBK) * n_tiles) % kSms != 0 || n_tiles < kSms;
+  return t + 2.5 + 3.0 + (split ? 7.0 : 0.0);
+}
+
+int planned_launches(int M, int N, int K, int epilogue) {
+  const Plan pl = make_plan(M, N, K, epilogue, caps_for_device());
+  if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(N, K, epilogue)) return 0;
+  return 1;
+}
+
+int launch_if_better(const Request& r) {
+  const int M = r.m_primary + r.m_aux;
+  const ClusterCaps* caps = caps_for_device();
+  if (!caps) return 0;
+  const Plan pl = make_plan(M, r.N, r.K, r.epilogue, caps);
+  if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(r.N, r.K, r.epilogue))
+    return 0;
+  const bool swiglu = r.epilogue == DF_EPI_SWIGLU;
+  Params p{};
+  p.M = M;
+  p.m_primary = r.m_primary;
+  p.n_out = swiglu ? r.N / 2 : r.N;
+  p.n_aux = r.n_aux;
+  p.epilogue = r.epilogue;
+  p.kblocks = r.K / kBK;
+  p.BN = pl.BN;
+  p.half = swiglu ? pl.BN / 2 : 0;
+  p.out_per_tile = swiglu ? pl.BN / 2 : pl.BN;
+  p.n_tiles = pl.n_tiles;
+  p.C = pl.C;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  p.idesc = make_idesc(kBM, pl.BN);
+  p.F = r.N / 2;
+  p.y = static_cast<__nv_bfloat16*>(r.y);
+  p.ldy = r.ldy;
+  p.coupling = static_cast<const __nv_bfloat16*>(r.coupling);
+  p.residual = static_cast<const __nv_bfloat16*>(r.residual);
+  p.ldr = r.ldr;
+  p.err = r.err;
+  CUtensorMap tmX, tmW;
+  if (!encode_tmap_bf16_2d(&tmX, r.x, static_cast<uint64_t>(M), static_cast<uint64_t>(r.K),
+                           static_cast<uint64_t>(r.ldx) * 2, kBM, kBK) ||
+      !encode_tmap_bf16_2d(&tmW, r.w, static_cast<uint64_t>(r.N), static_cast<uint64_t>(r.K),
+                           static_cast<uint64_t>(r.K) * 2, swiglu ? pl.BN / 2 : pl.BN, kBK))
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = r.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = pl.C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, tile_gemm_kernel, tmX, tmW, p) != cudaSuccess) return -1;
+  return 1;
+}
+
+}  // namespace tgemm
+}  // namespace df

@@ -1,0 +1,36 @@
+// Internal interface between the grouped-projection entry point and its
+// tile-parallel / cluster split-K plan (grouped_proj_tiles.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace df {
+namespace tgemm {
+
+struct Request {
+  const void* x;
+  int64_t ldx;
+  int m_primary, m_aux;
+  const void* w;
+  int N, K, n_aux;
+  void* y;
+  int64_t ldy;
+  int epilogue;
+  const void* coupling;
+  const void* residual;
+  int64_t ldr;
+  int32_t* err;
+  cudaStream_t stream;
+};
+
+// Launches the tile plan when it is modelled to beat stream-K on this device.
+// Returns 1 when launched, 0 when the caller should use stream-K, -1 on a CUDA
+// error. Arguments must already be validated.
+int launch_if_better(const Request& r);
+
+// 1 if the tile plan would be used for this shape on the current device, else 0.
+int planned_launches(int M, int N, int K, int epilogue);
+
+}  // namespace tgemm
+}  // namespace df

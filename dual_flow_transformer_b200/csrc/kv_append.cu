@@ -26,6 +26,8 @@ struct Params {
 
 __global__ void __launch_bounds__(256) kv_append_kernel(const Params p) {
   const int b = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int pos = p.positions[b];
   if (pos < 0 || pos / p.block_size >= p.max_blocks_per_seq) {
     if (threadIdx.x == 0) set_err(p.err, DF_DEVERR_POSITION);
@@ -86,6 +88,8 @@ extern "C" df_status dualflow_kv_append(const void* k_new, const void* v_new, in
   p.err = err_flag;
   const int nvec = Hkv * (D * esize / 16);
   const int threads = nvec >= 256 ? 256 : ((nvec + 31) / 32) * 32;
-  append::kv_append_kernel<<<B, threads, 0, static_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+  if (launch_pdl(append::kv_append_kernel, dim3(B), dim3(threads), 0,
+                 static_cast<cudaStream_t>(stream), p) != cudaSuccess)
+    return DF_ERR_CUDA;
+  return DF_OK;
 }

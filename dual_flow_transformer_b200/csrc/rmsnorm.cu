@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const __nv_bfloat16* 
                                                            __nv_bfloat16* y, int64_t ldy, int cols,
                                                            float eps) {
   const int r = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const uint4* xr = reinterpret_cast<const uint4*>(x + r * ldx);
   const int nvec = cols / 8;
   float ss = 0.f;
@@ -76,8 +78,10 @@ extern "C" df_status dualflow_rmsnorm(const void* x, int64_t ldx, const void* ga
   if (lx % 8 != 0 || ly % 8 != 0 || !aligned(x, 16) || !aligned(y, 16) ||
       (gain && !aligned(gain, 16)))
     return DF_ERR_ALIGN;
-  norm::rmsnorm_kernel<<<rows, norm::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), lx, static_cast<const __nv_bfloat16*>(gain),
-      static_cast<__nv_bfloat16*>(y), ly, cols, eps);
-  return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+  if (launch_pdl(norm::rmsnorm_kernel, dim3(rows), dim3(norm::kThreads), 0,
+                 static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(x), lx,
+                 static_cast<const __nv_bfloat16*>(gain), static_cast<__nv_bfloat16*>(y), ly, cols,
+                 eps) != cudaSuccess)
+    return DF_ERR_CUDA;
+  return DF_OK;
 }

@@ -1,0 +1,137 @@
+// tcgen05 (5th-generation tensor core) helpers for sm_100a: shared-memory
+// matrix descriptors, instruction descriptors, MMA issue/commit, TMEM loads,
+// plus bf16 vector load/store helpers used by the GEMM epilogues.
+#pragma once
+
+#include "common.cuh"
+
+namespace df {
+namespace umma {
+
+// Descriptor of a K-major bf16 tile with 128-byte swizzle: 8-row core groups
+// 1024 bytes apart (stride byte offset), leading offset unused (1), version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// kind::f16 instruction descriptor: D fp32 (bits 4-5), A and B bf16 (bits 7-9,
+// 10-12), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Load N consecutive fp32 TMEM columns of this thread's lane (32x32b shape:
+// lane = TMEM lane of the warp's quarter). Waits for completion.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  __syncwarp();
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  __syncwarp();
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int NV>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* src, float (&v)[NV]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < NV / 8; ++q) {
+    const uint4 u = s[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[q * 8 + 2 * k] = bf16_bits_to_float(static_cast<uint16_t>(w[k] & 0xffffu));
+      v[q * 8 + 2 * k + 1] = bf16_bits_to_float(static_cast<uint16_t>(w[k] >> 16));
+    }
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NV]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < NV / 8; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = pack_bf16x2(__float2bfloat16_rn(v[q * 8 + 2 * k]),
+                         __float2bfloat16_rn(v[q * 8 + 2 * k + 1]));
+    d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// SiLU(g) = g / (1 + exp(-g)) with the fast exponential and fast division
+// intrinsics (relative error a few ulp of fp32, far below the bf16 rounding of
+// the stored result; for very negative g the denominator overflows and the
+// fast division returns 0, the correct limit).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// 4 bf16 <-> 4 floats (8-byte accesses)
+__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* src, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(src);
+  v[0] = bf16_bits_to_float(static_cast<uint16_t>(u.x & 0xffffu));
+  v[1] = bf16_bits_to_float(static_cast<uint16_t>(u.x >> 16));
+  v[2] = bf16_bits_to_float(static_cast<uint16_t>(u.y & 0xffffu));
+  v[3] = bf16_bits_to_float(static_cast<uint16_t>(u.y >> 16));
+}
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(dst) =
+      make_uint2(pack_bf16x2(__float2bfloat16_rn(v[0]), __float2bfloat16_rn(v[1])),
+                 pack_bf16x2(__float2bfloat16_rn(v[2]), __float2bfloat16_rn(v[3])));
+}
+
+}  // namespace umma
+}  // namespace df

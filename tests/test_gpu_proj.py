@@ -134,3 +134,35 @@ def test_full_size_layer_projections_sampled(cuda_device, name, wkey, epi):
         ref = _oracle(x, w[cols], mp, epi, None if cpl is None else cpl[cols],
                       None if res is None else res[:, cols])
     assert_close(y[:, cols], ref, "bf16", name)
+
+
+MEDIUM = [  # (m_primary, m_aux, N, K): shapes that exercise the tile-parallel and
+            # cluster split-K plans (several tiles, k-ranges split over clusters)
+    (64, 64, 4096, 4096),
+    (64, 64, 8192, 4096),
+    (16, 16, 6144, 2048),
+    (64, 64, 2048, 14336),
+    (32, 32, 3200, 4096),   # tile width that does not divide N (tail tile)
+]
+
+
+@pytest.mark.parametrize("shape", MEDIUM)
+@pytest.mark.parametrize("epi,coupled", [("none", False), ("swiglu", True), ("residual", True)])
+def test_medium_shapes_sampled(cuda_device, shape, epi, coupled):
+    mp, ma, N, K = shape
+    g = torch.Generator().manual_seed(sum(shape) + len(epi))
+    x = _rand(g, (mp + ma, K))
+    w = _rand(g, (N, K), 0.02)
+    n_out = N // 2 if epi == "swiglu" else N
+    cpl = _rand(g, (n_out,), 0.1) if coupled else None
+    res = _rand(g, (mp + ma, n_out)) if epi == "residual" else None
+    y = _gpu(cuda_device, x, w, mp, epi, cpl, res).cpu()
+    torch.cuda.synchronize()
+    cols = np.unique(np.concatenate([np.arange(0, 48), np.arange(n_out - 48, n_out),
+                                     np.random.default_rng(1).integers(0, n_out, 192)]))
+    if epi == "swiglu":
+        ref = _oracle(x, torch.cat([w[cols], w[n_out + cols]]), mp, "swiglu", cpl[cols], None)
+    else:
+        ref = _oracle(x, w[cols], mp, epi, None if cpl is None else cpl[cols],
+                      None if res is None else res[:, cols])
+    assert_close(y[:, cols], ref, "bf16", "medium %s %s" % (shape, epi))
