@@ -220,7 +220,7 @@ class LayerRun:
                                    "head_dim %d, SwiGLU %d, batch %d per flow (M=%d), cache %d+1"
                                    % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
                        "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
-                       "attended": L, "attn_splits": self.layer.splits,
+                       "attended": L, "attn_launches": self.layer.attn_launches,
                        "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
                              % (self.kv_bytes / 1e9, 436207616 / 1e9)}
         self.dominant = "dualflow_decode_attn (split + combine kernels)"
@@ -257,14 +257,13 @@ class AttnRun:
         self.d = d
         self.max_len = int(self.host["seqlens"].max())
         self.ns = args.num_splits
-        nb = api.decode_attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, self.max_len, self.ns)
-        self.ws = torch.empty(max(256, nb), dtype=torch.uint8, device=dev)
+        self.ws = api.new_attn_workspace(w.B, w.Hq, w.Hkv, w.D, self.max_len, self.ns, dev)
         self.o1 = torch.empty_like(d["q1"])
         self.o2 = torch.empty_like(d["q1"])
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        S = api.decode_attn_num_splits(w.B, w.Hkv, self.max_len, self.ns)
+        n_attn = api.decode_attn_num_launches(w.B, w.Hkv, self.max_len, self.ns, w.torch_dtype)
         self.tokens_per_step = w.B
-        self.launches_per_step = (1 if S == 1 else 2) + (1 if w.append else 0)
+        self.launches_per_step = n_attn + (1 if w.append else 0)
         esize = 4 if w.dtype == "fp32" else 2
         tot = int(self.host["seqlens"].sum())
         self.attn_bytes = attn_algorithmic_bytes(w.B, w.Hq, w.Hkv, w.D, tot, esize)
@@ -275,7 +274,7 @@ class AttnRun:
                                    "head_dim %d, %s, lengths %d..%d%s" % (
                                        name, w.B, w.Hq, w.Hkv, w.D, w.dtype, w.len_lo, w.len_hi,
                                        ", random block table" if w.random_table else ""),
-                       "attn_splits": S,
+                       "attn_launches": n_attn,
                        "l2": "inputs larger than L2" if self.kv_bytes > 126e6
                              else "inputs smaller than L2 (not flushed)"}
         self.dominant = "dualflow_decode_attn (split + combine kernels)"

@@ -6,12 +6,14 @@ package is its thin binding plus the layer-step composition.
 
 from .api import (  # noqa: F401
     decode_attn,
+    decode_attn_num_launches,
     decode_attn_num_splits,
     decode_attn_workspace_size,
     grouped_proj,
     grouped_proj_num_launches,
     grouped_proj_workspace_size,
     kv_append,
+    new_attn_workspace,
     new_proj_workspace,
     rmsnorm,
 )

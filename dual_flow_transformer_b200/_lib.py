@@ -29,6 +29,7 @@ SIGNATURES = {
     "dualflow_status_string": (ctypes.c_char_p, [_c_int]),
     "dualflow_decode_attn_num_splits": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "dualflow_decode_attn_workspace_size": (_c_size, [_c_int] * 7),
+    "dualflow_decode_attn_num_launches": (_c_int, [_c_int] * 6),
     "dualflow_decode_attn": (_c_int, [
         _vp, _vp, _vp, _c_i64,          # q1, q2raw, a, q_stride_b
         _vp, _vp,                       # k_cache, v_cache

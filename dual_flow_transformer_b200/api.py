@@ -50,6 +50,20 @@ def decode_attn_num_splits(B, Hkv, max_seqlen, num_splits=0, block_size=64) -> i
     return _lib().dualflow_decode_attn_num_splits(B, Hkv, max_seqlen, block_size, num_splits)
 
 
+def decode_attn_num_launches(B, Hkv, max_seqlen, num_splits=0, dtype=torch.bfloat16,
+                             block_size=64) -> int:
+    return _lib().dualflow_decode_attn_num_launches(B, Hkv, max_seqlen, block_size, num_splits,
+                                                    dtype_code(dtype))
+
+
+def new_attn_workspace(B, Hq, Hkv, D, max_seqlen, num_splits=0, device="cuda"):
+    """Zero-filled decode-attention workspace for these sizes (bf16 keeps the
+    split-combine arrival counters in it; every completed call leaves them at
+    zero, so later calls with the same sizes can reuse it)."""
+    n = max(256, decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, num_splits))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
 def decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, num_splits=0, block_size=64) -> int:
     return _lib().dualflow_decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size,
                                                       num_splits)
@@ -88,9 +102,8 @@ def decode_attn(q1, q2raw, a, k_cache, v_cache, block_table, seqlens, max_seqlen
     for o in (o1, o2):
         if o is not None and (not _heads_view_ok(o, Hq, D) or o.stride(0) != os_b):
             raise ValueError("outputs must be [B, Hq, D] with contiguous heads and equal strides")
-    need = decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, num_splits, bs)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = new_attn_workspace(B, Hq, Hkv, D, max_seqlen, num_splits, dev)
     st = _lib().dualflow_decode_attn(
         _ptr(q1), _ptr(q2raw), _ptr(a), q1.stride(0), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_table), block_table.shape[1], _ptr(seqlens), int(max_seqlen),

@@ -1,7 +1,6 @@
 // Dual-flow decode attention: asymmetric shared-KV attention of the primary
 // query Q1 and the coupled auxiliary query Q2 = Q2raw + a (.) Q1 over the single
-// primary cache (K1, V1), split over the sequence (flash-decoding), plus the
-// split-combine kernel.
+// primary cache (K1, V1), optionally split over the sequence (flash-decoding).
 //
 // Method: "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi
 // Chiave" -- the auxiliary flow attends to the primary flow's keys and values
@@ -17,11 +16,16 @@
 //    (bf16(Q2 - hi)), 8..11 = the primary lo part (zero, Q1 is bf16-exact).
 //    The m16n8k16 fragment keeps row r and r+8 in the same thread, so hi + lo
 //    scores add in registers: Q2 enters the scores at ~16 significant bits;
-//  * QK^T and PV run on mma.sync (bf16 in, fp32 accumulate). The softmax
-//    weights P are split the same way (hi in rows r, lo in rows r+8) so PV
-//    also sees ~16-bit weights. Each warp owns 16 tokens of every page and
-//    keeps its own running max / sum per row (online softmax in the exp2
-//    domain, quad shuffles), merged across warps through shared memory;
+//  * QK^T and PV run on mma.sync (bf16 in, fp32 accumulate; one 16-row tile
+//    per page needs a small fraction of the tensor rate the HBM stream
+//    allows). The softmax weights P are split the same way (hi in rows r, lo
+//    in rows r+8) so PV also sees ~16-bit weights. Each warp owns 16 tokens of
+//    every page and keeps its own running max / sum per row (online softmax
+//    in the exp2 domain, quad shuffles), merged across warps through shared
+//    memory;
+//  * splits only when the (b, g) units cannot fill the two resident CTAs per
+//    SM (see make_plan); split partials are combined inside the kernel by the
+//    last split CTA of each unit to finish (arrival counter, split order);
 //  * every query row's arithmetic is independent of every other row's, and
 //    the split plan depends only on (B, Hkv, max_seqlen), so O1 is
 //    bit-identical whatever the auxiliary inputs are.
@@ -39,13 +43,9 @@ constexpr int kPage = 64;                 // tokens per page (block_size)
 constexpr int kConsumerWarps = 4;         // each owns 16 tokens of a page
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStagesBf16 = 3;            // pipeline depth of the bf16 kernel
-constexpr int kTargetCtas = 148 * 2 * 8;  // ~8 waves of 2 resident CTAs per SM
+constexpr int kSlots = 148 * 2;            // resident split CTAs (two per SM)
+constexpr int kSplitWaves = 2;             // split plans aim at ~2 waves of CTAs
 constexpr int kMinChunkPages = 8;         // >= 512 tokens per split
-// KV pages prefetched into L2 this many pages ahead of the shared-memory ring.
-#ifndef DF_ATTN_PREFETCH_PAGES
-#define DF_ATTN_PREFETCH_PAGES 0
-#endif
-constexpr int kPrefetchPages = DF_ATTN_PREFETCH_PAGES;
 
 struct Params {
   const void* q1;
@@ -66,7 +66,8 @@ struct Params {
   int chunk_pages;   // pages per split
   int num_splits;
   float* part_o;     // [B][2Hq][S][D]
-  float* part_ml;    // [B][2Hq][S][2] (running max in log2 units, sum)
+  float* part_ml;
+  int* counters;     // bf16 path with splits: [B][Hkv] arrival counters (zero between calls)    // [B][2Hq][S][2] (running max in log2 units, sum)
   int32_t* err;
   int dual;          // auxiliary rows computed
   int write1;        // store O1
@@ -84,8 +85,14 @@ inline Plan make_plan(int B, int Hkv, int max_seqlen, int block_size, int reques
   if (requested > 0) {
     s0 = requested < max_pages ? requested : max_pages;
   } else {
+    // Measured on B200: a CTA that streams a whole (sequence, KV head) unit
+    // ends at no cost (its successor's start overlaps the other CTA of the
+    // SM), while a split CTA adds ~3-6 us of slot time (partials, fence,
+    // arrival, merge). So one CTA per unit whenever the units fill every
+    // slot; otherwise enough splits for ~kSplitWaves waves at the longest
+    // length, each of at least kMinChunkPages pages.
     const int64_t units = static_cast<int64_t>(B) * Hkv;
-    int64_t want = ceil_div(kTargetCtas, units);
+    int64_t want = units >= kSlots ? 1 : ceil_div(int64_t(kSplitWaves) * kSlots, units);
     int64_t cap = max_pages / kMinChunkPages;
     if (cap < 1) cap = 1;
     if (want > cap) want = cap;
@@ -184,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int pg0 = split * p.chunk_pages;
   const int pg1 = min(npages, pg0 + p.chunk_pages);
   if (pg0 >= pg1) {
-    if (p.num_splits == 1)
-      write_zero_rows<__nv_bfloat16, D>(p, b, g, threadIdx.x, blockDim.x);
+    // no page in this split; split 0 owns the zero output of an empty sequence
+    if (split == 0) write_zero_rows<__nv_bfloat16, D>(p, b, g, threadIdx.x, blockDim.x);
     return;
   }
   const int ntiles = pg1 - pg0;
@@ -206,23 +213,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tensormap(&tmV);
       const uint64_t policy = l2_policy_evict_first();
       const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
-      auto prefetch_page = [&](int i) {
-        const int page = tbl[pg0 + i];
-        if (page < 0 || page >= p.num_blocks) return;
-        const int row = (page * p.Hkv + g) * kPage;
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          tma_prefetch_2d(&tmK, h * 64, row);
-          tma_prefetch_2d(&tmV, h * 64, row);
-        }
-      };
-      if (kPrefetchPages > 0)
-        for (int i = STAGES; i < ntiles && i < STAGES + kPrefetchPages; ++i) prefetch_page(i);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % STAGES;
-        if (kPrefetchPages > 0 && i + STAGES + kPrefetchPages < ntiles)
-          prefetch_page(i + STAGES + kPrefetchPages);
         if (i >= STAGES && !mbar_wait(&empty[st], ((i / STAGES) - 1) & 1)) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
           break;
@@ -473,6 +466,89 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
+  if (p.num_splits == 1) return;
+
+  // Split combine, done by whichever split of (b, g) finishes last: every
+  // split publishes its partial (fence, then one arrival on the unit's
+  // counter); the last arrival rewinds the counter for the next call and
+  // merges the splits in split order:
+  //   O = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),  M = max_s m_s.
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  __shared__ int last_arrival;
+  const int nsplit = (npages + p.chunk_pages - 1) / p.chunk_pages;
+  if (threadIdx.x == 0) {
+    int* ctr = p.counters + b * p.Hkv + g;
+    const int last = (atomicAdd(ctr, 1) == nsplit - 1);
+    if (last) atomicExch(ctr, 0);
+    last_arrival = last;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  if (!last_arrival) return;
+  __threadfence();
+  {
+    // thread t: row t / 16, columns [(t % 16) * D / 16, +D / 16)
+    constexpr int kCols = D / 16;
+    constexpr int kFastMerge = 8;
+    const int row = threadIdx.x >> 4, c0 = (threadIdx.x & 15) * kCols;
+    const int flow = row >> 2, j = row & 3;
+    if (j >= G || (flow == 1 && !p.dual)) return;
+    const int h = g * G + j;
+    const int64_t slot0 = (static_cast<int64_t>(b) * 2 * p.Hq + flow * p.Hq + h) * p.num_splits;
+    float M = kNegInf, Ls = 0.f, o[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) o[c] = 0.f;
+    auto accumulate = [&](float ms2, float ls2, const float4* v) {
+      const float wt = (ms2 == kNegInf) ? 0.f : exp2f(ms2 - M);
+      Ls += wt * ls2;
+#pragma unroll
+      for (int c = 0; c < kCols / 4; ++c) {
+        o[4 * c + 0] += wt * v[c].x;
+        o[4 * c + 1] += wt * v[c].y;
+        o[4 * c + 2] += wt * v[c].z;
+        o[4 * c + 3] += wt * v[c].w;
+      }
+    };
+    if (nsplit <= kFastMerge) {
+      // every load issued before the first use: one L2 round trip
+      float mv[kFastMerge], lv[kFastMerge];
+      float4 ov[kFastMerge][kCols / 4];
+#pragma unroll
+      for (int s2 = 0; s2 < kFastMerge; ++s2) {
+        if (s2 >= nsplit) break;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot0 + s2) * 2));
+        mv[s2] = ml.x;
+        lv[s2] = ml.y;
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + (slot0 + s2) * D + c0);
+#pragma unroll
+        for (int c = 0; c < kCols / 4; ++c) ov[s2][c] = __ldcg(src + c);
+      }
+#pragma unroll
+      for (int s2 = 0; s2 < kFastMerge; ++s2)
+        if (s2 < nsplit) M = max_nan(M, mv[s2]);
+#pragma unroll
+      for (int s2 = 0; s2 < kFastMerge; ++s2)
+        if (s2 < nsplit) accumulate(mv[s2], lv[s2], ov[s2]);
+    } else {
+      for (int s2 = 0; s2 < nsplit; ++s2) M = max_nan(M, __ldcg(p.part_ml + (slot0 + s2) * 2));
+      for (int s2 = 0; s2 < nsplit; ++s2) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot0 + s2) * 2));
+        float4 v[kCols / 4];
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + (slot0 + s2) * D + c0);
+#pragma unroll
+        for (int c = 0; c < kCols / 4; ++c) v[c] = __ldcg(src + c);
+        accumulate(ml.x, ml.y, v);
+      }
+    }
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(flow == 0 ? (p.write1 ? p.o1 : nullptr)
+                                                               : (p.write2 ? p.o2 : nullptr));
+    if (dst == nullptr) return;
+    uint32_t* out = reinterpret_cast<uint32_t*>(dst + b * p.o_stride_b + h * D + c0);
+#pragma unroll
+    for (int c = 0; c < kCols / 2; ++c)
+      out[c] = pack_bf16x2(__float2bfloat16_rn(safe_div(o[2 * c], Ls)),
+                           __float2bfloat16_rn(safe_div(o[2 * c + 1], Ls)));
+  }
 }
 
 // ------------------------------------------------------------------ fp32 split
@@ -605,8 +681,8 @@ __global__ void __launch_bounds__(128) split_f32_kernel(const Params p) {
 }
 
 // ------------------------------------------------------------------ combine
-// O = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s, in split
-// order (deterministic), then one rounding to the output dtype.
+// fp32 path: O = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s,
+// in split order (deterministic), then one rounding to the output dtype.
 
 template <typename T, int D>
 __global__ void __launch_bounds__(D) combine_kernel(const Params p) {
@@ -647,6 +723,23 @@ size_t f32_smem_bytes() {
   return sizeof(float) * (8 * D + 2 * kPage * D + 8 * kPage + 24);
 }
 
+// Workspace carve-up when there are splits: the bf16 arrival counters first
+// (the part that must start at zero), then the partial outputs and (max, sum).
+struct WsLayout {
+  size_t counters, part_o, part_ml;
+  size_t total() const { return counters + part_o + part_ml; }
+};
+
+inline WsLayout ws_layout(int B, int Hq, int Hkv, int D, int splits) {
+  WsLayout l{0, 0, 0};
+  if (splits <= 1) return l;
+  const size_t rows = static_cast<size_t>(B) * 2 * Hq * splits;
+  l.counters = round_up(static_cast<size_t>(B) * Hkv * sizeof(int), 256);
+  l.part_o = round_up(rows * D * sizeof(float), 256);
+  l.part_ml = round_up(rows * 2 * sizeof(float), 256);
+  return l;
+}
+
 template <int D>
 cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUtensorMap* tmV,
                    cudaStream_t stream) {
@@ -664,10 +757,6 @@ cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUt
     cudaError_t e = launch_pdl(split_bf16_kernel<D, kStagesBf16>, grid, dim3(kThreads), smem, stream,
                                *tmK, *tmV, p);
     if (e != cudaSuccess) return e;
-    if (p.num_splits > 1) {
-      e = launch_pdl(combine_kernel<__nv_bfloat16, D>, dim3(2 * p.Hq, p.B), dim3(D), 0, stream, p);
-      if (e != cudaSuccess) return e;
-    }
   } else {
     const size_t smem = f32_smem_bytes<D>();
     static bool attr_set = false;
@@ -700,15 +789,21 @@ extern "C" int dualflow_decode_attn_num_splits(int B, int Hkv, int max_seqlen, i
   return make_plan(B, Hkv, max_seqlen, block_size, num_splits).splits;
 }
 
+extern "C" int dualflow_decode_attn_num_launches(int B, int Hkv, int max_seqlen, int block_size,
+                                                 int num_splits, int dtype) {
+  if (B < 1 || Hkv < 1 || max_seqlen < 1 || block_size < 1 || num_splits < 0) return 0;
+  if (dtype == DF_BF16) return 1;  // the split combine runs inside the kernel
+  if (dtype != DF_FP32) return 0;
+  return make_plan(B, Hkv, max_seqlen, block_size, num_splits).splits > 1 ? 2 : 1;
+}
+
 extern "C" size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, int D,
                                                       int max_seqlen, int block_size,
                                                       int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || max_seqlen < 1 || block_size < 1 || num_splits < 0)
     return 0;
   const Plan pl = make_plan(B, Hkv, max_seqlen, block_size, num_splits);
-  if (pl.splits <= 1) return 0;
-  const size_t rows = static_cast<size_t>(B) * 2 * Hq * pl.splits;
-  return df::round_up(rows * D * sizeof(float), 256) + df::round_up(rows * 2 * sizeof(float), 256);
+  return df::attn::ws_layout(B, Hq, Hkv, D, pl.splits).total();
 }
 
 extern "C" df_status dualflow_decode_attn(
@@ -774,13 +869,13 @@ extern "C" df_status dualflow_decode_attn(
   p.write1 = o1 ? 1 : 0;
   p.write2 = want2 ? 1 : 0;
   if (pl.splits > 1) {
-    const size_t need = dualflow_decode_attn_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size,
-                                                            num_splits);
-    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DF_ERR_WORKSPACE;
-    const size_t rows = static_cast<size_t>(B) * 2 * Hq * pl.splits;
-    p.part_o = static_cast<float*>(workspace);
-    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                         round_up(rows * D * sizeof(float), 256));
+    const attn::WsLayout l = attn::ws_layout(B, Hq, Hkv, D, pl.splits);
+    if (!workspace || workspace_bytes < l.total() || !aligned(workspace, 256))
+      return DF_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    p.counters = reinterpret_cast<int*>(w);
+    p.part_o = reinterpret_cast<float*>(w + l.counters);
+    p.part_ml = reinterpret_cast<float*>(w + l.counters + l.part_o);
   }
 
   CUtensorMap tmK, tmV;
@@ -846,6 +941,13 @@ extern "C" df_status dualflow_decode_attn_noalloc(
   if (need > 0) {
     const df_status st = df::noalloc::scratch_address(&scratch);
     if (st != DF_OK) return st;
+    // the bf16 arrival counters (start of the layout) must start at zero
+    if (dtype == DF_BF16) {
+      const df::attn::Plan pl = make_plan(B, Hkv, max_seqlen, block_size, num_splits);
+      const size_t counters = df::attn::ws_layout(B, Hq, Hkv, D, pl.splits).counters;
+      if (cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DF_ERR_CUDA;
+    }
   }
   return dualflow_decode_attn(q1, q2raw, a, q_stride_b, k_cache, v_cache, block_table,
                               max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq,

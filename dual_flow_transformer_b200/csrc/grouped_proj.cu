@@ -248,9 +248,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int KB = p.kblocks;
-  // set-up above overlaps the previous kernel; global memory only from here on
-  pdl_wait();
-  pdl_trigger();
+  // Set-up above overlaps the previous kernel (programmatic dependent launch).
+  // Global memory that it may write (activations, residual, coupling,
+  // partials, the output) only after the wait; the producer waits after its
+  // first weights.
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -259,18 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmW);
       const uint64_t pol_w = l2_policy_evict_first();  // weights: streamed once
       const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read by every CTA
-      long long n = 0;  // stages issued
-      for (long long it = it_begin; it < it_end; ++it, ++n) {
-        const int s = static_cast<int>(n % kStages);
-        if (n >= kStages && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / kStages) - 1) & 1))) {
-          set_err(p.err, DF_DEVERR_TIMEOUT);
-          break;
-        }
+      auto load_w = [&](int s, long long it) {
         const int tile = static_cast<int>(it / KB), kb = static_cast<int>(it % KB);
-        uint8_t* sa = smem + s * kStageBytes;
-        uint8_t* sb = sa + kTileA;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+        uint8_t* sb = smem + s * kStageBytes + kTileA;
         if (p.epilogue == DF_EPI_SWIGLU) {
           tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * (kBN / 2), pol_w);
           tma_load_2d_hint(sb + kTileB / 2, &tmW, &full[s], kb * kBK, p.F + tile * (kBN / 2),
@@ -278,6 +274,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, tile * kBN, pol_w);
         }
+      };
+      // The weights are no product of the previous kernel: the first ring
+      // stages start streaming them before the wait for it.
+      long long pre = 0;
+      for (long long it = it_begin; it < it_end && pre < kStages; ++it, ++pre) {
+        mbar_arrive_expect_tx(&full[pre], kStageBytes);
+        load_w(static_cast<int>(pre), it);
+      }
+      pdl_wait();
+      pdl_trigger();
+      long long n = 0;  // stages issued
+      for (long long it = it_begin; it < it_end; ++it, ++n) {
+        const int s = static_cast<int>(n % kStages);
+        const int kb = static_cast<int>(it % KB);
+        uint8_t* sa = smem + s * kStageBytes;
+        if (n < pre) {  // weights already on their way
+          tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+          continue;
+        }
+        if (n >= kStages && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / kStages) - 1) & 1))) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+        load_w(s, it);
       }
       // drain own copies still in flight
       for (long long i = (n > kStages ? n - kStages : 0); i < n; ++i)

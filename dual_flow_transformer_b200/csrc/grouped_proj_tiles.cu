@@ -342,8 +342,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
+  // Set-up above overlaps the previous kernel (programmatic dependent launch).
+  // Global memory that it may write (activations, residual, coupling, the
+  // output) only after the wait; the producer waits after its first weights.
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -352,26 +357,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmW);
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
+      auto load_w = [&](int s, int t, int kb) {
+        uint8_t* sb = smem + s * p.stage_bytes + kTileX;
+        if (p.epilogue == DF_EPI_SWIGLU) {
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.half, pol_w);
+          tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + t * p.half, pol_w);
+        } else {
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.BN, pol_w);
+        }
+      };
+      // The weights are no product of the previous kernel: the first ring
+      // stages start streaming them before the wait for it.
+      long long pre = 0;
+      for (int t = tile_first; t < p.n_tiles && pre < S; t += tile_stride)
+        for (int kb = kb0; kb < kb1 && pre < S; ++kb, ++pre) {
+          mbar_arrive_expect_tx(&full[pre], p.stage_bytes);
+          load_w(static_cast<int>(pre), t, kb);
+        }
+      pdl_wait();
+      pdl_trigger();
       long long n = 0;
       bool ok = true;
       for (int t = tile_first; t < p.n_tiles && ok; t += tile_stride) {
         for (int kb = kb0; kb < kb1; ++kb, ++n) {
           const int s = static_cast<int>(n % S);
+          uint8_t* sa = smem + s * p.stage_bytes;
+          if (n < pre) {  // weights already on their way
+            tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+            continue;
+          }
           if (n >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / S) - 1) & 1))) {
             set_err(p.err, DF_DEVERR_TIMEOUT);
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * p.stage_bytes;
-          uint8_t* sb = sa + kTileX;
           mbar_arrive_expect_tx(&full[s], p.stage_bytes);
           tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
-          if (p.epilogue == DF_EPI_SWIGLU) {
-            tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.half, pol_w);
-            tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + t * p.half, pol_w);
-          } else {
-            tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.BN, pol_w);
-          }
+          load_w(s, t, kb);
         }
       }
       for (long long i = (n > S ? n - S : 0); i < n; ++i)

@@ -55,10 +55,9 @@ class DualFlowLayer:
                  api.grouped_proj_workspace_size(M, *weights["w_gu"].shape, "swiglu"),
                  api.grouped_proj_workspace_size(M, *weights["w_down"].shape, "residual"))
         self.proj_ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
-        aw = api.decode_attn_workspace_size(B, Hq, Hkv, D, self.max_seqlen, num_splits)
-        self.attn_ws = torch.empty(max(aw, 256), dtype=torch.uint8, device=dev)
+        self.attn_ws = api.new_attn_workspace(B, Hq, Hkv, D, self.max_seqlen, num_splits, dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.splits = api.decode_attn_num_splits(B, Hkv, self.max_seqlen, num_splits)
+        self.attn_launches = api.decode_attn_num_launches(B, Hkv, self.max_seqlen, num_splits)
         self._gemm_launches = (
             api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
             + api.grouped_proj_num_launches(M, *weights["w_o"].shape, "residual")
@@ -67,9 +66,9 @@ class DualFlowLayer:
 
     @property
     def launches_per_step(self) -> int:
-        """Kernel launches of one step: 2 norms, append, attention split (+ combine),
-        and the grouped projections (1 or 2 launches each)."""
-        return 3 + (2 if self.splits > 1 else 1) + self._gemm_launches
+        """Kernel launches of one step: 2 norms, append, attention, and the
+        grouped projections (1 or 2 launches each)."""
+        return 3 + self.attn_launches + self._gemm_launches
 
     # ------------------------------------------------------------ CUDA graphs
     def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):

@@ -108,11 +108,21 @@ const char* dualflow_status_string(int status);
 /* num_splits: 0 = automatic; otherwise the requested number of splits.      */
 /* workspace : device scratch, 256-byte aligned, at least                    */
 /*             dualflow_decode_attn_workspace_size(...) bytes (0 when the    */
-/*             plan has one split, then workspace may be NULL).               */
+/*             plan has one split, then workspace may be NULL). bf16: its    */
+/*             first bytes are per-(sequence, KV head) arrival counters of   */
+/*             the in-kernel split combine, so a new workspace must be       */
+/*             ZERO-FILLED once; every completed call leaves them at zero    */
+/*             again (re-zero after a call that set a device error code).    */
+/*             Calls sharing one workspace must be ordered on the GPU.       */
 /* Supported: D in {64, 128}, block_size 64, Hq/Hkv in {1,2,3,4}.            */
 /* ------------------------------------------------------------------------ */
 int dualflow_decode_attn_num_splits(int B, int Hkv, int max_seqlen, int block_size,
                                     int num_splits);
+/* Kernel launches one dualflow_decode_attn call makes with these arguments:*/
+/* bf16 1 (the split combine runs in the kernel); fp32 1 (one split) or 2   */
+/* (split kernel + combine kernel); 0 for invalid arguments.                 */
+int dualflow_decode_attn_num_launches(int B, int Hkv, int max_seqlen, int block_size,
+                                      int num_splits, int dtype);
 size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, int D, int max_seqlen,
                                            int block_size, int num_splits);
 df_status dualflow_decode_attn(const void* q1, const void* q2raw, const void* a,
@@ -144,9 +154,10 @@ df_status dualflow_decode_attn(const void* q1, const void* q2raw, const void* a,
 /*    that device current (cudaGetSymbolAddress) and caches it; make that    */
 /*    first call before any stream capture. A failed lookup: DF_ERR_CUDA.    */
 /*  - All calls on a device share the one array, which keeps the last call's */
-/*    contents (nothing in it needs to start at zero: every partial that the */
-/*    combine reads is written first by the same call). Calls that overlap   */
-/*    on the GPU (different streams, no ordering) race on it: order them.    */
+/*    contents. A bf16 call first clears, on its stream, the part that must  */
+/*    start at zero (the arrival counters; cudaMemsetAsync, no allocation).  */
+/*    Calls that overlap on the GPU (different streams, no ordering) race on */
+/*    it: order them.                                                        */
 /* ------------------------------------------------------------------------ */
 #define DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 df_status dualflow_decode_attn_noalloc(const void* q1, const void* q2raw, const void* a,
@@ -199,6 +210,10 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
 /*  DF_EPI_RESIDUAL : y[M][N] = residual + x w^T, and aux rows add            */
 /*                    coupling[n] * (x w^T)[j][n] before the residual (c_l).   */
 /* y and residual may alias (in-place residual add). All bf16.               */
+/* w is treated as constant: every launch is a programmatic dependent launch */
+/* that starts streaming w BEFORE it waits for the kernel launched ahead of  */
+/* it on the stream (x, residual and coupling are read only after the wait),*/
+/* so that kernel must not write w.                                          */
 /* Supported: M = m_primary + m_aux in [1, 128]; K % 64 == 0; N % 128 == 0    */
 /* (SWIGLU: F % 64 == 0); ldx, ldy, ldr multiples of 8 elements; x, w        */
 /* 16-byte aligned; n_aux a multiple of 32 or the full output width.          */

@@ -93,10 +93,20 @@ def test_decode_attn_plan(lib):
         chunk = -(-pages // s)
         assert 1 <= s <= pages and -(-pages // chunk) == s
         if s > 1:
-            assert ws(B, 2 * Hkv, Hkv, 128, L_, 64, 0) >= B * 2 * 2 * Hkv * s * 130 * 4
+            # arrival counters + partials (o and (max, sum)) of every split
+            assert ws(B, 2 * Hkv, Hkv, 128, L_, 64, 0) >= B * Hkv * 4 + B * 2 * 2 * Hkv * s * 130 * 4
         else:
             assert ws(B, 2 * Hkv, Hkv, 128, L_, 64, 0) == 0
     assert ns(0, 1, 10, 64, 0) == 0 and ws(0, 1, 1, 64, 10, 64, 0) == 0
+    nl = lib.dualflow_decode_attn_num_launches
+    assert nl(8, 8, 131072, 64, 0, L.DF_BF16) == 1  # the combine runs inside the kernel
+    assert nl(8, 8, 131072, 64, 0, L.DF_FP32) == 2 and nl(1, 2, 129, 64, 1, L.DF_FP32) == 1
+    # automatic plan: one CTA per (sequence, KV head) unit once the units fill
+    # the 296 resident slots (2 per SM); otherwise ~2 waves, chunks >= 8 pages
+    assert ns(64, 8, 4097, 64, 0) == 1 and ns(32, 32, 2048, 64, 0) == 1
+    assert ns(8, 8, 131072, 64, 0) == 10           # ceil(592 / 64) splits
+    assert ns(4, 2, 4096, 64, 0) == 8               # capped: 64 pages / 8
+    assert nl(0, 8, 4097, 64, 0, L.DF_BF16) == 0 and nl(1, 1, 64, 64, 0, 9) == 0
 
 
 def _append(lib, **over):

@@ -25,12 +25,19 @@ def _small(name, **kw):
 
 
 def _run(inp, dev, num_splits=0, primary_out=True, aux=True, err=None):
+    """One decode_attn call. Without an `err` from the caller the device error
+    flag (bad lengths or pages, a wait that gave up) must stay clear."""
     d = to_dev(inp, dev)
     max_len = int(inp["seqlens"].max())
+    own = err is None
+    if own:
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
     o1, o2 = api.decode_attn(d["q1"], d["q2raw"] if aux else None, d["a"] if aux else None,
                              d["k_cache"], d["v_cache"], d["block_table"], d["seqlens"], max_len,
                              primary_out=primary_out, num_splits=num_splits, err_flag=err)
     torch.cuda.synchronize()
+    if own:
+        assert int(err.item()) == 0, "device error flag %d" % int(err.item())
     return o1, o2
 
 
@@ -79,6 +86,8 @@ CASES = {
     "gqa_g3": dict(name="gqa", B=3, Hq=6, Hkv=2, len_lo=60, len_hi=260, seed=24),
     "long_small": dict(name="long", B=2, Hq=4, Hkv=1, len_lo=3000, len_hi=5100, seed=25),
     "edge_lengths": dict(name="gqa", B=8, Hq=8, Hkv=2, len_lo=1, len_hi=130, seed=26),
+    # 16..63 pages per unit: several chunks per split at every split count
+    "many_pages": dict(name="gqa", B=8, Hq=8, Hkv=2, len_lo=1000, len_hi=4000, seed=29),
 }
 
 
@@ -93,6 +102,34 @@ def test_bf16_parity(cuda_device, case, num_splits):
     r1, r2 = oracle_attn(inp)
     assert_close(o1, r1, "bf16", case + " o1")
     assert_close(o2, r2, "bf16", case + " o2")
+
+
+@pytest.mark.parametrize("num_splits", [0, 1])
+def test_bf16_workspace_reuse_is_deterministic(cuda_device, num_splits):
+    """Back-to-back calls on one workspace give the same bits: the arrival
+    counters return to zero after every call, every call rewrites the split
+    partials it reads, and the combine order is fixed."""
+    kw = dict(CASES["many_pages"])
+    w = _small(kw.pop("name"), **kw)
+    inp = synth.make_attn_inputs(w)
+    d = to_dev(inp, cuda_device)
+    max_len = int(inp["seqlens"].max())
+    ws = api.new_attn_workspace(w.B, w.Hq, w.Hkv, w.D, max_len, num_splits, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    outs = []
+    for _ in range(3):
+        o1, o2 = api.decode_attn(d["q1"], d["q2raw"], d["a"], d["k_cache"], d["v_cache"],
+                                 d["block_table"], d["seqlens"], max_len, num_splits=num_splits,
+                                 workspace=ws, err_flag=err)
+        outs.append((o1.clone(), o2.clone()))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for o1, o2 in outs[1:]:
+        assert torch.equal(o1.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(o2.view(torch.int16), outs[0][1].view(torch.int16))
+    r1, r2 = oracle_attn(inp)
+    assert_close(outs[0][0], r1, "bf16", "o1")
+    assert_close(outs[0][1], r2, "bf16", "o2")
 
 
 def test_bf16_stale_nan_tail_slots_do_not_leak(cuda_device):
