@@ -223,7 +223,7 @@ class LayerRun:
                        "attended": L, "attn_launches": self.layer.attn_launches,
                        "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
                              % (self.kv_bytes / 1e9, 436207616 / 1e9)}
-        self.dominant = "dualflow_decode_attn (split + combine kernels)"
+        self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"
 
     def step(self, timers=None):
         self.layer.replay(timers)
@@ -277,7 +277,7 @@ class AttnRun:
                        "attn_launches": n_attn,
                        "l2": "inputs larger than L2" if self.kv_bytes > 126e6
                              else "inputs smaller than L2 (not flushed)"}
-        self.dominant = "dualflow_decode_attn (split + combine kernels)"
+        self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"
         # CUDA graphs: [append] and [attention], replayed every step
         self._append()
         self._attn()
