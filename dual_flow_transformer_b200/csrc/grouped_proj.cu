@@ -530,9 +530,9 @@ extern "C" size_t dualflow_grouped_proj_workspace_size(int M, int N, int K, int 
 extern "C" int dualflow_grouped_proj_num_launches(int M, int N, int K, int epilogue) {
   using namespace df::gemm;
   if (M < 1 || N < 1 || K < 1 || epilogue < 0 || epilogue > 2) return 0;
-  if (df::tgemm::planned_launches(M, N, K, epilogue)) return 1;
   const Layout l = make_layout(N, K, epilogue);
   if (l.total < 1) return 0;
+  if (df::tgemm::planned_launches(M, N, K, epilogue, l.partial_bytes)) return 1;
   Params p{};
   p.total_iters = l.total;
   p.ctas = l.ctas;
@@ -600,7 +600,7 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   {
     // tile-parallel / cluster split-K plan when it is modelled to be faster
     tgemm::Request rq{x, lx, m_primary, m_aux, w, N, K, n_aux, y, ly, epilogue, coupling,
-                      residual, lr, err_flag, st};
+                      residual, lr, err_flag, st, workspace, workspace_bytes};
     const int launched = tgemm::launch_if_better(rq);
     if (launched < 0) return DF_ERR_CUDA;
     if (launched > 0) return DF_OK;

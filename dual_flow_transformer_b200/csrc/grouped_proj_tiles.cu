@@ -9,10 +9,13 @@
 //    shape so that the tile count fills the 148 SMs; with C = 1 each CTA owns
 //    whole tiles (persistent over tiles, two TMEM accumulators);
 //  * when there are too few tiles, a thread-block cluster of C <= 8 CTAs
-//    splits one tile's k-range. Each CTA parks its fp32 accumulator in its own
-//    shared memory, and after a cluster barrier every CTA sums its share of the
-//    tile's rows across the cluster through distributed shared memory (in rank
-//    order, so the result is deterministic), applies the epilogue and stores.
+//    splits one tile's k-range. Each CTA parks its fp32 accumulator in shared
+//    memory and writes it with one bulk TMA store to its slot of an
+//    L2-resident workspace; after a cluster barrier each CTA bulk-loads the C
+//    partials of its share of the tile's rows, sums them in rank order
+//    (deterministic), applies the epilogue and stores. (Distributed shared
+//    memory moves these ~100 KB per CTA at only ~20 GB/s per SM on B200; the
+//    TMA engine through L2 is several times faster.)
 // The producer/MMA/epilogue warp roles, the TMA ring and the bounded waits are
 // as in the stream-K kernel.
 #include <math.h>
@@ -55,6 +58,7 @@ struct Params {
   const __nv_bfloat16* coupling;
   const __nv_bfloat16* residual;
   int64_t ldr;
+  float* part;  // C > 1: [ctas][kBM][BN + 4] fp32 partial accumulators
   int32_t* err;
 };
 
@@ -67,21 +71,34 @@ __device__ __forceinline__ void cluster_sync_all() {
                    : "memory");
 }
 
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
+// Bulk (untiled) TMA copies; addresses 16-byte aligned, sizes multiples of 16.
+__device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          sdst),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Distributed-shared-memory load. No memory clobber: ordering against the
-// cluster barrier comes from both being volatile asm, and leaving the clobber
-// out lets independent loads be issued back to back.
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr));
-  return v;
+// Cluster plan (C > 1): rank q owns rows [lo, hi) of the rows it splits --
+// the primary rows when a coupling pairs aux row m_primary + j with primary
+// row j (both then belong to the same rank), else all M rows.
+__device__ __forceinline__ void owned_rows(const Params& p, int q, int& lo, int& hi) {
+  const int base = p.coupling != nullptr ? p.m_primary : p.M;
+  lo = q * base / p.C;
+  hi = (q + 1) * base / p.C;
 }
 
 __device__ __forceinline__ bool store_ok(const Params& p, int row, int col) {
@@ -183,80 +200,62 @@ __device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, 
   }
 }
 
-// C > 1: this CTA's share of the tile's rows, summed over the cluster's
-// accumulators (parked in each CTA's shared memory) in rank order, then the
-// epilogue. All threads of the CTA take part, two items (4 output columns of
-// one row each) at a time with every remote load issued before any sum.
-__device__ void cluster_epilogue(const Params& p, int tile, int rank, uint32_t acc_local,
-                                 float* prim, int tid, int nthreads,
-                                 const __nv_bfloat16* res_s, const float* cpl_s) {
-  constexpr int kBatch = 2;
+// C > 1: this CTA's rows of the tile, summed over the C partials loaded into
+// `recv` ([src rank][own row][BN + 4] fp32, own primary rows first), in rank
+// order, then the epilogue. Thread t keeps one 4-column group (t % groups)
+// and walks rows t / groups, + nthreads / groups, ... two at a time, with
+// the C partial loads of both rows issued before any sum (this loop runs on
+// six warps, so its latency is not hidden by other warps).
+template <int C>
+__device__ void cluster_epilogue_c(const Params& p, int tile, int rank, const float* recv,
+                                   float* prim, int tid, int nthreads,
+                                   const __nv_bfloat16* res_s, const float* cpl_s) {
   const int pitch = p.BN + 4;
   const bool coupled = p.coupling != nullptr;
   const bool swiglu = p.epilogue == DF_EPI_SWIGLU;
   const bool resid = p.epilogue == DF_EPI_RESIDUAL;
   const int opt = p.out_per_tile;
   const int groups = opt / 4;  // 4-column groups per row
-  int r0, r1;                  // primary (or all) rows of this rank
-  if (coupled) {
-    r0 = rank * p.m_primary / p.C;
-    r1 = (rank + 1) * p.m_primary / p.C;
-  } else {
-    r0 = rank * p.M / p.C;
-    r1 = (rank + 1) * p.M / p.C;
+  int r0, r1;
+  owned_rows(p, rank, r0, r1);
+  const int n = r1 - r0;
+  const int nloc = coupled ? 2 * n : n;
+  const int rstep = nthreads / groups;
+  const int g = tid % groups, rfirst = tid / groups;
+  const int j = g * 4;
+  const int col = tile * opt + j;
+  const bool active = rfirst < rstep;
+  float cv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (coupled && col < p.n_out) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cv[i] = cpl_s[j + i];
   }
-  const int col_base = tile * opt;
-  const int total = (r1 - r0) * groups;
   for (int pass = 0; pass < (coupled ? 2 : 1); ++pass) {
     const int row_off = (pass == 1 ? p.m_primary : 0) + r0;
-    for (int base = tid; base < total; base += nthreads * kBatch) {
-      float4 va[kBatch][kMaxCluster], vu[kBatch][kMaxCluster];
-      float rv[kBatch][4], cv[kBatch][4];
+    for (int rl0 = rfirst; active && rl0 < n; rl0 += 2 * rstep) {
+      float4 va[2][C], vu[2][C];
 #pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int item = base + b * nthreads;
-        if (item >= total) continue;
-        const int rl = item / groups, j = (item % groups) * 4;
-        const int row = row_off + rl, col = col_base + j;
-        const uint32_t off_a = acc_local + (row * pitch + j) * 4;
-        const uint32_t off_u = acc_local + (row * pitch + p.half + j) * 4;
+      for (int k = 0; k < 2; ++k) {
+        const int rl = rl0 + k * rstep;
+        if (rl >= n) continue;
+        const float* src = recv + (pass * n + rl) * pitch + j;
 #pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) {
-          if (q < p.C) {
-            va[b][q] = ld_cluster_f4(map_to_rank(off_a, q));
-            if (swiglu) vu[b][q] = ld_cluster_f4(map_to_rank(off_u, q));
-          }
-        }
-        if (resid && store_ok(p, row, col)) {
-          if (res_s != nullptr) {
-            load_bf16x4(res_s + (pass * (r1 - r0) + rl) * opt + j, rv[b]);
-          } else {
-            load_bf16x4(p.residual + row * p.ldr + col, rv[b]);
-          }
-        } else {
-          rv[b][0] = rv[b][1] = rv[b][2] = rv[b][3] = 0.f;
-        }
-        if (coupled && pass == 1 && col < p.n_out) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) cv[b][i] = cpl_s[j + i];
-        } else {
-          cv[b][0] = cv[b][1] = cv[b][2] = cv[b][3] = 0.f;
+        for (int q = 0; q < C; ++q) {
+          va[k][q] = *reinterpret_cast<const float4*>(src + q * nloc * pitch);
+          if (swiglu) vu[k][q] = *reinterpret_cast<const float4*>(src + q * nloc * pitch + p.half);
         }
       }
 #pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int item = base + b * nthreads;
-        if (item >= total) continue;
-        const int rl = item / groups, j = (item % groups) * 4;
-        const int row = row_off + rl, col = col_base + j;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), u = a;
+      for (int k = 0; k < 2; ++k) {
+        const int rl = rl0 + k * rstep;
+        if (rl >= n) continue;
+        const int row = row_off + rl;
+        float4 a = va[k][0], u = vu[k][0];
 #pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) {
-          if (q < p.C) {
-            a.x += va[b][q].x; a.y += va[b][q].y; a.z += va[b][q].z; a.w += va[b][q].w;
-            if (swiglu) {
-              u.x += vu[b][q].x; u.y += vu[b][q].y; u.z += vu[b][q].z; u.w += vu[b][q].w;
-            }
+        for (int q = 1; q < C; ++q) {
+          a.x += va[k][q].x; a.y += va[k][q].y; a.z += va[k][q].z; a.w += va[k][q].w;
+          if (swiglu) {
+            u.x += vu[k][q].x; u.y += vu[k][q].y; u.z += vu[k][q].z; u.w += vu[k][q].w;
           }
         }
         float o[4] = {a.x, a.y, a.z, a.w};
@@ -272,15 +271,37 @@ __device__ void cluster_epilogue(const Params& p, int tile, int rank, uint32_t a
         }
         if (coupled && pass == 1) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = fmaf(cv[b][i], prim[rl * opt + j + i], o[i]);
+          for (int i = 0; i < 4; ++i) o[i] = fmaf(cv[i], prim[rl * opt + j + i], o[i]);
         }
         if (!store_ok(p, row, col)) continue;
+        if (resid) {
+          float rv[4];
+          if (res_s != nullptr) {
+            load_bf16x4(res_s + (pass * n + rl) * opt + j, rv);
+          } else {
+            load_bf16x4(p.residual + row * p.ldr + col, rv);
+          }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o[i] += rv[b][i];
+          for (int i = 0; i < 4; ++i) o[i] += rv[i];
+        }
         store_bf16x4(p.y + row * p.ldy + col, o);
       }
     }
     if (coupled && pass == 0) __syncthreads();
+  }
+}
+
+__device__ void cluster_epilogue(const Params& p, int tile, int rank, const float* recv,
+                                 float* prim, int tid, int nthreads,
+                                 const __nv_bfloat16* res_s, const float* cpl_s) {
+  switch (p.C) {
+    case 2: cluster_epilogue_c<2>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 3: cluster_epilogue_c<3>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 4: cluster_epilogue_c<4>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 5: cluster_epilogue_c<5>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 6: cluster_epilogue_c<6>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 7: cluster_epilogue_c<7>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    default: cluster_epilogue_c<8>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
   }
 }
 
@@ -297,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + kMaxStages;
   uint64_t* acc_full = empty + kMaxStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* red_full = acc_empty + 2;  // C > 1: the partials of this CTA's rows have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
   int* flags = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -328,7 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], kEpiThreads / 32);
     }
-    flags[0] = 0;
+    mbar_init(red_full, 1);
+    flags[0] = 0;  // a wait gave up
+    flags[1] = 0;  // C > 1: the residual rows were prefetched into the staging area
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -440,6 +464,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int et = threadIdx.x - 64;
     float* stg = stg_all + (warp - 2) * 32 * kStgPitch;
+    if (p.C > 1) {
+      // While the MMAs run: this rank's epilogue inputs into the (idle)
+      // staging area -- the tile's coupling slice and, when they fit, the
+      // residual rows it will write.
+      const int opt = p.out_per_tile;
+      const int col0 = tile_first * opt;
+      const bool coupled = p.coupling != nullptr;
+      const int rows_base = coupled ? p.m_primary : p.M;
+      const int r0 = rank * rows_base / p.C, r1 = (rank + 1) * rows_base / p.C;
+      const int nrows = (r1 - r0) * (coupled ? 2 : 1);
+      if (coupled) {
+        for (int i = et; i < opt; i += kEpiThreads)
+          cpl_s[i] = (col0 + i < p.n_out) ? __bfloat162float(p.coupling[col0 + i]) : 0.f;
+      }
+      if (p.epilogue == DF_EPI_RESIDUAL && nrows * opt * 2 <= 4 * 32 * kStgPitch * 4) {
+        __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(stg_all);
+        const int vec = opt / 8;  // 16-byte vectors per row
+        for (int i = et; i < nrows * vec; i += kEpiThreads) {
+          const int rl = i / vec, v = i % vec;
+          const int pass = rl / (r1 - r0), rr = rl % (r1 - r0);
+          const int row = (pass == 1 ? p.m_primary : 0) + r0 + rr;
+          const int col = col0 + v * 8;
+          uint4 val = make_uint4(0u, 0u, 0u, 0u);
+          if (row < p.M && col < p.n_out)
+            val = *reinterpret_cast<const uint4*>(p.residual + row * p.ldr + col);
+          reinterpret_cast<uint4*>(rs)[i] = val;
+        }
+        if (et == 0) flags[1] = 1;
+      }
+    }
     int seg = 0;
     for (int t = tile_first; t < p.n_tiles; t += tile_stride, ++seg) {
       const int acc = seg & 1;
@@ -479,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           reinterpret_cast<float4*>(arow + c)[0] = make_float4(v[0], v[1], v[2], v[3]);
           reinterpret_cast<float4*>(arow + c)[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
+        fence_proxy_async_smem();  // the parked rows leave through a bulk TMA store
       }
       tc_fence_before();
       __syncwarp();
@@ -489,45 +544,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const __nv_bfloat16* res_s = nullptr;
-  if (p.C > 1 && !flags[0]) {
-    // Prefetch this rank's epilogue inputs into the (idle) staging area: the
-    // tile's coupling slice and, when they fit, the residual rows it will write.
-    const int opt = p.out_per_tile;
-    const int col0 = tile_first * opt;
-    const bool coupled = p.coupling != nullptr;
-    const int rows_base = coupled ? p.m_primary : p.M;
-    const int r0 = rank * rows_base / p.C, r1 = (rank + 1) * rows_base / p.C;
-    const int nrows = (r1 - r0) * (coupled ? 2 : 1);
-    if (coupled) {
-      for (int i = threadIdx.x; i < opt; i += kThreads)
-        cpl_s[i] = (col0 + i < p.n_out) ? __bfloat162float(p.coupling[col0 + i]) : 0.f;
-    }
-    if (p.epilogue == DF_EPI_RESIDUAL &&
-        nrows * opt * 2 <= 4 * 32 * kStgPitch * 4) {
-      __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(stg_all);
-      const int vec = opt / 8;  // 16-byte vectors per row
-      for (int i = threadIdx.x; i < nrows * vec; i += kThreads) {
-        const int rl = i / vec, v = i % vec;
-        const int pass = rl / (r1 - r0), rr = rl % (r1 - r0);
-        const int row = (pass == 1 ? p.m_primary : 0) + r0 + rr;
-        const int col = col0 + v * 8;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (row < p.M && col < p.n_out)
-          val = *reinterpret_cast<const uint4*>(p.residual + row * p.ldr + col);
-        reinterpret_cast<uint4*>(rs)[i] = val;
-      }
-      res_s = rs;
-    }
-  }
+  const __nv_bfloat16* res_s =
+      flags[1] ? reinterpret_cast<const __nv_bfloat16*>(stg_all) : nullptr;
   if (p.C > 1) {
-    cluster_sync_all();  // every accumulator of the cluster is parked
-    if (!flags[0]) {
-      float* prim = reinterpret_cast<float*>(smem) + kBM * (p.BN + 4);
-      cluster_epilogue(p, tile_first, rank, smem_u32(smem), prim, threadIdx.x, kThreads, res_s,
-                       cpl_s);
+    const int pitch = p.BN + 4;
+    const size_t slot_floats = static_cast<size_t>(kBM) * pitch;
+    if (threadIdx.x == 0) {
+      // parked rows -> this CTA's slot (every parking thread fenced its writes
+      // toward the async proxy before the CTA barrier above)
+      bulk_store_s2g(p.part + blockIdx.x * slot_floats, smem_u32(smem),
+                     static_cast<uint32_t>(slot_floats * 4));
+      bulk_store_commit_and_wait();
+      fence_proxy_async_global();
     }
-    cluster_sync_all();  // no CTA leaves while others still read its shared memory
+    cluster_sync_all();  // every slot of the cluster is written; the rings are free
+    int r0, r1;
+    owned_rows(p, rank, r0, r1);
+    const int n = r1 - r0;
+    const bool coupled = p.coupling != nullptr;
+    const int nloc = (coupled ? 2 : 1) * n;
+    float* recv = reinterpret_cast<float*>(smem);  // [C][nloc][pitch]
+    float* prim = recv + p.C * nloc * pitch;       // [n][out_per_tile]
+    bool ok = !flags[0];
+    if (threadIdx.x == 0) {
+      fence_proxy_async_global();
+      const uint32_t row_bytes = static_cast<uint32_t>(pitch * 4);
+      mbar_arrive_expect_tx(red_full, static_cast<uint32_t>(p.C * nloc) * row_bytes);
+      if (n > 0) {
+        const float* base = p.part + (blockIdx.x - rank) * slot_floats;  // rank 0's slot
+        for (int q = 0; q < p.C; ++q) {
+          const float* slot = base + q * slot_floats;
+          bulk_load_g2s(smem_u32(recv + (q * nloc) * pitch), slot + r0 * pitch,
+                        static_cast<uint32_t>(n) * row_bytes, red_full);
+          if (coupled)
+            bulk_load_g2s(smem_u32(recv + (q * nloc + n) * pitch),
+                          slot + (p.m_primary + r0) * pitch, static_cast<uint32_t>(n) * row_bytes,
+                          red_full);
+        }
+      }
+    }
+    if (!mbar_wait(red_full, 0)) ok = false;
+    ok = __syncthreads_and(ok) != 0;  // uniform: cluster_epilogue has CTA barriers
+    if (!ok) {
+      if (threadIdx.x == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+    } else {
+      cluster_epilogue(p, tile_first, rank, recv, prim, threadIdx.x, kThreads, res_s, cpl_s);
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -596,7 +658,7 @@ struct Plan {
 // ~46 GB/s of DRAM and ~77 GB/s of total TMA traffic per SM (measured with a
 // TMA streaming probe on B200), plus fixed costs for the cluster exchange and
 // per-tile epilogues.
-Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps) {
+Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_t ws_bytes) {
   Plan best{};
   best.ok = false;
   best.est_us = 1e30;
@@ -617,7 +679,11 @@ Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps) {
         tpc = static_cast<int>(ceil_div(n_tiles, ctas));
       } else {
         if (!caps || n_tiles > caps->max_clusters[C]) continue;
-        if (C > 1 && kBM * (BN + 4) * 4 + 32 * BN * 4 > kRingBytes) continue;
+        // parked tile; then C partials of <= ceil(rows / C) (x2 coupled) own
+        // rows plus the coupled primary results, all within the ring
+        if (kBM * (BN + 4) * 4 > kRingBytes) continue;
+        if ((kBM + 2 * C) * (BN + 4) * 4 + 32 * BN * 4 > kRingBytes) continue;
+        if (static_cast<size_t>(n_tiles) * C * kBM * (BN + 4) * 4 > ws_bytes) continue;
         ctas = n_tiles * C;
         tpc = 1;
       }
@@ -651,8 +717,8 @@ double stream_k_estimate(int N, int K, int epilogue) {
   return t + 2.5 + 3.0 + (split ? 7.0 : 0.0);
 }
 
-int planned_launches(int M, int N, int K, int epilogue) {
-  const Plan pl = make_plan(M, N, K, epilogue, caps_for_device());
+int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes) {
+  const Plan pl = make_plan(M, N, K, epilogue, caps_for_device(), ws_bytes);
   if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(N, K, epilogue)) return 0;
   return 1;
 }
@@ -661,7 +727,7 @@ int launch_if_better(const Request& r) {
   const int M = r.m_primary + r.m_aux;
   const ClusterCaps* caps = caps_for_device();
   if (!caps) return 0;
-  const Plan pl = make_plan(M, r.N, r.K, r.epilogue, caps);
+  const Plan pl = make_plan(M, r.N, r.K, r.epilogue, caps, r.workspace ? r.workspace_bytes : 0);
   if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(r.N, r.K, r.epilogue))
     return 0;
   const bool swiglu = r.epilogue == DF_EPI_SWIGLU;
@@ -686,6 +752,7 @@ int launch_if_better(const Request& r) {
   p.coupling = static_cast<const __nv_bfloat16*>(r.coupling);
   p.residual = static_cast<const __nv_bfloat16*>(r.residual);
   p.ldr = r.ldr;
+  p.part = static_cast<float*>(r.workspace);
   p.err = r.err;
   CUtensorMap tmX, tmW;
   if (!encode_tmap_bf16_2d(&tmX, r.x, static_cast<uint64_t>(M), static_cast<uint64_t>(r.K),

@@ -22,6 +22,8 @@ struct Request {
   int64_t ldr;
   int32_t* err;
   cudaStream_t stream;
+  void* workspace;  // fp32 partial slots of the cluster split-K reduction
+  size_t workspace_bytes;
 };
 
 // Launches the tile plan when it is modelled to beat stream-K on this device.
@@ -29,8 +31,9 @@ struct Request {
 // error. Arguments must already be validated.
 int launch_if_better(const Request& r);
 
-// 1 if the tile plan would be used for this shape on the current device, else 0.
-int planned_launches(int M, int N, int K, int epilogue);
+// 1 if the tile plan would be used for this shape on the current device with
+// a workspace of ws_bytes, else 0.
+int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes);
 
 }  // namespace tgemm
 }  // namespace df

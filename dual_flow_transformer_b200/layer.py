@@ -72,15 +72,20 @@ class DualFlowLayer:
 
     # ------------------------------------------------------------ CUDA graphs
     def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):
-        """Capture the step as three CUDA graphs (before attention, attention,
-        after attention) over fixed buffers, so a step costs three graph
-        launches instead of nine library calls from Python. The step runs once
-        eagerly first, so one-time host set-up happens outside the capture.
-        Events recorded between the graphs time the attention on the stream."""
+        """Capture the step over fixed buffers as one CUDA graph (one launch
+        per step; consecutive kernels keep their programmatic-dependent-launch
+        overlap) and, for timing the attention alone, as three graphs (before
+        attention, attention, after attention) with events between them. The
+        step runs once eagerly first, so one-time host set-up happens outside
+        the captures."""
         args = (X, k_cache, v_cache, block_table, positions, seqlens)
         self.step(*args)
         torch.cuda.synchronize()
         self._graph_args = args
+        self.graph_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_full):
+            for part in ("pre", "attn", "post"):
+                self._step_part(part, *args)
         self.graphs = []
         for part in ("pre", "attn", "post"):
             g = torch.cuda.CUDAGraph()
@@ -90,14 +95,16 @@ class DualFlowLayer:
         torch.cuda.synchronize()
 
     def replay(self, timers=None):
-        """One captured step on the current stream. timers: optional
-        {"attn": (start_event, end_event)} recorded around the attention."""
+        """One captured step on the current stream: the single-graph step, or
+        with timers ({"attn": (start_event, end_event)}) the three-graph step
+        with the events recorded around the attention."""
+        if timers is None:
+            self.graph_full.replay()
+            return self.x_out
         self.graphs[0].replay()
-        if timers is not None:
-            timers["attn"][0].record()
+        timers["attn"][0].record()
         self.graphs[1].replay()
-        if timers is not None:
-            timers["attn"][1].record()
+        timers["attn"][1].record()
         self.graphs[2].replay()
         return self.x_out
 
