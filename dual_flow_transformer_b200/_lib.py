@@ -54,6 +54,14 @@ SIGNATURES = {
         _vp, _c_i64,                    # y, ldy
         _c_int, _vp, _vp, _c_i64,       # epilogue, coupling, residual, ldr
         _vp, _c_size, _vp, _vp]),       # workspace, bytes, err_flag, stream
+    "dualflow_grouped_proj_chain": (_c_int, [
+        _vp, _c_i64, _c_int, _c_int,    # x, ldx, m_primary, m_aux
+        _vp, _c_int, _c_int, _c_int,    # w, N, K, n_aux
+        _vp, _c_i64,                    # y, ldy
+        _c_int, _vp, _vp, _c_i64,       # epilogue, coupling, residual, ldr
+        _vp, _c_size,                   # workspace, bytes
+        _vp, _c_int, _c_int, _c_int,    # w_next, N_next, K_next, epilogue_next
+        _vp, _vp]),                     # err_flag, stream
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
 }
 

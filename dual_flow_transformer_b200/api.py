@@ -153,13 +153,17 @@ def new_proj_workspace(M, N, K, epilogue="none", device="cuda"):
 
 
 def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupling=None,
-                 residual=None, workspace=None, err_flag=None, stream=None):
+                 residual=None, workspace=None, err_flag=None, stream=None, next_w=None,
+                 next_epilogue="none"):
     """y = epilogue(x w^T) for both flows' rows in one GEMM.
 
     x: bf16 [M, K] (row stride multiple of 8), rows [0, m_primary) primary,
     the rest auxiliary; w: bf16 [N, K] contiguous. epilogue "swiglu": w is
     [W_gate; W_up] and y is [M, N/2]; "residual": y = residual + x w^T.
     coupling: b (swiglu) or c (residual) vector, bf16, or None.
+    next_w / next_epilogue: the projection launched next on this stream (same
+    rows and workspace size); its first weight blocks are prefetched into L2
+    while this one finishes. A cache hint only: results do not change.
     """
     M, K = x.shape
     N, K2 = w.shape
@@ -171,12 +175,20 @@ def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupli
         y = torch.empty((M, n_out), dtype=x.dtype, device=x.device)
     if workspace is None:
         workspace = new_proj_workspace(M, N, K, epilogue, x.device)
-    st = _lib().dualflow_grouped_proj(
-        _ptr(x), x.stride(0), int(m_primary), int(M - m_primary), _ptr(w), N, K,
-        n_out if n_aux is None else int(n_aux), _ptr(y), y.stride(0), epi, _ptr(coupling),
-        _ptr(residual), 0 if residual is None else residual.stride(0), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream))
-    L.check("dualflow_grouped_proj", st)
+    args = (_ptr(x), x.stride(0), int(m_primary), int(M - m_primary), _ptr(w), N, K,
+            n_out if n_aux is None else int(n_aux), _ptr(y), y.stride(0), epi, _ptr(coupling),
+            _ptr(residual), 0 if residual is None else residual.stride(0), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    if next_w is None:
+        st = _lib().dualflow_grouped_proj(*args, _ptr(err_flag), _stream(stream))
+        L.check("dualflow_grouped_proj", st)
+    else:
+        if not next_w.is_contiguous() or next_w.dtype != torch.bfloat16:
+            raise ValueError("next_w must be a contiguous bf16 [N, K] weight")
+        st = _lib().dualflow_grouped_proj_chain(*args, _ptr(next_w), next_w.shape[0],
+                                                next_w.shape[1], EPILOGUES[next_epilogue],
+                                                _ptr(err_flag), _stream(stream))
+        L.check("dualflow_grouped_proj_chain", st)
     return y
 
 

@@ -543,15 +543,23 @@ extern "C" int dualflow_grouped_proj_num_launches(int M, int N, int K, int epilo
   return 1;
 }
 
-extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
-                                           const void* w, int N, int K, int n_aux, void* y,
-                                           int64_t ldy, int epilogue, const void* coupling,
-                                           const void* residual, int64_t ldr, void* workspace,
-                                           size_t workspace_bytes, int32_t* err_flag,
-                                           void* stream) {
+namespace {
+
+df_status grouped_proj_impl(const void* x, int64_t ldx, int m_primary, int m_aux, const void* w,
+                            int N, int K, int n_aux, void* y, int64_t ldy, int epilogue,
+                            const void* coupling, const void* residual, int64_t ldr,
+                            void* workspace, size_t workspace_bytes, const void* w_next,
+                            int N_next, int K_next, int epilogue_next, int32_t* err_flag,
+                            void* stream) {
   using namespace df;
   using namespace df::gemm;
   if (!x || !w || !y) return DF_ERR_NULL;
+  if (w_next) {
+    if (epilogue_next < DF_EPI_NONE || epilogue_next > DF_EPI_RESIDUAL) return DF_ERR_UNSUPPORTED;
+    if (N_next < 128 || K_next < kBK || N_next % 128 != 0 || K_next % kBK != 0)
+      return DF_ERR_UNSUPPORTED;
+    if (!aligned(w_next, 16)) return DF_ERR_ALIGN;
+  }
   if (epilogue < DF_EPI_NONE || epilogue > DF_EPI_RESIDUAL) return DF_ERR_UNSUPPORTED;
   if (epilogue == DF_EPI_RESIDUAL && !residual) return DF_ERR_NULL;
   if (epilogue == DF_EPI_NONE && (coupling || residual)) return DF_ERR_SHAPE;
@@ -600,7 +608,8 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   {
     // tile-parallel / cluster split-K plan when it is modelled to be faster
     tgemm::Request rq{x, lx, m_primary, m_aux, w, N, K, n_aux, y, ly, epilogue, coupling,
-                      residual, lr, err_flag, st, workspace, workspace_bytes};
+                      residual, lr, err_flag, st, workspace, workspace_bytes,
+                      w_next, N_next, K_next, epilogue_next};
     const int launched = tgemm::launch_if_better(rq);
     if (launched < 0) return DF_ERR_CUDA;
     if (launched > 0) return DF_OK;
@@ -636,4 +645,27 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
       return DF_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m_aux,
+                                           const void* w, int N, int K, int n_aux, void* y,
+                                           int64_t ldy, int epilogue, const void* coupling,
+                                           const void* residual, int64_t ldr, void* workspace,
+                                           size_t workspace_bytes, int32_t* err_flag,
+                                           void* stream) {
+  return grouped_proj_impl(x, ldx, m_primary, m_aux, w, N, K, n_aux, y, ldy, epilogue, coupling,
+                           residual, ldr, workspace, workspace_bytes, nullptr, 0, 0, 0, err_flag,
+                           stream);
+}
+
+extern "C" df_status dualflow_grouped_proj_chain(
+    const void* x, int64_t ldx, int m_primary, int m_aux, const void* w, int N, int K, int n_aux,
+    void* y, int64_t ldy, int epilogue, const void* coupling, const void* residual, int64_t ldr,
+    void* workspace, size_t workspace_bytes, const void* w_next, int N_next, int K_next,
+    int epilogue_next, int32_t* err_flag, void* stream) {
+  return grouped_proj_impl(x, ldx, m_primary, m_aux, w, N, K, n_aux, y, ldy, epilogue, coupling,
+                           residual, ldr, workspace, workspace_bytes, w_next, N_next, K_next,
+                           epilogue_next, err_flag, stream);
 }

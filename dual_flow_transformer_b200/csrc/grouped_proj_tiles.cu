@@ -19,6 +19,7 @@
 // The producer/MMA/epilogue warp roles, the TMA ring and the bounded waits are
 // as in the stream-K kernel.
 #include <math.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -60,6 +61,11 @@ struct Params {
   int64_t ldr;
   float* part;  // C > 1: [ctas][kBM][BN + 4] fp32 partial accumulators
   int32_t* err;
+  // L2 prefetch for the next projection (pf_stages 0 = none): its plan's tile
+  // width, cluster size, tile and CTA counts, k-blocks, SwiGLU half width and
+  // gate/up offset; pf_stages k-blocks from the start of each of its CTAs'
+  // slices.
+  int pf_stages, pf_BN, pf_C, pf_ntiles, pf_ctas, pf_kblocks, pf_half, pf_F;
 };
 
 __device__ __forceinline__ void epi_bar() {
@@ -307,7 +313,8 @@ __device__ void cluster_epilogue(const Params& p, int tile, int rank, const floa
 
 __global__ void __launch_bounds__(kThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
-                     const __grid_constant__ CUtensorMap tmW, const Params p) {
+                     const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmWn, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -422,6 +429,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (long long i = (n > S ? n - S : 0); i < n; ++i)
         mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1));
+      // This CTA's weights have landed: while the tile finishes (DRAM is
+      // otherwise idle in the tail), warm L2 with the first k-blocks that the
+      // next projection's CTAs j = blockIdx.x (mod gridDim.x) stream first.
+      if (ok && p.pf_stages > 0) {
+        prefetch_tensormap(&tmWn);
+        for (int j = blockIdx.x; j < p.pf_ctas; j += gridDim.x) {
+          int t = j, k0 = 0, k1 = p.pf_kblocks;
+          if (p.pf_C > 1) {
+            t = j / p.pf_C;
+            const int r = j % p.pf_C;
+            k0 = r * p.pf_kblocks / p.pf_C;
+            k1 = (r + 1) * p.pf_kblocks / p.pf_C;
+          }
+          if (t >= p.pf_ntiles) continue;
+          for (int kb = k0; kb < k1 && kb < k0 + p.pf_stages; ++kb) {
+            if (p.pf_half > 0) {
+              tma_prefetch_2d(&tmWn, kb * kBK, t * p.pf_half);
+              tma_prefetch_2d(&tmWn, kb * kBK, p.pf_F + t * p.pf_half);
+            } else {
+              tma_prefetch_2d(&tmWn, kb * kBK, t * p.pf_BN);
+            }
+          }
+        }
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -754,6 +785,32 @@ int launch_if_better(const Request& r) {
   p.ldr = r.ldr;
   p.part = static_cast<float*>(r.workspace);
   p.err = r.err;
+  CUtensorMap tmWn;
+  memset(&tmWn, 0, sizeof(tmWn));
+  if (r.w_next != nullptr) {
+    const size_t ws = r.workspace ? r.workspace_bytes : 0;
+    const Plan nx = make_plan(M, r.N_next, r.K_next, r.epilogue_next, caps, ws);
+    const bool nx_tiles = nx.ok && nx.ctas >= kSms * 3 / 4 &&
+                          nx.est_us < stream_k_estimate(r.N_next, r.K_next, r.epilogue_next);
+    const bool nx_swiglu = r.epilogue_next == DF_EPI_SWIGLU;
+    const int box_rows = nx_swiglu ? nx.BN / 2 : nx.BN;
+    if (nx_tiles &&
+        encode_tmap_bf16_2d(&tmWn, r.w_next, static_cast<uint64_t>(r.N_next),
+                            static_cast<uint64_t>(r.K_next), static_cast<uint64_t>(r.K_next) * 2,
+                            box_rows, kBK)) {
+      // ~28 MB in all: what DRAM delivers in a few microseconds of tail
+      const double per_stage = static_cast<double>(nx.ctas) * nx.BN * kBK * 2;
+      int st = static_cast<int>(28.0 * 1024 * 1024 / per_stage);
+      p.pf_stages = st < 1 ? 1 : (st > 16 ? 16 : st);
+      p.pf_BN = nx.BN;
+      p.pf_C = nx.C;
+      p.pf_ntiles = nx.n_tiles;
+      p.pf_ctas = nx.ctas;
+      p.pf_kblocks = r.K_next / kBK;
+      p.pf_half = nx_swiglu ? nx.BN / 2 : 0;
+      p.pf_F = r.N_next / 2;
+    }
+  }
   CUtensorMap tmX, tmW;
   if (!encode_tmap_bf16_2d(&tmX, r.x, static_cast<uint64_t>(M), static_cast<uint64_t>(r.K),
                            static_cast<uint64_t>(r.ldx) * 2, kBM, kBK) ||
@@ -774,7 +831,7 @@ int launch_if_better(const Request& r) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, tile_gemm_kernel, tmX, tmW, p) != cudaSuccess) return -1;
+  if (cudaLaunchKernelEx(&cfg, tile_gemm_kernel, tmX, tmW, tmWn, p) != cudaSuccess) return -1;
   return 1;
 }
 

@@ -24,6 +24,11 @@ struct Request {
   cudaStream_t stream;
   void* workspace;  // fp32 partial slots of the cluster split-K reduction
   size_t workspace_bytes;
+  // Optional: the projection launched next on the stream (same rows and
+  // workspace size); its first k-blocks are prefetched into L2 during this
+  // launch's tail. w_next NULL = none.
+  const void* w_next;
+  int N_next, K_next, epilogue_next;
 };
 
 // Launches the tile plan when it is modelled to beat stream-K on this device.

@@ -130,6 +130,9 @@ class DualFlowLayer:
         qd, kvd = Hq * D, Hkv * D
         w = self.w
         qkv = self.qkv
+        # Each projection warms L2 with the first weight blocks of the next one
+        # (o -> gate/up -> down -> the next step's QKV); none after the QKV
+        # projection, whose successor is the HBM-bound attention.
         if part == "pre":
             api.rmsnorm(X, y=self.xn, eps=self.eps, stream=stream)
             api.grouped_proj(self.xn, B, w["w_qkv"], n_aux=qd, y=qkv, workspace=self.proj_ws,
@@ -146,14 +149,15 @@ class DualFlowLayer:
         else:
             api.grouped_proj(self.attn, B, w["w_o"], y=self.x_mid, epilogue="residual",
                              residual=X, workspace=self.proj_ws, err_flag=self.err,
-                             stream=stream)
+                             stream=stream, next_w=w["w_gu"], next_epilogue="swiglu")
             api.rmsnorm(self.x_mid, y=self.xn2, eps=self.eps, stream=stream)
             api.grouped_proj(self.xn2, B, w["w_gu"], y=self.h, epilogue="swiglu",
                              coupling=w["b"], workspace=self.proj_ws, err_flag=self.err,
-                             stream=stream)
+                             stream=stream, next_w=w["w_down"], next_epilogue="residual")
             api.grouped_proj(self.h, B, w["w_down"], y=self.x_out, epilogue="residual",
                              coupling=w["c"], residual=self.x_mid, workspace=self.proj_ws,
-                             err_flag=self.err, stream=stream)
+                             err_flag=self.err, stream=stream, next_w=w["w_qkv"],
+                             next_epilogue="none")
 
 
     def step_host(self, x_host, out_host, k_cache, v_cache, block_table, positions, seqlens,

@@ -232,6 +232,23 @@ df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_primary, int m
                                 int64_t ldr, void* workspace, size_t workspace_bytes,
                                 int32_t* err_flag, void* stream);
 
+/* Same projection, and a hint for the projection that will be launched next */
+/* on the same stream with the same rows and workspace size: weight w_next   */
+/* (bf16 [N_next][K_next], 16-byte aligned, K_next % 64 == 0, N_next % 128   */
+/* == 0) and epilogue_next. While this call's tiles finish (the weights have */
+/* streamed, HBM is idle), its CTAs prefetch into L2 the first k-blocks that  */
+/* each CTA of the next call will read, so the next call starts from L2      */
+/* instead of a cold HBM pipeline. Results are identical with or without the */
+/* hint; w_next NULL = no hint. The prefetch is a cache hint only: w_next is */
+/* never written, and a next call with other arguments is still correct.     */
+df_status dualflow_grouped_proj_chain(const void* x, int64_t ldx, int m_primary, int m_aux,
+                                      const void* w, int N, int K, int n_aux, void* y,
+                                      int64_t ldy, int epilogue, const void* coupling,
+                                      const void* residual, int64_t ldr, void* workspace,
+                                      size_t workspace_bytes, const void* w_next, int N_next,
+                                      int K_next, int epilogue_next, int32_t* err_flag,
+                                      void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Row RMS normalisation (layer step, pre-attention and pre-MLP).            */
 /*                                                                           */

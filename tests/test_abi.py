@@ -138,3 +138,14 @@ def test_rmsnorm_rejects_invalid_arguments(lib):
     assert f(FAKE, 0, None, FAKE, 0, 4, 60, 1e-5, None) == L.DF_ERR_UNSUPPORTED
     assert f(FAKE + 2, 0, None, FAKE, 0, 4, 64, 1e-5, None) == L.DF_ERR_ALIGN
     assert f(FAKE, 0, None, FAKE, 0, 4, 64, -1.0, None) == L.DF_ERR_SHAPE
+
+
+def test_grouped_proj_chain_rejects_invalid_next_projection(lib):
+    f = lib.dualflow_grouped_proj_chain
+    base = [FAKE, 0, 64, 64, FAKE, 4096, 4096, 4096, FAKE, 0, 0, None, None, 0, FAKE, 1 << 30]
+    tail = [None, None]
+    assert f(*base, FAKE, 4000, 4096, 0, *tail) == L.DF_ERR_UNSUPPORTED   # N_next % 128
+    assert f(*base, FAKE, 4096, 4000, 0, *tail) == L.DF_ERR_UNSUPPORTED   # K_next % 64
+    assert f(*base, FAKE, 4096, 4096, 7, *tail) == L.DF_ERR_UNSUPPORTED   # epilogue_next
+    assert f(*base, FAKE + 8, 4096, 4096, 0, *tail) == L.DF_ERR_ALIGN     # w_next alignment
+    assert f(None, *base[1:], FAKE, 4096, 4096, 0, *tail) == L.DF_ERR_NULL

@@ -166,3 +166,37 @@ def test_medium_shapes_sampled(cuda_device, shape, epi, coupled):
         ref = _oracle(x, w[cols], mp, epi, None if cpl is None else cpl[cols],
                       None if res is None else res[:, cols])
     assert_close(y[:, cols], ref, "bf16", "medium %s %s" % (shape, epi))
+
+
+@pytest.mark.parametrize("cur,nxt", [(("w_o", "residual"), ("w_gu", "swiglu")),
+                                     (("w_gu", "swiglu"), ("w_down", "residual")),
+                                     (("w_down", "residual"), ("w_qkv", "none"))])
+def test_next_projection_hint_changes_no_bit(cuda_device, cur, nxt):
+    """The chained entry (L2 prefetch of the next projection's first weight
+    blocks) gives the same bits as the plain call, at the layer's shapes; the
+    next projection, run after it, is unchanged too."""
+    dev = cuda_device
+    shapes = {"w_qkv": (6144, 4096), "w_o": (4096, 4096), "w_gu": (2 * 14336, 4096),
+              "w_down": (4096, 14336)}
+    g = torch.Generator().manual_seed(41)
+    (wk, epi), (nk, nepi) = cur, nxt
+    N, K = shapes[wk]
+    Nn, Kn = shapes[nk]
+    n_out = N // 2 if epi == "swiglu" else N
+    x = _rand(g, (128, K)).to(dev)
+    w = _rand(g, (N, K), 0.02).to(dev)
+    wn = _rand(g, (Nn, Kn), 0.02).to(dev)
+    xn = _rand(g, (128, Kn)).to(dev)
+    cpl = _rand(g, (n_out,), 0.1).to(dev) if epi != "none" else None
+    res = _rand(g, (128, n_out)).to(dev) if epi == "residual" else None
+    ws = api.new_proj_workspace(128, max(N, Nn), max(K, Kn), "swiglu", dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    kw = dict(epilogue=epi, coupling=cpl, residual=res, workspace=ws, err_flag=err)
+    y_plain = api.grouped_proj(x, 64, w, **kw)
+    yn_plain = api.grouped_proj(xn, 64, wn, epilogue="none", workspace=ws, err_flag=err)
+    y_hint = api.grouped_proj(x, 64, w, next_w=wn, next_epilogue=nepi, **kw)
+    yn_hint = api.grouped_proj(xn, 64, wn, epilogue="none", workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(y_plain.view(torch.int16), y_hint.view(torch.int16))
+    assert torch.equal(yn_plain.view(torch.int16), yn_hint.view(torch.int16))
