@@ -19,4 +19,8 @@ from .dualflow_oracle import (  # noqa: F401
     residual_couple,
     rmsnorm,
     layer_step,
+    softmax_rows,
+    collision_probability,
+    mixture_weight,
+    mixture_head,
 )

@@ -27,6 +27,11 @@ of the function that takes it:
 * Layer step      pre-attention and pre-MLP RMSNorm (unit gain, eps 1e-5),
   residual adds, SwiGLU MLP, no positional rotation.
   PARITY UNPINNED against the pages (the pages name no norm, no MLP form).
+* Mixture head    p_mix = alpha p1 + (1 - alpha) p2 is the pages' formula;
+  the map from the primary's collision probability to alpha is a reading,
+  alpha = 1/2 + 1/2 sum(p1^2). Pinned by its limits (uniform and one-hot
+  primary) and invariants; the map itself is PARITY UNPINNED against the
+  pages beyond those limits.
 
 Attention itself (scores, softmax, weighted sum of V) is the textbook
 definition written out, so it is pinned by brute force, closed forms and a
@@ -309,3 +314,50 @@ def layer_step(x1, x2, w_qkv, w_o, w_gu, w_down, a, b, c, k_cache, v_cache,
         "xn": xn, "qkv": qkv, "k_cache": kc, "v_cache": vc, "attn": attn,
         "x_mid": x_mid, "xn2": xn2, "h": h, "x_out": x_out,
     }
+
+
+# ----------------------------------------------------------------- mixture head
+
+def softmax_rows(logits):
+    """Row softmax p_v = exp(l_v - max l) / sum_u exp(l_u - max l), in fp64."""
+    l = np.asarray(logits, dtype=F64)
+    m = l.max(axis=-1, keepdims=True)
+    e = np.exp(l - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def collision_probability(p):
+    """sum_v p_v^2 per row: the chance that two independent draws from p agree
+    (1 for a one-hot p, 1/V for a uniform p over V outcomes)."""
+    p = np.asarray(p, dtype=F64)
+    return (p * p).sum(axis=-1)
+
+
+def mixture_weight(p1):
+    """Weight of the primary distribution in the mixture.
+
+    "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi Chiave"
+    (mixture objective): the weight follows the primary distribution's
+    confidence, measured by its collision probability, and keeps the primary
+    at least half of the mixture at inference. The map is not printed; the
+    reading taken here is the plainest monotone one onto [1/2, 1]:
+        alpha = 1/2 + 1/2 * sum_v p1_v^2.
+    """
+    return 0.5 + 0.5 * collision_probability(p1)
+
+
+def mixture_head(logits, B):
+    """Mixed next-token distribution of both flows.
+
+    logits: [2B][V], primary rows 0..B-1, auxiliary rows B..2B-1 (the grouped
+    LM-head projection's output; same section as `mixture_weight`):
+        p1 = softmax(logits[b]), p2 = softmax(logits[B + b]),
+        alpha_b = mixture_weight(p1),
+        p_mix[b] = alpha_b * p1 + (1 - alpha_b) * p2.
+    Returns (p_mix [B][V], alpha [B]), fp64.
+    """
+    l = np.asarray(logits, dtype=F64)
+    p1 = softmax_rows(l[:B])
+    p2 = softmax_rows(l[B:2 * B])
+    alpha = mixture_weight(p1)
+    return alpha[:, None] * p1 + (1.0 - alpha[:, None]) * p2, alpha

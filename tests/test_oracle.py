@@ -23,8 +23,14 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 def _num(s):
-    table = {"sqrt2ln3": math.sqrt(2) * math.log(3), "sqrt2ln3/2": math.sqrt(2) * math.log(3) / 2}
-    return table[s] if s in table else float(s)
+    table = {"sqrt2ln3": math.sqrt(2) * math.log(3), "sqrt2ln3/2": math.sqrt(2) * math.log(3) / 2,
+             "ln2": math.log(2), "ln3": math.log(3)}
+    if s in table:
+        return table[s]
+    if "/" in s:
+        num, den = s.split("/")
+        return float(int(num)) / float(int(den))
+    return float(s)
 
 
 def _arr(x):
@@ -431,3 +437,57 @@ def test_layer_with_zero_output_weights_is_identity_on_hidden_state():
     r = oracle.layer_step(**p, **dims)
     np.testing.assert_array_equal(r["x_out"], np.concatenate([p["x1"], p["x2"]]))
     np.testing.assert_array_equal(r["x_mid"], np.concatenate([p["x1"], p["x2"]]))
+
+
+# ---------------------------------------------------------------- mixture head
+
+def test_golden_mixture_worked_examples():
+    with open(os.path.join(GOLDEN, "mixture_worked_example.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        logits = _arr(c["logits"])
+        p_mix, alpha = oracle.mixture_head(logits, 1)
+        np.testing.assert_allclose(alpha, _arr(c["alpha"]), rtol=0, atol=1e-14, err_msg=c["name"])
+        np.testing.assert_allclose(p_mix, _arr(c["p_mix"]), rtol=0, atol=1e-14, err_msg=c["name"])
+
+
+def test_mixture_of_identical_flows_is_the_flow():
+    rng = np.random.default_rng(70)
+    l = rng.normal(size=(3, 50)) * 3
+    p_mix, alpha = oracle.mixture_head(np.concatenate([l, l]), 3)
+    e = np.exp(l - l.max(axis=1, keepdims=True))
+    np.testing.assert_allclose(p_mix, e / e.sum(axis=1, keepdims=True), rtol=1e-13, atol=0)
+    assert np.all(alpha > 0.5) and np.all(alpha < 1.0)
+
+
+def test_mixture_weight_limits():
+    V = 1000
+    # uniform primary: collision probability 1/V, alpha = 1/2 + 1/(2V)
+    l = np.concatenate([np.full((1, V), -2.5), np.zeros((1, V))])
+    _, alpha = oracle.mixture_head(l, 1)
+    assert alpha[0] == pytest.approx(0.5 + 0.5 / V, abs=1e-15)
+    # one-hot primary (a logit 1000 above the rest): alpha = 1, the mixture is
+    # the primary distribution (a swapped weight would give the aux one)
+    l1 = np.zeros(V)
+    l1[17] = 1000.0
+    l2 = np.linspace(-1, 1, V)
+    p_mix, alpha = oracle.mixture_head(np.stack([l1, l2]), 1)
+    assert alpha[0] == 1.0
+    assert p_mix[0, 17] == 1.0 and np.all(np.delete(p_mix[0], 17) == 0.0)
+
+
+def test_mixture_invariants_and_primary_only_weight():
+    rng = np.random.default_rng(71)
+    B, V = 4, 257
+    l = rng.normal(size=(2 * B, V)) * rng.uniform(0.1, 6, size=(2 * B, 1))
+    p_mix, alpha = oracle.mixture_head(l, B)
+    np.testing.assert_allclose(p_mix.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+    assert np.all(p_mix >= 0) and np.all((alpha >= 0.5) & (alpha <= 1.0))
+    # alpha reads only the primary rows: any aux logits (NaN included) leave it unchanged
+    l_bad = l.copy()
+    l_bad[B:] = np.nan
+    _, alpha_bad = oracle.mixture_head(l_bad, B)
+    np.testing.assert_array_equal(alpha, alpha_bad)
+    # a flow swap is visible: exchanging the rows changes the mixture
+    p_swap, _ = oracle.mixture_head(np.concatenate([l[B:], l[:B]]), B)
+    assert not np.allclose(p_swap, p_mix)
