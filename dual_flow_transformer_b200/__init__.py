@@ -13,6 +13,8 @@ from .api import (  # noqa: F401
     grouped_proj_num_launches,
     grouped_proj_workspace_size,
     kv_append,
+    mixture_head,
+    mixture_head_slices,
     new_attn_workspace,
     new_proj_workspace,
     rmsnorm,

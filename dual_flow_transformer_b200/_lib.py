@@ -62,6 +62,9 @@ SIGNATURES = {
         _vp, _c_size,                   # workspace, bytes
         _vp, _c_int, _c_int, _c_int,    # w_next, N_next, K_next, epilogue_next
         _vp, _vp]),                     # err_flag, stream
+    "dualflow_mixture_head": (_c_int, [_vp, _c_i64, _c_int, _c_int, _c_int, _vp, _c_i64, _vp,
+                                       _vp]),
+    "dualflow_mixture_head_slices": (_c_int, [_c_int, _c_int]),
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
 }
 

@@ -192,6 +192,33 @@ def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupli
     return y
 
 
+# ----------------------------------------------------------------- mixture head
+
+def mixture_head(logits, B, *, p_mix=None, alpha=None, stream=None):
+    """Mixed next-token distribution of both flows.
+
+    logits: [2B, V] bf16 or fp32 (primary rows, then auxiliary rows; unit
+    column stride). Returns (p_mix fp32 [B, V], alpha fp32 [B]) with
+    p_mix = alpha p1 + (1 - alpha) p2, alpha = 1/2 + 1/2 sum(p1^2).
+    """
+    rows, V = logits.shape
+    if rows < 2 * B or logits.stride(1) != 1:
+        raise ValueError("logits must be [2B, V] with unit column stride")
+    if p_mix is None:
+        p_mix = torch.empty((B, V), dtype=torch.float32, device=logits.device)
+    if alpha is None:
+        alpha = torch.empty((B,), dtype=torch.float32, device=logits.device)
+    st = _lib().dualflow_mixture_head(_ptr(logits), logits.stride(0), int(B), int(V),
+                                      dtype_code(logits.dtype), _ptr(p_mix), p_mix.stride(0),
+                                      _ptr(alpha), _stream(stream))
+    L.check("dualflow_mixture_head", st)
+    return p_mix, alpha
+
+
+def mixture_head_slices(B, V) -> int:
+    return _lib().dualflow_mixture_head_slices(int(B), int(V))
+
+
 # ----------------------------------------------------------------- norm
 
 def rmsnorm(x, gain=None, y=None, eps=1e-5, stream=None):

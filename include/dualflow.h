@@ -250,6 +250,30 @@ df_status dualflow_grouped_proj_chain(const void* x, int64_t ldx, int m_primary,
                                       void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Mixture head: the mixed next-token distribution of both flows.            */
+/*                                                                           */
+/* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi        */
+/* Chiave" (mixture objective): p_mix = alpha p1 + (1 - alpha) p2, the       */
+/* weight alpha set by the primary distribution's confidence (collision      */
+/* probability) and keeping the primary at least half of the mixture. The    */
+/* map is not printed; this library reads it as                               */
+/*   alpha_b = 1/2 + 1/2 * sum_v p1[b][v]^2   (in [1/2, 1]).                  */
+/* logits : [2B][V] row stride ld (0 = V), dtype DF_BF16 or DF_FP32; rows     */
+/*          0..B-1 primary, B..2B-1 auxiliary (the grouped LM-head           */
+/*          projection of both flows' final hidden states, one shared         */
+/*          output matrix); p1/p2 = softmax of the rows, fp32 arithmetic.      */
+/* p_mix  : fp32 [B][V] row stride ldp (0 = V), written.                     */
+/* alpha  : fp32 [B] written, or NULL. alpha reads only the primary rows, so  */
+/*          it is bit-identical for any auxiliary logits (NaN included).      */
+/* Supported: V % 8 == 0; ld % 8 == 0, ldp % 4 == 0; logits and p_mix        */
+/* 16-byte aligned. One kernel launch (thread-block clusters of              */
+/* dualflow_mixture_head_slices(B, V) CTAs per sequence); no workspace.      */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_mixture_head(const void* logits, int64_t ld, int B, int V, int dtype,
+                                float* p_mix, int64_t ldp, float* alpha, void* stream);
+int dualflow_mixture_head_slices(int B, int V);
+
+/* ------------------------------------------------------------------------ */
 /* Row RMS normalisation (layer step, pre-attention and pre-MLP).            */
 /*                                                                           */
 /* y[r][:] = x[r][:] / sqrt(mean(x[r][:]^2) + eps) * gain[:] (gain NULL = 1), */

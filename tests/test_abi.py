@@ -149,3 +149,25 @@ def test_grouped_proj_chain_rejects_invalid_next_projection(lib):
     assert f(*base, FAKE, 4096, 4096, 7, *tail) == L.DF_ERR_UNSUPPORTED   # epilogue_next
     assert f(*base, FAKE + 8, 4096, 4096, 0, *tail) == L.DF_ERR_ALIGN     # w_next alignment
     assert f(None, *base[1:], FAKE, 4096, 4096, 0, *tail) == L.DF_ERR_NULL
+
+
+def test_mixture_head_rejects_invalid_arguments(lib):
+    f = lib.dualflow_mixture_head
+    ok = dict(lg=FAKE, ld=0, B=4, V=4096, dt=L.DF_BF16, p=FAKE, ldp=0, a=FAKE, st=None)
+
+    def call(**over):
+        a = dict(ok)
+        a.update(over)
+        return f(a["lg"], a["ld"], a["B"], a["V"], a["dt"], a["p"], a["ldp"], a["a"], a["st"])
+
+    assert call(lg=None) == L.DF_ERR_NULL
+    assert call(p=None) == L.DF_ERR_NULL
+    assert call(B=0) == L.DF_ERR_SHAPE
+    assert call(ld=100) == L.DF_ERR_SHAPE          # row stride below V
+    assert call(V=4100) == L.DF_ERR_UNSUPPORTED    # V % 8
+    assert call(dt=7) == L.DF_ERR_UNSUPPORTED
+    assert call(lg=FAKE + 8) == L.DF_ERR_ALIGN
+    assert call(ldp=4098) == L.DF_ERR_ALIGN
+    assert call(ld=4100) == L.DF_ERR_ALIGN
+    sl = lib.dualflow_mixture_head_slices
+    assert sl(64, 32000) == 5 and sl(1, 32000) == 8 and sl(4, 1024) == 1 and sl(0, 8) == 0
