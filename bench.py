@@ -49,7 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "mha", "gqa", "long", "tiny"], default="layer")
+    ap.add_argument("--workload", choices=["layer", "mha", "gqa", "long", "tiny", "mixture"],
+                    default="layer")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -331,6 +332,91 @@ class AttnRun:
         return int(self.err.item())
 
 
+class MixtureRun:
+    """Mixture head step: grouped LM-head projection of both flows' final
+    hidden states (shared output matrix) + the mixed next-token distribution."""
+
+    timer_keys = ("proj", "mix")
+    dominant_key = "proj"
+
+    def __init__(self, args, dev, seed):
+        import torch
+        from dual_flow_transformer_b200 import api, synth
+        w = synth.WORKLOADS["mixture"]
+        self.w = w
+        self.api = api
+        self.host = synth.make_mixture_inputs(w, seed=seed)
+        h = self.host
+        self.X = torch.cat([h["h1"], h["h2"]]).contiguous().to(dev)
+        self.W = h["w_head"].to(dev)
+        B, V, d = w.B, w.V, w.d_model
+        self.ws = api.new_proj_workspace(2 * B, V, d, "none", dev)
+        self.logits = torch.empty((2 * B, V), dtype=torch.bfloat16, device=dev)
+        self.p_mix = torch.empty((B, V), dtype=torch.float32, device=dev)
+        self.alpha = torch.empty((B,), dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.tokens_per_step = B
+        self.launches_per_step = api.grouped_proj_num_launches(2 * B, V, d, "none") + 1
+        # LM-head projection: weights once (one [d] row per vocabulary entry),
+        # activations in, bf16 logits out
+        self.units = V
+        self.bytes_per_unit = d * 2
+        self.dom_bytes = V * d * 2 + 2 * B * d * 2 + 2 * B * V * 2
+        # mixture kernel: logits read once, p_mix and alpha written once
+        self.mix_bytes = 2 * B * V * 2 + B * V * 4 + B * 4
+        self.config = {"workload": "dual-flow mixture head: LM-head projection of both flows "
+                                   "(batch %d per flow, M=%d, d_model %d, vocabulary %d, bf16 "
+                                   "weights %.1f MB) + mixed next-token distribution (fp32)"
+                                   % (B, 2 * B, d, V, V * d * 2 / 1e6),
+                       "l2": "inputs larger than L2 (%.0f MB of weights per step)"
+                             % (V * d * 2 / 1e6)}
+        self.dominant = "dualflow_grouped_proj (LM head, tcgen05)"
+        self._proj()
+        self._mix()
+        torch.cuda.synchronize()
+        self.g_full, self.g_proj, self.g_mix = (torch.cuda.CUDAGraph() for _ in range(3))
+        with torch.cuda.graph(self.g_full):
+            self._proj()
+            self._mix()
+        with torch.cuda.graph(self.g_proj):
+            self._proj()
+        with torch.cuda.graph(self.g_mix):
+            self._mix()
+        torch.cuda.synchronize()
+
+    def _proj(self):
+        self.api.grouped_proj(self.X, self.w.B, self.W, y=self.logits, workspace=self.ws,
+                              err_flag=self.err)
+
+    def _mix(self):
+        self.api.mixture_head(self.logits, self.w.B, p_mix=self.p_mix, alpha=self.alpha)
+
+    def step(self, timers=None):
+        if timers is None:
+            self.g_full.replay()
+            return
+        timers["proj"][0].record()
+        self.g_proj.replay()
+        timers["proj"][1].record()
+        timers["mix"][0].record()
+        self.g_mix.replay()
+        timers["mix"][1].record()
+
+    def host_io(self):
+        import torch
+        x = self.X.cpu().pin_memory()
+        o = torch.empty(tuple(self.p_mix.shape), dtype=torch.float32).pin_memory()
+        return x, o
+
+    def step_host(self, x_host, o_host):
+        self.X.copy_(x_host, non_blocking=True)
+        self.step()
+        o_host.copy_(self.p_mix, non_blocking=True)
+
+    def check_err(self):
+        return int(self.err.item())
+
+
 # ----------------------------------------------------------------------------- oracle timing
 
 def _threads_used():
@@ -393,6 +479,8 @@ def time_oracle(run, workload, budget_s, max_steps=None):
                   "full weights, cache %d+1; weights pre-widened to fp64 outside the timing"
                   % (steps, n_seq, run.w.B, run.w.cache_len))
         return n_seq * steps / el, sample, el, steps
+    if workload == "mixture":
+        return time_oracle_mixture(run.host, budget_s)
     B = run.w.B
     sel, el, k = [], 0.0, 0
     inp_all = None
@@ -405,6 +493,36 @@ def time_oracle(run, workload, budget_s, max_steps=None):
         k += 1
     sample = "fp64 oracle decode attention (both flows) on %d of %d sequences" % (k, B)
     del inp_all
+    return k / el, sample, el, k
+
+
+def oracle_mixture_sequence(host, b):
+    """One sequence of the mixture head on the oracle: fp64 LM-head projection
+    of both flows' rows, logits rounded to bf16 (the GPU stores them so), then
+    the mixture."""
+    import numpy as np
+    import oracle
+    import torch
+    x = torch.stack([host["h1"][b], host["h2"][b]]).to(torch.float32).numpy().astype(np.float64)
+    w = host["w_head_f64"]
+    logits = oracle.bf16_round(oracle.grouped_proj(x, w, 1))
+    return oracle.mixture_head(logits, 1)
+
+
+def time_oracle_mixture(host, budget_s):
+    import numpy as np
+    import torch
+    if "w_head_f64" not in host:
+        host["w_head_f64"] = host["w_head"].to(torch.float32).numpy().astype(np.float64)
+    B = host["B"]
+    k, el = 0, 0.0
+    while el < budget_s and k < 4 * B:
+        t0 = time.perf_counter()
+        oracle_mixture_sequence(host, k % B)
+        el += time.perf_counter() - t0
+        k += 1
+    sample = ("fp64 oracle mixture head (LM-head projection of both flows + mixture) on %d "
+              "sequence(s) of %d; weights pre-widened to fp64 outside the timing" % (k, B))
     return k / el, sample, el, k
 
 
@@ -422,6 +540,21 @@ def run_reference(args):
         pass
 
     h = Host()
+    if args.workload == "mixture":
+        h.w = synth.WORKLOADS["mixture"]
+        h.host = synth.make_mixture_inputs(h.w)
+        v, sample, el, steps = time_oracle_mixture(h.host, 20.0)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": world, "steps": steps, "steps_requested": args.steps,
+                "warmup": args.warmup, "ms_per_step": el / steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": args.workload},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads_used(),
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     if args.workload == "layer":
         h.w = synth.WORKLOADS["layer"]
         h.host = synth.make_layer_inputs(h.w)
@@ -489,8 +622,12 @@ def main(argv=None):
     torch.cuda.set_device(dev)
     seed_base = synth_seed(args.workload)
     seed = rank_seed(seed_base, rank)
-    run = LayerRun(args, dev, seed) if args.workload == "layer" else \
-        AttnRun(args, dev, seed, args.workload)
+    if args.workload == "layer":
+        run = LayerRun(args, dev, seed)
+    elif args.workload == "mixture":
+        run = MixtureRun(args, dev, seed)
+    else:
+        run = AttnRun(args, dev, seed, args.workload)
 
     for _ in range(args.warmup):
         run.step()
@@ -500,8 +637,9 @@ def main(argv=None):
         return 3
 
     # ---------------------------------------------------------------- timed region
-    timers = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    keys = getattr(run, "timer_keys", ("attn",))
+    timers = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for k in keys} for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -520,12 +658,13 @@ def main(argv=None):
     # (the step then runs as separate graphs, so it is not used for `value`).
     torch.cuda.synchronize()
     for i in range(args.steps):
-        run.step(timers={"attn": timers[i]})
+        run.step(timers=timers[i])
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if (not args.no_clocks and rank == 0) else None
-    attn_ms = sum(s.elapsed_time(e) for s, e in timers) / args.steps
-    attn_ms = max_over_ranks(attn_ms, world)
+    kernel_ms = {k: max_over_ranks(sum(t[k][0].elapsed_time(t[k][1]) for t in timers) / args.steps,
+                                   world) for k in keys}
+    attn_ms = kernel_ms[getattr(run, "dominant_key", "attn")]
     err = run.check_err()
 
     # ---------------------------------------------------------------- end to end (host buffers)
@@ -562,7 +701,8 @@ def main(argv=None):
             dist.destroy_process_group()
         return 0
     peak, peak_kind = measured_hbm_peak()
-    achieved = run.attn_bytes / (attn_ms / 1e3) / 1e9
+    dom_bytes = getattr(run, "dom_bytes", None) or run.attn_bytes
+    achieved = dom_bytes / (attn_ms / 1e3) / 1e9
     value = world * run.tokens_per_step * args.steps / (ms_max / 1e3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -570,22 +710,29 @@ def main(argv=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations/cache, N(0,0.02) weights, N(0,0.1) couplings)",
         "config": dict(run.config, parallelism="replicas" if world > 1 else "single GPU"),
-        "kv_read_gbs": run.kv_bytes / (attn_ms / 1e3) / 1e9,
-        "kv_frac_of_hbm_peak": run.kv_bytes / (attn_ms / 1e3) / 1e9 / peak,
-        "attn_ms_per_launch": attn_ms,
-        "attn_timing": "second pass of the same %d steps, attention graph bracketed by CUDA "
-                       "events on the launching stream (value uses the single-graph step)"
-                       % args.steps,
+        "dominant_ms_per_launch": attn_ms,
+        "kernel_timing": "second pass of the same %d steps, the timed kernels' graphs bracketed "
+                         "by CUDA events on the launching stream (value uses the single-graph "
+                         "step)" % args.steps,
         "roofline": {"kernel": run.dominant, "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind + " (STREAM-style copy, MEASURED_PEAKS.json)"
                      if peak_kind == "measured" else peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic_from_profile(args.workload),
-                     "algorithmic_bytes_per_launch": run.attn_bytes,
+                     "algorithmic_bytes_per_launch": dom_bytes,
                      "units_per_launch": run.units, "bytes_per_unit": run.bytes_per_unit},
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": run.launches_per_step * args.steps,
         "clocks": clk, "device_error_flag": err,
     }
+    if hasattr(run, "kv_bytes"):
+        line["kv_read_gbs"] = run.kv_bytes / (attn_ms / 1e3) / 1e9
+        line["kv_frac_of_hbm_peak"] = run.kv_bytes / (attn_ms / 1e3) / 1e9 / peak
+    if hasattr(run, "mix_bytes"):
+        mix_gbs = run.mix_bytes / (kernel_ms["mix"] / 1e3) / 1e9
+        line["mixture_kernel"] = {"kernel": "dualflow_mixture_head", "bound": "hbm",
+                                  "ms_per_launch": kernel_ms["mix"], "achieved": mix_gbs,
+                                  "peak": peak, "unit": "GB/s", "frac": mix_gbs / peak,
+                                  "algorithmic_bytes_per_launch": run.mix_bytes}
     if clk is None and not args.no_clocks:
         line["clocks"] = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
     print(json.dumps(line), flush=True)

@@ -14,15 +14,18 @@
 // written once):
 //  * one thread-block cluster of S <= 8 CTAs per sequence splits the
 //    vocabulary into S slices so that B * S CTAs fill the GPU;
-//  * pass 1: each thread keeps online statistics over its elements -- running
-//    max m, sum z = sum 2^(x - m) and, for the primary flow, the sum of
-//    squares c = sum 2^(2 (x - m)) (x = logit * log2(e)); warps and CTAs merge
-//    them by rescaling to the larger max;
+//  * pass 1: per CTA, the maximum m of each row's slice, then z = sum 2^(x - m)
+//    and, for the primary flow, the sum of squares c = sum 2^(2 (x - m))
+//    (x = logit * log2(e)); the slice stays in registers as packed bf16
+//    between the passes (slices longer than 8192 logits stream twice, with
+//    online statistics); CTAs merge by rescaling to the larger max;
 //  * the S CTAs exchange their 5 statistics through distributed shared memory
-//    and combine them in rank order, so every CTA derives the same alpha;
-//  * pass 2 re-reads the slice (an L2 hit: it was just read) and writes
-//    p_mix = (alpha / z1) 2^(x1 - m1) + ((1 - alpha) / z2) 2^(x2 - m2) with
-//    16-byte stores.
+//    (one remote load per thread) and combine them in rank order, so every
+//    CTA derives the same alpha;
+//  * pass 2 writes p_mix = (alpha / z1) 2^(x1 - m1) + ((1 - alpha) / z2)
+//    2^(x2 - m2) with 16-byte stores, from registers when each thread holds
+//    at most 4 vectors of 8 logits per row, else re-reading the slice (an L2
+//    hit: it was just read).
 // alpha reads only the primary rows, so it is bit-identical whatever the
 // auxiliary logits are (NaN included).
 #include <math.h>
@@ -35,7 +38,7 @@ namespace mix {
 
 constexpr int kThreads = 256;
 constexpr int kMaxCluster = 8;
-constexpr int kTargetCtas = 148 * 2;
+constexpr int kTargetCtas = 148 * 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Params {
@@ -122,10 +125,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
 __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
   uint32_t addr;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(local)), "r"(rank));
@@ -134,10 +133,65 @@ __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t ran
   return v;
 }
 
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 8 consecutive logits kept in their storage type (bf16: one 16-byte vector
+// in 4 registers), decoded to the log2 domain on use.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* src) {
+    u = *reinterpret_cast<const uint4*>(src);
+  }
+  __device__ __forceinline__ float get(int i) const {
+    const uint32_t w = (i < 2) ? u.x : (i < 4) ? u.y : (i < 6) ? u.z : u.w;
+    return bf16_bits_to_float(static_cast<uint16_t>((i & 1) ? (w >> 16) : (w & 0xffffu))) * kLog2e;
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* src) {
+    a = reinterpret_cast<const float4*>(src)[0];
+    b = reinterpret_cast<const float4*>(src)[1];
+  }
+  __device__ __forceinline__ float get(int i) const {
+    const float v = (i == 0) ? a.x : (i == 1) ? a.y : (i == 2) ? a.z : (i == 3) ? a.w
+                  : (i == 4) ? b.x : (i == 5) ? b.y : (i == 6) ? b.z : b.w;
+    return v * kLog2e;
+  }
+};
+
+// Vectors of 8 logits per row held in registers by each thread when the slice
+// is short enough (every CTA of the launch resident at once); longer slices
+// take the streaming path, which reads the slice twice.
+constexpr int kRegVecs = 4;
+
+__device__ __forceinline__ float warp_max_nan(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) mixture_kernel(const Params p) {
-  __shared__ Stat warp_st[2][kThreads / 32];
-  __shared__ float cta_st[5];  // this CTA's (m1, z1, c1, m2, z2), read by the cluster
+  constexpr int kWarps = kThreads / 32;
+  __shared__ float red[5][kWarps];
+  __shared__ float cta_st[5];                 // this CTA's (m1, z1, c1, m2, z2)
+  __shared__ float all_st[kMaxCluster][5];    // every rank's, gathered in one round trip
+  __shared__ float fin[4];
   const int b = blockIdx.y;
   const uint32_t rank = cluster_rank();
   const int S = static_cast<int>(gridDim.x);
@@ -145,75 +199,180 @@ __global__ void __launch_bounds__(kThreads) mixture_kernel(const Params p) {
   const int v1 = min(p.V, v0 + p.chunk);
   const T* row1 = static_cast<const T*>(p.logits) + static_cast<int64_t>(b) * p.ld;
   const T* row2 = static_cast<const T*>(p.logits) + static_cast<int64_t>(p.B + b) * p.ld;
+  float* out = p.p_mix + static_cast<int64_t>(b) * p.ldp;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool in_regs = (v1 - v0) <= kRegVecs * kThreads * 8;
   pdl_wait();
   pdl_trigger();
 
-  // ---- pass 1: statistics of this slice
-  Stat s1 = stat_empty(), s2 = stat_empty();
-  for (int v = v0 + tid * 8; v < v1; v += kThreads * 8) {
-    float x1[8], x2[8];
-    load8<T>(row1 + v, x1);
-    load8<T>(row2 + v, x2);
-    stat_add<8>(s1, x1, true);
-    stat_add<8>(s2, x2, false);
-  }
+  float m1 = -INFINITY, m2 = -INFINITY;  // this CTA's maxima (after the first reduction)
+  float z1 = 0.f, c1 = 0.f, z2 = 0.f;
+  Raw8<T> r1[kRegVecs], r2[kRegVecs];
+  if (in_regs) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    s1 = stat_merge(s1, stat_shfl_xor(s1, o));
-    s2 = stat_merge(s2, stat_shfl_xor(s2, o));
+    for (int it = 0; it < kRegVecs; ++it) {  // every load issued before any use
+      const int v = v0 + (it * kThreads + tid) * 8;
+      if (v < v1) {
+        r1[it].load(row1 + v);
+        r2[it].load(row2 + v);
+      }
+    }
+    // local maxima
+#pragma unroll
+    for (int it = 0; it < kRegVecs; ++it) {
+      if (v0 + (it * kThreads + tid) * 8 < v1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          m1 = max_nan(m1, r1[it].get(i));
+          m2 = max_nan(m2, r2[it].get(i));
+        }
+      }
+    }
+    m1 = warp_max_nan(m1);
+    m2 = warp_max_nan(m2);
+    if (lane == 0) {
+      red[0][warp] = m1;
+      red[1][warp] = m2;
+    }
+    __syncthreads();
+    m1 = red[0][0];
+    m2 = red[1][0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      m1 = max_nan(m1, red[0][w]);
+      m2 = max_nan(m2, red[1][w]);
+    }
+    // sums against the CTA maxima (an all -inf slice contributes nothing)
+    const float u1 = (m1 == -INFINITY) ? 0.f : m1, u2 = (m2 == -INFINITY) ? 0.f : m2;
+#pragma unroll
+    for (int it = 0; it < kRegVecs; ++it) {
+      if (v0 + (it * kThreads + tid) * 8 < v1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float e1 = exp2f(r1[it].get(i) - u1);
+          z1 += e1;
+          c1 = fmaf(e1, e1, c1);
+          z2 += exp2f(r2[it].get(i) - u2);
+        }
+      }
+    }
+  } else {
+    // streaming: online statistics with rescaling, two vectors per step
+    Stat s1 = stat_empty(), s2 = stat_empty();
+    for (int v = v0 + tid * 8; v < v1; v += 2 * kThreads * 8) {
+      float x1[8], x2[8], y1[8], y2[8];
+      const int w = v + kThreads * 8;
+      load8<T>(row1 + v, x1);
+      load8<T>(row2 + v, x2);
+      if (w < v1) {
+        load8<T>(row1 + w, y1);
+        load8<T>(row2 + w, y2);
+      }
+      stat_add<8>(s1, x1, true);
+      stat_add<8>(s2, x2, false);
+      if (w < v1) {
+        stat_add<8>(s1, y1, true);
+        stat_add<8>(s2, y2, false);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 = stat_merge(s1, stat_shfl_xor(s1, o));
+      s2 = stat_merge(s2, stat_shfl_xor(s2, o));
+    }
+    if (lane == 0) {
+      red[0][warp] = s1.m;
+      red[1][warp] = s2.m;
+    }
+    __syncthreads();
+    m1 = red[0][0];
+    m2 = red[1][0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      m1 = max_nan(m1, red[0][w]);
+      m2 = max_nan(m2, red[1][w]);
+    }
+    // this warp's sums rescaled to the CTA maxima
+    const float f1 = (s1.m == -INFINITY) ? 0.f : exp2f(s1.m - m1);
+    const float f2 = (s2.m == -INFINITY) ? 0.f : exp2f(s2.m - m2);
+    if (lane == 0) {
+      z1 = s1.z * f1;
+      c1 = s1.c * f1 * f1;
+      z2 = s2.z * f2;
+    }
   }
+  z1 = warp_sum(z1);
+  c1 = warp_sum(c1);
+  z2 = warp_sum(z2);
+  __syncthreads();  // the maxima in red[] have been read
   if (lane == 0) {
-    warp_st[0][warp] = s1;
-    warp_st[1][warp] = s2;
+    red[2][warp] = z1;
+    red[3][warp] = c1;
+    red[4][warp] = z2;
   }
   __syncthreads();
   if (tid == 0) {
-    Stat a = warp_st[0][0], c = warp_st[1][0];
-    for (int w = 1; w < kThreads / 32; ++w) {
-      a = stat_merge(a, warp_st[0][w]);
-      c = stat_merge(c, warp_st[1][w]);
+    float a = 0.f, c = 0.f, d = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      a += red[2][w];
+      c += red[3][w];
+      d += red[4][w];
     }
-    cta_st[0] = a.m;
-    cta_st[1] = a.z;
-    cta_st[2] = a.c;
-    cta_st[3] = c.m;
-    cta_st[4] = c.z;
+    cta_st[0] = m1;
+    cta_st[1] = a;
+    cta_st[2] = c;
+    cta_st[3] = m2;
+    cta_st[4] = d;
   }
-  // ---- combine the cluster's statistics in rank order (same result everywhere)
-  cluster_sync();
-  __shared__ float fin[5];
+  // ---- gather the cluster's statistics (one remote load per thread), combine
+  // them in rank order (the same result in every CTA)
+  cluster_arrive();
+  cluster_wait();
+  if (tid < 5 * S) all_st[tid / 5][tid % 5] = ld_cluster_f32(&cta_st[tid % 5], tid / 5);
+  cluster_arrive();  // this CTA is done reading remote statistics
+  __syncthreads();
   if (tid == 0) {
     Stat a = stat_empty(), c = stat_empty();
     for (int q = 0; q < S; ++q) {
-      const Stat qa{ld_cluster_f32(&cta_st[0], q), ld_cluster_f32(&cta_st[1], q),
-                    ld_cluster_f32(&cta_st[2], q)};
-      const Stat qc{ld_cluster_f32(&cta_st[3], q), ld_cluster_f32(&cta_st[4], q), 0.f};
-      a = stat_merge(a, qa);
-      c = stat_merge(c, qc);
+      a = stat_merge(a, Stat{all_st[q][0], all_st[q][1], all_st[q][2]});
+      c = stat_merge(c, Stat{all_st[q][3], all_st[q][4], 0.f});
     }
     const float alpha = 0.5f + 0.5f * (a.c / (a.z * a.z));
     fin[0] = a.m;
     fin[1] = alpha / a.z;
     fin[2] = c.m;
     fin[3] = (1.0f - alpha) / c.z;
-    fin[4] = alpha;
     if (rank == 0 && p.alpha != nullptr) p.alpha[b] = alpha;
   }
-  cluster_sync();  // no CTA leaves while others may still read its statistics
-  const float m1 = fin[0], k1 = fin[1], m2 = fin[2], k2 = fin[3];
+  __syncthreads();
+  const float M1 = fin[0], k1 = fin[1], M2 = fin[2], k2 = fin[3];
 
   // ---- pass 2: p_mix of this slice
-  float* out = p.p_mix + static_cast<int64_t>(b) * p.ldp;
-  for (int v = v0 + tid * 8; v < v1; v += kThreads * 8) {
-    float x1[8], x2[8], o[8];
-    load8<T>(row1 + v, x1);
-    load8<T>(row2 + v, x2);
+  if (in_regs) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = k1 * exp2f(x1[i] - m1) + k2 * exp2f(x2[i] - m2);
-    reinterpret_cast<float4*>(out + v)[0] = make_float4(o[0], o[1], o[2], o[3]);
-    reinterpret_cast<float4*>(out + v)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    for (int it = 0; it < kRegVecs; ++it) {
+      const int v = v0 + (it * kThreads + tid) * 8;
+      if (v < v1) {
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          o[i] = k1 * exp2f(r1[it].get(i) - M1) + k2 * exp2f(r2[it].get(i) - M2);
+        reinterpret_cast<float4*>(out + v)[0] = make_float4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<float4*>(out + v)[1] = make_float4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  } else {
+    for (int v = v0 + tid * 8; v < v1; v += kThreads * 8) {
+      float x1[8], x2[8], o[8];
+      load8<T>(row1 + v, x1);
+      load8<T>(row2 + v, x2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = k1 * exp2f(x1[i] - M1) + k2 * exp2f(x2[i] - M2);
+      reinterpret_cast<float4*>(out + v)[0] = make_float4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<float4*>(out + v)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
   }
+  cluster_wait();  // no CTA leaves while another may still read its statistics
 }
 
 // Slices per sequence: enough CTAs to fill two per SM, at most 8 (a portable

@@ -68,12 +68,24 @@ class LayerWorkload:
     coupled_mlp: bool = True   # b, c ~ N(0, 0.1); False -> b = c = 0
 
 
+@dataclasses.dataclass(frozen=True)
+class MixtureWorkload:
+    """Mixture head: grouped LM-head projection of both flows' final hidden
+    states (one shared output matrix) and the mixed next-token distribution."""
+    name: str
+    B: int          # sequences per flow (2B rows in the projection)
+    d_model: int
+    V: int          # vocabulary (multiple of 128)
+    seed: int = 6
+
+
 WORKLOADS = {
     "tiny": AttnWorkload("tiny", 1, 2, 2, 64, "fp32", 128, 128, append=True, seed=1),
     "mha": AttnWorkload("mha", 32, 32, 32, 128, "bf16", 2048, 2048, seed=2),
     "gqa": AttnWorkload("gqa", 64, 32, 8, 128, "bf16", 1024, 8192, random_table=True, seed=3),
     "long": AttnWorkload("long", 8, 32, 8, 128, "bf16", 32768, 131072, seed=4),
     "layer": LayerWorkload("layer", 64, 4096, 32, 8, 128, 14336, 4096, seed=5),
+    "mixture": MixtureWorkload("mixture", 64, 4096, 32000, seed=6),
 }
 
 
@@ -213,3 +225,15 @@ def make_layer_inputs(w: LayerWorkload, seed: Optional[int] = None, B: Optional[
 def to_numpy_f32(t: torch.Tensor):
     """Exact widening of a host bf16/fp32 tensor to a float32 numpy array."""
     return t.detach().to("cpu").to(torch.float32).numpy()
+
+
+def make_mixture_inputs(w: MixtureWorkload, seed: Optional[int] = None):
+    """Host tensors for one mixture-head step of workload ``w`` (bf16):
+    h1, h2 [B, d_model] ~ N(0, 1) (final hidden states of the two flows) and
+    the shared output matrix w_head [V, d_model] ~ N(0, 0.02), so logits have
+    a standard deviation of about 0.02 sqrt(d_model) (1.3 at d_model 4096)."""
+    g = _gen(w.seed if seed is None else seed)
+    h1 = _randn(g, (w.B, w.d_model))
+    h2 = _randn(g, (w.B, w.d_model))
+    w_head = _randn(g, (w.V, w.d_model), std=0.02, chunk_rows=2048)
+    return dict(h1=h1, h2=h2, w_head=w_head, B=w.B, d_model=w.d_model, V=w.V)

@@ -170,4 +170,4 @@ def test_mixture_head_rejects_invalid_arguments(lib):
     assert call(ldp=4098) == L.DF_ERR_ALIGN
     assert call(ld=4100) == L.DF_ERR_ALIGN
     sl = lib.dualflow_mixture_head_slices
-    assert sl(64, 32000) == 5 and sl(1, 32000) == 8 and sl(4, 1024) == 1 and sl(0, 8) == 0
+    assert sl(64, 32000) == 8 and sl(1, 32000) == 8 and sl(4, 1024) == 1 and sl(0, 8) == 0

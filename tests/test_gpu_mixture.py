@@ -41,7 +41,7 @@ CASES = [  # (B, V, dtype)
     (3, 1000, torch.float32),
     (1, 8, torch.float32),
     (1, 32000, torch.bfloat16),      # one sequence: a cluster of 8 slices
-    (64, 32000, torch.bfloat16),     # full size: 5 slices per sequence
+    (64, 32000, torch.bfloat16),     # full size: 8 slices per sequence
     (64, 32008, torch.bfloat16),     # ragged last slice
     (5, 50304, torch.float32),
 ]
