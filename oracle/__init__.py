@@ -23,4 +23,7 @@ from .dualflow_oracle import (  # noqa: F401
     collision_probability,
     mixture_weight,
     mixture_head,
+    moe_route,
+    moe_expert,
+    moe_forward,
 )

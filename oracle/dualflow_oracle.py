@@ -27,6 +27,12 @@ of the function that takes it:
 * Layer step      pre-attention and pre-MLP RMSNorm (unit gain, eps 1e-5),
   residual adds, SwiGLU MLP, no positional rotation.
   PARITY UNPINNED against the pages (the pages name no norm, no MLP form).
+* MoE router replay  the auxiliary flow uses the primary router's expert
+  set with its own gate weights (the pages' statement); the router matrix is
+  shared, gates are the softmax of each flow's router logits over the set,
+  experts are SwiGLU MLPs, and with a larger auxiliary fan-out the auxiliary
+  set is the primary ranking's top k_aux. Those details are readings:
+  PARITY UNPINNED against the pages beyond the invariants in the tests.
 * Mixture head    p_mix = alpha p1 + (1 - alpha) p2 is the pages' formula;
   the map from the primary's collision probability to alpha is a reading,
   alpha = 1/2 + 1/2 sum(p1^2). Pinned by its limits (uniform and one-hot
@@ -361,3 +367,83 @@ def mixture_head(logits, B):
     p2 = softmax_rows(l[B:2 * B])
     alpha = mixture_weight(p1)
     return alpha[:, None] * p1 + (1.0 - alpha[:, None]) * p2, alpha
+
+
+# ----------------------------------------------------------------- MoE router replay
+
+def moe_route(x1, x2, w_router, k, k_aux=None):
+    """Expert selection and gate weights of both flows (router replay).
+
+    "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi Chiave"
+    (router replay for MoE): the auxiliary flow reuses the set of experts that
+    the primary router selected, applied with its own mixing weights; section
+    "Contributi Chiave" (phase-specific MoE allocation): the two flows may
+    have independent expert fan-outs. Readings taken:
+      * router logits r_f = x_f W_router^T (one router matrix shared by both
+        flows, like every other matrix of the model);
+      * ids = the primary's top-k_aux experts by descending r_1 (ties: lower
+        expert index first); the primary uses the first k of them, the
+        auxiliary all k_aux (k_aux = k is router replay proper);
+      * gates: softmax of each flow's own logits over its set,
+        g1 = softmax(r_1[ids[:k]]), g2 = softmax(r_2[ids[:k_aux]]).
+    x1, x2: [B][d]; w_router: [E][d]. Returns (ids int [B][k_aux],
+    g1 [B][k], g2 [B][k_aux], r1 [B][E], r2 [B][E]), fp64.
+    """
+    k_aux = k if k_aux is None else k_aux
+    w = np.asarray(w_router, dtype=F64)
+    r1 = np.asarray(x1, dtype=F64) @ w.T
+    r2 = np.asarray(x2, dtype=F64) @ w.T
+    B, E = r1.shape
+    ids = np.zeros((B, k_aux), dtype=np.int64)
+    for t in range(B):
+        # stable sort of (-logit, index): descending logit, lower index first on ties
+        order = sorted(range(E), key=lambda e: (-r1[t, e], e))
+        ids[t] = order[:k_aux]
+    g1 = softmax_rows(np.take_along_axis(r1, ids[:, :k], axis=1))
+    g2 = softmax_rows(np.take_along_axis(r2, ids, axis=1))
+    return ids, g1, g2, r1, r2
+
+
+def moe_expert(x, w_gu, w_down, round_bf16=True):
+    """One SwiGLU expert applied to rows x: W_down (SiLU(x W_gate^T) * (x W_up^T)),
+    w_gu = [W_gate; W_up] ([2F][d]), w_down [d][F]. With round_bf16 the
+    intermediate and the result are rounded to bf16, where the CUDA path
+    stores bf16 tensors."""
+    x = np.asarray(x, dtype=F64)
+    gu = x @ np.asarray(w_gu, dtype=F64).T
+    F = gu.shape[1] // 2
+    h = silu(gu[:, :F]) * gu[:, F:]
+    if round_bf16:
+        h = bf16_round(h)  # the intermediate is stored bf16
+    y = h @ np.asarray(w_down, dtype=F64).T
+    return bf16_round(y) if round_bf16 else y
+
+
+def moe_forward(x1, x2, w_router, w_gu, w_down, k, k_aux=None, residual1=None,
+                residual2=None, round_bf16=True):
+    """MoE MLP block of both flows with router replay:
+        y1[t] = sum_j g1[t][j] E_{ids[t][j]}(x1[t])       (j < k)
+        y2[t] = sum_j g2[t][j] E_{ids[t][j]}(x2[t])       (j < k_aux)
+    plus the residual when given, rounded once to bf16 (round_bf16).
+    w_gu: [E][2F][d], w_down: [E][d][F]. Returns (y1, y2, ids, g1, g2)."""
+    k_aux = k if k_aux is None else k_aux
+    ids, g1, g2, _, _ = moe_route(x1, x2, w_router, k, k_aux)
+    x1 = np.asarray(x1, dtype=F64)
+    x2 = np.asarray(x2, dtype=F64)
+    B, d = x1.shape
+    y1 = np.zeros((B, d))
+    y2 = np.zeros((B, d))
+    for e in np.unique(ids):
+        t1, j1 = np.nonzero(ids[:, :k] == e)
+        if t1.size:
+            y1[t1] += g1[t1, j1][:, None] * moe_expert(x1[t1], w_gu[e], w_down[e], round_bf16)
+        t2, j2 = np.nonzero(ids == e)
+        if t2.size:
+            y2[t2] += g2[t2, j2][:, None] * moe_expert(x2[t2], w_gu[e], w_down[e], round_bf16)
+    if residual1 is not None:
+        y1 = y1 + np.asarray(residual1, dtype=F64)
+    if residual2 is not None:
+        y2 = y2 + np.asarray(residual2, dtype=F64)
+    if round_bf16:
+        y1, y2 = bf16_round(y1), bf16_round(y2)
+    return y1, y2, ids, g1, g2

@@ -491,3 +491,81 @@ def test_mixture_invariants_and_primary_only_weight():
     # a flow swap is visible: exchanging the rows changes the mixture
     p_swap, _ = oracle.mixture_head(np.concatenate([l[B:], l[:B]]), B)
     assert not np.allclose(p_swap, p_mix)
+
+
+# ---------------------------------------------------------------- MoE router replay
+
+def _moe_fixture_experts(u):
+    E = len(u)
+    w_gu = np.zeros((E, 2, 2))
+    w_gu[:, 0, 0] = 40.0          # gate row (40, 0)
+    w_gu[:, 1, 0] = u             # up row (u_e, 0)
+    w_down = np.zeros((E, 2, 1))
+    w_down[:, 0, 0] = 1.0         # down column (1, 0)
+    return w_gu, w_down
+
+
+def test_golden_moe_router_replay():
+    with open(os.path.join(GOLDEN, "moe_router_replay_worked_example.json")) as f:
+        fx = json.load(f)
+    w_r = _arr(fx["w_router"])
+    u = _arr(fx["u"])
+    w_gu, w_down = _moe_fixture_experts(u)
+    S = 40.0 / (1.0 + math.exp(-40.0))
+    for c in fx["cases"]:
+        y1, y2, ids, g1, g2 = oracle.moe_forward(_arr(fx["x1"]), _arr(fx["x2"]), w_r, w_gu, w_down,
+                                                 c["k"], c["k_aux"], round_bf16=False)
+        np.testing.assert_array_equal(ids, np.array(c["ids"]), err_msg=c["name"])
+        np.testing.assert_allclose(g1, _arr(c["g1"]), rtol=0, atol=1e-15, err_msg=c["name"])
+        np.testing.assert_allclose(g2, _arr(c["g2"]), rtol=0, atol=1e-15, err_msg=c["name"])
+        np.testing.assert_allclose(y1, S * _arr(c["y1_over_S"]), rtol=1e-14, atol=0, err_msg=c["name"])
+        np.testing.assert_allclose(y2, S * _arr(c["y2_over_S"]), rtol=1e-14, atol=0, err_msg=c["name"])
+
+
+def _moe_case(seed, B=6, d=32, E=5, F=16):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(B, d)), rng.normal(size=(B, d)), rng.normal(size=(E, d)),
+            rng.normal(size=(E, 2 * F, d)) * 0.2, rng.normal(size=(E, d, F)) * 0.2)
+
+
+def test_moe_identical_flows_and_primary_blind_to_aux():
+    x1, x2, wr, wgu, wd = _moe_case(90)
+    y1, y2, ids, g1, g2 = oracle.moe_forward(x1, x1, wr, wgu, wd, 2)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(g1, g2)
+    ya, _, ida, ga, _ = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 4)
+    bad = np.full_like(x2, np.nan)
+    yb, y2b, idb, gb, g2b = oracle.moe_forward(x1, bad, wr, wgu, wd, 2, 4)
+    np.testing.assert_array_equal(ida, idb)
+    np.testing.assert_array_equal(ga, gb)
+    np.testing.assert_array_equal(ya, yb)
+    assert np.isnan(y2b).all() and np.isnan(g2b).all()
+    np.testing.assert_allclose(g1.sum(axis=1), 1.0, atol=1e-15)
+
+
+def test_moe_relabelled_experts_give_the_same_outputs():
+    x1, x2, wr, wgu, wd = _moe_case(91)
+    perm = np.array([3, 0, 4, 1, 2])
+    y1, y2, ids, _, _ = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 3)
+    z1, z2, jds, _, _ = oracle.moe_forward(x1, x2, wr[perm], wgu[perm], wd[perm], 2, 3)
+    np.testing.assert_allclose(z1, y1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z2, y2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(perm[jds], ids)   # same experts under the new labels
+
+
+def test_moe_limits_reduce_to_the_dense_mlp():
+    x1, x2, wr, wgu, wd = _moe_case(92, E=4)
+    # a zero router: every logit ties, gates are uniform over k = E experts;
+    # with identical experts the block is that expert
+    same_gu = np.repeat(wgu[:1], 4, axis=0)
+    same_d = np.repeat(wd[:1], 4, axis=0)
+    y1, _, ids, g1, _ = oracle.moe_forward(x1, x2, np.zeros_like(wr), same_gu, same_d, 4,
+                                           round_bf16=False)
+    np.testing.assert_array_equal(ids, np.tile(np.arange(4), (x1.shape[0], 1)))
+    np.testing.assert_allclose(g1, 0.25, atol=1e-15)
+    # one expert, k = 1: the dense SwiGLU MLP (matmul, SiLU(gate) * up, matmul)
+    y1, y2, _, _, _ = oracle.moe_forward(x1, x2, wr[:1], wgu[:1], wd[:1], 1, round_bf16=False)
+    gu = oracle.grouped_proj(np.concatenate([x1, x2]), wgu[0], x1.shape[0])
+    h = oracle.swiglu_couple(gu, wgu.shape[1] // 2, x1.shape[0])
+    dense = oracle.grouped_proj(h, wd[0], x1.shape[0])
+    np.testing.assert_allclose(np.concatenate([y1, y2]), dense, rtol=1e-12, atol=1e-12)
