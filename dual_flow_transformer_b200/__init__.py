@@ -15,6 +15,9 @@ from .api import (  # noqa: F401
     kv_append,
     mixture_head,
     mixture_head_slices,
+    moe_combine,
+    moe_dispatch,
+    moe_route,
     new_attn_workspace,
     new_proj_workspace,
     rmsnorm,

@@ -65,6 +65,12 @@ SIGNATURES = {
     "dualflow_mixture_head": (_c_int, [_vp, _c_i64, _c_int, _c_int, _c_int, _vp, _c_i64, _vp,
                                        _vp]),
     "dualflow_mixture_head_slices": (_c_int, [_c_int, _c_int]),
+    "dualflow_moe_route": (_c_int, [_vp, _c_i64, _c_int, _c_int, _vp, _c_int, _c_int, _c_int,
+                                    _vp, _vp, _vp, _vp, _vp]),
+    "dualflow_moe_dispatch": (_c_int, [_vp, _c_i64, _c_int, _c_int, _vp, _c_int, _c_int, _c_int,
+                                       _vp, _vp, _vp, _vp, _vp, _vp]),
+    "dualflow_moe_combine": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                      _c_int, _c_int, _vp, _c_i64, _vp, _c_i64, _vp, _vp]),
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
 }
 

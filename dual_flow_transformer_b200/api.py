@@ -192,6 +192,62 @@ def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupli
     return y
 
 
+# ----------------------------------------------------------------- MoE router replay
+
+MOE_ROWS = 64  # rows per flow in an expert block: at most 64 tokens per call
+
+
+def moe_route(x, B, w_router, k, k_aux=None, *, ids=None, g1=None, g2=None, logits=None,
+              stream=None):
+    """Router of both flows (router replay). x: bf16 [2B, d] (primary rows,
+    then auxiliary rows); w_router: bf16 [E, d]. Returns (ids int32 [B, k_aux],
+    g1 fp32 [B, k], g2 fp32 [B, k_aux]); logits (fp32 [2B, E]) is filled when
+    given."""
+    k_aux = k if k_aux is None else k_aux
+    E, d = w_router.shape
+    dev = x.device
+    ids = torch.empty((B, k_aux), dtype=torch.int32, device=dev) if ids is None else ids
+    g1 = torch.empty((B, k), dtype=torch.float32, device=dev) if g1 is None else g1
+    g2 = torch.empty((B, k_aux), dtype=torch.float32, device=dev) if g2 is None else g2
+    st = _lib().dualflow_moe_route(_ptr(x), x.stride(0), int(B), int(d), _ptr(w_router), int(E),
+                                   int(k), int(k_aux), _ptr(ids), _ptr(g1), _ptr(g2),
+                                   _ptr(logits), _stream(stream))
+    L.check("dualflow_moe_route", st)
+    return ids, g1, g2
+
+
+def moe_dispatch(x, B, ids, E, k, k_aux=None, *, xe=None, slot1=None, slot2=None, counts=None,
+                 err_flag=None, stream=None):
+    """Pack each expert's rows: xe bf16 [E, 128, d] (primary rows from 0,
+    auxiliary rows from 64), slot1 int32 [B, k], slot2 int32 [B, k_aux]."""
+    k_aux = k if k_aux is None else k_aux
+    d = x.shape[1]
+    dev = x.device
+    xe = torch.zeros((E, 2 * MOE_ROWS, d), dtype=torch.bfloat16, device=dev) if xe is None else xe
+    slot1 = torch.empty((B, k), dtype=torch.int32, device=dev) if slot1 is None else slot1
+    slot2 = torch.empty((B, k_aux), dtype=torch.int32, device=dev) if slot2 is None else slot2
+    st = _lib().dualflow_moe_dispatch(_ptr(x), x.stride(0), int(B), int(d), _ptr(ids), int(E),
+                                      int(k), int(k_aux), _ptr(xe), _ptr(slot1), _ptr(slot2),
+                                      _ptr(counts), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_moe_dispatch", st)
+    return xe, slot1, slot2
+
+
+def moe_combine(ye, ids, g1, g2, slot1, slot2, B, k, k_aux=None, *, residual=None, y=None,
+                err_flag=None, stream=None):
+    """y bf16 [2B, d] = gate-weighted sum of the experts' output rows (+ residual)."""
+    k_aux = k if k_aux is None else k_aux
+    E, _, d = ye.shape
+    if y is None:
+        y = torch.empty((2 * B, d), dtype=torch.bfloat16, device=ye.device)
+    st = _lib().dualflow_moe_combine(_ptr(ye), _ptr(ids), _ptr(g1), _ptr(g2), _ptr(slot1),
+                                     _ptr(slot2), int(B), int(d), int(E), int(k), int(k_aux),
+                                     _ptr(residual), 0 if residual is None else residual.stride(0),
+                                     _ptr(y), y.stride(0), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_moe_combine", st)
+    return y
+
+
 # ----------------------------------------------------------------- mixture head
 
 def mixture_head(logits, B, *, p_mix=None, alpha=None, stream=None):

@@ -250,6 +250,53 @@ df_status dualflow_grouped_proj_chain(const void* x, int64_t ldx, int m_primary,
                                       void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* MoE MLP block with router replay.                                         */
+/*                                                                           */
+/* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi        */
+/* Chiave" (router replay: the auxiliary flow applies the experts selected   */
+/* by the primary router with its own mixing weights) and section            */
+/* "Contributi Chiave" (independent expert fan-outs). Readings: one router    */
+/* matrix shared by both flows; ids = the primary's top-k_aux experts by      */
+/* descending router logit (ties: lower expert index); the primary uses the  */
+/* first k, the auxiliary all k_aux (k_aux = k: router replay proper); gates */
+/* = softmax of each flow's own router logits over its set; SwiGLU experts.  */
+/* A block is: route -> dispatch -> per expert e, dualflow_grouped_proj of    */
+/* xe[e] ([128][d], m_primary = 64) with W_gate/up[e] (SWIGLU) and then        */
+/* W_down[e] (NONE) into ye[e] -> combine. Each expert's weights stream once  */
+/* for both flows; the projections' shapes do not depend on the routing.     */
+/* Limits: 1 <= B <= 64 tokens per flow per call, E <= 256,                  */
+/* 1 <= k <= k_aux <= min(E, 8), d % 8 == 0, 16-byte aligned rows.             */
+/*                                                                           */
+/* route:    x bf16 [2B][d] (primary rows, then auxiliary rows; stride ldx,  */
+/*           0 = d), w_router bf16 [E][d]. Writes ids int32 [B][k_aux],      */
+/*           g1 fp32 [B][k], g2 fp32 [B][k_aux] and, if non-NULL, the router  */
+/*           logits fp32 [2B][E] (fp32 dot products of the bf16 rows).        */
+/* dispatch: copies, for every expert e, the primary rows of the tokens that  */
+/*           chose it (first k choices), in token order, into rows 0.. of    */
+/*           xe[e] = xe + e*128*d, and the auxiliary rows (all k_aux choices) */
+/*           into rows 64.. ; writes the row of every (token, choice):        */
+/*           slot1 [B][k] (0..63), slot2 [B][k_aux] (64..127), and counts     */
+/*           [E][2] if non-NULL. ids must be distinct per token; an id        */
+/*           outside [0, E) sets DF_DEVERR_BLOCK in err_flag and is skipped.  */
+/*           Rows of xe past the counts are left as they were (each output    */
+/*           row of a projection depends only on its own input row).          */
+/* combine:  y[f*B + t] = sum_j g_f[t][j] * ye[ids[t][j]][slot_f[t][j]]       */
+/*           (+ residual[f*B + t]) in fp32, stored bf16; ye bf16 [E][128][d]. */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_moe_route(const void* x, int64_t ldx, int B, int d, const void* w_router,
+                             int E, int k, int k_aux, int32_t* ids, float* g1, float* g2,
+                             float* logits, void* stream);
+df_status dualflow_moe_dispatch(const void* x, int64_t ldx, int B, int d, const int32_t* ids,
+                                int E, int k, int k_aux, void* xe, int32_t* slot1,
+                                int32_t* slot2, int32_t* counts, int32_t* err_flag,
+                                void* stream);
+df_status dualflow_moe_combine(const void* ye, const int32_t* ids, const float* g1,
+                               const float* g2, const int32_t* slot1, const int32_t* slot2,
+                               int B, int d, int E, int k, int k_aux, const void* residual,
+                               int64_t ldr, void* y, int64_t ldy, int32_t* err_flag,
+                               void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Mixture head: the mixed next-token distribution of both flows.            */
 /*                                                                           */
 /* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi        */

@@ -171,3 +171,28 @@ def test_mixture_head_rejects_invalid_arguments(lib):
     assert call(ld=4100) == L.DF_ERR_ALIGN
     sl = lib.dualflow_mixture_head_slices
     assert sl(64, 32000) == 8 and sl(1, 32000) == 8 and sl(4, 1024) == 1 and sl(0, 8) == 0
+
+
+def test_moe_entry_points_reject_invalid_arguments(lib):
+    r = lib.dualflow_moe_route
+    assert r(None, 0, 4, 256, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_NULL
+    assert r(FAKE, 0, 65, 256, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_UNSUPPORTED
+    assert r(FAKE, 0, 4, 256, FAKE, 8, 3, 2, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_SHAPE
+    assert r(FAKE, 0, 4, 256, FAKE, 8, 2, 9, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_UNSUPPORTED
+    assert r(FAKE, 0, 4, 252, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_UNSUPPORTED
+    assert r(FAKE + 8, 0, 4, 256, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None) == L.DF_ERR_ALIGN
+    dsp = lib.dualflow_moe_dispatch
+    assert dsp(FAKE, 0, 4, 256, FAKE, 8, 2, 2, None, FAKE, FAKE, None, None, None) == L.DF_ERR_NULL
+    assert dsp(FAKE, 0, 0, 256, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None, None) == L.DF_ERR_SHAPE
+    assert dsp(FAKE, 100, 4, 256, FAKE, 8, 2, 2, FAKE, FAKE, FAKE, None, None, None) == L.DF_ERR_SHAPE
+    c = lib.dualflow_moe_combine
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 8, 2, 2, None, 0, FAKE, 0, None, None]
+    bad = list(args)
+    bad[13] = None
+    assert c(*bad) == L.DF_ERR_NULL
+    bad = list(args)
+    bad[14] = 100
+    assert c(*bad) == L.DF_ERR_SHAPE
+    bad = list(args)
+    bad[13] = FAKE + 8
+    assert c(*bad) == L.DF_ERR_ALIGN

@@ -1,0 +1,138 @@
+"""GPU parity of the MoE MLP block with router replay against the fp64 oracle,
+through the C ABI (route, dispatch, grouped tcgen05 expert projections,
+combine). Inputs come from seeded generators; expected values from the
+oracle only.
+
+Expert selection is an integer decision taken from router logits: both sides
+compute the logits (the GPU in fp32, the oracle in fp64) and the ids are
+compared exactly wherever the oracle's margin between consecutive ranks
+exceeds fp32 rounding; tokens with a closer call are checked for validity
+instead (every GPU choice within that margin of the oracle's ranking).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dual_flow_transformer_b200 import api
+from dual_flow_transformer_b200.moe import DualFlowMoE
+from tests.helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+MARGIN = 1e-3  # logit gap below which the ranking is treated as a near tie
+
+
+def _bf(g, shape, std=1.0):
+    return (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+
+
+def _f64(t):
+    return t.to(torch.float32).numpy().astype(np.float64)
+
+
+def _case(seed, B, d, F, E):
+    g = torch.Generator().manual_seed(seed)
+    x = _bf(g, (2 * B, d))
+    w_r = _bf(g, (E, d), 0.05)
+    w_gu = _bf(g, (E, 2 * F, d), 0.02)
+    w_down = _bf(g, (E, d, F), 0.02)
+    return x, w_r, w_gu, w_down
+
+
+def _decided(r1, k_aux):
+    """Tokens whose oracle ranking of the first k_aux + 1 places has no gap
+    below MARGIN (their ids are unique up to fp32 rounding)."""
+    srt = -np.sort(-r1, axis=1)
+    n = min(k_aux + 1, r1.shape[1])
+    gaps = srt[:, :n - 1] - srt[:, 1:n]
+    return (gaps > MARGIN).all(axis=1)
+
+
+@pytest.mark.parametrize("B,d,E,k,k_aux", [(8, 256, 4, 2, 2), (64, 2048, 8, 2, 2),
+                                           (33, 512, 16, 1, 3), (5, 64, 8, 8, 8)])
+def test_route_parity(cuda_device, B, d, E, k, k_aux):
+    x, w_r, _, _ = _case(100 + B, B, d, 16, E)
+    logits = torch.empty((2 * B, E), dtype=torch.float32, device=cuda_device)
+    ids, g1, g2 = api.moe_route(x.to(cuda_device), B, w_r.to(cuda_device), k, k_aux, logits=logits)
+    torch.cuda.synchronize()
+    r_ids, r_g1, r_g2, r1, r2 = oracle.moe_route(_f64(x[:B]), _f64(x[B:]), _f64(w_r), k, k_aux)
+    np.testing.assert_allclose(logits.cpu().numpy()[:B], r1, rtol=0, atol=1e-4)
+    np.testing.assert_allclose(logits.cpu().numpy()[B:], r2, rtol=0, atol=1e-4)
+    ok = _decided(r1, k_aux)
+    assert ok.sum() >= B - 2, "too many near ties for this seed"
+    got = ids.cpu().numpy()
+    np.testing.assert_array_equal(got[ok], r_ids[ok])
+    np.testing.assert_allclose(g1.cpu().numpy()[ok], r_g1[ok], rtol=0, atol=1e-5)
+    np.testing.assert_allclose(g2.cpu().numpy()[ok], r_g2[ok], rtol=0, atol=1e-5)
+    # undecided tokens: the GPU's choices are still a valid top-k_aux within the margin
+    for t in np.nonzero(~ok)[0]:
+        kth = -np.sort(-r1[t])[k_aux - 1]
+        assert (r1[t, got[t]] >= kth - MARGIN).all()
+        assert len(set(got[t].tolist())) == k_aux
+
+
+def test_dispatch_packs_rows_bit_exact(cuda_device):
+    B, d, E, k, k_aux = 48, 512, 8, 2, 3
+    x, w_r, _, _ = _case(110, B, d, 16, E)
+    xd = x.to(cuda_device)
+    ids, _, _ = api.moe_route(xd, B, w_r.to(cuda_device), k, k_aux)
+    counts = torch.zeros((E, 2), dtype=torch.int32, device=cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    xe, s1, s2 = api.moe_dispatch(xd, B, ids, E, k, k_aux, counts=counts, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ids, xe, s1, s2 = ids.cpu().numpy(), xe.cpu(), s1.cpu().numpy(), s2.cpu().numpy()
+    for t in range(B):
+        for j in range(k_aux):
+            e = ids[t, j]
+            if j < k:
+                assert 0 <= s1[t, j] < 64
+                assert torch.equal(xe[e, s1[t, j]].view(torch.int16), x[t].view(torch.int16))
+            assert 64 <= s2[t, j] < 128
+            assert torch.equal(xe[e, s2[t, j]].view(torch.int16), x[B + t].view(torch.int16))
+    exp1 = np.bincount(ids[:, :k].ravel(), minlength=E)
+    exp2 = np.bincount(ids.ravel(), minlength=E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), np.stack([exp1, exp2], axis=1))
+
+
+def _block(dev, x, w_r, w_gu, w_down, k, k_aux, B, residual=None):
+    moe = DualFlowMoE(w_r.to(dev), w_gu.to(dev), w_down.to(dev), k, k_aux, B=B, device=dev)
+    y = moe.forward(x.to(dev), residual=None if residual is None else residual.to(dev))
+    torch.cuda.synchronize()
+    assert int(moe.err.item()) == 0
+    return y.cpu(), moe
+
+
+@pytest.mark.parametrize("B,d,F,E,k,k_aux", [(8, 256, 512, 4, 2, 2), (16, 512, 768, 8, 1, 3),
+                                             (64, 2048, 5632, 8, 2, 2)])
+def test_moe_block_parity(cuda_device, B, d, F, E, k, k_aux):
+    x, w_r, w_gu, w_down = _case(120 + B, B, d, F, E)
+    g = torch.Generator().manual_seed(121)
+    res = _bf(g, (2 * B, d))
+    y, _ = _block(cuda_device, x, w_r, w_gu, w_down, k, k_aux, B, residual=res)
+    r1, r2, r_ids, _, _ = oracle.moe_forward(_f64(x[:B]), _f64(x[B:]), _f64(w_r), _f64(w_gu),
+                                             _f64(w_down), k, k_aux, _f64(res[:B]), _f64(res[B:]))
+    _, _, _, rl1, _ = oracle.moe_route(_f64(x[:B]), _f64(x[B:]), _f64(w_r), k, k_aux)
+    ok = _decided(rl1, k_aux)
+    assert ok.sum() >= B - 2
+    ok2 = np.concatenate([ok, ok])
+    ref = np.concatenate([r1, r2])
+    assert_close(y[torch.from_numpy(ok2)], ref[ok2], "bf16", "moe block B=%d d=%d E=%d" % (B, d, E))
+
+
+def test_primary_blind_to_aux_and_identical_flows(cuda_device):
+    B, d, F, E, k, k_aux = 16, 256, 512, 8, 2, 4
+    x, w_r, w_gu, w_down = _case(130, B, d, F, E)
+    y0, m0 = _block(cuda_device, x, w_r, w_gu, w_down, k, k_aux, B)
+    ids0 = m0.ids.cpu().clone()
+    bad = x.clone()
+    bad[B:] = float("nan")
+    y1, m1 = _block(cuda_device, bad, w_r, w_gu, w_down, k, k_aux, B)
+    assert torch.equal(m1.ids.cpu(), ids0)
+    assert torch.equal(y1[:B].view(torch.int16), y0[:B].view(torch.int16))
+    assert torch.isnan(y1[B:].float()).all()
+    same = torch.cat([x[:B], x[:B]])
+    y2, _ = _block(cuda_device, same, w_r, w_gu, w_down, k, k, B)
+    assert torch.equal(y2[:B].view(torch.int16), y2[B:].view(torch.int16))
