@@ -49,7 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "mha", "gqa", "long", "tiny", "mixture"],
+    ap.add_argument("--workload",
+                    choices=["layer", "mha", "gqa", "long", "tiny", "mixture", "moe"],
                     default="layer")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -417,6 +418,97 @@ class MixtureRun:
         return int(self.err.item())
 
 
+class MoERun:
+    """MoE MLP block of both flows with router replay: route, dispatch, the
+    experts' grouped projections, combine (+ residual)."""
+
+    timer_keys = ("experts",)
+    dominant_key = "experts"
+
+    def __init__(self, args, dev, seed):
+        import torch
+        from dual_flow_transformer_b200 import api, synth
+        from dual_flow_transformer_b200.moe import DualFlowMoE
+        w = synth.WORKLOADS["moe"]
+        self.w = w
+        self.api = api
+        self.host = synth.make_moe_inputs(w, seed=seed)
+        h = self.host
+        self.x = h["x"].to(dev)
+        self.moe = DualFlowMoE(h["w_router"].to(dev), h["w_gu"].to(dev), h["w_down"].to(dev),
+                               w.k, w.k_aux, B=w.B, device=dev)
+        self.err = self.moe.err
+        B, d, F, E = w.B, w.d_model, w.F, w.E
+        self.tokens_per_step = B
+        self.launches_per_step = self.moe.launches
+        self.units = E
+        self.bytes_per_unit = 3 * F * d * 2
+        rows = 2 * api.MOE_ROWS
+        self.dom_bytes = E * (self.bytes_per_unit + rows * d * 2 + rows * F * 2 * 2 + rows * d * 2)
+        self.config = {"workload": "dual-flow MoE MLP block with router replay: %d tokens per "
+                                   "flow, d_model %d, %d SwiGLU experts of width %d, primary "
+                                   "top-%d, auxiliary fan-out %d (%.1f MB of expert weights)"
+                                   % (B, d, E, F, w.k, w.k_aux, E * 3 * F * d * 2 / 1e6),
+                       "l2": "inputs larger than L2 (%.0f MB of expert weights per step)"
+                             % (E * 3 * F * d * 2 / 1e6)}
+        self.dominant = "dualflow_grouped_proj (expert SwiGLU projections, tcgen05)"
+        self._all()
+        torch.cuda.synchronize()
+        self.g_full, self.g_pre, self.g_exp, self.g_post = (torch.cuda.CUDAGraph() for _ in range(4))
+        with torch.cuda.graph(self.g_full):
+            self._all()
+        with torch.cuda.graph(self.g_pre):
+            self._pre()
+        with torch.cuda.graph(self.g_exp):
+            self._experts()
+        with torch.cuda.graph(self.g_post):
+            self._post()
+        torch.cuda.synchronize()
+
+    def _pre(self):
+        m, w = self.moe, self.w
+        self.api.moe_route(self.x, w.B, m.w_router, w.k, w.k_aux, ids=m.ids, g1=m.g1, g2=m.g2)
+        self.api.moe_dispatch(self.x, w.B, m.ids, w.E, w.k, w.k_aux, xe=m.xe, slot1=m.slot1,
+                              slot2=m.slot2, counts=m.counts, err_flag=m.err)
+
+    def _experts(self):
+        self.moe.experts()
+
+    def _post(self):
+        m, w = self.moe, self.w
+        self.api.moe_combine(m.ye, m.ids, m.g1, m.g2, m.slot1, m.slot2, w.B, w.k, w.k_aux,
+                             residual=self.x, y=m.y, err_flag=m.err)
+
+    def _all(self):
+        self._pre()
+        self._experts()
+        self._post()
+
+    def step(self, timers=None):
+        if timers is None:
+            self.g_full.replay()
+            return
+        self.g_pre.replay()
+        timers["experts"][0].record()
+        self.g_exp.replay()
+        timers["experts"][1].record()
+        self.g_post.replay()
+
+    def host_io(self):
+        import torch
+        x = self.x.cpu().pin_memory()
+        o = torch.empty(tuple(self.moe.y.shape), dtype=torch.bfloat16).pin_memory()
+        return x, o
+
+    def step_host(self, x_host, o_host):
+        self.x.copy_(x_host, non_blocking=True)
+        self.step()
+        o_host.copy_(self.moe.y, non_blocking=True)
+
+    def check_err(self):
+        return int(self.err.item())
+
+
 # ----------------------------------------------------------------------------- oracle timing
 
 def _threads_used():
@@ -481,6 +573,8 @@ def time_oracle(run, workload, budget_s, max_steps=None):
         return n_seq * steps / el, sample, el, steps
     if workload == "mixture":
         return time_oracle_mixture(run.host, budget_s)
+    if workload == "moe":
+        return time_oracle_moe(run.host, budget_s)
     B = run.w.B
     sel, el, k = [], 0.0, 0
     inp_all = None
@@ -526,6 +620,32 @@ def time_oracle_mixture(host, budget_s):
     return k / el, sample, el, k
 
 
+def time_oracle_moe(host, budget_s, tokens_per_call=4):
+    """The oracle MoE block on a few tokens per call (both flows); the
+    experts' weights are widened to fp64 once, outside the timing."""
+    import numpy as np
+    import oracle
+    import torch
+    if "w64" not in host:
+        f = lambda t: t.to(torch.float32).numpy().astype(np.float64)
+        host["w64"] = (f(host["w_router"]), f(host["w_gu"]), f(host["w_down"]))
+    wr, wgu, wd = host["w64"]
+    x = host["x"].to(torch.float32).numpy().astype(np.float64)
+    B = host["B"]
+    k, el, calls = 0, 0.0, 0
+    while el < budget_s and calls < 64:
+        sel = [(k + i) % B for i in range(tokens_per_call)]
+        t0 = time.perf_counter()
+        oracle.moe_forward(x[sel], x[[B + s for s in sel]], wr, wgu, wd, host["k"], host["k_aux"],
+                           x[sel], x[[B + s for s in sel]])
+        el += time.perf_counter() - t0
+        k += tokens_per_call
+        calls += 1
+    sample = ("fp64 oracle MoE block (both flows, router replay) on %d token(s) in calls of %d; "
+              "expert weights pre-widened to fp64 outside the timing" % (k, tokens_per_call))
+    return k / el, sample, el, k
+
+
 # ----------------------------------------------------------------------------- main
 
 def run_reference(args):
@@ -540,10 +660,14 @@ def run_reference(args):
         pass
 
     h = Host()
-    if args.workload == "mixture":
-        h.w = synth.WORKLOADS["mixture"]
-        h.host = synth.make_mixture_inputs(h.w)
-        v, sample, el, steps = time_oracle_mixture(h.host, 20.0)
+    if args.workload in ("mixture", "moe"):
+        h.w = synth.WORKLOADS[args.workload]
+        if args.workload == "mixture":
+            h.host = synth.make_mixture_inputs(h.w)
+            v, sample, el, steps = time_oracle_mixture(h.host, 20.0)
+        else:
+            h.host = synth.make_moe_inputs(h.w)
+            v, sample, el, steps = time_oracle_moe(h.host, 20.0)
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
                 "n_gpus": world, "steps": steps, "steps_requested": args.steps,
                 "warmup": args.warmup, "ms_per_step": el / steps * 1e3, "higher_is_better": True,
@@ -626,6 +750,8 @@ def main(argv=None):
         run = LayerRun(args, dev, seed)
     elif args.workload == "mixture":
         run = MixtureRun(args, dev, seed)
+    elif args.workload == "moe":
+        run = MoERun(args, dev, seed)
     else:
         run = AttnRun(args, dev, seed, args.workload)
 

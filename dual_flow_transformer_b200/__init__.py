@@ -10,6 +10,7 @@ from .api import (  # noqa: F401
     decode_attn_num_splits,
     decode_attn_workspace_size,
     grouped_proj,
+    grouped_proj_batched,
     grouped_proj_num_launches,
     grouped_proj_workspace_size,
     kv_append,

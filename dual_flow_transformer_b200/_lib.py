@@ -71,6 +71,14 @@ SIGNATURES = {
                                        _vp, _vp, _vp, _vp, _vp, _vp]),
     "dualflow_moe_combine": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _vp, _c_i64, _vp, _c_i64, _vp, _vp]),
+    "dualflow_grouped_proj_batched": (_c_int, [
+        _vp, _c_i64, _c_i64, _c_int, _c_int,    # x, ldx, x_bstride, m_primary, m_aux
+        _vp, _c_int, _c_int, _c_i64,            # w, N, K, w_bstride
+        _vp, _c_i64, _c_i64, _c_int, _c_int,    # y, ldy, y_bstride, batch, epilogue
+        _vp, _c_size,                           # workspace, bytes
+        _vp, _c_int, _c_int, _c_int, _c_int, _c_i64,  # next: w, N, K, epilogue, batch, bstride
+        _vp, _vp]),                             # err_flag, stream
+    "dualflow_grouped_proj_batched_num_launches": (_c_int, [_c_int] * 5),
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
 }
 

@@ -192,6 +192,42 @@ def grouped_proj(x, m_primary, w, *, n_aux=None, y=None, epilogue="none", coupli
     return y
 
 
+def grouped_proj_batched(x, m_primary, w, *, y=None, epilogue="none", workspace=None,
+                         err_flag=None, stream=None, next_w=None, next_epilogue="none"):
+    """A batch of projections of one shape in one launch: y[b] = epilogue(x[b]
+    w[b]^T) for x bf16 [batch, M, K], w bf16 [batch, N, K] (contiguous), y
+    bf16 [batch, M, n_out]; epilogue "none" or "swiglu" (no coupling, no
+    residual). next_w ([N', K'] or [batch', N', K']) hints the next projection
+    on the stream for an L2 prefetch (results do not change)."""
+    batch, M, K = x.shape
+    _, N, K2 = w.shape
+    if K2 != K or not x.is_contiguous() or not w.is_contiguous():
+        raise ValueError("x [batch, M, K] and w [batch, N, K] contiguous required")
+    epi = EPILOGUES[epilogue]
+    n_out = N // 2 if epi == L.DF_EPI_SWIGLU else N
+    if y is None:
+        y = torch.empty((batch, M, n_out), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        workspace = new_proj_workspace(M, N, K, epilogue, x.device)
+    if next_w is None:
+        nw, nN, nK, nb, nbs = None, 0, 0, 1, 0
+    else:
+        nw3 = next_w if next_w.dim() == 3 else next_w.unsqueeze(0)
+        nb, nN, nK = nw3.shape
+        nw, nbs = next_w, nN * nK
+    st = _lib().dualflow_grouped_proj_batched(
+        _ptr(x), x.stride(1), x.stride(0), int(m_primary), int(M - m_primary), _ptr(w), N, K,
+        w.stride(0), _ptr(y), y.stride(1), y.stride(0), batch, epi, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(nw), nN, nK,
+        EPILOGUES[next_epilogue], nb, nbs, _ptr(err_flag), _stream(stream))
+    L.check("dualflow_grouped_proj_batched", st)
+    return y
+
+
+def grouped_proj_batched_num_launches(M, N, K, epilogue, batch) -> int:
+    return _lib().dualflow_grouped_proj_batched_num_launches(M, N, K, EPILOGUES[epilogue], batch)
+
+
 # ----------------------------------------------------------------- MoE router replay
 
 MOE_ROWS = 64  # rows per flow in an expert block: at most 64 tokens per call

@@ -550,7 +550,9 @@ df_status grouped_proj_impl(const void* x, int64_t ldx, int m_primary, int m_aux
                             const void* coupling, const void* residual, int64_t ldr,
                             void* workspace, size_t workspace_bytes, const void* w_next,
                             int N_next, int K_next, int epilogue_next, int32_t* err_flag,
-                            void* stream) {
+                            void* stream, int batch = 1, int64_t x_bstride = 0,
+                            int64_t w_bstride = 0, int64_t y_bstride = 0, int batch_next = 1,
+                            int64_t w_next_bstride = 0) {
   using namespace df;
   using namespace df::gemm;
   if (!x || !w || !y) return DF_ERR_NULL;
@@ -609,10 +611,22 @@ df_status grouped_proj_impl(const void* x, int64_t ldx, int m_primary, int m_aux
     // tile-parallel / cluster split-K plan when it is modelled to be faster
     tgemm::Request rq{x, lx, m_primary, m_aux, w, N, K, n_aux, y, ly, epilogue, coupling,
                       residual, lr, err_flag, st, workspace, workspace_bytes,
-                      w_next, N_next, K_next, epilogue_next};
+                      w_next, N_next, K_next, epilogue_next, batch, x_bstride, w_bstride,
+                      y_bstride, batch_next, w_next_bstride};
     const int launched = tgemm::launch_if_better(rq);
     if (launched < 0) return DF_ERR_CUDA;
     if (launched > 0) return DF_OK;
+  }
+  if (batch > 1) {  // no single-launch plan: one projection per batch entry
+    for (int b = 0; b < batch; ++b) {
+      const df_status sb = grouped_proj_impl(
+          static_cast<const __nv_bfloat16*>(x) + b * x_bstride, ldx, m_primary, m_aux,
+          static_cast<const __nv_bfloat16*>(w) + b * w_bstride, N, K, n_aux,
+          static_cast<__nv_bfloat16*>(y) + b * y_bstride, ldy, epilogue, nullptr, nullptr, 0,
+          workspace, workspace_bytes, nullptr, 0, 0, 0, err_flag, stream);
+      if (sb != DF_OK) return sb;
+    }
+    return DF_OK;
   }
   CUtensorMap tmX, tmW;
   if (!encode_tmap_bf16_2d(&tmX, x, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -658,6 +672,45 @@ extern "C" df_status dualflow_grouped_proj(const void* x, int64_t ldx, int m_pri
   return grouped_proj_impl(x, ldx, m_primary, m_aux, w, N, K, n_aux, y, ldy, epilogue, coupling,
                            residual, ldr, workspace, workspace_bytes, nullptr, 0, 0, 0, err_flag,
                            stream);
+}
+
+extern "C" df_status dualflow_grouped_proj_batched(
+    const void* x, int64_t ldx, int64_t x_bstride, int m_primary, int m_aux, const void* w, int N,
+    int K, int64_t w_bstride, void* y, int64_t ldy, int64_t y_bstride, int batch, int epilogue,
+    void* workspace, size_t workspace_bytes, const void* w_next, int N_next, int K_next,
+    int epilogue_next, int batch_next, int64_t w_next_bstride, int32_t* err_flag, void* stream) {
+  using namespace df;
+  if (!x || !w || !y) return DF_ERR_NULL;
+  if (batch < 1 || batch > 65535 || (w_next && (batch_next < 1 || batch_next > 65535)))
+    return DF_ERR_SHAPE;
+  if (epilogue != DF_EPI_NONE && epilogue != DF_EPI_SWIGLU) return DF_ERR_UNSUPPORTED;
+  const int M = m_primary + m_aux;
+  const int n_out = epilogue == DF_EPI_SWIGLU ? N / 2 : N;
+  const int64_t lx = ldx ? ldx : K, ly = ldy ? ldy : n_out;
+  const int64_t xs = x_bstride ? x_bstride : lx * M;
+  const int64_t wsd = w_bstride ? w_bstride : static_cast<int64_t>(N) * K;
+  const int64_t ys = y_bstride ? y_bstride : ly * M;
+  if (M < 1 || N < 1 || K < 1 || xs < lx * M || wsd < static_cast<int64_t>(N) * K ||
+      ys < ly * M)
+    return DF_ERR_SHAPE;
+  if (xs % 8 || wsd % 8 || ys % 8) return DF_ERR_ALIGN;
+  const int64_t wns = w_next_bstride ? w_next_bstride : static_cast<int64_t>(N_next) * K_next;
+  if (w_next && (wns < static_cast<int64_t>(N_next) * K_next || wns % 8)) return DF_ERR_SHAPE;
+  return grouped_proj_impl(x, lx, m_primary, m_aux, w, N, K, n_out, y, ly, epilogue, nullptr,
+                           nullptr, 0, workspace, workspace_bytes, w_next, N_next, K_next,
+                           epilogue_next, err_flag, stream, batch, xs, wsd, ys,
+                           w_next ? batch_next : 1, wns);
+}
+
+extern "C" int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue,
+                                                          int batch) {
+  using namespace df::gemm;
+  if (M < 1 || N < 1 || K < 1 || batch < 1 || (epilogue != DF_EPI_NONE && epilogue != DF_EPI_SWIGLU))
+    return 0;
+  const Layout l = make_layout(N, K, epilogue);
+  if (l.total < 1) return 0;
+  if (df::tgemm::planned_launches(M, N, K, epilogue, l.partial_bytes, batch)) return 1;
+  return batch * dualflow_grouped_proj_num_launches(M, N, K, epilogue);
 }
 
 extern "C" df_status dualflow_grouped_proj_chain(

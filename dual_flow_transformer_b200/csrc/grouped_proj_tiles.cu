@@ -52,6 +52,8 @@ constexpr size_t kSmemBytes =
 struct Params {
   int M, m_primary, n_out, n_aux, epilogue;
   int kblocks, BN, half, out_per_tile, n_tiles, C, stages, stage_bytes;
+  int tpb;            // tiles per batch entry: tile t is (batch t / tpb, column tile t % tpb)
+  int64_t ystride_b;  // output batch stride (elements)
   uint32_t idesc;
   int F;
   __nv_bfloat16* y;
@@ -65,7 +67,7 @@ struct Params {
   // width, cluster size, tile and CTA counts, k-blocks, SwiGLU half width and
   // gate/up offset; pf_stages k-blocks from the start of each of its CTAs'
   // slices.
-  int pf_stages, pf_BN, pf_C, pf_ntiles, pf_ctas, pf_kblocks, pf_half, pf_F;
+  int pf_stages, pf_BN, pf_C, pf_ntiles, pf_ctas, pf_kblocks, pf_half, pf_F, pf_tpb;
 };
 
 __device__ __forceinline__ void epi_bar() {
@@ -116,9 +118,9 @@ __device__ __forceinline__ bool store_ok(const Params& p, int row, int col) {
 // bf16 store. W = 32 goes through the warp's staging tile so that stores are
 // row-contiguous; W = 8 (tile tails) stores per row.
 template <int W>
-__device__ __forceinline__ void finish_chunk(const Params& p, int quarter, int lane, int col0,
-                                             float (&val)[W], float* xbuf, float* stg,
-                                             const float* cpl) {
+__device__ __forceinline__ void finish_chunk(const Params& p, __nv_bfloat16* y, int quarter,
+                                             int lane, int col0, float (&val)[W], float* xbuf,
+                                             float* stg, const float* cpl) {
   const int row = quarter * 32 + lane;
   if (p.coupling != nullptr) {
     if (row < p.m_primary) {
@@ -152,7 +154,7 @@ __device__ __forceinline__ void finish_chunk(const Params& p, int quarter, int l
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[i] += rv[i];
       }
-      store_bf16x4(p.y + r * p.ldy + col0 + cg, o);
+      store_bf16x4(y + r * p.ldy + col0 + cg, o);
     }
     __syncwarp();
   } else {
@@ -163,14 +165,15 @@ __device__ __forceinline__ void finish_chunk(const Params& p, int quarter, int l
 #pragma unroll
         for (int i = 0; i < W; ++i) val[i] += rv[i];
       }
-      store_bf16<W>(p.y + row * p.ldy + col0, val);
+      store_bf16<W>(y + row * p.ldy + col0, val);
     }
   }
 }
 
-// Epilogue of a whole tile straight from TMEM (C = 1).
-__device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, uint32_t taddr,
-                              float* xbuf, float* stg, const float* cpl_s) {
+// Epilogue of a whole tile straight from TMEM (C = 1); tile = column tile,
+// y = the output matrix of its batch entry.
+__device__ void tile_epilogue(const Params& p, int tile, __nv_bfloat16* y, int quarter, int lane,
+                              uint32_t taddr, float* xbuf, float* stg, const float* cpl_s) {
   const int col0 = tile * p.out_per_tile;
   if (p.epilogue == DF_EPI_SWIGLU) {
     const int H = p.half;
@@ -181,7 +184,7 @@ __device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, 
       tmem_ld<32>(taddr + H + c, u);
 #pragma unroll
       for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
-      finish_chunk<32>(p, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
+      finish_chunk<32>(p, y, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
     }
     for (; c < H; c += 8) {
       float g[8], u[8];
@@ -189,19 +192,19 @@ __device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, 
       tmem_ld<8>(taddr + H + c, u);
 #pragma unroll
       for (int i = 0; i < 8; ++i) g[i] = silu_f(g[i]) * u[i];
-      finish_chunk<8>(p, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
+      finish_chunk<8>(p, y, quarter, lane, col0 + c, g, xbuf, stg, cpl_s + c);
     }
   } else {
     int c = 0;
     for (; c + 32 <= p.BN; c += 32) {
       float v[32];
       tmem_ld<32>(taddr + c, v);
-      finish_chunk<32>(p, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
+      finish_chunk<32>(p, y, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
     }
     for (; c < p.BN; c += 8) {
       float v[8];
       tmem_ld<8>(taddr + c, v);
-      finish_chunk<8>(p, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
+      finish_chunk<8>(p, y, quarter, lane, col0 + c, v, xbuf, stg, cpl_s + c);
     }
   }
 }
@@ -213,8 +216,8 @@ __device__ void tile_epilogue(const Params& p, int tile, int quarter, int lane, 
 // the C partial loads of both rows issued before any sum (this loop runs on
 // six warps, so its latency is not hidden by other warps).
 template <int C>
-__device__ void cluster_epilogue_c(const Params& p, int tile, int rank, const float* recv,
-                                   float* prim, int tid, int nthreads,
+__device__ void cluster_epilogue_c(const Params& p, int tile, __nv_bfloat16* y, int rank,
+                                   const float* recv, float* prim, int tid, int nthreads,
                                    const __nv_bfloat16* res_s, const float* cpl_s) {
   const int pitch = p.BN + 4;
   const bool coupled = p.coupling != nullptr;
@@ -290,24 +293,24 @@ __device__ void cluster_epilogue_c(const Params& p, int tile, int rank, const fl
 #pragma unroll
           for (int i = 0; i < 4; ++i) o[i] += rv[i];
         }
-        store_bf16x4(p.y + row * p.ldy + col, o);
+        store_bf16x4(y + row * p.ldy + col, o);
       }
     }
     if (coupled && pass == 0) __syncthreads();
   }
 }
 
-__device__ void cluster_epilogue(const Params& p, int tile, int rank, const float* recv,
-                                 float* prim, int tid, int nthreads,
+__device__ void cluster_epilogue(const Params& p, int tile, __nv_bfloat16* y, int rank,
+                                 const float* recv, float* prim, int tid, int nthreads,
                                  const __nv_bfloat16* res_s, const float* cpl_s) {
   switch (p.C) {
-    case 2: cluster_epilogue_c<2>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    case 3: cluster_epilogue_c<3>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    case 4: cluster_epilogue_c<4>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    case 5: cluster_epilogue_c<5>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    case 6: cluster_epilogue_c<6>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    case 7: cluster_epilogue_c<7>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
-    default: cluster_epilogue_c<8>(p, tile, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 2: cluster_epilogue_c<2>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 3: cluster_epilogue_c<3>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 4: cluster_epilogue_c<4>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 5: cluster_epilogue_c<5>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 6: cluster_epilogue_c<6>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    case 7: cluster_epilogue_c<7>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
+    default: cluster_epilogue_c<8>(p, tile, y, rank, recv, prim, tid, nthreads, res_s, cpl_s); break;
   }
 }
 
@@ -389,12 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       auto load_w = [&](int s, int t, int kb) {
+        const int e = t / p.tpb, tn = t - e * p.tpb;
         uint8_t* sb = smem + s * p.stage_bytes + kTileX;
         if (p.epilogue == DF_EPI_SWIGLU) {
-          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.half, pol_w);
-          tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + t * p.half, pol_w);
+          tma_load_3d_hint(sb, &tmW, &full[s], kb * kBK, tn * p.half, e, pol_w);
+          tma_load_3d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + tn * p.half, e,
+                           pol_w);
         } else {
-          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, t * p.BN, pol_w);
+          tma_load_3d_hint(sb, &tmW, &full[s], kb * kBK, tn * p.BN, e, pol_w);
         }
       };
       // The weights are no product of the previous kernel: the first ring
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = static_cast<int>(n % S);
           uint8_t* sa = smem + s * p.stage_bytes;
           if (n < pre) {  // weights already on their way
-            tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+            tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
             continue;
           }
           if (n >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / S) - 1) & 1))) {
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], p.stage_bytes);
-          tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
+          tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
           load_w(s, t, kb);
         }
       }
@@ -443,12 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             k1 = (r + 1) * p.pf_kblocks / p.pf_C;
           }
           if (t >= p.pf_ntiles) continue;
+          const int e = t / p.pf_tpb, tn = t - e * p.pf_tpb;
           for (int kb = k0; kb < k1 && kb < k0 + p.pf_stages; ++kb) {
             if (p.pf_half > 0) {
-              tma_prefetch_2d(&tmWn, kb * kBK, t * p.pf_half);
-              tma_prefetch_2d(&tmWn, kb * kBK, p.pf_F + t * p.pf_half);
+              tma_prefetch_3d(&tmWn, kb * kBK, tn * p.pf_half, e);
+              tma_prefetch_3d(&tmWn, kb * kBK, p.pf_F + tn * p.pf_half, e);
             } else {
-              tma_prefetch_2d(&tmWn, kb * kBK, t * p.pf_BN);
+              tma_prefetch_3d(&tmWn, kb * kBK, tn * p.pf_BN, e);
             }
           }
         }
@@ -500,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // staging area -- the tile's coupling slice and, when they fit, the
       // residual rows it will write.
       const int opt = p.out_per_tile;
-      const int col0 = tile_first * opt;
+      const int col0 = (tile_first % p.tpb) * opt;  // coupling / residual: one batch entry
       const bool coupled = p.coupling != nullptr;
       const int rows_base = coupled ? p.m_primary : p.M;
       const int r0 = rank * rows_base / p.C, r1 = (rank + 1) * rows_base / p.C;
@@ -530,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = seg & 1;
       if (p.C == 1 && p.coupling != nullptr) {
         // this tile's coupling vector, fetched while the MMAs run
-        const int c0 = t * p.out_per_tile;
+        const int c0 = (t % p.tpb) * p.out_per_tile;
         for (int i = et; i < p.out_per_tile; i += kEpiThreads)
           cpl_s[i] = (c0 + i < p.n_out) ? __bfloat162float(p.coupling[c0 + i]) : 0.f;
       }
@@ -544,7 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * p.BN;
       if (p.C == 1) {
-        tile_epilogue(p, t, quarter, lane, taddr, xbuf, stg, cpl_s);
+        tile_epilogue(p, t % p.tpb, p.y + (t / p.tpb) * p.ystride_b, quarter, lane, taddr, xbuf,
+                      stg, cpl_s);
       } else {
         // park the fp32 accumulator rows in this CTA's shared memory (the ring
         // is idle: every stage has been consumed by the MMAs that completed)
@@ -619,7 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       if (threadIdx.x == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
     } else {
-      cluster_epilogue(p, tile_first, rank, recv, prim, threadIdx.x, kThreads, res_s, cpl_s);
+      cluster_epilogue(p, tile_first % p.tpb, p.y + (tile_first / p.tpb) * p.ystride_b, rank,
+                       recv, prim, threadIdx.x, kThreads, res_s, cpl_s);
     }
   }
   if (warp == 1) {
@@ -683,13 +691,15 @@ struct Plan {
   bool ok;
   int BN, C, n_tiles, ctas, stages, stage_bytes;
   double est_us;
+  int tpb;  // tiles per batch entry (n_tiles = batch * tpb)
 };
 
 // Pick the tile width and cluster size with the lowest modelled time. Rates:
 // ~46 GB/s of DRAM and ~77 GB/s of total TMA traffic per SM (measured with a
 // TMA streaming probe on B200), plus fixed costs for the cluster exchange and
 // per-tile epilogues.
-Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_t ws_bytes) {
+Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_t ws_bytes,
+               int batch = 1) {
   Plan best{};
   best.ok = false;
   best.est_us = 1e30;
@@ -698,7 +708,8 @@ Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_
   const int KB = K / kBK;
   for (int BN = 256; BN >= 64; BN -= 16) {
     const int opt = swiglu ? BN / 2 : BN;
-    const int n_tiles = static_cast<int>(ceil_div(n_out, opt));
+    const int tpb = static_cast<int>(ceil_div(n_out, opt));
+    const int n_tiles = tpb * batch;
     const int stage_bytes = kTileX + BN * 128;
     int stages = kRingBytes / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
@@ -726,7 +737,7 @@ Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_
       if (tot / 77e3 > t) t = tot / 77e3;
       t += (C > 1 ? 2.5 : 0.0) + tpc * 1.5 + 2.5;
       if (t < best.est_us) {
-        best = Plan{true, BN, C, n_tiles, ctas, stages, stage_bytes, t};
+        best = Plan{true, BN, C, n_tiles, ctas, stages, stage_bytes, t, tpb};
       }
     }
   }
@@ -748,19 +759,26 @@ double stream_k_estimate(int N, int K, int epilogue) {
   return t + 2.5 + 3.0 + (split ? 7.0 : 0.0);
 }
 
-int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes) {
-  const Plan pl = make_plan(M, N, K, epilogue, caps_for_device(), ws_bytes);
-  if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(N, K, epilogue)) return 0;
-  return 1;
+// The tile plan is taken when it fills at least 3/4 of the SMs and beats the
+// stream-K kernel run once per batch entry.
+bool tile_plan_wins(const Plan& pl, int N, int K, int epilogue, int batch) {
+  return pl.ok && pl.ctas >= kSms * 3 / 4 &&
+         pl.est_us < batch * stream_k_estimate(N, K, epilogue);
+}
+
+int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes, int batch) {
+  const Plan pl = make_plan(M, N, K, epilogue, caps_for_device(), ws_bytes, batch);
+  return tile_plan_wins(pl, N, K, epilogue, batch) ? 1 : 0;
 }
 
 int launch_if_better(const Request& r) {
   const int M = r.m_primary + r.m_aux;
   const ClusterCaps* caps = caps_for_device();
   if (!caps) return 0;
-  const Plan pl = make_plan(M, r.N, r.K, r.epilogue, caps, r.workspace ? r.workspace_bytes : 0);
-  if (!pl.ok || pl.ctas < kSms * 3 / 4 || pl.est_us >= stream_k_estimate(r.N, r.K, r.epilogue))
-    return 0;
+  const int batch = r.batch > 0 ? r.batch : 1;
+  const Plan pl =
+      make_plan(M, r.N, r.K, r.epilogue, caps, r.workspace ? r.workspace_bytes : 0, batch);
+  if (!tile_plan_wins(pl, r.N, r.K, r.epilogue, batch)) return 0;
   const bool swiglu = r.epilogue == DF_EPI_SWIGLU;
   Params p{};
   p.M = M;
@@ -773,6 +791,8 @@ int launch_if_better(const Request& r) {
   p.half = swiglu ? pl.BN / 2 : 0;
   p.out_per_tile = swiglu ? pl.BN / 2 : pl.BN;
   p.n_tiles = pl.n_tiles;
+  p.tpb = pl.tpb;
+  p.ystride_b = r.y_bstride;
   p.C = pl.C;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
@@ -789,15 +809,18 @@ int launch_if_better(const Request& r) {
   memset(&tmWn, 0, sizeof(tmWn));
   if (r.w_next != nullptr) {
     const size_t ws = r.workspace ? r.workspace_bytes : 0;
-    const Plan nx = make_plan(M, r.N_next, r.K_next, r.epilogue_next, caps, ws);
-    const bool nx_tiles = nx.ok && nx.ctas >= kSms * 3 / 4 &&
-                          nx.est_us < stream_k_estimate(r.N_next, r.K_next, r.epilogue_next);
+    const int nb = r.batch_next > 0 ? r.batch_next : 1;
+    const Plan nx = make_plan(M, r.N_next, r.K_next, r.epilogue_next, caps, ws, nb);
+    const bool nx_tiles = tile_plan_wins(nx, r.N_next, r.K_next, r.epilogue_next, nb);
     const bool nx_swiglu = r.epilogue_next == DF_EPI_SWIGLU;
     const int box_rows = nx_swiglu ? nx.BN / 2 : nx.BN;
+    const int64_t wn_stride =
+        r.w_next_bstride > 0 ? r.w_next_bstride : static_cast<int64_t>(r.N_next) * r.K_next;
     if (nx_tiles &&
-        encode_tmap_bf16_2d(&tmWn, r.w_next, static_cast<uint64_t>(r.N_next),
-                            static_cast<uint64_t>(r.K_next), static_cast<uint64_t>(r.K_next) * 2,
-                            box_rows, kBK)) {
+        encode_tmap_bf16_3d(&tmWn, r.w_next, static_cast<uint64_t>(nb),
+                            static_cast<uint64_t>(r.N_next), static_cast<uint64_t>(r.K_next),
+                            static_cast<uint64_t>(r.K_next) * 2,
+                            static_cast<uint64_t>(wn_stride) * 2, box_rows, kBK)) {
       // ~28 MB in all: what DRAM delivers in a few microseconds of tail
       const double per_stage = static_cast<double>(nx.ctas) * nx.BN * kBK * 2;
       int st = static_cast<int>(28.0 * 1024 * 1024 / per_stage);
@@ -809,13 +832,18 @@ int launch_if_better(const Request& r) {
       p.pf_kblocks = r.K_next / kBK;
       p.pf_half = nx_swiglu ? nx.BN / 2 : 0;
       p.pf_F = r.N_next / 2;
+      p.pf_tpb = nx.tpb;
     }
   }
   CUtensorMap tmX, tmW;
-  if (!encode_tmap_bf16_2d(&tmX, r.x, static_cast<uint64_t>(M), static_cast<uint64_t>(r.K),
-                           static_cast<uint64_t>(r.ldx) * 2, kBM, kBK) ||
-      !encode_tmap_bf16_2d(&tmW, r.w, static_cast<uint64_t>(r.N), static_cast<uint64_t>(r.K),
-                           static_cast<uint64_t>(r.K) * 2, swiglu ? pl.BN / 2 : pl.BN, kBK))
+  const int64_t xs = r.x_bstride > 0 ? r.x_bstride : static_cast<int64_t>(M) * r.ldx;
+  const int64_t wsd = r.w_bstride > 0 ? r.w_bstride : static_cast<int64_t>(r.N) * r.K;
+  if (!encode_tmap_bf16_3d(&tmX, r.x, static_cast<uint64_t>(batch), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.ldx) * 2,
+                           static_cast<uint64_t>(xs) * 2, kBM, kBK) ||
+      !encode_tmap_bf16_3d(&tmW, r.w, static_cast<uint64_t>(batch), static_cast<uint64_t>(r.N),
+                           static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.K) * 2,
+                           static_cast<uint64_t>(wsd) * 2, swiglu ? pl.BN / 2 : pl.BN, kBK))
     return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.ctas);

@@ -29,6 +29,13 @@ struct Request {
   // launch's tail. w_next NULL = none.
   const void* w_next;
   int N_next, K_next, epilogue_next;
+  // Batched form (batch > 1): `batch` independent projections of the same
+  // shape, entry b at x + b*x_bstride, w + b*w_bstride, y + b*y_bstride
+  // (elements); the next projection may be batched too.
+  int batch;
+  int64_t x_bstride, w_bstride, y_bstride;
+  int batch_next;
+  int64_t w_next_bstride;
 };
 
 // Launches the tile plan when it is modelled to beat stream-K on this device.
@@ -38,7 +45,7 @@ int launch_if_better(const Request& r);
 
 // 1 if the tile plan would be used for this shape on the current device with
 // a workspace of ws_bytes, else 0.
-int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes);
+int planned_launches(int M, int N, int K, int epilogue, size_t ws_bytes, int batch = 1);
 
 }  // namespace tgemm
 }  // namespace df

@@ -23,6 +23,12 @@ inline bool aligned(const void* p, uintptr_t n) {
 bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                          uint64_t row_pitch_bytes, uint32_t box_rows, uint32_t box_cols);
 
+// 3-D variant: `batch` matrices of [rows][cols], batch_pitch_bytes apart
+// (a multiple of 16); boxes of [box_rows][box_cols] in one matrix.
+bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t batch, uint64_t rows,
+                         uint64_t cols, uint64_t row_pitch_bytes, uint64_t batch_pitch_bytes,
+                         uint32_t box_rows, uint32_t box_cols);
+
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();
 

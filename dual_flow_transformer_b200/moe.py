@@ -4,10 +4,10 @@ Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi Chiave"
 (router replay) and section "Contributi Chiave" (independent expert fan-outs
 of the two flows). One block call: route (primary top-k_aux, gates of both
 flows) -> dispatch (each expert's rows packed into a fixed [128][d] block) ->
-per expert, the gate/up projection with the SwiGLU epilogue and the down
-projection on the grouped tcgen05 kernel, each hinting the next projection's
-weights into L2 -> combine (+ residual). Every expert's weights stream from
-HBM once per call for both flows.
+the gate/up projections of all experts in one batched launch (SwiGLU
+epilogue), then the down projections of all experts in one batched launch,
+each hinting the other's weights into L2 -> combine (+ residual). Every
+expert's weights stream from HBM once per call for both flows.
 """
 
 from __future__ import annotations
@@ -32,7 +32,7 @@ class DualFlowMoE:
         dev = torch.device(device)
         rows = 2 * api.MOE_ROWS
         self.xe = torch.zeros((E, rows, d), dtype=torch.bfloat16, device=dev)
-        self.h = torch.empty((rows, self.F), dtype=torch.bfloat16, device=dev)
+        self.h = torch.empty((E, rows, self.F), dtype=torch.bfloat16, device=dev)
         self.ye = torch.zeros((E, rows, d), dtype=torch.bfloat16, device=dev)
         self.ids = torch.empty((B, self.k_aux), dtype=torch.int32, device=dev)
         self.g1 = torch.empty((B, self.k), dtype=torch.float32, device=dev)
@@ -45,8 +45,8 @@ class DualFlowMoE:
         ws = max(api.grouped_proj_workspace_size(rows, 2 * self.F, d, "swiglu"),
                  api.grouped_proj_workspace_size(rows, d, self.F, "none"))
         self.ws = torch.zeros(max(256, ws), dtype=torch.uint8, device=dev)
-        self.launches = 3 + E * (api.grouped_proj_num_launches(rows, 2 * self.F, d, "swiglu")
-                                 + api.grouped_proj_num_launches(rows, d, self.F, "none"))
+        self.launches = 3 + (api.grouped_proj_batched_num_launches(rows, 2 * self.F, d, "swiglu", E)
+                             + api.grouped_proj_batched_num_launches(rows, d, self.F, "none", E))
 
     def forward(self, x, residual=None, stream=None):
         """x: bf16 [2B, d] (primary rows, then auxiliary rows). Returns the
@@ -56,14 +56,18 @@ class DualFlowMoE:
                       g2=self.g2, stream=stream)
         api.moe_dispatch(x, B, self.ids, E, self.k, self.k_aux, xe=self.xe, slot1=self.slot1,
                          slot2=self.slot2, counts=self.counts, err_flag=self.err, stream=stream)
-        for e in range(E):
-            api.grouped_proj(self.xe[e], api.MOE_ROWS, self.w_gu[e], y=self.h, epilogue="swiglu",
-                             workspace=self.ws, err_flag=self.err, stream=stream,
-                             next_w=self.w_down[e], next_epilogue="none")
-            nxt = self.w_gu[e + 1] if e + 1 < E else None
-            api.grouped_proj(self.h, api.MOE_ROWS, self.w_down[e], y=self.ye[e], workspace=self.ws,
-                             err_flag=self.err, stream=stream, next_w=nxt,
-                             next_epilogue="swiglu")
+        self.experts(stream)
         return api.moe_combine(self.ye, self.ids, self.g1, self.g2, self.slot1, self.slot2, B,
                                self.k, self.k_aux, residual=residual, y=self.y,
                                err_flag=self.err, stream=stream)
+
+    def experts(self, stream=None):
+        """The experts' SwiGLU MLPs: all gate/up projections in one batched
+        launch, then all down projections (each hinting the other's weights,
+        the down launch the next call's gate/up)."""
+        api.grouped_proj_batched(self.xe, api.MOE_ROWS, self.w_gu, y=self.h, epilogue="swiglu",
+                                 workspace=self.ws, err_flag=self.err, stream=stream,
+                                 next_w=self.w_down, next_epilogue="none")
+        api.grouped_proj_batched(self.h, api.MOE_ROWS, self.w_down, y=self.ye, workspace=self.ws,
+                                 err_flag=self.err, stream=stream, next_w=self.w_gu,
+                                 next_epilogue="swiglu")

@@ -79,6 +79,19 @@ class MixtureWorkload:
     seed: int = 6
 
 
+@dataclasses.dataclass(frozen=True)
+class MoEWorkload:
+    """MoE MLP block of both flows with router replay (one decode step)."""
+    name: str
+    B: int          # tokens per flow
+    d_model: int
+    F: int          # expert SwiGLU width
+    E: int          # experts
+    k: int          # primary fan-out
+    k_aux: int      # auxiliary fan-out (k_aux = k: router replay proper)
+    seed: int = 7
+
+
 WORKLOADS = {
     "tiny": AttnWorkload("tiny", 1, 2, 2, 64, "fp32", 128, 128, append=True, seed=1),
     "mha": AttnWorkload("mha", 32, 32, 32, 128, "bf16", 2048, 2048, seed=2),
@@ -86,6 +99,7 @@ WORKLOADS = {
     "long": AttnWorkload("long", 8, 32, 8, 128, "bf16", 32768, 131072, seed=4),
     "layer": LayerWorkload("layer", 64, 4096, 32, 8, 128, 14336, 4096, seed=5),
     "mixture": MixtureWorkload("mixture", 64, 4096, 32000, seed=6),
+    "moe": MoEWorkload("moe", 64, 2048, 5632, 8, 2, 2, seed=7),
 }
 
 
@@ -237,3 +251,21 @@ def make_mixture_inputs(w: MixtureWorkload, seed: Optional[int] = None):
     h2 = _randn(g, (w.B, w.d_model))
     w_head = _randn(g, (w.V, w.d_model), std=0.02, chunk_rows=2048)
     return dict(h1=h1, h2=h2, w_head=w_head, B=w.B, d_model=w.d_model, V=w.V)
+
+
+def make_moe_inputs(w: MoEWorkload, seed: Optional[int] = None):
+    """Host tensors for one MoE block step of workload ``w`` (bf16): x [2B, d]
+    ~ N(0, 1) (primary rows, then auxiliary rows; also the residual), the
+    shared router w_router [E, d] ~ N(0, 0.05) (router logits of standard
+    deviation ~2.3 at d = 2048), w_gu [E, 2F, d] and w_down [E, d, F]
+    ~ N(0, 0.02)."""
+    g = _gen(w.seed if seed is None else seed)
+    x = _randn(g, (2 * w.B, w.d_model))
+    w_router = _randn(g, (w.E, w.d_model), std=0.05)
+    w_gu = torch.empty((w.E, 2 * w.F, w.d_model), dtype=torch.bfloat16)
+    w_down = torch.empty((w.E, w.d_model, w.F), dtype=torch.bfloat16)
+    for e in range(w.E):
+        w_gu[e] = _randn(g, (2 * w.F, w.d_model), std=0.02, chunk_rows=2048)
+        w_down[e] = _randn(g, (w.d_model, w.F), std=0.02, chunk_rows=2048)
+    return dict(x=x, w_router=w_router, w_gu=w_gu, w_down=w_down, B=w.B, d_model=w.d_model,
+                F=w.F, E=w.E, k=w.k, k_aux=w.k_aux)

@@ -249,6 +249,22 @@ df_status dualflow_grouped_proj_chain(const void* x, int64_t ldx, int m_primary,
                                       int K_next, int epilogue_next, int32_t* err_flag,
                                       void* stream);
 
+/* Batched form: `batch` projections of one shape in one launch (the MoE    */
+/* experts: every expert's weights stream once, all experts share one       */
+/* pipeline fill and one tail). Entry b reads x + b*x_bstride and             */
+/* w + b*w_bstride and writes y + b*y_bstride (elements; 0 = packed). Only    */
+/* DF_EPI_NONE and DF_EPI_SWIGLU, no coupling or residual; auxiliary rows     */
+/* store every output column. The optional next-projection hint may itself    */
+/* be batched (batch_next, w_next_bstride). Without a single-launch plan the  */
+/* call runs one projection per entry.                                        */
+df_status dualflow_grouped_proj_batched(
+    const void* x, int64_t ldx, int64_t x_bstride, int m_primary, int m_aux, const void* w, int N,
+    int K, int64_t w_bstride, void* y, int64_t ldy, int64_t y_bstride, int batch, int epilogue,
+    void* workspace, size_t workspace_bytes, const void* w_next, int N_next, int K_next,
+    int epilogue_next, int batch_next, int64_t w_next_bstride, int32_t* err_flag, void* stream);
+/* Kernel launches one batched call makes: 1 with a single-launch plan.      */
+int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue, int batch);
+
 /* ------------------------------------------------------------------------ */
 /* MoE MLP block with router replay.                                         */
 /*                                                                           */

@@ -196,3 +196,23 @@ def test_moe_entry_points_reject_invalid_arguments(lib):
     bad = list(args)
     bad[13] = FAKE + 8
     assert c(*bad) == L.DF_ERR_ALIGN
+
+
+def test_grouped_proj_batched_rejects_invalid_arguments(lib):
+    f = lib.dualflow_grouped_proj_batched
+    ok = [FAKE, 0, 0, 64, 64, FAKE, 1024, 512, 0, FAKE, 0, 0, 4, 0, FAKE, 1 << 30,
+          None, 0, 0, 0, 1, 0, None, None]
+
+    def call(**over):
+        a = list(ok)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return f(*a)
+
+    assert call(a0=None) == L.DF_ERR_NULL
+    assert call(a12=0) == L.DF_ERR_SHAPE                    # batch
+    assert call(a13=2) == L.DF_ERR_UNSUPPORTED              # residual epilogue
+    assert call(a2=100) == L.DF_ERR_SHAPE                   # x batch stride below M * K
+    assert call(a8=1024 * 512 + 4) == L.DF_ERR_ALIGN        # w batch stride not 16-byte
+    nl = lib.dualflow_grouped_proj_batched_num_launches
+    assert nl(128, 1024, 512, 2, 4) == 0 and nl(0, 1024, 512, 0, 4) == 0

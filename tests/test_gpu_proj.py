@@ -200,3 +200,30 @@ def test_next_projection_hint_changes_no_bit(cuda_device, cur, nxt):
     assert int(err.item()) == 0
     assert torch.equal(y_plain.view(torch.int16), y_hint.view(torch.int16))
     assert torch.equal(yn_plain.view(torch.int16), yn_hint.view(torch.int16))
+
+
+@pytest.mark.parametrize("batch,mp,ma,N,K,epi", [(3, 64, 64, 1024, 512, "swiglu"),
+                                                 (8, 64, 64, 2048, 5632, "none"),
+                                                 (8, 64, 64, 11264, 2048, "swiglu"),
+                                                 (2, 5, 3, 256, 128, "none")])
+def test_batched_projection_parity(cuda_device, batch, mp, ma, N, K, epi):
+    """One launch for a batch of same-shape projections (the MoE experts):
+    every entry matches the oracle, on sampled columns at the larger shapes."""
+    g = torch.Generator().manual_seed(batch * 1000 + N)
+    x = _rand(g, (batch, mp + ma, K))
+    w = _rand(g, (batch, N, K), 0.02)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    y = api.grouped_proj_batched(x.to(cuda_device), mp, w.to(cuda_device), epilogue=epi,
+                                 err_flag=err).cpu()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    n_out = N // 2 if epi == "swiglu" else N
+    cols = np.unique(np.concatenate([np.arange(0, min(48, n_out)),
+                                     np.arange(max(0, n_out - 48), n_out),
+                                     np.random.default_rng(2).integers(0, n_out, 128)]))
+    for b in range(batch):
+        if epi == "swiglu":
+            ref = _oracle(x[b], torch.cat([w[b][cols], w[b][n_out + cols]]), mp, "swiglu", None, None)
+        else:
+            ref = _oracle(x[b], w[b][cols], mp, "none", None, None)
+        assert_close(y[b][:, cols], ref, "bf16", "batched entry %d" % b)
