@@ -28,6 +28,7 @@ constexpr int kRows = 64;      // rows per flow in an expert block (max tokens p
 constexpr int kMaxK = 8;       // max experts per token
 constexpr int kMaxE = 256;     // max experts
 constexpr int kThreads = 256;
+constexpr int kCopySplit = 16;  // CTAs per expert in the dispatch copy
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ routing
@@ -57,7 +58,8 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const RouteParams p) {
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(f) * p.B + t) * p.ldx);
     const uint4* wr = reinterpret_cast<const uint4*>(p.w + static_cast<int64_t>(e) * p.d);
     float acc = 0.f;
-    for (int v = lane; v < nvec; v += 32) {
+#pragma unroll 8
+    for (int v = lane; v < nvec; v += 32) {  // loads of 8 iterations in flight
       const uint4 a = xr[v], b = wr[v];
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -128,15 +130,17 @@ struct DispatchParams {
   int32_t* err;
 };
 
-// One CTA per expert: the tokens routed to it in token order (ballot prefix
-// over the <= 64 tokens), their row slots, and the copy of their rows into
-// the expert's block. Rows past the counts are left as they were: every
-// output row of the projections depends only on its own input row, and the
-// combine reads only the rows listed in the slots.
+// kCopySplit CTAs per expert: each finds the tokens routed to it in token
+// order (ballot prefix over the <= 64 tokens) and copies its share of their
+// rows into the expert's block; the first also writes the row slots and
+// counts. Rows past the counts are left as they were: every output row of the
+// projections depends only on its own input row, and the combine reads only
+// the rows listed in the slots.
 __global__ void __launch_bounds__(kThreads) dispatch_kernel(const DispatchParams p) {
   __shared__ int rows1[kRows], rows2[kRows];
   __shared__ int n_s[2];
   const int e = blockIdx.x;
+  const bool writer = blockIdx.y == 0;
   const int tid = threadIdx.x;
   pdl_wait();
   pdl_trigger();
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(const DispatchParams
       for (int j = 0; j < p.k_aux; ++j) {
         const int id = p.ids[static_cast<int64_t>(t) * p.k_aux + j];
         if (id < 0 || id >= p.E) {
-          set_err(p.err, DF_DEVERR_BLOCK);
+          if (writer) set_err(p.err, DF_DEVERR_BLOCK);
           continue;
         }
         if (id == e) {
@@ -170,12 +174,12 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(const DispatchParams
     if (j1 >= 0) {
       const int row = base1 + __popc(m1 & below);
       rows1[row] = t;
-      p.slot1[static_cast<int64_t>(t) * p.k + j1] = row;
+      if (writer) p.slot1[static_cast<int64_t>(t) * p.k + j1] = row;
     }
     if (j2 >= 0) {
       const int row = base2 + __popc(m2 & below);
       rows2[row] = t;
-      p.slot2[static_cast<int64_t>(t) * p.k_aux + j2] = kRows + row;
+      if (writer) p.slot2[static_cast<int64_t>(t) * p.k_aux + j2] = kRows + row;
     }
     if (t == 0) {
       n_s[0] = c1[0] + c1[1];
@@ -184,13 +188,16 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(const DispatchParams
   }
   __syncthreads();
   const int n1 = n_s[0], n2 = n_s[1];
-  if (tid == 0 && p.counts) {
+  if (tid == 0 && writer && p.counts) {
     p.counts[2 * e] = n1;
     p.counts[2 * e + 1] = n2;
   }
   const int nvec = p.d / 8;
   uint4* dst = reinterpret_cast<uint4*>(p.xe + static_cast<int64_t>(e) * 2 * kRows * p.d);
-  for (int i = tid; i < (n1 + n2) * nvec; i += kThreads) {
+  const int total = (n1 + n2) * nvec;
+  const int per = (total + gridDim.y - 1) / gridDim.y;
+  const int i0 = blockIdx.y * per, i1 = min(total, i0 + per);
+  for (int i = i0 + tid; i < i1; i += kThreads) {
     const int rr = i / nvec, v = i % nvec;
     const bool aux = rr >= n1;
     const int row = aux ? kRows + (rr - n1) : rr;
@@ -316,7 +323,7 @@ extern "C" df_status dualflow_moe_dispatch(const void* x, int64_t ldx, int B, in
   if (lx % 8 != 0 || !aligned(x, 16) || !aligned(xe, 16)) return DF_ERR_ALIGN;
   moe::DispatchParams p{static_cast<const __nv_bfloat16*>(x), lx, B, d, E, k, k_aux, ids,
                         static_cast<__nv_bfloat16*>(xe), slot1, slot2, counts, err_flag};
-  if (launch_pdl(moe::dispatch_kernel, dim3(E), dim3(moe::kThreads), 0,
+  if (launch_pdl(moe::dispatch_kernel, dim3(E, moe::kCopySplit), dim3(moe::kThreads), 0,
                  static_cast<cudaStream_t>(stream), p) != cudaSuccess)
     return DF_ERR_CUDA;
   return DF_OK;
