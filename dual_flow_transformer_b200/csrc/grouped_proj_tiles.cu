@@ -54,6 +54,8 @@ struct Params {
   int kblocks, BN, half, out_per_tile, n_tiles, C, stages, stage_bytes;
   int tpb;            // tiles per batch entry: tile t is (batch t / tpb, column tile t % tpb)
   int64_t ystride_b;  // output batch stride (elements)
+  int batched;        // X / W tensor maps are 3-D (batch > 1); 2-D otherwise
+  int pf_batched;     // the next projection's W map is 3-D
   uint32_t idesc;
   int F;
   __nv_bfloat16* y;
@@ -394,13 +396,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_w = [&](int s, int t, int kb) {
         const int e = t / p.tpb, tn = t - e * p.tpb;
         uint8_t* sb = smem + s * p.stage_bytes + kTileX;
-        if (p.epilogue == DF_EPI_SWIGLU) {
-          tma_load_3d_hint(sb, &tmW, &full[s], kb * kBK, tn * p.half, e, pol_w);
-          tma_load_3d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, p.F + tn * p.half, e,
-                           pol_w);
+        const int r0 = p.epilogue == DF_EPI_SWIGLU ? tn * p.half : tn * p.BN;
+        const int r1 = p.F + tn * p.half;
+        if (p.batched) {
+          tma_load_3d_hint(sb, &tmW, &full[s], kb * kBK, r0, e, pol_w);
+          if (p.epilogue == DF_EPI_SWIGLU)
+            tma_load_3d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, r1, e, pol_w);
         } else {
-          tma_load_3d_hint(sb, &tmW, &full[s], kb * kBK, tn * p.BN, e, pol_w);
+          tma_load_2d_hint(sb, &tmW, &full[s], kb * kBK, r0, pol_w);
+          if (p.epilogue == DF_EPI_SWIGLU)
+            tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, r1, pol_w);
         }
+      };
+      auto load_x = [&](uint8_t* sa, int s, int t, int kb) {
+        if (p.batched)
+          tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
+        else
+          tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
       };
       // The weights are no product of the previous kernel: the first ring
       // stages start streaming them before the wait for it.
@@ -419,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = static_cast<int>(n % S);
           uint8_t* sa = smem + s * p.stage_bytes;
           if (n < pre) {  // weights already on their way
-            tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
+            load_x(sa, s, t, kb);
             continue;
           }
           if (n >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / S) - 1) & 1))) {
@@ -428,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], p.stage_bytes);
-          tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
+          load_x(sa, s, t, kb);
           load_w(s, t, kb);
         }
       }
@@ -449,12 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (t >= p.pf_ntiles) continue;
           const int e = t / p.pf_tpb, tn = t - e * p.pf_tpb;
+          const int r0 = p.pf_half > 0 ? tn * p.pf_half : tn * p.pf_BN;
+          const int r1 = p.pf_F + tn * p.pf_half;
           for (int kb = k0; kb < k1 && kb < k0 + p.pf_stages; ++kb) {
-            if (p.pf_half > 0) {
-              tma_prefetch_3d(&tmWn, kb * kBK, tn * p.pf_half, e);
-              tma_prefetch_3d(&tmWn, kb * kBK, p.pf_F + tn * p.pf_half, e);
+            if (p.pf_batched) {
+              tma_prefetch_3d(&tmWn, kb * kBK, r0, e);
+              if (p.pf_half > 0) tma_prefetch_3d(&tmWn, kb * kBK, r1, e);
             } else {
-              tma_prefetch_3d(&tmWn, kb * kBK, tn * p.pf_BN, e);
+              tma_prefetch_2d(&tmWn, kb * kBK, r0);
+              if (p.pf_half > 0) tma_prefetch_2d(&tmWn, kb * kBK, r1);
             }
           }
         }
@@ -816,11 +831,17 @@ int launch_if_better(const Request& r) {
     const int box_rows = nx_swiglu ? nx.BN / 2 : nx.BN;
     const int64_t wn_stride =
         r.w_next_bstride > 0 ? r.w_next_bstride : static_cast<int64_t>(r.N_next) * r.K_next;
-    if (nx_tiles &&
-        encode_tmap_bf16_3d(&tmWn, r.w_next, static_cast<uint64_t>(nb),
-                            static_cast<uint64_t>(r.N_next), static_cast<uint64_t>(r.K_next),
-                            static_cast<uint64_t>(r.K_next) * 2,
-                            static_cast<uint64_t>(wn_stride) * 2, box_rows, kBK)) {
+    const bool nx_map =
+        nb > 1 ? encode_tmap_bf16_3d(&tmWn, r.w_next, static_cast<uint64_t>(nb),
+                                     static_cast<uint64_t>(r.N_next),
+                                     static_cast<uint64_t>(r.K_next),
+                                     static_cast<uint64_t>(r.K_next) * 2,
+                                     static_cast<uint64_t>(wn_stride) * 2, box_rows, kBK)
+               : encode_tmap_bf16_2d(&tmWn, r.w_next, static_cast<uint64_t>(r.N_next),
+                                     static_cast<uint64_t>(r.K_next),
+                                     static_cast<uint64_t>(r.K_next) * 2, box_rows, kBK);
+    if (nx_tiles && nx_map) {
+      p.pf_batched = nb > 1 ? 1 : 0;
       // ~28 MB in all: what DRAM delivers in a few microseconds of tail
       const double per_stage = static_cast<double>(nx.ctas) * nx.BN * kBK * 2;
       int st = static_cast<int>(28.0 * 1024 * 1024 / per_stage);
@@ -838,13 +859,25 @@ int launch_if_better(const Request& r) {
   CUtensorMap tmX, tmW;
   const int64_t xs = r.x_bstride > 0 ? r.x_bstride : static_cast<int64_t>(M) * r.ldx;
   const int64_t wsd = r.w_bstride > 0 ? r.w_bstride : static_cast<int64_t>(r.N) * r.K;
-  if (!encode_tmap_bf16_3d(&tmX, r.x, static_cast<uint64_t>(batch), static_cast<uint64_t>(M),
-                           static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.ldx) * 2,
-                           static_cast<uint64_t>(xs) * 2, kBM, kBK) ||
-      !encode_tmap_bf16_3d(&tmW, r.w, static_cast<uint64_t>(batch), static_cast<uint64_t>(r.N),
-                           static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.K) * 2,
-                           static_cast<uint64_t>(wsd) * 2, swiglu ? pl.BN / 2 : pl.BN, kBK))
-    return -1;
+  // batch 1 keeps 2-D maps and loads (measured faster than a 3-D map whose
+  // third dimension is 1)
+  p.batched = batch > 1 ? 1 : 0;
+  const uint32_t wbox = swiglu ? pl.BN / 2 : pl.BN;
+  const bool maps_ok =
+      batch > 1
+          ? encode_tmap_bf16_3d(&tmX, r.x, static_cast<uint64_t>(batch), static_cast<uint64_t>(M),
+                                static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.ldx) * 2,
+                                static_cast<uint64_t>(xs) * 2, kBM, kBK) &&
+                encode_tmap_bf16_3d(&tmW, r.w, static_cast<uint64_t>(batch),
+                                    static_cast<uint64_t>(r.N), static_cast<uint64_t>(r.K),
+                                    static_cast<uint64_t>(r.K) * 2,
+                                    static_cast<uint64_t>(wsd) * 2, wbox, kBK)
+          : encode_tmap_bf16_2d(&tmX, r.x, static_cast<uint64_t>(M), static_cast<uint64_t>(r.K),
+                                static_cast<uint64_t>(r.ldx) * 2, kBM, kBK) &&
+                encode_tmap_bf16_2d(&tmW, r.w, static_cast<uint64_t>(r.N),
+                                    static_cast<uint64_t>(r.K), static_cast<uint64_t>(r.K) * 2,
+                                    wbox, kBK);
+  if (!maps_ok) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.ctas);
   cfg.blockDim = dim3(kThreads);
