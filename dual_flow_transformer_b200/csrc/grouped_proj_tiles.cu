@@ -393,8 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmW);
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      auto load_w = [&](int s, int t, int kb) {
-        const int e = t / p.tpb, tn = t - e * p.tpb;
+      // (e, tn) = (batch entry, column tile) of tile t, split once per tile:
+      // nothing on the per-stage issue path divides (the ring is only a few
+      // DRAM round trips deep, so issue latency costs bandwidth)
+      auto load_w = [&](int s, int e, int tn, int kb) {
         uint8_t* sb = smem + s * p.stage_bytes + kTileX;
         const int r0 = p.epilogue == DF_EPI_SWIGLU ? tn * p.half : tn * p.BN;
         const int r1 = p.F + tn * p.half;
@@ -408,40 +410,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d_hint(sb + p.half * 128, &tmW, &full[s], kb * kBK, r1, pol_w);
         }
       };
-      auto load_x = [&](uint8_t* sa, int s, int t, int kb) {
+      auto load_x = [&](uint8_t* sa, int s, int e, int kb) {
         if (p.batched)
-          tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, t / p.tpb, pol_x);
+          tma_load_3d_hint(sa, &tmX, &full[s], kb * kBK, 0, e, pol_x);
         else
           tma_load_2d_hint(sa, &tmX, &full[s], kb * kBK, 0, pol_x);
       };
       // The weights are no product of the previous kernel: the first ring
       // stages start streaming them before the wait for it.
       long long pre = 0;
-      for (int t = tile_first; t < p.n_tiles && pre < S; t += tile_stride)
+      for (int t = tile_first; t < p.n_tiles && pre < S; t += tile_stride) {
+        const int e = t / p.tpb, tn = t - e * p.tpb;
         for (int kb = kb0; kb < kb1 && pre < S; ++kb, ++pre) {
           mbar_arrive_expect_tx(&full[pre], p.stage_bytes);
-          load_w(static_cast<int>(pre), t, kb);
+          load_w(static_cast<int>(pre), e, tn, kb);
         }
+      }
       pdl_wait();
       pdl_trigger();
       long long n = 0;
+      int s = 0;         // n % S
+      uint32_t ph = 0;   // (n / S) & 1
       bool ok = true;
       for (int t = tile_first; t < p.n_tiles && ok; t += tile_stride) {
+        const int e = t / p.tpb, tn = t - e * p.tpb;
         for (int kb = kb0; kb < kb1; ++kb, ++n) {
-          const int s = static_cast<int>(n % S);
           uint8_t* sa = smem + s * p.stage_bytes;
           if (n < pre) {  // weights already on their way
-            load_x(sa, s, t, kb);
-            continue;
+            load_x(sa, s, e, kb);
+          } else {
+            if (n >= S && !mbar_wait(&empty[s], ph ^ 1u)) {
+              set_err(p.err, DF_DEVERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], p.stage_bytes);
+            load_x(sa, s, e, kb);
+            load_w(s, e, tn, kb);
           }
-          if (n >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((n / S) - 1) & 1))) {
-            set_err(p.err, DF_DEVERR_TIMEOUT);
-            ok = false;
-            break;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
           }
-          mbar_arrive_expect_tx(&full[s], p.stage_bytes);
-          load_x(sa, s, t, kb);
-          load_w(s, t, kb);
         }
       }
       for (long long i = (n > S ? n - S : 0); i < n; ++i)
@@ -479,6 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       long long n = 0;
+      int ms = 0;        // n % S
+      uint32_t mph = 0;  // (n / S) & 1
       int seg = 0;
       bool ok = true;
       for (int t = tile_first; t < p.n_tiles && ok; t += tile_stride, ++seg) {
@@ -490,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * p.BN;
         for (int kb = kb0; kb < kb1; ++kb, ++n) {
-          const int s = static_cast<int>(n % S);
-          if (!mbar_wait(&full[s], static_cast<uint32_t>((n / S) & 1))) {
+          const int s = ms;  // n % S and (n / S) & 1, kept as counters
+          if (!mbar_wait(&full[s], mph)) {
             set_err(p.err, DF_DEVERR_TIMEOUT);
             ok = false;
             break;
@@ -505,6 +517,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
+          if (++ms == S) {
+            ms = 0;
+            mph ^= 1u;
+          }
         }
         if (!ok) break;
         umma_commit(&acc_full[acc]);
