@@ -13,6 +13,7 @@ from .dualflow_oracle import (  # noqa: F401
     attn_weights,
     decode_attn,
     kv_append,
+    prefill,
     grouped_proj,
     silu,
     swiglu_couple,

@@ -24,6 +24,10 @@ of the function that takes it:
   The general formula is a reading: PARITY UNPINNED against the pages.
 * MLP coupling    h2 += b ⊙ h1 ;  m2 += c ⊙ m1  (same additive form).
   PARITY UNPINNED against the pages beyond the b = c = 0 reduction.
+* Prefill         the primary flow's causal attention over the prompt,
+  writing the cache; the auxiliary query only at the last prompt position.
+  Both are the pages' statements; the chunked form (a cache that already
+  holds a prefix) is the plain extension of the causal mask.
 * Layer step      pre-attention and pre-MLP RMSNorm (unit gain, eps 1e-5),
   residual adds, SwiGLU MLP, no positional rotation.
   PARITY UNPINNED against the pages (the pages name no norm, no MLP form).
@@ -197,6 +201,97 @@ def kv_append(k_new, v_new, k_cache, v_cache, block_table, positions, block_size
         kc[page, :, p % block_size, :] = k_new[b]
         vc[page, :, p % block_size, :] = v_new[b]
     return kc, vc
+
+
+def prefill(q1, k_new, v_new, k_cache, v_cache, block_table, cu_seqlens, ctx_lens=None,
+            q2raw=None, a=None, scale=None, block_size=None):
+    """Prompt processing of the primary flow, then the auxiliary query at the
+    last prompt position.
+
+    Page "Sintesi Tecnica: Dual-Flow Transformers", section "Architettura
+    Core": the primary flow is a standard causal Transformer that processes
+    the whole prompt and writes the persistent KV cache; the auxiliary flow is
+    skipped while the prompt is processed and switched on only at the last
+    prompt position (to predict the first continuation token). Section
+    "Costi di Inferenza vs. Addestramento": prefill costs what a standard
+    Transformer's does. The page "プライマリパスとデコード処理を分離する
+    Dual-Flow Transformers", section "提案手法の詳細", says the same (the auxiliary
+    flow is skipped during prompt processing and starts at the final position).
+
+    Sequence b holds the prompt tokens t in [cu_seqlens[b], cu_seqlens[b+1]);
+    its cache already holds ctx_lens[b] tokens (0 for a fresh prompt), so
+    token i of the chunk sits at position p = ctx_lens[b] + i. Steps:
+
+    1. append: the chunk's K1/V1 rows go to positions ctx_lens[b] + i of the
+       paged cache (the ``kv_append`` rule, one position per token);
+    2. primary attention, causal: the query at position p attends to cache
+       positions j <= p,
+           O1[t, h] = softmax_j(scale * q1[t, h] . k_j) V, j in [0, p];
+    3. auxiliary query at the last position P = ctx_lens[b] + n_b - 1 only,
+       coupled to that position's primary query (``couple_query``) and
+       attending to positions j <= P of the same cache:
+           O2[b, h] = softmax_j(scale * q2[b, h] . k_j) V.
+
+    q1 [T, Hq, D]; k_new, v_new [T, Hkv, D]; q2raw [B, Hq, D] or None;
+    a [Hq, D] or None; caches [num_blocks, Hkv, bs, D]; block_table
+    [B, max_blocks]; cu_seqlens [B + 1] with every chunk non-empty.
+    Returns (o1 float64 [T, Hq, D], o2 float64 [B, Hq, D] or None,
+    k_cache, v_cache) -- the caches as new arrays of the input dtype.
+    """
+    q1 = np.asarray(q1, dtype=F64)
+    T, Hq, D = q1.shape
+    Hkv = k_cache.shape[1]
+    if block_size is None:
+        block_size = k_cache.shape[2]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cu = [int(x) for x in cu_seqlens]
+    B = len(cu) - 1
+    ctx = [0] * B if ctx_lens is None else [int(x) for x in ctx_lens]
+    if cu[0] != 0 or cu[-1] != T or any(cu[b + 1] - cu[b] < 1 for b in range(B)):
+        raise ValueError("cu_seqlens must split the T tokens into non-empty chunks")
+
+    # 1. primary-only cache write, one position per prompt token (the
+    #    ``kv_append`` rule: page table[b][p // bs], slot p % bs, all KV heads)
+    kc = np.array(k_cache, copy=True)
+    vc = np.array(v_cache, copy=True)
+    table = np.asarray(block_table)
+    for b in range(B):
+        for i in range(cu[b + 1] - cu[b]):
+            t, p = cu[b] + i, ctx[b] + i
+            page = int(table[b][p // block_size])
+            kc[page, :, p % block_size, :] = k_new[t]
+            vc[page, :, p % block_size, :] = v_new[t]
+
+    o1 = np.zeros((T, Hq, D), dtype=F64)
+    o2 = None if q2raw is None else np.zeros((B, Hq, D), dtype=F64)
+    for b in range(B):
+        n = cu[b + 1] - cu[b]
+        L = ctx[b] + n
+        pos = ctx[b] + np.arange(n)                      # position of each query row
+        keep = np.arange(L)[None, :] <= pos[:, None]     # causal mask [n, L]
+        last = cu[b + 1] - 1
+        for g in range(Hkv):
+            K = gather_kv(kc, block_table, b, g, L, block_size)
+            V = gather_kv(vc, block_table, b, g, L, block_size)
+            for h in range(g * G, (g + 1) * G):
+                # 2. masked softmax over keys j <= p for every query row
+                s = scale * (q1[cu[b]:cu[b + 1], h, :] @ K.T)
+                s = np.where(keep, s, -np.inf)
+                s = s - s.max(axis=1, keepdims=True)
+                e = np.exp(s)
+                o1[cu[b]:cu[b + 1], h, :] = (e / e.sum(axis=1, keepdims=True)) @ V
+            if q2raw is not None:
+                # 3. auxiliary query of the last prompt position, every key
+                heads = slice(g * G, (g + 1) * G)
+                q2 = couple_query(q1[last:last + 1, heads, :],
+                                  np.asarray(q2raw, dtype=F64)[b:b + 1, heads, :],
+                                  None if a is None else np.asarray(a, dtype=F64)[heads])
+                o2[b, heads] = attn_weights(q2[0], K, scale) @ V
+    return o1, o2, kc, vc
 
 
 def grouped_proj(x, w, m_primary, n_aux=None):

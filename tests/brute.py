@@ -52,3 +52,13 @@ def dual_decode(q1, q2raw, a, kc, vc, table, seqlens, block_size, Hq, Hkv):
 def matmul_nt(x, w):
     """x [M][K], w [N][K] -> x w^T as nested lists."""
     return [[math.fsum(xi * wi for xi, wi in zip(row, wrow)) for wrow in w] for row in x]
+
+
+def causal_prefill(q_rows, keys, values, ctx, scale):
+    """q_rows: list[n][D] queries of positions ctx .. ctx+n-1; keys, values:
+    list[ctx+n][D] in position order. Row i attends to keys 0..ctx+i."""
+    out = []
+    for i, q in enumerate(q_rows):
+        stop = ctx + i + 1
+        out.append(softmax_attention(q, keys[:stop], values[:stop], scale))
+    return out
