@@ -39,8 +39,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "dual-flow decode tokens/s and KV-read GB/s (% of B200 HBM peak), 1 GPU"
+PREFILL_METRIC = ("primary prefill prompt tokens/s (one layer's causal attention, cache write "
+                  "and last-position auxiliary query), 1 GPU")
 FALLBACK_HBM_GBS = 6650.0
-ATTN_SRC = os.path.join(ROOT, "dual_flow_transformer_b200", "csrc", "decode_attn.cu")
+FALLBACK_BF16_TFLOPS = 1590.0
+CSRC = os.path.join(ROOT, "dual_flow_transformer_b200", "csrc")
+ATTN_SRC = os.path.join(CSRC, "decode_attn.cu")
 
 
 def parse_args(argv=None):
@@ -50,7 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload",
-                    choices=["layer", "mha", "gqa", "long", "tiny", "mixture", "moe"],
+                    choices=["layer", "mha", "gqa", "long", "tiny", "mixture", "moe",
+                             "prefill"],
                     default="layer")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -73,13 +78,26 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_from_profile(workload):
-    """DRAM bytes per attention launch from the committed ncu summary, or None
-    when there is none or the kernel source changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", "decode_attn_%s.md" % workload)
+def measured_tensor_peak():
+    """Dense bf16 tensor-core peak: the burst cuBLAS figure (a kernel timed on
+    its own), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["bf16_tflops"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def traffic_from_profile(workload, prefix="decode_attn", src=ATTN_SRC):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when there is none or the kernel source changed since it
+    was captured."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (prefix, workload))
     if not os.path.exists(path):
         return None
-    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in open(path):
         if line.startswith("- ") and ":" in line:
@@ -509,6 +527,106 @@ class MoERun:
         return int(self.err.item())
 
 
+class PrefillRun:
+    """Primary prefill of fresh prompts: cache write, causal attention of the
+    primary queries, auxiliary query at each last prompt position (one
+    dualflow_prefill call = 4 kernels)."""
+
+    timer_keys = ("attn",)
+    dominant_key = "attn"
+    roof_bound = "tensor"
+    metric = PREFILL_METRIC
+    profile_prefix = "prefill_attn"
+    profile_src = os.path.join(CSRC, "prefill.cu")
+
+    def __init__(self, args, dev, seed):
+        import torch
+        from dual_flow_transformer_b200 import api, synth
+        w = synth.WORKLOADS["prefill"]
+        self.w = w
+        self.api = api
+        self.host = synth.make_prefill_inputs(w, seed=seed)
+        h = self.host
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in h.items()}
+        self.d = d
+        self.ws = api.new_prefill_workspace(h["B"], w.Hq, w.Hkv, w.D, h["max_seqlen"], dev)
+        self.o1 = torch.empty_like(d["q1"])
+        self.o2 = torch.empty_like(d["q2raw"])
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        lens = (h["cu_seqlens"][1:] - h["cu_seqlens"][:-1]).tolist()
+        ctx = h["ctx_lens"].tolist()
+        pairs = sum(n * c + n * (n + 1) // 2 for n, c in zip(lens, ctx))
+        self.tokens_per_step = h["T"]
+        self.launches_per_step = api.prefill_num_launches(True, True)
+        self.units = w.Hq * pairs                  # (query row, visible key) pairs, all heads
+        self.flops_per_unit = 4 * w.D              # q.k and p*v, multiply-add each
+        self.dom_flops = self.units * self.flops_per_unit
+        self.config = {"workload": "dual-flow primary prefill: %d fresh prompts of %d..%d tokens, "
+                                   "%d/%d heads, head_dim %d, bf16, 64-token pages in a random "
+                                   "block table, auxiliary query at each last position"
+                                   % (h["B"], w.len_lo, w.len_hi, w.Hq, w.Hkv, w.D),
+                       "l2": "inputs larger than L2 (%.0f MB of queries, %.0f MB of new K/V)"
+                             % (h["q1"].numel() * 2 / 1e6, 2 * h["k_new"].numel() * 2 / 1e6)}
+        self.dominant = "dualflow_prefill attention kernel (mma.sync, TMA page ring)"
+        self._full()
+        torch.cuda.synchronize()
+        self.g_full, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_full):
+            self._full()
+        with torch.cuda.graph(self.g_attn):
+            self._attn_only()
+        torch.cuda.synchronize()
+
+    def _call(self, append, aux):
+        d = self.d
+        self.api.prefill(d["q1"], d["k_new"] if append else None, d["v_new"] if append else None,
+                         d["k_cache"], d["v_cache"], d["block_table"], d["cu_seqlens"],
+                         d["max_q_len"], d["max_seqlen"], ctx_lens=d["ctx_lens"],
+                         q2raw=d["q2raw"] if aux else None, a=d["a"] if aux else None,
+                         o1=self.o1, o2=self.o2 if aux else None, workspace=self.ws,
+                         err_flag=self.err)
+
+    def _full(self):
+        self._call(True, True)
+
+    def _attn_only(self):
+        self._call(False, False)   # one launch: the attention kernel alone
+
+    def step(self, timers=None):
+        if timers is None:
+            self.g_full.replay()
+            return
+        timers["attn"][0].record()
+        self.g_attn.replay()
+        timers["attn"][1].record()
+
+    def host_io(self):
+        import torch
+        h = self.host
+        parts = [h["q1"], h["k_new"], h["v_new"], h["q2raw"]]
+        n = sum(p.numel() for p in parts)
+        x = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+        off = 0
+        self._views = []
+        for p in parts:
+            v = x[off:off + p.numel()].view(p.shape)
+            v.copy_(p)
+            self._views.append(v)
+            off += p.numel()
+        o = torch.empty(tuple(self.o1.shape), dtype=torch.bfloat16).pin_memory()
+        return x, o
+
+    def step_host(self, x_host, o_host):
+        d = self.d
+        for dst, src in zip((d["q1"], d["k_new"], d["v_new"], d["q2raw"]), self._views):
+            dst.copy_(src, non_blocking=True)
+        self.step()
+        o_host.copy_(self.o1, non_blocking=True)
+
+    def check_err(self):
+        return int(self.err.item())
+
+
 # ----------------------------------------------------------------------------- oracle timing
 
 def _threads_used():
@@ -575,6 +693,8 @@ def time_oracle(run, workload, budget_s, max_steps=None):
         return time_oracle_mixture(run.host, budget_s)
     if workload == "moe":
         return time_oracle_moe(run.host, budget_s)
+    if workload == "prefill":
+        return time_oracle_prefill(run.host, budget_s)
     B = run.w.B
     sel, el, k = [], 0.0, 0
     inp_all = None
@@ -646,6 +766,49 @@ def time_oracle_moe(host, budget_s, tokens_per_call=4):
     return k / el, sample, el, k
 
 
+def oracle_prefill_group(host, b, g):
+    """Oracle inputs for KV head g of sequence b of a prefill workload: the
+    query heads of that group, that head's new K/V and cached pages (input
+    selection and dtype widening only, no arithmetic)."""
+    import numpy as np
+    import torch
+    f = lambda t: t.to(torch.float32).numpy()
+    Hq, Hkv = host["Hq"], host["Hkv"]
+    G = Hq // Hkv
+    cu = host["cu_seqlens"].tolist()
+    t0, t1 = cu[b], cu[b + 1]
+    row = [int(p) for p in host["block_table"][b].tolist() if p >= 0]
+    heads = slice(g * G, (g + 1) * G)
+    return dict(q1=f(host["q1"][t0:t1, heads]), k_new=f(host["k_new"][t0:t1, g:g + 1]),
+                v_new=f(host["v_new"][t0:t1, g:g + 1]),
+                k_cache=f(host["k_cache"][row][:, g:g + 1]),
+                v_cache=f(host["v_cache"][row][:, g:g + 1]),
+                block_table=np.arange(len(row))[None, :], cu_seqlens=np.array([0, t1 - t0]),
+                ctx_lens=host["ctx_lens"][b:b + 1].numpy(), q2raw=f(host["q2raw"][b:b + 1, heads]),
+                a=f(host["a"][heads]))
+
+
+def time_oracle_prefill(host, budget_s):
+    """The oracle prefill, one (sequence, KV head) group per call: 1/Hkv of
+    the work of that sequence's prompt tokens, counted as such."""
+    import oracle
+    Hkv = host["Hkv"]
+    cu = host["cu_seqlens"].tolist()
+    el, tokens, calls = 0.0, 0.0, 0
+    while el < budget_s and calls < 64:
+        b, g = (calls // Hkv) % host["B"], calls % Hkv
+        inp = oracle_prefill_group(host, b, g)
+        t0 = time.perf_counter()
+        oracle.prefill(**inp)
+        el += time.perf_counter() - t0
+        tokens += (cu[b + 1] - cu[b]) / Hkv
+        calls += 1
+    sample = ("fp64 oracle prefill (cache write, causal attention, last-position auxiliary "
+              "query) on %d (sequence, KV head) group(s) of %d query heads, each counted as 1/%d "
+              "of its sequence's prompt tokens" % (calls, host["Hq"] // Hkv, Hkv))
+    return tokens / el, sample, el, calls
+
+
 # ----------------------------------------------------------------------------- main
 
 def run_reference(args):
@@ -660,15 +823,20 @@ def run_reference(args):
         pass
 
     h = Host()
-    if args.workload in ("mixture", "moe"):
+    if args.workload in ("mixture", "moe", "prefill"):
         h.w = synth.WORKLOADS[args.workload]
         if args.workload == "mixture":
             h.host = synth.make_mixture_inputs(h.w)
             v, sample, el, steps = time_oracle_mixture(h.host, 20.0)
+        elif args.workload == "prefill":
+            h.host = synth.make_prefill_inputs(h.w)
+            v, sample, el, steps = time_oracle_prefill(h.host, 20.0)
         else:
             h.host = synth.make_moe_inputs(h.w)
             v, sample, el, steps = time_oracle_moe(h.host, 20.0)
-        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        line = {"impl": "reference",
+                "metric": PREFILL_METRIC if args.workload == "prefill" else METRIC,
+                "value": v, "unit": "tokens/s",
                 "n_gpus": world, "steps": steps, "steps_requested": args.steps,
                 "warmup": args.warmup, "ms_per_step": el / steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -752,6 +920,8 @@ def main(argv=None):
         run = MixtureRun(args, dev, seed)
     elif args.workload == "moe":
         run = MoERun(args, dev, seed)
+    elif args.workload == "prefill":
+        run = PrefillRun(args, dev, seed)
     else:
         run = AttnRun(args, dev, seed, args.workload)
 
@@ -826,12 +996,33 @@ def main(argv=None):
             import torch.distributed as dist
             dist.destroy_process_group()
         return 0
-    peak, peak_kind = measured_hbm_peak()
-    dom_bytes = getattr(run, "dom_bytes", None) or run.attn_bytes
-    achieved = dom_bytes / (attn_ms / 1e3) / 1e9
     value = world * run.tokens_per_step * args.steps / (ms_max / 1e3)
+    if getattr(run, "roof_bound", "hbm") == "tensor":
+        peak, peak_kind = measured_tensor_peak()
+        achieved = run.dom_flops / (attn_ms / 1e3) / 1e12
+        roofline = {"kernel": run.dominant, "bound": "tensor", "achieved": achieved,
+                    "peak": peak, "peak_kind": peak_kind + " (cuBLAS bf16 GEMM, burst, "
+                    "MEASURED_PEAKS.json)" if peak_kind == "measured" else peak_kind,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": traffic_from_profile(args.workload, run.profile_prefix,
+                                                    run.profile_src),
+                    "algorithmic_flops_per_launch": run.dom_flops,
+                    "units_per_launch": run.units, "flops_per_unit": run.flops_per_unit}
+        peak, peak_kind = measured_hbm_peak()
+    else:
+        peak, peak_kind = measured_hbm_peak()
+        dom_bytes = getattr(run, "dom_bytes", None) or run.attn_bytes
+        achieved = dom_bytes / (attn_ms / 1e3) / 1e9
+        roofline = {"kernel": run.dominant, "bound": "hbm", "achieved": achieved,
+                    "peak": peak, "peak_kind": peak_kind + " (STREAM-style copy, "
+                    "MEASURED_PEAKS.json)" if peak_kind == "measured" else peak_kind,
+                    "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": traffic_from_profile(args.workload),
+                    "algorithmic_bytes_per_launch": dom_bytes,
+                    "units_per_launch": run.units, "bytes_per_unit": run.bytes_per_unit}
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": getattr(run, "metric", METRIC), "value": value, "unit": "tokens/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations/cache, N(0,0.02) weights, N(0,0.1) couplings)",
@@ -840,12 +1031,7 @@ def main(argv=None):
         "kernel_timing": "second pass of the same %d steps, the timed kernels' graphs bracketed "
                          "by CUDA events on the launching stream (value uses the single-graph "
                          "step)" % args.steps,
-        "roofline": {"kernel": run.dominant, "bound": "hbm", "achieved": achieved,
-                     "peak": peak, "peak_kind": peak_kind + " (STREAM-style copy, MEASURED_PEAKS.json)"
-                     if peak_kind == "measured" else peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic_from_profile(args.workload),
-                     "algorithmic_bytes_per_launch": dom_bytes,
-                     "units_per_launch": run.units, "bytes_per_unit": run.bytes_per_unit},
+        "roofline": roofline,
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": run.launches_per_step * args.steps,
         "clocks": clk, "device_error_flag": err,

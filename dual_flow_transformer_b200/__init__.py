@@ -20,6 +20,10 @@ from .api import (  # noqa: F401
     moe_dispatch,
     moe_route,
     new_attn_workspace,
+    new_prefill_workspace,
     new_proj_workspace,
+    prefill,
+    prefill_num_launches,
+    prefill_workspace_size,
     rmsnorm,
 )

@@ -46,6 +46,17 @@ SIGNATURES = {
     "dualflow_kv_append": (_c_int, [
         _vp, _vp, _c_i64, _vp, _vp, _vp, _c_int, _vp,
         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+    "dualflow_prefill_workspace_size": (_c_size, [_c_int] * 6),
+    "dualflow_prefill_num_launches": (_c_int, [_c_int, _c_int]),
+    "dualflow_prefill": (_c_int, [
+        _vp, _c_i64, _vp, _vp, _c_i64,  # q1, q_stride_t, k_new, v_new, kv_stride_t
+        _vp, _vp, _vp, _vp,             # q2raw, a, k_cache, v_cache
+        _vp, _c_int, _vp, _vp,          # block_table, max_blocks_per_seq, cu_seqlens, ctx_lens
+        _c_int, _c_int,                 # max_q_len, max_seqlen
+        _vp, _c_i64, _vp,               # o1, o_stride_t, o2
+        _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,  # B, T, Hq, Hkv, D, bs, nblocks
+        _c_float, _c_int,               # scale, dtype
+        _vp, _c_size, _vp, _vp]),       # workspace, bytes, err_flag, stream
     "dualflow_grouped_proj_workspace_size": (_c_size, [_c_int] * 4),
     "dualflow_grouped_proj_num_launches": (_c_int, [_c_int] * 4),
     "dualflow_grouped_proj": (_c_int, [

@@ -115,6 +115,76 @@ def decode_attn(q1, q2raw, a, k_cache, v_cache, block_table, seqlens, max_seqlen
     return o1, o2
 
 
+# ----------------------------------------------------------------- prefill
+
+def prefill_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size=64) -> int:
+    return _lib().dualflow_prefill_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size)
+
+
+def prefill_num_launches(with_append=True, with_aux=True) -> int:
+    return _lib().dualflow_prefill_num_launches(int(bool(with_append)), int(bool(with_aux)))
+
+
+def new_prefill_workspace(B, Hq, Hkv, D, max_seqlen, device="cuda"):
+    """Zero-filled prefill workspace (the auxiliary step's decode counters
+    start at zero and every completed call leaves them there)."""
+    n = max(256, prefill_workspace_size(B, Hq, Hkv, D, max_seqlen))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def prefill(q1, k_new, v_new, k_cache, v_cache, block_table, cu_seqlens, max_q_len, max_seqlen,
+            *, ctx_lens=None, q2raw=None, a=None, o1=None, o2=None, scale=0.0, workspace=None,
+            err_flag=None, stream=None):
+    """Primary prefill of the chunks cu_seqlens describes; returns (o1, o2).
+
+    q1 [T, Hq, D]; k_new, v_new [T, Hkv, D] (or both None when the cache
+    already holds the chunk); caches [num_blocks, Hkv, 64, D]; block_table
+    int32 [B, max_blocks]; cu_seqlens int32 [B + 1]; ctx_lens int32 [B] or
+    None; q2raw [B, Hq, D] (auxiliary query of each last prompt position) or
+    None; a [Hq, D] or None. max_q_len, max_seqlen: host bounds.
+    """
+    T, Hq, D = q1.shape
+    num_blocks, Hkv, bs, Dk = k_cache.shape
+    B = cu_seqlens.shape[0] - 1
+    if Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("cache shape mismatch")
+    if not _heads_view_ok(q1, Hq, D):
+        raise ValueError("q1 must be [T, Hq, D] with contiguous heads")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new or neither")
+    if k_new is not None and (tuple(k_new.shape) != (T, Hkv, D) or v_new.stride() != k_new.stride()
+                              or not _heads_view_ok(k_new, Hkv, D)):
+        raise ValueError("k_new/v_new must be [T, Hkv, D] with contiguous heads")
+    if not (k_cache.is_contiguous() and v_cache.is_contiguous() and block_table.is_contiguous()):
+        raise ValueError("caches and block table must be contiguous")
+    dev = q1.device
+    if o1 is None:
+        o1 = torch.empty((T, Hq, D), dtype=q1.dtype, device=dev)
+    if not _heads_view_ok(o1, Hq, D):
+        raise ValueError("o1 must be [T, Hq, D] with contiguous heads")
+    if q2raw is None:
+        o2 = None
+    else:
+        if not (q2raw.is_contiguous() and tuple(q2raw.shape) == (B, Hq, D)):
+            raise ValueError("q2raw must be a contiguous [B, Hq, D] tensor")
+        if o2 is None:
+            o2 = torch.empty((B, Hq, D), dtype=q1.dtype, device=dev)
+        if not (o2.is_contiguous() and tuple(o2.shape) == (B, Hq, D)):
+            raise ValueError("o2 must be a contiguous [B, Hq, D] tensor")
+        if workspace is None:
+            workspace = new_prefill_workspace(B, Hq, Hkv, D, max_seqlen, dev)
+    st = _lib().dualflow_prefill(
+        _ptr(q1), q1.stride(0), _ptr(k_new), _ptr(v_new),
+        0 if k_new is None else k_new.stride(0), _ptr(q2raw), _ptr(a), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_table), block_table.shape[1], _ptr(cu_seqlens), _ptr(ctx_lens),
+        int(max_q_len), int(max_seqlen), _ptr(o1), o1.stride(0), _ptr(o2), B, T, Hq, Hkv, D, bs,
+        num_blocks, float(scale), dtype_code(q1.dtype), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    L.check("dualflow_prefill", st)
+    return o1, o2
+
+
 # ----------------------------------------------------------------- append
 
 def kv_append(k_new, v_new, k_cache, v_cache, block_table, positions, *, err_flag=None,

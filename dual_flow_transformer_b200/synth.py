@@ -16,6 +16,9 @@ Workloads (the decode-step shapes studied for the method):
   lengths uniform in [1024, 8192], 64-token pages in a random block table.
 * ``long``  -- B 8, 32/8 heads, head_dim 128, bf16, lengths uniform in
   [32768, 131072], identity block table (split over the sequence needed).
+* ``prefill`` -- primary prefill of 16 fresh prompts of 4096 tokens (the
+  layer workload's cache length), 32/8 heads, head_dim 128, bf16, 64-token
+  pages in a random block table; auxiliary query at each last position.
 * ``layer`` -- full decoder layer at one generated position: d_model 4096,
   32/8 heads, head_dim 128, SwiGLU width 14336, bf16 weights ~ N(0, 0.02),
   B 64 per flow (M = 128 rows), cache 4096 tokens before the step.
@@ -80,6 +83,23 @@ class MixtureWorkload:
 
 
 @dataclasses.dataclass(frozen=True)
+class PrefillWorkload:
+    """Primary prefill of prompt chunks (one layer's attention), with the
+    auxiliary query at each chunk's last position."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    len_lo: int                # chunk length range (inclusive)
+    len_hi: int
+    ctx_lo: int = 0            # tokens already cached before the chunk
+    ctx_hi: int = 0
+    random_table: bool = True
+    seed: int = 8
+
+
+@dataclasses.dataclass(frozen=True)
 class MoEWorkload:
     """MoE MLP block of both flows with router replay (one decode step)."""
     name: str
@@ -100,6 +120,7 @@ WORKLOADS = {
     "layer": LayerWorkload("layer", 64, 4096, 32, 8, 128, 14336, 4096, seed=5),
     "mixture": MixtureWorkload("mixture", 64, 4096, 32000, seed=6),
     "moe": MoEWorkload("moe", 64, 2048, 5632, 8, 2, 2, seed=7),
+    "prefill": PrefillWorkload("prefill", 16, 32, 8, 128, 4096, 4096, seed=8),
 }
 
 
@@ -269,3 +290,45 @@ def make_moe_inputs(w: MoEWorkload, seed: Optional[int] = None):
         w_down[e] = _randn(g, (w.d_model, w.F), std=0.02, chunk_rows=2048)
     return dict(x=x, w_router=w_router, w_gu=w_gu, w_down=w_down, B=w.B, d_model=w.d_model,
                 F=w.F, E=w.E, k=w.k, k_aux=w.k_aux)
+
+
+def make_prefill_inputs(w: PrefillWorkload, seed: Optional[int] = None, lengths=None, ctx=None):
+    """Host tensors for one prefill call of workload ``w`` (bf16).
+
+    Chunk lengths n_b ~ U{len_lo..len_hi} and cached prefixes c_b ~
+    U{ctx_lo..ctx_hi} (or the given ``lengths`` / ``ctx``); the block table
+    covers c_b + n_b tokens per sequence. Returns q1 [T, Hq, D], k_new, v_new
+    [T, Hkv, D], q2raw [B, Hq, D], a [Hq, D] (std 0.1), k_cache, v_cache
+    [num_blocks, Hkv, 64, D] (every slot drawn; the prefix slots are the
+    cached tokens), block_table, cu_seqlens [B + 1], ctx_lens [B] (int32),
+    max_q_len and max_seqlen.
+    """
+    g = _gen(w.seed if seed is None else seed)
+    dt = torch.bfloat16
+    if lengths is not None:
+        lens = torch.as_tensor(lengths, dtype=torch.int32)
+    else:
+        lens = make_lengths(g, w.B, w.len_lo, w.len_hi)
+    B = lens.numel()
+    if ctx is not None:
+        ctx_lens = torch.as_tensor(ctx, dtype=torch.int32)
+    elif w.ctx_hi > 0:
+        ctx_lens = make_lengths(g, B, w.ctx_lo, w.ctx_hi)
+    else:
+        ctx_lens = torch.zeros(B, dtype=torch.int32)
+    caps = (ctx_lens + lens).tolist()
+    table, nblocks = make_block_table(g, caps, BLOCK_SIZE, w.random_table)
+    T = int(lens.sum())
+    cu = torch.zeros(B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    q1 = _randn(g, (T, w.Hq, w.D), dtype=dt, chunk_rows=4096)
+    k_new = _randn(g, (T, w.Hkv, w.D), dtype=dt, chunk_rows=4096)
+    v_new = _randn(g, (T, w.Hkv, w.D), dtype=dt, chunk_rows=4096)
+    q2raw = _randn(g, (B, w.Hq, w.D), dtype=dt)
+    a = _randn(g, (w.Hq, w.D), std=0.1, dtype=dt)
+    kc = _randn(g, (nblocks, w.Hkv, BLOCK_SIZE, w.D), dtype=dt, chunk_rows=1024)
+    vc = _randn(g, (nblocks, w.Hkv, BLOCK_SIZE, w.D), dtype=dt, chunk_rows=1024)
+    return dict(q1=q1, k_new=k_new, v_new=v_new, q2raw=q2raw, a=a, k_cache=kc, v_cache=vc,
+                block_table=table, cu_seqlens=cu, ctx_lens=ctx_lens, num_blocks=nblocks, B=B,
+                T=T, Hq=w.Hq, Hkv=w.Hkv, D=w.D, max_q_len=int(lens.max()),
+                max_seqlen=int(max(caps)))

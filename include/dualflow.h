@@ -86,7 +86,8 @@ const char* dualflow_status_string(int status);
 /*   seqlens[b] tokens of the cache.                                         */
 /* Each KV page is read from HBM once for all 2 * Hq/Hkv query rows of its    */
 /* KV head. Split over the sequence (flash-decoding) with per-split fp32     */
-/* partials in `workspace`, then a separate combine kernel.                  */
+/* partials in `workspace`, merged by the last split to finish (bf16) or by  */
+/* a separate combine kernel (fp32).                                         */
 /*                                                                           */
 /* q1, q2raw : [B][Hq][D] (dtype), sequence b at q + b*q_stride_b elements   */
 /*             (q_stride_b = 0 means Hq*D). 4-byte aligned; q_stride_b even. */
@@ -188,6 +189,64 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
                              int max_blocks_per_seq, const int32_t* positions, int B, int Hkv,
                              int D, int block_size, int num_blocks, int dtype,
                              int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Primary prefill (prompt processing), with the auxiliary query at the last */
+/* prompt position.                                                          */
+/*                                                                           */
+/* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Architettura      */
+/* Core": the primary flow is a standard causal Transformer that processes   */
+/* the whole prompt and writes the persistent cache; the auxiliary flow is   */
+/* skipped over the prompt and switched on only at the last prompt position. */
+/* Section "Costi di Inferenza vs. Addestramento": prefill costs the same as  */
+/* a standard Transformer's.                                                 */
+/*                                                                           */
+/* Sequence b's chunk is the token rows t in [cu_seqlens[b],                 */
+/* cu_seqlens[b+1]) (n_b >= 1 tokens); its cache already holds ctx_lens[b]   */
+/* tokens (ctx_lens NULL = 0: a fresh prompt), so chunk token i is position  */
+/* p = ctx_lens[b] + i. The call                                             */
+/*  1. writes k_new/v_new row t to cache position p (as dualflow_kv_append); */
+/*     k_new = v_new = NULL skips this (the cache already holds the chunk);  */
+/*  2. O1[t,h] = softmax_j(scale * q1[t,h] . k_j) V over positions j <= p of */
+/*     KV head g = h / (Hq/Hkv) (causal; prefix + chunk);                    */
+/*  3. if q2raw and o2 are given: O2[b,h] = the decode step's auxiliary      */
+/*     output for the last position P = ctx_lens[b] + n_b - 1, i.e. Q2 =     */
+/*     q2raw[b] + a (.) q1[last row of b] over positions j <= P (computed by */
+/*     the decode attention kernel in auxiliary-only mode).                  */
+/*                                                                           */
+/* q1        : bf16 [T][Hq][D], token row t at q1 + t*q_stride_t elements    */
+/*             (0 = Hq*D); 16-byte aligned, q_stride_t % 8 == 0.              */
+/* k_new, v_new : bf16 [T][Hkv][D] at + t*kv_stride_t (0 = Hkv*D), 16-byte   */
+/*             aligned, kv_stride_t % 8 == 0; or both NULL.                  */
+/* q2raw, a  : bf16 [B][Hq][D] (the auxiliary query of the last position,    */
+/*             before coupling) and [Hq][D] (or NULL: no coupling).          */
+/* cu_seqlens: int32 [B+1], device; ctx_lens: int32 [B], device, or NULL.    */
+/* max_q_len : host bound of every n_b (sets the grid); max_seqlen: host     */
+/*             bound of every ctx_lens[b] + n_b, <= max_blocks_per_seq * 64. */
+/*             A chunk outside these bounds (or with n_b < 1, or rows past T)*/
+/*             sets DF_DEVERR_SEQLEN and is skipped (its rows unwritten).    */
+/* o1        : bf16 [T][Hq][D] at + t*o_stride_t (0 = Hq*D), 4-byte aligned. */
+/* o2        : bf16 [B][Hq][D] or NULL.                                      */
+/* workspace : only with the auxiliary step: 256-byte aligned, at least      */
+/*             dualflow_prefill_workspace_size(...) bytes, ZERO-FILLED once  */
+/*             (its first bytes are the decode kernel's arrival counters,    */
+/*             which every completed call leaves at zero).                   */
+/* Supported: dtype DF_BF16, D in {64, 128}, block_size 64; with the         */
+/* auxiliary step also Hq/Hkv <= 4. Kernel launches per call:                */
+/* dualflow_prefill_num_launches(k_new != NULL, auxiliary step).             */
+/* ------------------------------------------------------------------------ */
+size_t dualflow_prefill_workspace_size(int B, int Hq, int Hkv, int D, int max_seqlen,
+                                       int block_size);
+int dualflow_prefill_num_launches(int with_append, int with_aux);
+df_status dualflow_prefill(const void* q1, int64_t q_stride_t, const void* k_new,
+                           const void* v_new, int64_t kv_stride_t, const void* q2raw,
+                           const void* a, void* k_cache, void* v_cache,
+                           const int32_t* block_table, int max_blocks_per_seq,
+                           const int32_t* cu_seqlens, const int32_t* ctx_lens, int max_q_len,
+                           int max_seqlen, void* o1, int64_t o_stride_t, void* o2, int B, int T,
+                           int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+                           int dtype, void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                           void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Grouped shared-weight projection (tcgen05 tensor cores, TMEM accumulator).*/

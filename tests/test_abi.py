@@ -216,3 +216,50 @@ def test_grouped_proj_batched_rejects_invalid_arguments(lib):
     assert call(a8=1024 * 512 + 4) == L.DF_ERR_ALIGN        # w batch stride not 16-byte
     nl = lib.dualflow_grouped_proj_batched_num_launches
     assert nl(128, 1024, 512, 2, 4) == 0 and nl(0, 1024, 512, 0, 4) == 0
+
+
+def _prefill(lib, **over):
+    a = dict(q1=FAKE, qs=0, kn=FAKE, vn=FAKE, kvs=0, q2=FAKE, av=FAKE, kc=FAKE, vc=FAKE,
+             tbl=FAKE, mbps=8, cu=FAKE, ctx=None, mql=256, msl=400, o1=FAKE, os=0, o2=FAKE,
+             B=2, T=300, Hq=8, Hkv=2, D=128, bs=64, nb=16, scale=0.0, dtype=L.DF_BF16,
+             ws=FAKE, wsb=1 << 30, err=None, stream=None)
+    a.update(over)
+    return lib.dualflow_prefill(a["q1"], a["qs"], a["kn"], a["vn"], a["kvs"], a["q2"], a["av"],
+                                a["kc"], a["vc"], a["tbl"], a["mbps"], a["cu"], a["ctx"],
+                                a["mql"], a["msl"], a["o1"], a["os"], a["o2"], a["B"], a["T"],
+                                a["Hq"], a["Hkv"], a["D"], a["bs"], a["nb"], a["scale"],
+                                a["dtype"], a["ws"], a["wsb"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q1=None), L.DF_ERR_NULL),
+    (dict(o1=None), L.DF_ERR_NULL),
+    (dict(cu=None), L.DF_ERR_NULL),
+    (dict(vn=None), L.DF_ERR_NULL),               # k_new without v_new
+    (dict(T=1), L.DF_ERR_SHAPE),                  # fewer tokens than sequences
+    (dict(mql=301), L.DF_ERR_SHAPE),              # chunk bound above T
+    (dict(msl=100), L.DF_ERR_SHAPE),              # max_seqlen below max_q_len
+    (dict(msl=600), L.DF_ERR_SHAPE),              # beyond the block table
+    (dict(Hq=7), L.DF_ERR_SHAPE),
+    (dict(qs=8), L.DF_ERR_SHAPE),                 # token stride below Hq * D
+    (dict(dtype=L.DF_FP32), L.DF_ERR_UNSUPPORTED),
+    (dict(D=96), L.DF_ERR_UNSUPPORTED),
+    (dict(bs=32, msl=256), L.DF_ERR_UNSUPPORTED),
+    (dict(Hq=16, Hkv=2), L.DF_ERR_UNSUPPORTED),   # auxiliary step needs Hq/Hkv <= 4
+    (dict(q1=FAKE + 8), L.DF_ERR_ALIGN),
+    (dict(qs=8 * 128 + 4), L.DF_ERR_ALIGN),
+    (dict(kn=FAKE + 4), L.DF_ERR_ALIGN),
+    (dict(ws=None), L.DF_ERR_WORKSPACE),
+    (dict(wsb=16), L.DF_ERR_WORKSPACE),
+    (dict(ws=FAKE + 64), L.DF_ERR_WORKSPACE),
+])
+def test_prefill_rejects_invalid_arguments(lib, over, status):
+    assert _prefill(lib, **over) == status
+
+
+def test_prefill_sizes(lib):
+    assert lib.dualflow_prefill_num_launches(1, 1) == 4
+    assert lib.dualflow_prefill_num_launches(0, 1) == 3
+    assert lib.dualflow_prefill_num_launches(1, 0) == 2
+    assert lib.dualflow_prefill_workspace_size(2, 8, 2, 128, 400, 64) > 0
+    assert lib.dualflow_prefill_workspace_size(2, 8, 2, 128, 400, 32) == 0
