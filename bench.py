@@ -248,6 +248,27 @@ class LayerRun:
     def step(self, timers=None):
         self.layer.replay(timers)
 
+    def attn_graphs(self):
+        """(dual attention graph, primary-only attention graph) on this step's
+        buffers: the same call with q2raw = NULL writes O1 only."""
+        import torch
+        from dual_flow_transformer_b200 import api
+        L, d = self.layer, self.d
+        B, Hq, D = L.B, L.Hq, L.D
+        o1 = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=L.qkv.device)
+
+        def call():
+            api.decode_attn(L.qkv[:B, :Hq * D].view(B, Hq, D), None, None, d["k_cache"],
+                            d["v_cache"], d["block_table"], self.seqlens, L.max_seqlen, o1=o1,
+                            num_splits=L.num_splits, workspace=L.attn_ws, err_flag=L.err)
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        self._primary_o1 = o1
+        return L.graphs[1], g
+
     def step_host(self, x_host, out_host):
         d = self.d
         self.layer.step_host(x_host, out_host, d["k_cache"], d["v_cache"], d["block_table"],
@@ -332,6 +353,24 @@ class AttnRun:
         self.g_attn.replay()
         if timers is not None:
             timers["attn"][1].record()
+
+    def attn_graphs(self):
+        """(dual attention graph, primary-only attention graph)."""
+        import torch
+        d = self.d
+        o1 = torch.empty_like(d["q1"])
+
+        def call():
+            self.api.decode_attn(d["q1"], None, None, d["k_cache"], d["v_cache"],
+                                 d["block_table"], d["seqlens"], self.max_len, o1=o1,
+                                 num_splits=self.ns, workspace=self.ws, err_flag=self.err)
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        self._primary_o1 = o1
+        return self.g_attn, g
 
     def host_io(self):
         import torch
@@ -961,6 +1000,30 @@ def main(argv=None):
     kernel_ms = {k: max_over_ranks(sum(t[k][0].elapsed_time(t[k][1]) for t in timers) / args.steps,
                                    world) for k in keys}
     attn_ms = kernel_ms[getattr(run, "dominant_key", "attn")]
+
+    # ---------------------------------------------------------------- aux overhead
+    # Decode attention alone, dual call vs the same call with q2raw = NULL,
+    # replayed back to back in A B A B order.
+    aux_overhead = None
+    if hasattr(run, "attn_graphs"):
+        g_dual, g_prim = run.attn_graphs()
+        n_rep = max(20, min(args.steps, 400))
+        tot = {"dual": 0.0, "primary_only": 0.0}
+        for name, g in (("dual", g_dual), ("primary_only", g_prim)) * 2:
+            s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            torch.cuda.synchronize()
+            s_ev.record()
+            for _ in range(n_rep):
+                g.replay()
+            e_ev.record()
+            torch.cuda.synchronize()
+            tot[name] += max_over_ranks(s_ev.elapsed_time(e_ev), world) / (2 * n_rep)
+        aux_overhead = {"dual_ms": tot["dual"], "primary_only_ms": tot["primary_only"],
+                        "ratio": tot["dual"] / tot["primary_only"], "target": 1.15,
+                        "replays": 2 * n_rep,
+                        "how": "decode attention graphs alone, dual vs q2raw = NULL, "
+                               "ABAB back-to-back replays, CUDA events"}
     err = run.check_err()
 
     # ---------------------------------------------------------------- end to end (host buffers)
@@ -1036,6 +1099,8 @@ def main(argv=None):
         "gpu_launches": run.launches_per_step * args.steps,
         "clocks": clk, "device_error_flag": err,
     }
+    if aux_overhead is not None:
+        line["aux_overhead"] = aux_overhead
     if hasattr(run, "kv_bytes"):
         line["kv_read_gbs"] = run.kv_bytes / (attn_ms / 1e3) / 1e9
         line["kv_frac_of_hbm_peak"] = run.kv_bytes / (attn_ms / 1e3) / 1e9 / peak

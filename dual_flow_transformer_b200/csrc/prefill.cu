@@ -20,7 +20,8 @@
 //     first. 4 consumer warps own 16 query rows each; 1 producer warp streams
 //     64-token K and V pages by TMA (128-byte swizzle) through a 3-stage
 //     mbarrier ring. S = Q K^T and O += P V run on mma.sync (bf16 in, fp32
-//     accumulate), online softmax in the exp2 domain per row;
+//     accumulate), online softmax in the exp2 domain per row (P rounded once
+//     to bf16 for P V, fp32 row sums);
 //  3. gather_last_kernel: copies each sequence's last-position primary query
 //     row and writes the attended length ctx + n, the inputs of
 //  4. the decode attention kernel in auxiliary-only mode: the coupled
@@ -141,9 +142,6 @@ struct AttnParams {
   int32_t* err;
 };
 
-// max that propagates NaN (fmaxf drops it), so NaN inputs give NaN outputs.
-__device__ __forceinline__ float max_nan(float a, float b) { return (a != a || a > b) ? a : b; }
-
 // Byte address of 16-byte chunk `ch` of token row `tok` in a TMA-written
 // [64 tokens][D] bf16 page stored as D/64 column halves of [64][128 B] with the
 // 128-byte swizzle (chunk index XOR row index within each 8-row group).
@@ -152,7 +150,8 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int tok, int ch) {
 }
 
 __device__ __forceinline__ uint32_t pack_f32_bf16x2(float lo, float hi) {
-  return pack_bf16x2(__float2bfloat16_rn(lo), __float2bfloat16_rn(hi));
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // lo in the low half
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // Zero the bf16 halves of a P V operand register whose key index is >= kend:
@@ -292,103 +291,114 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t kb = smem_u32(smem + st * kStageBytes);
       const uint32_t vb = kb + kTileBytes;
       const int kbase = i * kPage;
-
-      // S = Q K^T: 16 rows x 64 keys (8 n-tiles of 8 keys).
-      float sc[8][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-        for (int kg = 0; kg < 4; ++kg) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(swz(kb, kg * 16 + (mi >> 1) * 8 + r8, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-          mma_bf16_16816(sc[2 * kg], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-          mma_bf16_16816(sc[2 * kg + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
-        }
-      }
-
-      // Causal mask (key j visible to the row at position pos iff j <= pos),
-      // needed only where the page reaches past the warp's first row.
-      const bool need_mask = kbase + kPage - 1 > w_first;
-      float mx_lo = kNegInf, mx_hi = kNegInf;
-#pragma unroll
-      for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = kbase + n * 8 + 2 * tq + e;
-          float s0 = sc[n][e] * p.scale_log2, s1 = sc[n][e + 2] * p.scale_log2;
-          if (need_mask) {
-            if (j > pos_lo) s0 = kNegInf;
-            if (j > pos_hi) s1 = kNegInf;
-          }
-          sc[n][e] = s0;
-          sc[n][e + 2] = s1;
-          mx_lo = max_nan(mx_lo, s0);
-          mx_hi = max_nan(mx_hi, s1);
-        }
-      mx_lo = max_nan(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-      mx_lo = max_nan(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-      mx_hi = max_nan(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-      mx_hi = max_nan(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-      const float mn_lo = max_nan(m_lo, mx_lo), mn_hi = max_nan(m_hi, mx_hi);
-      const float mu_lo = (mn_lo == kNegInf) ? 0.f : mn_lo;
-      const float mu_hi = (mn_hi == kNegInf) ? 0.f : mn_hi;
-      const float al_lo = exp2f(m_lo - mu_lo), al_hi = exp2f(m_hi - mu_hi);
-      m_lo = mn_lo;
-      m_hi = mn_hi;
-
-      // P in bf16 as the A operand of P V (k-step ks = keys 16 ks .. 16 ks + 15);
-      // the row sums add the same rounded weights the products use.
-      uint32_t pa[4][4];
-      float ps_lo = 0.f, ps_hi = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int n = 2 * ks + half;
-          const __nv_bfloat16 p0 = __float2bfloat16_rn(exp2f(sc[n][0] - mu_lo));
-          const __nv_bfloat16 p1 = __float2bfloat16_rn(exp2f(sc[n][1] - mu_lo));
-          const __nv_bfloat16 p2 = __float2bfloat16_rn(exp2f(sc[n][2] - mu_hi));
-          const __nv_bfloat16 p3 = __float2bfloat16_rn(exp2f(sc[n][3] - mu_hi));
-          ps_lo += __bfloat162float(p0) + __bfloat162float(p1);
-          ps_hi += __bfloat162float(p2) + __bfloat162float(p3);
-          pa[ks][2 * half + 0] = pack_bf16x2(p0, p1);
-          pa[ks][2 * half + 1] = pack_bf16x2(p2, p3);
-        }
-      l_lo = l_lo * al_lo + ps_lo;
-      l_hi = l_hi * al_hi + ps_hi;
-      if (!__all_sync(0xffffffffu, al_lo == 1.f && al_hi == 1.f)) {
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          acc[n][0] *= al_lo;
-          acc[n][1] *= al_lo;
-          acc[n][2] *= al_hi;
-          acc[n][3] *= al_hi;
-        }
-      }
-
-      // O += P V. Keys at or past kend hold other tokens' bytes (possibly NaN
-      // patterns); their weights are 0, and their V halves are zeroed too, as
-      // 0 * NaN would still be NaN.
       const bool v_tail = kbase + kPage > kend;
       const int kend_rel = kend - kbase;
+
+      // The page in two halves of 32 keys (fewer live registers); a half that
+      // lies wholly past the warp's last row is skipped.
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
+      for (int hk = 0; hk < 2; ++hk) {
+        const int hbase = kbase + hk * 32;
+        if (hbase > w_last) break;
+
+        // S = Q K^T: 16 rows x 32 keys (4 n-tiles of 8 keys).
+        float sc[4][4];
 #pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_trans(swz(vb, ks * 16 + (mi & 1) * 8 + r8, 2 * np + (mi >> 1)), v0, v1, v2,
-                        v3);
-          if (v_tail) {
-            const int k0 = ks * 16 + 2 * tq;
-            v0 = keep_keys(v0, k0, kend_rel);
-            v2 = keep_keys(v2, k0, kend_rel);
-            v1 = keep_keys(v1, k0 + 8, kend_rel);
-            v3 = keep_keys(v3, k0 + 8, kend_rel);
+        for (int n = 0; n < 4; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+          for (int kg = 0; kg < 2; ++kg) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(swz(kb, hk * 32 + kg * 16 + (mi >> 1) * 8 + r8, 2 * ks + (mi & 1)), b0, b1,
+                    b2, b3);
+            mma_bf16_16816(sc[2 * kg], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+            mma_bf16_16816(sc[2 * kg + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
           }
-          mma_bf16_16816(acc[2 * np], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], v0, v1);
-          mma_bf16_16816(acc[2 * np + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], v2, v3);
+        }
+
+        // Causal mask (key j visible to the row at position pos iff j <= pos),
+        // needed only where the half reaches past the warp's first row.
+        if (hbase + 31 > w_first) {
+#pragma unroll
+          for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int j = hbase + n * 8 + 2 * tq + e;
+              if (j > pos_lo) sc[n][e] = kNegInf;
+              if (j > pos_hi) sc[n][e + 2] = kNegInf;
+            }
+        }
+        // Row maxima of the raw scores as a tree (scale > 0 keeps the order).
+        // fmaxf skips a NaN score, but the NaN still reaches the output
+        // through its weight exp2(NaN) and the sums.
+        float mx_lo = fmaxf(fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])),
+                            fmaxf(fmaxf(sc[2][0], sc[2][1]), fmaxf(sc[3][0], sc[3][1])));
+        float mx_hi = fmaxf(fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3])),
+                            fmaxf(fmaxf(sc[2][2], sc[2][3]), fmaxf(sc[3][2], sc[3][3])));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+        // running maxima in log2 units
+        const float mn_lo = fmaxf(m_lo, mx_lo * p.scale_log2);
+        const float mn_hi = fmaxf(m_hi, mx_hi * p.scale_log2);
+        const float mu_lo = (mn_lo == kNegInf) ? 0.f : mn_lo;
+        const float mu_hi = (mn_hi == kNegInf) ? 0.f : mn_hi;
+        const float al_lo = exp2f(m_lo - mu_lo), al_hi = exp2f(m_hi - mu_hi);
+        m_lo = mn_lo;
+        m_hi = mn_hi;
+
+        // P = 2^(s * scale_log2 - m) in bf16 as the A operand of P V (k-step
+        // ks = keys 16 ks .. 16 ks + 15 of the half); fp32 row sums.
+        uint32_t pa[2][4];
+        float ps_lo = 0.f, ps_hi = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int n = 2 * ks + half;
+            const float p0 = exp2f(fmaf(sc[n][0], p.scale_log2, -mu_lo));
+            const float p1 = exp2f(fmaf(sc[n][1], p.scale_log2, -mu_lo));
+            const float p2 = exp2f(fmaf(sc[n][2], p.scale_log2, -mu_hi));
+            const float p3 = exp2f(fmaf(sc[n][3], p.scale_log2, -mu_hi));
+            ps_lo += p0 + p1;
+            ps_hi += p2 + p3;
+            pa[ks][2 * half + 0] = pack_f32_bf16x2(p0, p1);
+            pa[ks][2 * half + 1] = pack_f32_bf16x2(p2, p3);
+          }
+        l_lo = fmaf(l_lo, al_lo, ps_lo);
+        l_hi = fmaf(l_hi, al_hi, ps_hi);
+        if (!__all_sync(0xffffffffu, al_lo == 1.f && al_hi == 1.f)) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            acc[n][0] *= al_lo;
+            acc[n][1] *= al_lo;
+            acc[n][2] *= al_hi;
+            acc[n][3] *= al_hi;
+          }
+        }
+
+        // O += P V. Keys at or past kend hold other tokens' bytes (possibly
+        // NaN patterns); their weights are 0, and their V halves are zeroed
+        // too, as 0 * NaN would still be NaN.
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+          for (int np = 0; np < NT / 2; ++np) {
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_trans(swz(vb, hk * 32 + ks * 16 + (mi & 1) * 8 + r8, 2 * np + (mi >> 1)), v0,
+                          v1, v2, v3);
+            if (v_tail) {
+              const int k0 = hk * 32 + ks * 16 + 2 * tq;
+              v0 = keep_keys(v0, k0, kend_rel);
+              v2 = keep_keys(v2, k0, kend_rel);
+              v1 = keep_keys(v1, k0 + 8, kend_rel);
+              v3 = keep_keys(v3, k0 + 8, kend_rel);
+            }
+            mma_bf16_16816(acc[2 * np], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], v0, v1);
+            mma_bf16_16816(acc[2 * np + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], v2, v3);
+          }
         }
       }
     }
