@@ -606,7 +606,11 @@ class PrefillRun:
                                    % (h["B"], w.len_lo, w.len_hi, w.Hq, w.Hkv, w.D),
                        "l2": "inputs larger than L2 (%.0f MB of queries, %.0f MB of new K/V)"
                              % (h["q1"].numel() * 2 / 1e6, 2 * h["k_new"].numel() * 2 / 1e6)}
-        self.dominant = "dualflow_prefill attention kernel (mma.sync, TMA page ring)"
+        kern = api.prefill_kernel(w.D, h["T"], self.o1, w.Hq)
+        self.dominant = ("dualflow_prefill attention kernel (%s)"
+                         % ("tcgen05, TMEM accumulators" if kern == "tcgen05"
+                            else "mma.sync, TMA page ring"))
+        self.config["attn_kernel"] = kern
         self._full()
         torch.cuda.synchronize()
         self.g_full, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()

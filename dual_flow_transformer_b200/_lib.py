@@ -19,6 +19,7 @@ DF_FP32, DF_BF16 = 0, 1
 DF_EPI_NONE, DF_EPI_SWIGLU, DF_EPI_RESIDUAL = 0, 1, 2
 DF_DEVERR_SEQLEN, DF_DEVERR_BLOCK, DF_DEVERR_POSITION, DF_DEVERR_TIMEOUT = 1, 2, 4, 8
 DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+DF_PREFILL_KERNEL_AUTO, DF_PREFILL_KERNEL_MMA_SYNC, DF_PREFILL_KERNEL_TCGEN05 = 0, 1, 2
 
 _c_int, _c_i64, _c_size, _c_float, _vp = (ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
                                            ctypes.c_float, ctypes.c_void_p)
@@ -48,6 +49,12 @@ SIGNATURES = {
         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "dualflow_prefill_workspace_size": (_c_size, [_c_int] * 6),
     "dualflow_prefill_num_launches": (_c_int, [_c_int, _c_int]),
+    "dualflow_prefill_kernel": (_c_int, [_c_int, _c_int, _vp, _c_i64, _c_int]),
+    "dualflow_prefill_ex": (_c_int, [
+        _vp, _c_i64, _vp, _vp, _c_i64, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int,
+        _vp, _c_i64, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+        _c_float, _c_int, _c_int,       # scale, dtype, kernel
+        _vp, _c_size, _vp, _vp]),
     "dualflow_prefill": (_c_int, [
         _vp, _c_i64, _vp, _vp, _c_i64,  # q1, q_stride_t, k_new, v_new, kv_stride_t
         _vp, _vp, _vp, _vp,             # q2raw, a, k_cache, v_cache

@@ -121,6 +121,12 @@ def prefill_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size=64) -> int:
     return _lib().dualflow_prefill_workspace_size(B, Hq, Hkv, D, max_seqlen, block_size)
 
 
+def prefill_kernel(D, T, o1, Hq) -> str:
+    """The attention kernel an automatic prefill call uses for these sizes."""
+    k = _lib().dualflow_prefill_kernel(D, T, _ptr(o1), o1.stride(0), Hq)
+    return "tcgen05" if k == L.DF_PREFILL_KERNEL_TCGEN05 else "mma_sync"
+
+
 def prefill_num_launches(with_append=True, with_aux=True) -> int:
     return _lib().dualflow_prefill_num_launches(int(bool(with_append)), int(bool(with_aux)))
 
@@ -134,7 +140,7 @@ def new_prefill_workspace(B, Hq, Hkv, D, max_seqlen, device="cuda"):
 
 def prefill(q1, k_new, v_new, k_cache, v_cache, block_table, cu_seqlens, max_q_len, max_seqlen,
             *, ctx_lens=None, q2raw=None, a=None, o1=None, o2=None, scale=0.0, workspace=None,
-            err_flag=None, stream=None):
+            err_flag=None, stream=None, kernel="auto"):
     """Primary prefill of the chunks cu_seqlens describes; returns (o1, o2).
 
     q1 [T, Hq, D]; k_new, v_new [T, Hkv, D] (or both None when the cache
@@ -142,7 +148,10 @@ def prefill(q1, k_new, v_new, k_cache, v_cache, block_table, cu_seqlens, max_q_l
     int32 [B, max_blocks]; cu_seqlens int32 [B + 1]; ctx_lens int32 [B] or
     None; q2raw [B, Hq, D] (auxiliary query of each last prompt position) or
     None; a [Hq, D] or None. max_q_len, max_seqlen: host bounds.
+    kernel: "auto", "mma_sync" or "tcgen05" (the attention kernel).
     """
+    kcode = {"auto": L.DF_PREFILL_KERNEL_AUTO, "mma_sync": L.DF_PREFILL_KERNEL_MMA_SYNC,
+             "tcgen05": L.DF_PREFILL_KERNEL_TCGEN05}[kernel]
     T, Hq, D = q1.shape
     num_blocks, Hkv, bs, Dk = k_cache.shape
     B = cu_seqlens.shape[0] - 1
@@ -173,15 +182,15 @@ def prefill(q1, k_new, v_new, k_cache, v_cache, block_table, cu_seqlens, max_q_l
             raise ValueError("o2 must be a contiguous [B, Hq, D] tensor")
         if workspace is None:
             workspace = new_prefill_workspace(B, Hq, Hkv, D, max_seqlen, dev)
-    st = _lib().dualflow_prefill(
+    st = _lib().dualflow_prefill_ex(
         _ptr(q1), q1.stride(0), _ptr(k_new), _ptr(v_new),
         0 if k_new is None else k_new.stride(0), _ptr(q2raw), _ptr(a), _ptr(k_cache),
         _ptr(v_cache), _ptr(block_table), block_table.shape[1], _ptr(cu_seqlens), _ptr(ctx_lens),
         int(max_q_len), int(max_seqlen), _ptr(o1), o1.stride(0), _ptr(o2), B, T, Hq, Hkv, D, bs,
-        num_blocks, float(scale), dtype_code(q1.dtype), _ptr(workspace),
+        num_blocks, float(scale), dtype_code(q1.dtype), kcode, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(),
         _ptr(err_flag), _stream(stream))
-    L.check("dualflow_prefill", st)
+    L.check("dualflow_prefill_ex", st)
     return o1, o2
 
 

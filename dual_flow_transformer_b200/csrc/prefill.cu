@@ -13,8 +13,10 @@
 // programmatic dependent launch:
 //  1. append_kernel: token t of sequence b goes to cache position
 //     ctx_lens[b] + (t - cu_seqlens[b]) (one CTA per token, 16-byte copies);
-//  2. attn_kernel: causal flash attention of the chunk's primary queries over
-//     the cache (prefix + chunk). One CTA per (query head, 64-row tile,
+//  2. causal flash attention of the chunk's primary queries over the cache
+//     (prefix + chunk): tc::attn_kernel on the tcgen05 tensor cores (D = 128,
+//     at least 128 token rows, 16-byte aligned output rows; described at the
+//     kernel), otherwise attn_kernel: one CTA per (query head, 64-row tile,
 //     sequence), heads fastest so that the CTAs sharing a KV head run side by
 //     side and meet its pages in L2; tiles of one sequence are issued longest
 //     first. 4 consumer warps own 16 query rows each; 1 producer warp streams
@@ -31,6 +33,7 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "umma.cuh"
 
 extern "C" size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, int D,
                                                       int max_seqlen, int block_size,
@@ -430,6 +433,386 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
+
+// ------------------------------------------------------------------ 2'. attention, tcgen05
+//
+// The same computation on the 5th-generation tensor cores, for D = 128. One
+// CTA per (query head, 128-row tile, sequence); 6 warps:
+//  * warp 0, one thread: TMA producer -- the tile's Q rows once (two K-major
+//    [128][64] boxes, 128-byte swizzle), then the K and V pages of the key
+//    range through the 3-stage ring;
+//  * warp 1, one thread: MMA issuer -- S_i = Q K_i^T (M 128, N 64, K 128)
+//    into one of two 64-column TMEM buffers, and O += P_i V_i (M 128, K 64,
+//    two N = 64 halves) into a 128-column TMEM accumulator; S_{i+1} is issued
+//    before waiting for P_i, so it overlaps the softmax of page i;
+//  * warps 2-5: one thread per query row (its TMEM lane): S row by
+//    tcgen05.ld, causal mask, row max, P = 2^(s scale_log2 - m) written to
+//    shared memory as bf16 in the K-major swizzled layout the MMA reads. The
+//    reference max m is updated (and O rescaled in TMEM) only when a row's max
+//    exceeds it by more than 2^8, so P stays <= 256 and O is rarely touched.
+//    After the last page: O / l from TMEM to bf16 rows in global memory.
+namespace tc {
+
+constexpr int kRows = 128;          // query rows per CTA (= TMEM lanes)
+constexpr int kThreads = 192;       // producer warp, MMA warp, 4 softmax warps
+constexpr uint32_t kTmemCols = 256; // S double buffer (2 x 64 columns) + O (128)
+constexpr uint32_t kOCol = 128;     // first TMEM column of O
+constexpr float kRescaleLog2 = 8.f; // keep a stale reference max up to 2^8 below
+
+template <int D>
+struct Layout {
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kPageBytes = kPage * D * 2;   // one K (or V) page
+  static constexpr int kStageBytes = 2 * kPageBytes;
+  static constexpr int kPBytes = kRows * kPage * 2;  // P of one page: [128 rows][64 keys]
+  static constexpr int kOffStages = kQBytes;
+  static constexpr int kOffP = kOffStages + kStages * kStageBytes;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 + 1;
+  static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
+};
+
+// Descriptor of an MN-major bf16 operand with 128-byte swizzle that is one
+// swizzle atom (64 elements) wide along N: 8-row atoms along K are 1024 bytes
+// apart; both byte-offset fields carry that stride (the N extent needs none).
+__device__ __forceinline__ uint64_t smem_desc_mn64(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1024 >> 4) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// Store 32 consecutive fp32 TMEM columns of this thread's lane and wait.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float t[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    t[q] = fmaxf(fmaxf(v[4 * q], v[4 * q + 1]), fmaxf(v[4 * q + 2], v[4 * q + 3]));
+  return fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])), fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
+}
+
+// P of 32 keys (chunks c0 .. c0 + 3 of 8 keys) of row r: bf16 into the
+// swizzled row (16-byte chunk c of row r at chunk c ^ (r & 7)); returns the
+// fp32 sum of the weights.
+__device__ __forceinline__ float write_p32(uint8_t* prow, int r, int c0, const float (&s)[32],
+                                           float scale_log2, float mu) {
+  float sum[2] = {0.f, 0.f};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = exp2f(fmaf(s[8 * q + 2 * k], scale_log2, -mu));
+      const float b = exp2f(fmaf(s[8 * q + 2 * k + 1], scale_log2, -mu));
+      sum[k & 1] += a + b;
+      w[k] = pack_f32_bf16x2(a, b);
+    }
+    *reinterpret_cast<uint4*>(prow + (((c0 + q) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  return sum[0] + sum[1];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using Lay = Layout<D>;
+  constexpr int H = D / 64;  // 64-column halves of Q, K and V
+  constexpr float kNegInf = -INFINITY;
+  static_assert(D == 128, "the tcgen05 prefill kernel is built for head_dim 128");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = full + kStages;
+  uint64_t* s_full = empty + kStages;  // [2] S_i landed in TMEM buffer i & 1
+  uint64_t* s_free = s_full + 2;       // [2] the softmax warps have read it
+  uint64_t* p_full = s_free + 2;       // [2] P_i written to P buffer i & 1
+  uint64_t* pv_done = p_full + 2;      // [2] O += P_i V_i completed
+  uint64_t* mma_done = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int h = blockIdx.x;
+  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
+  const int b = blockIdx.z;
+  const int g = h / p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+
+  const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
+  if (!c.ok) {
+    if (h == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
+    return;
+  }
+  const int i0 = tile * kRows;
+  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
+  const int rows = min(kRows, c.n - i0);
+  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
+  const int npages = (kend + kPage - 1) / kPage;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_arrive_expect_tx(q_full, Lay::kQBytes);
+#pragma unroll
+      for (int hf = 0; hf < H; ++hf)
+        tma_load_2d(smem + hf * (kRows * 128), &tmQ, q_full, h * D + hf * 64, c.t0 + i0);
+      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      int issued = 0;
+      for (int i = 0; i < npages; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        int page = tbl[i];
+        if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
+          set_err(p.err, DF_DEVERR_BLOCK);
+          page = 0;
+        }
+        mbar_arrive_expect_tx(&full[st], Lay::kStageBytes);
+        const int row = (page * p.Hkv + g) * kPage;
+        uint8_t* sK = smem + Lay::kOffStages + st * Lay::kStageBytes;
+        uint8_t* sV = sK + Lay::kPageBytes;
+#pragma unroll
+        for (int hf = 0; hf < H; ++hf) {
+          tma_load_2d(sK + hf * kPage * 128, &tmK, &full[st], hf * 64, row);
+          tma_load_2d(sV + hf * kPage * 128, &tmV, &full[st], hf * 64, row);
+        }
+        ++issued;
+      }
+      // Leave no copy in flight (bounded waits).
+      mbar_wait(q_full, 0);
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = umma::make_idesc(kRows, kPage);                 // Q K^T
+      constexpr uint32_t kIdPV = umma::make_idesc(kRows, 64) | (1u << 16);      // P V, V MN-major
+      const uint32_t q_addr = smem_u32(smem);
+      bool ok = mbar_wait(q_full, 0);
+      auto issue_s = [&](int i) -> bool {
+        const int st = i % kStages, sb = i & 1;
+        if (!mbar_wait(&full[st], (i / kStages) & 1)) return false;
+        if (i >= 2 && !mbar_wait(&s_free[sb], ((i >> 1) - 1) & 1)) return false;
+        umma::tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk >> 2, kq = kk & 3;
+          umma::umma_bf16(tmem + sb * kPage,
+                          umma::smem_desc(q_addr + hf * (kRows * 128) + kq * 32),
+                          umma::smem_desc(k_addr + hf * (kPage * 128) + kq * 32), kIdS,
+                          kk > 0 ? 1u : 0u);
+        }
+        umma::umma_commit(&s_full[sb]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int i = 0; ok && i < npages; ++i) {
+        if (i + 1 < npages && !issue_s(i + 1)) {
+          ok = false;
+          break;
+        }
+        const int pb = i & 1, st = i % kStages;
+        if (!mbar_wait(&p_full[pb], (i >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        umma::tc_fence_after();
+        const uint32_t p_addr = smem_u32(smem + Lay::kOffP + pb * Lay::kPBytes);
+        const uint32_t v_addr =
+            smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes);
+#pragma unroll
+        for (int kk = 0; kk < kPage / 16; ++kk) {
+#pragma unroll
+          for (int hf = 0; hf < H; ++hf)
+            umma::umma_bf16(tmem + kOCol + hf * 64, umma::smem_desc(p_addr + kk * 32),
+                            smem_desc_mn64(v_addr + hf * (kPage * 128) + kk * 2048), kIdPV,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma::umma_commit(&pv_done[pb]);
+        umma::umma_commit(&empty[st]);
+      }
+      if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
+      umma::umma_commit(mma_done);  // completes when every MMA issued above has
+      mbar_wait(mma_done, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int quarter = warp & 3;  // this warp may access TMEM lanes 32 quarter .. + 31
+    const int r = quarter * 32 + lane;
+    const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint8_t* p_base = smem + Lay::kOffP + r * 128;
+    float m_ref = kNegInf, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < npages; ++i) {
+      const int sb = i & 1, st = i % kStages, kbase = i * kPage;
+      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      umma::tc_fence_after();
+      float s0[32], s1[32];
+      umma::tmem_ld<32>(t_lane + sb * kPage, s0);
+      umma::tmem_ld<32>(t_lane + sb * kPage + 32, s1);
+      umma::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+
+      if (kbase + kPage - 1 > pos) {  // causal mask (and keys past the chunk end)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (kbase + j > pos) s0[j] = kNegInf;
+          if (kbase + 32 + j > pos) s1[j] = kNegInf;
+        }
+      }
+      const float m_cand = fmaxf(max32(s0), max32(s1)) * p.scale_log2;
+      const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
+      if (m_ref == kNegInf) m_ref = m_cand;  // first page: O holds nothing yet
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold P_{i-1} V_{i-1} before it is rescaled in place.
+        if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        umma::tc_fence_after();
+        const float alpha = rescale ? exp2f(m_ref - m_cand) : 1.f;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          float o[32];
+          umma::tmem_ld<32>(t_lane + kOCol + cc, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_lane + kOCol + cc, o);
+        }
+        if (rescale) {
+          l *= alpha;
+          m_ref = m_cand;
+        }
+      }
+      const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
+
+      // P buffer sb is free once O += P_{i-2} V_{i-2} has completed.
+      if (i >= 2 && !mbar_wait_warp(&pv_done[sb], ((i >> 1) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = p_base + sb * Lay::kPBytes;
+      l += write_p32(prow, r, 0, s0, p.scale_log2, mu);
+      l += write_p32(prow, r, 4, s1, p.scale_log2, mu);
+
+      // Keys at or past kend on the last page hold other tokens' bytes
+      // (possibly NaN patterns): their weights are 0, and their V rows are
+      // zeroed, as 0 * NaN would still be NaN in the accumulator.
+      if (kbase + kPage > kend) {
+        if (!mbar_wait_warp(&full[st], (i / kStages) & 1)) {  // the page has landed
+          ok = false;
+          break;
+        }
+        const int kend_rel = kend - kbase;
+        uint8_t* sV = smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes;
+        const int nvec = (kPage - kend_rel) * H * 8;  // 16-byte chunks to clear
+        for (int v = r; v < nvec; v += kRows) {
+          const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
+          *reinterpret_cast<uint4*>(sV + hf * (kPage * 128) + row * 128 + ch * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // P (and cleared V rows) -> the tensor core's proxy
+      umma::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+    }
+    if (ok) {
+      const int last = npages - 1;
+      ok = mbar_wait_warp(&pv_done[last & 1], (last >> 1) & 1);
+    }
+    if (ok) {
+      umma::tc_fence_after();
+      __nv_bfloat16* orow =
+          p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t + h * D;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        float o[32];
+        umma::tmem_ld<32>(t_lane + kOCol + cc, o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
+        if (r < rows) umma::store_bf16<32>(orow + cc, o);
+      }
+    } else if (lane == 0) {
+      set_err(p.err, DF_DEVERR_TIMEOUT);
+    }
+  }
+
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace tc
+
 // ------------------------------------------------------------------ 3. last-row gather
 
 struct GatherParams {
@@ -480,6 +863,21 @@ cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* t
                     p);
 }
 
+cudaError_t launch_attn_tc(const AttnParams& p, int Hq, int B, const CUtensorMap* tmQ,
+                           const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
+  constexpr size_t smem = tc::Layout<128>::kSmem;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(tc::attn_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return launch_pdl(tc::attn_kernel<128>, dim3(Hq, p.tiles, B), dim3(tc::kThreads), smem, stream,
+                    *tmQ, *tmK, *tmV, p);
+}
+
 // Workspace of the auxiliary step: the decode workspace (its arrival counters
 // first), then the gathered last-position queries, then the attended lengths.
 struct WsLayout {
@@ -509,12 +907,24 @@ extern "C" int dualflow_prefill_num_launches(int with_append, int with_aux) {
   return (with_append ? 1 : 0) + 1 + (with_aux ? 2 : 0);
 }
 
-extern "C" df_status dualflow_prefill(
+// The tcgen05 attention kernel serves D = 128 with at least one full tile of
+// token rows and 16-byte aligned output rows; anything else takes the
+// mma.sync kernel.
+static bool tc_kernel_fits(int D, int T, const void* o1, int64_t o_stride_t) {
+  return D == 128 && T >= df::prefill::tc::kRows && df::aligned(o1, 16) && o_stride_t % 8 == 0;
+}
+
+extern "C" int dualflow_prefill_kernel(int D, int T, const void* o1, int64_t o_stride_t, int Hq) {
+  const int64_t os = o_stride_t ? o_stride_t : static_cast<int64_t>(Hq) * D;
+  return tc_kernel_fits(D, T, o1, os) ? DF_PREFILL_KERNEL_TCGEN05 : DF_PREFILL_KERNEL_MMA_SYNC;
+}
+
+extern "C" df_status dualflow_prefill_ex(
     const void* q1, int64_t q_stride_t, const void* k_new, const void* v_new, int64_t kv_stride_t,
     const void* q2raw, const void* a, void* k_cache, void* v_cache, const int32_t* block_table,
     int max_blocks_per_seq, const int32_t* cu_seqlens, const int32_t* ctx_lens, int max_q_len,
     int max_seqlen, void* o1, int64_t o_stride_t, void* o2, int B, int T, int Hq, int Hkv, int D,
-    int block_size, int num_blocks, float scale, int dtype, void* workspace,
+    int block_size, int num_blocks, float scale, int dtype, int kernel, void* workspace,
     size_t workspace_bytes, int32_t* err_flag, void* stream) {
   using namespace df;
   using namespace df::prefill;
@@ -545,6 +955,11 @@ extern "C" df_status dualflow_prefill(
     return DF_ERR_ALIGN;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return DF_ERR_ALIGN;
   if (aux && (!aligned(q2raw, 4) || (a && !aligned(a, 4)) || !aligned(o2, 4))) return DF_ERR_ALIGN;
+  if (kernel < DF_PREFILL_KERNEL_AUTO || kernel > DF_PREFILL_KERNEL_TCGEN05) return DF_ERR_SHAPE;
+  const bool tc_fits = tc_kernel_fits(D, T, o1, os);
+  if (kernel == DF_PREFILL_KERNEL_TCGEN05 && !tc_fits) return DF_ERR_UNSUPPORTED;
+  const bool use_tc = kernel == DF_PREFILL_KERNEL_TCGEN05 ||
+                      (kernel == DF_PREFILL_KERNEL_AUTO && tc_fits);
   WsLayout wl{};
   if (aux) {
     wl = ws_layout(B, Hq, Hkv, D, max_seqlen);
@@ -600,12 +1015,21 @@ extern "C" df_status dualflow_prefill(
   p.num_blocks = num_blocks;
   p.max_q_len = max_q_len;
   p.max_seqlen = max_seqlen;
-  p.tiles = tiles;
+  p.tiles = use_tc ? static_cast<int>(ceil_div(max_q_len, tc::kRows)) : tiles;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D));
   p.scale_log2 = sc * 1.4426950408889634f;
   p.err = err_flag;
-  cudaError_t e = (D == 64) ? launch_attn<64>(p, Hq, B, &tmK, &tmV, st)
-                            : launch_attn<128>(p, Hq, B, &tmK, &tmV, st);
+  cudaError_t e;
+  if (use_tc) {
+    CUtensorMap tmQ;  // token rows x (Hq * D) columns; boxes of 128 rows x 64 columns
+    if (!encode_tmap_bf16_2d(&tmQ, q1, static_cast<uint64_t>(T), static_cast<uint64_t>(Hq) * D,
+                             static_cast<uint64_t>(qs) * 2, tc::kRows, 64))
+      return DF_ERR_CUDA;
+    e = launch_attn_tc(p, Hq, B, &tmQ, &tmK, &tmV, st);
+  } else {
+    e = (D == 64) ? launch_attn<64>(p, Hq, B, &tmK, &tmV, st)
+                  : launch_attn<128>(p, Hq, B, &tmK, &tmV, st);
+  }
   if (e != cudaSuccess) return DF_ERR_CUDA;
   if (!aux) return DF_OK;
 
@@ -628,4 +1052,18 @@ extern "C" df_status dualflow_prefill(
                               max_blocks_per_seq, gp.seqlens, max_seqlen, nullptr, o2, 0, B, Hq,
                               Hkv, D, block_size, num_blocks, sc, DF_BF16, 0,
                               wl.decode ? workspace : nullptr, wl.decode, err_flag, stream);
+}
+
+extern "C" df_status dualflow_prefill(
+    const void* q1, int64_t q_stride_t, const void* k_new, const void* v_new, int64_t kv_stride_t,
+    const void* q2raw, const void* a, void* k_cache, void* v_cache, const int32_t* block_table,
+    int max_blocks_per_seq, const int32_t* cu_seqlens, const int32_t* ctx_lens, int max_q_len,
+    int max_seqlen, void* o1, int64_t o_stride_t, void* o2, int B, int T, int Hq, int Hkv, int D,
+    int block_size, int num_blocks, float scale, int dtype, void* workspace,
+    size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  return dualflow_prefill_ex(q1, q_stride_t, k_new, v_new, kv_stride_t, q2raw, a, k_cache, v_cache,
+                             block_table, max_blocks_per_seq, cu_seqlens, ctx_lens, max_q_len,
+                             max_seqlen, o1, o_stride_t, o2, B, T, Hq, Hkv, D, block_size,
+                             num_blocks, scale, dtype, DF_PREFILL_KERNEL_AUTO, workspace,
+                             workspace_bytes, err_flag, stream);
 }

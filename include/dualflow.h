@@ -225,6 +225,8 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
 /*             bound of every ctx_lens[b] + n_b, <= max_blocks_per_seq * 64. */
 /*             A chunk outside these bounds (or with n_b < 1, or rows past T)*/
 /*             sets DF_DEVERR_SEQLEN and is skipped (its rows unwritten).    */
+/*             A block_table entry outside [0, num_blocks) sets             */
+/*             DF_DEVERR_BLOCK; that sequence's outputs are then invalid.    */
 /* o1        : bf16 [T][Hq][D] at + t*o_stride_t (0 = Hq*D), 4-byte aligned. */
 /* o2        : bf16 [B][Hq][D] or NULL.                                      */
 /* workspace : only with the auxiliary step: 256-byte aligned, at least      */
@@ -237,6 +239,17 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
 /* ------------------------------------------------------------------------ */
 size_t dualflow_prefill_workspace_size(int B, int Hq, int Hkv, int D, int max_seqlen,
                                        int block_size);
+/* Attention kernel of a prefill call. DF_PREFILL_KERNEL_TCGEN05: tensor    */
+/* cores with TMEM accumulators, 128-row tiles; used (automatically) when    */
+/* D = 128, T >= 128, o1 is 16-byte aligned and o_stride_t % 8 == 0.          */
+/* DF_PREFILL_KERNEL_MMA_SYNC: warp-level mma.sync, 64-row tiles, any        */
+/* supported shape. Both compute the same result within the tolerance; the   */
+/* cache write and the auxiliary step are the same code.                     */
+#define DF_PREFILL_KERNEL_AUTO 0
+#define DF_PREFILL_KERNEL_MMA_SYNC 1
+#define DF_PREFILL_KERNEL_TCGEN05 2
+/* The kernel dualflow_prefill picks for these arguments (o_stride_t 0 = Hq*D). */
+int dualflow_prefill_kernel(int D, int T, const void* o1, int64_t o_stride_t, int Hq);
 int dualflow_prefill_num_launches(int with_append, int with_aux);
 df_status dualflow_prefill(const void* q1, int64_t q_stride_t, const void* k_new,
                            const void* v_new, int64_t kv_stride_t, const void* q2raw,
@@ -247,6 +260,18 @@ df_status dualflow_prefill(const void* q1, int64_t q_stride_t, const void* k_new
                            int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
                            int dtype, void* workspace, size_t workspace_bytes, int32_t* err_flag,
                            void* stream);
+/* The same call with the attention kernel chosen by the caller (kernel =   */
+/* DF_PREFILL_KERNEL_*; TCGEN05 where it does not fit: DF_ERR_UNSUPPORTED;  */
+/* another value: DF_ERR_SHAPE).                                             */
+df_status dualflow_prefill_ex(const void* q1, int64_t q_stride_t, const void* k_new,
+                              const void* v_new, int64_t kv_stride_t, const void* q2raw,
+                              const void* a, void* k_cache, void* v_cache,
+                              const int32_t* block_table, int max_blocks_per_seq,
+                              const int32_t* cu_seqlens, const int32_t* ctx_lens, int max_q_len,
+                              int max_seqlen, void* o1, int64_t o_stride_t, void* o2, int B,
+                              int T, int Hq, int Hkv, int D, int block_size, int num_blocks,
+                              float scale, int dtype, int kernel, void* workspace,
+                              size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Grouped shared-weight projection (tcgen05 tensor cores, TMEM accumulator).*/

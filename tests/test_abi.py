@@ -263,3 +263,18 @@ def test_prefill_sizes(lib):
     assert lib.dualflow_prefill_num_launches(1, 0) == 2
     assert lib.dualflow_prefill_workspace_size(2, 8, 2, 128, 400, 64) > 0
     assert lib.dualflow_prefill_workspace_size(2, 8, 2, 128, 400, 32) == 0
+
+
+def test_prefill_kernel_choice_is_checked(lib):
+    def ex(kernel, D=128, T=300, o1=FAKE):
+        return lib.dualflow_prefill_ex(FAKE, 0, FAKE, FAKE, 0, None, None, FAKE, FAKE, FAKE, 8,
+                                       FAKE, None, 256, 400, o1, 0, None, 2, T, 8, 2, D, 64, 16,
+                                       0.0, L.DF_BF16, kernel, None, 0, None, None)
+    assert ex(7) == L.DF_ERR_SHAPE
+    assert ex(L.DF_PREFILL_KERNEL_TCGEN05, D=64) == L.DF_ERR_UNSUPPORTED
+    assert ex(L.DF_PREFILL_KERNEL_TCGEN05, T=100, o1=FAKE) == L.DF_ERR_SHAPE  # max_q_len > T
+    assert ex(L.DF_PREFILL_KERNEL_TCGEN05, o1=FAKE + 4) == L.DF_ERR_UNSUPPORTED
+    assert lib.dualflow_prefill_kernel(128, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_TCGEN05
+    assert lib.dualflow_prefill_kernel(128, 100, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
+    assert lib.dualflow_prefill_kernel(64, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
+    assert lib.dualflow_prefill_kernel(128, 300, FAKE + 4, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC

@@ -64,17 +64,42 @@ def _check_all(inp, d, o1, o2, what):
     return r1, r2
 
 
+KERNELS = ["mma_sync", "tcgen05"]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("Hq,Hkv,D,lengths,ctx", [
     (8, 2, 128, (1, 63, 65, 200), (0, 37, 64, 130)),   # ragged chunks, prefixes, tile edges
     (16, 4, 64, (130, 7), (0, 0)),                     # D 64, 4 query heads per KV head
     (4, 4, 128, (256, 129), (0, 0)),                   # MHA, fresh prompts
     (6, 2, 128, (64, 128, 191), (1, 63, 0)),           # G = 3
+    (8, 2, 128, (127, 128, 129, 300), (0, 5, 200, 64)),  # 128-row tile edges
 ])
-def test_prefill_matches_oracle(cuda_device, Hq, Hkv, D, lengths, ctx):
+def test_prefill_matches_oracle(cuda_device, Hq, Hkv, D, lengths, ctx, kernel):
+    if kernel == "tcgen05" and D != 128:
+        pytest.skip("the tcgen05 prefill kernel is built for head_dim 128")
     inp = synth.make_prefill_inputs(_w(Hq=Hq, Hkv=Hkv, D=D), lengths=lengths, ctx=ctx)
     d = _dev(inp, cuda_device)
-    o1, o2 = _run(d)
-    _check_all(inp, d, o1, o2, "G=%d D=%d" % (Hq // Hkv, D))
+    o1, o2 = _run(d, kernel=kernel)
+    _check_all(inp, d, o1, o2, "%s G=%d D=%d" % (kernel, Hq // Hkv, D))
+
+
+def test_automatic_kernel_choice(cuda_device):
+    o1 = torch.empty((256, 8, 128), dtype=torch.bfloat16, device=cuda_device)
+    assert api.prefill_kernel(128, 256, o1, 8) == "tcgen05"
+    assert api.prefill_kernel(64, 256, o1[:, :, :64], 8) == "mma_sync"
+    assert api.prefill_kernel(128, 100, o1[:100], 8) == "mma_sync"
+
+
+def test_both_kernels_agree_within_tolerance(cuda_device):
+    inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(400, 250), ctx=(30, 0))
+    d = _dev(inp, cuda_device)
+    a1, a2 = _run(d, kernel="mma_sync")
+    b1, b2 = _run(d, kernel="tcgen05", append=False)
+    assert torch.equal(a2, b2)   # the auxiliary step is the same code
+    r1, _, _, _ = _oracle(inp)
+    assert_close(a1, r1, "bf16", "mma_sync O1")
+    assert_close(b1, r1, "bf16", "tcgen05 O1")
 
 
 def test_aux_output_is_the_decode_step_of_the_last_position(cuda_device):
@@ -104,7 +129,8 @@ def test_primary_output_ignores_aux_inputs_even_nan(cuda_device):
     assert torch.isnan(o2.float()).all()
 
 
-def test_stale_nan_slots_around_the_chunk_are_masked(cuda_device):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_stale_nan_slots_around_the_chunk_are_masked(cuda_device, kernel):
     """Every cache slot that is neither prefix nor chunk holds NaN: the tail
     of the last page must not leak into any output."""
     inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(37, 100, 1), ctx=(3, 0, 70))
@@ -119,12 +145,13 @@ def test_stale_nan_slots_around_the_chunk_are_masked(cuda_device):
             nan_v[page, :, slot] = vc[page, :, slot]
     inp["k_cache"], inp["v_cache"] = nan_k, nan_v
     d = _dev(inp, cuda_device)
-    o1, o2 = _run(d)
+    o1, o2 = _run(d, kernel=kernel)
     assert torch.isfinite(o1.float()).all() and torch.isfinite(o2.float()).all()
-    _check_all(inp, d, o1, o2, "NaN stale slots")
+    _check_all(inp, d, o1, o2, "%s NaN stale slots" % kernel)
 
 
-def test_chunked_prefill_equals_whole_prompt(cuda_device):
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_chunked_prefill_equals_whole_prompt(cuda_device, kernel):
     inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(300,), ctx=(0,))
     r1, r2, _, _ = _oracle(inp)
     d = _dev(inp, cuda_device)
@@ -132,12 +159,12 @@ def test_chunked_prefill_equals_whole_prompt(cuda_device):
     first = dict(d, q1=d["q1"][:m], k_new=d["k_new"][:m], v_new=d["v_new"][:m],
                  cu_seqlens=torch.tensor([0, m], dtype=torch.int32, device=cuda_device),
                  max_q_len=m)
-    a1, _ = _run(first, aux=False)
+    a1, _ = _run(first, aux=False, kernel=kernel)
     second = dict(d, q1=d["q1"][m:], k_new=d["k_new"][m:], v_new=d["v_new"][m:],
                   cu_seqlens=torch.tensor([0, 300 - m], dtype=torch.int32, device=cuda_device),
                   ctx_lens=torch.tensor([m], dtype=torch.int32, device=cuda_device),
                   max_q_len=300 - m)
-    a2, b2 = _run(second)
+    a2, b2 = _run(second, kernel=kernel)
     assert_close(torch.cat([a1, a2]), r1, "bf16", "chunked O1")
     assert_close(b2, r2, "bf16", "chunked O2")
 
@@ -174,13 +201,14 @@ def test_invalid_chunk_is_flagged_and_the_others_are_computed(cuda_device):
         assert_close(o2[b:b + 1], r2, "bf16", "sequence %d O2" % b)
 
 
-def test_out_of_range_page_is_flagged(cuda_device):
-    inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(100,), ctx=(0,))
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_out_of_range_page_is_flagged(cuda_device, kernel):
+    inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(200,), ctx=(0,))
     inp["block_table"] = inp["block_table"].clone()
     inp["block_table"][0, 1] = inp["num_blocks"] + 5
     d = _dev(inp, cuda_device)
     err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
-    _run(d, err=err)
+    _run(d, err=err, kernel=kernel)
     assert int(err.item()) & L.DF_DEVERR_BLOCK
     assert not int(err.item()) & L.DF_DEVERR_TIMEOUT
 
@@ -197,7 +225,7 @@ def test_full_size_prefill_sampled_rows(cuda_device):
     and sampled output rows against the oracle's attention of that row."""
     inp = synth.make_prefill_inputs(W)
     d = _dev(inp, cuda_device)
-    o1, o2 = _run(d)
+    o1, o2 = _run(d)   # automatic choice: the tcgen05 kernel at these sizes
     kc, vc = d["k_cache"].cpu(), d["v_cache"].cpu()
     tbl, cu = inp["block_table"], inp["cu_seqlens"].tolist()
     G = W.Hq // W.Hkv
