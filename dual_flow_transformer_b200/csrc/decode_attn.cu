@@ -746,28 +746,17 @@ cudaError_t launch(const Params& p, int dtype, const CUtensorMap* tmK, const CUt
   const dim3 grid(p.num_splits, p.Hkv, p.B);
   if (dtype == DF_BF16) {
     const size_t smem = bf16_smem_bytes<D>();
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(split_bf16_kernel<D, kStagesBf16>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
-    cudaError_t e = launch_pdl(split_bf16_kernel<D, kStagesBf16>, grid, dim3(kThreads), smem, stream,
-                               *tmK, *tmV, p);
+    cudaError_t e = ensure_dynamic_smem(
+        reinterpret_cast<const void*>(split_bf16_kernel<D, kStagesBf16>), smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(split_bf16_kernel<D, kStagesBf16>, grid, dim3(kThreads), smem, stream, *tmK,
+                   *tmV, p);
     if (e != cudaSuccess) return e;
   } else {
     const size_t smem = f32_smem_bytes<D>();
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(split_f32_kernel<D>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
-    cudaError_t e = launch_pdl(split_f32_kernel<D>, grid, dim3(128), smem, stream, p);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_f32_kernel<D>), smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(split_f32_kernel<D>, grid, dim3(128), smem, stream, p);
     if (e != cudaSuccess) return e;
     if (p.num_splits > 1) {
       e = launch_pdl(combine_kernel<float, D>, dim3(2 * p.Hq, p.B), dim3(D), 0, stream, p);

@@ -635,13 +635,9 @@ df_status grouped_proj_impl(const void* x, int64_t ldx, int m_primary, int m_aux
                            static_cast<uint64_t>(K) * 2,
                            epilogue == DF_EPI_SWIGLU ? kBN / 2 : kBN, kBK))
     return DF_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(grouped_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-      return DF_ERR_CUDA;
-    attr_set = true;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(grouped_proj_kernel), kSmemBytes) !=
+      cudaSuccess)
+    return DF_ERR_CUDA;
   if (launch_pdl(grouped_proj_kernel, dim3(l.ctas), dim3(kThreads), kSmemBytes, st, tmX, tmW, p) !=
       cudaSuccess)
     return DF_ERR_CUDA;

@@ -7,7 +7,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
+#include <vector>
 
 namespace df {
 
@@ -28,6 +30,24 @@ bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint
 bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t batch, uint64_t rows,
                          uint64_t cols, uint64_t row_pitch_bytes, uint64_t batch_pitch_bytes,
                          uint32_t box_rows, uint32_t box_cols);
+
+// Opt `kernel` into `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to the device, so it is set once per (kernel,
+// device) pair; later calls only look the pair up.
+inline cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == kernel && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  return e;
+}
 
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();

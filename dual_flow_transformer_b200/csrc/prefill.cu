@@ -852,13 +852,8 @@ template <int D>
 cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* tmK,
                         const CUtensorMap* tmV, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes<D>();
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(attn_kernel<D>), smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(attn_kernel<D>, dim3(Hq, p.tiles, B), dim3(kThreads), smem, stream, *tmK, *tmV,
                     p);
 }
@@ -866,14 +861,8 @@ cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* t
 cudaError_t launch_attn_tc(const AttnParams& p, int Hq, int B, const CUtensorMap* tmQ,
                            const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
   constexpr size_t smem = tc::Layout<128>::kSmem;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc::attn_kernel<128>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::attn_kernel<128>), smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(tc::attn_kernel<128>, dim3(Hq, p.tiles, B), dim3(tc::kThreads), smem, stream,
                     *tmQ, *tmK, *tmV, p);
 }

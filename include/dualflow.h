@@ -12,7 +12,11 @@
  * per-layer vector a_l, and attends to the primary K1/V1 without ever writing
  * the cache or feeding back into the primary flow. Because both flows share
  * the weights and the cache, one pass over each weight matrix and each KV page
- * can serve both ("grouped execution"). This library is that decode step.
+ * can serve both ("grouped execution"). This library is that decode step
+ * (attention, append, grouped projections, norms), the primary prefill that
+ * precedes it (the auxiliary flow joining at the last prompt position), the
+ * mixture head that combines both flows' next-token distributions, and the
+ * MoE MLP block with router replay.
  *
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller. The library
