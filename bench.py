@@ -42,6 +42,7 @@ METRIC = "dual-flow decode tokens/s and KV-read GB/s (% of B200 HBM peak), 1 GPU
 PREFILL_METRIC = ("primary prefill prompt tokens/s (one layer's causal attention, cache write "
                   "and last-position auxiliary query), 1 GPU")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, NVIDIA's nominal figure
 FALLBACK_BF16_TFLOPS = 1590.0
 CSRC = os.path.join(ROOT, "dual_flow_transformer_b200", "csrc")
 ATTN_SRC = os.path.join(CSRC, "decode_attn.cu")
@@ -1108,6 +1109,7 @@ def main(argv=None):
     if hasattr(run, "kv_bytes"):
         line["kv_read_gbs"] = run.kv_bytes / (attn_ms / 1e3) / 1e9
         line["kv_frac_of_hbm_peak"] = run.kv_bytes / (attn_ms / 1e3) / 1e9 / peak
+        line["kv_frac_of_nominal_8tbs"] = run.kv_bytes / (attn_ms / 1e3) / 1e9 / NOMINAL_HBM_GBS
     if hasattr(run, "mix_bytes"):
         mix_gbs = run.mix_bytes / (kernel_ms["mix"] / 1e3) / 1e9
         line["mixture_kernel"] = {"kernel": "dualflow_mixture_head", "bound": "hbm",
