@@ -196,3 +196,42 @@ def test_primary_prefill_ignores_aux_inputs_even_nan():
     assert np.array_equal(kc, nkc) and np.array_equal(vc, nvc)
     p1, p2, _, _ = oracle.prefill(**dict(args, q2raw=None))
     assert np.array_equal(o1, p1) and p2 is None
+
+
+def _golden_num(s):
+    table = {"sqrt2ln2": math.sqrt(2) * math.log(2), "sqrt2ln3": math.sqrt(2) * math.log(3)}
+    if s in table:
+        return table[s]
+    if "/" in s:
+        n, d = s.split("/")
+        return float(int(n)) / float(int(d))
+    return float(s)
+
+
+def _golden_arr(x):
+    return np.vectorize(_golden_num, otypes=[np.float64])(np.array(x, dtype=object))
+
+
+def test_golden_prefill_worked_example():
+    import json
+    import os
+    spec = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                       "prefill_worked_example.json")))
+    bs = spec["block_size"]
+    table = np.array(spec["block_table"])
+    kc = np.full((3, 1, bs, 2), 9.0)   # page 2 is spare: its marker must survive
+    vc = np.full((3, 1, bs, 2), 9.0)
+    for j, (kr, vr) in enumerate(zip(spec["cached_k"], spec["cached_v"])):
+        kc[table[0, j // bs], 0, j % bs] = _golden_arr(kr)
+        vc[table[0, j // bs], 0, j % bs] = _golden_arr(vr)
+    o1, o2, kc2, vc2 = oracle.prefill(
+        _golden_arr(spec["q1"]), _golden_arr(spec["k_new"]), _golden_arr(spec["v_new"]), kc, vc,
+        table, np.array(spec["cu_seqlens"]), np.array(spec["ctx_lens"]),
+        q2raw=_golden_arr(spec["q2raw"]), a=_golden_arr(spec["a"]))
+    np.testing.assert_allclose(o1, _golden_arr(spec["o1"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o2, _golden_arr(spec["o2"]), rtol=0, atol=1e-12)
+    for page, rows in spec["k_pages_after"].items():
+        np.testing.assert_array_equal(kc2[int(page), 0], _golden_arr(rows))
+    for page, rows in spec["v_pages_after"].items():
+        np.testing.assert_array_equal(vc2[int(page), 0], _golden_arr(rows))
+    assert (kc2[2] == 9.0).all() and (vc2[2] == 9.0).all()
