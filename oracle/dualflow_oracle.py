@@ -30,7 +30,9 @@ of the function that takes it:
   holds a prefix) is the plain extension of the causal mask.
 * Layer step      pre-attention and pre-MLP RMSNorm (unit gain, eps 1e-5),
   residual adds, SwiGLU MLP, no positional rotation.
-  PARITY UNPINNED against the pages (the pages name no norm, no MLP form).
+  PARITY UNPINNED against the pages (the pages name no norm, no MLP form);
+  the wiring of that reading (which tensor feeds which step) is pinned by a
+  hand-derived worked example with every intermediate in closed form.
 * MoE router replay  the auxiliary flow uses the primary router's expert
   set with its own gate weights (the pages' statement); the router matrix is
   shared, gates are the softmax of each flow's router logits over the set,
