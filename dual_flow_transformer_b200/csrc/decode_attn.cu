@@ -31,7 +31,11 @@
 //    bit-identical whatever the auxiliary inputs are.
 #include <math.h>
 
+#include <cudaTypedefs.h>
+
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "host_util.h"
@@ -795,12 +799,18 @@ extern "C" size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, in
   return df::attn::ws_layout(B, Hq, Hkv, D, pl.splits).total();
 }
 
-extern "C" df_status dualflow_decode_attn(
+namespace {
+
+// Both entry points: every argument check first, then (only for the no-alloc
+// entry point, clear_counters) the clearing of the bf16 arrival counters, then
+// the launch. A call rejected by a check has issued no device work.
+df_status decode_attn_impl(
     const void* q1, const void* q2raw, const void* a, int64_t q_stride_b, const void* k_cache,
     const void* v_cache, const int32_t* block_table, int max_blocks_per_seq,
     const int32_t* seqlens, int max_seqlen, void* o1, void* o2, int64_t o_stride_b, int B, int Hq,
     int Hkv, int D, int block_size, int num_blocks, float scale, int dtype, int num_splits,
-    void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream) {
+    void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream,
+    bool clear_counters) {
   using namespace df;
   if (!q1 || !k_cache || !v_cache || !block_table || !seqlens) return DF_ERR_NULL;
   const bool want2 = (o2 != nullptr) && (q2raw != nullptr);
@@ -875,9 +885,27 @@ extern "C" df_status dualflow_decode_attn(
       return DF_ERR_CUDA;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (clear_counters && dtype == DF_BF16 && pl.splits > 1) {
+    const size_t counters = attn::ws_layout(B, Hq, Hkv, D, pl.splits).counters;
+    if (cudaMemsetAsync(p.counters, 0, counters, st) != cudaSuccess) return DF_ERR_CUDA;
+  }
   cudaError_t e = (D == 64) ? attn::launch<64>(p, dtype, &tmK, &tmV, st)
                             : attn::launch<128>(p, dtype, &tmK, &tmV, st);
   return e == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" df_status dualflow_decode_attn(
+    const void* q1, const void* q2raw, const void* a, int64_t q_stride_b, const void* k_cache,
+    const void* v_cache, const int32_t* block_table, int max_blocks_per_seq,
+    const int32_t* seqlens, int max_seqlen, void* o1, void* o2, int64_t o_stride_b, int B, int Hq,
+    int Hkv, int D, int block_size, int num_blocks, float scale, int dtype, int num_splits,
+    void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  return decode_attn_impl(q1, q2raw, a, q_stride_b, k_cache, v_cache, block_table,
+                          max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq, Hkv,
+                          D, block_size, num_blocks, scale, dtype, num_splits, workspace,
+                          workspace_bytes, err_flag, stream, false);
 }
 
 // ------------------------------------------------------------------ no-alloc variant
@@ -894,21 +922,65 @@ namespace noalloc {
 
 static __device__ __align__(256) uint8_t g_scratch[DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_mu;
-void* g_addr[64] = {};  // device address of g_scratch, per device ordinal
+// The array's device address belongs to a CUDA context (the module is loaded
+// into each context separately): after a device reset, or under another
+// driver-API context, the same device ordinal has a different address. So
+// the looked-up address is cached per context, keyed by the context's unique
+// id (never reused within a process), not per device ordinal.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_fn_once;
 
-// Device address of the scratch array on the current device; looked up once
-// per device (with that device current) and cached.
+void load_ctx_fns() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) ==
+          cudaSuccess && q == cudaDriverEntryPointSuccess)
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  fn = nullptr;
+  q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess && q == cudaDriverEntryPointSuccess)
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+}
+
+// Unique id of the calling thread's current context; 0 if there is none or
+// the driver cannot say.
+unsigned long long current_ctx_id() {
+  std::call_once(g_fn_once, load_ctx_fns);
+  if (!g_ctx_current || !g_ctx_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+std::mutex g_mu;
+std::vector<std::pair<unsigned long long, void*>> g_addr;  // (context id, address)
+
+// Device address of the scratch array in the current context: looked up with
+// cudaGetSymbolAddress the first time a context calls (which also loads the
+// module there, so make that first call before any stream capture), then
+// taken from the cache. Without a context id the lookup runs on every call.
 df_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return DF_ERR_CUDA;
-    g_addr[dev] = p;
+  unsigned long long id = current_ctx_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (const auto& e : g_addr)
+      if (e.first == id) {
+        *out = e.second;
+        return DF_OK;
+      }
   }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return DF_ERR_CUDA;
+  if (id == 0) id = current_ctx_id();  // the lookup made the primary context current
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_addr.emplace_back(id, p);
+  }
+  *out = p;
   return DF_OK;
 }
 
@@ -930,17 +1002,12 @@ extern "C" df_status dualflow_decode_attn_noalloc(
   if (need > 0) {
     const df_status st = df::noalloc::scratch_address(&scratch);
     if (st != DF_OK) return st;
-    // the bf16 arrival counters (start of the layout) must start at zero
-    if (dtype == DF_BF16) {
-      const df::attn::Plan pl = make_plan(B, Hkv, max_seqlen, block_size, num_splits);
-      const size_t counters = df::attn::ws_layout(B, Hq, Hkv, D, pl.splits).counters;
-      if (cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return DF_ERR_CUDA;
-    }
   }
-  return dualflow_decode_attn(q1, q2raw, a, q_stride_b, k_cache, v_cache, block_table,
-                              max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq,
-                              Hkv, D, block_size, num_blocks, scale, dtype, num_splits, scratch,
-                              need > 0 ? DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES : 0, err_flag,
-                              stream);
+  // the counters at the start of the scratch are cleared after the argument
+  // checks, just before the launch (bf16 split calls only)
+  return decode_attn_impl(q1, q2raw, a, q_stride_b, k_cache, v_cache, block_table,
+                          max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq, Hkv,
+                          D, block_size, num_blocks, scale, dtype, num_splits, scratch,
+                          need > 0 ? DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES : 0, err_flag, stream,
+                          true);
 }

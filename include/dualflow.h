@@ -155,14 +155,18 @@ df_status dualflow_decode_attn(const void* q1, const void* q2raw, const void* a,
 /*  - A request whose workspace would exceed that size (see                  */
 /*    dualflow_decode_attn_workspace_size) returns DF_ERR_WORKSPACE before    */
 /*    any launch.                                                            */
-/*  - The first call on a device looks up the array's device address with    */
-/*    that device current (cudaGetSymbolAddress) and caches it; make that    */
-/*    first call before any stream capture. A failed lookup: DF_ERR_CUDA.    */
+/*  - The array's device address belongs to a CUDA context. The first call  */
+/*    made in a context (the device's primary context, or a driver-API       */
+/*    context made current by the caller; again after a device reset) looks  */
+/*    it up with cudaGetSymbolAddress, which also loads the library's module */
+/*    there, and caches it under the context's unique id; make that first   */
+/*    call before any stream capture. A failed lookup: DF_ERR_CUDA.          */
 /*  - All calls on a device share the one array, which keeps the last call's */
-/*    contents. A bf16 call first clears, on its stream, the part that must  */
-/*    start at zero (the arrival counters; cudaMemsetAsync, no allocation).  */
-/*    Calls that overlap on the GPU (different streams, no ordering) race on */
-/*    it: order them.                                                        */
+/*    contents. After every argument check has passed, a bf16 call that      */
+/*    splits clears, on its stream, the part that must start at zero (the    */
+/*    arrival counters; cudaMemsetAsync, no allocation). A rejected call     */
+/*    touches nothing. Calls that overlap on the GPU (different streams, no  */
+/*    ordering) race on the array: order them.                              */
 /* ------------------------------------------------------------------------ */
 #define DF_DECODE_ATTN_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 df_status dualflow_decode_attn_noalloc(const void* q1, const void* q2raw, const void* a,
