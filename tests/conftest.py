@@ -19,3 +19,18 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected but no CUDA device is visible")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """One line per full-size parity comparison: the observed errors."""
+    try:
+        from tests.helpers import PARITY_LOG
+    except Exception:
+        return
+    rows = [e for e in PARITY_LOG if e[0].startswith("full ")]
+    if not rows:
+        return
+    terminalreporter.write_line("parity at full size (max-abs, max row-relative error):")
+    for what, mx, rel in rows:
+        terminalreporter.write_line("  %-28s max-abs %.3e%s" % (
+            what, mx, "" if rel is None else "  row-rel %.3e" % rel))

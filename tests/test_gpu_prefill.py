@@ -14,7 +14,7 @@ import torch
 import oracle
 from dual_flow_transformer_b200 import api, synth
 from dual_flow_transformer_b200 import _lib as L
-from tests.helpers import assert_close
+from tests.helpers import assert_attn_close
 
 pytestmark = pytest.mark.gpu
 
@@ -55,9 +55,9 @@ def _oracle(inp, aux=True):
 
 def _check_all(inp, d, o1, o2, what):
     r1, r2, kc, vc = _oracle(inp, aux=o2 is not None)
-    assert_close(o1, r1, "bf16", what + " O1")
+    assert_attn_close(o1, r1, "bf16", what + " O1")
     if o2 is not None:
-        assert_close(o2, r2, "bf16", what + " O2")
+        assert_attn_close(o2, r2, "bf16", what + " O2")
     # byte copies: equal values, NaN slots (stale-slot tests) equal as NaN
     assert np.array_equal(f32(d["k_cache"]), kc, equal_nan=True), what + ": K cache differs"
     assert np.array_equal(f32(d["v_cache"]), vc, equal_nan=True), what + ": V cache differs"
@@ -98,8 +98,8 @@ def test_both_kernels_agree_within_tolerance(cuda_device):
     b1, b2 = _run(d, kernel="tcgen05", append=False)
     assert torch.equal(a2, b2)   # the auxiliary step is the same code
     r1, _, _, _ = _oracle(inp)
-    assert_close(a1, r1, "bf16", "mma_sync O1")
-    assert_close(b1, r1, "bf16", "tcgen05 O1")
+    assert_attn_close(a1, r1, "bf16", "mma_sync O1")
+    assert_attn_close(b1, r1, "bf16", "tcgen05 O1")
 
 
 def test_aux_output_is_the_decode_step_of_the_last_position(cuda_device):
@@ -114,8 +114,8 @@ def test_aux_output_is_the_decode_step_of_the_last_position(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(d2, o2)          # the same kernel on the same cache
     r1, _, _, _ = _oracle(inp)
-    assert_close(d1, r1[last.numpy()], "bf16", "decode O1 at the last position")
-    assert_close(o1[last.to(cuda_device)], r1[last.numpy()], "bf16", "prefill O1 last rows")
+    assert_attn_close(d1, r1[last.numpy()], "bf16", "decode O1 at the last position")
+    assert_attn_close(o1[last.to(cuda_device)], r1[last.numpy()], "bf16", "prefill O1 last rows")
 
 
 def test_primary_output_ignores_aux_inputs_even_nan(cuda_device):
@@ -165,8 +165,8 @@ def test_chunked_prefill_equals_whole_prompt(cuda_device, kernel):
                   ctx_lens=torch.tensor([m], dtype=torch.int32, device=cuda_device),
                   max_q_len=300 - m)
     a2, b2 = _run(second, kernel=kernel)
-    assert_close(torch.cat([a1, a2]), r1, "bf16", "chunked O1")
-    assert_close(b2, r2, "bf16", "chunked O2")
+    assert_attn_close(torch.cat([a1, a2]), r1, "bf16", "chunked O1")
+    assert_attn_close(b2, r2, "bf16", "chunked O2")
 
 
 def test_without_append_reads_the_cached_chunk(cuda_device):
@@ -197,8 +197,8 @@ def test_invalid_chunk_is_flagged_and_the_others_are_computed(cuda_device):
                    cu_seqlens=torch.tensor([0, t1 - t0], dtype=torch.int32),
                    ctx_lens=inp["ctx_lens"][b:b + 1])
         r1, r2, _, _ = _oracle(one)
-        assert_close(o1[t0:t1], r1, "bf16", "sequence %d O1" % b)
-        assert_close(o2[b:b + 1], r2, "bf16", "sequence %d O2" % b)
+        assert_attn_close(o1[t0:t1], r1, "bf16", "sequence %d O1" % b)
+        assert_attn_close(o2[b:b + 1], r2, "bf16", "sequence %d O2" % b)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
@@ -243,7 +243,7 @@ def test_full_size_prefill_sampled_rows(cuda_device):
                 K = f32(inp["k_new"][t0:t + 1, g])
                 V = f32(inp["v_new"][t0:t + 1, g])
                 ref = oracle.attn_weights(f32(inp["q1"][t, h])[None], K, scale) @ V
-                assert_close(o1[t, h][None], ref, "bf16", "row b=%d i=%d h=%d" % (b, i, h))
+                assert_attn_close(o1[t, h][None], ref, "bf16", "row b=%d i=%d h=%d" % (b, i, h))
         last = t0 + n - 1
         q2 = oracle.couple_query(f32(inp["q1"][last])[None], f32(inp["q2raw"][b])[None],
                                  f32(inp["a"]))[0]
@@ -252,4 +252,4 @@ def test_full_size_prefill_sampled_rows(cuda_device):
             K = f32(inp["k_new"][t0:last + 1, g])
             V = f32(inp["v_new"][t0:last + 1, g])
             ref = oracle.attn_weights(q2[h][None], K, scale) @ V
-            assert_close(o2[b, h][None], ref, "bf16", "aux b=%d h=%d" % (b, h))
+            assert_attn_close(o2[b, h][None], ref, "bf16", "aux b=%d h=%d" % (b, h))
