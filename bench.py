@@ -31,7 +31,6 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -112,54 +111,100 @@ def traffic_from_profile(workload, prefix="decode_attn", src=ATTN_SRC):
         return None
 
 
-class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+_SAMPLER_SRC = r"""
+import sys, time
+import pynvml as N
+pynvml_bus, idx = sys.argv[1], int(sys.argv[2])
+N.nvmlInit()
+try:
+    h = N.nvmlDeviceGetHandleByPciBusId(pynvml_bus) if pynvml_bus else N.nvmlDeviceGetHandleByIndex(idx)
+except Exception:
+    h = N.nvmlDeviceGetHandleByIndex(idx)
+smax = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+print("ready %d" % smax, flush=True)
+while True:
+    t = time.time()
+    sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+    try:
+        r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+    except Exception:
+        r = N.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+    print("%.6f %d %d" % (t, sm, r), flush=True)
+    time.sleep(0.002)
+"""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+# NVML clock-event reason bits (nvml.h)
+_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled by NVML every ~2 ms from a
+    separate process (read-only queries), kept only for the host-time window
+    that brackets the timed GPU work (start() ... stop())."""
+
+    def __init__(self, device):
+        self.device = device
         self.proc = None
-        self.file = None
+        self.smax = None
+        self.t0 = self.t1 = None
 
     def start(self):
+        import torch
+        bus = ""
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.file, stderr=subprocess.DEVNULL)
+            pr = torch.cuda.get_device_properties(self.device)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        except Exception:
+            pass
+        idx = self.device.index or 0
+        try:
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, bus, str(idx)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            line = self.proc.stdout.readline().split()
+            self.smax = float(line[1]) if len(line) == 2 and line[0] == "ready" else None
+            if self.smax is None:
+                self.proc.kill()
+                self.proc = None
         except Exception:
             self.proc = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def stop(self):
+        """{"sm_mhz": median, "sm_max_mhz", "reasons", "samples", "window_ms"}
+        over the timed window, or a record saying why there is none."""
         if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.file.flush()
-        self.file.seek(0)
-        rows = [r.strip().split(",") for r in self.file.read().splitlines() if r.strip()]
-        os.unlink(self.file.name)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML sampler unavailable"}
+        self.proc.kill()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, reasons = [], set()
+        for row in out.splitlines():
+            f = row.split()
             try:
-                sm.append(float(r[1]))
-                smax = float(r[2])
-                for n, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
+                t, mhz, bits = float(f[0]), float(f[1]), int(f[2])
             except (IndexError, ValueError):
                 continue
+            if self.t0 is None or self.t1 is None or not (self.t0 <= t <= self.t1):
+                continue
+            sm.append(mhz)
+            for name, bit in _REASON_BITS.items():
+                if bits & bit:
+                    reasons.add(name)
+        rec = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+               "reasons": sorted(reasons), "samples": len(sm),
+               "window_ms": None if self.t0 is None else round((self.t1 - self.t0) * 1e3, 2),
+               "how": "NVML every ~2 ms from a separate process, host-time window around the "
+                      "timed passes"}
         if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            rec["note"] = "no sample fell inside the timed window"
+        return rec
 
 
 def dist_setup(args):
@@ -674,6 +719,7 @@ class PrefillRun:
 # ----------------------------------------------------------------------------- oracle timing
 
 def _threads_used():
+    """Threads the oracle's BLAS uses (its pool size), else the usable cores."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
@@ -682,6 +728,24 @@ def _threads_used():
     except Exception:
         pass
     return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline_record(run, workload, budget_s):
+    """The oracle timed on the host: once with the BLAS pool as it stands and
+    once limited to one thread (half the budget)."""
+    v, sample, el, steps = time_oracle(run, workload, budget_s)
+    rec = {"value": v, "unit": "tokens/s", "cores": _threads_used(),
+           "usable_cores": len(os.sched_getaffinity(0)), "blas_threads": _threads_used(),
+           "kind": "oracle", "sample": sample, "seconds": round(el, 2)}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, sample1, el1, _ = time_oracle(run, workload, budget_s / 2)
+        rec["one_thread"] = {"value": v1, "unit": "tokens/s", "blas_threads": 1,
+                             "sample": sample1, "seconds": round(el1, 2)}
+    except Exception as e:  # threadpoolctl missing: say so, do not guess
+        rec["one_thread"] = {"value": None, "note": "not measured: %s" % e}
+    return rec
 
 
 def oracle_layer_sample(host, n_seq):
@@ -980,11 +1044,12 @@ def main(argv=None):
     keys = getattr(run, "timer_keys", ("attn",))
     timers = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for k in keys} for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
     if not args.no_clocks and rank == 0:
         clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark_start()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for i in range(args.steps):
@@ -1000,6 +1065,7 @@ def main(argv=None):
     for i in range(args.steps):
         run.step(timers=timers[i])
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier(world)
     clk = clocks.stop() if (not args.no_clocks and rank == 0) else None
     kernel_ms = {k: max_over_ranks(sum(t[k][0].elapsed_time(t[k][1]) for t in timers) / args.steps,
@@ -1055,9 +1121,7 @@ def main(argv=None):
     # ---------------------------------------------------------------- CPU baseline (oracle)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, el, steps = time_oracle(run, args.workload, args.cpu_budget_s)
-        cpu = {"value": v, "unit": "tokens/s", "cores": _threads_used(), "kind": "oracle",
-               "sample": sample, "seconds": round(el, 2)}
+        cpu = cpu_baseline_record(run, args.workload, args.cpu_budget_s)
 
     if rank != 0:
         if world > 1:
@@ -1116,8 +1180,6 @@ def main(argv=None):
                                   "ms_per_launch": kernel_ms["mix"], "achieved": mix_gbs,
                                   "peak": peak, "unit": "GB/s", "frac": mix_gbs / peak,
                                   "algorithmic_bytes_per_launch": run.mix_bytes}
-    if clk is None and not args.no_clocks:
-        line["clocks"] = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
