@@ -468,7 +468,7 @@ def mixture_head(logits, B):
 
 # ----------------------------------------------------------------- MoE router replay
 
-def moe_route(x1, x2, w_router, k, k_aux=None):
+def moe_route(x1, x2, w_router, k, k_aux=None, ids=None):
     """Expert selection and gate weights of both flows (router replay).
 
     "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi Chiave"
@@ -485,17 +485,26 @@ def moe_route(x1, x2, w_router, k, k_aux=None):
         g1 = softmax(r_1[ids[:k]]), g2 = softmax(r_2[ids[:k_aux]]).
     x1, x2: [B][d]; w_router: [E][d]. Returns (ids int [B][k_aux],
     g1 [B][k], g2 [B][k_aux], r1 [B][E], r2 [B][E]), fp64.
+
+    ids (optional, int [B][k_aux]): a selection made elsewhere, used as
+    given instead of this function's own ranking. Where two logits are closer
+    than the rounding of another implementation's arithmetic, several
+    selections are equally correct; the gates and outputs of that selection
+    are then checked with the same formulas.
     """
     k_aux = k if k_aux is None else k_aux
     w = np.asarray(w_router, dtype=F64)
     r1 = np.asarray(x1, dtype=F64) @ w.T
     r2 = np.asarray(x2, dtype=F64) @ w.T
     B, E = r1.shape
-    ids = np.zeros((B, k_aux), dtype=np.int64)
-    for t in range(B):
-        # stable sort of (-logit, index): descending logit, lower index first on ties
-        order = sorted(range(E), key=lambda e: (-r1[t, e], e))
-        ids[t] = order[:k_aux]
+    if ids is not None:
+        ids = np.asarray(ids, dtype=np.int64).reshape(B, k_aux)
+    else:
+        ids = np.zeros((B, k_aux), dtype=np.int64)
+        for t in range(B):
+            # stable sort of (-logit, index): descending logit, lower index first on ties
+            order = sorted(range(E), key=lambda e: (-r1[t, e], e))
+            ids[t] = order[:k_aux]
     g1 = softmax_rows(np.take_along_axis(r1, ids[:, :k], axis=1))
     g2 = softmax_rows(np.take_along_axis(r2, ids, axis=1))
     return ids, g1, g2, r1, r2
@@ -517,14 +526,15 @@ def moe_expert(x, w_gu, w_down, round_bf16=True):
 
 
 def moe_forward(x1, x2, w_router, w_gu, w_down, k, k_aux=None, residual1=None,
-                residual2=None, round_bf16=True):
+                residual2=None, round_bf16=True, ids=None):
     """MoE MLP block of both flows with router replay:
         y1[t] = sum_j g1[t][j] E_{ids[t][j]}(x1[t])       (j < k)
         y2[t] = sum_j g2[t][j] E_{ids[t][j]}(x2[t])       (j < k_aux)
     plus the residual when given, rounded once to bf16 (round_bf16).
-    w_gu: [E][2F][d], w_down: [E][d][F]. Returns (y1, y2, ids, g1, g2)."""
+    w_gu: [E][2F][d], w_down: [E][d][F]. Returns (y1, y2, ids, g1, g2).
+    ids: an expert selection to use as given (see ``moe_route``)."""
     k_aux = k if k_aux is None else k_aux
-    ids, g1, g2, _, _ = moe_route(x1, x2, w_router, k, k_aux)
+    ids, g1, g2, _, _ = moe_route(x1, x2, w_router, k, k_aux, ids=ids)
     x1 = np.asarray(x1, dtype=F64)
     x2 = np.asarray(x2, dtype=F64)
     B, d = x1.shape

@@ -6,8 +6,11 @@ oracle only.
 Expert selection is an integer decision taken from router logits: both sides
 compute the logits (the GPU in fp32, the oracle in fp64) and the ids are
 compared exactly wherever the oracle's margin between consecutive ranks
-exceeds fp32 rounding; tokens with a closer call are checked for validity
-instead (every GPU choice within that margin of the oracle's ranking).
+exceeds fp32 rounding. Tokens with a closer call are checked for validity
+instead: the GPU's ids must be a descending ranking of the oracle's logits
+up to that margin, with no excluded expert clearly above a chosen one, and
+their gates and block outputs must match the oracle evaluated on the GPU's
+own ids.
 """
 
 import numpy as np
@@ -66,11 +69,29 @@ def test_route_parity(cuda_device, B, d, E, k, k_aux):
     np.testing.assert_array_equal(got[ok], r_ids[ok])
     np.testing.assert_allclose(g1.cpu().numpy()[ok], r_g1[ok], rtol=0, atol=1e-5)
     np.testing.assert_allclose(g2.cpu().numpy()[ok], r_g2[ok], rtol=0, atol=1e-5)
-    # undecided tokens: the GPU's choices are still a valid top-k_aux within the margin
-    for t in np.nonzero(~ok)[0]:
-        kth = -np.sort(-r1[t])[k_aux - 1]
-        assert (r1[t, got[t]] >= kth - MARGIN).all()
-        assert len(set(got[t].tolist())) == k_aux
+    # every token: the GPU's choices are a valid ranking within the margin,
+    # and the gates are the oracle's on those very ids
+    _assert_valid_ranking(got, r1, k_aux)
+    _, o_g1, o_g2, _, _ = oracle.moe_route(_f64(x[:B]), _f64(x[B:]), _f64(w_r), k, k_aux,
+                                           ids=got)
+    np.testing.assert_allclose(g1.cpu().numpy(), o_g1, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(g2.cpu().numpy(), o_g2, rtol=0, atol=1e-5)
+
+
+def _assert_valid_ranking(got, r1, k_aux):
+    """ids[t] is a top-k_aux of the logits r1[t] in descending order, up to
+    MARGIN: distinct experts, each chosen one at least the next chosen one
+    minus MARGIN, and no excluded expert above the last chosen one plus
+    MARGIN."""
+    B, E = r1.shape
+    for t in range(B):
+        sel = got[t].tolist()
+        assert len(set(sel)) == k_aux and all(0 <= e < E for e in sel), (t, sel)
+        vals = r1[t, sel]
+        assert (vals[:-1] >= vals[1:] - MARGIN).all(), (t, sel, vals)
+        rest = [e for e in range(E) if e not in sel]
+        if rest:
+            assert r1[t, rest].max() <= vals.min() + MARGIN, (t, sel)
 
 
 def test_dispatch_packs_rows_bit_exact(cuda_device):
@@ -111,15 +132,20 @@ def test_moe_block_parity(cuda_device, B, d, F, E, k, k_aux):
     x, w_r, w_gu, w_down = _case(120 + B, B, d, F, E)
     g = torch.Generator().manual_seed(121)
     res = _bf(g, (2 * B, d))
-    y, _ = _block(cuda_device, x, w_r, w_gu, w_down, k, k_aux, B, residual=res)
-    r1, r2, r_ids, _, _ = oracle.moe_forward(_f64(x[:B]), _f64(x[B:]), _f64(w_r), _f64(w_gu),
-                                             _f64(w_down), k, k_aux, _f64(res[:B]), _f64(res[B:]))
-    _, _, _, rl1, _ = oracle.moe_route(_f64(x[:B]), _f64(x[B:]), _f64(w_r), k, k_aux)
+    y, moe = _block(cuda_device, x, w_r, w_gu, w_down, k, k_aux, B, residual=res)
+    got = moe.ids.cpu().numpy()
+    o_ids, _, _, rl1, _ = oracle.moe_route(_f64(x[:B]), _f64(x[B:]), _f64(w_r), k, k_aux)
     ok = _decided(rl1, k_aux)
     assert ok.sum() >= B - 2
-    ok2 = np.concatenate([ok, ok])
+    # decided tokens: the GPU chose the oracle's ids; every token: a valid ranking
+    np.testing.assert_array_equal(got[ok], o_ids[ok])
+    _assert_valid_ranking(got, rl1, k_aux)
+    # every token's output against the oracle block on the GPU's own selection
+    r1, r2, _, _, _ = oracle.moe_forward(_f64(x[:B]), _f64(x[B:]), _f64(w_r), _f64(w_gu),
+                                         _f64(w_down), k, k_aux, _f64(res[:B]), _f64(res[B:]),
+                                         ids=got)
     ref = np.concatenate([r1, r2])
-    assert_close(y[torch.from_numpy(ok2)], ref[ok2], "bf16", "moe block B=%d d=%d E=%d" % (B, d, E))
+    assert_close(y, ref, "bf16", "moe block B=%d d=%d E=%d" % (B, d, E))
 
 
 def test_primary_blind_to_aux_and_identical_flows(cuda_device):

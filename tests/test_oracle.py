@@ -569,3 +569,29 @@ def test_moe_limits_reduce_to_the_dense_mlp():
     h = oracle.swiglu_couple(gu, wgu.shape[1] // 2, x1.shape[0])
     dense = oracle.grouped_proj(h, wd[0], x1.shape[0])
     np.testing.assert_allclose(np.concatenate([y1, y2]), dense, rtol=1e-12, atol=1e-12)
+
+
+def test_moe_given_selection():
+    # The selection passed in replaces the oracle's own ranking: its own ids
+    # reproduce every output bit for bit; the same set in another order
+    # permutes the gates with it and leaves each flow's sum over the set as it
+    # was; a different set changes the outputs.
+    x1, x2, wr, wgu, wd = _moe_case(93)
+    y1, y2, ids, g1, g2 = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 2, round_bf16=False)
+    z1, z2, jds, h1, h2 = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 2, round_bf16=False, ids=ids)
+    for a, b in ((y1, z1), (y2, z2), (ids, jds), (g1, h1), (g2, h2)):
+        np.testing.assert_array_equal(a, b)
+    swapped = ids[:, ::-1].copy()
+    s1, s2, _, sg1, sg2 = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 2, round_bf16=False,
+                                             ids=swapped)
+    np.testing.assert_allclose(sg1, g1[:, ::-1], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(sg2, g2[:, ::-1], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(s1, y1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s2, y2, rtol=1e-12, atol=1e-12)
+    other = ids.copy()
+    other[:, 1] = [next(e for e in range(5) if e not in ids[t]) for t in range(ids.shape[0])]
+    o1, _, _, og1, _ = oracle.moe_forward(x1, x2, wr, wgu, wd, 2, 2, round_bf16=False, ids=other)
+    assert np.abs(o1 - y1).max() > 1e-3
+    r1 = x1 @ wr.T
+    np.testing.assert_allclose(og1, oracle.softmax_rows(np.take_along_axis(r1, other, axis=1)),
+                               rtol=0, atol=1e-15)
