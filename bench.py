@@ -130,7 +130,6 @@ while True:
     except Exception:
         r = N.nvmlDeviceGetCurrentClocksThrottleReasons(h)
     print("%.6f %d %d" % (t, sm, r), flush=True)
-    time.sleep(0.002)
 """
 
 # NVML clock-event reason bits (nvml.h)
@@ -139,9 +138,10 @@ _REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 
 
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled by NVML every ~2 ms from a
-    separate process (read-only queries), kept only for the host-time window
-    that brackets the timed GPU work (start() ... stop())."""
+    """SM clock and clock-event reasons sampled by NVML back to back (each
+    sample is two read-only queries) from a separate process, kept only for
+    the host-time window that brackets the timed GPU work (start() ...
+    stop())."""
 
     def __init__(self, device):
         self.device = device
@@ -200,8 +200,8 @@ class ClockSampler:
         rec = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
                "reasons": sorted(reasons), "samples": len(sm),
                "window_ms": None if self.t0 is None else round((self.t1 - self.t0) * 1e3, 2),
-               "how": "NVML every ~2 ms from a separate process, host-time window around the "
-                      "timed passes"}
+               "how": "NVML queries back to back from a separate process, host-time window "
+                      "around the timed passes"}
         if not sm:
             rec["note"] = "no sample fell inside the timed window"
         return rec
