@@ -31,6 +31,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -114,7 +115,7 @@ def traffic_from_profile(workload, prefix="decode_attn", src=ATTN_SRC):
 _SAMPLER_SRC = r"""
 import sys, time
 import pynvml as N
-pynvml_bus, idx = sys.argv[1], int(sys.argv[2])
+pynvml_bus, idx, out = sys.argv[1], int(sys.argv[2]), open(sys.argv[3], "w")
 N.nvmlInit()
 try:
     h = N.nvmlDeviceGetHandleByPciBusId(pynvml_bus) if pynvml_bus else N.nvmlDeviceGetHandleByIndex(idx)
@@ -129,7 +130,9 @@ while True:
         r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
     except Exception:
         r = N.nvmlDeviceGetCurrentClocksThrottleReasons(h)
-    print("%.6f %d %d" % (t, sm, r), flush=True)
+    out.write("%.6f %d %d\n" % (t, sm, r))
+    out.flush()
+    time.sleep(0.0005)
 """
 
 # NVML clock-event reason bits (nvml.h)
@@ -138,10 +141,10 @@ _REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 
 
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled by NVML back to back (each
-    sample is two read-only queries) from a separate process, kept only for
-    the host-time window that brackets the timed GPU work (start() ...
-    stop())."""
+    """SM clock and clock-event reasons sampled by NVML every ~0.5 ms (each
+    sample is two read-only queries) from a separate process into a file,
+    kept only for the host-time window that brackets the timed GPU work
+    (start() ... stop())."""
 
     def __init__(self, device):
         self.device = device
@@ -159,7 +162,11 @@ class ClockSampler:
             pass
         idx = self.device.index or 0
         try:
-            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, bus, str(idx)],
+            # samples go to a file (a pipe left unread would fill and stall the sampler)
+            fd, self.path = tempfile.mkstemp(suffix=".clk")
+            os.close(fd)
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, bus, str(idx),
+                                          self.path],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
             line = self.proc.stdout.readline().split()
@@ -183,7 +190,10 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
                     "note": "NVML sampler unavailable"}
         self.proc.kill()
-        out, _ = self.proc.communicate(timeout=10)
+        self.proc.communicate(timeout=10)
+        with open(self.path) as f:
+            out = f.read()
+        os.unlink(self.path)
         sm, reasons = [], set()
         for row in out.splitlines():
             f = row.split()
@@ -200,7 +210,7 @@ class ClockSampler:
         rec = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
                "reasons": sorted(reasons), "samples": len(sm),
                "window_ms": None if self.t0 is None else round((self.t1 - self.t0) * 1e3, 2),
-               "how": "NVML queries back to back from a separate process, host-time window "
+               "how": "NVML queries every ~0.5 ms from a separate process, host-time window "
                       "around the timed passes"}
         if not sm:
             rec["note"] = "no sample fell inside the timed window"

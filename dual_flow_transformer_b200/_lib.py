@@ -98,6 +98,13 @@ SIGNATURES = {
         _vp, _vp]),                             # err_flag, stream
     "dualflow_grouped_proj_batched_num_launches": (_c_int, [_c_int] * 5),
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
+    "dualflow_layer_post_attention_workspace_size": (_c_size, [_c_int] * 4),
+    "dualflow_layer_post_attention": (_c_int, [
+        _vp, _vp, _vp, _vp, _vp, _vp, _vp,  # attn, x, w_o, w_gu, w_down, b, c
+        _c_int, _c_int, _c_int, _c_int,     # m_primary, d_model, q_dim, F
+        _c_float,                           # eps
+        _vp, _vp, _vp, _vp,                 # x_mid, xn2, h, x_out
+        _vp, _c_size, _vp, _vp]),           # workspace, bytes, err_flag, stream
 }
 
 _lib = None

@@ -400,3 +400,54 @@ def rmsnorm(x, gain=None, y=None, eps=1e-5, stream=None):
                                  float(eps), _stream(stream))
     L.check("dualflow_rmsnorm", st)
     return y
+
+
+def layer_post_attention_workspace_size(m_primary, d_model, q_dim, F) -> int:
+    return _lib().dualflow_layer_post_attention_workspace_size(int(m_primary), int(d_model),
+                                                               int(q_dim), int(F))
+
+
+def new_post_attention_workspace(m_primary, d_model, q_dim, F, device="cuda"):
+    """Zero-filled workspace of layer_post_attention (its leading grid counters
+    must start at zero; every completed call leaves them at zero)."""
+    n = layer_post_attention_workspace_size(m_primary, d_model, q_dim, F)
+    if n == 0:
+        raise ValueError("layer_post_attention does not support these sizes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=None, xn2=None,
+                         h=None, x_out=None, workspace=None, err_flag=None, stream=None):
+    """x_mid = x + attn W_o^T; xn2 = RMSNorm(x_mid); h = SwiGLU(xn2) (+ b
+    coupling); x_out = x_mid + h W_down^T (+ c coupling), in one launch.
+
+    attn: bf16 [2m, q_dim]; x: bf16 [2m, d_model] (primary rows first); w_o
+    [d_model, q_dim], w_gu [2F, d_model], w_down [d_model, F]; b [F], c
+    [d_model] or None. Returns (x_out, x_mid, xn2, h)."""
+    M, q_dim = attn.shape
+    d_model = x.shape[1]
+    F = w_down.shape[1]
+    mp = M // 2
+    for t in (attn, x, w_o, w_gu, w_down):
+        if not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("bf16 contiguous tensors required")
+    if M % 2 or x.shape[0] != M or tuple(w_o.shape) != (d_model, q_dim) or \
+            tuple(w_gu.shape) != (2 * F, d_model):
+        raise ValueError("shape mismatch")
+    dev = x.device
+    bf = torch.bfloat16
+    x_mid = torch.empty((M, d_model), dtype=bf, device=dev) if x_mid is None else x_mid
+    xn2 = torch.empty((M, d_model), dtype=bf, device=dev) if xn2 is None else xn2
+    h = torch.empty((M, F), dtype=bf, device=dev) if h is None else h
+    x_out = torch.empty((M, d_model), dtype=bf, device=dev) if x_out is None else x_out
+    for t in (x_mid, xn2, h, x_out):
+        if not t.is_contiguous():
+            raise ValueError("outputs must be contiguous")
+    if workspace is None:
+        workspace = new_post_attention_workspace(mp, d_model, q_dim, F, dev)
+    st = _lib().dualflow_layer_post_attention(
+        _ptr(attn), _ptr(x), _ptr(w_o), _ptr(w_gu), _ptr(w_down), _ptr(b), _ptr(c), mp, d_model,
+        q_dim, F, float(eps), _ptr(x_mid), _ptr(xn2), _ptr(h), _ptr(x_out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_layer_post_attention", st)
+    return x_out, x_mid, xn2, h

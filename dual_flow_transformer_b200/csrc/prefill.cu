@@ -811,6 +811,326 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ two tiles per CTA
+// The same computation for two query heads h0 = 2x, h1 = 2x + 1 of one KV
+// group and one 128-row tile: both tiles read the same K/V pages (one load per
+// page serves 256 query rows), and the tensor core alternates between them,
+// so that it computes one tile's S or P V while the other tile's softmax
+// warps work (one tile alone leaves the tensor core idle during its softmax).
+// Warp 0: TMA producer; warp 1: MMA issuer; warps 2-5: softmax of tile 0;
+// warps 6-9: softmax of tile 1 (two softmax warps per SM sub-partition).
+// TMEM: tile t at columns t * 256: S double buffer [0, 128), O [128, 256).
+
+constexpr int kPairThreads = 320;
+constexpr uint32_t kPairTmemCols = 512;
+
+template <int D>
+struct PairLayout {
+  static constexpr int kQBytes = kRows * D * 2;      // one tile's Q
+  static constexpr int kPageBytes = kPage * D * 2;   // one K (or V) page
+  static constexpr int kStageBytes = 2 * kPageBytes;
+  static constexpr int kPBytes = kRows * kPage * 2;  // P of one page of one tile
+  static constexpr int kOffStages = 2 * kQBytes;
+  static constexpr int kOffP = kOffStages + kStages * kStageBytes;  // [tile][buffer]
+  static constexpr int kOffBar = kOffP + 4 * kPBytes;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 * 2 + 1;
+  static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using Lay = PairLayout<D>;
+  constexpr int H = D / 64;
+  constexpr float kNegInf = -INFINITY;
+  static_assert(D == 128, "the two-tile prefill kernel is built for head_dim 128");
+  static_assert(PairLayout<D>::kSmem <= 227 * 1024, "shared memory budget");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = full + kStages;
+  uint64_t* s_full = empty + kStages;  // [tile][2] S_i landed in TMEM buffer i & 1
+  uint64_t* s_free = s_full + 4;       // [tile][2] that tile's softmax warps have read it
+  uint64_t* p_full = s_free + 4;       // [tile][2] P_i written to P buffer i & 1
+  uint64_t* pv_done = p_full + 4;      // [tile][2] O += P_i V_i completed
+  uint64_t* mma_done = pv_done + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int h0 = 2 * static_cast<int>(blockIdx.x);
+  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
+  const int b = blockIdx.z;
+  const int g = h0 / p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+
+  const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
+  if (!c.ok) {
+    if (h0 == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
+    return;
+  }
+  const int i0 = tile * kRows;
+  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
+  const int rows = min(kRows, c.n - i0);
+  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
+  const int npages = (kend + kPage - 1) / kPage;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kPairTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_arrive_expect_tx(q_full, 2 * Lay::kQBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int hf = 0; hf < H; ++hf)
+          tma_load_2d(smem + t * Lay::kQBytes + hf * (kRows * 128), &tmQ, q_full,
+                      (h0 + t) * D + hf * 64, c.t0 + i0);
+      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      int issued = 0;
+      for (int i = 0; i < npages; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        int page = tbl[i];
+        if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
+          set_err(p.err, DF_DEVERR_BLOCK);
+          page = 0;
+        }
+        mbar_arrive_expect_tx(&full[st], Lay::kStageBytes);
+        const int row = (page * p.Hkv + g) * kPage;
+        uint8_t* sK = smem + Lay::kOffStages + st * Lay::kStageBytes;
+        uint8_t* sV = sK + Lay::kPageBytes;
+#pragma unroll
+        for (int hf = 0; hf < H; ++hf) {
+          tma_load_2d(sK + hf * kPage * 128, &tmK, &full[st], hf * 64, row);
+          tma_load_2d(sV + hf * kPage * 128, &tmV, &full[st], hf * 64, row);
+        }
+        ++issued;
+      }
+      // Leave no copy in flight (bounded waits).
+      mbar_wait(q_full, 0);
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = umma::make_idesc(kRows, kPage);             // Q K^T
+      constexpr uint32_t kIdPV = umma::make_idesc(kRows, 64) | (1u << 16);  // P V, V MN-major
+      bool ok = mbar_wait(q_full, 0);
+      // S_i of tile t into its TMEM buffer i & 1
+      auto issue_s = [&](int t, int i) -> bool {
+        const int st = i % kStages, sb = i & 1;
+        if (!mbar_wait(&full[st], (i / kStages) & 1)) return false;
+        if (i >= 2 && !mbar_wait(&s_free[2 * t + sb], ((i >> 1) - 1) & 1)) return false;
+        umma::tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + t * Lay::kQBytes);
+        const uint32_t k_addr = smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk >> 2, kq = kk & 3;
+          umma::umma_bf16(tmem + t * 256 + sb * kPage,
+                          umma::smem_desc(q_addr + hf * (kRows * 128) + kq * 32),
+                          umma::smem_desc(k_addr + hf * (kPage * 128) + kq * 32), kIdS,
+                          kk > 0 ? 1u : 0u);
+        }
+        umma::umma_commit(&s_full[2 * t + sb]);
+        return true;
+      };
+      // O_t += P_i V_i once tile t's softmax has written P_i
+      auto issue_pv = [&](int t, int i) -> bool {
+        const int pb = i & 1, st = i % kStages;
+        if (!mbar_wait(&p_full[2 * t + pb], (i >> 1) & 1)) return false;
+        umma::tc_fence_after();
+        const uint32_t p_addr = smem_u32(smem + Lay::kOffP + (2 * t + pb) * Lay::kPBytes);
+        const uint32_t v_addr =
+            smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes);
+#pragma unroll
+        for (int kk = 0; kk < kPage / 16; ++kk) {
+#pragma unroll
+          for (int hf = 0; hf < H; ++hf)
+            umma::umma_bf16(tmem + t * 256 + kOCol + hf * 64, umma::smem_desc(p_addr + kk * 32),
+                            smem_desc_mn64(v_addr + hf * (kPage * 128) + kk * 2048), kIdPV,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma::umma_commit(&pv_done[2 * t + pb]);
+        return true;
+      };
+      if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+      for (int i = 0; ok && i < npages; ++i) {
+        const bool more = i + 1 < npages;
+        if (more && !issue_s(0, i + 1)) ok = false;
+        if (ok && !issue_pv(0, i)) ok = false;
+        if (ok && more && !issue_s(1, i + 1)) ok = false;
+        if (ok && !issue_pv(1, i)) ok = false;
+        if (ok) umma::umma_commit(&empty[i % kStages]);  // page i read by both tiles
+      }
+      if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
+      umma::umma_commit(mma_done);  // completes when every MMA issued above has
+      mbar_wait(mma_done, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int t = warp >= 6 ? 1 : 0;  // the tile this warp serves
+    const int quarter = warp & 3;     // this warp may access TMEM lanes 32 quarter .. + 31
+    const int r = quarter * 32 + lane;
+    const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
+    uint8_t* p_base = smem + Lay::kOffP + 2 * t * Lay::kPBytes + r * 128;
+    uint64_t* my_s_full = s_full + 2 * t;
+    uint64_t* my_s_free = s_free + 2 * t;
+    uint64_t* my_p_full = p_full + 2 * t;
+    uint64_t* my_pv_done = pv_done + 2 * t;
+    float m_ref = kNegInf, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < npages; ++i) {
+      const int sb = i & 1, st = i % kStages, kbase = i * kPage;
+      if (!mbar_wait_warp(&my_s_full[sb], (i >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      umma::tc_fence_after();
+      float s0[32], s1[32];
+      umma::tmem_ld<32>(t_lane + sb * kPage, s0);
+      umma::tmem_ld<32>(t_lane + sb * kPage + 32, s1);
+      umma::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&my_s_free[sb]);
+
+      if (kbase + kPage - 1 > pos) {  // causal mask (and keys past the chunk end)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (kbase + j > pos) s0[j] = kNegInf;
+          if (kbase + 32 + j > pos) s1[j] = kNegInf;
+        }
+      }
+      const float m_cand = fmaxf(max32(s0), max32(s1)) * p.scale_log2;
+      const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
+      if (m_ref == kNegInf) m_ref = m_cand;  // first page: O holds nothing yet
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold P_{i-1} V_{i-1} before it is rescaled in place.
+        if (!mbar_wait_warp(&my_pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        umma::tc_fence_after();
+        const float alpha = rescale ? exp2f(m_ref - m_cand) : 1.f;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          float o[32];
+          umma::tmem_ld<32>(t_lane + kOCol + cc, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_lane + kOCol + cc, o);
+        }
+        if (rescale) {
+          l *= alpha;
+          m_ref = m_cand;
+        }
+      }
+      const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
+
+      // P buffer sb of this tile is free once O += P_{i-2} V_{i-2} has completed.
+      if (i >= 2 && !mbar_wait_warp(&my_pv_done[sb], ((i >> 1) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = p_base + sb * Lay::kPBytes;
+      l += write_p32(prow, r, 0, s0, p.scale_log2, mu);
+      l += write_p32(prow, r, 4, s1, p.scale_log2, mu);
+
+      // Keys at or past kend on the last page hold other tokens' bytes
+      // (possibly NaN patterns): their weights are 0, and their V rows are
+      // zeroed, as 0 * NaN would still be NaN in the accumulator. Both tiles'
+      // warps clear the same rows (the same zero bytes), each before its own
+      // P is published, so neither tile's P V can read the old bytes.
+      if (kbase + kPage > kend) {
+        if (!mbar_wait_warp(&full[st], (i / kStages) & 1)) {  // the page has landed
+          ok = false;
+          break;
+        }
+        const int kend_rel = kend - kbase;
+        uint8_t* sV = smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes;
+        const int nvec = (kPage - kend_rel) * H * 8;  // 16-byte chunks to clear
+        for (int v = r; v < nvec; v += kRows) {
+          const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
+          *reinterpret_cast<uint4*>(sV + hf * (kPage * 128) + row * 128 + ch * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // P (and cleared V rows) -> the tensor core's proxy
+      umma::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&my_p_full[sb]);
+    }
+    if (ok) {
+      const int last = npages - 1;
+      ok = mbar_wait_warp(&my_pv_done[last & 1], (last >> 1) & 1);
+    }
+    if (ok) {
+      umma::tc_fence_after();
+      __nv_bfloat16* orow = p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t +
+                            (h0 + t) * D;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        float o[32];
+        umma::tmem_ld<32>(t_lane + kOCol + cc, o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
+        if (r < rows) umma::store_bf16<32>(orow + cc, o);
+      }
+    } else if (lane == 0) {
+      set_err(p.err, DF_DEVERR_TIMEOUT);
+    }
+  }
+
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kPairTmemCols)
+                 : "memory");
+  }
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------------ 3. last-row gather
@@ -858,8 +1178,18 @@ cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* t
                     p);
 }
 
+// Two query heads of one KV group per CTA when the group has an even number
+// of heads (both tiles then read the same pages), else one head per CTA.
 cudaError_t launch_attn_tc(const AttnParams& p, int Hq, int B, const CUtensorMap* tmQ,
                            const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
+  if (p.G % 2 == 0) {
+    constexpr size_t smem2 = tc::PairLayout<128>::kSmem;
+    cudaError_t e2 =
+        ensure_dynamic_smem(reinterpret_cast<const void*>(tc::pair_kernel<128>), smem2);
+    if (e2 != cudaSuccess) return e2;
+    return launch_pdl(tc::pair_kernel<128>, dim3(Hq / 2, p.tiles, B), dim3(tc::kPairThreads),
+                      smem2, stream, *tmQ, *tmK, *tmV, p);
+  }
   constexpr size_t smem = tc::Layout<128>::kSmem;
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::attn_kernel<128>), smem);
   if (e != cudaSuccess) return e;

@@ -14,6 +14,11 @@ Composition of library calls only (each step is a libdualflow kernel):
   7. H = SiLU(X'n W_gate^T) * (X'n W_up^T), aux += b_l H1    dualflow_grouped_proj (swiglu)
   8. X'' = X' + H W_down^T, aux += c_l (H1 W_down^T)         dualflow_grouped_proj (residual)
 
+With fused_post=True, steps 5-8 run as one persistent launch
+(dualflow_layer_post_attention) when the sizes allow it: its weight producers
+stream W_o, W_gate/up and W_down back to back instead of four launches each
+ramping up and draining. The default keeps the four calls.
+
 Pages: "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
 Core" (shared matrices, primary-only cache writes, auxiliary flow active at
 generated positions), "Meccanismi Chiave" (asymmetric shared-KV attention and
@@ -31,7 +36,7 @@ from . import api
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
-                 num_splits=0):
+                 num_splits=0, fused_post=False):
         self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
         self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
         self.d_model = weights["w_o"].shape[0]
@@ -58,17 +63,27 @@ class DualFlowLayer:
         self.attn_ws = api.new_attn_workspace(B, Hq, Hkv, D, self.max_seqlen, num_splits, dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.attn_launches = api.decode_attn_num_launches(B, Hkv, self.max_seqlen, num_splits)
-        self._gemm_launches = (
-            api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
-            + api.grouped_proj_num_launches(M, *weights["w_o"].shape, "residual")
-            + api.grouped_proj_num_launches(M, *weights["w_gu"].shape, "swiglu")
-            + api.grouped_proj_num_launches(M, *weights["w_down"].shape, "residual"))
+        self.fused_post = bool(fused_post) and \
+            api.layer_post_attention_workspace_size(B, self.d_model, qd, F) > 0
+        self.post_ws = (api.new_post_attention_workspace(B, self.d_model, qd, F, dev)
+                        if self.fused_post else None)
+        if self.fused_post:
+            post_launches = 1
+        else:
+            post_launches = (api.grouped_proj_num_launches(M, *weights["w_o"].shape, "residual")
+                             + 1
+                             + api.grouped_proj_num_launches(M, *weights["w_gu"].shape, "swiglu")
+                             + api.grouped_proj_num_launches(M, *weights["w_down"].shape,
+                                                             "residual"))
+        self._gemm_launches = (api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
+                               + post_launches)
 
     @property
     def launches_per_step(self) -> int:
-        """Kernel launches of one step: 2 norms, append, attention, and the
-        grouped projections (1 or 2 launches each)."""
-        return 3 + self.attn_launches + self._gemm_launches
+        """Kernel launches of one step: the first norm, the QKV projection,
+        the append, the attention and the post-attention half (one launch
+        fused, else W_o, the second norm, gate/up and down)."""
+        return 2 + self.attn_launches + self._gemm_launches
 
     # ------------------------------------------------------------ CUDA graphs
     def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):
@@ -146,6 +161,11 @@ class DualFlowLayer:
                             o1=self.attn[:B].view(B, Hq, D), o2=self.attn[B:].view(B, Hq, D),
                             num_splits=self.num_splits, workspace=self.attn_ws,
                             err_flag=self.err, stream=stream)
+        elif self.fused_post:
+            api.layer_post_attention(self.attn, X, w["w_o"], w["w_gu"], w["w_down"], w["b"],
+                                     w["c"], eps=self.eps, x_mid=self.x_mid, xn2=self.xn2,
+                                     h=self.h, x_out=self.x_out, workspace=self.post_ws,
+                                     err_flag=self.err, stream=stream)
         else:
             api.grouped_proj(self.attn, B, w["w_o"], y=self.x_mid, epilogue="residual",
                              residual=X, workspace=self.proj_ws, err_flag=self.err,

@@ -23,9 +23,13 @@ class _FakeProc:
         return self.text, ""
 
 
-def _sampler(lines, t0, t1):
+def _sampler(lines, t0, t1, tmp_path=None):
+    import tempfile
     s = bench.ClockSampler(device=None)
-    s.proc = _FakeProc("\n".join(lines))
+    fd, s.path = tempfile.mkstemp(suffix=".clk")
+    with os.fdopen(fd, "w") as f:
+        f.write("\n".join(lines))
+    s.proc = _FakeProc("")
     s.smax = 1965.0
     s.t0, s.t1 = t0, t1
     return s

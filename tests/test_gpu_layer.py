@@ -18,12 +18,14 @@ SMALL = dataclasses.replace(synth.WORKLOADS["layer"], B=8, d_model=512, Hq=4, Hk
                             F=1024, cache_len=200, seed=50)
 
 
-def _run_gpu(inp, dev, num_splits=0):
+def _run_gpu(inp, dev, num_splits=0, fused_post=True):
     d = to_dev(inp, dev)
     w = {k: d[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
     B = inp["B"]
     layer = DualFlowLayer(w, inp["Hq"], inp["Hkv"], inp["D"], inp["F"], B,
-                          int(inp["positions"].max()) + 1, device=dev, num_splits=num_splits)
+                          int(inp["positions"].max()) + 1, device=dev, num_splits=num_splits,
+                          fused_post=fused_post)
+    assert layer.fused_post == fused_post
     X = torch.cat([d["x1"], d["x2"]]).contiguous()
     seqlens = (d["positions"] + 1).to(torch.int32)
     out = layer.step(X, d["k_cache"], d["v_cache"], d["block_table"], d["positions"], seqlens)
@@ -45,13 +47,16 @@ def _oracle(inp, rows=None):
     return r
 
 
+@pytest.mark.parametrize("fused_post", [True, False])
 @pytest.mark.parametrize("coupled", [True, False])
-def test_layer_step_small(cuda_device, coupled):
+def test_layer_step_small(cuda_device, coupled, fused_post):
     w = dataclasses.replace(SMALL, coupled_mlp=coupled)
     inp = synth.make_layer_inputs(w)
-    out, d, _ = _run_gpu(inp, cuda_device)
+    out, d, layer = _run_gpu(inp, cuda_device, fused_post=fused_post)
     ref = _oracle(inp)
     assert_close(out, ref["x_out"], "bf16", "layer x_out")
+    assert_close(layer.x_mid.cpu(), ref["x_mid"], "bf16", "layer x_mid")
+    assert_close(layer.h.cpu(), ref["h"], "bf16", "layer h")
 
 
 def test_layer_primary_flow_is_self_sufficient(cuda_device):
