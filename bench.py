@@ -59,6 +59,9 @@ def parse_args(argv=None):
                              "prefill"],
                     default="layer")
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--fused-post", type=int, choices=[0, 1], default=None,
+                    help="layer workload: 1 = the post-attention half as one persistent launch, "
+                         "0 = four launches (default: the layer's own default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -277,8 +280,9 @@ class LayerRun:
         d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.host.items()}
         self.d = d
         W = {k: d[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
+        kw = {} if args.fused_post is None else {"fused_post": bool(args.fused_post)}
         self.layer = DualFlowLayer(W, w.Hq, w.Hkv, w.D, w.F, w.B, w.cache_len + 1, device=dev,
-                                   num_splits=args.num_splits)
+                                   num_splits=args.num_splits, **kw)
         self.X = torch.cat([d["x1"], d["x2"]]).contiguous()
         self.seqlens = (d["positions"] + 1).to(torch.int32)
         # the step runs as CUDA-graph replays over fixed buffers (X lives in x_in)
@@ -297,6 +301,8 @@ class LayerRun:
                                    % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
                        "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
                        "attended": L, "attn_launches": self.layer.attn_launches,
+                       "post_attention": "one persistent launch" if self.layer.fused_post
+                                         else "four launches",
                        "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
                              % (self.kv_bytes / 1e9, 436207616 / 1e9)}
         self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"

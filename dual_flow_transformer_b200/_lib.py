@@ -103,7 +103,7 @@ SIGNATURES = {
         _vp, _vp, _vp, _vp, _vp, _vp, _vp,  # attn, x, w_o, w_gu, w_down, b, c
         _c_int, _c_int, _c_int, _c_int,     # m_primary, d_model, q_dim, F
         _c_float,                           # eps
-        _vp, _vp, _vp, _vp,                 # x_mid, xn2, h, x_out
+        _vp, _vp, _vp,                      # x_mid, h, x_out
         _vp, _c_size, _vp, _vp]),           # workspace, bytes, err_flag, stream
 }
 

@@ -416,14 +416,15 @@ def new_post_attention_workspace(m_primary, d_model, q_dim, F, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=None, xn2=None,
-                         h=None, x_out=None, workspace=None, err_flag=None, stream=None):
-    """x_mid = x + attn W_o^T; xn2 = RMSNorm(x_mid); h = SwiGLU(xn2) (+ b
-    coupling); x_out = x_mid + h W_down^T (+ c coupling), in one launch.
+def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=None, h=None,
+                         x_out=None, workspace=None, err_flag=None, stream=None):
+    """x_mid = x + attn W_o^T; r = RMSNorm row scale of x_mid; h = SiLU(r
+    x_mid W_gate^T) * (r x_mid W_up^T) (+ b coupling); x_out = x_mid + h
+    W_down^T (+ c coupling), in one launch.
 
     attn: bf16 [2m, q_dim]; x: bf16 [2m, d_model] (primary rows first); w_o
     [d_model, q_dim], w_gu [2F, d_model], w_down [d_model, F]; b [F], c
-    [d_model] or None. Returns (x_out, x_mid, xn2, h)."""
+    [d_model] or None. Returns (x_out, x_mid, h)."""
     M, q_dim = attn.shape
     d_model = x.shape[1]
     F = w_down.shape[1]
@@ -437,17 +438,16 @@ def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=No
     dev = x.device
     bf = torch.bfloat16
     x_mid = torch.empty((M, d_model), dtype=bf, device=dev) if x_mid is None else x_mid
-    xn2 = torch.empty((M, d_model), dtype=bf, device=dev) if xn2 is None else xn2
     h = torch.empty((M, F), dtype=bf, device=dev) if h is None else h
     x_out = torch.empty((M, d_model), dtype=bf, device=dev) if x_out is None else x_out
-    for t in (x_mid, xn2, h, x_out):
+    for t in (x_mid, h, x_out):
         if not t.is_contiguous():
             raise ValueError("outputs must be contiguous")
     if workspace is None:
         workspace = new_post_attention_workspace(mp, d_model, q_dim, F, dev)
     st = _lib().dualflow_layer_post_attention(
         _ptr(attn), _ptr(x), _ptr(w_o), _ptr(w_gu), _ptr(w_down), _ptr(b), _ptr(c), mp, d_model,
-        q_dim, F, float(eps), _ptr(x_mid), _ptr(xn2), _ptr(h), _ptr(x_out), _ptr(workspace),
+        q_dim, F, float(eps), _ptr(x_mid), _ptr(h), _ptr(x_out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream))
     L.check("dualflow_layer_post_attention", st)
-    return x_out, x_mid, xn2, h
+    return x_out, x_mid, h

@@ -6,11 +6,12 @@
 // "Costi di Inferenza vs. Addestramento" (grouped decode reads the unique
 // weights once for both flows). With X = [primary rows; auxiliary rows]:
 //   x_mid = x + attn W_o^T                                   (residual)
-//   xn2   = x_mid / sqrt(mean(x_mid^2) + eps)                 (RMSNorm, unit gain)
-//   h     = SiLU(xn2 W_gate^T) * (xn2 W_up^T);  h_aux += b (.) h_primary
+//   r     = 1 / sqrt(mean(x_mid^2) + eps)                    (RMSNorm, unit gain)
+//   h     = SiLU(r x_mid W_gate^T) * (r x_mid W_up^T);  h_aux += b (.) h_primary
 //   x_out = x_mid + h W_down^T;  aux rows add c (.) (h W_down^T)_primary
-// x_mid, xn2, h and x_out are stored as bf16 (the same interfaces as the
-// four-launch form of the same step).
+// x_mid, h and x_out are stored as bf16. The norm's row scale r is applied to
+// the gate/up accumulators (r (x_mid W^T) = (r x_mid) W^T), so the normalised
+// rows are never rounded to bf16 and stored: the gate/up product reads x_mid.
 //
 // Why one kernel: at M = 128 rows every projection is a weight stream (about
 // 128 flop per weight byte, below the B200 ridge). Separate launches leave
@@ -24,14 +25,26 @@
 // grid = SM count), each wait bounded.
 //
 // Phases (units are spread over the CTAs, CTA i takes units i, i + G, ...):
-//   P0  W_o:    16 column tiles of 256 x S0 k-ranges -> fp32 partials
-//   --- counter A --- R0: CTA r < M sums row r's partials in split order, adds
-//                     the residual, stores x_mid, then xn2 (row-local norm)
-//   --- counter B --- P1  W_gate/W_up: one tile of 2*H1 weight rows per CTA,
-//                     SwiGLU + b coupling straight from TMEM -> h
+//   P0  W_o:    column tiles of 256 x S0 k-ranges -> fp32 partials
+//   --- counter A --- R0: 4-column groups over all CTAs: x_mid = x + the sum
+//                     of the partials (split order), and each CTA's partial
+//                     sum of squares per row
+//   --- counter A2 --- P1 may read x_mid; CTA r < M sums row r's squares in
+//                     CTA order -> r_row   --- counter I ---
+//   P1  W_gate/W_up: one tile of 2*H1 weight rows per CTA, SwiGLU (row scale
+//                     r) + b coupling straight from TMEM -> h
 //   --- counter C --- P2  W_down: column tiles of 256 x S2 k-ranges -> partials
-//   --- counter D --- R2: (sequence, column half) units: residual + c
+//   --- counter D --- R2: 4-column groups over all CTAs: residual + c
 //                     coupling -> x_out
+// Partials are stored [unit][column group of 4][row][4] fp32: a warp's store
+// (32 consecutive rows of one group) is one contiguous 512-byte segment, and a
+// (group, split) item is one contiguous 2 KB block. The reductions bring all
+// their items into the idle 192 KB weight ring with bulk TMA copies, one
+// round trip at the layer's sizes (a latency-bound loop of loads took 13 us);
+// the gate/up weight loads wait for the ring, and the gap is covered by L2
+// prefetches of the next phase's first weight tiles, issued at each phase
+// boundary only (prefetching ahead all the time took TMA bandwidth from the
+// loads).
 // Roles (224 threads): warp 0 weight producer, warp 1 MMA issuer (one thread,
 // tcgen05.mma M = 128 into two 256-column TMEM accumulators), warp 2
 // activation producer, warps 3-6 epilogue (TMEM lane quarter = warp % 4).
@@ -59,17 +72,19 @@ constexpr int kStages = 4;
 constexpr int kXBytes = kBM * kBK * 2;            // 16 KB activation tile
 constexpr int kSlot = kXBytes + 256 * kBK * 2;    // + up to 32 KB of weights
 constexpr int kTileN = 256;                       // W_o / W_down column tile
-constexpr int kMaxHalf = 112;                     // SwiGLU output columns per tile
-constexpr int kStgPitch = 36;                     // fp32 staging row pitch
-constexpr int kXchgFloats = 64 * (kMaxHalf + 1);  // >= 4 * 32 * kStgPitch
-constexpr int kCounters = 8;                      // A, B, C, D, exit
+constexpr int kMaxHalf = 128;                     // SwiGLU output columns per tile
+constexpr int kXchgPitch = 33;                    // coupling exchange: [64 rows][32 + 1]
+constexpr int kXchgFloats = 64 * kXchgPitch;
+constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
+constexpr int kGroupBytes = kBM * 4 * 4;          // one 4-column group of a partial: 2 KB
+constexpr int kRedItems = kStages * kSlot / kGroupBytes;  // reduction batch: the whole ring
+constexpr int kBoundaryPrefetch = 16;             // next-phase weight stages prefetched to L2
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kSlot + kXchgFloats * 4 +
-                              16 * 4 + 256;  // + barriers, TMEM slot and flags
-static_assert(kXchgFloats >= 4 * 32 * kStgPitch, "staging must fit in the exchange area");
+                              kEpiThreads * 4 + kMaxHalf * 4 + 256;  // + barriers, flags
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-enum { kCntA = 0, kCntB = 1, kCntC = 2, kCntD = 3, kCntExit = 4 };
+enum { kCntA = 0, kCntA2 = 1, kCntI = 2, kCntC = 3, kCntD = 4, kCntExit = 5 };
 
 struct Gemm {
   int units, splits, kblocks;
@@ -83,16 +98,16 @@ struct Params {
   int M, mp, d, qd, F;
   float eps;
   Gemm g[3];
-  int r2_units;  // mp * 2 (sequence, column half)
   const __nv_bfloat16* x;
   const __nv_bfloat16* b;
   const __nv_bfloat16* c;
   __nv_bfloat16* x_mid;
-  __nv_bfloat16* xn2;
   __nv_bfloat16* h;
   __nv_bfloat16* x_out;
-  float* part;  // [units][128][256] fp32
-  int* cnt;     // [kCounters]
+  float* part;     // [units][64 groups][128 rows][4] fp32
+  float* ss_part;  // [G][128] per-CTA partial sums of squares of x_mid rows
+  float* rscale;   // [128] RMSNorm row scales
+  int* cnt;        // [kCounters]
   int32_t* err;
 };
 
@@ -124,22 +139,6 @@ __device__ __forceinline__ void st_cg4(float* p, float4 v) {
                : "memory");
 }
 
-// 16 bf16 values through L2 only (rows written by other CTAs of this grid).
-__device__ __forceinline__ void load_bf16x16_cg(const __nv_bfloat16* src, float (&v)[16]) {
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint32_t w[4];
-    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                 : "l"(src + 8 * q));
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[q * 8 + 2 * k] = bf16_bits_to_float(static_cast<uint16_t>(w[k] & 0xffffu));
-      v[q * 8 + 2 * k + 1] = bf16_bits_to_float(static_cast<uint16_t>(w[k] >> 16));
-    }
-  }
-}
-
 // Single-thread bounded wait until *cnt >= target (every CTA of the grid has
 // passed the corresponding point). false: gave up.
 __device__ bool wait_count(const int* cnt, int target) {
@@ -166,6 +165,40 @@ __device__ __forceinline__ void unit_range(const Gemm& g, int u, int& tile, int&
   }
 }
 
+// Walks this CTA's stage sequence (GEMM q, its units u = cta, cta + G, ...,
+// their k-blocks) in the order the producers and the MMA issuer use.
+struct StageCursor {
+  int q, u, kb, k1, tile;
+  bool done;
+  __device__ StageCursor(const Params& p, int cta, int G) : q(0), u(cta), kb(0), k1(0), tile(0),
+                                                          done(false) {
+    seek(p, G);
+  }
+  // first stage of unit u of GEMM q, or of the next GEMM that has one
+  __device__ void seek(const Params& p, int G) {
+    while (q < 3 && u >= p.g[q].units) {
+      ++q;
+      u = u % G;  // this CTA's index
+    }
+    if (q >= 3) {
+      done = true;
+      return;
+    }
+    int k0;
+    unit_range(p.g[q], u, tile, k0, k1);
+    kb = k0;
+  }
+  __device__ void next(const Params& p, int cta, int G) {
+    if (++kb < k1) return;
+    u += G;
+    if (u >= p.g[q].units) {
+      ++q;
+      u = cta;
+    }
+    seek(p, G);
+  }
+};
+
 // The epilogue threads' arrival at a grid counter: every thread's stores are
 // made visible (also to TMA reads of other CTAs) before one thread adds.
 __device__ __forceinline__ void arrive_count(int* cnt, int et) {
@@ -187,181 +220,323 @@ __device__ __forceinline__ bool epi_wait_count(const int* cnt, int target, int e
   return ok;
 }
 
-// Accumulator (this warp's 32 rows, BN = 256 columns) -> fp32 partial slab
-// part[unit][row][256], staged through shared memory so that each store
-// instruction writes whole 128-byte row segments.
-__device__ void store_partial(const Params& p, float* slab, uint32_t taddr, int quarter, int lane,
-                              float* stg) {
-  for (int c = 0; c < kTileN; c += 32) {
-    float v[32];
-    tmem_ld<32>(taddr + c, v);
-    float4* srow = reinterpret_cast<float4*>(stg + lane * kStgPitch);
+// Two 32-column TMEM loads (this thread's lane), one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  __syncwarp();
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr + 32));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      srow[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    __syncwarp();
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Accumulator (row = this thread's TMEM lane, 256 columns) -> the unit's fp32
+// partial slab [64 groups][128 rows][4]: for each group the warp's 32 lanes
+// store one contiguous 512-byte segment, straight from registers.
+__device__ void store_partial(const Params& p, float* slab, uint32_t taddr, int row) {
+  for (int c = 0; c < kTileN; c += 64) {
+    float v[64];
+    tmem_ld64(taddr + c, v);
+    if (row < p.M) {
 #pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      const int rl = rr * 4 + (lane >> 3), cg = (lane & 7) * 4;
-      const int r = quarter * 32 + rl;
-      if (r < p.M)
-        st_cg4(slab + static_cast<size_t>(r) * kTileN + c + cg,
-               *reinterpret_cast<const float4*>(stg + rl * kStgPitch + cg));
+      for (int q = 0; q < 16; ++q)
+        st_cg4(slab + (static_cast<size_t>(c / 4 + q) * kBM + row) * 4,
+               make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
     }
-    __syncwarp();
   }
 }
 
-// P1 epilogue of tile t: h[row][t*H + j] = SiLU(gate) * up (+ b * primary row's
-// value for auxiliary rows). Pass 1 stores the primary rows (and every row
-// without coupling) and parks the primary values in `xchg`; pass 2 re-reads
-// the accumulator for the auxiliary rows and adds the coupling.
-__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int quarter, int lane,
-                                float* xchg) {
-  const int H = p.g[1].half;
-  const int row = quarter * 32 + lane;
-  const int col0 = t * H;
-  const bool coupled = p.b != nullptr;
-  const int pitch = H + 1;
-  // pass 1
-  if (!coupled || quarter * 32 < p.mp) {
-    for (int c = 0; c < H; c += 8) {
-      float g[8], u[8];
-      tmem_ld<8>(taddr + c, g);
-      tmem_ld<8>(taddr + H + c, u);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) g[i] = silu_f(g[i]) * u[i];
-      const bool prim = row < p.mp;
-      if (coupled && prim) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) xchg[row * pitch + c + i] = g[i];
-      }
-      if ((!coupled || prim) && row < p.M && col0 + c < p.F)
-        store_bf16<8>(p.h + static_cast<size_t>(row) * p.F + col0 + c, g);
-    }
-  }
-  if (!coupled) return;
-  epi_bar();
-  // pass 2: auxiliary rows mp .. 2mp-1, paired with primary row row - mp
-  if (quarter * 32 + 31 >= p.mp) {
-    for (int c = 0; c < H; c += 8) {
-      float g[8], u[8];
-      tmem_ld<8>(taddr + c, g);
-      tmem_ld<8>(taddr + H + c, u);
-      const bool aux = row >= p.mp && row < p.M;
-      if (aux && col0 + c < p.F) {
-        float bv[8];
-        load_bf16<8>(p.b + col0 + c, bv);
-        const float* src = xchg + (row - p.mp) * pitch + c;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) g[i] = fmaf(bv[i], src[i], silu_f(g[i]) * u[i]);
-        store_bf16<8>(p.h + static_cast<size_t>(row) * p.F + col0 + c, g);
-      }
-    }
-  }
-  epi_bar();  // xchg is reused by the next tile / the staging of P2
+__device__ __forceinline__ void load_bf16x4_cg(const __nv_bfloat16* src, float (&v)[4]) {
+  uint32_t w0, w1;
+  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "l"(src));
+  v[0] = bf16_bits_to_float(static_cast<uint16_t>(w0 & 0xffffu));
+  v[1] = bf16_bits_to_float(static_cast<uint16_t>(w0 >> 16));
+  v[2] = bf16_bits_to_float(static_cast<uint16_t>(w1 & 0xffffu));
+  v[3] = bf16_bits_to_float(static_cast<uint16_t>(w1 >> 16));
 }
 
-// R0 for row r: x_mid = x + sum of the W_o partials (split order), stored
-// bf16; then xn2 = bf16(x_mid / sqrt(mean(x_mid^2) + eps)) from the stored
-// (rounded) values.
-__device__ void reduce_o_row(const Params& p, int r, int et, float* red) {
-  const Gemm& g = p.g[0];
-  const int groups = p.d / 32;
+__device__ __forceinline__ void bulk_g2s(uint32_t sdst, const void* gsrc, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          sdst),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Streams the S split partials of each of this CTA's 4-column groups (gi =
+// cta, cta + G, ...) into shared memory by bulk TMA copies (one 2 KB copy
+// per (group, split): all 128 rows of those 4 columns), as many at once as
+// the idle weight ring holds (all of them at the layer's sizes: one round
+// trip), and hands every item to on_item(gi, s, bytes) in split order, then
+// on_group(gi) after its last split. Thread et == 0 issues the copies;
+// `batches` counts the batches of earlier calls (it sets the barrier phase).
+// Returns false if a wait gave up. The caller guarantees that no weight or
+// activation copy targets the ring meanwhile.
+template <class OnItem, class OnGroup>
+__device__ bool stream_partials(const Params& p, int S, int cta, int G, uint8_t* rbuf,
+                                uint64_t* rfull, int& batches, int et, OnItem on_item,
+                                OnGroup on_group) {
+  const int groups = p.d / 4;
+  const int mine = groups > cta ? (groups - cta + G - 1) / G : 0;
+  const int n = mine * S;
+  const int nb = (n + kRedItems - 1) / kRedItems;
+  bool ok = true;
+  for (int b = 0; b < nb; ++b) {
+    const int gb = batches + b;
+    const int k0 = b * kRedItems, k1 = min(n, k0 + kRedItems);
+    if (et == 0) {
+      if (b == 0) fence_proxy_async_global();  // partials stored by other CTAs -> bulk copies
+      mbar_arrive_expect_tx(rfull, static_cast<uint32_t>((k1 - k0) * kGroupBytes));
+      for (int k = k0; k < k1; ++k) {
+        const int gi = cta + (k / S) * G, sp = k % S;
+        const int tile = gi / (kTileN / 4), g = gi - tile * (kTileN / 4);
+        const float* src =
+            p.part + (static_cast<size_t>(tile * S + sp) * (kTileN / 4) + g) * (kBM * 4);
+        bulk_g2s(smem_u32(rbuf + (k - k0) * kGroupBytes), src, kGroupBytes, rfull);
+      }
+    }
+    if (!mbar_wait(rfull, static_cast<uint32_t>(gb & 1))) ok = false;
+    if (ok) {
+      for (int k = k0; k < k1; ++k) {
+        const int gi = cta + (k / S) * G, sp = k % S;
+        on_item(gi, sp, rbuf + (k - k0) * kGroupBytes);
+        if (sp == S - 1) on_group(gi);
+      }
+    }
+    epi_bar();  // every thread is done with the batch before the next one lands
+  }
+  batches += nb;
+  return ok;
+}
+
+// R0 on this CTA's 4-column groups (thread = row): x_mid = bf16(x + sum of the
+// W_o partials in split order); this CTA's sum of squares of each row's
+// stored values goes to ss_part[cta][row].
+constexpr int kPreGroups = 8;  // residual values of up to this many groups held in registers
+
+__device__ bool reduce_o(const Params& p, int cta, int G, int et, uint8_t* rbuf, uint64_t* rfull,
+                         int& batches) {
+  const int row = et;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float ss = 0.f;
-  for (int cg = et; cg < groups; cg += kEpiThreads) {
-    const int col = cg * 32;
-    const int tile = col / kTileN, off = col - tile * kTileN;
-    float acc[32];
+  const bool live = row < p.M;
+  // The residual values of this thread's groups are loaded before the partials
+  // arrive, so no group waits for a load of its own.
+  const int groups = p.d / 4;
+  uint2 pre[kPreGroups];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    for (int s = 0; s < g.splits; ++s) {
-      const float* src =
-          p.part + (static_cast<size_t>(tile * g.splits + s) * kBM + r) * kTileN + off;
-      float4 v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = ld_cg4(src + 4 * i);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        acc[4 * i] += v[i].x;
-        acc[4 * i + 1] += v[i].y;
-        acc[4 * i + 2] += v[i].z;
-        acc[4 * i + 3] += v[i].w;
-      }
-    }
-    float res[32];
-    load_bf16<32>(p.x + static_cast<size_t>(r) * p.d + col, res);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      acc[i] += res[i];
-      const float q = __bfloat162float(__float2bfloat16_rn(acc[i]));
-      ss = fmaf(q, q, ss);
-    }
-    store_bf16<32>(p.x_mid + static_cast<size_t>(r) * p.d + col, acc);
+  for (int i = 0; i < kPreGroups; ++i) {
+    const int gi = cta + i * G;
+    pre[i] = (live && gi < groups)
+                 ? *reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(row) * p.d + gi * 4)
+                 : make_uint2(0u, 0u);
   }
+  const bool ok = stream_partials(
+      p, p.g[0].splits, cta, G, rbuf, rfull, batches, et,
+      [&](int, int, const uint8_t* item) {
+        const float4 v = *reinterpret_cast<const float4*>(item + row * 16);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      },
+      [&](int gi) {
+        if (live) {
+          const int i = (gi - cta) / G;
+          float res[4];
+          if (i < kPreGroups) {
+            uint2 w = make_uint2(0u, 0u);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((et & 31) == 0) red[et >> 5] = ss;
-  epi_bar();
-  const float tot = red[0] + red[1] + red[2] + red[3];
-  const float inv = 1.0f / sqrtf(tot / static_cast<float>(p.d) + p.eps);
-  for (int cg = et; cg < groups; cg += kEpiThreads) {
-    const int col = cg * 32;
-    float v[32];
-    load_bf16<32>(p.x_mid + static_cast<size_t>(r) * p.d + col, v);  // this thread's own stores
+            for (int k = 0; k < kPreGroups; ++k)
+              if (k == i) w = pre[k];
+            res[0] = bf16_bits_to_float(static_cast<uint16_t>(w.x & 0xffffu));
+            res[1] = bf16_bits_to_float(static_cast<uint16_t>(w.x >> 16));
+            res[2] = bf16_bits_to_float(static_cast<uint16_t>(w.y & 0xffffu));
+            res[3] = bf16_bits_to_float(static_cast<uint16_t>(w.y >> 16));
+          } else {
+            load_bf16x4(p.x + static_cast<size_t>(row) * p.d + gi * 4, res);
+          }
+          float o[4] = {acc.x + res[0], acc.y + res[1], acc.z + res[2], acc.w + res[3]};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] *= inv;
-    store_bf16<32>(p.xn2 + static_cast<size_t>(r) * p.d + col, v);
-  }
-  epi_bar();  // red is reused
+          for (int i = 0; i < 4; ++i) {
+            o[i] = __bfloat162float(__float2bfloat16_rn(o[i]));
+            ss = fmaf(o[i], o[i], ss);
+          }
+          store_bf16x4(p.x_mid + static_cast<size_t>(row) * p.d + gi * 4, o);
+        }
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      });
+  p.ss_part[static_cast<size_t>(cta) * kBM + row] = ss;
+  return ok;
 }
 
-// R2 for unit v = (sequence j, column half hf): x_out rows j (primary) and
-// mp + j (auxiliary) over that half: residual x_mid + sum of the W_down
-// partials (split order); the auxiliary row adds c * (primary row's sum).
-__device__ void reduce_down_pair(const Params& p, int v, int et) {
-  const Gemm& g = p.g[2];
-  const int j = v >> 1, hf = v & 1;
-  const int half_cols = p.d / 2;
-  const int rp = j, ra = p.mp + j;
-  for (int cg = et; cg < half_cols / 16; cg += kEpiThreads) {
-    const int col = hf * half_cols + cg * 16;
-    const int tile = col / kTileN, off = col - tile * kTileN;
-    float ap[16], aa[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ap[i] = aa[i] = 0.f;
-    for (int s = 0; s < g.splits; ++s) {
-      const float* base = p.part + static_cast<size_t>(tile * g.splits + s) * kBM * kTileN + off;
-      float4 vp[4], va[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        vp[i] = ld_cg4(base + static_cast<size_t>(rp) * kTileN + 4 * i);
-        va[i] = ld_cg4(base + static_cast<size_t>(ra) * kTileN + 4 * i);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ap[4 * i] += vp[i].x; ap[4 * i + 1] += vp[i].y; ap[4 * i + 2] += vp[i].z;
-        ap[4 * i + 3] += vp[i].w;
-        aa[4 * i] += va[i].x; aa[4 * i + 1] += va[i].y; aa[4 * i + 2] += va[i].z;
-        aa[4 * i + 3] += va[i].w;
-      }
-    }
-    if (p.c != nullptr) {
-      float cv[16];
-      load_bf16<16>(p.c + col, cv);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) aa[i] = fmaf(cv[i], ap[i], aa[i]);
-    }
-    float rv[16];
-    load_bf16x16_cg(p.x_mid + static_cast<size_t>(rp) * p.d + col, rv);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ap[i] += rv[i];
-    load_bf16x16_cg(p.x_mid + static_cast<size_t>(ra) * p.d + col, rv);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) aa[i] += rv[i];
-    store_bf16<16>(p.x_out + static_cast<size_t>(rp) * p.d + col, ap);
-    store_bf16<16>(p.x_out + static_cast<size_t>(ra) * p.d + col, aa);
+// Row scale of row r: 1 / sqrt(sum over CTAs of ss_part[.][r] / d + eps),
+// summed in a fixed order (thread et adds CTAs et, et + 128, ...; then a
+// fixed tree over the 128 threads).
+__device__ void row_scale(const Params& p, int G, int r, int et, float* red) {
+  float v = 0.f;
+  for (int k = et; k < G; k += kEpiThreads) v += __ldcg(p.ss_part + static_cast<size_t>(k) * kBM + r);
+  red[et] = v;
+  epi_bar();
+  for (int w = kEpiThreads / 2; w > 0; w >>= 1) {
+    if (et < w) red[et] += red[et + w];
+    epi_bar();
   }
+  if (et == 0) p.rscale[r] = 1.0f / sqrtf(red[0] / static_cast<float>(p.d) + p.eps);
+  epi_bar();
+}
+
+// P1 epilogue of tile t: h[row][t*H + j] = SiLU(rs g) * (rs u) (+ b * primary
+// row's value for auxiliary rows), in 32-column chunks (8-column tail); the
+// primary rows' values reach their auxiliary rows through `xchg`.
+template <int W>
+__device__ __forceinline__ void swiglu_chunk(const Params& p, uint32_t taddr, int H, int c, int col0,
+                                             int row, float rs, float* xchg, const float* bsl) {
+  float g[W], u[W];
+  tmem_ld<W>(taddr + c, g);
+  tmem_ld<W>(taddr + H + c, u);
+#pragma unroll
+  for (int i = 0; i < W; ++i) g[i] = silu_f(rs * g[i]) * (rs * u[i]);
+  if (p.b != nullptr) {
+    if (row < p.mp) {
+#pragma unroll
+      for (int i = 0; i < W; ++i) xchg[row * kXchgPitch + i] = g[i];
+    }
+    epi_bar();
+    if (row >= p.mp && row < p.M && col0 + c < p.F) {
+#pragma unroll
+      for (int i = 0; i < W; ++i) g[i] = fmaf(bsl[c + i], xchg[(row - p.mp) * kXchgPitch + i], g[i]);
+    }
+    epi_bar();
+  }
+  if (row < p.M) {
+    // a chunk of the last tile may reach past F: store its 8-column groups
+    // that lie inside (F and H are multiples of 8)
+#pragma unroll
+    for (int q = 0; q < W / 8; ++q) {
+      if (col0 + c + 8 * q >= p.F) break;
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = g[8 * q + i];
+      store_bf16<8>(p.h + static_cast<size_t>(row) * p.F + col0 + c + 8 * q, o);
+    }
+  }
+}
+
+__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int row, float rs,
+                                float* xchg, const float* bsl) {
+  const int H = p.g[1].half;
+  const int col0 = t * H;
+  int c = 0;
+  for (; c + 32 <= H; c += 32) swiglu_chunk<32>(p, taddr, H, c, col0, row, rs, xchg, bsl);
+  for (; c < H; c += 8) swiglu_chunk<8>(p, taddr, H, c, col0, row, rs, xchg, bsl);
+}
+
+// Tile t's slice of the coupling vector b into shared memory (zeros past F),
+// fetched while the tile's MMAs run.
+__device__ void load_b_slice(const Params& p, int t, int et, float* bsl) {
+  const int H = p.g[1].half;
+  for (int i = et; i < H; i += kEpiThreads) {
+    const int col = t * H + i;
+    bsl[i] = (p.b != nullptr && col < p.F) ? __bfloat162float(p.b[col]) : 0.f;
+  }
+  epi_bar();
+}
+
+// R2 on this CTA's 4-column groups: thread et handles sequence j = et % 64
+// (rows j and mp + j), columns 2 (et / 64) .. + 1 of each group: x_out =
+// x_mid + the sum of the W_down partials in split order, the auxiliary row
+// adding c * (primary row's sum) first.
+__device__ bool reduce_down(const Params& p, int cta, int G, int et, uint8_t* rbuf,
+                            uint64_t* rfull, int& batches) {
+  const int j = et & 63, hc = (et >> 6) * 2;
+  const bool live = j < p.mp;
+  float2 ap = make_float2(0.f, 0.f), aa = make_float2(0.f, 0.f);
+  // residual (x_mid, written by other CTAs: read through L2) and coupling
+  // values of this thread's groups, loaded before the partials arrive
+  const int groups = p.d / 4;
+  uint32_t pre_p[kPreGroups], pre_a[kPreGroups], pre_c[kPreGroups];
+#pragma unroll
+  for (int i = 0; i < kPreGroups; ++i) {
+    const int gi = cta + i * G;
+    const bool in = live && gi < groups;
+    const int col = gi * 4 + hc;
+    pre_p[i] = in ? __ldcg(reinterpret_cast<const unsigned int*>(
+                        p.x_mid + static_cast<size_t>(j) * p.d + col))
+                  : 0u;
+    pre_a[i] = in ? __ldcg(reinterpret_cast<const unsigned int*>(
+                        p.x_mid + static_cast<size_t>(p.mp + j) * p.d + col))
+                  : 0u;
+    pre_c[i] = (in && p.c != nullptr) ? *reinterpret_cast<const uint32_t*>(p.c + col) : 0u;
+  }
+  return stream_partials(
+      p, p.g[2].splits, cta, G, rbuf, rfull, batches, et,
+      [&](int, int, const uint8_t* item) {
+        if (!live) return;
+        const float2 vp = *reinterpret_cast<const float2*>(item + j * 16 + hc * 4);
+        const float2 va = *reinterpret_cast<const float2*>(item + (p.mp + j) * 16 + hc * 4);
+        ap.x += vp.x;
+        ap.y += vp.y;
+        aa.x += va.x;
+        aa.y += va.y;
+      },
+      [&](int gi) {
+        if (live) {
+          const int col = gi * 4 + hc;
+          const int i = (gi - cta) / G;
+          uint32_t wp = 0u, wa = 0u, wc = 0u;
+          if (i < kPreGroups) {
+#pragma unroll
+            for (int k = 0; k < kPreGroups; ++k)
+              if (k == i) {
+                wp = pre_p[k];
+                wa = pre_a[k];
+                wc = pre_c[k];
+              }
+          } else {
+            wp = __ldcg(reinterpret_cast<const unsigned int*>(p.x_mid + static_cast<size_t>(j) * p.d + col));
+            wa = __ldcg(reinterpret_cast<const unsigned int*>(
+                p.x_mid + static_cast<size_t>(p.mp + j) * p.d + col));
+            if (p.c != nullptr) wc = *reinterpret_cast<const uint32_t*>(p.c + col);
+          }
+          float op[2] = {ap.x, ap.y}, oa[2] = {aa.x, aa.y};
+          if (p.c != nullptr) {
+            oa[0] = fmaf(bf16_bits_to_float(static_cast<uint16_t>(wc & 0xffffu)), op[0], oa[0]);
+            oa[1] = fmaf(bf16_bits_to_float(static_cast<uint16_t>(wc >> 16)), op[1], oa[1]);
+          }
+          op[0] += bf16_bits_to_float(static_cast<uint16_t>(wp & 0xffffu));
+          op[1] += bf16_bits_to_float(static_cast<uint16_t>(wp >> 16));
+          oa[0] += bf16_bits_to_float(static_cast<uint16_t>(wa & 0xffffu));
+          oa[1] += bf16_bits_to_float(static_cast<uint16_t>(wa >> 16));
+          *reinterpret_cast<__nv_bfloat162*>(p.x_out + static_cast<size_t>(j) * p.d + col) =
+              __floats2bfloat162_rn(op[0], op[1]);
+          *reinterpret_cast<__nv_bfloat162*>(p.x_out + static_cast<size_t>(p.mp + j) * p.d + col) =
+              __floats2bfloat162_rn(oa[0], oa[1]);
+        }
+        ap = make_float2(0.f, 0.f);
+        aa = make_float2(0.f, 0.f);
+      });
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -372,14 +547,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  uint8_t* rbuf = smem;  // the weight ring, while a reduction has it
   float* xchg = reinterpret_cast<float*>(smem + static_cast<size_t>(kStages) * kSlot);
-  float* red = xchg + kXchgFloats;                                // [16]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + 16);         // [kStages]
+  float* red = xchg + kXchgFloats;                                // [kEpiThreads]
+  float* bsl = red + kEpiThreads;                                 // [kMaxHalf] b of a tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);   // [kStages]
   uint64_t* empty = full + kStages;                               // [kStages]
   uint64_t* acc_full = empty + kStages;                           // [2]
   uint64_t* acc_empty = acc_full + 2;                             // [2]
   uint64_t* mma_done = acc_empty + 2;                             // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* rfull = mma_done + 1;     // reduction batch landed
+  uint64_t* ring_free = rfull + 1;    // R0 is done with the ring: gate/up weights may load
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_free + 1);
   // [0] abort, [1] epilogue broadcast, [2] / [3] stages issued by the weight /
   // activation producer
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -397,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], kEpiThreads / 32);
     }
     mbar_init(mma_done, 1);
+    mbar_init(rfull, 1);
+    mbar_init(ring_free, 1);
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
@@ -425,6 +606,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmWg);
       prefetch_tensormap(&tmWd);
       const uint64_t pol = l2_policy_evict_first();
+      // At a phase boundary the MMAs wait for the next phase's activations:
+      // the next phase's first weight tiles are prefetched into L2 there, so
+      // DRAM keeps streaming and those stages later load from L2. Before the
+      // first gate/up stage the ring is lent to the W_o reduction (R0): its
+      // loads wait until R0 has released it.
+      auto prefetch_phase = [&](int q, int count) {
+        StageCursor pf(p, cta, G);
+        while (!pf.done && pf.q < q) pf.next(p, cta, G);
+        for (int i = 0; i < count && !pf.done && pf.q == q; ++i) {
+          const Gemm& gq = p.g[q];
+          const CUtensorMap* tq = q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd);
+          if (q == 1) {
+            tma_prefetch_2d(tq, pf.kb * kBK, pf.tile * gq.half);
+            tma_prefetch_2d(tq, pf.kb * kBK, p.F + pf.tile * gq.half);
+          } else {
+            tma_prefetch_2d(tq, pf.kb * kBK, pf.tile * kTileN);
+          }
+          pf.next(p, cta, G);
+        }
+      };
       int s = 0;
       uint32_t ph = 0;
       long long n = 0;
@@ -432,6 +633,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
         const CUtensorMap* tm = q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd);
+        if (q >= 1) prefetch_phase(q, kBoundaryPrefetch);
+        if (q == 1 && !mbar_wait(ring_free, 0)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          flags[0] = 1;
+          ok = false;
+          break;
+        }
         for (int u = cta; u < g.units && ok; u += G) {
           int tile, k0, k1;
           unit_range(g, u, tile, k0, k1);
@@ -484,8 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           int tile, k0, k1;
           unit_range(g, u, tile, k0, k1);
           if (!ready) {
-            // P1 needs every row's xn2 (counter B), P2 every column of h (C)
-            if (!wait_count(p.cnt + (q == 1 ? kCntB : kCntC), G)) {
+            // P1 reads x_mid (counter A2), P2 every column of h (C)
+            if (!wait_count(p.cnt + (q == 1 ? kCntA2 : kCntC), G)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
               ok = false;
@@ -572,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue warps
     const int quarter = warp & 3;
     const int et = threadIdx.x - 3 * 32;
-    float* stg = xchg + (warp - 3) * 32 * kStgPitch;
+    const int row = quarter * 32 + lane;  // this thread's TMEM lane = accumulator row
     volatile int* eflag = flags + 1;
     int seg = 0;
     bool ok = true;
@@ -589,6 +797,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
     };
+    auto grid_wait = [&](int which) -> bool {
+      if (epi_wait_count(p.cnt + which, G, et, eflag)) return true;
+      if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+      flags[0] = 1;
+      return false;
+    };
+    auto acc_addr = [&](int acc) -> uint32_t {
+      return tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+             static_cast<uint32_t>(acc * 256);
+    };
     // P0: W_o partials
     for (int u = cta; u < p.g[0].units && ok; u += G, ++seg) {
       const int acc = seg & 1;
@@ -597,33 +815,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, taddr, quarter, lane, stg);
+      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, acc_addr(acc), row);
       give_acc(acc);
     }
     arrive_count(p.cnt + kCntA, et);
-    // R0: rows
-    for (int r = cta; r < p.M; r += G) {
-      if (!epi_wait_count(p.cnt + kCntA, G, et, eflag)) {
-        if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
-        flags[0] = 1;
-        break;
-      }
-      if (!flags[0]) reduce_o_row(p, r, et, red);
+    // R0: x_mid and this CTA's row sums of squares
+    // (the ring is idle: every W_o stage has been consumed, and the producers
+    // hold back the gate/up stages until ring_free)
+    int rbatches = 0;
+    if (grid_wait(kCntA) && !flags[0] && !reduce_o(p, cta, G, et, rbuf, rfull, rbatches)) {
+      if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+      flags[0] = 1;
     }
-    arrive_count(p.cnt + kCntB, et);
+    if (et == 0) mbar_arrive(ring_free);
+    arrive_count(p.cnt + kCntA2, et);
+    // row scales of the norm (CTA r < M computes row r)
+    if (cta < p.M && grid_wait(kCntA2) && !flags[0]) row_scale(p, G, cta, et, red);
+    arrive_count(p.cnt + kCntI, et);
     // P1: SwiGLU tiles straight from TMEM
+    float rs = 0.f;
+    bool have_rs = false;
     for (int u = cta; u < p.g[1].units && ok; u += G, ++seg) {
       const int acc = seg & 1;
+      if (!have_rs) {
+        if (!grid_wait(kCntI)) {
+          ok = false;
+          break;
+        }
+        rs = row < p.M ? __ldcg(p.rscale + row) : 0.f;
+        have_rs = true;
+      }
+      if (p.b != nullptr) load_b_slice(p, u, et, bsl);
       if (!take_acc(acc, seg)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      swiglu_epilogue(p, u, taddr, quarter, lane, xchg);
+      swiglu_epilogue(p, u, acc_addr(acc), row, rs, xchg, bsl);
       give_acc(acc);
     }
     arrive_count(p.cnt + kCntC, et);
@@ -635,20 +863,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * 256);
-      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, taddr, quarter, lane, stg);
+      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, acc_addr(acc), row);
       give_acc(acc);
     }
     arrive_count(p.cnt + kCntD, et);
-    // R2: (sequence, column half) units
-    for (int v = cta; v < p.r2_units; v += G) {
-      if (!epi_wait_count(p.cnt + kCntD, G, et, eflag)) {
-        if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
-        flags[0] = 1;
-        break;
-      }
-      if (!flags[0]) reduce_down_pair(p, v, et);
+    // R2: x_out (the ring is idle again: every W_down stage has been consumed)
+    if (grid_wait(kCntD) && !flags[0] && !reduce_down(p, cta, G, et, rbuf, rfull, rbatches)) {
+      if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
+      flags[0] = 1;
     }
   }
 
@@ -717,9 +939,19 @@ Plan make_plan(int M, int mp, int d, int qd, int F) {
   return pl;
 }
 
-size_t workspace_bytes(const Plan& pl) {
+// Workspace: counters | ss_part [G][128] | rscale [128] | partials.
+struct WsLayout {
+  size_t ss, rscale, part, total;
+};
+
+WsLayout ws_layout(const Plan& pl) {
   const int units = pl.T0 * pl.S0 > pl.T2 * pl.S2 ? pl.T0 * pl.S0 : pl.T2 * pl.S2;
-  return kCounterBytes + static_cast<size_t>(units) * kBM * kTileN * 4;
+  WsLayout l;
+  l.ss = kCounterBytes;
+  l.rscale = l.ss + round_up(static_cast<size_t>(pl.G) * kBM * 4, 256);
+  l.part = l.rscale + round_up(kBM * 4, 256);
+  l.total = l.part + static_cast<size_t>(units) * kBM * kTileN * 4;
+  return l;
 }
 
 std::mutex g_mu;
@@ -731,27 +963,28 @@ bool g_attr[64] = {};
 extern "C" size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model,
                                                                int q_dim, int F) {
   const df::post::Plan pl = df::post::make_plan(2 * m_primary, m_primary, d_model, q_dim, F);
-  return pl.ok ? df::post::workspace_bytes(pl) : 0;
+  return pl.ok ? df::post::ws_layout(pl).total : 0;
 }
 
 extern "C" df_status dualflow_layer_post_attention(
     const void* attn, const void* x, const void* w_o, const void* w_gu, const void* w_down,
     const void* b, const void* c, int m_primary, int d_model, int q_dim, int F, float eps,
-    void* x_mid, void* xn2, void* h, void* x_out, void* workspace, size_t workspace_bytes,
+    void* x_mid, void* h, void* x_out, void* workspace, size_t workspace_bytes,
     int32_t* err_flag, void* stream) {
   using namespace df;
   using namespace df::post;
-  if (!attn || !x || !w_o || !w_gu || !w_down || !x_mid || !xn2 || !h || !x_out)
+  if (!attn || !x || !w_o || !w_gu || !w_down || !x_mid || !h || !x_out)
     return DF_ERR_NULL;
   if (m_primary < 1 || d_model < 1 || q_dim < 1 || F < 1 || !(eps >= 0.f)) return DF_ERR_SHAPE;
   const int M = 2 * m_primary;
   const Plan pl = make_plan(M, m_primary, d_model, q_dim, F);
   if (!pl.ok) return DF_ERR_UNSUPPORTED;
-  const void* ptrs[] = {attn, x, w_o, w_gu, w_down, x_mid, xn2, h, x_out};
+  const void* ptrs[] = {attn, x, w_o, w_gu, w_down, x_mid, h, x_out};
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DF_ERR_ALIGN;
   if ((b && !aligned(b, 16)) || (c && !aligned(c, 16))) return DF_ERR_ALIGN;
-  if (!workspace || workspace_bytes < df::post::workspace_bytes(pl) || !aligned(workspace, 256))
+  const WsLayout wl = ws_layout(pl);
+  if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 256))
     return DF_ERR_WORKSPACE;
 
   Params p{};
@@ -767,16 +1000,17 @@ extern "C" df_status dualflow_layer_post_attention(
                 make_idesc(kBM, 2 * pl.H1)};
   p.g[2] = Gemm{pl.T2 * pl.S2, pl.S2, F / kBK, kTileN, 0, kTileN * kBK * 2,
                 make_idesc(kBM, kTileN)};
-  p.r2_units = 2 * m_primary;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.b = static_cast<const __nv_bfloat16*>(b);
   p.c = static_cast<const __nv_bfloat16*>(c);
   p.x_mid = static_cast<__nv_bfloat16*>(x_mid);
-  p.xn2 = static_cast<__nv_bfloat16*>(xn2);
   p.h = static_cast<__nv_bfloat16*>(h);
   p.x_out = static_cast<__nv_bfloat16*>(x_out);
-  p.cnt = static_cast<int*>(workspace);
-  p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  p.cnt = reinterpret_cast<int*>(w8);
+  p.ss_part = reinterpret_cast<float*>(w8 + wl.ss);
+  p.rscale = reinterpret_cast<float*>(w8 + wl.rscale);
+  p.part = reinterpret_cast<float*>(w8 + wl.part);
   p.err = err_flag;
 
   CUtensorMap tmXo, tmWo, tmXg, tmWg, tmXd, tmWd;
@@ -784,7 +1018,7 @@ extern "C" df_status dualflow_layer_post_attention(
                  qu = static_cast<uint64_t>(q_dim), Fu = static_cast<uint64_t>(F);
   if (!encode_tmap_bf16_2d(&tmXo, attn, Mu, qu, qu * 2, kBM, kBK) ||
       !encode_tmap_bf16_2d(&tmWo, w_o, du, qu, qu * 2, kTileN, kBK) ||
-      !encode_tmap_bf16_2d(&tmXg, xn2, Mu, du, du * 2, kBM, kBK) ||
+      !encode_tmap_bf16_2d(&tmXg, x_mid, Mu, du, du * 2, kBM, kBK) ||
       !encode_tmap_bf16_2d(&tmWg, w_gu, 2 * Fu, du, du * 2, static_cast<uint32_t>(pl.H1), kBK) ||
       !encode_tmap_bf16_2d(&tmXd, h, Mu, Fu, Fu * 2, kBM, kBK) ||
       !encode_tmap_bf16_2d(&tmWd, w_down, du, Fu, Fu * 2, kTileN, kBK))

@@ -510,6 +510,15 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
   return fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])), fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
 }
 
+// 2^x by the SFU's approximate base-2 exponential (relative error near
+// 2^-22, far below the bf16 rounding of P; results under 2^-126 flush to 0,
+// which only drops weights below 2^-126 of the row's largest).
+__device__ __forceinline__ float exp2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // P of 32 keys (chunks c0 .. c0 + 3 of 8 keys) of row r: bf16 into the
 // swizzled row (16-byte chunk c of row r at chunk c ^ (r & 7)); returns the
 // fp32 sum of the weights.
@@ -521,8 +530,8 @@ __device__ __forceinline__ float write_p32(uint8_t* prow, int r, int c0, const f
     uint32_t w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float a = exp2f(fmaf(s[8 * q + 2 * k], scale_log2, -mu));
-      const float b = exp2f(fmaf(s[8 * q + 2 * k + 1], scale_log2, -mu));
+      const float a = exp2_sfu(fmaf(s[8 * q + 2 * k], scale_log2, -mu));
+      const float b = exp2_sfu(fmaf(s[8 * q + 2 * k + 1], scale_log2, -mu));
       sum[k & 1] += a + b;
       w[k] = pack_f32_bf16x2(a, b);
     }
@@ -710,8 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma::tc_fence_after();
       float s0[32], s1[32];
-      umma::tmem_ld<32>(t_lane + sb * kPage, s0);
-      umma::tmem_ld<32>(t_lane + sb * kPage + 32, s1);
+      umma::tmem_ld32x2(t_lane + sb * kPage, s0, s1);
       umma::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
@@ -955,21 +963,28 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       constexpr uint32_t kIdS = umma::make_idesc(kRows, kPage);             // Q K^T
       constexpr uint32_t kIdPV = umma::make_idesc(kRows, 64) | (1u << 16);  // P V, V MN-major
       bool ok = mbar_wait(q_full, 0);
+      // Descriptors are affine in the byte address (its bits 4..17 sit in the
+      // low field): each one below is a base plus a constant, so the issue
+      // loop spends its instructions on the MMAs.
+      const uint64_t dq0 = umma::smem_desc(smem_u32(smem));
+      const uint64_t dstage0 = umma::smem_desc(smem_u32(smem + Lay::kOffStages));
+      const uint64_t dv0 =
+          smem_desc_mn64(smem_u32(smem + Lay::kOffStages + Lay::kPageBytes));
+      const uint64_t dp0 = umma::smem_desc(smem_u32(smem + Lay::kOffP));
       // S_i of tile t into its TMEM buffer i & 1
       auto issue_s = [&](int t, int i) -> bool {
         const int st = i % kStages, sb = i & 1;
         if (!mbar_wait(&full[st], (i / kStages) & 1)) return false;
         if (i >= 2 && !mbar_wait(&s_free[2 * t + sb], ((i >> 1) - 1) & 1)) return false;
         umma::tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + t * Lay::kQBytes);
-        const uint32_t k_addr = smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes);
+        const uint64_t dq = dq0 + static_cast<uint64_t>((t * Lay::kQBytes) >> 4);
+        const uint64_t dk = dstage0 + static_cast<uint64_t>((st * Lay::kStageBytes) >> 4);
+        const uint32_t d_tmem = tmem + t * 256 + sb * kPage;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int hf = kk >> 2, kq = kk & 3;
-          umma::umma_bf16(tmem + t * 256 + sb * kPage,
-                          umma::smem_desc(q_addr + hf * (kRows * 128) + kq * 32),
-                          umma::smem_desc(k_addr + hf * (kPage * 128) + kq * 32), kIdS,
-                          kk > 0 ? 1u : 0u);
+          umma::umma_bf16(d_tmem, dq + ((hf * (kRows * 128) + kq * 32) >> 4),
+                          dk + ((hf * (kPage * 128) + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
         }
         umma::umma_commit(&s_full[2 * t + sb]);
         return true;
@@ -979,15 +994,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const int pb = i & 1, st = i % kStages;
         if (!mbar_wait(&p_full[2 * t + pb], (i >> 1) & 1)) return false;
         umma::tc_fence_after();
-        const uint32_t p_addr = smem_u32(smem + Lay::kOffP + (2 * t + pb) * Lay::kPBytes);
-        const uint32_t v_addr =
-            smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes);
+        const uint64_t dp = dp0 + static_cast<uint64_t>(((2 * t + pb) * Lay::kPBytes) >> 4);
+        const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kStageBytes) >> 4);
+        const uint32_t d_tmem = tmem + t * 256 + kOCol;
 #pragma unroll
         for (int kk = 0; kk < kPage / 16; ++kk) {
 #pragma unroll
           for (int hf = 0; hf < H; ++hf)
-            umma::umma_bf16(tmem + t * 256 + kOCol + hf * 64, umma::smem_desc(p_addr + kk * 32),
-                            smem_desc_mn64(v_addr + hf * (kPage * 128) + kk * 2048), kIdPV,
+            umma::umma_bf16(d_tmem + hf * 64, dp + ((kk * 32) >> 4),
+                            dv + ((hf * (kPage * 128) + kk * 2048) >> 4), kIdPV,
                             (i > 0 || kk > 0) ? 1u : 0u);
         }
         umma::umma_commit(&pv_done[2 * t + pb]);
@@ -1028,8 +1043,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       umma::tc_fence_after();
       float s0[32], s1[32];
-      umma::tmem_ld<32>(t_lane + sb * kPage, s0);
-      umma::tmem_ld<32>(t_lane + sb * kPage + 32, s1);
+      umma::tmem_ld32x2(t_lane + sb * kPage, s0, s1);
       umma::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&my_s_free[sb]);

@@ -17,7 +17,9 @@ Composition of library calls only (each step is a libdualflow kernel):
 With fused_post=True, steps 5-8 run as one persistent launch
 (dualflow_layer_post_attention) when the sizes allow it: its weight producers
 stream W_o, W_gate/up and W_down back to back instead of four launches each
-ramping up and draining. The default keeps the four calls.
+ramping up and draining, and the norm's row scale multiplies the gate/up
+accumulators (the normalised rows are not stored). The default keeps the four
+calls.
 
 Pages: "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
 Core" (shared matrices, primary-only cache writes, auxiliary flow active at
@@ -163,8 +165,8 @@ class DualFlowLayer:
                             err_flag=self.err, stream=stream)
         elif self.fused_post:
             api.layer_post_attention(self.attn, X, w["w_o"], w["w_gu"], w["w_down"], w["b"],
-                                     w["c"], eps=self.eps, x_mid=self.x_mid, xn2=self.xn2,
-                                     h=self.h, x_out=self.x_out, workspace=self.post_ws,
+                                     w["c"], eps=self.eps, x_mid=self.x_mid, h=self.h,
+                                     x_out=self.x_out, workspace=self.post_ws,
                                      err_flag=self.err, stream=stream)
         else:
             api.grouped_proj(self.attn, B, w["w_o"], y=self.x_mid, epilogue="residual",

@@ -367,42 +367,45 @@ int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue
 /* [0, m_primary) primary and [m_primary, 2 m_primary) auxiliary (sequence j */
 /* = rows j and m_primary + j), M = 2 m_primary:                             */
 /*   x_mid = x + attn W_o^T                                                  */
-/*   xn2   = x_mid / sqrt(mean_row(x_mid^2) + eps)        (unit gain)         */
-/*   h     = SiLU(xn2 W_gate^T) * (xn2 W_up^T); aux rows += b (.) primary h   */
+/*   r     = 1 / sqrt(mean_row(x_mid^2) + eps)   (RMSNorm, unit gain)         */
+/*   h     = SiLU(r x_mid W_gate^T) * (r x_mid W_up^T); aux rows += b (.)     */
+/*           primary h                                                       */
 /*   x_out = x_mid + h W_down^T; aux rows += c (.) (h W_down^T) of primary   */
 /* which is dualflow_grouped_proj (residual) -> dualflow_rmsnorm ->          */
 /* dualflow_grouped_proj (swiglu, b) -> dualflow_grouped_proj (residual, c)  */
 /* computed by one grid of one CTA per SM whose TMA producers stream the     */
 /* three weights back to back; the dependencies between the steps are       */
-/* grid-wide counters in the workspace (bounded waits). Each split-k sum is  */
-/* taken in a fixed order, so results are deterministic and primary rows    */
-/* never depend on auxiliary rows. The result matches the four-call form    */
-/* within the bf16 tolerance, not bit for bit (other split-k orders).        */
+/* grid-wide counters in the workspace (bounded waits). The norm's row scale */
+/* multiplies the gate/up accumulators (the normalised rows are not rounded  */
+/* to bf16 and stored). Each split-k sum is taken in a fixed order, so the   */
+/* results are deterministic and primary rows never depend on auxiliary      */
+/* rows. They match the four-call form within the bf16 tolerance, not bit    */
+/* for bit (other split-k orders, no bf16 rounding of the normalised rows).  */
 /*                                                                           */
 /* attn  : bf16 [M][q_dim] (the attention output, O1 rows then O2 rows).      */
 /* x     : bf16 [M][d_model] (the layer input, residual of W_o).             */
 /* w_o [d_model][q_dim], w_gu [2F][d_model] (gate rows, then up rows),       */
 /* w_down [d_model][F]: bf16, row-major. b [F], c [d_model] bf16 or NULL.     */
-/* x_mid, xn2 [M][d_model], h [M][F], x_out [M][d_model]: bf16, written      */
-/* (all rows packed, 16-byte aligned). w_* are read before the wait for the  */
-/* kernel launched ahead on the stream (programmatic dependent launch), so   */
-/* that kernel must not write them.                                          */
+/* x_mid [M][d_model], h [M][F], x_out [M][d_model]: bf16, written (all rows */
+/* packed, 16-byte aligned). w_* are read before the wait for the kernel     */
+/* launched ahead on the stream (programmatic dependent launch), so that     */
+/* kernel must not write them.                                               */
 /* workspace: >= dualflow_layer_post_attention_workspace_size(...) bytes,     */
 /* 256-byte aligned, ZERO-FILLED once: its first bytes are grid counters     */
 /* that every completed call leaves at zero (after a DF_DEVERR_TIMEOUT,      */
-/* zero it again); the rest holds fp32 split-k partials. Calls sharing one  */
-/* workspace must not overlap on the GPU.                                    */
+/* zero it again); the rest holds fp32 split-k partials and the row sums of  */
+/* the norm. Calls sharing one workspace must not overlap on the GPU.        */
 /* Supported (else DF_ERR_UNSUPPORTED; the size query returns 0):            */
 /* 1 <= m_primary <= 64, d_model % 256 == 0, q_dim % 64 == 0, F % 64 == 0,   */
-/* F <= 112 * (SM count). One kernel launch.                                  */
+/* F <= 128 * (SM count). One kernel launch.                                  */
 /* ------------------------------------------------------------------------ */
 size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model, int q_dim,
                                                     int F);
 df_status dualflow_layer_post_attention(const void* attn, const void* x, const void* w_o,
                                         const void* w_gu, const void* w_down, const void* b,
                                         const void* c, int m_primary, int d_model, int q_dim,
-                                        int F, float eps, void* x_mid, void* xn2, void* h,
-                                        void* x_out, void* workspace, size_t workspace_bytes,
+                                        int F, float eps, void* x_mid, void* h, void* x_out,
+                                        void* workspace, size_t workspace_bytes,
                                         int32_t* err_flag, void* stream);
 
 /* ------------------------------------------------------------------------ */

@@ -20,6 +20,7 @@ from .dualflow_oracle import (  # noqa: F401
     residual_couple,
     rmsnorm,
     layer_step,
+    LAYER_INTERFACES,
     softmax_rows,
     collision_probability,
     mixture_weight,

@@ -372,8 +372,12 @@ def rmsnorm(x, gain=None, eps=1e-5):
     return y
 
 
+LAYER_INTERFACES = ("xn", "qkv", "attn", "x_mid", "xn2", "h", "x_out")
+
+
 def layer_step(x1, x2, w_qkv, w_o, w_gu, w_down, a, b, c, k_cache, v_cache,
-               block_table, positions, Hq, Hkv, D, F, round_bf16=True, eps=1e-5):
+               block_table, positions, Hq, Hkv, D, F, round_bf16=True, eps=1e-5,
+               rounded=LAYER_INTERFACES):
     """One Dual-Flow decoder layer at one generated position, both flows.
 
     Composition (pages "Sintesi Tecnica", sections "Architettura Core",
@@ -388,19 +392,27 @@ def layer_step(x1, x2, w_qkv, w_o, w_gu, w_down, a, b, c, k_cache, v_cache,
     w_qkv [(Hq + 2 Hkv) D, d_model]; w_o [d_model, Hq D];
     w_gu [2F, d_model] (gate rows then up rows); w_down [d_model, F].
     positions[b]: cache length before this step (the slot the append writes).
-    With round_bf16, every intermediate that the CUDA path stores as a bf16
-    tensor is rounded to bf16 here too (same interfaces, same order).
+    With round_bf16, every intermediate named in `rounded` (by default all
+    the tensors a four-call layer step stores as bf16) is rounded to bf16
+    here too, in the same order; an implementation that keeps an intermediate
+    in fp32 (a normalised row scaled inside a GEMM epilogue instead of stored)
+    is compared with that name left out.
     Returns a dict of float64 arrays (and the updated caches).
     """
-    r = bf16_round if round_bf16 else (lambda t: np.asarray(t, dtype=F64))
+    exact = lambda t: np.asarray(t, dtype=F64)  # noqa: E731
+    rset = frozenset(rounded) if round_bf16 else frozenset()
+    unknown = rset - frozenset(LAYER_INTERFACES)
+    if unknown:
+        raise ValueError("unknown interfaces %s" % sorted(unknown))
+    rd = {name: (bf16_round if name in rset else exact) for name in LAYER_INTERFACES}
     x1 = np.asarray(x1, dtype=F64)
     x2 = np.asarray(x2, dtype=F64)
     B = x1.shape[0]
     X = np.concatenate([x1, x2], axis=0)
     qd, kvd = Hq * D, Hkv * D
 
-    xn = r(rmsnorm(X, eps=eps))
-    qkv = r(grouped_proj(xn, w_qkv, B, n_aux=qd))
+    xn = rd["xn"](rmsnorm(X, eps=eps))
+    qkv = rd["qkv"](grouped_proj(xn, w_qkv, B, n_aux=qd))
     k_new = qkv[:B, qd:qd + kvd].reshape(B, Hkv, D)
     v_new = qkv[:B, qd + kvd:qd + 2 * kvd].reshape(B, Hkv, D)
     kc, vc = kv_append(k_new, v_new, k_cache, v_cache, block_table, positions)
@@ -408,11 +420,11 @@ def layer_step(x1, x2, w_qkv, w_o, w_gu, w_down, a, b, c, k_cache, v_cache,
     q1 = qkv[:B, :qd].reshape(B, Hq, D)
     q2raw = qkv[B:, :qd].reshape(B, Hq, D)
     o1, o2 = decode_attn(q1, q2raw, a, kc, vc, block_table, seqlens)
-    attn = r(np.concatenate([o1.reshape(B, qd), o2.reshape(B, qd)], axis=0))
-    x_mid = r(residual_couple(grouped_proj(attn, w_o, B), X, B, None))
-    xn2 = r(rmsnorm(x_mid, eps=eps))
-    h = r(swiglu_couple(grouped_proj(xn2, w_gu, B), F, B, b))
-    x_out = r(residual_couple(grouped_proj(h, w_down, B), x_mid, B, c))
+    attn = rd["attn"](np.concatenate([o1.reshape(B, qd), o2.reshape(B, qd)], axis=0))
+    x_mid = rd["x_mid"](residual_couple(grouped_proj(attn, w_o, B), X, B, None))
+    xn2 = rd["xn2"](rmsnorm(x_mid, eps=eps))
+    h = rd["h"](swiglu_couple(grouped_proj(xn2, w_gu, B), F, B, b))
+    x_out = rd["x_out"](residual_couple(grouped_proj(h, w_down, B), x_mid, B, c))
     return {
         "xn": xn, "qkv": qkv, "k_cache": kc, "v_cache": vc, "attn": attn,
         "x_mid": x_mid, "xn2": xn2, "h": h, "x_out": x_out,

@@ -123,7 +123,7 @@ MUTATIONS = {
     "MLP fed from the first norm xn": ("grouped_proj(xn2, w_gu, B)", "grouped_proj(xn, w_gu, B)"),
     "QKV built from X, not xn": ("grouped_proj(xn, w_qkv, B, n_aux=qd)",
                                  "grouped_proj(X, w_qkv, B, n_aux=qd)"),
-    "second norm dropped": ("xn2 = r(rmsnorm(x_mid, eps=eps))", "xn2 = r(x_mid)"),
+    "second norm dropped": ('xn2 = rd["xn2"](rmsnorm(x_mid, eps=eps))', 'xn2 = rd["xn2"](x_mid)'),
     "attention residual taken from xn": ("grouped_proj(attn, w_o, B), X, B, None)",
                                          "grouped_proj(attn, w_o, B), xn, B, None)"),
     "MLP residual taken from X": ("grouped_proj(h, w_down, B), x_mid, B, c)",
@@ -158,6 +158,30 @@ def test_worked_example_catches_planted_wiring_mistake(name):
 def test_unmutated_copy_passes():
     # the mutation harness itself: a copy with a no-op substitution is exact
     spec = _spec()
-    out = _mutant("xn2 = r(rmsnorm(x_mid, eps=eps))", "xn2 = r(rmsnorm(x_mid, eps=eps))")(
-        **_inputs(spec))
+    same = 'xn2 = rd["xn2"](rmsnorm(x_mid, eps=eps))'
+    out = _mutant(same, same)(**_inputs(spec))
     assert _mismatches(out, spec) == []
+
+
+def test_rounded_interfaces_option():
+    # `rounded` names the intermediates rounded to bf16: all of them by
+    # default, none equals round_bf16=False, one left out differs from the
+    # default only from that point on (here xn2: x_mid is unchanged, h is not).
+    spec = _spec()
+    inp = _inputs(spec)
+    inp["round_bf16"] = True
+    inp["eps"] = 1e-5
+    full = oracle.layer_step(**inp)
+    same = oracle.layer_step(**dict(inp, rounded=oracle.LAYER_INTERFACES))
+    none = oracle.layer_step(**dict(inp, rounded=()))
+    exact = oracle.layer_step(**dict(inp, round_bf16=False))
+    keep = oracle.layer_step(**dict(inp, rounded=tuple(n for n in oracle.LAYER_INTERFACES
+                                                        if n != "xn2")))
+    for k in ("xn", "qkv", "attn", "x_mid", "xn2", "h", "x_out"):
+        np.testing.assert_array_equal(full[k], same[k])
+        np.testing.assert_array_equal(none[k], exact[k])
+    np.testing.assert_array_equal(keep["x_mid"], full["x_mid"])
+    assert not np.array_equal(keep["xn2"], full["xn2"])
+    np.testing.assert_array_equal(keep["xn2"], oracle.rmsnorm(full["x_mid"], eps=1e-5))
+    with pytest.raises(ValueError):
+        oracle.layer_step(**dict(inp, rounded=("xn3",)))
