@@ -1,4 +1,5 @@
-// Post-attention half of the Dual-Flow decoder layer as ONE persistent kernel.
+// Post-attention half of the Dual-Flow decoder layer as ONE persistent kernel
+// launched as clusters of 4 CTAs.
 //
 // Method: "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
 // Core" (both flows share the output and MLP matrices), "Meccanismi Chiave"
@@ -15,40 +16,41 @@
 //
 // Why one kernel: at M = 128 rows every projection is a weight stream (about
 // 128 flop per weight byte, below the B200 ridge). Separate launches leave
-// HBM idle at every boundary: the next launch's CTAs cannot become resident
-// until the previous launch's CTAs (one per SM) have run their tails, and
-// then each pays a first TMA round trip. Here one CTA per SM walks all three
-// GEMMs in order and its TMA producer streams the weights continuously, into
-// a 4-stage ring, across the phase boundaries; only the activation tiles of a
-// phase wait for the phase before it. The dependencies between phases are
-// grid-wide counters in the workspace (every CTA is resident: one per SM,
-// grid = SM count), each wait bounded.
+// HBM idle at every boundary. Here one CTA per SM walks all three GEMMs in
+// order and its TMA producer streams the weights continuously, into a 4-stage
+// ring, across the phase boundaries; only the activation tiles of a phase
+// wait for the phase before it.
 //
-// Phases (units are spread over the CTAs, CTA i takes units i, i + G, ...):
-//   P0  W_o:    column tiles of 256 x S0 k-ranges -> fp32 partials
-//   --- counter A --- R0: 4-column groups over all CTAs: x_mid = x + the sum
-//                     of the partials (split order), and each CTA's partial
-//                     sum of squares per row
-//   --- counter A2 --- P1 may read x_mid; CTA r < M sums row r's squares in
-//                     CTA order -> r_row   --- counter I ---
-//   P1  W_gate/W_up: one tile of 2*H1 weight rows per CTA, SwiGLU (row scale
-//                     r) + b coupling straight from TMEM -> h
-//   --- counter C --- P2  W_down: column tiles of 256 x S2 k-ranges -> partials
-//   --- counter D --- R2: 4-column groups over all CTAs: residual + c
-//                     coupling -> x_out
-// Partials are stored [unit][column group of 4][row][4] fp32: a warp's store
-// (32 consecutive rows of one group) is one contiguous 512-byte segment, and a
-// (group, split) item is one contiguous 2 KB block. The reductions bring all
-// their items into the idle 192 KB weight ring with bulk TMA copies, one
-// round trip at the layer's sizes (a latency-bound loop of loads took 13 us);
-// the gate/up weight loads wait for the ring, and the gap is covered by L2
-// prefetches of the next phase's first weight tiles, issued at each phase
-// boundary only (prefetching ahead all the time took TMA bandwidth from the
-// loads).
+// Why clusters: W_o and W_down have only d / 128 output tiles of 128 columns,
+// too few for the SMs, so their K dimension is split 4 ways. The 4 splits of
+// a tile run on the 4 CTAs of one cluster, and the split sum is a
+// reduce-scatter through distributed shared memory: rank r owns columns
+// 32 r .. 32 r + 31 of the tile, every other rank writes its fp32 slice of
+// those columns straight from its TMEM accumulator into r's receive buffer
+// (st.async, completing on r's mbarrier), and r adds the four slices in rank
+// order. No partial sum goes through global memory and no grid-wide barrier
+// is needed for a split reduction.
+//
+// Phases (cluster c = blockIdx.x / 4, rank = blockIdx.x % 4, G CTAs):
+//   P0  W_o: cluster c < d/128 takes column tile c, rank r the r-th quarter
+//       of K; reduce-scatter; the owner of a 32-column slice stores x_mid =
+//       bf16(x + sum) and its rows' sums of squares over the slice
+//   --- grid counter A2: x_mid and every slice's sums of squares are stored
+//   P1  W_gate/W_up: tiles of 2*H1 weight rows spread over all CTAs (CTA i
+//       takes i, i + G, ...); each CTA sums the slices' squares of its rows
+//       (slice order) for r; SwiGLU + b coupling straight from TMEM -> h
+//   --- grid counter C: every column of h is stored
+//   P2  W_down: as P0 over K = F; the owner adds x_mid and the c coupling
+//       (the primary row's sum reaches its auxiliary row through shared
+//       memory) -> x_out
+// Every cluster is resident (one CTA per SM, grid = 4 x the device's maximum
+// of co-resident 4-CTA clusters), so the grid counters cannot deadlock; every
+// wait is bounded.
 // Roles (224 threads): warp 0 weight producer, warp 1 MMA issuer (one thread,
 // tcgen05.mma M = 128 into two 256-column TMEM accumulators), warp 2
-// activation producer, warps 3-6 epilogue (TMEM lane quarter = warp % 4).
-// Every split reduction sums in a fixed order: results are deterministic, and
+// activation producer, warps 3-6 epilogue (TMEM lane quarter = warp % 4,
+// thread = accumulator row).
+// Every split sum is taken in a fixed order: results are deterministic, and
 // primary rows never read auxiliary rows.
 #include <math.h>
 #include <string.h>
@@ -69,25 +71,30 @@ constexpr int kBK = 64;
 constexpr int kThreads = 224;
 constexpr int kEpiThreads = 128;
 constexpr int kStages = 4;
-constexpr int kXBytes = kBM * kBK * 2;            // 16 KB activation tile
-constexpr int kSlot = kXBytes + 256 * kBK * 2;    // + up to 32 KB of weights
-constexpr int kTileN = 256;                       // W_o / W_down column tile
-constexpr int kMaxHalf = 128;                     // SwiGLU output columns per tile
-constexpr int kXchgPitch = 33;                    // coupling exchange: [64 rows][32 + 1]
-constexpr int kXchgFloats = 64 * kXchgPitch;
+constexpr int kCluster = 4;                          // CTAs per cluster = K splits
+constexpr int kTileN = 128;                          // W_o / W_down columns per cluster
+constexpr int kSliceN = kTileN / kCluster;           // columns a rank owns: 32
+constexpr int kMaxHalf = 112;                        // SwiGLU output columns per tile
+constexpr int kXBytes = kBM * kBK * 2;               // 16 KB activation tile
+constexpr int kSlot = kXBytes + 2 * kMaxHalf * kBK * 2;  // + up to 28 KB of weights
+constexpr int kRecvSlotBytes = kBM * kSliceN * 4;    // one sender's slice: 16 KB
+constexpr int kRecvBytes = (kCluster - 1) * kRecvSlotBytes;
+constexpr int kXchgPitch = 33;                       // coupling exchange: [64 rows][32 + 1]
+constexpr int kXchgFloats = 64 * kXchgPitch;         // aliases the receive buffer
 constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
-constexpr int kGroupBytes = kBM * 4 * 4;          // one 4-column group of a partial: 2 KB
-constexpr int kRedItems = kStages * kSlot / kGroupBytes;  // reduction batch: the whole ring
-constexpr int kBoundaryPrefetch = 16;             // next-phase weight stages prefetched to L2
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kSlot + kXchgFloats * 4 +
-                              kEpiThreads * 4 + kMaxHalf * 4 + 256;  // + barriers, flags
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kSlot + kRecvBytes +
+                              kMaxHalf * 4 + 256;    // + barriers, flags
+static_assert(kSlot % 1024 == 0, "ring slots keep the 1024-byte swizzle alignment");
+static_assert(kTileN * kBK * 2 <= kSlot - kXBytes, "W_o / W_down stage fits a slot");
+static_assert(kXchgFloats * 4 <= kRecvBytes, "exchange fits the receive buffer");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-enum { kCntA = 0, kCntA2 = 1, kCntI = 2, kCntC = 3, kCntD = 4, kCntExit = 5 };
+enum { kCntA2 = 0, kCntC = 1, kCntExit = 2 };
 
 struct Gemm {
-  int units, splits, kblocks;
+  int units;    // P0 / P2: column tiles (one per cluster); P1: SwiGLU tiles
+  int kblocks;  // 64-wide K blocks of the whole product
   int BN;       // MMA N
   int half;     // SwiGLU output columns per tile (0: plain)
   int w_bytes;  // weight bytes per stage
@@ -104,15 +111,28 @@ struct Params {
   __nv_bfloat16* x_mid;
   __nv_bfloat16* h;
   __nv_bfloat16* x_out;
-  float* part;     // [units][64 groups][128 rows][4] fp32
-  float* ss_part;  // [G][128] per-CTA partial sums of squares of x_mid rows
-  float* rscale;   // [128] RMSNorm row scales
+  float* ss_part;  // [d / 32 slices][128 rows] sums of squares of stored x_mid values
   int* cnt;        // [kCounters]
   int32_t* err;
 };
 
 __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+// Epilogue barrier that also ANDs a predicate over the epilogue threads, so
+// that a wait which gave up in one thread stops all of them together.
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -125,18 +145,56 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
-__device__ __forceinline__ float4 ld_cg4(const float* p) {
-  float4 v;
-  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
 
-__device__ __forceinline__ void st_cg4(float* p, float4 v) {
-  asm volatile("st.global.cg.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
-               : "memory");
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+
+// All threads of all CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The address of this CTA's shared-memory location `addr` in cluster rank `rank`.
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// 16 bytes into another CTA's shared memory, counted on its mbarrier.
+__device__ __forceinline__ void st_async16(uint32_t raddr, float a, float b, float c, float d,
+                                           uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, "
+      "[%5];" ::"r"(raddr),
+      "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
+      "r"(__float_as_uint(d)), "r"(rbar)
+      : "memory");
+}
+
+// 32 bf16 values written by other CTAs of this launch (read through L2).
+__device__ __forceinline__ void load_bf16x32_cg(const __nv_bfloat16* src, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "l"(src + 8 * q));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * q + 2 * k] = bf16_bits_to_float(static_cast<uint16_t>(w[k] & 0xffffu));
+      v[8 * q + 2 * k + 1] = bf16_bits_to_float(static_cast<uint16_t>(w[k] >> 16));
+    }
+  }
 }
 
 // Single-thread bounded wait until *cnt >= target (every CTA of the grid has
@@ -151,53 +209,25 @@ __device__ bool wait_count(const int* cnt, int target) {
   return true;
 }
 
-// (tile, first k-block, end k-block) of unit u of GEMM g.
-__device__ __forceinline__ void unit_range(const Gemm& g, int u, int& tile, int& k0, int& k1) {
-  if (g.splits > 1) {
-    tile = u / g.splits;
-    const int s = u - tile * g.splits;
-    k0 = s * g.kblocks / g.splits;
-    k1 = (s + 1) * g.kblocks / g.splits;
-  } else {
-    tile = u;
+// This CTA's units of GEMM q: P0 / P2 one column tile per cluster (the
+// cluster's index, if it has one), P1 tiles cta, cta + G, ...; and the
+// k-blocks [k0, k1) of a unit (rank r's quarter for P0 / P2; may be empty
+// when the product has fewer than 4 k-blocks).
+struct Units {
+  int first, step;
+};
+__device__ __forceinline__ Units units_of(const Gemm& g, int q, int cta, int cid, int G) {
+  return q == 1 ? Units{cta, G} : Units{cid, g.units};
+}
+__device__ __forceinline__ void k_range(const Gemm& g, int q, int rank, int& k0, int& k1) {
+  if (q == 1) {
     k0 = 0;
     k1 = g.kblocks;
+  } else {
+    k0 = rank * g.kblocks / kCluster;
+    k1 = (rank + 1) * g.kblocks / kCluster;
   }
 }
-
-// Walks this CTA's stage sequence (GEMM q, its units u = cta, cta + G, ...,
-// their k-blocks) in the order the producers and the MMA issuer use.
-struct StageCursor {
-  int q, u, kb, k1, tile;
-  bool done;
-  __device__ StageCursor(const Params& p, int cta, int G) : q(0), u(cta), kb(0), k1(0), tile(0),
-                                                          done(false) {
-    seek(p, G);
-  }
-  // first stage of unit u of GEMM q, or of the next GEMM that has one
-  __device__ void seek(const Params& p, int G) {
-    while (q < 3 && u >= p.g[q].units) {
-      ++q;
-      u = u % G;  // this CTA's index
-    }
-    if (q >= 3) {
-      done = true;
-      return;
-    }
-    int k0;
-    unit_range(p.g[q], u, tile, k0, k1);
-    kb = k0;
-  }
-  __device__ void next(const Params& p, int cta, int G) {
-    if (++kb < k1) return;
-    u += G;
-    if (u >= p.g[q].units) {
-      ++q;
-      u = cta;
-    }
-    seek(p, G);
-  }
-};
 
 // The epilogue threads' arrival at a grid counter: every thread's stores are
 // made visible (also to TMA reads of other CTAs) before one thread adds.
@@ -220,191 +250,91 @@ __device__ __forceinline__ bool epi_wait_count(const int* cnt, int target, int e
   return ok;
 }
 
-// Two 32-column TMEM loads (this thread's lane), one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
-  __syncwarp();
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
-        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
-        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
-        "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr + 32));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+// Receive slot of sender s in owner o's buffer (0..2).
+__device__ __forceinline__ uint32_t recv_slot(uint32_t s, uint32_t o) {
+  return (s - o - 1u) & 3u;
 }
 
-// Accumulator (row = this thread's TMEM lane, 256 columns) -> the unit's fp32
-// partial slab [64 groups][128 rows][4]: for each group the warp's 32 lanes
-// store one contiguous 512-byte segment, straight from registers.
-__device__ void store_partial(const Params& p, float* slab, uint32_t taddr, int row) {
-  for (int c = 0; c < kTileN; c += 64) {
-    float v[64];
-    tmem_ld64(taddr + c, v);
-    if (row < p.M) {
+// Reduce-scatter of a split-K accumulator over the cluster (thread = row).
+// reduce_send writes the other ranks' 32-column slices of this thread's row
+// into their receive buffers and returns this rank's own slice in `own`; the
+// TMEM accumulator may be reused once it returns. `empty`: this rank had no
+// k-blocks (its partial is 0). A receive slot is laid out [8 chunks of 4
+// columns][128 rows][16 bytes], so the 32 lanes of a warp (32 consecutive
+// rows) write, and later read, one contiguous 512-byte block per chunk.
+__device__ __forceinline__ void reduce_send(uint32_t taddr, bool empty, int row, uint32_t rank,
+                                            uint8_t* recv, uint64_t* red_full, float (&own)[32]) {
+#pragma unroll 1
+  for (uint32_t o = 0; o < kCluster; ++o) {
+    if (o == rank) continue;
+    float v[32];
+    if (empty) {
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        st_cg4(slab + (static_cast<size_t>(c / 4 + q) * kBM + row) * 4,
-               make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    } else {
+      tmem_ld<32>(taddr + o * kSliceN, v);
     }
+    const uint32_t base =
+        map_rank(smem_u32(recv + recv_slot(rank, o) * kRecvSlotBytes + row * 16), o);
+    const uint32_t rbar = map_rank(smem_u32(red_full), o);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      st_async16(base + c * (kBM * 16), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], rbar);
+  }
+  if (empty) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) own[i] = 0.f;
+  } else {
+    tmem_ld<32>(taddr + rank * kSliceN, own);
   }
 }
 
-__device__ __forceinline__ void load_bf16x4_cg(const __nv_bfloat16* src, float (&v)[4]) {
-  uint32_t w0, w1;
-  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "l"(src));
-  v[0] = bf16_bits_to_float(static_cast<uint16_t>(w0 & 0xffffu));
-  v[1] = bf16_bits_to_float(static_cast<uint16_t>(w0 >> 16));
-  v[2] = bf16_bits_to_float(static_cast<uint16_t>(w1 & 0xffffu));
-  v[3] = bf16_bits_to_float(static_cast<uint16_t>(w1 >> 16));
-}
-
-__device__ __forceinline__ void bulk_g2s(uint32_t sdst, const void* gsrc, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          sdst),
-      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Streams the S split partials of each of this CTA's 4-column groups (gi =
-// cta, cta + G, ...) into shared memory by bulk TMA copies (one 2 KB copy
-// per (group, split): all 128 rows of those 4 columns), as many at once as
-// the idle weight ring holds (all of them at the layer's sizes: one round
-// trip), and hands every item to on_item(gi, s, bytes) in split order, then
-// on_group(gi) after its last split. Thread et == 0 issues the copies;
-// `batches` counts the batches of earlier calls (it sets the barrier phase).
-// Returns false if a wait gave up. The caller guarantees that no weight or
-// activation copy targets the ring meanwhile.
-template <class OnItem, class OnGroup>
-__device__ bool stream_partials(const Params& p, int S, int cta, int G, uint8_t* rbuf,
-                                uint64_t* rfull, int& batches, int et, OnItem on_item,
-                                OnGroup on_group) {
-  const int groups = p.d / 4;
-  const int mine = groups > cta ? (groups - cta + G - 1) / G : 0;
-  const int n = mine * S;
-  const int nb = (n + kRedItems - 1) / kRedItems;
-  bool ok = true;
-  for (int b = 0; b < nb; ++b) {
-    const int gb = batches + b;
-    const int k0 = b * kRedItems, k1 = min(n, k0 + kRedItems);
-    if (et == 0) {
-      if (b == 0) fence_proxy_async_global();  // partials stored by other CTAs -> bulk copies
-      mbar_arrive_expect_tx(rfull, static_cast<uint32_t>((k1 - k0) * kGroupBytes));
-      for (int k = k0; k < k1; ++k) {
-        const int gi = cta + (k / S) * G, sp = k % S;
-        const int tile = gi / (kTileN / 4), g = gi - tile * (kTileN / 4);
-        const float* src =
-            p.part + (static_cast<size_t>(tile * S + sp) * (kTileN / 4) + g) * (kBM * 4);
-        bulk_g2s(smem_u32(rbuf + (k - k0) * kGroupBytes), src, kGroupBytes, rfull);
+// reduce_gather waits (phase `parity`) for the other ranks' slices and sums
+// the four in rank order into `sum`; false (for every epilogue thread) if the
+// wait gave up.
+__device__ __forceinline__ bool reduce_gather(int row, uint32_t rank, const uint8_t* recv,
+                                              uint64_t* red_full, uint32_t parity,
+                                              const float (&own)[32], float (&sum)[32]) {
+  bool ok = mbar_wait(red_full, parity);
+  ok = epi_bar_and(ok);
+  if (!ok) return false;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) sum[i] = 0.f;
+#pragma unroll 1
+  for (uint32_t k = 0; k < kCluster; ++k) {
+    if (k == rank) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sum[i] += own[i];
+    } else {
+      const uint8_t* src = recv + recv_slot(k, rank) * kRecvSlotBytes + row * 16;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 v = *reinterpret_cast<const float4*>(src + c * (kBM * 16));
+        sum[4 * c] += v.x;
+        sum[4 * c + 1] += v.y;
+        sum[4 * c + 2] += v.z;
+        sum[4 * c + 3] += v.w;
       }
     }
-    if (!mbar_wait(rfull, static_cast<uint32_t>(gb & 1))) ok = false;
-    if (ok) {
-      for (int k = k0; k < k1; ++k) {
-        const int gi = cta + (k / S) * G, sp = k % S;
-        on_item(gi, sp, rbuf + (k - k0) * kGroupBytes);
-        if (sp == S - 1) on_group(gi);
-      }
-    }
-    epi_bar();  // every thread is done with the batch before the next one lands
   }
-  batches += nb;
-  return ok;
+  return true;
 }
 
-// R0 on this CTA's 4-column groups (thread = row): x_mid = bf16(x + sum of the
-// W_o partials in split order); this CTA's sum of squares of each row's
-// stored values goes to ss_part[cta][row].
-constexpr int kPreGroups = 8;  // residual values of up to this many groups held in registers
-
-__device__ bool reduce_o(const Params& p, int cta, int G, int et, uint8_t* rbuf, uint64_t* rfull,
-                         int& batches) {
-  const int row = et;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float ss = 0.f;
-  const bool live = row < p.M;
-  // The residual values of this thread's groups are loaded before the partials
-  // arrive, so no group waits for a load of its own.
-  const int groups = p.d / 4;
-  uint2 pre[kPreGroups];
+// Row scale of this thread's row: 1 / sqrt(sum over the d/32 slices of their
+// sums of squares (slice order) / d + eps).
+__device__ float row_scale(const Params& p, int row) {
+  const int slices = p.d / kSliceN;
+  float s = 0.f;
+  int k = 0;
+  for (; k + 16 <= slices; k += 16) {
+    float v[16];
 #pragma unroll
-  for (int i = 0; i < kPreGroups; ++i) {
-    const int gi = cta + i * G;
-    pre[i] = (live && gi < groups)
-                 ? *reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(row) * p.d + gi * 4)
-                 : make_uint2(0u, 0u);
+    for (int i = 0; i < 16; ++i) v[i] = __ldcg(p.ss_part + static_cast<size_t>(k + i) * kBM + row);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s += v[i];
   }
-  const bool ok = stream_partials(
-      p, p.g[0].splits, cta, G, rbuf, rfull, batches, et,
-      [&](int, int, const uint8_t* item) {
-        const float4 v = *reinterpret_cast<const float4*>(item + row * 16);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      },
-      [&](int gi) {
-        if (live) {
-          const int i = (gi - cta) / G;
-          float res[4];
-          if (i < kPreGroups) {
-            uint2 w = make_uint2(0u, 0u);
-#pragma unroll
-            for (int k = 0; k < kPreGroups; ++k)
-              if (k == i) w = pre[k];
-            res[0] = bf16_bits_to_float(static_cast<uint16_t>(w.x & 0xffffu));
-            res[1] = bf16_bits_to_float(static_cast<uint16_t>(w.x >> 16));
-            res[2] = bf16_bits_to_float(static_cast<uint16_t>(w.y & 0xffffu));
-            res[3] = bf16_bits_to_float(static_cast<uint16_t>(w.y >> 16));
-          } else {
-            load_bf16x4(p.x + static_cast<size_t>(row) * p.d + gi * 4, res);
-          }
-          float o[4] = {acc.x + res[0], acc.y + res[1], acc.z + res[2], acc.w + res[3]};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            o[i] = __bfloat162float(__float2bfloat16_rn(o[i]));
-            ss = fmaf(o[i], o[i], ss);
-          }
-          store_bf16x4(p.x_mid + static_cast<size_t>(row) * p.d + gi * 4, o);
-        }
-        acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      });
-  p.ss_part[static_cast<size_t>(cta) * kBM + row] = ss;
-  return ok;
-}
-
-// Row scale of row r: 1 / sqrt(sum over CTAs of ss_part[.][r] / d + eps),
-// summed in a fixed order (thread et adds CTAs et, et + 128, ...; then a
-// fixed tree over the 128 threads).
-__device__ void row_scale(const Params& p, int G, int r, int et, float* red) {
-  float v = 0.f;
-  for (int k = et; k < G; k += kEpiThreads) v += __ldcg(p.ss_part + static_cast<size_t>(k) * kBM + r);
-  red[et] = v;
-  epi_bar();
-  for (int w = kEpiThreads / 2; w > 0; w >>= 1) {
-    if (et < w) red[et] += red[et + w];
-    epi_bar();
-  }
-  if (et == 0) p.rscale[r] = 1.0f / sqrtf(red[0] / static_cast<float>(p.d) + p.eps);
-  epi_bar();
+  for (; k < slices; ++k) s += __ldcg(p.ss_part + static_cast<size_t>(k) * kBM + row);
+  return 1.0f / sqrtf(s / static_cast<float>(p.d) + p.eps);
 }
 
 // P1 epilogue of tile t: h[row][t*H + j] = SiLU(rs g) * (rs u) (+ b * primary
@@ -464,81 +394,6 @@ __device__ void load_b_slice(const Params& p, int t, int et, float* bsl) {
   epi_bar();
 }
 
-// R2 on this CTA's 4-column groups: thread et handles sequence j = et % 64
-// (rows j and mp + j), columns 2 (et / 64) .. + 1 of each group: x_out =
-// x_mid + the sum of the W_down partials in split order, the auxiliary row
-// adding c * (primary row's sum) first.
-__device__ bool reduce_down(const Params& p, int cta, int G, int et, uint8_t* rbuf,
-                            uint64_t* rfull, int& batches) {
-  const int j = et & 63, hc = (et >> 6) * 2;
-  const bool live = j < p.mp;
-  float2 ap = make_float2(0.f, 0.f), aa = make_float2(0.f, 0.f);
-  // residual (x_mid, written by other CTAs: read through L2) and coupling
-  // values of this thread's groups, loaded before the partials arrive
-  const int groups = p.d / 4;
-  uint32_t pre_p[kPreGroups], pre_a[kPreGroups], pre_c[kPreGroups];
-#pragma unroll
-  for (int i = 0; i < kPreGroups; ++i) {
-    const int gi = cta + i * G;
-    const bool in = live && gi < groups;
-    const int col = gi * 4 + hc;
-    pre_p[i] = in ? __ldcg(reinterpret_cast<const unsigned int*>(
-                        p.x_mid + static_cast<size_t>(j) * p.d + col))
-                  : 0u;
-    pre_a[i] = in ? __ldcg(reinterpret_cast<const unsigned int*>(
-                        p.x_mid + static_cast<size_t>(p.mp + j) * p.d + col))
-                  : 0u;
-    pre_c[i] = (in && p.c != nullptr) ? *reinterpret_cast<const uint32_t*>(p.c + col) : 0u;
-  }
-  return stream_partials(
-      p, p.g[2].splits, cta, G, rbuf, rfull, batches, et,
-      [&](int, int, const uint8_t* item) {
-        if (!live) return;
-        const float2 vp = *reinterpret_cast<const float2*>(item + j * 16 + hc * 4);
-        const float2 va = *reinterpret_cast<const float2*>(item + (p.mp + j) * 16 + hc * 4);
-        ap.x += vp.x;
-        ap.y += vp.y;
-        aa.x += va.x;
-        aa.y += va.y;
-      },
-      [&](int gi) {
-        if (live) {
-          const int col = gi * 4 + hc;
-          const int i = (gi - cta) / G;
-          uint32_t wp = 0u, wa = 0u, wc = 0u;
-          if (i < kPreGroups) {
-#pragma unroll
-            for (int k = 0; k < kPreGroups; ++k)
-              if (k == i) {
-                wp = pre_p[k];
-                wa = pre_a[k];
-                wc = pre_c[k];
-              }
-          } else {
-            wp = __ldcg(reinterpret_cast<const unsigned int*>(p.x_mid + static_cast<size_t>(j) * p.d + col));
-            wa = __ldcg(reinterpret_cast<const unsigned int*>(
-                p.x_mid + static_cast<size_t>(p.mp + j) * p.d + col));
-            if (p.c != nullptr) wc = *reinterpret_cast<const uint32_t*>(p.c + col);
-          }
-          float op[2] = {ap.x, ap.y}, oa[2] = {aa.x, aa.y};
-          if (p.c != nullptr) {
-            oa[0] = fmaf(bf16_bits_to_float(static_cast<uint16_t>(wc & 0xffffu)), op[0], oa[0]);
-            oa[1] = fmaf(bf16_bits_to_float(static_cast<uint16_t>(wc >> 16)), op[1], oa[1]);
-          }
-          op[0] += bf16_bits_to_float(static_cast<uint16_t>(wp & 0xffffu));
-          op[1] += bf16_bits_to_float(static_cast<uint16_t>(wp >> 16));
-          oa[0] += bf16_bits_to_float(static_cast<uint16_t>(wa & 0xffffu));
-          oa[1] += bf16_bits_to_float(static_cast<uint16_t>(wa >> 16));
-          *reinterpret_cast<__nv_bfloat162*>(p.x_out + static_cast<size_t>(j) * p.d + col) =
-              __floats2bfloat162_rn(op[0], op[1]);
-          *reinterpret_cast<__nv_bfloat162*>(p.x_out + static_cast<size_t>(p.mp + j) * p.d + col) =
-              __floats2bfloat162_rn(oa[0], oa[1]);
-        }
-        ap = make_float2(0.f, 0.f);
-        aa = make_float2(0.f, 0.f);
-      });
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     post_kernel(const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
                 const __grid_constant__ CUtensorMap tmXg, const __grid_constant__ CUtensorMap tmWg,
@@ -547,24 +402,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* rbuf = smem;  // the weight ring, while a reduction has it
-  float* xchg = reinterpret_cast<float*>(smem + static_cast<size_t>(kStages) * kSlot);
-  float* red = xchg + kXchgFloats;                                // [kEpiThreads]
-  float* bsl = red + kEpiThreads;                                 // [kMaxHalf] b of a tile
-  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);   // [kStages]
-  uint64_t* empty = full + kStages;                               // [kStages]
-  uint64_t* acc_full = empty + kStages;                           // [2]
-  uint64_t* acc_empty = acc_full + 2;                             // [2]
-  uint64_t* mma_done = acc_empty + 2;                             // [1]
-  uint64_t* rfull = mma_done + 1;     // reduction batch landed
-  uint64_t* ring_free = rfull + 1;    // R0 is done with the ring: gate/up weights may load
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_free + 1);
+  uint8_t* recv = smem + static_cast<size_t>(kStages) * kSlot;   // [3][128 rows][32] fp32
+  float* xchg = reinterpret_cast<float*>(recv);                  // aliases recv (never both)
+  float* bsl = reinterpret_cast<float*>(recv + kRecvBytes);      // [kMaxHalf] b of a tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);  // [kStages]
+  uint64_t* empty = full + kStages;                              // [kStages]
+  uint64_t* acc_full = empty + kStages;                          // [2]
+  uint64_t* acc_empty = acc_full + 2;                            // [2]
+  uint64_t* mma_done = acc_empty + 2;                            // [1]
+  uint64_t* red_full = mma_done + 1;  // this rank's slices from the other 3 ranks have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
   // [0] abort, [1] epilogue broadcast, [2] / [3] stages issued by the weight /
   // activation producer
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
+  const uint32_t rank = cluster_rank();
+  const int cid = static_cast<int>(cluster_index());
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -576,8 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], kEpiThreads / 32);
     }
     mbar_init(mma_done, 1);
-    mbar_init(rfull, 1);
-    mbar_init(ring_free, 1);
+    mbar_init(red_full, 1);  // this rank's expect_tx arrival + the senders' bytes
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
@@ -592,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();
+  // every CTA of the cluster has initialised its barriers before any remote write
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Only the weight producer may run ahead of the kernel launched before this
@@ -606,26 +461,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmWg);
       prefetch_tensormap(&tmWd);
       const uint64_t pol = l2_policy_evict_first();
-      // At a phase boundary the MMAs wait for the next phase's activations:
-      // the next phase's first weight tiles are prefetched into L2 there, so
-      // DRAM keeps streaming and those stages later load from L2. Before the
-      // first gate/up stage the ring is lent to the W_o reduction (R0): its
-      // loads wait until R0 has released it.
-      auto prefetch_phase = [&](int q, int count) {
-        StageCursor pf(p, cta, G);
-        while (!pf.done && pf.q < q) pf.next(p, cta, G);
-        for (int i = 0; i < count && !pf.done && pf.q == q; ++i) {
-          const Gemm& gq = p.g[q];
-          const CUtensorMap* tq = q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd);
-          if (q == 1) {
-            tma_prefetch_2d(tq, pf.kb * kBK, pf.tile * gq.half);
-            tma_prefetch_2d(tq, pf.kb * kBK, p.F + pf.tile * gq.half);
-          } else {
-            tma_prefetch_2d(tq, pf.kb * kBK, pf.tile * kTileN);
-          }
-          pf.next(p, cta, G);
-        }
-      };
       int s = 0;
       uint32_t ph = 0;
       long long n = 0;
@@ -633,16 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
         const CUtensorMap* tm = q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd);
-        if (q >= 1) prefetch_phase(q, kBoundaryPrefetch);
-        if (q == 1 && !mbar_wait(ring_free, 0)) {
-          set_err(p.err, DF_DEVERR_TIMEOUT);
-          flags[0] = 1;
-          ok = false;
-          break;
-        }
-        for (int u = cta; u < g.units && ok; u += G) {
-          int tile, k0, k1;
-          unit_range(g, u, tile, k0, k1);
+        const Units us = units_of(g, q, cta, cid, G);
+        for (int u = us.first; u < g.units && ok; u += us.step) {
+          int k0, k1;
+          k_range(g, q, static_cast<int>(rank), k0, k1);
           for (int kb = k0; kb < k1; ++kb, ++n) {
             if (n >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
@@ -657,11 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* wdst = smem + static_cast<size_t>(s) * kSlot + kXBytes;
             mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(g.w_bytes));
             if (q == 1) {
-              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, tile * g.half, pol);
-              tma_load_2d_hint(wdst + g.half * 128, tm, &full[s], kb * kBK,
-                               p.F + tile * g.half, pol);
+              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, u * g.half, pol);
+              tma_load_2d_hint(wdst + g.half * 128, tm, &full[s], kb * kBK, p.F + u * g.half,
+                               pol);
             } else {
-              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, tile * kTileN, pol);
+              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, u * kTileN, pol);
             }
             if (++s == kStages) {
               s = 0;
@@ -688,10 +517,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Gemm& g = p.g[q];
         const CUtensorMap* tm = q == 0 ? &tmXo : (q == 1 ? &tmXg : &tmXd);
         bool ready = q == 0;  // P0 reads the attention output: pdl_wait above
-        for (int u = cta; u < g.units && ok; u += G) {
-          int tile, k0, k1;
-          unit_range(g, u, tile, k0, k1);
-          if (!ready) {
+        const Units us = units_of(g, q, cta, cid, G);
+        for (int u = us.first; u < g.units && ok; u += us.step) {
+          int k0, k1;
+          k_range(g, q, static_cast<int>(rank), k0, k1);
+          if (!ready && k1 > k0) {
             // P1 reads x_mid (counter A2), P2 every column of h (C)
             if (!wait_count(p.cnt + (q == 1 ? kCntA2 : kCntC), G)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
@@ -734,9 +564,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
-        for (int u = cta; u < g.units && ok; u += G, ++seg) {
-          int tile, k0, k1;
-          unit_range(g, u, tile, k0, k1);
+        const Units us = units_of(g, q, cta, cid, G);
+        for (int u = us.first; u < g.units && ok; u += us.step, ++seg) {
+          int k0, k1;
+          k_range(g, q, static_cast<int>(rank), k0, k1);
           const int acc = seg & 1;
           if (seg >= 2 &&
               !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
@@ -768,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
+          // (a unit without k-blocks commits at once: its partial is zero)
           umma_commit(&acc_full[acc]);
         }
       }
@@ -781,16 +613,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int et = threadIdx.x - 3 * 32;
     const int row = quarter * 32 + lane;  // this thread's TMEM lane = accumulator row
+    const bool live = row < p.M;
     volatile int* eflag = flags + 1;
     int seg = 0;
     bool ok = true;
+    // (uniform over the epilogue threads, like every other epilogue wait, so
+    // that all of them pass the same named barriers on every path)
     auto take_acc = [&](int acc, int sg) -> bool {
       const bool got = mbar_wait_warp(&acc_full[acc], static_cast<uint32_t>((sg >> 1) & 1));
-      if (!got && lane == 0) {
-        set_err(p.err, DF_DEVERR_TIMEOUT);
-        flags[0] = 1;
-      }
-      return got;
+      return epi_bar_and(got);
     };
     auto give_acc = [&](int acc) {
       tc_fence_before();
@@ -807,70 +638,128 @@ __global__ void __launch_bounds__(kThreads, 1)
       return tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
              static_cast<uint32_t>(acc * 256);
     };
-    // P0: W_o partials
-    for (int u = cta; u < p.g[0].units && ok; u += G, ++seg) {
-      const int acc = seg & 1;
-      if (!take_acc(acc, seg)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, acc_addr(acc), row);
-      give_acc(acc);
-    }
-    arrive_count(p.cnt + kCntA, et);
-    // R0: x_mid and this CTA's row sums of squares
-    // (the ring is idle: every W_o stage has been consumed, and the producers
-    // hold back the gate/up stages until ring_free)
-    int rbatches = 0;
-    if (grid_wait(kCntA) && !flags[0] && !reduce_o(p, cta, G, et, rbuf, rfull, rbatches)) {
+    auto fail = [&]() {
       if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
       flags[0] = 1;
+      ok = false;
+    };
+    // P0: W_o tile `cid` over this rank's K quarter; reduce-scatter; x_mid
+    if (cid < p.g[0].units) {
+      const int acc = seg & 1;
+      int k0, k1;
+      k_range(p.g[0], 0, static_cast<int>(rank), k0, k1);
+      const int col0 = cid * kTileN + static_cast<int>(rank) * kSliceN;
+      float res[32];  // residual, loaded while the MMAs run
+      if (live) {
+        load_bf16<32>(p.x + static_cast<size_t>(row) * p.d + col0, res);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) res[i] = 0.f;
+      }
+      if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
+      if (!take_acc(acc, seg)) {
+        fail();
+      } else {
+        tc_fence_after();
+        float own[32], sum[32];
+        reduce_send(acc_addr(acc), k1 == k0, row, rank, recv, red_full, own);
+        give_acc(acc);
+        if (!reduce_gather(row, rank, recv, red_full, 0, own, sum)) {
+          fail();
+        } else {
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            sum[i] = __bfloat162float(__float2bfloat16_rn(sum[i] + res[i]));
+            ss = fmaf(sum[i], sum[i], ss);
+          }
+          if (live) store_bf16<32>(p.x_mid + static_cast<size_t>(row) * p.d + col0, sum);
+          p.ss_part[static_cast<size_t>(cid * kCluster + rank) * kBM + row] = live ? ss : 0.f;
+        }
+      }
+      ++seg;
     }
-    if (et == 0) mbar_arrive(ring_free);
+    ok = epi_bar_and(ok);
     arrive_count(p.cnt + kCntA2, et);
-    // row scales of the norm (CTA r < M computes row r)
-    if (cta < p.M && grid_wait(kCntA2) && !flags[0]) row_scale(p, G, cta, et, red);
-    arrive_count(p.cnt + kCntI, et);
     // P1: SwiGLU tiles straight from TMEM
     float rs = 0.f;
     bool have_rs = false;
     for (int u = cta; u < p.g[1].units && ok; u += G, ++seg) {
       const int acc = seg & 1;
+      if (p.b != nullptr) load_b_slice(p, u, et, bsl);
       if (!have_rs) {
-        if (!grid_wait(kCntI)) {
+        if (!grid_wait(kCntA2)) {
           ok = false;
           break;
         }
-        rs = row < p.M ? __ldcg(p.rscale + row) : 0.f;
+        rs = live ? row_scale(p, row) : 0.f;
         have_rs = true;
       }
-      if (p.b != nullptr) load_b_slice(p, u, et, bsl);
       if (!take_acc(acc, seg)) {
-        ok = false;
+        fail();
         break;
       }
       tc_fence_after();
       swiglu_epilogue(p, u, acc_addr(acc), row, rs, xchg, bsl);
       give_acc(acc);
     }
+    ok = epi_bar_and(ok);
     arrive_count(p.cnt + kCntC, et);
-    // P2: W_down partials
-    for (int u = cta; u < p.g[2].units && ok; u += G, ++seg) {
+    // P2: W_down tile `cid` over this rank's K quarter; reduce-scatter; x_out.
+    // The other ranks' receive buffers hold their gate/up coupling exchange
+    // until every CTA is past P1 (counter C); a rank without k-blocks would
+    // otherwise send before that.
+    if (ok && cid < p.g[2].units && grid_wait(kCntC)) {
       const int acc = seg & 1;
+      int k0, k1;
+      k_range(p.g[2], 2, static_cast<int>(rank), k0, k1);
+      const int col0 = cid * kTileN + static_cast<int>(rank) * kSliceN;
+      if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
       if (!take_acc(acc, seg)) {
-        ok = false;
-        break;
+        fail();
+      } else {
+        tc_fence_after();
+        float own[32], sum[32];
+        reduce_send(acc_addr(acc), k1 == k0, row, rank, recv, red_full, own);
+        give_acc(acc);
+        // residual (x_mid, written by other CTAs) and coupling, while the
+        // other ranks' slices arrive
+        float res[32], cc[32];
+        if (live) {
+          load_bf16x32_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) res[i] = 0.f;
+        }
+        const bool aux = row >= p.mp && live;
+        if (aux && p.c != nullptr) {
+          load_bf16<32>(p.c + col0, cc);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cc[i] = 0.f;
+        }
+        if (!reduce_gather(row, rank, recv, red_full, 1, own, sum)) {
+          fail();
+        } else {
+          if (p.c != nullptr) {
+            epi_bar();  // every thread is done with the receive buffer (xchg aliases it)
+            if (row < p.mp) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) xchg[row * kXchgPitch + i] = sum[i];
+            }
+            epi_bar();
+            if (aux) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                sum[i] = fmaf(cc[i], xchg[(row - p.mp) * kXchgPitch + i], sum[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sum[i] += res[i];
+          if (live) store_bf16<32>(p.x_out + static_cast<size_t>(row) * p.d + col0, sum);
+        }
       }
-      tc_fence_after();
-      store_partial(p, p.part + static_cast<size_t>(u) * kBM * kTileN, acc_addr(acc), row);
-      give_acc(acc);
-    }
-    arrive_count(p.cnt + kCntD, et);
-    // R2: x_out (the ring is idle again: every W_down stage has been consumed)
-    if (grid_wait(kCntD) && !flags[0] && !reduce_down(p, cta, G, et, rbuf, rfull, rbatches)) {
-      if (et == 0) set_err(p.err, DF_DEVERR_TIMEOUT);
-      flags[0] = 1;
+      ++seg;
     }
   }
 
@@ -898,6 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
     }
   }
+  // no CTA leaves while another rank may still write into its shared memory
+  cluster_sync();
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "n"(512)
                  : "memory");
@@ -906,30 +797,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ planning
 
+std::mutex g_mu;
+bool g_attr[64] = {};
+int g_clusters[64] = {};  // co-resident 4-CTA clusters per device (0: not queried)
+
+// Sets the kernel's shared-memory attribute on the current device and returns
+// how many 4-CTA clusters of it fit on the device at once (0 on error).
+int max_clusters() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_attr[dev]) {
+    if (cudaFuncSetAttribute(post_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return 0;
+    g_attr[dev] = true;
+  }
+  if (g_clusters[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kCluster * 64);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, post_kernel, &cfg) != cudaSuccess || n < 1) return 0;
+    g_clusters[dev] = n;
+  }
+  return g_clusters[dev];
+}
+
 struct Plan {
   bool ok;
-  int G, S0, T0, S2, T2, H1, T1;
+  int G, T0, H1, T1;
 };
 
 Plan make_plan(int M, int mp, int d, int qd, int F) {
   Plan pl{};
   pl.ok = false;
-  const int G = device_sm_count();
   if (M != 2 * mp || mp < 1 || mp > 64 || d % kTileN != 0 || qd % kBK != 0 || F % kBK != 0 ||
-      d < kTileN)
+      d < kTileN || qd < kBK || F < kBK)
     return pl;
-  pl.G = G;
+  const int nc = max_clusters();
   pl.T0 = d / kTileN;
-  const int kb0 = qd / kBK, kb2 = F / kBK;
-  pl.S0 = G / pl.T0;
-  if (pl.S0 < 1) pl.S0 = 1;
-  if (pl.S0 > kb0) pl.S0 = kb0;
-  pl.T2 = pl.T0;
-  pl.S2 = G / pl.T2;
-  if (pl.S2 < 1) pl.S2 = 1;
-  if (pl.S2 > kb2) pl.S2 = kb2;
+  if (nc < 1 || pl.T0 > nc) return pl;  // one W_o / W_down tile per cluster
+  pl.G = nc * kCluster;
   // smallest multiple of 8 with at most G SwiGLU tiles
-  int H = static_cast<int>(ceil_div(F, G));
+  int H = static_cast<int>(ceil_div(F, pl.G));
   H = static_cast<int>(ceil_div(H, 8)) * 8;
   if (H < 8) H = 8;
   if (H > kMaxHalf) return pl;
@@ -939,23 +858,10 @@ Plan make_plan(int M, int mp, int d, int qd, int F) {
   return pl;
 }
 
-// Workspace: counters | ss_part [G][128] | rscale [128] | partials.
-struct WsLayout {
-  size_t ss, rscale, part, total;
-};
-
-WsLayout ws_layout(const Plan& pl) {
-  const int units = pl.T0 * pl.S0 > pl.T2 * pl.S2 ? pl.T0 * pl.S0 : pl.T2 * pl.S2;
-  WsLayout l;
-  l.ss = kCounterBytes;
-  l.rscale = l.ss + round_up(static_cast<size_t>(pl.G) * kBM * 4, 256);
-  l.part = l.rscale + round_up(kBM * 4, 256);
-  l.total = l.part + static_cast<size_t>(units) * kBM * kTileN * 4;
-  return l;
+// Workspace: counters | ss_part [d / 32][128].
+size_t ws_bytes(int d) {
+  return kCounterBytes + static_cast<size_t>(d / kSliceN) * kBM * 4;
 }
-
-std::mutex g_mu;
-bool g_attr[64] = {};
 
 }  // namespace post
 }  // namespace df
@@ -963,7 +869,7 @@ bool g_attr[64] = {};
 extern "C" size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model,
                                                                int q_dim, int F) {
   const df::post::Plan pl = df::post::make_plan(2 * m_primary, m_primary, d_model, q_dim, F);
-  return pl.ok ? df::post::ws_layout(pl).total : 0;
+  return pl.ok ? df::post::ws_bytes(d_model) : 0;
 }
 
 extern "C" df_status dualflow_layer_post_attention(
@@ -983,8 +889,7 @@ extern "C" df_status dualflow_layer_post_attention(
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DF_ERR_ALIGN;
   if ((b && !aligned(b, 16)) || (c && !aligned(c, 16))) return DF_ERR_ALIGN;
-  const WsLayout wl = ws_layout(pl);
-  if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 256))
+  if (!workspace || workspace_bytes < ws_bytes(d_model) || !aligned(workspace, 256))
     return DF_ERR_WORKSPACE;
 
   Params p{};
@@ -994,12 +899,10 @@ extern "C" df_status dualflow_layer_post_attention(
   p.qd = q_dim;
   p.F = F;
   p.eps = eps;
-  p.g[0] = Gemm{pl.T0 * pl.S0, pl.S0, q_dim / kBK, kTileN, 0, kTileN * kBK * 2,
-                make_idesc(kBM, kTileN)};
-  p.g[1] = Gemm{pl.T1, 1, d_model / kBK, 2 * pl.H1, pl.H1, 2 * pl.H1 * kBK * 2,
+  p.g[0] = Gemm{pl.T0, q_dim / kBK, kTileN, 0, kTileN * kBK * 2, make_idesc(kBM, kTileN)};
+  p.g[1] = Gemm{pl.T1, d_model / kBK, 2 * pl.H1, pl.H1, 2 * pl.H1 * kBK * 2,
                 make_idesc(kBM, 2 * pl.H1)};
-  p.g[2] = Gemm{pl.T2 * pl.S2, pl.S2, F / kBK, kTileN, 0, kTileN * kBK * 2,
-                make_idesc(kBM, kTileN)};
+  p.g[2] = Gemm{pl.T0, F / kBK, kTileN, 0, kTileN * kBK * 2, make_idesc(kBM, kTileN)};
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.b = static_cast<const __nv_bfloat16*>(b);
   p.c = static_cast<const __nv_bfloat16*>(c);
@@ -1008,9 +911,7 @@ extern "C" df_status dualflow_layer_post_attention(
   p.x_out = static_cast<__nv_bfloat16*>(x_out);
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
   p.cnt = reinterpret_cast<int*>(w8);
-  p.ss_part = reinterpret_cast<float*>(w8 + wl.ss);
-  p.rscale = reinterpret_cast<float*>(w8 + wl.rscale);
-  p.part = reinterpret_cast<float*>(w8 + wl.part);
+  p.ss_part = reinterpret_cast<float*>(w8 + kCounterBytes);
   p.err = err_flag;
 
   CUtensorMap tmXo, tmWo, tmXg, tmWg, tmXd, tmWd;
@@ -1024,27 +925,20 @@ extern "C" df_status dualflow_layer_post_attention(
       !encode_tmap_bf16_2d(&tmWd, w_down, du, Fu, Fu * 2, kTileN, kBK))
     return DF_ERR_CUDA;
 
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF_ERR_CUDA;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_attr[dev]) {
-      if (cudaFuncSetAttribute(post_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemBytes)) != cudaSuccess)
-        return DF_ERR_CUDA;
-      g_attr[dev] = true;
-    }
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.G);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, post_kernel, tmXo, tmWo, tmXg, tmWg, tmXd, tmWd, p) != cudaSuccess)
     return DF_ERR_CUDA;
   return DF_OK;

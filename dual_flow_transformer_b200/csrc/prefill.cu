@@ -831,7 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr int kPairThreads = 320;
 constexpr uint32_t kPairTmemCols = 512;
+constexpr int kPairStages = 4;  // K/V page ring depth
 
+// One P buffer per tile: a tile's softmax writes P_i only after its own
+// O += P_{i-1} V_{i-1} has completed, which by then it long has (that MMA is
+// issued as soon as P_{i-1} is published, and P_i takes a whole softmax to
+// compute); the 32 KB this saves buys the fourth K/V stage.
 template <int D>
 struct PairLayout {
   static constexpr int kQBytes = kRows * D * 2;      // one tile's Q
@@ -839,9 +844,9 @@ struct PairLayout {
   static constexpr int kStageBytes = 2 * kPageBytes;
   static constexpr int kPBytes = kRows * kPage * 2;  // P of one page of one tile
   static constexpr int kOffStages = 2 * kQBytes;
-  static constexpr int kOffP = kOffStages + kStages * kStageBytes;  // [tile][buffer]
-  static constexpr int kOffBar = kOffP + 4 * kPBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 * 2 + 1;
+  static constexpr int kOffP = kOffStages + kPairStages * kStageBytes;  // [tile]
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kNumBars = 1 + 2 * kPairStages + 2 * 4 * 2 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
 };
 
@@ -861,8 +866,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* full = bars + 1;
-  uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;  // [tile][2] S_i landed in TMEM buffer i & 1
+  uint64_t* empty = full + kPairStages;
+  uint64_t* s_full = empty + kPairStages;  // [tile][2] S_i landed in TMEM buffer i & 1
   uint64_t* s_free = s_full + 4;       // [tile][2] that tile's softmax warps have read it
   uint64_t* p_full = s_free + 4;       // [tile][2] P_i written to P buffer i & 1
   uint64_t* pv_done = p_full + 4;      // [tile][2] O += P_i V_i completed
@@ -890,7 +895,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kPairStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -931,8 +936,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
       int issued = 0;
       for (int i = 0; i < npages; ++i) {
-        const int st = i % kStages;
-        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
+        const int st = i % kPairStages;
+        if (i >= kPairStages && !mbar_wait(&empty[st], ((i / kPairStages) - 1) & 1)) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
           break;
         }
@@ -954,8 +959,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       // Leave no copy in flight (bounded waits).
       mbar_wait(q_full, 0);
-      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
-        mbar_wait(&full[i % kStages], (i / kStages) & 1);
+      for (int i = issued > kPairStages ? issued - kPairStages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kPairStages], (i / kPairStages) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -973,8 +978,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t dp0 = umma::smem_desc(smem_u32(smem + Lay::kOffP));
       // S_i of tile t into its TMEM buffer i & 1
       auto issue_s = [&](int t, int i) -> bool {
-        const int st = i % kStages, sb = i & 1;
-        if (!mbar_wait(&full[st], (i / kStages) & 1)) return false;
+        const int st = i % kPairStages, sb = i & 1;
+        if (!mbar_wait(&full[st], (i / kPairStages) & 1)) return false;
         if (i >= 2 && !mbar_wait(&s_free[2 * t + sb], ((i >> 1) - 1) & 1)) return false;
         umma::tc_fence_after();
         const uint64_t dq = dq0 + static_cast<uint64_t>((t * Lay::kQBytes) >> 4);
@@ -991,10 +996,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       };
       // O_t += P_i V_i once tile t's softmax has written P_i
       auto issue_pv = [&](int t, int i) -> bool {
-        const int pb = i & 1, st = i % kStages;
+        const int pb = i & 1, st = i % kPairStages;
         if (!mbar_wait(&p_full[2 * t + pb], (i >> 1) & 1)) return false;
         umma::tc_fence_after();
-        const uint64_t dp = dp0 + static_cast<uint64_t>(((2 * t + pb) * Lay::kPBytes) >> 4);
+        const uint64_t dp = dp0 + static_cast<uint64_t>((t * Lay::kPBytes) >> 4);
         const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kStageBytes) >> 4);
         const uint32_t d_tmem = tmem + t * 256 + kOCol;
 #pragma unroll
@@ -1015,7 +1020,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (ok && !issue_pv(0, i)) ok = false;
         if (ok && more && !issue_s(1, i + 1)) ok = false;
         if (ok && !issue_pv(1, i)) ok = false;
-        if (ok) umma::umma_commit(&empty[i % kStages]);  // page i read by both tiles
+        if (ok) umma::umma_commit(&empty[i % kPairStages]);  // page i read by both tiles
       }
       if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
       umma::umma_commit(mma_done);  // completes when every MMA issued above has
@@ -1028,7 +1033,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int r = quarter * 32 + lane;
     const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
-    uint8_t* p_base = smem + Lay::kOffP + 2 * t * Lay::kPBytes + r * 128;
+    uint8_t* prow = smem + Lay::kOffP + t * Lay::kPBytes + r * 128;
     uint64_t* my_s_full = s_full + 2 * t;
     uint64_t* my_s_free = s_free + 2 * t;
     uint64_t* my_p_full = p_full + 2 * t;
@@ -1036,7 +1041,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     float m_ref = kNegInf, l = 0.f;
     bool ok = true;
     for (int i = 0; i < npages; ++i) {
-      const int sb = i & 1, st = i % kStages, kbase = i * kPage;
+      const int sb = i & 1, st = i % kPairStages, kbase = i * kPage;
       if (!mbar_wait_warp(&my_s_full[sb], (i >> 1) & 1)) {
         ok = false;
         break;
@@ -1081,12 +1086,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
 
-      // P buffer sb of this tile is free once O += P_{i-2} V_{i-2} has completed.
-      if (i >= 2 && !mbar_wait_warp(&my_pv_done[sb], ((i >> 1) - 1) & 1)) {
+      // This tile's P buffer is free once O += P_{i-1} V_{i-1} has completed.
+      if (i >= 1 && !mbar_wait_warp(&my_pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
         ok = false;
         break;
       }
-      uint8_t* prow = p_base + sb * Lay::kPBytes;
       l += write_p32(prow, r, 0, s0, p.scale_log2, mu);
       l += write_p32(prow, r, 4, s1, p.scale_log2, mu);
 
@@ -1096,7 +1100,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // warps clear the same rows (the same zero bytes), each before its own
       // P is published, so neither tile's P V can read the old bytes.
       if (kbase + kPage > kend) {
-        if (!mbar_wait_warp(&full[st], (i / kStages) & 1)) {  // the page has landed
+        if (!mbar_wait_warp(&full[st], (i / kPairStages) & 1)) {  // the page has landed
           ok = false;
           break;
         }

@@ -373,14 +373,18 @@ int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue
 /*   x_out = x_mid + h W_down^T; aux rows += c (.) (h W_down^T) of primary   */
 /* which is dualflow_grouped_proj (residual) -> dualflow_rmsnorm ->          */
 /* dualflow_grouped_proj (swiglu, b) -> dualflow_grouped_proj (residual, c)  */
-/* computed by one grid of one CTA per SM whose TMA producers stream the     */
-/* three weights back to back; the dependencies between the steps are       */
-/* grid-wide counters in the workspace (bounded waits). The norm's row scale */
-/* multiplies the gate/up accumulators (the normalised rows are not rounded  */
-/* to bf16 and stored). Each split-k sum is taken in a fixed order, so the   */
-/* results are deterministic and primary rows never depend on auxiliary      */
-/* rows. They match the four-call form within the bf16 tolerance, not bit    */
-/* for bit (other split-k orders, no bf16 rounding of the normalised rows).  */
+/* computed by one grid of one CTA per SM, launched as clusters of 4 CTAs,   */
+/* whose TMA producers stream the three weights back to back. W_o and W_down */
+/* are split 4 ways along K over the CTAs of a cluster and their split sums  */
+/* are reduced inside the cluster through distributed shared memory; the    */
+/* steps that need every column of the step before (x_mid for gate/up, h for */
+/* W_down) wait on grid-wide counters in the workspace (bounded waits). The  */
+/* norm's row scale multiplies the gate/up accumulators (the normalised rows */
+/* are not rounded to bf16 and stored). Each split-k sum is taken in a fixed */
+/* order, so the results are deterministic and primary rows never depend on  */
+/* auxiliary rows. They match the four-call form within the bf16 tolerance,  */
+/* not bit for bit (other split-k orders, no bf16 rounding of the normalised */
+/* rows).                                                                    */
 /*                                                                           */
 /* attn  : bf16 [M][q_dim] (the attention output, O1 rows then O2 rows).      */
 /* x     : bf16 [M][d_model] (the layer input, residual of W_o).             */
@@ -390,14 +394,17 @@ int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue
 /* packed, 16-byte aligned). w_* are read before the wait for the kernel     */
 /* launched ahead on the stream (programmatic dependent launch), so that     */
 /* kernel must not write them.                                               */
-/* workspace: >= dualflow_layer_post_attention_workspace_size(...) bytes,     */
-/* 256-byte aligned, ZERO-FILLED once: its first bytes are grid counters     */
-/* that every completed call leaves at zero (after a DF_DEVERR_TIMEOUT,      */
-/* zero it again); the rest holds fp32 split-k partials and the row sums of  */
-/* the norm. Calls sharing one workspace must not overlap on the GPU.        */
+/* workspace: >= dualflow_layer_post_attention_workspace_size(...) bytes     */
+/* (256 + d_model * 16), 256-byte aligned, ZERO-FILLED once: its first bytes */
+/* are grid counters that every completed call leaves at zero (after a       */
+/* DF_DEVERR_TIMEOUT, zero it again); the rest holds the row sums of squares */
+/* of the norm. Calls sharing one workspace must not overlap on the GPU.     */
 /* Supported (else DF_ERR_UNSUPPORTED; the size query returns 0):            */
-/* 1 <= m_primary <= 64, d_model % 256 == 0, q_dim % 64 == 0, F % 64 == 0,   */
-/* F <= 128 * (SM count). One kernel launch.                                  */
+/* 1 <= m_primary <= 64, d_model % 128 == 0 with d_model / 128 at most the   */
+/* number of 4-CTA clusters the device holds at once (33 on a 148-SM B200:   */
+/* d_model <= 4224), q_dim % 64 == 0, F % 64 == 0, F <= 112 * 4 * (that     */
+/* cluster count). Needs a current CUDA device (the size query too). One    */
+/* kernel launch.                                                            */
 /* ------------------------------------------------------------------------ */
 size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model, int q_dim,
                                                     int F);

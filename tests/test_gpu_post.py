@@ -166,6 +166,10 @@ def test_post_attention_rejects_unsupported_sizes(cuda_device):
     d = _dev(_inputs(s), cuda_device)
     assert api.layer_post_attention_workspace_size(65, 512, 512, 1024) == 0
     assert api.layer_post_attention_workspace_size(8, 320, 512, 1024) == 0
+    # one 128-column W_o / W_down tile per 4-CTA cluster: d_model 8192 needs 64
+    assert api.layer_post_attention_workspace_size(8, 8192, 512, 1024) == 0
+    # counters + one fp32 sum of squares per (32-column slice, row)
+    assert api.layer_post_attention_workspace_size(8, 512, 512, 1024) == 256 + 512 * 16
     ws = torch.zeros(256, dtype=torch.uint8, device=cuda_device)
     with pytest.raises(L.DualflowError) as e:
         _post(d, workspace=ws)
