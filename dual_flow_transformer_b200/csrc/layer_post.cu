@@ -50,6 +50,12 @@
 // tcgen05.mma M = 128 into two 256-column TMEM accumulators), warp 2
 // activation producer, warps 3-6 epilogue (TMEM lane quarter = warp % 4,
 // thread = accumulator row).
+// One 176 KB ring holds a k-block's activation tile and weight tile per
+// stage; its stage size follows the phase (5 stages of 32 KB for W_o and
+// W_down, 4 of 44 KB for gate/up), so every phase keeps the whole ring in
+// flight: at these loads the DRAM and L2 latency under full HBM traffic
+// (1.5-2 us) needs all of it. The producers drain the ring at each phase
+// boundary, where the MMAs wait for the phase before anyway.
 // Every split sum is taken in a fixed order: results are deterministic, and
 // primary rows never read auxiliary rows.
 #include <math.h>
@@ -70,23 +76,23 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 224;
 constexpr int kEpiThreads = 128;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;                        // ring stages (barrier pairs)
 constexpr int kCluster = 4;                          // CTAs per cluster = K splits
 constexpr int kTileN = 128;                          // W_o / W_down columns per cluster
 constexpr int kSliceN = kTileN / kCluster;           // columns a rank owns: 32
 constexpr int kMaxHalf = 112;                        // SwiGLU output columns per tile
 constexpr int kXBytes = kBM * kBK * 2;               // 16 KB activation tile
-constexpr int kSlot = kXBytes + 2 * kMaxHalf * kBK * 2;  // + up to 28 KB of weights
 constexpr int kRecvSlotBytes = kBM * kSliceN * 4;    // one sender's slice: 16 KB
 constexpr int kRecvBytes = (kCluster - 1) * kRecvSlotBytes;
 constexpr int kXchgPitch = 33;                       // coupling exchange: [64 rows][32 + 1]
 constexpr int kXchgFloats = 64 * kXchgPitch;         // aliases the receive buffer
 constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kSlot + kRecvBytes +
-                              kMaxHalf * 4 + 256;    // + barriers, flags
-static_assert(kSlot % 1024 == 0, "ring slots keep the 1024-byte swizzle alignment");
-static_assert(kTileN * kBK * 2 <= kSlot - kXBytes, "W_o / W_down stage fits a slot");
+// the ring: 4 SwiGLU stages of 16 + 28 KB, or 5 W_o / W_down stages of 16 + 16 KB
+constexpr size_t kRingBytes = 4 * (kXBytes + 2 * kMaxHalf * kBK * 2);
+constexpr size_t kSmemBytes = 1024 + kRingBytes + kRecvBytes + kMaxHalf * 4 +
+                              512;                   // + barriers, fill counts, flags
+static_assert(kRingBytes % 1024 == 0 && kXBytes % 1024 == 0, "1024-byte swizzle alignment");
 static_assert(kXchgFloats * 4 <= kRecvBytes, "exchange fits the receive buffer");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -98,6 +104,8 @@ struct Gemm {
   int BN;       // MMA N
   int half;     // SwiGLU output columns per tile (0: plain)
   int w_bytes;  // weight bytes per stage
+  int stage;    // bytes per ring stage (activation tile first; multiple of 1024)
+  int nst;      // ring stages in this phase
   uint32_t idesc;
 };
 
@@ -402,18 +410,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* recv = smem + static_cast<size_t>(kStages) * kSlot;   // [3][128 rows][32] fp32
+  uint8_t* recv = smem + kRingBytes;                             // [3][8 chunks][128 rows][16 B]
   float* xchg = reinterpret_cast<float*>(recv);                  // aliases recv (never both)
   float* bsl = reinterpret_cast<float*>(recv + kRecvBytes);      // [kMaxHalf] b of a tile
-  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);  // [kStages]
-  uint64_t* empty = full + kStages;                              // [kStages]
-  uint64_t* acc_full = empty + kStages;                          // [2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);  // [kMaxStages]
+  uint64_t* empty = full + kMaxStages;                           // [kMaxStages]
+  uint64_t* acc_full = empty + kMaxStages;                       // [2]
   uint64_t* acc_empty = acc_full + 2;                            // [2]
   uint64_t* mma_done = acc_empty + 2;                            // [1]
   uint64_t* red_full = mma_done + 1;  // this rank's slices from the other 3 ranks have landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
-  // [0] abort, [1] epilogue broadcast, [2] / [3] stages issued by the weight /
-  // activation producer
+  int* wfills = reinterpret_cast<int*>(red_full + 1);  // [kMaxStages] fills per slot: weights
+  int* xfills = wfills + kMaxStages;                     // [kMaxStages] activation tiles
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfills + kMaxStages);
+  // [0] abort, [1] epilogue broadcast
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -422,9 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cid = static_cast<int>(cluster_index());
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kMaxStages; ++i) {
       mbar_init(&full[i], 2);  // weight producer + activation producer
       mbar_init(&empty[i], 1);
+      wfills[i] = 0;
+      xfills[i] = 0;
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -434,8 +445,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(red_full, 1);  // this rank's expect_tx arrival + the senders' bytes
     flags[0] = 0;
     flags[1] = 0;
-    flags[2] = 0;
-    flags[3] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -454,69 +463,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   // one (the weights are constants); every other role waits for it first.
   if (warp != 0) pdl_wait();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ weight producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    // warp 0: weights (may run ahead of the kernel launched before this one:
+    // the weights are constants); warp 2: activation tiles.
     if (lane == 0) {
-      prefetch_tensormap(&tmWo);
-      prefetch_tensormap(&tmWg);
-      prefetch_tensormap(&tmWd);
-      const uint64_t pol = l2_policy_evict_first();
-      int s = 0;
-      uint32_t ph = 0;
-      long long n = 0;
+      const bool wrole = warp == 0;
+      if (wrole) {
+        prefetch_tensormap(&tmWo);
+        prefetch_tensormap(&tmWg);
+        prefetch_tensormap(&tmWd);
+      } else {
+        prefetch_tensormap(&tmXo);
+        prefetch_tensormap(&tmXg);
+        prefetch_tensormap(&tmXd);
+      }
+      const uint64_t pol = wrole ? l2_policy_evict_first() : l2_policy_evict_last();
+      int* fills = wrole ? wfills : xfills;
+      uint32_t par = 0;  // bit i: parity of this producer's fills of slot i
       bool ok = true;
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
-        const CUtensorMap* tm = q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd);
-        const Units us = units_of(g, q, cta, cid, G);
-        for (int u = us.first; u < g.units && ok; u += us.step) {
-          int k0, k1;
-          k_range(g, q, static_cast<int>(rank), k0, k1);
-          for (int kb = k0; kb < k1; ++kb, ++n) {
-            if (n >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
+        const CUtensorMap* tm = wrole ? (q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd))
+                                      : (q == 0 ? &tmXo : (q == 1 ? &tmXg : &tmXd));
+        // The ring changes its stage size at a phase boundary: every earlier
+        // fill of every slot must have been consumed first.
+        if (q > 0) {
+          for (int i = 0; i < kMaxStages && ok; ++i) {
+            if (!mbar_wait(&empty[i], ((par >> i) & 1u) ^ 1u)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
               ok = false;
-              break;
-            }
-            if (flags[0]) {
-              ok = false;
-              break;
-            }
-            uint8_t* wdst = smem + static_cast<size_t>(s) * kSlot + kXBytes;
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(g.w_bytes));
-            if (q == 1) {
-              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, u * g.half, pol);
-              tma_load_2d_hint(wdst + g.half * 128, tm, &full[s], kb * kBK, p.F + u * g.half,
-                               pol);
-            } else {
-              tma_load_2d_hint(wdst, tm, &full[s], kb * kBK, u * kTileN, pol);
-            }
-            if (++s == kStages) {
-              s = 0;
-              ph ^= 1u;
             }
           }
         }
-      }
-      flags[2] = static_cast<int>(n);
-      pdl_trigger();
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ activation producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmXo);
-      prefetch_tensormap(&tmXg);
-      prefetch_tensormap(&tmXd);
-      const uint64_t pol = l2_policy_evict_last();
-      int s = 0;
-      uint32_t ph = 0;
-      long long n = 0;
-      bool ok = true;
-      for (int q = 0; q < 3 && ok; ++q) {
-        const Gemm& g = p.g[q];
-        const CUtensorMap* tm = q == 0 ? &tmXo : (q == 1 ? &tmXg : &tmXd);
-        bool ready = q == 0;  // P0 reads the attention output: pdl_wait above
+        bool ready = wrole || q == 0;  // P0 reads the attention output: pdl_wait above
+        int s = 0;
         const Units us = units_of(g, q, cta, cid, G);
         for (int u = us.first; u < g.units && ok; u += us.step) {
           int k0, k1;
@@ -532,8 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_global();
             ready = true;
           }
-          for (int kb = k0; kb < k1; ++kb, ++n) {
-            if (n >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
+          for (int kb = k0; kb < k1; ++kb) {
+            if (!mbar_wait(&empty[s], ((par >> s) & 1u) ^ 1u)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
               ok = false;
@@ -543,27 +525,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], kXBytes);
-            tma_load_2d_hint(smem + static_cast<size_t>(s) * kSlot, tm, &full[s], kb * kBK, 0,
-                             pol);
-            if (++s == kStages) {
-              s = 0;
-              ph ^= 1u;
+            uint8_t* st = smem + static_cast<size_t>(s) * g.stage;
+            if (wrole) {
+              mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(g.w_bytes));
+              if (q == 1) {
+                tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * g.half, pol);
+                tma_load_2d_hint(st + kXBytes + g.half * 128, tm, &full[s], kb * kBK,
+                                 p.F + u * g.half, pol);
+              } else {
+                tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * kTileN, pol);
+              }
+            } else {
+              mbar_arrive_expect_tx(&full[s], kXBytes);
+              tma_load_2d_hint(st, tm, &full[s], kb * kBK, 0, pol);
             }
+            ++fills[s];
+            par ^= 1u << s;
+            if (++s == g.nst) s = 0;
           }
         }
       }
-      flags[3] = static_cast<int>(n);
+      if (wrole) pdl_trigger();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
+      uint32_t par = 0;  // bit i: parity of the next phase of full[i] to wait for
       int seg = 0;
       bool ok = true;
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
+        int s = 0;  // the producers restart the ring at every phase
         const Units us = units_of(g, q, cta, cid, G);
         for (int u = us.first; u < g.units && ok; u += us.step, ++seg) {
           int k0, k1;
@@ -579,24 +571,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
           for (int kb = k0; kb < k1; ++kb) {
-            if (!mbar_wait(&full[s], ph) || flags[0]) {
+            if (!mbar_wait(&full[s], (par >> s) & 1u) || flags[0]) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
               ok = false;
               break;
             }
+            par ^= 1u << s;
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * kSlot);
+            const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * g.stage);
             const uint32_t b_addr = a_addr + kXBytes;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk)
               umma_bf16(d_tmem, smem_desc(a_addr + kk * 32), smem_desc(b_addr + kk * 32), g.idesc,
                         (kb > k0 || kk > 0) ? 1u : 0u);
             umma_commit(&empty[s]);
-            if (++s == kStages) {
-              s = 0;
-              ph ^= 1u;
-            }
+            if (++s == g.nst) s = 0;
           }
           if (!ok) break;
           // (a unit without k-blocks commits at once: its partial is zero)
@@ -714,6 +704,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k0, k1;
       k_range(p.g[2], 2, static_cast<int>(rank), k0, k1);
       const int col0 = cid * kTileN + static_cast<int>(rank) * kSliceN;
+      // residual (x_mid, stored by other CTAs before counter A2) and coupling,
+      // loaded while the MMAs run
+      float res[32], cc[32];
+      if (live) {
+        load_bf16x32_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) res[i] = 0.f;
+      }
+      const bool aux = row >= p.mp && live;
+      if (aux && p.c != nullptr) {
+        load_bf16<32>(p.c + col0, cc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cc[i] = 0.f;
+      }
       if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
       if (!take_acc(acc, seg)) {
         fail();
@@ -722,22 +728,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         float own[32], sum[32];
         reduce_send(acc_addr(acc), k1 == k0, row, rank, recv, red_full, own);
         give_acc(acc);
-        // residual (x_mid, written by other CTAs) and coupling, while the
-        // other ranks' slices arrive
-        float res[32], cc[32];
-        if (live) {
-          load_bf16x32_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) res[i] = 0.f;
-        }
-        const bool aux = row >= p.mp && live;
-        if (aux && p.c != nullptr) {
-          load_bf16<32>(p.c + col0, cc);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) cc[i] = 0.f;
-        }
         if (!reduce_gather(row, rank, recv, red_full, 1, own, sum)) {
           fail();
         } else {
@@ -769,15 +759,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (threadIdx.x == 0 && flags[0]) {
-    // A wait gave up: a stage may have been filled by one producer only. The
-    // missing arrivals are made here so that those phases complete once the
-    // copies already issued have landed, and the last kStages stages are
-    // awaited (bounded): no copy is left in flight into shared memory.
-    const int nw = flags[2], nx = flags[3];
-    const int lo = nw < nx ? nw : nx, hi = nw < nx ? nx : nw;
-    for (int n = lo; n < hi; ++n) mbar_arrive(&full[n % kStages]);
-    for (int n = hi > kStages ? hi - kStages : 0; n < hi; ++n)
-      mbar_wait(&full[n % kStages], static_cast<uint32_t>((n / kStages) & 1));
+    // A wait gave up: a stage may have been filled by one producer only. Its
+    // missing arrival is made here, so that the phase completes once the copy
+    // already issued has landed, and the last fill of every slot is awaited
+    // (bounded): no copy is left in flight into shared memory.
+    for (int i = 0; i < kMaxStages; ++i) {
+      const int nw = wfills[i], nx = xfills[i];
+      if (nw != nx) mbar_arrive(&full[i]);
+      const int n = nw > nx ? nw : nx;
+      if (n > 0) mbar_wait(&full[i], static_cast<uint32_t>((n - 1) & 1));
+    }
   }
   if (threadIdx.x == 0) {
     __threadfence();
@@ -847,15 +838,32 @@ Plan make_plan(int M, int mp, int d, int qd, int F) {
   pl.T0 = d / kTileN;
   if (nc < 1 || pl.T0 > nc) return pl;  // one W_o / W_down tile per cluster
   pl.G = nc * kCluster;
-  // smallest multiple of 8 with at most G SwiGLU tiles
+  // smallest multiple of 8 with at most G SwiGLU tiles (the MMA's N = 2 H
+  // steps by 16 at M = 128)
   int H = static_cast<int>(ceil_div(F, pl.G));
   H = static_cast<int>(ceil_div(H, 8)) * 8;
-  if (H < 8) H = 8;
   if (H > kMaxHalf) return pl;
   pl.H1 = H;
   pl.T1 = static_cast<int>(ceil_div(F, H));
   pl.ok = true;
   return pl;
+}
+
+// A phase's GEMM: MMA N = BN (weight rows per k-block), ring stages of the
+// activation tile plus BN x 64 weights, as many as the ring holds (at most
+// kMaxStages).
+Gemm ring_gemm(int units, int kblocks, int BN, int half) {
+  Gemm g{};
+  g.units = units;
+  g.kblocks = kblocks;
+  g.BN = BN;
+  g.half = half;
+  g.w_bytes = BN * kBK * 2;
+  g.stage = static_cast<int>(round_up(static_cast<size_t>(kXBytes + g.w_bytes), 1024));
+  g.nst = static_cast<int>(kRingBytes / static_cast<size_t>(g.stage));
+  if (g.nst > kMaxStages) g.nst = kMaxStages;
+  g.idesc = make_idesc(kBM, BN);
+  return g;
 }
 
 // Workspace: counters | ss_part [d / 32][128].
@@ -899,10 +907,9 @@ extern "C" df_status dualflow_layer_post_attention(
   p.qd = q_dim;
   p.F = F;
   p.eps = eps;
-  p.g[0] = Gemm{pl.T0, q_dim / kBK, kTileN, 0, kTileN * kBK * 2, make_idesc(kBM, kTileN)};
-  p.g[1] = Gemm{pl.T1, d_model / kBK, 2 * pl.H1, pl.H1, 2 * pl.H1 * kBK * 2,
-                make_idesc(kBM, 2 * pl.H1)};
-  p.g[2] = Gemm{pl.T0, F / kBK, kTileN, 0, kTileN * kBK * 2, make_idesc(kBM, kTileN)};
+  p.g[0] = ring_gemm(pl.T0, q_dim / kBK, kTileN, 0);
+  p.g[1] = ring_gemm(pl.T1, d_model / kBK, 2 * pl.H1, pl.H1);
+  p.g[2] = ring_gemm(pl.T0, F / kBK, kTileN, 0);
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.b = static_cast<const __nv_bfloat16*>(b);
   p.c = static_cast<const __nv_bfloat16*>(c);

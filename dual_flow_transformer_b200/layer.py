@@ -14,12 +14,13 @@ Composition of library calls only (each step is a libdualflow kernel):
   7. H = SiLU(X'n W_gate^T) * (X'n W_up^T), aux += b_l H1    dualflow_grouped_proj (swiglu)
   8. X'' = X' + H W_down^T, aux += c_l (H1 W_down^T)         dualflow_grouped_proj (residual)
 
-With fused_post=True, steps 5-8 run as one persistent launch
+By default (fused_post=True) steps 5-8 run as one persistent launch
 (dualflow_layer_post_attention) when the sizes allow it: its weight producers
 stream W_o, W_gate/up and W_down back to back instead of four launches each
-ramping up and draining, and the norm's row scale multiplies the gate/up
-accumulators (the normalised rows are not stored). The default keeps the four
-calls.
+ramping up and draining, the W_o and W_down split-k sums are reduced inside
+4-CTA clusters, and the norm's row scale multiplies the gate/up accumulators
+(the normalised rows are not stored). fused_post=False, or sizes the fused
+launch does not take, use the four calls.
 
 Pages: "Sintesi Tecnica: Dual-Flow Transformers", sections "Architettura
 Core" (shared matrices, primary-only cache writes, auxiliary flow active at
@@ -38,7 +39,7 @@ from . import api
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
-                 num_splits=0, fused_post=False):
+                 num_splits=0, fused_post=True):
         self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
         self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
         self.d_model = weights["w_o"].shape[0]
