@@ -98,6 +98,11 @@ SIGNATURES = {
         _vp, _vp]),                             # err_flag, stream
     "dualflow_grouped_proj_batched_num_launches": (_c_int, [_c_int] * 5),
     "dualflow_rmsnorm": (_c_int, [_vp, _c_i64, _vp, _vp, _c_i64, _c_int, _c_int, _c_float, _vp]),
+    "dualflow_layer_pre_attention_supported": (_c_int, [_c_int] * 5),
+    "dualflow_layer_pre_attention": (_c_int, [
+        _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,  # x, w_qkv, m, d, Hq, Hkv, D
+        _c_float, _vp, _vp, _vp, _vp, _c_int, _vp,         # eps, qkv, caches, table, mbps, pos
+        _c_int, _c_int, _vp, _vp]),                        # block_size, num_blocks, err, stream
     "dualflow_layer_post_attention_workspace_size": (_c_size, [_c_int] * 4),
     "dualflow_layer_post_attention": (_c_int, [
         _vp, _vp, _vp, _vp, _vp, _vp, _vp,  # attn, x, w_o, w_gu, w_down, b, c

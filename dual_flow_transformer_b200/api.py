@@ -402,6 +402,46 @@ def rmsnorm(x, gain=None, y=None, eps=1e-5, stream=None):
     return y
 
 
+def layer_pre_attention_supported(m_primary, d_model, Hq, Hkv, D) -> bool:
+    return bool(_lib().dualflow_layer_pre_attention_supported(int(m_primary), int(d_model),
+                                                               int(Hq), int(Hkv), int(D)))
+
+
+def layer_pre_attention(x, w_qkv, Hq, Hkv, k_cache, v_cache, block_table, positions, *, eps=1e-5,
+                        qkv=None, err_flag=None, stream=None):
+    """r = RMSNorm row scale of x; qkv = bf16(r x W_qkv^T) (auxiliary rows: Q
+    columns only); the primary rows' K / V columns appended to the cache at
+    positions[b], in one launch.
+
+    x: bf16 [2m, d_model] (primary rows first); w_qkv: bf16 [Hq D + 2 Hkv D,
+    d_model]; caches bf16 [num_blocks, Hkv, block_size, D]; block_table int32
+    [m, max_blocks]; positions int32 [m]. Returns qkv [2m, Hq D + 2 Hkv D]."""
+    M, d_model = x.shape
+    num_blocks, Hkv2, bs, D = k_cache.shape
+    mp = M // 2
+    nout = (Hq + 2 * Hkv) * D
+    for t in (x, w_qkv, k_cache, v_cache):
+        if not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("bf16 contiguous tensors required")
+    if M % 2 or Hkv2 != Hkv or tuple(w_qkv.shape) != (nout, d_model) or \
+            v_cache.shape != k_cache.shape or block_table.shape[0] != mp or \
+            positions.numel() != mp:
+        raise ValueError("shape mismatch")
+    if block_table.dtype != torch.int32 or positions.dtype != torch.int32 or \
+            not block_table.is_contiguous():
+        raise ValueError("int32 contiguous block_table / positions required")
+    if qkv is None:
+        qkv = torch.empty((M, nout), dtype=torch.bfloat16, device=x.device)
+    if not qkv.is_contiguous() or tuple(qkv.shape) != (M, nout):
+        raise ValueError("qkv must be contiguous [2m, N]")
+    st = _lib().dualflow_layer_pre_attention(
+        _ptr(x), _ptr(w_qkv), mp, d_model, int(Hq), int(Hkv), D, float(eps), _ptr(qkv),
+        _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1], _ptr(positions),
+        bs, num_blocks, _ptr(err_flag), _stream(stream))
+    L.check("dualflow_layer_pre_attention", st)
+    return qkv
+
+
 def layer_post_attention_workspace_size(m_primary, d_model, q_dim, F) -> int:
     return _lib().dualflow_layer_post_attention_workspace_size(int(m_primary), int(d_model),
                                                                int(q_dim), int(F))

@@ -63,6 +63,7 @@
 
 #include <mutex>
 
+#include "cluster.cuh"
 #include "common.cuh"
 #include "host_util.h"
 #include "umma.cuh"
@@ -71,11 +72,12 @@ namespace df {
 namespace post {
 
 using namespace umma;
+using namespace cl;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 224;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiThreads = 128;  // the epilogue named barrier (cl::epi_bar) counts 128
 constexpr int kMaxStages = 8;                        // ring stages (barrier pairs)
 constexpr int kCluster = 4;                          // CTAs per cluster = K splits
 constexpr int kTileN = 128;                          // W_o / W_down columns per cluster
@@ -124,25 +126,6 @@ struct Params {
   int32_t* err;
 };
 
-__device__ __forceinline__ void epi_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-}
-
-// Epilogue barrier that also ANDs a predicate over the epilogue threads, so
-// that a wait which gave up in one thread stops all of them together.
-__device__ __forceinline__ bool epi_bar_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, 1, %2, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
-      : "memory");
-  return r != 0;
-}
-
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -151,42 +134,6 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_index() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-
-// All threads of all CTAs of the cluster.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// The address of this CTA's shared-memory location `addr` in cluster rank `rank`.
-__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-
-// 16 bytes into another CTA's shared memory, counted on its mbarrier.
-__device__ __forceinline__ void st_async16(uint32_t raddr, float a, float b, float c, float d,
-                                           uint32_t rbar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, "
-      "[%5];" ::"r"(raddr),
-      "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
-      "r"(__float_as_uint(d)), "r"(rbar)
-      : "memory");
 }
 
 // 32 bf16 values written by other CTAs of this launch (read through L2).
@@ -256,11 +203,6 @@ __device__ __forceinline__ bool epi_wait_count(const int* cnt, int target, int e
   const bool ok = *flag != 0;
   epi_bar();
   return ok;
-}
-
-// Receive slot of sender s in owner o's buffer (0..2).
-__device__ __forceinline__ uint32_t recv_slot(uint32_t s, uint32_t o) {
-  return (s - o - 1u) & 3u;
 }
 
 // Reduce-scatter of a split-K accumulator over the cluster (thread = row).

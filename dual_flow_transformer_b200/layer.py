@@ -14,6 +14,13 @@ Composition of library calls only (each step is a libdualflow kernel):
   7. H = SiLU(X'n W_gate^T) * (X'n W_up^T), aux += b_l H1    dualflow_grouped_proj (swiglu)
   8. X'' = X' + H W_down^T, aux += c_l (H1 W_down^T)         dualflow_grouped_proj (residual)
 
+By default (fused_pre=True) steps 1-3 run as one launch
+(dualflow_layer_pre_attention) when the sizes allow it: 4-CTA clusters split
+the QKV product along K and reduce it through distributed shared memory, the
+first norm's row scale multiplies the accumulator (the normalised rows are
+not stored) and the primary K/V columns go straight into the cache.
+fused_pre=False, or sizes the fused launch does not take, use the three calls.
+
 By default (fused_post=True) steps 5-8 run as one persistent launch
 (dualflow_layer_post_attention) when the sizes allow it: its weight producers
 stream W_o, W_gate/up and W_down back to back instead of four launches each
@@ -39,7 +46,7 @@ from . import api
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
-                 num_splits=0, fused_post=True):
+                 num_splits=0, fused_pre=True, fused_post=True):
         self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
         self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
         self.d_model = weights["w_o"].shape[0]
@@ -66,6 +73,8 @@ class DualFlowLayer:
         self.attn_ws = api.new_attn_workspace(B, Hq, Hkv, D, self.max_seqlen, num_splits, dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.attn_launches = api.decode_attn_num_launches(B, Hkv, self.max_seqlen, num_splits)
+        self.fused_pre = bool(fused_pre) and \
+            api.layer_pre_attention_supported(B, self.d_model, Hq, Hkv, D)
         self.fused_post = bool(fused_post) and \
             api.layer_post_attention_workspace_size(B, self.d_model, qd, F) > 0
         self.post_ws = (api.new_post_attention_workspace(B, self.d_model, qd, F, dev)
@@ -78,15 +87,17 @@ class DualFlowLayer:
                              + api.grouped_proj_num_launches(M, *weights["w_gu"].shape, "swiglu")
                              + api.grouped_proj_num_launches(M, *weights["w_down"].shape,
                                                              "residual"))
-        self._gemm_launches = (api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
-                               + post_launches)
+        pre_launches = 1 if self.fused_pre else \
+            2 + api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
+        self._launches = pre_launches + self.attn_launches + post_launches
 
     @property
     def launches_per_step(self) -> int:
-        """Kernel launches of one step: the first norm, the QKV projection,
-        the append, the attention and the post-attention half (one launch
-        fused, else W_o, the second norm, gate/up and down)."""
-        return 2 + self.attn_launches + self._gemm_launches
+        """Kernel launches of one step: the pre-attention half (one launch
+        fused, else the first norm, the QKV projection and the append), the
+        attention and the post-attention half (one launch fused, else W_o, the
+        second norm, gate/up and down)."""
+        return self._launches
 
     # ------------------------------------------------------------ CUDA graphs
     def capture(self, X, k_cache, v_cache, block_table, positions, seqlens):
@@ -151,7 +162,11 @@ class DualFlowLayer:
         # Each projection warms L2 with the first weight blocks of the next one
         # (o -> gate/up -> down -> the next step's QKV); none after the QKV
         # projection, whose successor is the HBM-bound attention.
-        if part == "pre":
+        if part == "pre" and self.fused_pre:
+            api.layer_pre_attention(X, w["w_qkv"], Hq, Hkv, k_cache, v_cache, block_table,
+                                    positions, eps=self.eps, qkv=qkv, err_flag=self.err,
+                                    stream=stream)
+        elif part == "pre":
             api.rmsnorm(X, y=self.xn, eps=self.eps, stream=stream)
             api.grouped_proj(self.xn, B, w["w_qkv"], n_aux=qd, y=qkv, workspace=self.proj_ws,
                              err_flag=self.err, stream=stream)

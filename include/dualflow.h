@@ -358,6 +358,50 @@ df_status dualflow_grouped_proj_batched(
 int dualflow_grouped_proj_batched_num_launches(int M, int N, int K, int epilogue, int batch);
 
 /* ------------------------------------------------------------------------ */
+/* Pre-attention half of the decoder layer in ONE launch.                    */
+/*                                                                           */
+/* Pages "Sintesi Tecnica" ("Architettura Core": the flows share the         */
+/* projection matrices, only the primary flow writes the persistent KV      */
+/* cache, the auxiliary flow needs only its query; "Costi di Inferenza":     */
+/* grouped decode reads the unique weights once for both flows). With rows   */
+/* [0, m_primary) primary and [m_primary, 2 m_primary) auxiliary, M =        */
+/* 2 m_primary, q_dim = Hq D, kv_dim = Hkv D, N = q_dim + 2 kv_dim:          */
+/*   r   = 1 / sqrt(mean_row(x^2) + eps)          (RMSNorm, unit gain)       */
+/*   qkv = bf16(r (x W_qkv^T)): primary rows all N columns, auxiliary rows   */
+/*         the q_dim Q columns only (their K / V columns are not written)    */
+/*   and, as dualflow_kv_append, primary row b's K and V columns (the same   */
+/*   bf16 values) into the cache slot of positions[b].                       */
+/* which is dualflow_rmsnorm -> dualflow_grouped_proj (n_aux = q_dim) ->     */
+/* dualflow_kv_append computed by one launch of 4-CTA clusters: each         */
+/* cluster owns a column tile, its 4 CTAs multiply the 4 quarters of K and   */
+/* reduce the partial sums (and the row sums of squares of the norm)        */
+/* through distributed shared memory. The row scale multiplies the          */
+/* accumulator (the normalised rows are not rounded to bf16 and stored), so */
+/* the result matches the three-call form within the bf16 tolerance, not     */
+/* bit for bit. Sums are taken in a fixed order (deterministic); primary     */
+/* rows never depend on auxiliary rows.                                      */
+/*                                                                           */
+/* x     : bf16 [M][d_model]; w_qkv : bf16 [N][d_model] (Q rows, K rows, V   */
+/* rows), row-major. qkv : bf16 [M][N], written as above (16-byte aligned).  */
+/* k_cache, v_cache, block_table, max_blocks_per_seq, positions, block_size, */
+/* num_blocks: as dualflow_kv_append (bf16 cache); an out-of-table position  */
+/* or page is skipped and flagged in err_flag. w_qkv is read before the wait */
+/* for the kernel launched ahead on the stream (programmatic dependent       */
+/* launch), so that kernel must not write it. No workspace.                  */
+/* Supported (else DF_ERR_UNSUPPORTED; dualflow_layer_pre_attention_supported*/
+/* returns 0): 1 <= m_primary <= 64, d_model % 64 == 0, D % 8 == 0, and N at */
+/* most 256 x the number of 4-CTA clusters the device holds at once (33 on  */
+/* a 148-SM B200: N <= 8448). Needs a current CUDA device. One launch.       */
+/* ------------------------------------------------------------------------ */
+int dualflow_layer_pre_attention_supported(int m_primary, int d_model, int Hq, int Hkv, int D);
+df_status dualflow_layer_pre_attention(const void* x, const void* w_qkv, int m_primary,
+                                       int d_model, int Hq, int Hkv, int D, float eps, void* qkv,
+                                       void* k_cache, void* v_cache, const int32_t* block_table,
+                                       int max_blocks_per_seq, const int32_t* positions,
+                                       int block_size, int num_blocks, int32_t* err_flag,
+                                       void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Post-attention half of the decoder layer in ONE persistent launch.        */
 /*                                                                           */
 /* Pages "Sintesi Tecnica" ("Architettura Core": the flows share the output  */

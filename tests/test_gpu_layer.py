@@ -18,14 +18,14 @@ SMALL = dataclasses.replace(synth.WORKLOADS["layer"], B=8, d_model=512, Hq=4, Hk
                             F=1024, cache_len=200, seed=50)
 
 
-def _run_gpu(inp, dev, num_splits=0, fused_post=False):
+def _run_gpu(inp, dev, num_splits=0, fused=False):
     d = to_dev(inp, dev)
     w = {k: d[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
     B = inp["B"]
     layer = DualFlowLayer(w, inp["Hq"], inp["Hkv"], inp["D"], inp["F"], B,
                           int(inp["positions"].max()) + 1, device=dev, num_splits=num_splits,
-                          fused_post=fused_post)
-    assert layer.fused_post == fused_post
+                          fused_pre=fused, fused_post=fused)
+    assert layer.fused_pre == fused and layer.fused_post == fused
     X = torch.cat([d["x1"], d["x2"]]).contiguous()
     seqlens = (d["positions"] + 1).to(torch.int32)
     out = layer.step(X, d["k_cache"], d["v_cache"], d["block_table"], d["positions"], seqlens)
@@ -34,10 +34,10 @@ def _run_gpu(inp, dev, num_splits=0, fused_post=False):
     return out.cpu(), d, layer
 
 
-# The fused post-attention launch keeps the normalised rows of the second
-# norm in fp32 (its row scale multiplies the gate/up accumulators): compare it
-# with the oracle rounded at every other stored interface.
-FUSED_ROUNDED = tuple(n for n in oracle.LAYER_INTERFACES if n != "xn2")
+# The fused launches keep the normalised rows of both norms in fp32 (their row
+# scales multiply the QKV and gate/up accumulators): compare them with the
+# oracle rounded at every other stored interface.
+FUSED_ROUNDED = tuple(n for n in oracle.LAYER_INTERFACES if n not in ("xn", "xn2"))
 
 
 def _oracle(inp, rows=None, rounded=oracle.LAYER_INTERFACES):
@@ -53,28 +53,28 @@ def _oracle(inp, rows=None, rounded=oracle.LAYER_INTERFACES):
     return r
 
 
-@pytest.mark.parametrize("fused_post", [True, False])
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("coupled", [True, False])
-def test_layer_step_small(cuda_device, coupled, fused_post):
+def test_layer_step_small(cuda_device, coupled, fused):
     w = dataclasses.replace(SMALL, coupled_mlp=coupled)
     inp = synth.make_layer_inputs(w)
-    out, d, layer = _run_gpu(inp, cuda_device, fused_post=fused_post)
-    ref = _oracle(inp, rounded=FUSED_ROUNDED if fused_post else oracle.LAYER_INTERFACES)
+    out, d, layer = _run_gpu(inp, cuda_device, fused=fused)
+    ref = _oracle(inp, rounded=FUSED_ROUNDED if fused else oracle.LAYER_INTERFACES)
     assert_close(out, ref["x_out"], "bf16", "layer x_out")
     assert_close(layer.x_mid.cpu(), ref["x_mid"], "bf16", "layer x_mid")
     assert_close(layer.h.cpu(), ref["h"], "bf16", "layer h")
 
 
-@pytest.mark.parametrize("fused_post", [False, True])
-def test_layer_primary_flow_is_self_sufficient(cuda_device, fused_post):
+@pytest.mark.parametrize("fused", [False, True])
+def test_layer_primary_flow_is_self_sufficient(cuda_device, fused):
     inp = synth.make_layer_inputs(SMALL)
-    out1, _, _ = _run_gpu(inp, cuda_device, fused_post=fused_post)
+    out1, _, _ = _run_gpu(inp, cuda_device, fused=fused)
     other = dict(inp)
     other["x2"] = inp["x2"] * 3
     other["a"] = -inp["a"]
     other["b"] = inp["b"] * 2
     other["c"] = -inp["c"]
-    out2, _, _ = _run_gpu(other, cuda_device, fused_post=fused_post)
+    out2, _, _ = _run_gpu(other, cuda_device, fused=fused)
     B = inp["B"]
     assert torch.equal(out1[:B].view(torch.int16), out2[:B].view(torch.int16))
 
@@ -94,16 +94,16 @@ def test_layer_append_writes_primary_rows_only(cuda_device):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("fused_post", [False, True])
-def test_layer_step_full_size_sampled(cuda_device, fused_post):
+@pytest.mark.parametrize("fused", [False, True])
+def test_layer_step_full_size_sampled(cuda_device, fused):
     """The 4096/14336 layer, B = 64 per flow, cache 4096 + 1, in the launch
     configurations the benchmark can time; the oracle recomputes 17 of the 64
     sequences (every fourth and the last), both flows."""
     inp = synth.make_layer_inputs(synth.WORKLOADS["layer"])
-    out, _, _ = _run_gpu(inp, cuda_device, fused_post=fused_post)
+    out, _, _ = _run_gpu(inp, cuda_device, fused=fused)
     rows = list(range(0, 64, 4)) + [63]
-    ref = _oracle(inp, rows, rounded=FUSED_ROUNDED if fused_post else oracle.LAYER_INTERFACES)
+    ref = _oracle(inp, rows, rounded=FUSED_ROUNDED if fused else oracle.LAYER_INTERFACES)
     B = inp["B"]
     got = torch.cat([out[rows], out[[B + r for r in rows]]])
     assert_close(got, ref["x_out"], "bf16",
-                 "full layer x_out (17 seq%s)" % (", fused" if fused_post else ""))
+                 "full layer x_out (17 seq%s)" % (", fused" if fused else ""))
