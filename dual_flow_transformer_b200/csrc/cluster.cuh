@@ -64,6 +64,19 @@ __device__ __forceinline__ void st_async16(uint32_t raddr, float a, float b, flo
       : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// this CTA's shared memory into another CTA's (dst, rbar: shared::cluster
+// addresses from map_rank), counted (complete_tx) on its mbarrier. The source
+// must have been made visible to the async proxy (fence.proxy.async) first.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t rbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(dst),
+      "r"(smem_u32(src)), "r"(bytes), "r"(rbar)
+      : "memory");
+}
+
 // Receive slot of sender s in owner o's buffer (0..2) in a 4-CTA cluster.
 __device__ __forceinline__ uint32_t recv_slot(uint32_t s, uint32_t o) {
   return (s - o - 1u) & 3u;

@@ -31,6 +31,13 @@ bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t batch, uin
                          uint64_t cols, uint64_t row_pitch_bytes, uint64_t batch_pitch_bytes,
                          uint32_t box_rows, uint32_t box_cols);
 
+// General 3-D tensor map (128-byte swizzle): dims[0] contiguous elements,
+// dims[1], dims[2] at the given byte strides (multiples of 16, in any
+// order), box[0..2] elements per dimension. The box lands in shared memory
+// dimension 0 fastest, then 1, then 2.
+bool encode_tmap_bf16_3d_box(CUtensorMap* map, const void* base, const uint64_t dims[3],
+                             const uint64_t strides_bytes[2], const uint32_t box[3]);
+
 // Opt `kernel` into `bytes` of dynamic shared memory on the current device.
 // The attribute belongs to the device, so it is set once per (kernel,
 // device) pair; later calls only look the pair up.

@@ -41,8 +41,11 @@
 //       (slice order) for r; SwiGLU + b coupling straight from TMEM -> h
 //   --- grid counter C: every column of h is stored
 //   P2  W_down: as P0 over K = F; the owner adds x_mid and the c coupling
-//       (the primary row's sum reaches its auxiliary row through shared
-//       memory) -> x_out
+//       -> x_out
+// The activation tiles interleave the flows (sequence j's primary row at tile
+// row 2j, its auxiliary row at 2j + 1, by a [sequence][flow][K] tensor map),
+// so both rows of a sequence sit in neighbouring TMEM lanes of one warp and
+// the one-way b and c couplings are a warp shuffle from the primary lane.
 // Every cluster is resident (one CTA per SM, grid = 4 x the device's maximum
 // of co-resident 4-CTA clusters), so the grid counters cannot deadlock; every
 // wait is bounded.
@@ -55,7 +58,9 @@
 // W_down, 4 of 44 KB for gate/up), so every phase keeps the whole ring in
 // flight: at these loads the DRAM and L2 latency under full HBM traffic
 // (1.5-2 us) needs all of it. The producers drain the ring at each phase
-// boundary, where the MMAs wait for the phase before anyway.
+// boundary, where the MMAs wait for the phase before anyway. (L2 prefetches
+// of the next phase's weights at a boundary were measured to delay the grid
+// counters behind them by more than they saved.)
 // Every split sum is taken in a fixed order: results are deterministic, and
 // primary rows never read auxiliary rows.
 #include <math.h>
@@ -86,8 +91,6 @@ constexpr int kMaxHalf = 112;                        // SwiGLU output columns pe
 constexpr int kXBytes = kBM * kBK * 2;               // 16 KB activation tile
 constexpr int kRecvSlotBytes = kBM * kSliceN * 4;    // one sender's slice: 16 KB
 constexpr int kRecvBytes = (kCluster - 1) * kRecvSlotBytes;
-constexpr int kXchgPitch = 33;                       // coupling exchange: [64 rows][32 + 1]
-constexpr int kXchgFloats = 64 * kXchgPitch;         // aliases the receive buffer
 constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
 // the ring: 4 SwiGLU stages of 16 + 28 KB, or 5 W_o / W_down stages of 16 + 16 KB
@@ -95,7 +98,6 @@ constexpr size_t kRingBytes = 4 * (kXBytes + 2 * kMaxHalf * kBK * 2);
 constexpr size_t kSmemBytes = 1024 + kRingBytes + kRecvBytes + kMaxHalf * 4 +
                               512;                   // + barriers, fill counts, flags
 static_assert(kRingBytes % 1024 == 0 && kXBytes % 1024 == 0, "1024-byte swizzle alignment");
-static_assert(kXchgFloats * 4 <= kRecvBytes, "exchange fits the receive buffer");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum { kCntA2 = 0, kCntC = 1, kCntExit = 2 };
@@ -288,29 +290,26 @@ __device__ float row_scale(const Params& p, int row) {
 }
 
 // P1 epilogue of tile t: h[row][t*H + j] = SiLU(rs g) * (rs u) (+ b * primary
-// row's value for auxiliary rows), in 32-column chunks (8-column tail); the
-// primary rows' values reach their auxiliary rows through `xchg`.
+// row's value for auxiliary rows), in 32-column chunks (8-column tail). The
+// primary row of a sequence is the neighbouring TMEM lane of its auxiliary
+// row (lanes 2j, 2j + 1), so its values arrive by one warp shuffle.
 template <int W>
 __device__ __forceinline__ void swiglu_chunk(const Params& p, uint32_t taddr, int H, int c, int col0,
-                                             int row, float rs, float* xchg, const float* bsl) {
+                                             int row, bool live, bool aux, float rs,
+                                             const float* bsl) {
   float g[W], u[W];
   tmem_ld<W>(taddr + c, g);
   tmem_ld<W>(taddr + H + c, u);
 #pragma unroll
   for (int i = 0; i < W; ++i) g[i] = silu_f(rs * g[i]) * (rs * u[i]);
   if (p.b != nullptr) {
-    if (row < p.mp) {
 #pragma unroll
-      for (int i = 0; i < W; ++i) xchg[row * kXchgPitch + i] = g[i];
+    for (int i = 0; i < W; ++i) {
+      const float pv = __shfl_xor_sync(0xffffffffu, g[i], 1);
+      if (aux) g[i] = fmaf(bsl[c + i], pv, g[i]);
     }
-    epi_bar();
-    if (row >= p.mp && row < p.M && col0 + c < p.F) {
-#pragma unroll
-      for (int i = 0; i < W; ++i) g[i] = fmaf(bsl[c + i], xchg[(row - p.mp) * kXchgPitch + i], g[i]);
-    }
-    epi_bar();
   }
-  if (row < p.M) {
+  if (live) {
     // a chunk of the last tile may reach past F: store its 8-column groups
     // that lie inside (F and H are multiples of 8)
 #pragma unroll
@@ -324,13 +323,13 @@ __device__ __forceinline__ void swiglu_chunk(const Params& p, uint32_t taddr, in
   }
 }
 
-__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int row, float rs,
-                                float* xchg, const float* bsl) {
+__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int row, bool live,
+                                bool aux, float rs, const float* bsl) {
   const int H = p.g[1].half;
   const int col0 = t * H;
   int c = 0;
-  for (; c + 32 <= H; c += 32) swiglu_chunk<32>(p, taddr, H, c, col0, row, rs, xchg, bsl);
-  for (; c < H; c += 8) swiglu_chunk<8>(p, taddr, H, c, col0, row, rs, xchg, bsl);
+  for (; c + 32 <= H; c += 32) swiglu_chunk<32>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
+  for (; c < H; c += 8) swiglu_chunk<8>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
 }
 
 // Tile t's slice of the coupling vector b into shared memory (zeros past F),
@@ -353,7 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* recv = smem + kRingBytes;                             // [3][8 chunks][128 rows][16 B]
-  float* xchg = reinterpret_cast<float*>(recv);                  // aliases recv (never both)
   float* bsl = reinterpret_cast<float*>(recv + kRecvBytes);      // [kMaxHalf] b of a tile
   uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);  // [kMaxStages]
   uint64_t* empty = full + kMaxStages;                           // [kMaxStages]
@@ -479,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             } else {
               mbar_arrive_expect_tx(&full[s], kXBytes);
-              tma_load_2d_hint(st, tm, &full[s], kb * kBK, 0, pol);
+              tma_load_3d_hint(st, tm, &full[s], kb * kBK, 0, 0, pol);
             }
             ++fills[s];
             par ^= 1u << s;
@@ -544,8 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue warps
     const int quarter = warp & 3;
     const int et = threadIdx.x - 3 * 32;
-    const int row = quarter * 32 + lane;  // this thread's TMEM lane = accumulator row
-    const bool live = row < p.M;
+    // The activation tiles hold the rows interleaved, sequence j's primary
+    // row at tile row 2j and its auxiliary row at 2j + 1: this thread's TMEM
+    // lane tl is tile row tl, which is `row` of x / x_mid / h / x_out.
+    const int tl = quarter * 32 + lane;
+    const int seq = tl >> 1;
+    const bool aux = (tl & 1) != 0;
+    const bool live = seq < p.mp;
+    const int row = aux ? p.mp + seq : seq;
     volatile int* eflag = flags + 1;
     int seg = 0;
     bool ok = true;
@@ -594,9 +598,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tc_fence_after();
         float own[32], sum[32];
-        reduce_send(acc_addr(acc), k1 == k0, row, rank, recv, red_full, own);
+        reduce_send(acc_addr(acc), k1 == k0, tl, rank, recv, red_full, own);
         give_acc(acc);
-        if (!reduce_gather(row, rank, recv, red_full, 0, own, sum)) {
+        if (!reduce_gather(tl, rank, recv, red_full, 0, own, sum)) {
           fail();
         } else {
           float ss = 0.f;
@@ -606,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ss = fmaf(sum[i], sum[i], ss);
           }
           if (live) store_bf16<32>(p.x_mid + static_cast<size_t>(row) * p.d + col0, sum);
-          p.ss_part[static_cast<size_t>(cid * kCluster + rank) * kBM + row] = live ? ss : 0.f;
+          if (live) p.ss_part[static_cast<size_t>(cid * kCluster + rank) * kBM + row] = ss;
         }
       }
       ++seg;
@@ -632,15 +636,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      swiglu_epilogue(p, u, acc_addr(acc), row, rs, xchg, bsl);
+      swiglu_epilogue(p, u, acc_addr(acc), row, live, aux, rs, bsl);
       give_acc(acc);
     }
     ok = epi_bar_and(ok);
     arrive_count(p.cnt + kCntC, et);
     // P2: W_down tile `cid` over this rank's K quarter; reduce-scatter; x_out.
-    // The other ranks' receive buffers hold their gate/up coupling exchange
-    // until every CTA is past P1 (counter C); a rank without k-blocks would
-    // otherwise send before that.
+    // (A rank without k-blocks sends at once: counter C orders its sends
+    // after the receivers' last use of P0's data, like everyone else's.)
     if (ok && cid < p.g[2].units && grid_wait(kCntC)) {
       const int acc = seg & 1;
       int k0, k1;
@@ -655,8 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) res[i] = 0.f;
       }
-      const bool aux = row >= p.mp && live;
-      if (aux && p.c != nullptr) {
+      if (aux && live && p.c != nullptr) {
         load_bf16<32>(p.c + col0, cc);
       } else {
 #pragma unroll
@@ -668,22 +670,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tc_fence_after();
         float own[32], sum[32];
-        reduce_send(acc_addr(acc), k1 == k0, row, rank, recv, red_full, own);
+        reduce_send(acc_addr(acc), k1 == k0, tl, rank, recv, red_full, own);
         give_acc(acc);
-        if (!reduce_gather(row, rank, recv, red_full, 1, own, sum)) {
+        if (!reduce_gather(tl, rank, recv, red_full, 1, own, sum)) {
           fail();
         } else {
           if (p.c != nullptr) {
-            epi_bar();  // every thread is done with the receive buffer (xchg aliases it)
-            if (row < p.mp) {
+            // the primary row's sum from the neighbouring lane
 #pragma unroll
-              for (int i = 0; i < 32; ++i) xchg[row * kXchgPitch + i] = sum[i];
-            }
-            epi_bar();
-            if (aux) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                sum[i] = fmaf(cc[i], xchg[(row - p.mp) * kXchgPitch + i], sum[i]);
+            for (int i = 0; i < 32; ++i) {
+              const float pv = __shfl_xor_sync(0xffffffffu, sum[i], 1);
+              if (aux) sum[i] = fmaf(cc[i], pv, sum[i]);
             }
           }
 #pragma unroll
@@ -864,13 +861,23 @@ extern "C" df_status dualflow_layer_post_attention(
   p.err = err_flag;
 
   CUtensorMap tmXo, tmWo, tmXg, tmWg, tmXd, tmWd;
-  const uint64_t Mu = static_cast<uint64_t>(M), du = static_cast<uint64_t>(d_model),
+  const uint64_t du = static_cast<uint64_t>(d_model),
                  qu = static_cast<uint64_t>(q_dim), Fu = static_cast<uint64_t>(F);
-  if (!encode_tmap_bf16_2d(&tmXo, attn, Mu, qu, qu * 2, kBM, kBK) ||
+  // Activations [M][K] viewed as [sequence][flow][K]: a 64 x 2 x 64 box puts
+  // sequence j's primary row at tile row 2j and its auxiliary row at 2j + 1
+  // (sequences past m_primary read as zeros).
+  const uint64_t mpu = static_cast<uint64_t>(m_primary);
+  auto x_map = [&](CUtensorMap* m, const void* base, uint64_t K) {
+    const uint64_t dims[3] = {K, 2, mpu};
+    const uint64_t strides[2] = {mpu * K * 2, K * 2};
+    const uint32_t box[3] = {kBK, 2, kBM / 2};
+    return encode_tmap_bf16_3d_box(m, base, dims, strides, box);
+  };
+  if (!x_map(&tmXo, attn, qu) ||
       !encode_tmap_bf16_2d(&tmWo, w_o, du, qu, qu * 2, kTileN, kBK) ||
-      !encode_tmap_bf16_2d(&tmXg, x_mid, Mu, du, du * 2, kBM, kBK) ||
+      !x_map(&tmXg, x_mid, du) ||
       !encode_tmap_bf16_2d(&tmWg, w_gu, 2 * Fu, du, du * 2, static_cast<uint32_t>(pl.H1), kBK) ||
-      !encode_tmap_bf16_2d(&tmXd, h, Mu, Fu, Fu * 2, kBM, kBK) ||
+      !x_map(&tmXd, h, Fu) ||
       !encode_tmap_bf16_2d(&tmWd, w_down, du, Fu, Fu * 2, kTileN, kBK))
     return DF_ERR_CUDA;
 

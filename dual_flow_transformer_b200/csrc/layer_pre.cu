@@ -53,10 +53,11 @@ constexpr int kCluster = 4;
 constexpr int kMaxTileN = 256;
 constexpr int kMaxStages = 8;
 constexpr int kXBytes = kBM * kBK * 2;     // 16 KB activation tile
-constexpr size_t kRingBytes = 200 * 1024;  // e.g. 5 stages of 16 + 24 KB at TN = 192
+constexpr size_t kRingBytes = 208 * 1024;  // e.g. 5 stages of 16 + 24 KB at TN = 192
 constexpr size_t kSmemBytes = 1024 + kRingBytes + 512;  // + barriers, flags
-// receive buffer (aliases the retired ring): [3 senders][TN/16 + 1 chunks][128 rows][16 B]
-static_assert(3 * (kMaxTileN / 16 + 1) * kBM * 16 <= kRingBytes, "receive buffer fits the ring");
+// The retired ring holds the receive buffer [3 senders][TN/16 + 1 chunks][128
+// rows][16 B] and, after it, the outgoing slices in the same layout.
+static_assert(6 * (kMaxTileN / 16 + 1) * kBM * 16 <= kRingBytes, "reduce buffers fit the ring");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Params {
@@ -76,10 +77,10 @@ struct Params {
   int32_t* err;
 };
 
-// Cache element offset of (primary row b, column c of the K or V block, i.e.
-// KV head c / D, dimension c % D) or -1 (and the error bit) when b's position
-// or page is outside the table.
-__device__ __forceinline__ int64_t cache_offset(const Params& p, int b, int c) {
+// Cache element offset of (sequence b, KV head 0, dimension 0) at b's
+// position (head g adds g block_size D), or -1 (and the error bit) when b's
+// position or page is outside the table.
+__device__ __forceinline__ int64_t cache_row_base(const Params& p, int b) {
   const int pos = p.positions[b];
   if (pos < 0 || pos / p.block_size >= p.max_blocks) {
     set_err(p.err, DF_DEVERR_POSITION);
@@ -91,9 +92,7 @@ __device__ __forceinline__ int64_t cache_offset(const Params& p, int b, int c) {
     set_err(p.err, DF_DEVERR_BLOCK);
     return -1;
   }
-  const int g = c / p.D, dim = c - g * p.D;
-  return ((static_cast<int64_t>(page) * p.Hkv + g) * p.block_size + pos % p.block_size) * p.D +
-         dim;
+  return (static_cast<int64_t>(page) * p.Hkv * p.block_size + pos % p.block_size) * p.D;
 }
 
 // 8 bf16 values (16 bytes) from 8 floats.
@@ -230,6 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this row's sum of squares over this rank's K quarter, from the
     // activation tiles in the ring (a row's 128 bytes in any chunk order)
     const int row = (warp & 3) * 32 + lane;
+    // a primary row's cache slot, looked up while the MMAs run
+    const int64_t cbase = row < p.mp ? cache_row_base(p, row) : -1;
     float ss = 0.f;
     int s = 0;
     uint32_t ph = 0;
@@ -275,13 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool empty_rank = k1 == k0;
       if (threadIdx.x == 3 * 32)
         mbar_arrive_expect_tx(red_full, static_cast<uint32_t>(3 * slot_bytes));
-      // send the other ranks' slices of this row, then its sum of squares
+      // the other ranks' slices of this row, then its sum of squares, into
+      // this rank's outgoing buffers (the layout of a receive slot), each
+      // then sent by one bulk copy
+      uint8_t* out = recv + 3 * slot_bytes;
 #pragma unroll 1
       for (uint32_t o = 0; o < kCluster; ++o) {
         if (o == rank) continue;
-        const uint32_t base =
-            map_rank(smem_u32(recv + recv_slot(rank, o) * slot_bytes + row * 16), o);
-        const uint32_t rbar = map_rank(smem_u32(red_full), o);
+        uint8_t* dst = out + ((o - rank - 1u) & 3u) * slot_bytes + row * 16;
 #pragma unroll 1
         for (int j = 0; j < W / 8; ++j) {
           float v[8];
@@ -291,10 +293,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tmem_ld<8>(taddr + o * W + 8 * j, v);
           }
-          st_async16(base + (2 * j) * (kBM * 16), v[0], v[1], v[2], v[3], rbar);
-          st_async16(base + (2 * j + 1) * (kBM * 16), v[4], v[5], v[6], v[7], rbar);
+          *reinterpret_cast<float4*>(dst + (2 * j) * (kBM * 16)) = make_float4(v[0], v[1], v[2], v[3]);
+          *reinterpret_cast<float4*>(dst + (2 * j + 1) * (kBM * 16)) =
+              make_float4(v[4], v[5], v[6], v[7]);
         }
-        st_async16(base + nchunk * (kBM * 16), ss, 0.f, 0.f, 0.f, rbar);
+        *reinterpret_cast<float4*>(dst + nchunk * (kBM * 16)) = make_float4(ss, 0.f, 0.f, 0.f);
+      }
+      fence_proxy_async_smem();  // the generic writes above -> the bulk copies' reads
+      epi_bar();
+      if (threadIdx.x == 3 * 32) {
+        for (uint32_t o = 0; o < kCluster; ++o) {
+          if (o == rank) continue;
+          bulk_s2cluster(map_rank(smem_u32(recv + recv_slot(rank, o) * slot_bytes), o),
+                         out + ((o - rank - 1u) & 3u) * slot_bytes,
+                         static_cast<uint32_t>(slot_bytes), map_rank(smem_u32(red_full), o));
+        }
       }
       ok = epi_bar_and(mbar_wait(red_full, 0));
       if (ok) {
@@ -336,13 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!live || c0 >= p.nout || (!primary && c0 >= p.nq)) continue;
           const uint4 packed = pack8(sum);
           *reinterpret_cast<uint4*>(p.qkv + static_cast<size_t>(row) * p.nout + c0) = packed;
-          if (primary && c0 >= p.nq) {
+          if (primary && c0 >= p.nq && cbase >= 0) {
             // primary K / V columns: also into the cache slot of this position
             const int kvd = p.Hkv * p.D;
             const bool is_v = c0 >= p.nq + kvd;
-            const int64_t off = cache_offset(p, row, c0 - p.nq - (is_v ? kvd : 0));
-            if (off >= 0)
-              *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) + off) = packed;
+            const int c = c0 - p.nq - (is_v ? kvd : 0);
+            const int g = c / p.D;
+            const int64_t off =
+                cbase + static_cast<int64_t>(g) * p.block_size * p.D + (c - g * p.D);
+            *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) + off) = packed;
           }
         }
       } else if (lane == 0) {
