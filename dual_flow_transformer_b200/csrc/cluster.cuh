@@ -9,20 +9,24 @@
 namespace df {
 namespace cl {
 
-// Named barrier 1 over the 128 epilogue threads (warps 3-6).
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier 1 over a kernel's N epilogue threads (whole warps).
+template <int N = 128>
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
+}
 
 // The same barrier, ANDing a predicate over the epilogue threads, so that a
 // wait which gave up in one thread stops all of them together.
+template <int N = 128>
 __device__ __forceinline__ bool epi_bar_and(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "bar.red.and.pred po, 1, %2, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(static_cast<uint32_t>(v)), "n"(N)
       : "memory");
   return r != 0;
 }

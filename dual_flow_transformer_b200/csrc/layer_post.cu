@@ -42,17 +42,21 @@
 //   --- grid counter C: every column of h is stored
 //   P2  W_down: as P0 over K = F; the owner adds x_mid and the c coupling
 //       -> x_out
+// (Per-tile readiness flags in place of the two counters were measured
+// slower: each flag read is an L2 round trip of a microsecond or more while
+// the weight stream fills the memory system, and the tiles finish together.)
 // The activation tiles interleave the flows (sequence j's primary row at tile
 // row 2j, its auxiliary row at 2j + 1, by a [sequence][flow][K] tensor map),
 // so both rows of a sequence sit in neighbouring TMEM lanes of one warp and
 // the one-way b and c couplings are a warp shuffle from the primary lane.
 // Every cluster is resident (one CTA per SM, grid = 4 x the device's maximum
-// of co-resident 4-CTA clusters), so the grid counters cannot deadlock; every
-// wait is bounded.
-// Roles (224 threads): warp 0 weight producer, warp 1 MMA issuer (one thread,
+// of co-resident 4-CTA clusters), so the grid counters cannot deadlock;
+// every wait is bounded.
+// Roles (352 threads): warp 0 weight producer, warp 1 MMA issuer (one thread,
 // tcgen05.mma M = 128 into two 256-column TMEM accumulators), warp 2
-// activation producer, warps 3-6 epilogue (TMEM lane quarter = warp % 4,
-// thread = accumulator row).
+// activation producer, warps 3-10 epilogue (TMEM lane quarter = warp % 4,
+// thread = accumulator row; the two warps of a quarter take one half of the
+// columns each, so two epilogue warps share each SM sub-partition).
 // One 176 KB ring holds a k-block's activation tile and weight tile per
 // stage; its stage size follows the phase (5 stages of 32 KB for W_o and
 // W_down, 4 of 44 KB for gate/up), so every phase keeps the whole ring in
@@ -81,12 +85,13 @@ using namespace cl;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 224;
-constexpr int kEpiThreads = 128;  // the epilogue named barrier (cl::epi_bar) counts 128
+constexpr int kThreads = 352;
+constexpr int kEpiThreads = 256;                     // warps 3-10: two per TMEM lane quarter
 constexpr int kMaxStages = 8;                        // ring stages (barrier pairs)
 constexpr int kCluster = 4;                          // CTAs per cluster = K splits
 constexpr int kTileN = 128;                          // W_o / W_down columns per cluster
 constexpr int kSliceN = kTileN / kCluster;           // columns a rank owns: 32
+constexpr int kHalfN = kSliceN / 2;                  // of which one epilogue thread takes 16
 constexpr int kMaxHalf = 112;                        // SwiGLU output columns per tile
 constexpr int kXBytes = kBM * kBK * 2;               // 16 KB activation tile
 constexpr int kRecvSlotBytes = kBM * kSliceN * 4;    // one sender's slice: 16 KB
@@ -95,11 +100,13 @@ constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
 // the ring: 4 SwiGLU stages of 16 + 28 KB, or 5 W_o / W_down stages of 16 + 16 KB
 constexpr size_t kRingBytes = 4 * (kXBytes + 2 * kMaxHalf * kBK * 2);
-constexpr size_t kSmemBytes = 1024 + kRingBytes + kRecvBytes + kMaxHalf * 4 +
+constexpr size_t kSmemBytes = 1024 + kRingBytes + kRecvBytes + kMaxHalf * 4 + kBM * 4 +
                               512;                   // + barriers, fill counts, flags
 static_assert(kRingBytes % 1024 == 0 && kXBytes % 1024 == 0, "1024-byte swizzle alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// grid counters: CTAs past P0 (x_mid and the sums of squares stored), past
+// P1 (h stored), done
 enum { kCntA2 = 0, kCntC = 1, kCntExit = 2 };
 
 struct Gemm {
@@ -138,10 +145,10 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
-// 32 bf16 values written by other CTAs of this launch (read through L2).
-__device__ __forceinline__ void load_bf16x32_cg(const __nv_bfloat16* src, float (&v)[32]) {
+// 16 bf16 values written by other CTAs of this launch (read through L2).
+__device__ __forceinline__ void load_bf16x16_cg(const __nv_bfloat16* src, float (&v)[16]) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < 2; ++q) {
     uint32_t w[4];
     asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
@@ -190,7 +197,7 @@ __device__ __forceinline__ void k_range(const Gemm& g, int q, int rank, int& k0,
 // made visible (also to TMA reads of other CTAs) before one thread adds.
 __device__ __forceinline__ void arrive_count(int* cnt, int et) {
   fence_proxy_async_global();
-  epi_bar();
+  epi_bar<kEpiThreads>();
   if (et == 0) {
     __threadfence();
     atomicAdd(cnt, 1);
@@ -201,66 +208,71 @@ __device__ __forceinline__ void arrive_count(int* cnt, int et) {
 __device__ __forceinline__ bool epi_wait_count(const int* cnt, int target, int et,
                                                volatile int* flag) {
   if (et == 0) *flag = wait_count(cnt, target) ? 1 : 0;
-  epi_bar();
+  epi_bar<kEpiThreads>();
   const bool ok = *flag != 0;
-  epi_bar();
+  epi_bar<kEpiThreads>();
   return ok;
 }
 
-// Reduce-scatter of a split-K accumulator over the cluster (thread = row).
-// reduce_send writes the other ranks' 32-column slices of this thread's row
-// into their receive buffers and returns this rank's own slice in `own`; the
-// TMEM accumulator may be reused once it returns. `empty`: this rank had no
+// Reduce-scatter of a split-K accumulator over the cluster (thread = row and
+// column half). reduce_send writes the given 16-column half of the other
+// ranks' 32-column slices of this thread's row into their receive buffers and
+// returns the same half of this rank's own slice in `own`; the TMEM
+// accumulator may be reused once it returns. `empty`: this rank had no
 // k-blocks (its partial is 0). A receive slot is laid out [8 chunks of 4
 // columns][128 rows][16 bytes], so the 32 lanes of a warp (32 consecutive
 // rows) write, and later read, one contiguous 512-byte block per chunk.
-__device__ __forceinline__ void reduce_send(uint32_t taddr, bool empty, int row, uint32_t rank,
-                                            uint8_t* recv, uint64_t* red_full, float (&own)[32]) {
+__device__ __forceinline__ void reduce_send(uint32_t taddr, bool empty, int row, int half,
+                                            uint32_t rank, uint8_t* recv, uint64_t* red_full,
+                                            float (&own)[kHalfN]) {
 #pragma unroll 1
   for (uint32_t o = 0; o < kCluster; ++o) {
     if (o == rank) continue;
-    float v[32];
+    float v[kHalfN];
     if (empty) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      for (int i = 0; i < kHalfN; ++i) v[i] = 0.f;
     } else {
-      tmem_ld<32>(taddr + o * kSliceN, v);
+      tmem_ld<kHalfN>(taddr + o * kSliceN + half * kHalfN, v);
     }
-    const uint32_t base =
-        map_rank(smem_u32(recv + recv_slot(rank, o) * kRecvSlotBytes + row * 16), o);
+    const uint32_t base = map_rank(
+        smem_u32(recv + recv_slot(rank, o) * kRecvSlotBytes + (half * 4) * (kBM * 16) + row * 16),
+        o);
     const uint32_t rbar = map_rank(smem_u32(red_full), o);
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
+    for (int c = 0; c < 4; ++c)
       st_async16(base + c * (kBM * 16), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], rbar);
   }
   if (empty) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) own[i] = 0.f;
+    for (int i = 0; i < kHalfN; ++i) own[i] = 0.f;
   } else {
-    tmem_ld<32>(taddr + rank * kSliceN, own);
+    tmem_ld<kHalfN>(taddr + rank * kSliceN + half * kHalfN, own);
   }
 }
 
 // reduce_gather waits (phase `parity`) for the other ranks' slices and sums
-// the four in rank order into `sum`; false (for every epilogue thread) if the
-// wait gave up.
-__device__ __forceinline__ bool reduce_gather(int row, uint32_t rank, const uint8_t* recv,
-                                              uint64_t* red_full, uint32_t parity,
-                                              const float (&own)[32], float (&sum)[32]) {
+// the four in rank order into `sum` (this thread's half); false (for every
+// epilogue thread) if the wait gave up.
+__device__ __forceinline__ bool reduce_gather(int row, int half, uint32_t rank,
+                                              const uint8_t* recv, uint64_t* red_full,
+                                              uint32_t parity, const float (&own)[kHalfN],
+                                              float (&sum)[kHalfN]) {
   bool ok = mbar_wait(red_full, parity);
-  ok = epi_bar_and(ok);
+  ok = epi_bar_and<kEpiThreads>(ok);
   if (!ok) return false;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) sum[i] = 0.f;
+  for (int i = 0; i < kHalfN; ++i) sum[i] = 0.f;
 #pragma unroll 1
   for (uint32_t k = 0; k < kCluster; ++k) {
     if (k == rank) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) sum[i] += own[i];
+      for (int i = 0; i < kHalfN; ++i) sum[i] += own[i];
     } else {
-      const uint8_t* src = recv + recv_slot(k, rank) * kRecvSlotBytes + row * 16;
+      const uint8_t* src =
+          recv + recv_slot(k, rank) * kRecvSlotBytes + (half * 4) * (kBM * 16) + row * 16;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         const float4 v = *reinterpret_cast<const float4*>(src + c * (kBM * 16));
         sum[4 * c] += v.x;
         sum[4 * c + 1] += v.y;
@@ -272,21 +284,36 @@ __device__ __forceinline__ bool reduce_gather(int row, uint32_t rank, const uint
   return true;
 }
 
-// Row scale of this thread's row: 1 / sqrt(sum over the d/32 slices of their
-// sums of squares (slice order) / d + eps).
-__device__ float row_scale(const Params& p, int row) {
+// Row scale of this thread's row: 1 / sqrt(sum over the d/32 column slices of
+// their sums of squares / d + eps). The two threads of a row (one per column
+// half) sum one half of the slices each, in slice order, and the halves are
+// added in a fixed order (uniform call: every epilogue thread).
+__device__ float row_scale(const Params& p, int row, int tl, int half, bool live, float* red) {
   const int slices = p.d / kSliceN;
+  const int k0 = half * (slices / 2), k1 = half ? slices : slices / 2;
   float s = 0.f;
-  int k = 0;
-  for (; k + 16 <= slices; k += 16) {
-    float v[16];
+  if (live) {
+    int k = k0;
+    for (; k + 16 <= k1; k += 16) {
+      float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __ldcg(p.ss_part + static_cast<size_t>(k + i) * kBM + row);
+      for (int i = 0; i < 16; ++i)
+        v[i] = __ldcg(p.ss_part + static_cast<size_t>(k + i) * kBM + row);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s += v[i];
+      for (int i = 0; i < 16; ++i) s += v[i];
+    }
+    for (; k < k1; ++k) s += __ldcg(p.ss_part + static_cast<size_t>(k) * kBM + row);
   }
-  for (; k < slices; ++k) s += __ldcg(p.ss_part + static_cast<size_t>(k) * kBM + row);
-  return 1.0f / sqrtf(s / static_cast<float>(p.d) + p.eps);
+  if (half == 1) red[tl] = s;
+  epi_bar<kEpiThreads>();
+  float r = 0.f;
+  if (half == 0) r = 1.0f / sqrtf((s + red[tl]) / static_cast<float>(p.d) + p.eps);
+  epi_bar<kEpiThreads>();
+  if (half == 0) red[tl] = r;
+  epi_bar<kEpiThreads>();
+  r = red[tl];
+  epi_bar<kEpiThreads>();
+  return live ? r : 0.f;
 }
 
 // P1 epilogue of tile t: h[row][t*H + j] = SiLU(rs g) * (rs u) (+ b * primary
@@ -323,13 +350,15 @@ __device__ __forceinline__ void swiglu_chunk(const Params& p, uint32_t taddr, in
   }
 }
 
-__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int row, bool live,
-                                bool aux, float rs, const float* bsl) {
+// (this thread's half of the tile's H columns: H is a multiple of 16)
+__device__ void swiglu_epilogue(const Params& p, int t, uint32_t taddr, int row, int half,
+                                bool live, bool aux, float rs, const float* bsl) {
   const int H = p.g[1].half;
   const int col0 = t * H;
-  int c = 0;
-  for (; c + 32 <= H; c += 32) swiglu_chunk<32>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
-  for (; c < H; c += 8) swiglu_chunk<8>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
+  int c = half * (H / 2);
+  const int c1 = c + H / 2;
+  for (; c + 32 <= c1; c += 32) swiglu_chunk<32>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
+  for (; c < c1; c += 8) swiglu_chunk<8>(p, taddr, H, c, col0, row, live, aux, rs, bsl);
 }
 
 // Tile t's slice of the coupling vector b into shared memory (zeros past F),
@@ -340,7 +369,7 @@ __device__ void load_b_slice(const Params& p, int t, int et, float* bsl) {
     const int col = t * H + i;
     bsl[i] = (p.b != nullptr && col < p.F) ? __bfloat162float(p.b[col]) : 0.f;
   }
-  epi_bar();
+  epi_bar<kEpiThreads>();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -353,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* recv = smem + kRingBytes;                             // [3][8 chunks][128 rows][16 B]
   float* bsl = reinterpret_cast<float*>(recv + kRecvBytes);      // [kMaxHalf] b of a tile
-  uint64_t* full = reinterpret_cast<uint64_t*>(bsl + kMaxHalf);  // [kMaxStages]
+  float* red = bsl + kMaxHalf;  // [128]: one value per TMEM lane passed between the halves
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + kBM);       // [kMaxStages]
   uint64_t* empty = full + kMaxStages;                           // [kMaxStages]
   uint64_t* acc_full = empty + kMaxStages;                       // [2]
   uint64_t* acc_empty = acc_full + 2;                            // [2]
@@ -437,14 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        bool ready = wrole || q == 0;  // P0 reads the attention output: pdl_wait above
         int s = 0;
         const Units us = units_of(g, q, cta, cid, G);
         for (int u = us.first; u < g.units && ok; u += us.step) {
           int k0, k1;
           k_range(g, q, static_cast<int>(rank), k0, k1);
-          if (!ready && k1 > k0) {
-            // P1 reads x_mid (counter A2), P2 every column of h (C)
+          if (!wrole && q > 0 && k1 > k0) {
+            // P1 reads x_mid (counter A2), P2 every column of h (counter C)
             if (!wait_count(p.cnt + (q == 1 ? kCntA2 : kCntC), G)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
@@ -452,9 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             fence_proxy_async_global();
-            ready = true;
           }
-          for (int kb = k0; kb < k1; ++kb) {
+          for (int kb = k0; kb < k1 && ok; ++kb) {
             if (!mbar_wait(&empty[s], ((par >> s) & 1u) ^ 1u)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
@@ -540,8 +568,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
+    // Two warps per TMEM lane quarter (warps q + 3 and q + 7 take quarter
+    // (q + 3) % 4), each taking one half of the columns.
     const int quarter = warp & 3;
     const int et = threadIdx.x - 3 * 32;
+    const int half = et >> 7;
     // The activation tiles hold the rows interleaved, sequence j's primary
     // row at tile row 2j and its auxiliary row at 2j + 1: this thread's TMEM
     // lane tl is tile row tl, which is `row` of x / x_mid / h / x_out.
@@ -557,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // that all of them pass the same named barriers on every path)
     auto take_acc = [&](int acc, int sg) -> bool {
       const bool got = mbar_wait_warp(&acc_full[acc], static_cast<uint32_t>((sg >> 1) & 1));
-      return epi_bar_and(got);
+      return epi_bar_and<kEpiThreads>(got);
     };
     auto give_acc = [&](int acc) {
       tc_fence_before();
@@ -584,38 +615,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = seg & 1;
       int k0, k1;
       k_range(p.g[0], 0, static_cast<int>(rank), k0, k1);
-      const int col0 = cid * kTileN + static_cast<int>(rank) * kSliceN;
-      float res[32];  // residual, loaded while the MMAs run
+      const int slice = (cid * kCluster + static_cast<int>(rank)) * 2 + half;  // 16 columns
+      const int col0 = slice * kHalfN;
+      float res[kHalfN];  // residual, loaded while the MMAs run
       if (live) {
-        load_bf16<32>(p.x + static_cast<size_t>(row) * p.d + col0, res);
+        load_bf16<kHalfN>(p.x + static_cast<size_t>(row) * p.d + col0, res);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) res[i] = 0.f;
+        for (int i = 0; i < kHalfN; ++i) res[i] = 0.f;
       }
       if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
       if (!take_acc(acc, seg)) {
         fail();
       } else {
         tc_fence_after();
-        float own[32], sum[32];
-        reduce_send(acc_addr(acc), k1 == k0, tl, rank, recv, red_full, own);
+        float own[kHalfN], sum[kHalfN];
+        reduce_send(acc_addr(acc), k1 == k0, tl, half, rank, recv, red_full, own);
         give_acc(acc);
-        if (!reduce_gather(tl, rank, recv, red_full, 0, own, sum)) {
+        if (!reduce_gather(tl, half, rank, recv, red_full, 0, own, sum)) {
           fail();
         } else {
           float ss = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < kHalfN; ++i) {
             sum[i] = __bfloat162float(__float2bfloat16_rn(sum[i] + res[i]));
             ss = fmaf(sum[i], sum[i], ss);
           }
-          if (live) store_bf16<32>(p.x_mid + static_cast<size_t>(row) * p.d + col0, sum);
-          if (live) p.ss_part[static_cast<size_t>(cid * kCluster + rank) * kBM + row] = ss;
+          if (live) store_bf16<kHalfN>(p.x_mid + static_cast<size_t>(row) * p.d + col0, sum);
+          // the 32-column slice's sum of squares: this half's, then the other's
+          if (half == 1) red[tl] = ss;
+          epi_bar<kEpiThreads>();
+          if (half == 0 && live)
+            p.ss_part[static_cast<size_t>(slice >> 1) * kBM + row] = ss + red[tl];
         }
       }
       ++seg;
     }
-    ok = epi_bar_and(ok);
+    ok = epi_bar_and<kEpiThreads>(ok);
     arrive_count(p.cnt + kCntA2, et);
     // P1: SwiGLU tiles straight from TMEM
     float rs = 0.f;
@@ -628,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        rs = live ? row_scale(p, row) : 0.f;
+        rs = row_scale(p, row, tl, half, live, red);
         have_rs = true;
       }
       if (!take_acc(acc, seg)) {
@@ -636,56 +672,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      swiglu_epilogue(p, u, acc_addr(acc), row, live, aux, rs, bsl);
+      swiglu_epilogue(p, u, acc_addr(acc), row, half, live, aux, rs, bsl);
       give_acc(acc);
     }
-    ok = epi_bar_and(ok);
+    ok = epi_bar_and<kEpiThreads>(ok);
     arrive_count(p.cnt + kCntC, et);
     // P2: W_down tile `cid` over this rank's K quarter; reduce-scatter; x_out.
-    // (A rank without k-blocks sends at once: counter C orders its sends
-    // after the receivers' last use of P0's data, like everyone else's.)
+    // (Counter C orders this rank's sends after the receivers' last use of
+    // P0's data; a rank without k-blocks would otherwise send at once.)
     if (ok && cid < p.g[2].units && grid_wait(kCntC)) {
       const int acc = seg & 1;
       int k0, k1;
       k_range(p.g[2], 2, static_cast<int>(rank), k0, k1);
-      const int col0 = cid * kTileN + static_cast<int>(rank) * kSliceN;
+      const int col0 = ((cid * kCluster + static_cast<int>(rank)) * 2 + half) * kHalfN;
       // residual (x_mid, stored by other CTAs before counter A2) and coupling,
       // loaded while the MMAs run
-      float res[32], cc[32];
+      float res[kHalfN], cc[kHalfN];
       if (live) {
-        load_bf16x32_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
+        load_bf16x16_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) res[i] = 0.f;
+        for (int i = 0; i < kHalfN; ++i) res[i] = 0.f;
       }
       if (aux && live && p.c != nullptr) {
-        load_bf16<32>(p.c + col0, cc);
+        load_bf16<kHalfN>(p.c + col0, cc);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) cc[i] = 0.f;
+        for (int i = 0; i < kHalfN; ++i) cc[i] = 0.f;
       }
       if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
       if (!take_acc(acc, seg)) {
         fail();
       } else {
         tc_fence_after();
-        float own[32], sum[32];
-        reduce_send(acc_addr(acc), k1 == k0, tl, rank, recv, red_full, own);
+        float own[kHalfN], sum[kHalfN];
+        reduce_send(acc_addr(acc), k1 == k0, tl, half, rank, recv, red_full, own);
         give_acc(acc);
-        if (!reduce_gather(tl, rank, recv, red_full, 1, own, sum)) {
+        if (!reduce_gather(tl, half, rank, recv, red_full, 1, own, sum)) {
           fail();
         } else {
           if (p.c != nullptr) {
             // the primary row's sum from the neighbouring lane
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < kHalfN; ++i) {
               const float pv = __shfl_xor_sync(0xffffffffu, sum[i], 1);
               if (aux) sum[i] = fmaf(cc[i], pv, sum[i]);
             }
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sum[i] += res[i];
-          if (live) store_bf16<32>(p.x_out + static_cast<size_t>(row) * p.d + col0, sum);
+          for (int i = 0; i < kHalfN; ++i) sum[i] += res[i];
+          if (live) store_bf16<kHalfN>(p.x_out + static_cast<size_t>(row) * p.d + col0, sum);
         }
       }
       ++seg;
@@ -777,10 +813,10 @@ Plan make_plan(int M, int mp, int d, int qd, int F) {
   pl.T0 = d / kTileN;
   if (nc < 1 || pl.T0 > nc) return pl;  // one W_o / W_down tile per cluster
   pl.G = nc * kCluster;
-  // smallest multiple of 8 with at most G SwiGLU tiles (the MMA's N = 2 H
-  // steps by 16 at M = 128)
+  // smallest multiple of 16 with at most G SwiGLU tiles (two epilogue warps
+  // take 8-column multiples each; the MMA's N = 2 H steps by 16 at M = 128)
   int H = static_cast<int>(ceil_div(F, pl.G));
-  H = static_cast<int>(ceil_div(H, 8)) * 8;
+  H = static_cast<int>(ceil_div(H, 16)) * 16;
   if (H > kMaxHalf) return pl;
   pl.H1 = H;
   pl.T1 = static_cast<int>(ceil_div(F, H));

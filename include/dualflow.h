@@ -439,10 +439,11 @@ df_status dualflow_layer_pre_attention(const void* x, const void* w_qkv, int m_p
 /* launched ahead on the stream (programmatic dependent launch), so that     */
 /* kernel must not write them.                                               */
 /* workspace: >= dualflow_layer_post_attention_workspace_size(...) bytes     */
-/* (256 + d_model * 16), 256-byte aligned, ZERO-FILLED once: its first bytes */
-/* are grid counters that every completed call leaves at zero (after a       */
-/* DF_DEVERR_TIMEOUT, zero it again); the rest holds the row sums of squares */
-/* of the norm. Calls sharing one workspace must not overlap on the GPU.     */
+/* (256 + d_model * 16), 256-byte aligned, ZERO-FILLED once: its first 256  */
+/* bytes are grid counters that every completed call leaves at zero         */
+/* (after a DF_DEVERR_TIMEOUT, zero it again); the rest holds the row sums   */
+/* of squares of the norm. Calls sharing one workspace must not overlap on   */
+/* the GPU.                                                                  */
 /* Supported (else DF_ERR_UNSUPPORTED; the size query returns 0):            */
 /* 1 <= m_primary <= 64, d_model % 128 == 0 with d_model / 128 at most the   */
 /* number of 4-CTA clusters the device holds at once (33 on a 148-SM B200:   */
