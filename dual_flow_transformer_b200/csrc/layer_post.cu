@@ -57,12 +57,16 @@
 // activation producer, warps 3-10 epilogue (TMEM lane quarter = warp % 4,
 // thread = accumulator row; the two warps of a quarter take one half of the
 // columns each, so two epilogue warps share each SM sub-partition).
-// One 176 KB ring holds a k-block's activation tile and weight tile per
-// stage; its stage size follows the phase (5 stages of 32 KB for W_o and
-// W_down, 4 of 44 KB for gate/up), so every phase keeps the whole ring in
-// flight: at these loads the DRAM and L2 latency under full HBM traffic
-// (1.5-2 us) needs all of it. The producers drain the ring at each phase
-// boundary, where the MMAs wait for the phase before anyway. (L2 prefetches
+// One ring holds a k-block's activation tile and weight tile per stage; its
+// stage size follows the phase (5 stages of 32 KB for W_o in the low 176 KB,
+// 5 of 44 KB for gate/up and 7 of 32 KB for W_down over 224 KB, whose top
+// 48 KB is the W_o / W_down receive buffer when a reduction needs it), so
+// every phase keeps the ring in flight: at these loads the DRAM and L2
+// latency under full HBM traffic (1.5-2 us) needs all of it. The producers
+// drain the ring at each phase boundary, where the MMAs wait for the phase
+// before anyway; the gate/up stage in the top is filled once the W_o
+// reduction has consumed its slices and counter A2 is complete (more weight
+// traffic in flight delays the counter). (L2 prefetches
 // of the next phase's weights at a boundary were measured to delay the grid
 // counters behind them by more than they saved.)
 // Every split sum is taken in a fixed order: results are deterministic, and
@@ -98,11 +102,15 @@ constexpr int kRecvSlotBytes = kBM * kSliceN * 4;    // one sender's slice: 16 K
 constexpr int kRecvBytes = (kCluster - 1) * kRecvSlotBytes;
 constexpr int kCounters = 8;
 constexpr size_t kCounterBytes = 256;
-// the ring: 4 SwiGLU stages of 16 + 28 KB, or 5 W_o / W_down stages of 16 + 16 KB
-constexpr size_t kRingBytes = 4 * (kXBytes + 2 * kMaxHalf * kBK * 2);
-constexpr size_t kSmemBytes = 1024 + kRingBytes + kRecvBytes + kMaxHalf * 4 + kBM * 4 +
+// The ring: P0 uses its low 176 KB (5 stages of 16 + 16 KB); P1 and P2 also
+// the top 48 KB, which is the W_o / W_down receive buffer when a reduction
+// needs it (P1: 5 stages of 16 + 28 KB, P2: 7 of 16 + 16 KB).
+constexpr size_t kRingLow = 4 * (kXBytes + 2 * kMaxHalf * kBK * 2);
+constexpr size_t kRingBytes = kRingLow + kRecvBytes;
+constexpr size_t kSmemBytes = 1024 + kRingBytes + kMaxHalf * 4 + kBM * 4 +
                               512;                   // + barriers, fill counts, flags
-static_assert(kRingBytes % 1024 == 0 && kXBytes % 1024 == 0, "1024-byte swizzle alignment");
+static_assert(kRingLow % 1024 == 0 && kRingBytes % 1024 == 0 && kXBytes % 1024 == 0,
+              "1024-byte swizzle alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // grid counters: CTAs past P0 (x_mid and the sums of squares stored), past
@@ -380,8 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* recv = smem + kRingBytes;                             // [3][8 chunks][128 rows][16 B]
-  float* bsl = reinterpret_cast<float*>(recv + kRecvBytes);      // [kMaxHalf] b of a tile
+  uint8_t* recv = smem + kRingLow;  // [3][8 chunks][128 rows][16 B], the ring's top in P1 / P2
+  float* bsl = reinterpret_cast<float*>(smem + kRingBytes);      // [kMaxHalf] b of a tile
   float* red = bsl + kMaxHalf;  // [128]: one value per TMEM lane passed between the halves
   uint64_t* full = reinterpret_cast<uint64_t*>(red + kBM);       // [kMaxStages]
   uint64_t* empty = full + kMaxStages;                           // [kMaxStages]
@@ -389,10 +397,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;                            // [2]
   uint64_t* mma_done = acc_empty + 2;                            // [1]
   uint64_t* red_full = mma_done + 1;  // this rank's slices from the other 3 ranks have landed
-  int* wfills = reinterpret_cast<int*>(red_full + 1);  // [kMaxStages] fills per slot: weights
+  uint64_t* recv_free = red_full + 1;  // P0's received slices are consumed: P1 may use the top
+  int* wfills = reinterpret_cast<int*>(recv_free + 1);  // [kMaxStages] fills per slot: weights
   int* xfills = wfills + kMaxStages;                     // [kMaxStages] activation tiles
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfills + kMaxStages);
-  // [0] abort, [1] epilogue broadcast
+  // [0] abort, [1] epilogue broadcast, [2] counter A2 seen by the activation producer
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -413,8 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(red_full, 1);  // this rank's expect_tx arrival + the senders' bytes
+    mbar_init(recv_free, 1);
     flags[0] = 0;
     flags[1] = 0;
+    flags[2] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -451,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = wrole ? l2_policy_evict_first() : l2_policy_evict_last();
       int* fills = wrole ? wfills : xfills;
       uint32_t par = 0;  // bit i: parity of this producer's fills of slot i
+      bool recv_ok = false;
       bool ok = true;
       for (int q = 0; q < 3 && ok; ++q) {
         const Gemm& g = p.g[q];
@@ -481,8 +493,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             fence_proxy_async_global();
+            if (q == 1) flags[2] = 1;  // counter A2 seen (see the weight producer)
           }
           for (int kb = k0; kb < k1 && ok; ++kb) {
+            if (!recv_ok && static_cast<size_t>(s + 1) * g.stage > kRingLow) {
+              // this slot reaches into the receive buffer: wait until this
+              // CTA's epilogue has consumed P0's received slices, and (the
+              // weights) until counter A2 is complete, so that the extra
+              // stage does not add to the traffic the counter waits behind
+              if (wrole && q == 1) {
+                const long long t0 = clock64();
+                while (flags[2] == 0) {
+                  if (clock64() - t0 > kWaitLimitCycles) {
+                    set_err(p.err, DF_DEVERR_TIMEOUT);
+                    flags[0] = 1;
+                    break;
+                  }
+                  __nanosleep(64);
+                }
+                if (flags[0]) {
+                  ok = false;
+                  break;
+                }
+              }
+              if (!mbar_wait(recv_free, 0)) {
+                set_err(p.err, DF_DEVERR_TIMEOUT);
+                flags[0] = 1;
+                ok = false;
+                break;
+              }
+              recv_ok = true;
+            }
             if (!mbar_wait(&empty[s], ((par >> s) & 1u) ^ 1u)) {
               set_err(p.err, DF_DEVERR_TIMEOUT);
               flags[0] = 1;
@@ -515,6 +556,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (wrole) pdl_trigger();
     }
+    // P2's reduction may write into this CTA's ring once every role of every
+    // rank is done with it (the epilogue meets this barrier after P2's MMAs)
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -566,6 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(mma_done);
       mbar_wait(mma_done, 0);
     }
+    tc_fence_before();
+    cluster_sync();  // the ring retires (see the producers)
+    tc_fence_after();
   } else {
     // ------------------------------------------------------------ epilogue warps
     // Two warps per TMEM lane quarter (warps q + 3 and q + 7 take quarter
@@ -652,6 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++seg;
     }
     ok = epi_bar_and<kEpiThreads>(ok);
+    if (et == 0) mbar_arrive(recv_free);  // every epilogue thread is done with recv
     arrive_count(p.cnt + kCntA2, et);
     // P1: SwiGLU tiles straight from TMEM
     float rs = 0.f;
@@ -680,14 +730,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P2: W_down tile `cid` over this rank's K quarter; reduce-scatter; x_out.
     // (Counter C orders this rank's sends after the receivers' last use of
     // P0's data; a rank without k-blocks would otherwise send at once.)
-    if (ok && cid < p.g[2].units && grid_wait(kCntC)) {
-      const int acc = seg & 1;
+    const bool p2 = ok && cid < p.g[2].units && grid_wait(kCntC);
+    bool got = false;
+    float res[kHalfN], cc[kHalfN];
+    int col0 = 0;
+    const int acc2 = seg & 1;
+    if (p2) {
+      const int acc = acc2;
       int k0, k1;
       k_range(p.g[2], 2, static_cast<int>(rank), k0, k1);
-      const int col0 = ((cid * kCluster + static_cast<int>(rank)) * 2 + half) * kHalfN;
+      col0 = ((cid * kCluster + static_cast<int>(rank)) * 2 + half) * kHalfN;
       // residual (x_mid, stored by other CTAs before counter A2) and coupling,
       // loaded while the MMAs run
-      float res[kHalfN], cc[kHalfN];
       if (live) {
         load_bf16x16_cg(p.x_mid + static_cast<size_t>(row) * p.d + col0, res);
       } else {
@@ -701,10 +755,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kHalfN; ++i) cc[i] = 0.f;
       }
       if (et == 0) mbar_arrive_expect_tx(red_full, kRecvBytes);
-      if (!take_acc(acc, seg)) {
-        fail();
-      } else {
-        tc_fence_after();
+      got = take_acc(acc, seg);
+      if (!got) fail();
+    }
+    // every role of every rank of the cluster is done with its ring (the
+    // receive buffer is its top in P2)
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (p2 && got) {
+      const int acc = acc2;
+      int k0, k1;
+      k_range(p.g[2], 2, static_cast<int>(rank), k0, k1);
+      {
         float own[kHalfN], sum[kHalfN];
         reduce_send(acc_addr(acc), k1 == k0, tl, half, rank, recv, red_full, own);
         give_acc(acc);
@@ -827,7 +890,7 @@ Plan make_plan(int M, int mp, int d, int qd, int F) {
 // A phase's GEMM: MMA N = BN (weight rows per k-block), ring stages of the
 // activation tile plus BN x 64 weights, as many as the ring holds (at most
 // kMaxStages).
-Gemm ring_gemm(int units, int kblocks, int BN, int half) {
+Gemm ring_gemm(int units, int kblocks, int BN, int half, size_t ring_bytes) {
   Gemm g{};
   g.units = units;
   g.kblocks = kblocks;
@@ -835,7 +898,7 @@ Gemm ring_gemm(int units, int kblocks, int BN, int half) {
   g.half = half;
   g.w_bytes = BN * kBK * 2;
   g.stage = static_cast<int>(round_up(static_cast<size_t>(kXBytes + g.w_bytes), 1024));
-  g.nst = static_cast<int>(kRingBytes / static_cast<size_t>(g.stage));
+  g.nst = static_cast<int>(ring_bytes / static_cast<size_t>(g.stage));
   if (g.nst > kMaxStages) g.nst = kMaxStages;
   g.idesc = make_idesc(kBM, BN);
   return g;
@@ -882,9 +945,9 @@ extern "C" df_status dualflow_layer_post_attention(
   p.qd = q_dim;
   p.F = F;
   p.eps = eps;
-  p.g[0] = ring_gemm(pl.T0, q_dim / kBK, kTileN, 0);
-  p.g[1] = ring_gemm(pl.T1, d_model / kBK, 2 * pl.H1, pl.H1);
-  p.g[2] = ring_gemm(pl.T0, F / kBK, kTileN, 0);
+  p.g[0] = ring_gemm(pl.T0, q_dim / kBK, kTileN, 0, kRingLow);
+  p.g[1] = ring_gemm(pl.T1, d_model / kBK, 2 * pl.H1, pl.H1, kRingBytes);
+  p.g[2] = ring_gemm(pl.T0, F / kBK, kTileN, 0, kRingBytes);
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.b = static_cast<const __nv_bfloat16*>(b);
   p.c = static_cast<const __nv_bfloat16*>(c);
