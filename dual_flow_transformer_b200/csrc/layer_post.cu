@@ -117,6 +117,10 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // P1 (h stored), done
 enum { kCntA2 = 0, kCntC = 1, kCntExit = 2 };
 
+// Weight stages filled before counter A2 (gate/up) and C (W_down) is seen.
+constexpr int kEarlyGateUpStages = 4;
+constexpr int kEarlyDownStages = 7;
+
 struct Gemm {
   int units;    // P0 / P2: column tiles (one per cluster); P1: SwiGLU tiles
   int kblocks;  // 64-wide K blocks of the whole product
@@ -141,6 +145,7 @@ struct Params {
   float* ss_part;  // [d / 32 slices][128 rows] sums of squares of stored x_mid values
   int* cnt;        // [kCounters]
   int32_t* err;
+  int early[3];    // weight stages of phase q filled before its grid counter is complete
 };
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -401,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* wfills = reinterpret_cast<int*>(recv_free + 1);  // [kMaxStages] fills per slot: weights
   int* xfills = wfills + kMaxStages;                     // [kMaxStages] activation tiles
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfills + kMaxStages);
-  // [0] abort, [1] epilogue broadcast, [2] counter A2 seen by the activation producer
+  // [0] abort, [1] epilogue broadcast, [2] / [3] counter A2 / C seen by the
+  // activation producer
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -426,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
+    flags[3] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -480,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         int s = 0;
+        int fills_q = 0;  // this producer's fills in this phase
         const Units us = units_of(g, q, cta, cid, G);
         for (int u = us.first; u < g.units && ok; u += us.step) {
           int k0, k1;
@@ -493,29 +501,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             fence_proxy_async_global();
-            if (q == 1) flags[2] = 1;  // counter A2 seen (see the weight producer)
+            flags[1 + q] = 1;  // counter A2 / C seen (see the weight producer)
           }
           for (int kb = k0; kb < k1 && ok; ++kb) {
+            if (wrole && q > 0 && fills_q == p.early[q]) {
+              // Weight traffic in flight delays the grid counter the phase's
+              // activations wait for: beyond p.early[q] stages, wait until
+              // the activation producer has seen it (counter A2 / C).
+              const long long t0 = clock64();
+              while (flags[1 + q] == 0 && !flags[0]) {
+                if (clock64() - t0 > kWaitLimitCycles) {
+                  set_err(p.err, DF_DEVERR_TIMEOUT);
+                  flags[0] = 1;
+                }
+                __nanosleep(64);
+              }
+              if (flags[0]) {
+                ok = false;
+                break;
+              }
+            }
             if (!recv_ok && static_cast<size_t>(s + 1) * g.stage > kRingLow) {
               // this slot reaches into the receive buffer: wait until this
-              // CTA's epilogue has consumed P0's received slices, and (the
-              // weights) until counter A2 is complete, so that the extra
-              // stage does not add to the traffic the counter waits behind
-              if (wrole && q == 1) {
-                const long long t0 = clock64();
-                while (flags[2] == 0) {
-                  if (clock64() - t0 > kWaitLimitCycles) {
-                    set_err(p.err, DF_DEVERR_TIMEOUT);
-                    flags[0] = 1;
-                    break;
-                  }
-                  __nanosleep(64);
-                }
-                if (flags[0]) {
-                  ok = false;
-                  break;
-                }
-              }
+              // CTA's epilogue has consumed P0's received slices
               if (!mbar_wait(recv_free, 0)) {
                 set_err(p.err, DF_DEVERR_TIMEOUT);
                 flags[0] = 1;
@@ -549,6 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d_hint(st, tm, &full[s], kb * kBK, 0, 0, pol);
             }
             ++fills[s];
+            ++fills_q;
             par ^= 1u << s;
             if (++s == g.nst) s = 0;
           }
@@ -958,6 +967,9 @@ extern "C" df_status dualflow_layer_post_attention(
   p.cnt = reinterpret_cast<int*>(w8);
   p.ss_part = reinterpret_cast<float*>(w8 + kCounterBytes);
   p.err = err_flag;
+  p.early[0] = 0;                    // (P0 waits for no counter)
+  p.early[1] = kEarlyGateUpStages;
+  p.early[2] = kEarlyDownStages;
 
   CUtensorMap tmXo, tmWo, tmXg, tmWg, tmXd, tmWd;
   const uint64_t du = static_cast<uint64_t>(d_model),
