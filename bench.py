@@ -62,6 +62,10 @@ def parse_args(argv=None):
     ap.add_argument("--fused-pre", type=int, choices=[0, 1], default=None,
                     help="layer workload: 1 = norm, QKV and the append as one launch, "
                          "0 = three launches (default: the layer's own default)")
+    ap.add_argument("--split-pre", type=int, choices=[0, 1], default=None,
+                    help="layer workload, with the one-launch pre-attention half: 1 = it "
+                         "stores fp32 partial products that the attention launch reduces, "
+                         "0 = it reduces them itself (default: the layer's own default)")
     ap.add_argument("--fused-post", type=int, choices=[0, 1], default=None,
                     help="layer workload: 1 = the post-attention half as one persistent launch, "
                          "0 = four launches (default: the layer's own default)")
@@ -286,6 +290,8 @@ class LayerRun:
         kw = {} if args.fused_post is None else {"fused_post": bool(args.fused_post)}
         if args.fused_pre is not None:
             kw["fused_pre"] = bool(args.fused_pre)
+        if args.split_pre is not None:
+            kw["split_pre"] = bool(args.split_pre)
         self.layer = DualFlowLayer(W, w.Hq, w.Hkv, w.D, w.F, w.B, w.cache_len + 1, device=dev,
                                    num_splits=args.num_splits, **kw)
         self.X = torch.cat([d["x1"], d["x2"]]).contiguous()
@@ -306,8 +312,9 @@ class LayerRun:
                                    % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
                        "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
                        "attended": L, "attn_launches": self.layer.attn_launches,
-                       "pre_attention": "one launch" if self.layer.fused_pre
-                                        else "three launches",
+                       "pre_attention": ("one launch, reduced in the attention launch"
+                                         if self.layer.split_pre else "one launch")
+                                        if self.layer.fused_pre else "three launches",
                        "post_attention": "one persistent launch" if self.layer.fused_post
                                          else "four launches",
                        "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"

@@ -103,6 +103,16 @@ SIGNATURES = {
         _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,  # x, w_qkv, m, d, Hq, Hkv, D
         _c_float, _vp, _vp, _vp, _vp, _c_int, _vp,         # eps, qkv, caches, table, mbps, pos
         _c_int, _c_int, _vp, _vp]),                        # block_size, num_blocks, err, stream
+    "dualflow_layer_qkv_partials": (_c_int, [
+        _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,  # x, w_qkv, m, d, Hq, Hkv, D
+        _vp, _vp, _vp, _vp]),                              # part, ss_part, err, stream
+    "dualflow_decode_attn_qkv_partials": (_c_int, [
+        _vp, _vp, _c_int, _c_int, _c_int, _c_float,  # part, ss_part, parts, m, d_model, eps
+        _vp, _vp, _vp, _vp, _c_int,          # a, k_cache, v_cache, block_table, mbps
+        _vp, _c_int, _vp, _vp, _c_i64,       # seqlens, max_seqlen, o1, o2, o_stride_b
+        _c_int, _c_int, _c_int, _c_int, _c_int,  # Hq, Hkv, D, block_size, num_blocks
+        _c_float, _c_int,                    # scale, num_splits
+        _vp, _c_size, _vp, _vp]),            # workspace, bytes, err_flag, stream
     "dualflow_layer_post_attention_workspace_size": (_c_size, [_c_int] * 4),
     "dualflow_layer_post_attention": (_c_int, [
         _vp, _vp, _vp, _vp, _vp, _vp, _vp,  # attn, x, w_o, w_gu, w_down, b, c

@@ -442,6 +442,76 @@ def layer_pre_attention(x, w_qkv, Hq, Hkv, k_cache, v_cache, block_table, positi
     return qkv
 
 
+def layer_qkv_partials(x, w_qkv, Hq, Hkv, D, *, part=None, ss_part=None, err_flag=None,
+                       stream=None):
+    """fp32 QKV partial products of the 4 quarters of d_model and the
+    quarters' row sums of squares, one launch: returns (part [4, 2m, N],
+    ss_part [4, 2m]). Summed in quarter order and scaled by the RMSNorm row
+    scale they give layer_pre_attention's qkv bit for bit."""
+    M, d_model = x.shape
+    nout = (Hq + 2 * Hkv) * D
+    for t in (x, w_qkv):
+        if not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("bf16 contiguous tensors required")
+    if M % 2 or tuple(w_qkv.shape) != (nout, d_model):
+        raise ValueError("shape mismatch")
+    if part is None:
+        part = torch.empty((4, M, nout), dtype=torch.float32, device=x.device)
+    if ss_part is None:
+        ss_part = torch.empty((4, M), dtype=torch.float32, device=x.device)
+    if tuple(part.shape) != (4, M, nout) or tuple(ss_part.shape) != (4, M) or \
+            part.dtype != torch.float32 or ss_part.dtype != torch.float32 or \
+            not part.is_contiguous() or not ss_part.is_contiguous():
+        raise ValueError("part must be fp32 [4, 2m, N] and ss_part fp32 [4, 2m], contiguous")
+    st = _lib().dualflow_layer_qkv_partials(
+        _ptr(x), _ptr(w_qkv), M // 2, d_model, int(Hq), int(Hkv), int(D), _ptr(part),
+        _ptr(ss_part), _ptr(err_flag), _stream(stream))
+    L.check("dualflow_layer_qkv_partials", st)
+    return part, ss_part
+
+
+def decode_attn_qkv_partials(part, ss_part, d_model, a, k_cache, v_cache, block_table, seqlens,
+                             max_seqlen, Hq, *, eps=1e-5, o1=None, o2=None, dual=True, scale=0.0,
+                             num_splits=0, workspace=None, err_flag=None, stream=None):
+    """Decode attention whose Q1 / Q2raw rows and appended K / V row are built
+    in its prologue from layer_qkv_partials' output; returns (o1, o2).
+    Equal bit for bit to layer_pre_attention (positions = seqlens - 1)
+    followed by decode_attn. dual=False: primary-only (o2 None)."""
+    parts, M, nout = part.shape
+    mp = M // 2
+    num_blocks, Hkv, bs, D = k_cache.shape
+    if M % 2 or nout != (Hq + 2 * Hkv) * D or tuple(ss_part.shape) != (parts, M):
+        raise ValueError("shape mismatch")
+    if part.dtype != torch.float32 or ss_part.dtype != torch.float32 or \
+            not part.is_contiguous() or not ss_part.is_contiguous():
+        raise ValueError("fp32 contiguous partials required")
+    if k_cache.dtype != torch.bfloat16 or v_cache.shape != k_cache.shape or \
+            not (k_cache.is_contiguous() and v_cache.is_contiguous() and
+                 block_table.is_contiguous()):
+        raise ValueError("bf16 contiguous caches and block table required")
+    dev = part.device
+    if o1 is None:
+        o1 = torch.empty((mp, Hq, D), dtype=torch.bfloat16, device=dev)
+    if dual and o2 is None:
+        o2 = torch.empty((mp, Hq, D), dtype=torch.bfloat16, device=dev)
+    if not dual:
+        o2 = None
+    for o in (o1, o2):
+        if o is not None and (not _heads_view_ok(o, Hq, D) or o.stride(0) != o1.stride(0)):
+            raise ValueError("outputs must be [m, Hq, D] with contiguous heads and equal strides")
+    if workspace is None:
+        workspace = new_attn_workspace(mp, Hq, Hkv, D, max_seqlen, num_splits, dev)
+    st = _lib().dualflow_decode_attn_qkv_partials(
+        _ptr(part), _ptr(ss_part), parts, mp, int(d_model), float(eps), _ptr(a), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_table), block_table.shape[1], _ptr(seqlens), int(max_seqlen),
+        _ptr(o1), _ptr(o2), o1.stride(0), int(Hq), Hkv, D, bs, num_blocks, float(scale),
+        int(num_splits), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    L.check("dualflow_decode_attn_qkv_partials", st)
+    return o1, o2
+
+
 def layer_post_attention_workspace_size(m_primary, d_model, q_dim, F) -> int:
     return _lib().dualflow_layer_post_attention_workspace_size(int(m_primary), int(d_model),
                                                                int(q_dim), int(F))

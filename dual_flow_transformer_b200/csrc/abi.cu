@@ -70,6 +70,21 @@ bool encode_tmap_bf16_3d_box(CUtensorMap* map, const void* base, const uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_f32_3d_box(CUtensorMap* map, const void* base, const uint64_t dims[3],
+                            const uint64_t strides_bytes[2], const uint32_t box[3]) {
+  std::call_once(g_encode_once, load_encode);
+  if (!g_encode) return false;
+  cuuint64_t gdims[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t gstrides[2] = {strides_bytes[0], strides_bytes[1]};
+  cuuint32_t gbox[3] = {box[0], box[1], box[2]};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), gdims,
+                        gstrides, gbox, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
   static int cached[64] = {0};
   int dev = 0;

@@ -76,12 +76,49 @@ struct Params {
   int dual;          // auxiliary rows computed
   int write1;        // store O1
   int write2;        // store O2
+  // Partials mode (qpart != nullptr; bf16 kernel): Q1, Q2raw and this
+  // step's K / V rows are not read from memory but built in the prologue
+  // from qparts fp32 partial products [part][row][column] of the QKV
+  // projection (row b primary, qmp + b auxiliary; columns: Q of head h at
+  // h D, K of KV head g at qkcol + g D, V at qvcol + g D) and the parts'
+  // row sums of squares qss [part][row]: with r = 1 / sqrt(sum qss / qd +
+  // qeps), each value is bf16(r (sum of the parts in part order)); K and V
+  // are appended to the cache at position seqlens[b] - 1 before its page is
+  // read.
+  const float* qpart;
+  const float* qss;
+  int qparts, qmp, qd, qkcol, qvcol;
+  int64_t qrow;   // floats between rows
+  int64_t qpstr;  // floats between parts
+  float qeps;
 };
 
 struct Plan {
   int splits;
   int chunk_pages;
 };
+
+// Partials mode: most partial products a call may sum (the QKV partials
+// launch writes 4, one per quarter of d_model).
+constexpr int kMaxParts = 4;
+
+__device__ __forceinline__ float4 ldg_f4(const float* ptr) {
+  return *reinterpret_cast<const float4*>(ptr);
+}
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+__device__ __forceinline__ float4 f4_scale(float4 a, float r) {
+  return make_float4(a.x * r, a.y * r, a.z * r, a.w * r);
+}
+// 4 bf16 (round to nearest even) to an 8-byte-aligned address
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
 
 inline Plan make_plan(int B, int Hkv, int max_seqlen, int block_size, int requested) {
   const int max_pages = static_cast<int>(ceil_div(max_seqlen, block_size));
@@ -183,6 +220,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
   uint64_t* empty = full + STAGES;
   int* stage_valid = reinterpret_cast<int*>(empty + STAGES);
+  uint64_t* kv_ready = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes + 64);
+  __nv_bfloat16* q1s = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * kStageBytes + 128);
+  __nv_bfloat16* q2s = q1s + 4 * D;  // partials mode: this KV head's Q1 / Q2raw rows
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -201,11 +241,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   const int ntiles = pg1 - pg0;
 
+  // Partials mode: the CTA whose pages include this step's position writes
+  // its K / V rows into the cache (page append_pg, relative to pg0).
+  int append_pg = -1;
+  if (p.qpart != nullptr && p.seqlens[b] >= 1 && p.seqlens[b] - 1 < L) {
+    const int pg = (p.seqlens[b] - 1) / kPage;
+    if (pg >= pg0 && pg < pg1) append_pg = pg - pg0;
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kConsumerWarps);
     }
+    mbar_init(kv_ready, 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -232,6 +280,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           ++issued;
           continue;
         }
+        // this step's K / V row lands in this page first (partials mode)
+        if (i == append_pg && !mbar_wait(kv_ready, 0)) set_err(p.err, DF_DEVERR_TIMEOUT);
         stage_valid[st] = 1;
         mbar_arrive_expect_tx(&full[st], kStageBytes);
         const int row = (page * p.Hkv + g) * kPage;
@@ -256,11 +306,81 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int gid = lane >> 2, tq = lane & 3;
   const int G = p.G;
 
+  if (p.qpart != nullptr) {
+    // Partials mode prologue: this KV head's Q1 / Q2raw rows into shared
+    // memory, and (the CTA holding this step's page) its K / V row into the
+    // cache, while the producer already streams the other pages. Every load
+    // of a thread is issued before the first sum (one L2 round trip): thread
+    // ct owns 4 consecutive Q columns of both rows and, for ct < D / 2, 4 of
+    // the 2 D K / V columns.
+    const int ct = threadIdx.x;  // 0 .. 127
+    const int M = 2 * p.qmp;
+    const int hcol = g * G * D;
+    const bool has_q = 4 * ct < G * D;
+    const bool has_kv = append_pg >= 0 && 4 * ct < 2 * D;
+    const float* pr1 = p.qpart + static_cast<int64_t>(b) * p.qrow;
+    const float* pr2 = p.qpart + static_cast<int64_t>(p.qmp + b) * p.qrow;
+    const int kvi = 4 * ct, kvsel = kvi >= D ? 1 : 0, kvd = kvi - kvsel * D;
+    const int kvcol = (kvsel ? p.qvcol : p.qkcol) + g * D + kvd;
+    float4 v1[kMaxParts], v2[kMaxParts], vk[kMaxParts];
+    float ss1[kMaxParts], ss2[kMaxParts];
+#pragma unroll
+    for (int k = 0; k < kMaxParts; ++k) {
+      const bool pk = k < p.qparts;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      v1[k] = pk && has_q ? ldg_f4(pr1 + k * p.qpstr + hcol + 4 * ct) : z;
+      v2[k] = pk && has_q && p.dual ? ldg_f4(pr2 + k * p.qpstr + hcol + 4 * ct) : z;
+      vk[k] = pk && has_kv ? ldg_f4(pr1 + k * p.qpstr + kvcol) : z;
+      ss1[k] = pk ? p.qss[k * M + b] : 0.f;
+      ss2[k] = pk ? p.qss[k * M + p.qmp + b] : 0.f;
+    }
+    float s1 = 0.f, s2 = 0.f;
+    float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), a2 = a1, ak = a1;
+#pragma unroll
+    for (int k = 0; k < kMaxParts; ++k) {
+      if (k < p.qparts) {
+        s1 += ss1[k];
+        s2 += ss2[k];
+        a1 = f4_add(a1, v1[k]);
+        a2 = f4_add(a2, v2[k]);
+        ak = f4_add(ak, vk[k]);
+      }
+    }
+    const float r1 = 1.0f / sqrtf(s1 / static_cast<float>(p.qd) + p.qeps);
+    const float r2 = 1.0f / sqrtf(s2 / static_cast<float>(p.qd) + p.qeps);
+    if (has_q) {
+      store_bf16x4(q1s + 4 * ct, f4_scale(a1, r1));
+      store_bf16x4(q2s + 4 * ct, f4_scale(a2, r2));
+    }
+    if (append_pg >= 0) {
+      const int pos = p.seqlens[b] - 1;
+      const int page = p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + pos / kPage];
+      if (page < 0 || page >= p.num_blocks) {
+        if (ct == 0) set_err(p.err, DF_DEVERR_BLOCK);
+      } else if (has_kv) {
+        const int64_t row = (static_cast<int64_t>(page) * p.Hkv + g) * kPage + pos % kPage;
+        __nv_bfloat16* cache =
+            static_cast<__nv_bfloat16*>(const_cast<void*>(kvsel ? p.v_cache : p.k_cache));
+        store_bf16x4(cache + row * D + kvd, f4_scale(ak, r1));
+      }
+      asm volatile("fence.proxy.async.global;" ::: "memory");  // -> the page's TMA load
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    if (ct == 0 && append_pg >= 0) {
+      __threadfence();
+      mbar_arrive(kv_ready);
+    }
+  }
+
   // Q fragments (A operand of Q K^T): rows gid and gid + 8 of the 16-row tile.
   uint32_t qa[KS][4];
   {
-    const __nv_bfloat16* q1 = static_cast<const __nv_bfloat16*>(p.q1) + b * p.q_stride_b;
-    const __nv_bfloat16* q2 = static_cast<const __nv_bfloat16*>(p.q2raw) + b * p.q_stride_b;
+    // (q1 / q2: this KV head's G rows, in shared memory in partials mode)
+    const bool own = p.qpart != nullptr;
+    const __nv_bfloat16* q1 =
+        own ? q1s : static_cast<const __nv_bfloat16*>(p.q1) + b * p.q_stride_b + g * G * D;
+    const __nv_bfloat16* q2 =
+        own ? q2s : static_cast<const __nv_bfloat16*>(p.q2raw) + b * p.q_stride_b + g * G * D;
     const __nv_bfloat16* av = static_cast<const __nv_bfloat16*>(p.a);
     const int j = gid & 3;
     const bool aux = gid >= 4;
@@ -276,11 +396,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int e = 0; e < 2; ++e) {
           __nv_bfloat16 top = __float2bfloat16_rn(0.f), bot = __float2bfloat16_rn(0.f);
           if (valid) {
-            const __nv_bfloat16 x1 = q1[h * D + d0 + e];
+            const __nv_bfloat16 x1 = q1[j * D + d0 + e];
             if (!aux) {
               top = x1;
             } else {
-              float q = __bfloat162float(q2[h * D + d0 + e]);
+              float q = __bfloat162float(q2[j * D + d0 + e]);
               if (av != nullptr) q = fmaf(__bfloat162float(av[h * D + d0 + e]), __bfloat162float(x1), q);
               split_bf16(q, top, bot);
             }
@@ -718,8 +838,9 @@ __global__ void __launch_bounds__(D) combine_kernel(const Params p) {
 
 template <int D>
 size_t bf16_smem_bytes() {
-  return 1024 + static_cast<size_t>(kStagesBf16) * 2 * kPage * D * 2 + 2 * kStagesBf16 * 8 +
-         kStagesBf16 * 4 + 64;
+  // ring | barriers, stage flags (64 B) | kv_ready (64 B) | Q1, Q2raw rows of
+  // one KV head (partials mode)
+  return 1024 + static_cast<size_t>(kStagesBf16) * 2 * kPage * D * 2 + 128 + 2 * 4 * D * 2;
 }
 
 template <int D>
@@ -801,7 +922,16 @@ extern "C" size_t dualflow_decode_attn_workspace_size(int B, int Hq, int Hkv, in
 
 namespace {
 
-// Both entry points: every argument check first, then (only for the no-alloc
+// Partials-mode source of Q1 / Q2raw and this step's K / V (see Params).
+struct QParts {
+  const float* part;
+  const float* ss;
+  int parts, mp, d, kcol, vcol;
+  int64_t row, pstr;
+  float eps;
+};
+
+// Every entry point: every argument check first, then (only for the no-alloc
 // entry point, clear_counters) the clearing of the bf16 arrival counters, then
 // the launch. A call rejected by a check has issued no device work.
 df_status decode_attn_impl(
@@ -810,10 +940,10 @@ df_status decode_attn_impl(
     const int32_t* seqlens, int max_seqlen, void* o1, void* o2, int64_t o_stride_b, int B, int Hq,
     int Hkv, int D, int block_size, int num_blocks, float scale, int dtype, int num_splits,
     void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream,
-    bool clear_counters) {
+    bool clear_counters, const QParts* qp = nullptr) {
   using namespace df;
-  if (!q1 || !k_cache || !v_cache || !block_table || !seqlens) return DF_ERR_NULL;
-  const bool want2 = (o2 != nullptr) && (q2raw != nullptr);
+  if ((!q1 && !qp) || !k_cache || !v_cache || !block_table || !seqlens) return DF_ERR_NULL;
+  const bool want2 = (o2 != nullptr) && (q2raw != nullptr || qp != nullptr);
   if (!o1 && !want2) return DF_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || num_blocks < 1 || max_blocks_per_seq < 1 ||
       max_seqlen < 1 || num_splits < 0)
@@ -833,7 +963,8 @@ df_status decode_attn_impl(
   if (qs < static_cast<int64_t>(Hq) * D || os < static_cast<int64_t>(Hq) * D) return DF_ERR_SHAPE;
   const uintptr_t esize = dtype == DF_BF16 ? 2 : 4;
   const uintptr_t qa_align = dtype == DF_BF16 ? 4 : 4;
-  if (!aligned(q1, qa_align) || (q2raw && !aligned(q2raw, qa_align)) || (a && !aligned(a, qa_align)) ||
+  if ((q1 && !aligned(q1, qa_align)) || (q2raw && !aligned(q2raw, qa_align)) ||
+      (a && !aligned(a, qa_align)) ||
       (o1 && !aligned(o1, esize)) || (o2 && !aligned(o2, esize)))
     return DF_ERR_ALIGN;
   if (dtype == DF_BF16 && (qs % 2 != 0)) return DF_ERR_ALIGN;
@@ -867,6 +998,19 @@ df_status decode_attn_impl(
   p.dual = want2 ? 1 : 0;
   p.write1 = o1 ? 1 : 0;
   p.write2 = want2 ? 1 : 0;
+  if (qp != nullptr) {
+    if (dtype != DF_BF16) return DF_ERR_UNSUPPORTED;
+    p.qpart = qp->part;
+    p.qss = qp->ss;
+    p.qparts = qp->parts;
+    p.qmp = qp->mp;
+    p.qd = qp->d;
+    p.qkcol = qp->kcol;
+    p.qvcol = qp->vcol;
+    p.qrow = qp->row;
+    p.qpstr = qp->pstr;
+    p.qeps = qp->eps;
+  }
   if (pl.splits > 1) {
     const attn::WsLayout l = attn::ws_layout(B, Hq, Hkv, D, pl.splits);
     if (!workspace || workspace_bytes < l.total() || !aligned(workspace, 256))
@@ -906,6 +1050,35 @@ extern "C" df_status dualflow_decode_attn(
                           max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, B, Hq, Hkv,
                           D, block_size, num_blocks, scale, dtype, num_splits, workspace,
                           workspace_bytes, err_flag, stream, false);
+}
+
+extern "C" df_status dualflow_decode_attn_qkv_partials(
+    const float* part, const float* ss_part, int parts, int m_primary, int d_model, float eps,
+    const void* a, const void* k_cache, const void* v_cache, const int32_t* block_table,
+    int max_blocks_per_seq, const int32_t* seqlens, int max_seqlen, void* o1, void* o2,
+    int64_t o_stride_b, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+    int num_splits, void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  using namespace df;
+  if (!part || !ss_part) return DF_ERR_NULL;
+  if (parts < 1 || parts > attn::kMaxParts || m_primary < 1 || d_model < 1 || !(eps >= 0.f) || Hq < 1 ||
+      Hkv < 1 || D < 1)
+    return DF_ERR_SHAPE;
+  if (!aligned(part, 16) || !aligned(ss_part, 4)) return DF_ERR_ALIGN;
+  QParts qp;
+  qp.part = part;
+  qp.ss = ss_part;
+  qp.parts = parts;
+  qp.mp = m_primary;
+  qp.d = d_model;
+  qp.kcol = Hq * D;
+  qp.vcol = (Hq + Hkv) * D;
+  qp.row = static_cast<int64_t>(Hq + 2 * Hkv) * D;
+  qp.pstr = 2 * static_cast<int64_t>(m_primary) * qp.row;
+  qp.eps = eps;
+  return decode_attn_impl(nullptr, nullptr, a, 0, k_cache, v_cache, block_table,
+                          max_blocks_per_seq, seqlens, max_seqlen, o1, o2, o_stride_b, m_primary,
+                          Hq, Hkv, D, block_size, num_blocks, scale, DF_BF16, num_splits,
+                          workspace, workspace_bytes, err_flag, stream, false, &qp);
 }
 
 // ------------------------------------------------------------------ no-alloc variant

@@ -38,6 +38,10 @@ bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t batch, uin
 bool encode_tmap_bf16_3d_box(CUtensorMap* map, const void* base, const uint64_t dims[3],
                              const uint64_t strides_bytes[2], const uint32_t box[3]);
 
+// The same for fp32 elements (box[0] * 4 bytes <= 128 with the swizzle).
+bool encode_tmap_f32_3d_box(CUtensorMap* map, const void* base, const uint64_t dims[3],
+                            const uint64_t strides_bytes[2], const uint32_t box[3]);
+
 // Opt `kernel` into `bytes` of dynamic shared memory on the current device.
 // The attribute belongs to the device, so it is set once per (kernel,
 // device) pair; later calls only look the pair up.

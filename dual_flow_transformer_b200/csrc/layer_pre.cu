@@ -75,6 +75,11 @@ struct Params {
   const int32_t* positions;
   int max_blocks, Hkv, D, block_size, num_blocks;
   int32_t* err;
+  // partials mode (part != nullptr): each rank stores its fp32 partial
+  // product [rank][row][column] and the first cluster each rank's row sums
+  // of squares ss_out [rank][row]; no reduction, no norm, no append here
+  float* part;
+  float* ss_out;
 };
 
 // Cache element offset of (sequence b, KV head 0, dimension 0) at b's
@@ -106,7 +111,7 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     pre_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-               const Params p) {
+               const __grid_constant__ CUtensorMap tmP, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // activation tiles in the ring (a row's 128 bytes in any chunk order)
     const int row = (warp & 3) * 32 + lane;
     // a primary row's cache slot, looked up while the MMAs run
-    const int64_t cbase = row < p.mp ? cache_row_base(p, row) : -1;
+    const int64_t cbase = (p.part == nullptr && row < p.mp) ? cache_row_base(p, row) : -1;
     float ss = 0.f;
     int s = 0;
     uint32_t ph = 0;
@@ -266,6 +271,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       set_err(p.err, DF_DEVERR_TIMEOUT);
       flags[0] = 1;
     }
+    if (p.part != nullptr) {
+      // Partials mode: this rank's fp32 partial product, staged in its own
+      // ring (retired: all its MMAs have completed) as boxes of 32 columns
+      // in the 128-byte-swizzled layout, then stored by TMA.
+      if (ok) {
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const bool empty_rank = k1 == k0;
+#pragma unroll 1
+        for (int j = 0; j < p.TN / 32; ++j) {
+          float v[32];
+          if (empty_rank) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          } else {
+            tmem_ld<32>(taddr + 32 * j, v);
+          }
+          uint8_t* box = smem + static_cast<size_t>(j) * (kBM * 128) + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(box + ((c ^ (row & 7)) * 16)) =
+                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
+        if (tile == 0 && row < p.M) p.ss_out[static_cast<size_t>(rank) * p.M + row] = ss;
+        fence_proxy_async_smem();  // the generic writes above -> the TMA stores' reads
+        epi_bar();
+        if (threadIdx.x == 3 * 32) {
+          for (int j = 0; j < p.TN / 32; ++j)
+            tma_store_3d(&tmP, smem + static_cast<size_t>(j) * (kBM * 128), tile * p.TN + 32 * j,
+                         0, static_cast<int>(rank));
+          bulk_commit_group();
+          bulk_wait_all();
+        }
+      }
+    } else {
     tc_fence_before();
     // every rank's ring is retired (all its MMAs have completed: the MMA
     // thread waited for them) before any rank writes into another's
@@ -364,8 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         set_err(p.err, DF_DEVERR_TIMEOUT);
       }
     }
+    }  // reduce mode
   }
-  if (warp < 3) {
+  if (warp < 3 && p.part == nullptr) {
     // the roles outside the epilogue meet the epilogue's cluster barrier
     tc_fence_before();
     cluster_sync();
@@ -468,6 +508,65 @@ extern "C" int dualflow_layer_pre_attention_supported(int m_primary, int d_model
   return df::pre::make_plan(m_primary, d_model, Hq, Hkv, D).ok ? 1 : 0;
 }
 
+namespace df {
+namespace pre {
+
+// Fills the shape fields of Params from the plan, encodes the tensor maps and
+// launches (tmP: the partials store map, or any valid map in reduce mode).
+df_status launch(Params& p, const Plan& pl, const void* x, const void* w_qkv, int m_primary,
+                 int d_model, void* stream) {
+  const int M = 2 * m_primary;
+  p.M = M;
+  p.mp = m_primary;
+  p.d = d_model;
+  p.nq = pl.nq;
+  p.nout = pl.nout;
+  p.TN = pl.TN;
+  p.kblocks = d_model / kBK;
+  p.w_bytes = pl.TN * kBK * 2;
+  p.stage = static_cast<int>(round_up(static_cast<size_t>(kXBytes + p.w_bytes), 1024));
+  p.nst = static_cast<int>(kRingBytes / static_cast<size_t>(p.stage));
+  if (p.nst > kMaxStages) p.nst = kMaxStages;
+  p.idesc = make_idesc(kBM, pl.TN);
+
+  CUtensorMap tmX, tmW, tmP;
+  const uint64_t du = static_cast<uint64_t>(d_model);
+  if (!encode_tmap_bf16_2d(&tmX, x, static_cast<uint64_t>(M), du, du * 2, kBM, kBK) ||
+      !encode_tmap_bf16_2d(&tmW, w_qkv, static_cast<uint64_t>(pl.nout), du, du * 2,
+                           static_cast<uint32_t>(pl.TN), kBK))
+    return DF_ERR_CUDA;
+  if (p.part != nullptr) {
+    // [rank][row][column] fp32, boxes of 32 columns x 128 rows of one rank
+    const uint64_t nout = static_cast<uint64_t>(pl.nout), Mu = static_cast<uint64_t>(M);
+    const uint64_t dims[3] = {nout, Mu, kCluster};
+    const uint64_t strides[2] = {nout * 4, Mu * nout * 4};
+    const uint32_t box[3] = {32, kBM, 1};
+    if (!encode_tmap_f32_3d_box(&tmP, p.part, dims, strides, box)) return DF_ERR_CUDA;
+  } else {
+    tmP = tmX;
+  }
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.T * kCluster);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, pre_kernel, tmX, tmW, tmP, p) != cudaSuccess) return DF_ERR_CUDA;
+  return DF_OK;
+}
+
+}  // namespace pre
+}  // namespace df
+
 extern "C" df_status dualflow_layer_pre_attention(
     const void* x, const void* w_qkv, int m_primary, int d_model, int Hq, int Hkv, int D,
     float eps, void* qkv, void* k_cache, void* v_cache, const int32_t* block_table,
@@ -485,21 +584,7 @@ extern "C" df_status dualflow_layer_pre_attention(
   const void* ptrs[] = {x, w_qkv, qkv, k_cache, v_cache};
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DF_ERR_ALIGN;
-  const int M = 2 * m_primary;
-
   Params p{};
-  p.M = M;
-  p.mp = m_primary;
-  p.d = d_model;
-  p.nq = pl.nq;
-  p.nout = pl.nout;
-  p.TN = pl.TN;
-  p.kblocks = d_model / kBK;
-  p.w_bytes = pl.TN * kBK * 2;
-  p.stage = static_cast<int>(round_up(static_cast<size_t>(kXBytes + p.w_bytes), 1024));
-  p.nst = static_cast<int>(kRingBytes / static_cast<size_t>(p.stage));
-  if (p.nst > kMaxStages) p.nst = kMaxStages;
-  p.idesc = make_idesc(kBM, pl.TN);
   p.eps = eps;
   p.qkv = static_cast<__nv_bfloat16*>(qkv);
   p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
@@ -512,28 +597,26 @@ extern "C" df_status dualflow_layer_pre_attention(
   p.block_size = block_size;
   p.num_blocks = num_blocks;
   p.err = err_flag;
+  return launch(p, pl, x, w_qkv, m_primary, d_model, stream);
+}
 
-  CUtensorMap tmX, tmW;
-  const uint64_t du = static_cast<uint64_t>(d_model);
-  if (!encode_tmap_bf16_2d(&tmX, x, static_cast<uint64_t>(M), du, du * 2, kBM, kBK) ||
-      !encode_tmap_bf16_2d(&tmW, w_qkv, static_cast<uint64_t>(pl.nout), du, du * 2,
-                           static_cast<uint32_t>(pl.TN), kBK))
-    return DF_ERR_CUDA;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.T * kCluster);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, pre_kernel, tmX, tmW, p) != cudaSuccess) return DF_ERR_CUDA;
-  return DF_OK;
+extern "C" df_status dualflow_layer_qkv_partials(const void* x, const void* w_qkv, int m_primary,
+                                                 int d_model, int Hq, int Hkv, int D, void* part,
+                                                 void* ss_part, int32_t* err_flag, void* stream) {
+  using namespace df;
+  using namespace df::pre;
+  if (!x || !w_qkv || !part || !ss_part) return DF_ERR_NULL;
+  if (m_primary < 1 || d_model < 1 || Hq < 1 || Hkv < 1 || D < 1) return DF_ERR_SHAPE;
+  const Plan pl = make_plan(m_primary, d_model, Hq, Hkv, D);
+  if (!pl.ok) return DF_ERR_UNSUPPORTED;
+  const void* ptrs[] = {x, w_qkv, part, ss_part};
+  for (const void* ptr : ptrs)
+    if (!aligned(ptr, 16)) return DF_ERR_ALIGN;
+  Params p{};
+  p.Hkv = Hkv;
+  p.D = D;
+  p.err = err_flag;
+  p.part = static_cast<float*>(part);
+  p.ss_out = static_cast<float*>(ss_part);
+  return launch(p, pl, x, w_qkv, m_primary, d_model, stream);
 }

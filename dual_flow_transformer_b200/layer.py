@@ -20,6 +20,13 @@ the QKV product along K and reduce it through distributed shared memory, the
 first norm's row scale multiplies the accumulator (the normalised rows are
 not stored) and the primary K/V columns go straight into the cache.
 fused_pre=False, or sizes the fused launch does not take, use the three calls.
+With split_pre=True (the default) the fused pre-attention launch stops short
+of the reduction (dualflow_layer_qkv_partials: fp32 partial products of the
+4 quarters of K and their row sums of squares) and the attention launch
+(dualflow_decode_attn_qkv_partials) sums, scales and rounds its KV head's
+query rows and appends the primary K/V row in its prologue: the same bits as
+the fused launch followed by dualflow_decode_attn, without the reduction's
+round trip between the cluster's shared memories on the critical path.
 
 By default (fused_post=True) steps 5-8 run as one persistent launch
 (dualflow_layer_post_attention) when the sizes allow it: its weight producers
@@ -46,7 +53,7 @@ from . import api
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
-                 num_splits=0, fused_pre=True, fused_post=True):
+                 num_splits=0, fused_pre=True, fused_post=True, split_pre=True):
         self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
         self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
         self.d_model = weights["w_o"].shape[0]
@@ -75,6 +82,11 @@ class DualFlowLayer:
         self.attn_launches = api.decode_attn_num_launches(B, Hkv, self.max_seqlen, num_splits)
         self.fused_pre = bool(fused_pre) and \
             api.layer_pre_attention_supported(B, self.d_model, Hq, Hkv, D)
+        self.split_pre = self.fused_pre and bool(split_pre)
+        self.qkv_part = (torch.empty(4, M, qd + 2 * kvd, dtype=torch.float32, device=dev)
+                         if self.split_pre else None)
+        self.ss_part = (torch.empty(4, M, dtype=torch.float32, device=dev)
+                        if self.split_pre else None)
         self.fused_post = bool(fused_post) and \
             api.layer_post_attention_workspace_size(B, self.d_model, qd, F) > 0
         self.post_ws = (api.new_post_attention_workspace(B, self.d_model, qd, F, dev)
@@ -162,7 +174,10 @@ class DualFlowLayer:
         # Each projection warms L2 with the first weight blocks of the next one
         # (o -> gate/up -> down -> the next step's QKV); none after the QKV
         # projection, whose successor is the HBM-bound attention.
-        if part == "pre" and self.fused_pre:
+        if part == "pre" and self.split_pre:
+            api.layer_qkv_partials(X, w["w_qkv"], Hq, Hkv, D, part=self.qkv_part,
+                                   ss_part=self.ss_part, err_flag=self.err, stream=stream)
+        elif part == "pre" and self.fused_pre:
             api.layer_pre_attention(X, w["w_qkv"], Hq, Hkv, k_cache, v_cache, block_table,
                                     positions, eps=self.eps, qkv=qkv, err_flag=self.err,
                                     stream=stream)
@@ -173,6 +188,12 @@ class DualFlowLayer:
             api.kv_append(qkv[:B, qd:qd + kvd].view(B, Hkv, D), qkv[:B, qd + kvd:].view(B, Hkv, D),
                           k_cache, v_cache, block_table, positions, err_flag=self.err,
                           stream=stream)
+        elif part == "attn" and self.split_pre:
+            api.decode_attn_qkv_partials(
+                self.qkv_part, self.ss_part, self.d_model, w["a"], k_cache, v_cache, block_table,
+                seqlens, self.max_seqlen, Hq, eps=self.eps, o1=self.attn[:B].view(B, Hq, D),
+                o2=self.attn[B:].view(B, Hq, D), num_splits=self.num_splits,
+                workspace=self.attn_ws, err_flag=self.err, stream=stream)
         elif part == "attn":
             api.decode_attn(qkv[:B, :qd].view(B, Hq, D), qkv[B:, :qd].view(B, Hq, D), w["a"],
                             k_cache, v_cache, block_table, seqlens, self.max_seqlen,

@@ -402,6 +402,66 @@ df_status dualflow_layer_pre_attention(const void* x, const void* w_qkv, int m_p
                                        void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Pre-attention half split across two launches: QKV partial products.       */
+/*                                                                           */
+/* Same operation as dualflow_layer_pre_attention (pages "Sintesi Tecnica",  */
+/* "Architettura Core" and "Costi di Inferenza"), but the split sums are     */
+/* not reduced here: this launch multiplies and stores, and                  */
+/* dualflow_decode_attn_qkv_partials (below) reduces, normalises, rounds     */
+/* and appends in its prologue, which removes the reduction's               */
+/* distributed-shared-memory round trip from the step. With M = 2 m_primary */
+/* and N = (Hq + 2 Hkv) D as in dualflow_layer_pre_attention:                */
+/*   part[k][row][n] = sum over K quarter k of x[row][j] w_qkv[n][j]  (fp32) */
+/*   ss_part[k][row] = sum over K quarter k of x[row][j]^2            (fp32) */
+/* for k = 0..3, the 4 quarters of d_model in order (a quarter past the end  */
+/* of K, when d_model / 64 < 4, holds zeros). All M rows and N columns are  */
+/* written. Summing the parts in order k = 0..3 from 0 and scaling by        */
+/* r = 1 / sqrt(sum_k ss_part[k][row] / d_model + eps) reproduces           */
+/* dualflow_layer_pre_attention's qkv bit for bit.                           */
+/*                                                                           */
+/* x, w_qkv : as dualflow_layer_pre_attention. part : fp32 [4][M][N],        */
+/* ss_part : fp32 [4][M], both 16-byte aligned, written completely; N * 4    */
+/* must be a multiple of 16 bytes (D % 8 == 0 guarantees it). w_qkv is read  */
+/* before the wait for the kernel launched ahead on the stream. Supported:   */
+/* as dualflow_layer_pre_attention_supported. One launch, no workspace.      */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_layer_qkv_partials(const void* x, const void* w_qkv, int m_primary,
+                                      int d_model, int Hq, int Hkv, int D, void* part,
+                                      void* ss_part, int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Dual-flow decode attention fed by QKV partial products.                   */
+/*                                                                           */
+/* Computes what dualflow_layer_pre_attention followed by                    */
+/* dualflow_decode_attn (bf16, q_stride_b = N, q2raw = the auxiliary rows'   */
+/* qkv) compute, with the same results bit for bit, in one launch: each CTA  */
+/* sums `parts` partial products in order, scales by the RMSNorm row scale   */
+/* and rounds to bf16 its KV head's Q1 and Q2raw rows (the pre-attention     */
+/* formulas above), and the CTA whose split holds position seqlens[b] - 1    */
+/* writes primary row b's K and V (same rounding) into that cache slot       */
+/* before its page is loaded; the other splits never read that slot.         */
+/*                                                                           */
+/* part, ss_part, parts : [parts][2 m_primary][(Hq + 2 Hkv) D] and           */
+/*            [parts][2 m_primary] fp32 as written by                        */
+/*            dualflow_layer_qkv_partials (parts = 4; 1..4 accepted);        */
+/*            row b primary, row m_primary + b auxiliary of sequence b.      */
+/*            16-byte and 4-byte aligned. d_model, eps: the norm's width     */
+/*            and epsilon.                                                   */
+/* The other arguments are dualflow_decode_attn's with B = m_primary and     */
+/* dtype bf16 (k_cache and v_cache are WRITTEN at the appended slot, so      */
+/* they must not be read by another kernel in flight). seqlens[b] counts the */
+/* appended token. An out-of-table page is skipped and flagged (             */
+/* DF_DEVERR_BLOCK), like a page the attention reads.                        */
+/* Supported: as dualflow_decode_attn (bf16). One launch.                    */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_decode_attn_qkv_partials(
+    const float* part, const float* ss_part, int parts, int m_primary, int d_model, float eps,
+    const void* a, const void* k_cache, const void* v_cache, const int32_t* block_table,
+    int max_blocks_per_seq, const int32_t* seqlens, int max_seqlen, void* o1, void* o2,
+    int64_t o_stride_b, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+    int num_splits, void* workspace, size_t workspace_bytes, int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Post-attention half of the decoder layer in ONE persistent launch.        */
 /*                                                                           */
 /* Pages "Sintesi Tecnica" ("Architettura Core": the flows share the output  */

@@ -18,14 +18,22 @@ SMALL = dataclasses.replace(synth.WORKLOADS["layer"], B=8, d_model=512, Hq=4, Hk
                             F=1024, cache_len=200, seed=50)
 
 
-def _run_gpu(inp, dev, num_splits=0, fused=False):
+MODES = ("split", "fused", "unfused")
+
+
+def _run_gpu(inp, dev, num_splits=0, mode="unfused"):
+    """mode: "split" (pre-attention partials reduced in the attention launch),
+    "fused" (one-launch pre- and post-attention halves), "unfused" (one call
+    per step of the layer)."""
+    fused = mode != "unfused"
     d = to_dev(inp, dev)
     w = {k: d[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
     B = inp["B"]
     layer = DualFlowLayer(w, inp["Hq"], inp["Hkv"], inp["D"], inp["F"], B,
                           int(inp["positions"].max()) + 1, device=dev, num_splits=num_splits,
-                          fused_pre=fused, fused_post=fused)
+                          fused_pre=fused, fused_post=fused, split_pre=mode == "split")
     assert layer.fused_pre == fused and layer.fused_post == fused
+    assert layer.split_pre == (mode == "split")
     X = torch.cat([d["x1"], d["x2"]]).contiguous()
     seqlens = (d["positions"] + 1).to(torch.int32)
     out = layer.step(X, d["k_cache"], d["v_cache"], d["block_table"], d["positions"], seqlens)
@@ -53,28 +61,28 @@ def _oracle(inp, rows=None, rounded=oracle.LAYER_INTERFACES):
     return r
 
 
-@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("coupled", [True, False])
-def test_layer_step_small(cuda_device, coupled, fused):
+def test_layer_step_small(cuda_device, coupled, mode):
     w = dataclasses.replace(SMALL, coupled_mlp=coupled)
     inp = synth.make_layer_inputs(w)
-    out, d, layer = _run_gpu(inp, cuda_device, fused=fused)
-    ref = _oracle(inp, rounded=FUSED_ROUNDED if fused else oracle.LAYER_INTERFACES)
+    out, d, layer = _run_gpu(inp, cuda_device, mode=mode)
+    ref = _oracle(inp, rounded=oracle.LAYER_INTERFACES if mode == "unfused" else FUSED_ROUNDED)
     assert_close(out, ref["x_out"], "bf16", "layer x_out")
     assert_close(layer.x_mid.cpu(), ref["x_mid"], "bf16", "layer x_mid")
     assert_close(layer.h.cpu(), ref["h"], "bf16", "layer h")
 
 
-@pytest.mark.parametrize("fused", [False, True])
-def test_layer_primary_flow_is_self_sufficient(cuda_device, fused):
+@pytest.mark.parametrize("mode", MODES)
+def test_layer_primary_flow_is_self_sufficient(cuda_device, mode):
     inp = synth.make_layer_inputs(SMALL)
-    out1, _, _ = _run_gpu(inp, cuda_device, fused=fused)
+    out1, _, _ = _run_gpu(inp, cuda_device, mode=mode)
     other = dict(inp)
     other["x2"] = inp["x2"] * 3
     other["a"] = -inp["a"]
     other["b"] = inp["b"] * 2
     other["c"] = -inp["c"]
-    out2, _, _ = _run_gpu(other, cuda_device, fused=fused)
+    out2, _, _ = _run_gpu(other, cuda_device, mode=mode)
     B = inp["B"]
     assert torch.equal(out1[:B].view(torch.int16), out2[:B].view(torch.int16))
 
@@ -94,16 +102,16 @@ def test_layer_append_writes_primary_rows_only(cuda_device):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("fused", [False, True])
-def test_layer_step_full_size_sampled(cuda_device, fused):
+@pytest.mark.parametrize("mode", MODES)
+def test_layer_step_full_size_sampled(cuda_device, mode):
     """The 4096/14336 layer, B = 64 per flow, cache 4096 + 1, in the launch
     configurations the benchmark can time; the oracle recomputes 17 of the 64
     sequences (every fourth and the last), both flows."""
     inp = synth.make_layer_inputs(synth.WORKLOADS["layer"])
-    out, _, _ = _run_gpu(inp, cuda_device, fused=fused)
+    out, _, _ = _run_gpu(inp, cuda_device, mode=mode)
     rows = list(range(0, 64, 4)) + [63]
-    ref = _oracle(inp, rows, rounded=FUSED_ROUNDED if fused else oracle.LAYER_INTERFACES)
+    ref = _oracle(inp, rows, rounded=oracle.LAYER_INTERFACES if mode == "unfused" else FUSED_ROUNDED)
     B = inp["B"]
     got = torch.cat([out[rows], out[[B + r for r in rows]]])
     assert_close(got, ref["x_out"], "bf16",
-                 "full layer x_out (17 seq%s)" % (", fused" if fused else ""))
+                 "full layer x_out (17 seq, %s)" % mode)
