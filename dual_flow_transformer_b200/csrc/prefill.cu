@@ -821,34 +821,109 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ two tiles per CTA
 // The same computation for two query heads h0 = 2x, h1 = 2x + 1 of one KV
-// group and one 128-row tile: both tiles read the same K/V pages (one load per
-// page serves 256 query rows), and the tensor core alternates between them,
-// so that it computes one tile's S or P V while the other tile's softmax
-// warps work (one tile alone leaves the tensor core idle during its softmax).
-// Warp 0: TMA producer; warp 1: MMA issuer; warps 2-5: softmax of tile 0;
-// warps 6-9: softmax of tile 1 (two softmax warps per SM sub-partition).
-// TMEM: tile t at columns t * 256: S double buffer [0, 128), O [128, 256).
+// group and one 128-row tile, over key blocks of 128 tokens (two cache pages).
+// Both tiles read the same K/V blocks (one load serves 256 query rows), and
+// the tensor core alternates between them: it computes one tile's P V and
+// next S while the other tile's softmax warps work.
+//  * S_t = Q_t K_j^T: M 128, N 128 (both pages of block j), K 128, both
+//    operands in shared memory, into tile t's 128-column TMEM region;
+//  * P_t, bf16 with two keys per 32-bit column, overwrites the first 64
+//    columns of that region, and O_t += P_t V_j reads P from TMEM (the A
+//    operand) and V from shared memory (MN-major, N 128 = all of D): P never
+//    passes through shared memory, and no MMA step reads more than 8 KB of
+//    it for its 128 x 128 x 16 multiply-adds;
+//  * per block j and tile t the MMA warp issues P V, then S of block j + 1
+//    into the same region: the MMAs of one thread run in issue order, so
+//    S_{j+1} overwrites P_j only after P_j V_j has read it, and the commit
+//    after S_{j+1} also tells the softmax warps that O_t holds P_j V_j (a
+//    rescale of O may then follow, and the next P may be written).
+// Warp 0: TMA producer (both Q tiles once; K blocks through a 2-stage ring,
+// V blocks through a 3-stage ring: a K block is released once both tiles'
+// S are computed, long before its V block); warp 1: MMA issuer; warps 2-5 /
+// 6-9: softmax of tile 0 / 1, one thread per query row. TMEM: S and P of
+// tile t at columns [128 t, 128 t + 128), O of tile t at [256 + 128 t, ...).
 
 constexpr int kPairThreads = 320;
 constexpr uint32_t kPairTmemCols = 512;
-constexpr int kPairStages = 4;  // K/V page ring depth
+constexpr int kBlk = 2 * kPage;       // keys per block
+constexpr int kKStages = 2;           // K block ring depth
+constexpr int kVStages = 3;           // V block ring depth
+constexpr uint32_t kPairOCol = 256;   // first TMEM column of O (tile 0)
 
-// One P buffer per tile: a tile's softmax writes P_i only after its own
-// O += P_{i-1} V_{i-1} has completed, which by then it long has (that MMA is
-// issued as soon as P_{i-1} is published, and P_i takes a whole softmax to
-// compute); the 32 KB this saves buys the fourth K/V stage.
 template <int D>
 struct PairLayout {
-  static constexpr int kQBytes = kRows * D * 2;      // one tile's Q
-  static constexpr int kPageBytes = kPage * D * 2;   // one K (or V) page
-  static constexpr int kStageBytes = 2 * kPageBytes;
-  static constexpr int kPBytes = kRows * kPage * 2;  // P of one page of one tile
-  static constexpr int kOffStages = 2 * kQBytes;
-  static constexpr int kOffP = kOffStages + kPairStages * kStageBytes;  // [tile]
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 1 + 2 * kPairStages + 2 * 4 * 2 + 1;
+  static constexpr int kQBytes = kRows * D * 2;   // one tile's Q: [D/64][128 rows][128 B]
+  static constexpr int kBlkBytes = kBlk * D * 2;  // one K or V block: [D/64][128 keys][128 B]
+  static constexpr int kHalf = kBlk * 128;        // bytes between a block's 64-column halves
+  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kBlkBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kBlkBytes;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 3 * 2 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
 };
+
+// Descriptor of an MN-major bf16 operand with 128-byte swizzle, two swizzle
+// atoms (128 elements) wide along N: 8-row groups along K 1024 bytes apart
+// (stride byte offset), the second 64-element atom along N `atom_stride`
+// bytes after the first (leading byte offset).
+__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t addr, uint32_t atom_stride) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((atom_stride >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// D (TMEM) (+)= A B with A in TMEM (K-major: lane = row, two bf16 of
+// consecutive k per 32-bit column) and B in shared memory (descriptor db).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 64 consecutive 32-bit TMEM columns of this thread's lane, waited for in the
+// same statement (the registers are defined once the wait has returned).
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, "
+      "%45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, "
+      "%62, %63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+        "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+        "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+        "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kPairThreads, 1)
@@ -865,13 +940,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = full + kPairStages;
-  uint64_t* s_full = empty + kPairStages;  // [tile][2] S_i landed in TMEM buffer i & 1
-  uint64_t* s_free = s_full + 4;       // [tile][2] that tile's softmax warps have read it
-  uint64_t* p_full = s_free + 4;       // [tile][2] P_i written to P buffer i & 1
-  uint64_t* pv_done = p_full + 4;      // [tile][2] O += P_i V_i completed
-  uint64_t* mma_done = pv_done + 4;
+  uint64_t* k_full = q_full + 1;          // [kKStages] K block landed
+  uint64_t* k_empty = k_full + kKStages;  // [kKStages] both tiles' S have read it
+  uint64_t* v_full = k_empty + kKStages;  // [kVStages]
+  uint64_t* v_empty = v_full + kVStages;  // [kVStages] both tiles' P V have read it
+  uint64_t* s_full = v_empty + kVStages;  // [tile] S_j in TMEM (and every earlier MMA done)
+  uint64_t* p_full = s_full + 2;          // [tile] P_j in TMEM (4 softmax warps)
+  uint64_t* pv_done = p_full + 2;         // [tile] O += P_j V_j completed
+  uint64_t* mma_done = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int h0 = 2 * static_cast<int>(blockIdx.x);
@@ -892,18 +968,22 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int rows = min(kRows, c.n - i0);
   const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
   const int npages = (kend + kPage - 1) / kPage;
+  const int nblk = (npages + 1) / 2;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kPairStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -934,93 +1014,100 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tma_load_2d(smem + t * Lay::kQBytes + hf * (kRows * 128), &tmQ, q_full,
                       (h0 + t) * D + hf * 64, c.t0 + i0);
       const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
-      int issued = 0;
-      for (int i = 0; i < npages; ++i) {
-        const int st = i % kPairStages;
-        if (i >= kPairStages && !mbar_wait(&empty[st], ((i / kPairStages) - 1) & 1)) {
+      // One block = pages 2j and (if the key range reaches it) 2j + 1; a
+      // missing second page leaves its rows stale: their keys are masked and
+      // their V rows cleared by the softmax warps.
+      auto load_block = [&](const CUtensorMap* tm, uint64_t* bar, uint8_t* dst, int j) {
+        const int np = min(2, npages - 2 * j);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(np * H * kPage * 128));
+        for (int q = 0; q < np; ++q) {
+          int page = tbl[2 * j + q];
+          if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
+            set_err(p.err, DF_DEVERR_BLOCK);
+            page = 0;
+          }
+          const int row = (page * p.Hkv + g) * kPage;
+#pragma unroll
+          for (int hf = 0; hf < H; ++hf)
+            tma_load_2d(dst + hf * Lay::kHalf + q * (kPage * 128), tm, bar, hf * 64, row);
+        }
+      };
+      int kissued = 0, vissued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int sk = j % kKStages, sv = j % kVStages;
+        if (j >= kKStages && !mbar_wait(&k_empty[sk], ((j / kKStages) - 1) & 1)) {
           set_err(p.err, DF_DEVERR_TIMEOUT);
           break;
         }
-        int page = tbl[i];
-        if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
-          set_err(p.err, DF_DEVERR_BLOCK);
-          page = 0;
+        load_block(&tmK, &k_full[sk], smem + Lay::kOffK + sk * Lay::kBlkBytes, j);
+        ++kissued;
+        if (j >= kVStages && !mbar_wait(&v_empty[sv], ((j / kVStages) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
         }
-        mbar_arrive_expect_tx(&full[st], Lay::kStageBytes);
-        const int row = (page * p.Hkv + g) * kPage;
-        uint8_t* sK = smem + Lay::kOffStages + st * Lay::kStageBytes;
-        uint8_t* sV = sK + Lay::kPageBytes;
-#pragma unroll
-        for (int hf = 0; hf < H; ++hf) {
-          tma_load_2d(sK + hf * kPage * 128, &tmK, &full[st], hf * 64, row);
-          tma_load_2d(sV + hf * kPage * 128, &tmV, &full[st], hf * 64, row);
-        }
-        ++issued;
+        load_block(&tmV, &v_full[sv], smem + Lay::kOffV + sv * Lay::kBlkBytes, j);
+        ++vissued;
       }
       // Leave no copy in flight (bounded waits).
       mbar_wait(q_full, 0);
-      for (int i = issued > kPairStages ? issued - kPairStages : 0; i < issued; ++i)
-        mbar_wait(&full[i % kPairStages], (i / kPairStages) & 1);
+      for (int j = kissued > kKStages ? kissued - kKStages : 0; j < kissued; ++j)
+        mbar_wait(&k_full[j % kKStages], (j / kKStages) & 1);
+      for (int j = vissued > kVStages ? vissued - kVStages : 0; j < vissued; ++j)
+        mbar_wait(&v_full[j % kVStages], (j / kVStages) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = umma::make_idesc(kRows, kPage);             // Q K^T
-      constexpr uint32_t kIdPV = umma::make_idesc(kRows, 64) | (1u << 16);  // P V, V MN-major
+      constexpr uint32_t kIdS = umma::make_idesc(kRows, kBlk);          // Q K^T, N 128
+      constexpr uint32_t kIdPV = umma::make_idesc(kRows, D) | (1u << 16);  // P V, V MN-major
       bool ok = mbar_wait(q_full, 0);
       // Descriptors are affine in the byte address (its bits 4..17 sit in the
-      // low field): each one below is a base plus a constant, so the issue
-      // loop spends its instructions on the MMAs.
+      // low field): each one below is a base plus a constant.
       const uint64_t dq0 = umma::smem_desc(smem_u32(smem));
-      const uint64_t dstage0 = umma::smem_desc(smem_u32(smem + Lay::kOffStages));
-      const uint64_t dv0 =
-          smem_desc_mn64(smem_u32(smem + Lay::kOffStages + Lay::kPageBytes));
-      const uint64_t dp0 = umma::smem_desc(smem_u32(smem + Lay::kOffP));
-      // S_i of tile t into its TMEM buffer i & 1
-      auto issue_s = [&](int t, int i) -> bool {
-        const int st = i % kPairStages, sb = i & 1;
-        if (!mbar_wait(&full[st], (i / kPairStages) & 1)) return false;
-        if (i >= 2 && !mbar_wait(&s_free[2 * t + sb], ((i >> 1) - 1) & 1)) return false;
+      const uint64_t dk0 = umma::smem_desc(smem_u32(smem + Lay::kOffK));
+      const uint64_t dv0 = smem_desc_mn(smem_u32(smem + Lay::kOffV), Lay::kHalf);
+      // S_j of tile t into its TMEM region (tile 0 first waits for the block)
+      auto issue_s = [&](int t, int j) -> bool {
+        const int st = j % kKStages;
+        if (t == 0 && !mbar_wait(&k_full[st], (j / kKStages) & 1)) return false;
         umma::tc_fence_after();
         const uint64_t dq = dq0 + static_cast<uint64_t>((t * Lay::kQBytes) >> 4);
-        const uint64_t dk = dstage0 + static_cast<uint64_t>((st * Lay::kStageBytes) >> 4);
-        const uint32_t d_tmem = tmem + t * 256 + sb * kPage;
+        const uint64_t dk = dk0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
+        const uint32_t d_tmem = tmem + t * kBlk;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int hf = kk >> 2, kq = kk & 3;
           umma::umma_bf16(d_tmem, dq + ((hf * (kRows * 128) + kq * 32) >> 4),
-                          dk + ((hf * (kPage * 128) + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
+                          dk + ((hf * Lay::kHalf + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
         }
-        umma::umma_commit(&s_full[2 * t + sb]);
+        umma::umma_commit(&s_full[t]);
+        if (t == 1) umma::umma_commit(&k_empty[st]);  // block j's K read by both tiles
         return true;
       };
-      // O_t += P_i V_i once tile t's softmax has written P_i
-      auto issue_pv = [&](int t, int i) -> bool {
-        const int pb = i & 1, st = i % kPairStages;
-        if (!mbar_wait(&p_full[2 * t + pb], (i >> 1) & 1)) return false;
+      // O_t += P_j V_j once tile t's softmax has written P_j
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int st = j % kVStages;
+        if (!mbar_wait(&p_full[t], j & 1)) return false;
+        if (t == 0 && !mbar_wait(&v_full[st], (j / kVStages) & 1)) return false;
         umma::tc_fence_after();
-        const uint64_t dp = dp0 + static_cast<uint64_t>((t * Lay::kPBytes) >> 4);
-        const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kStageBytes) >> 4);
-        const uint32_t d_tmem = tmem + t * 256 + kOCol;
+        const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
+        const uint32_t a_tmem = tmem + t * kBlk;
+        const uint32_t d_tmem = tmem + kPairOCol + t * D;
 #pragma unroll
-        for (int kk = 0; kk < kPage / 16; ++kk) {
-#pragma unroll
-          for (int hf = 0; hf < H; ++hf)
-            umma::umma_bf16(d_tmem + hf * 64, dp + ((kk * 32) >> 4),
-                            dv + ((hf * (kPage * 128) + kk * 2048) >> 4), kIdPV,
-                            (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma::umma_commit(&pv_done[2 * t + pb]);
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          umma_bf16_ts(d_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        umma::umma_commit(&pv_done[t]);
+        if (t == 1) umma::umma_commit(&v_empty[st]);  // block j's V read by both tiles
         return true;
       };
       if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
-      for (int i = 0; ok && i < npages; ++i) {
-        const bool more = i + 1 < npages;
-        if (more && !issue_s(0, i + 1)) ok = false;
-        if (ok && !issue_pv(0, i)) ok = false;
-        if (ok && more && !issue_s(1, i + 1)) ok = false;
-        if (ok && !issue_pv(1, i)) ok = false;
-        if (ok) umma::umma_commit(&empty[i % kPairStages]);  // page i read by both tiles
+      for (int j = 0; ok && j < nblk; ++j) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (ok && !issue_pv(t, j)) ok = false;
+          if (ok && j + 1 < nblk && !issue_s(t, j + 1)) ok = false;
+        }
       }
       if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
       umma::umma_commit(mma_done);  // completes when every MMA issued above has
@@ -1032,96 +1119,111 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int quarter = warp & 3;     // this warp may access TMEM lanes 32 quarter .. + 31
     const int r = quarter * 32 + lane;
     const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 256;
-    uint8_t* prow = smem + Lay::kOffP + t * Lay::kPBytes + r * 128;
-    uint64_t* my_s_full = s_full + 2 * t;
-    uint64_t* my_s_free = s_free + 2 * t;
-    uint64_t* my_p_full = p_full + 2 * t;
-    uint64_t* my_pv_done = pv_done + 2 * t;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t t_s = t_lane + t * kBlk;             // S / P of this tile
+    const uint32_t t_o = t_lane + kPairOCol + t * D;    // O of this tile
     float m_ref = kNegInf, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < npages; ++i) {
-      const int sb = i & 1, st = i % kPairStages, kbase = i * kPage;
-      if (!mbar_wait_warp(&my_s_full[sb], (i >> 1) & 1)) {
+    for (int j = 0; j < nblk; ++j) {
+      const int kbase = j * kBlk;
+      // S_j landed; every earlier MMA of this CTA (P_{j-1} V_{j-1} included)
+      // has completed with it.
+      if (!mbar_wait_warp(&s_full[t], j & 1)) {
         ok = false;
         break;
       }
       umma::tc_fence_after();
-      float s0[32], s1[32];
-      umma::tmem_ld32x2(t_lane + sb * kPage, s0, s1);
-      umma::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&my_s_free[sb]);
-
-      if (kbase + kPage - 1 > pos) {  // causal mask (and keys past the chunk end)
+      float s[kBlk];
+      {
+        uint32_t rr[64];
+        tmem_ld64_wait(t_s, rr);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (kbase + j > pos) s0[j] = kNegInf;
-          if (kbase + 32 + j > pos) s1[j] = kNegInf;
-        }
+        for (int k = 0; k < 64; ++k) s[k] = __uint_as_float(rr[k]);
+        tmem_ld64_wait(t_s + 64, rr);
+#pragma unroll
+        for (int k = 0; k < 64; ++k) s[64 + k] = __uint_as_float(rr[k]);
       }
-      const float m_cand = fmaxf(max32(s0), max32(s1)) * p.scale_log2;
+      if (kbase + kBlk - 1 > pos) {  // causal mask (and keys past the chunk end)
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k)
+          if (kbase + k > pos) s[k] = kNegInf;
+      }
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = s[q];
+#pragma unroll
+      for (int k = 8; k < kBlk; ++k) mx[k & 7] = fmaxf(mx[k & 7], s[k]);
+      const float m_cand =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
+      // The reference max moves (and O and l are rescaled) only when the
+      // block's max exceeds it by more than 2^kRescaleLog2.
       const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
-      if (m_ref == kNegInf) m_ref = m_cand;  // first page: O holds nothing yet
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold P_{i-1} V_{i-1} before it is rescaled in place.
-        if (!mbar_wait_warp(&my_pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        umma::tc_fence_after();
-        const float alpha = rescale ? exp2f(m_ref - m_cand) : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          float o[32];
-          umma::tmem_ld<32>(t_lane + kOCol + cc, o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= alpha;
-          tmem_st32(t_lane + kOCol + cc, o);
-        }
-        if (rescale) {
-          l *= alpha;
-          m_ref = m_cand;
-        }
+      float alpha = 1.f;
+      if (m_ref == kNegInf) {
+        m_ref = m_cand;  // first block: O holds nothing yet
+      } else if (rescale) {
+        alpha = exp2f(m_ref - m_cand);
+        m_ref = m_cand;
       }
       const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
 
-      // This tile's P buffer is free once O += P_{i-1} V_{i-1} has completed.
-      if (i >= 1 && !mbar_wait_warp(&my_pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-        ok = false;
-        break;
+      // P_j = 2^(s scale_log2 - mu) as bf16 pairs over the first 64 columns
+      // of the S region (this thread's lane); fp32 row sum of the weights.
+      float sum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < kBlk / 32; ++q) {
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float a = exp2_sfu(fmaf(s[32 * q + 2 * k], p.scale_log2, -mu));
+          const float bb = exp2_sfu(fmaf(s[32 * q + 2 * k + 1], p.scale_log2, -mu));
+          sum[k & 1] += a + bb;
+          w[k] = pack_f32_bf16x2(a, bb);
+        }
+        tmem_st16(t_s + 16 * q, w);
       }
-      l += write_p32(prow, r, 0, s0, p.scale_log2, mu);
-      l += write_p32(prow, r, 4, s1, p.scale_log2, mu);
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O holds P_{j-1} V_{j-1} (see the wait above): rescale it in place
+        // (alpha = 1 on the rows that keep their reference).
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          float o[32];
+          umma::tmem_ld<32>(t_o + cc, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_o + cc, o);
+        }
+      }
+      tmem_wait_st();
+      l = fmaf(l, alpha, sum[0] + sum[1]);
 
-      // Keys at or past kend on the last page hold other tokens' bytes
-      // (possibly NaN patterns): their weights are 0, and their V rows are
-      // zeroed, as 0 * NaN would still be NaN in the accumulator. Both tiles'
-      // warps clear the same rows (the same zero bytes), each before its own
-      // P is published, so neither tile's P V can read the old bytes.
-      if (kbase + kPage > kend) {
-        if (!mbar_wait_warp(&full[st], (i / kPairStages) & 1)) {  // the page has landed
+      // Keys at or past kend in the last block hold other tokens' bytes (or
+      // stale rows where the block has one page): their weights are 0, and
+      // their V rows are zeroed, as 0 * NaN would still be NaN in the
+      // accumulator. Both tiles' warps clear the same rows (the same zero
+      // bytes), each before its own P is published.
+      if (kbase + kBlk > kend) {
+        const int sv = j % kVStages;
+        if (!mbar_wait_warp(&v_full[sv], (j / kVStages) & 1)) {  // the block has landed
           ok = false;
           break;
         }
         const int kend_rel = kend - kbase;
-        uint8_t* sV = smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes;
-        const int nvec = (kPage - kend_rel) * H * 8;  // 16-byte chunks to clear
+        uint8_t* sV = smem + Lay::kOffV + sv * Lay::kBlkBytes;
+        const int nvec = (kBlk - kend_rel) * H * 8;  // 16-byte chunks to clear
         for (int v = r; v < nvec; v += kRows) {
           const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
-          *reinterpret_cast<uint4*>(sV + hf * (kPage * 128) + row * 128 + ch * 16) =
+          *reinterpret_cast<uint4*>(sV + hf * Lay::kHalf + row * 128 + ch * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();  // cleared V rows -> the tensor core's proxy
       }
-      fence_proxy_async_smem();  // P (and cleared V rows) -> the tensor core's proxy
       umma::tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&my_p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok) {
-      const int last = npages - 1;
-      ok = mbar_wait_warp(&my_pv_done[last & 1], (last >> 1) & 1);
-    }
+    if (ok) ok = mbar_wait_warp(&pv_done[t], (nblk - 1) & 1);
     if (ok) {
       umma::tc_fence_after();
       __nv_bfloat16* orow = p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t +
@@ -1129,7 +1231,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         float o[32];
-        umma::tmem_ld<32>(t_lane + kOCol + cc, o);
+        umma::tmem_ld<32>(t_o + cc, o);
 #pragma unroll
         for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
         if (r < rows) umma::store_bf16<32>(orow + cc, o);
