@@ -229,6 +229,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   pdl_wait();
   pdl_trigger();
 
+  // Partials mode: the query rows' partial products and row sums of squares
+  // are loaded first (one L2 round trip, overlapping the set-up below);
+  // consumer thread ct owns 4 consecutive Q columns of both rows.
+  const int G = p.G;
+  const bool has_q = p.qpart != nullptr && warp < kConsumerWarps && 4 * static_cast<int>(threadIdx.x) < G * D;
+  float4 v1[kMaxParts], v2[kMaxParts];
+  float ss1[kMaxParts], ss2[kMaxParts];
+#pragma unroll
+  for (int k = 0; k < kMaxParts; ++k) {
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool pk = has_q && k < p.qparts;
+    const int64_t o = static_cast<int64_t>(k) * p.qpstr + g * G * D + 4 * threadIdx.x;
+    v1[k] = pk ? ldg_f4(p.qpart + static_cast<int64_t>(b) * p.qrow + o) : z;
+    v2[k] = pk && p.dual ? ldg_f4(p.qpart + static_cast<int64_t>(p.qmp + b) * p.qrow + o) : z;
+    // (every consumer thread: those without Q columns may append K / V)
+    const bool sk = p.qpart != nullptr && warp < kConsumerWarps && k < p.qparts;
+    ss1[k] = sk ? p.qss[k * 2 * p.qmp + b] : 0.f;
+    ss2[k] = sk ? p.qss[k * 2 * p.qmp + p.qmp + b] : 0.f;
+  }
+
   if (split == 0 && g == 0 && threadIdx.x == 0) flag_len(p, b);
   const int L = attended_len(p, b);
   const int npages = (L + kPage - 1) / kPage;
@@ -304,36 +324,23 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // ------------------------------------------------------------ consumer warps
   const int gid = lane >> 2, tq = lane & 3;
-  const int G = p.G;
 
   if (p.qpart != nullptr) {
     // Partials mode prologue: this KV head's Q1 / Q2raw rows into shared
-    // memory, and (the CTA holding this step's page) its K / V row into the
-    // cache, while the producer already streams the other pages. Every load
-    // of a thread is issued before the first sum (one L2 round trip): thread
-    // ct owns 4 consecutive Q columns of both rows and, for ct < D / 2, 4 of
-    // the 2 D K / V columns.
+    // memory (their loads were issued at the start), and (the CTA holding
+    // this step's page) its K / V row into the cache, while the producer
+    // already streams the other pages. Thread ct owns 4 consecutive Q
+    // columns of both rows and, for ct < D / 2, 4 of the 2 D K / V columns.
     const int ct = threadIdx.x;  // 0 .. 127
-    const int M = 2 * p.qmp;
-    const int hcol = g * G * D;
-    const bool has_q = 4 * ct < G * D;
     const bool has_kv = append_pg >= 0 && 4 * ct < 2 * D;
     const float* pr1 = p.qpart + static_cast<int64_t>(b) * p.qrow;
-    const float* pr2 = p.qpart + static_cast<int64_t>(p.qmp + b) * p.qrow;
     const int kvi = 4 * ct, kvsel = kvi >= D ? 1 : 0, kvd = kvi - kvsel * D;
     const int kvcol = (kvsel ? p.qvcol : p.qkcol) + g * D + kvd;
-    float4 v1[kMaxParts], v2[kMaxParts], vk[kMaxParts];
-    float ss1[kMaxParts], ss2[kMaxParts];
+    float4 vk[kMaxParts];
 #pragma unroll
-    for (int k = 0; k < kMaxParts; ++k) {
-      const bool pk = k < p.qparts;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      v1[k] = pk && has_q ? ldg_f4(pr1 + k * p.qpstr + hcol + 4 * ct) : z;
-      v2[k] = pk && has_q && p.dual ? ldg_f4(pr2 + k * p.qpstr + hcol + 4 * ct) : z;
-      vk[k] = pk && has_kv ? ldg_f4(pr1 + k * p.qpstr + kvcol) : z;
-      ss1[k] = pk ? p.qss[k * M + b] : 0.f;
-      ss2[k] = pk ? p.qss[k * M + p.qmp + b] : 0.f;
-    }
+    for (int k = 0; k < kMaxParts; ++k)
+      vk[k] = has_kv && k < p.qparts ? ldg_f4(pr1 + k * p.qpstr + kvcol)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
     float s1 = 0.f, s2 = 0.f;
     float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), a2 = a1, ak = a1;
 #pragma unroll

@@ -34,6 +34,9 @@ SHAPES = {
                                       seed=82),
     "gqa": dataclasses.replace(BASE, B=16, d_model=1024, Hq=8, Hkv=2, D=128, cache_len=330,
                                seed=83),
+    # one query head per KV head: threads that append K / V own no Q columns
+    "g1": dataclasses.replace(BASE, B=6, d_model=256, Hq=4, Hkv=4, D=128, cache_len=140,
+                              seed=84),
 }
 
 
@@ -136,7 +139,7 @@ def test_partials_are_the_quarter_products(cuda_device, name):
 
 
 @pytest.mark.parametrize("num_splits", [0, 1, 3])
-@pytest.mark.parametrize("name", ["small", "odd", "gqa"])
+@pytest.mark.parametrize("name", ["small", "odd", "gqa", "g1", "one_kblock"])
 def test_split_path_bit_identical_to_fused_pre(cuda_device, name, num_splits):
     w = SHAPES[name]
     inp = synth.make_layer_inputs(w)
