@@ -28,6 +28,7 @@ _c_int, _c_i64, _c_size, _c_float, _vp = (ctypes.c_int, ctypes.c_int64, ctypes.c
 SIGNATURES = {
     "dualflow_abi_version": (_c_int, []),
     "dualflow_status_string": (ctypes.c_char_p, [_c_int]),
+    "dualflow_selftest_wait_timeout": (_c_int, [_vp, _vp]),
     "dualflow_decode_attn_num_splits": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "dualflow_decode_attn_workspace_size": (_c_size, [_c_int] * 7),
     "dualflow_decode_attn_num_launches": (_c_int, [_c_int] * 6),

@@ -114,3 +114,32 @@ extern "C" const char* dualflow_status_string(int status) {
     default: return "unknown dualflow status";
   }
 }
+
+// ------------------------------------------------------------------ failure-detection self-test
+
+namespace df {
+
+// One CTA of one warp waits, with the bounded waits every kernel of this
+// library uses (one thread, then the whole warp), on an mbarrier that nothing
+// ever arrives on. Each wait gives up after kWaitLimitCycles and the kernel
+// records DF_DEVERR_TIMEOUT and returns normally.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(int32_t* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0)) set_err(err, DF_DEVERR_TIMEOUT);
+  __syncwarp();
+  const bool ok = mbar_wait_warp(&bar, 0);
+  if (!ok && threadIdx.x == 0) set_err(err, DF_DEVERR_TIMEOUT);
+}
+
+}  // namespace df
+
+extern "C" df_status dualflow_selftest_wait_timeout(int32_t* err_flag, void* stream) {
+  if (err_flag == nullptr) return DF_ERR_NULL;
+  df::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err_flag);
+  return cudaGetLastError() == cudaSuccess ? DF_OK : DF_ERR_CUDA;
+}

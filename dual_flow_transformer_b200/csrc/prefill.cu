@@ -14,9 +14,10 @@
 //  1. append_kernel: token t of sequence b goes to cache position
 //     ctx_lens[b] + (t - cu_seqlens[b]) (one CTA per token, 16-byte copies);
 //  2. causal flash attention of the chunk's primary queries over the cache
-//     (prefix + chunk): tc::attn_kernel on the tcgen05 tensor cores (D = 128,
-//     at least 128 token rows, 16-byte aligned output rows; described at the
-//     kernel), otherwise attn_kernel: one CTA per (query head, 64-row tile,
+//     (prefix + chunk): tc::pair_kernel or tc::solo_kernel on the tcgen05
+//     tensor cores (D = 128, at least 128 token rows, 16-byte aligned output
+//     rows; described at the kernels), otherwise attn_kernel: one CTA per
+//     (query head, 64-row tile,
 //     sequence), heads fastest so that the CTAs sharing a KV head run side by
 //     side and meet its pages in L2; tiles of one sequence are issued longest
 //     first. 4 consumer warps own 16 query rows each; 1 producer warp streams
@@ -436,50 +437,20 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ------------------------------------------------------------------ 2'. attention, tcgen05
 //
-// The same computation on the 5th-generation tensor cores, for D = 128. One
-// CTA per (query head, 128-row tile, sequence); 6 warps:
-//  * warp 0, one thread: TMA producer -- the tile's Q rows once (two K-major
-//    [128][64] boxes, 128-byte swizzle), then the K and V pages of the key
-//    range through the 3-stage ring;
-//  * warp 1, one thread: MMA issuer -- S_i = Q K_i^T (M 128, N 64, K 128)
-//    into one of two 64-column TMEM buffers, and O += P_i V_i (M 128, K 64,
-//    two N = 64 halves) into a 128-column TMEM accumulator; S_{i+1} is issued
-//    before waiting for P_i, so it overlaps the softmax of page i;
-//  * warps 2-5: one thread per query row (its TMEM lane): S row by
-//    tcgen05.ld, causal mask, row max, P = 2^(s scale_log2 - m) written to
-//    shared memory as bf16 in the K-major swizzled layout the MMA reads. The
-//    reference max m is updated (and O rescaled in TMEM) only when a row's max
-//    exceeds it by more than 2^8, so P stays <= 256 and O is rarely touched.
-//    After the last page: O / l from TMEM to bf16 rows in global memory.
+// The same computation on the 5th-generation tensor cores, for D = 128, over
+// key blocks of 128 tokens (two cache pages): S = Q K^T (M 128, N 128) into
+// TMEM, the softmax warps write P as bf16 into TMEM, and O += P V takes P
+// from TMEM as its A operand. Two kernels: pair_kernel (two query heads of a
+// KV group per CTA, the tensor core alternating between their tiles) when the
+// group has an even number of heads, solo_kernel (one head per CTA, S and P
+// double-buffered) otherwise; both are described at their definitions. The
+// reference max m of a row changes (and O is rescaled in TMEM) only when the
+// row's max exceeds it by more than 2^8, so P stays <= 256 and O is rarely
+// touched. After the last block: O / l from TMEM to bf16 rows.
 namespace tc {
 
 constexpr int kRows = 128;          // query rows per CTA (= TMEM lanes)
-constexpr int kThreads = 192;       // producer warp, MMA warp, 4 softmax warps
-constexpr uint32_t kTmemCols = 256; // S double buffer (2 x 64 columns) + O (128)
-constexpr uint32_t kOCol = 128;     // first TMEM column of O
 constexpr float kRescaleLog2 = 8.f; // keep a stale reference max up to 2^8 below
-
-template <int D>
-struct Layout {
-  static constexpr int kQBytes = kRows * D * 2;
-  static constexpr int kPageBytes = kPage * D * 2;   // one K (or V) page
-  static constexpr int kStageBytes = 2 * kPageBytes;
-  static constexpr int kPBytes = kRows * kPage * 2;  // P of one page: [128 rows][64 keys]
-  static constexpr int kOffStages = kQBytes;
-  static constexpr int kOffP = kOffStages + kStages * kStageBytes;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 + 1;
-  static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
-};
-
-// Descriptor of an MN-major bf16 operand with 128-byte swizzle that is one
-// swizzle atom (64 elements) wide along N: 8-row atoms along K are 1024 bytes
-// apart; both byte-offset fields carry that stride (the N extent needs none).
-__device__ __forceinline__ uint64_t smem_desc_mn64(uint32_t addr) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1024 >> 4) << 16) |
-         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-         (static_cast<uint64_t>(2) << 61);
-}
 
 // Store 32 consecutive fp32 TMEM columns of this thread's lane and wait.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -502,14 +473,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float max32(const float (&v)[32]) {
-  float t[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-    t[q] = fmaxf(fmaxf(v[4 * q], v[4 * q + 1]), fmaxf(v[4 * q + 2], v[4 * q + 3]));
-  return fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])), fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
-}
-
 // 2^x by the SFU's approximate base-2 exponential (relative error near
 // 2^-22, far below the bf16 rounding of P; results under 2^-126 flush to 0,
 // which only drops weights below 2^-126 of the row's largest).
@@ -517,306 +480,6 @@ __device__ __forceinline__ float exp2_sfu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// P of 32 keys (chunks c0 .. c0 + 3 of 8 keys) of row r: bf16 into the
-// swizzled row (16-byte chunk c of row r at chunk c ^ (r & 7)); returns the
-// fp32 sum of the weights.
-__device__ __forceinline__ float write_p32(uint8_t* prow, int r, int c0, const float (&s)[32],
-                                           float scale_log2, float mu) {
-  float sum[2] = {0.f, 0.f};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float a = exp2_sfu(fmaf(s[8 * q + 2 * k], scale_log2, -mu));
-      const float b = exp2_sfu(fmaf(s[8 * q + 2 * k + 1], scale_log2, -mu));
-      sum[k & 1] += a + b;
-      w[k] = pack_f32_bf16x2(a, b);
-    }
-    *reinterpret_cast<uint4*>(prow + (((c0 + q) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  return sum[0] + sum[1];
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using Lay = Layout<D>;
-  constexpr int H = D / 64;  // 64-column halves of Q, K and V
-  constexpr float kNegInf = -INFINITY;
-  static_assert(D == 128, "the tcgen05 prefill kernel is built for head_dim 128");
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
-  uint64_t* q_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;  // [2] S_i landed in TMEM buffer i & 1
-  uint64_t* s_free = s_full + 2;       // [2] the softmax warps have read it
-  uint64_t* p_full = s_free + 2;       // [2] P_i written to P buffer i & 1
-  uint64_t* pv_done = p_full + 2;      // [2] O += P_i V_i completed
-  uint64_t* mma_done = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-
-  const int h = blockIdx.x;
-  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
-  const int b = blockIdx.z;
-  const int g = h / p.G;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();
-  pdl_trigger();
-
-  const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
-  if (!c.ok) {
-    if (h == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
-    return;
-  }
-  const int i0 = tile * kRows;
-  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
-  const int rows = min(kRows, c.n - i0);
-  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
-  const int npages = (kend + kPage - 1) / kPage;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
-    }
-    mbar_init(mma_done, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  umma::tc_fence_before();
-  __syncthreads();
-  umma::tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, Lay::kQBytes);
-#pragma unroll
-      for (int hf = 0; hf < H; ++hf)
-        tma_load_2d(smem + hf * (kRows * 128), &tmQ, q_full, h * D + hf * 64, c.t0 + i0);
-      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
-      int issued = 0;
-      for (int i = 0; i < npages; ++i) {
-        const int st = i % kStages;
-        if (i >= kStages && !mbar_wait(&empty[st], ((i / kStages) - 1) & 1)) {
-          set_err(p.err, DF_DEVERR_TIMEOUT);
-          break;
-        }
-        int page = tbl[i];
-        if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
-          set_err(p.err, DF_DEVERR_BLOCK);
-          page = 0;
-        }
-        mbar_arrive_expect_tx(&full[st], Lay::kStageBytes);
-        const int row = (page * p.Hkv + g) * kPage;
-        uint8_t* sK = smem + Lay::kOffStages + st * Lay::kStageBytes;
-        uint8_t* sV = sK + Lay::kPageBytes;
-#pragma unroll
-        for (int hf = 0; hf < H; ++hf) {
-          tma_load_2d(sK + hf * kPage * 128, &tmK, &full[st], hf * 64, row);
-          tma_load_2d(sV + hf * kPage * 128, &tmV, &full[st], hf * 64, row);
-        }
-        ++issued;
-      }
-      // Leave no copy in flight (bounded waits).
-      mbar_wait(q_full, 0);
-      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
-        mbar_wait(&full[i % kStages], (i / kStages) & 1);
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = umma::make_idesc(kRows, kPage);                 // Q K^T
-      constexpr uint32_t kIdPV = umma::make_idesc(kRows, 64) | (1u << 16);      // P V, V MN-major
-      const uint32_t q_addr = smem_u32(smem);
-      bool ok = mbar_wait(q_full, 0);
-      auto issue_s = [&](int i) -> bool {
-        const int st = i % kStages, sb = i & 1;
-        if (!mbar_wait(&full[st], (i / kStages) & 1)) return false;
-        if (i >= 2 && !mbar_wait(&s_free[sb], ((i >> 1) - 1) & 1)) return false;
-        umma::tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int hf = kk >> 2, kq = kk & 3;
-          umma::umma_bf16(tmem + sb * kPage,
-                          umma::smem_desc(q_addr + hf * (kRows * 128) + kq * 32),
-                          umma::smem_desc(k_addr + hf * (kPage * 128) + kq * 32), kIdS,
-                          kk > 0 ? 1u : 0u);
-        }
-        umma::umma_commit(&s_full[sb]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int i = 0; ok && i < npages; ++i) {
-        if (i + 1 < npages && !issue_s(i + 1)) {
-          ok = false;
-          break;
-        }
-        const int pb = i & 1, st = i % kStages;
-        if (!mbar_wait(&p_full[pb], (i >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        umma::tc_fence_after();
-        const uint32_t p_addr = smem_u32(smem + Lay::kOffP + pb * Lay::kPBytes);
-        const uint32_t v_addr =
-            smem_u32(smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes);
-#pragma unroll
-        for (int kk = 0; kk < kPage / 16; ++kk) {
-#pragma unroll
-          for (int hf = 0; hf < H; ++hf)
-            umma::umma_bf16(tmem + kOCol + hf * 64, umma::smem_desc(p_addr + kk * 32),
-                            smem_desc_mn64(v_addr + hf * (kPage * 128) + kk * 2048), kIdPV,
-                            (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma::umma_commit(&pv_done[pb]);
-        umma::umma_commit(&empty[st]);
-      }
-      if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
-      umma::umma_commit(mma_done);  // completes when every MMA issued above has
-      mbar_wait(mma_done, 0);
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax warps
-    const int quarter = warp & 3;  // this warp may access TMEM lanes 32 quarter .. + 31
-    const int r = quarter * 32 + lane;
-    const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint8_t* p_base = smem + Lay::kOffP + r * 128;
-    float m_ref = kNegInf, l = 0.f;
-    bool ok = true;
-    for (int i = 0; i < npages; ++i) {
-      const int sb = i & 1, st = i % kStages, kbase = i * kPage;
-      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      umma::tc_fence_after();
-      float s0[32], s1[32];
-      umma::tmem_ld32x2(t_lane + sb * kPage, s0, s1);
-      umma::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-
-      if (kbase + kPage - 1 > pos) {  // causal mask (and keys past the chunk end)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (kbase + j > pos) s0[j] = kNegInf;
-          if (kbase + 32 + j > pos) s1[j] = kNegInf;
-        }
-      }
-      const float m_cand = fmaxf(max32(s0), max32(s1)) * p.scale_log2;
-      const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
-      if (m_ref == kNegInf) m_ref = m_cand;  // first page: O holds nothing yet
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold P_{i-1} V_{i-1} before it is rescaled in place.
-        if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        umma::tc_fence_after();
-        const float alpha = rescale ? exp2f(m_ref - m_cand) : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          float o[32];
-          umma::tmem_ld<32>(t_lane + kOCol + cc, o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= alpha;
-          tmem_st32(t_lane + kOCol + cc, o);
-        }
-        if (rescale) {
-          l *= alpha;
-          m_ref = m_cand;
-        }
-      }
-      const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
-
-      // P buffer sb is free once O += P_{i-2} V_{i-2} has completed.
-      if (i >= 2 && !mbar_wait_warp(&pv_done[sb], ((i >> 1) - 1) & 1)) {
-        ok = false;
-        break;
-      }
-      uint8_t* prow = p_base + sb * Lay::kPBytes;
-      l += write_p32(prow, r, 0, s0, p.scale_log2, mu);
-      l += write_p32(prow, r, 4, s1, p.scale_log2, mu);
-
-      // Keys at or past kend on the last page hold other tokens' bytes
-      // (possibly NaN patterns): their weights are 0, and their V rows are
-      // zeroed, as 0 * NaN would still be NaN in the accumulator.
-      if (kbase + kPage > kend) {
-        if (!mbar_wait_warp(&full[st], (i / kStages) & 1)) {  // the page has landed
-          ok = false;
-          break;
-        }
-        const int kend_rel = kend - kbase;
-        uint8_t* sV = smem + Lay::kOffStages + st * Lay::kStageBytes + Lay::kPageBytes;
-        const int nvec = (kPage - kend_rel) * H * 8;  // 16-byte chunks to clear
-        for (int v = r; v < nvec; v += kRows) {
-          const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
-          *reinterpret_cast<uint4*>(sV + hf * (kPage * 128) + row * 128 + ch * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      fence_proxy_async_smem();  // P (and cleared V rows) -> the tensor core's proxy
-      umma::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-    }
-    if (ok) {
-      const int last = npages - 1;
-      ok = mbar_wait_warp(&pv_done[last & 1], (last >> 1) & 1);
-    }
-    if (ok) {
-      umma::tc_fence_after();
-      __nv_bfloat16* orow =
-          p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t + h * D;
-#pragma unroll
-      for (int cc = 0; cc < D; cc += 32) {
-        float o[32];
-        umma::tmem_ld<32>(t_lane + kOCol + cc, o);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
-        if (r < rows) umma::store_bf16<32>(orow + cc, o);
-      }
-    } else if (lane == 0) {
-      set_err(p.err, DF_DEVERR_TIMEOUT);
-    }
-  }
-
-  umma::tc_fence_before();
-  __syncthreads();
-  umma::tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
-  }
 }
 
 // ------------------------------------------------------------------ two tiles per CTA
@@ -1347,6 +1010,398 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ one tile per CTA
+// One query head and one 128-row tile per CTA (any number of query heads per
+// KV head), over key blocks of 128 tokens. S and P are double-buffered in
+// TMEM, so S of block j + 1 is computed while the softmax warps work on
+// block j; P_j (bf16 pairs) is the A operand of O += P_j V_j. Each query row
+// is shared by two softmax warps, one per 64-key half of the block (eight
+// softmax warps, two per SM sub-partition, so that one hides the other's
+// latencies): both read the whole S row for its maximum (the same bits, so
+// the same decisions), each writes the weights of its half, keeps its own
+// row sum, and owns half of O's columns for a rescale and the division.
+// Warp 0: TMA producer (Q once; K and V blocks through 3-stage rings);
+// warp 1: MMA issuer (S_0, S_1, then per block j: P_j V_j and S_{j+2} into
+// the S buffer block j used -- MMAs of one thread run in order, and the
+// softmax warps have read S_j before publishing P_j);
+// warps 2-9: softmax, half h = (warp - 2) / 4, TMEM lane quarter warp % 4.
+// TMEM: S buffers at columns [0, 128) and [128, 256), O at [256, 384), P
+// buffers at [384, 448) and [448, 512).
+
+constexpr int kSoloThreads = 320;
+constexpr uint32_t kSoloTmemCols = 512;
+constexpr int kSoloStages = 3;          // K and V block rings
+constexpr uint32_t kSoloOCol = 256;
+constexpr uint32_t kSoloPCol = 384;
+
+template <int D>
+struct SoloLayout {
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kBlkBytes = kBlk * D * 2;
+  static constexpr int kHalf = kBlk * 128;
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kSoloStages * kBlkBytes;
+  static constexpr int kOffX = kOffV + kSoloStages * kBlkBytes;  // [2 halves][128] row sums
+  static constexpr int kOffBar = kOffX + 2 * kRows * 4;
+  static constexpr int kNumBars = 1 + 4 * kSoloStages + 3 * 2 + 2;
+  static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSoloThreads, 1)
+    solo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using Lay = SoloLayout<D>;
+  constexpr int H = D / 64;
+  constexpr float kNegInf = -INFINITY;
+  static_assert(D == 128, "the one-tile prefill kernel is built for head_dim 128");
+  static_assert(SoloLayout<D>::kSmem <= 227 * 1024, "shared memory budget");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* xl = reinterpret_cast<float*>(smem + Lay::kOffX);  // [half][row] row sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + kSoloStages;
+  uint64_t* v_full = k_empty + kSoloStages;
+  uint64_t* v_empty = v_full + kSoloStages;
+  uint64_t* s_full = v_empty + kSoloStages;  // [buffer] S_j landed (and every earlier S / P V)
+  uint64_t* p_full = s_full + 2;             // [buffer] P_j written (8 softmax warps)
+  uint64_t* pv_done = p_full + 2;            // [buffer] O += P_j V_j completed
+  uint64_t* mma_done = pv_done + 2;
+  uint64_t* l_ready = mma_done + 1;          // both halves' row sums written (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_ready + 1);
+
+  const int h = blockIdx.x;
+  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
+  const int b = blockIdx.z;
+  const int g = h / p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+
+  const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
+  if (!c.ok) {
+    if (h == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
+    return;
+  }
+  const int i0 = tile * kRows;
+  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
+  const int rows = min(kRows, c.n - i0);
+  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
+  const int npages = (kend + kPage - 1) / kPage;
+  const int nblk = (npages + 1) / 2;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kSoloStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    mbar_init(l_ready, 8);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kSoloTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_arrive_expect_tx(q_full, Lay::kQBytes);
+#pragma unroll
+      for (int hf = 0; hf < H; ++hf)
+        tma_load_2d(smem + hf * (kRows * 128), &tmQ, q_full, h * D + hf * 64, c.t0 + i0);
+      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      // one block = pages 2j and (if the key range reaches it) 2j + 1; a
+      // missing second page leaves stale rows: masked keys, cleared V rows
+      auto load_block = [&](const CUtensorMap* tm, uint64_t* bar, uint8_t* dst, int j) {
+        const int np = min(2, npages - 2 * j);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(np * H * kPage * 128));
+        for (int q = 0; q < np; ++q) {
+          int page = tbl[2 * j + q];
+          if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
+            set_err(p.err, DF_DEVERR_BLOCK);
+            page = 0;
+          }
+          const int row = (page * p.Hkv + g) * kPage;
+#pragma unroll
+          for (int hf = 0; hf < H; ++hf)
+            tma_load_2d(dst + hf * Lay::kHalf + q * (kPage * 128), tm, bar, hf * 64, row);
+        }
+      };
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int st = j % kSoloStages;
+        if (j >= kSoloStages && !mbar_wait(&k_empty[st], ((j / kSoloStages) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          break;
+        }
+        load_block(&tmK, &k_full[st], smem + Lay::kOffK + st * Lay::kBlkBytes, j);
+        if (j >= kSoloStages && !mbar_wait(&v_empty[st], ((j / kSoloStages) - 1) & 1)) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          mbar_wait(&k_full[st], (j / kSoloStages) & 1);  // the K block issued above
+          break;
+        }
+        load_block(&tmV, &v_full[st], smem + Lay::kOffV + st * Lay::kBlkBytes, j);
+        ++issued;
+      }
+      // Leave no copy in flight (bounded waits).
+      mbar_wait(q_full, 0);
+      for (int j = issued > kSoloStages ? issued - kSoloStages : 0; j < issued; ++j) {
+        mbar_wait(&k_full[j % kSoloStages], (j / kSoloStages) & 1);
+        mbar_wait(&v_full[j % kSoloStages], (j / kSoloStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = umma::make_idesc(kRows, kBlk);
+      constexpr uint32_t kIdPV = umma::make_idesc(kRows, D) | (1u << 16);  // V MN-major
+      bool ok = mbar_wait(q_full, 0);
+      const uint64_t dq = umma::smem_desc(smem_u32(smem));
+      const uint64_t dk0 = umma::smem_desc(smem_u32(smem + Lay::kOffK));
+      const uint64_t dv0 = smem_desc_mn(smem_u32(smem + Lay::kOffV), Lay::kHalf);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % kSoloStages;
+        if (!mbar_wait(&k_full[st], (j / kSoloStages) & 1)) return false;
+        umma::tc_fence_after();
+        const uint64_t dk = dk0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
+        const uint32_t d_tmem = tmem + (j & 1) * kBlk;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk >> 2, kq = kk & 3;
+          umma::umma_bf16(d_tmem, dq + ((hf * (kRows * 128) + kq * 32) >> 4),
+                          dk + ((hf * Lay::kHalf + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
+        }
+        umma::umma_commit(&s_full[j & 1]);
+        umma::umma_commit(&k_empty[st]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && nblk > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int st = j % kSoloStages, bb = j & 1;
+        if (!mbar_wait(&p_full[bb], (j >> 1) & 1) ||
+            !mbar_wait(&v_full[st], (j / kSoloStages) & 1)) {
+          ok = false;
+          break;
+        }
+        umma::tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
+        const uint32_t a_tmem = tmem + kSoloPCol + bb * (kBlk / 2);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          umma_bf16_ts(tmem + kSoloOCol, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        umma::umma_commit(&pv_done[bb]);
+        umma::umma_commit(&v_empty[st]);
+        if (j + 2 < nblk && !issue_s(j + 2)) ok = false;
+      }
+      if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
+      umma::umma_commit(mma_done);  // completes when every MMA issued above has
+      mbar_wait(mma_done, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int hh = (warp - 2) >> 2;   // key half of each block this warp serves
+    const int quarter = warp & 3;     // TMEM lanes 32 quarter .. + 31
+    const int r = quarter * 32 + lane;
+    const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t t_o = t_lane + kSoloOCol + hh * 64;  // this half's 64 columns of O
+    float m_ref = kNegInf, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const int bb = j & 1;
+      const int kbase = j * kBlk + hh * 64;
+      if (!mbar_wait_warp(&s_full[bb], (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      umma::tc_fence_after();
+      const uint32_t t_s = t_lane + bb * kBlk;                       // S_j, both halves
+      const uint32_t t_p = t_lane + kSoloPCol + bb * (kBlk / 2) + hh * 32;  // this half's P
+      // the other half first, for the row maximum only
+      float omax;
+      {
+        uint32_t rr[64];
+        tmem_ld64_wait(t_s + (hh ^ 1) * 64, rr);
+        const int obase = j * kBlk + (hh ^ 1) * 64;
+        float mo[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mo[q] = obase + q > pos ? kNegInf : __uint_as_float(rr[q]);
+#pragma unroll
+        for (int k = 8; k < 64; k += 16) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float x0 = obase + k + q > pos ? kNegInf : __uint_as_float(rr[k + q]);
+            const float x1 = obase + k + 8 + q > pos ? kNegInf : __uint_as_float(rr[k + 8 + q]);
+            mo[q] = max3f(mo[q], x0, x1);
+          }
+        }
+        omax = fmaxf(max3f(mo[0], mo[1], mo[2]), max3f(max3f(mo[3], mo[4], mo[5]), mo[6], mo[7]));
+      }
+      float s[64];
+      {
+        uint32_t rr[64];
+        tmem_ld64_wait(t_s + hh * 64, rr);
+#pragma unroll
+        for (int k = 0; k < 64; ++k) s[k] = __uint_as_float(rr[k]);
+      }
+      if (kbase + 63 > pos) {  // causal mask (and keys past the chunk end)
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (kbase + k > pos) s[k] = kNegInf;
+      }
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = s[q];
+#pragma unroll
+      for (int k = 8; k < 64; k += 16) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx[q] = max3f(mx[q], s[k + q], s[k + 8 + q]);
+      }
+      // the row's maximum over both halves: the same value in both warps
+      const float m_cand =
+          max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), max3f(mx[6], mx[7], omax)) *
+          p.scale_log2;
+      const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
+      float alpha = 1.f;
+      if (m_ref == kNegInf) {
+        m_ref = m_cand;  // first block: O holds nothing yet
+      } else if (rescale) {
+        alpha = exp2f(m_ref - m_cand);
+        m_ref = m_cand;
+      }
+      const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
+
+      const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+      const uint64_t nmu2 = f2_pack(-mu, -mu);
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint64_t x2 = f2_fma(f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2, nmu2);
+          uint64_t e2;
+          if (poly_pair(k)) {
+            e2 = exp2_poly2(x2);
+          } else {
+            float xa, xb;
+            f2_unpack(x2, xa, xb);
+            e2 = f2_pack(exp2_sfu(xa), exp2_sfu(xb));
+          }
+          sum2[k & 3] = f2_add(sum2[k & 3], e2);
+          float a, a2;
+          f2_unpack(e2, a, a2);
+          w[k] = pack_f32_bf16x2(a, a2);
+        }
+        tmem_st16(t_p + 16 * q, w);
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold P_{j-1} V_{j-1} before it is rescaled in place
+        if (!mbar_wait_warp(&pv_done[bb ^ 1], ((j - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        umma::tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 32) {
+          float o[32];
+          umma::tmem_ld<32>(t_o + cc, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_o + cc, o);
+        }
+      }
+      tmem_wait_st();
+      {
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f2_unpack(sum2[i], e[2 * i], e[2 * i + 1]);
+        l = fmaf(l, alpha, ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7])));
+      }
+      // Keys at or past kend in the last block: zero weights, and their V
+      // rows cleared (0 * NaN would still be NaN); every softmax thread
+      // clears its share before the block's P is published.
+      if (j * kBlk + kBlk > kend) {
+        const int st = j % kSoloStages;
+        if (!mbar_wait_warp(&v_full[st], (j / kSoloStages) & 1)) {
+          ok = false;
+          break;
+        }
+        const int kend_rel = kend - j * kBlk;
+        uint8_t* sV = smem + Lay::kOffV + st * Lay::kBlkBytes;
+        const int nvec = (kBlk - kend_rel) * H * 8;
+        for (int v = hh * kRows + r; v < nvec; v += 2 * kRows) {
+          const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
+          *reinterpret_cast<uint4*>(sV + hf * Lay::kHalf + row * 128 + ch * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      umma::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[bb]);
+    }
+    if (ok) ok = mbar_wait_warp(&pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1);
+    // the row sum over both halves (every warp publishes its own, even after
+    // a failed wait, so that its partner's bounded wait ends)
+    xl[hh * kRows + r] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(l_ready);
+    if (ok) ok = mbar_wait_warp(l_ready, 0);
+    if (ok) {
+      l += xl[(hh ^ 1) * kRows + r];
+      umma::tc_fence_after();
+      __nv_bfloat16* orow =
+          p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t + h * D + hh * 64;
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 32) {
+        float o[32];
+        umma::tmem_ld<32>(t_o + cc, o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
+        if (r < rows) umma::store_bf16<32>(orow + cc, o);
+      }
+    } else if (lane == 0) {
+      set_err(p.err, DF_DEVERR_TIMEOUT);
+    }
+  }
+
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kSoloTmemCols)
+                 : "memory");
+  }
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------------ 3. last-row gather
@@ -1406,10 +1461,10 @@ cudaError_t launch_attn_tc(const AttnParams& p, int Hq, int B, const CUtensorMap
     return launch_pdl(tc::pair_kernel<128>, dim3(Hq / 2, p.tiles, B), dim3(tc::kPairThreads),
                       smem2, stream, *tmQ, *tmK, *tmV, p);
   }
-  constexpr size_t smem = tc::Layout<128>::kSmem;
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::attn_kernel<128>), smem);
+  constexpr size_t smem = tc::SoloLayout<128>::kSmem;
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::solo_kernel<128>), smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tc::attn_kernel<128>, dim3(Hq, p.tiles, B), dim3(tc::kThreads), smem, stream,
+  return launch_pdl(tc::solo_kernel<128>, dim3(Hq, p.tiles, B), dim3(tc::kSoloThreads), smem, stream,
                     *tmQ, *tmK, *tmV, p);
 }
 

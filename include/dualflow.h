@@ -78,6 +78,21 @@ int dualflow_abi_version(void);
 const char* dualflow_status_string(int status);
 
 /* ------------------------------------------------------------------------ */
+/* Failure-detection self-test (no counterpart in the pages).                */
+/*                                                                           */
+/* Every in-kernel wait of this library (on an mbarrier, a grid counter or a */
+/* peer CTA) gives up after about 2e9 SM cycles (1-2 s), ORs                 */
+/* DF_DEVERR_TIMEOUT into the call's err_flag and lets the kernel return, so */
+/* a lost arrival never hangs the GPU. This entry point exercises that       */
+/* mechanism without a fault: one launch of one warp waits, with the same    */
+/* bounded waits (single thread, then whole warp), on an mbarrier that       */
+/* nothing arrives on; after two time-outs (2-4 s) *err_flag has             */
+/* DF_DEVERR_TIMEOUT set and the context stays usable.                       */
+/* err_flag: int32 in device memory (ORed into). Asynchronous on `stream`.   */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_selftest_wait_timeout(int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Dual-flow decode attention (asymmetric shared-KV attention).              */
 /*                                                                           */
 /* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi       */

@@ -278,3 +278,28 @@ def test_prefill_kernel_choice_is_checked(lib):
     assert lib.dualflow_prefill_kernel(128, 100, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
     assert lib.dualflow_prefill_kernel(64, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
     assert lib.dualflow_prefill_kernel(128, 300, FAKE + 4, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
+
+
+def test_selftest_and_split_pre_entries_reject_invalid_arguments(lib):
+    # every check below returns before any CUDA call
+    assert lib.dualflow_selftest_wait_timeout(None, None) == L.DF_ERR_NULL
+    buf = 4096
+    assert lib.dualflow_layer_qkv_partials(None, buf, 8, 512, 4, 2, 128, buf, buf, None,
+                                           None) == L.DF_ERR_NULL
+    assert lib.dualflow_layer_qkv_partials(buf, buf, 0, 512, 4, 2, 128, buf, buf, None,
+                                           None) == L.DF_ERR_SHAPE
+
+    def attn(**kw):
+        a = dict(part=buf, ss=buf, parts=4, m=8, d=512, eps=1e-5)
+        a.update(kw)
+        return lib.dualflow_decode_attn_qkv_partials(
+            a["part"], a["ss"], a["parts"], a["m"], a["d"], a["eps"], None, buf, buf, buf, 4,
+            buf, 200, buf, buf, 0, 4, 2, 128, 64, 100, 0.0, 0, None, 0, None, None)
+
+    assert attn(part=None) == L.DF_ERR_NULL
+    assert attn(ss=None) == L.DF_ERR_NULL
+    assert attn(parts=0) == L.DF_ERR_SHAPE
+    assert attn(parts=5) == L.DF_ERR_SHAPE
+    assert attn(m=0) == L.DF_ERR_SHAPE
+    assert attn(eps=-1.0) == L.DF_ERR_SHAPE
+    assert attn(part=buf + 4) == L.DF_ERR_ALIGN
