@@ -43,15 +43,22 @@ constexpr int kXPitch = 33;
 constexpr int kStgPitch = 36;
 constexpr int kTileX = kBM * kBK * 2;  // 16 KB activation tile per stage
 constexpr int kRingBytes = 196 * 1024;
+// The ring plus the epilogue staging (the primary rows' results for the
+// coupling and the output staging). A CTA with one tile and no cluster
+// partner needs the staging only after its last MMA, when the ring is idle:
+// its ring then spans the whole region (one stage more at the wide tiles).
+constexpr int kStagingBytes = 64 * 33 * 4 + 4 * 32 * 36 * 4;
+constexpr int kRingRegion = kRingBytes + kStagingBytes;
 constexpr int kMaxCluster = 8;
 constexpr int kSms = 148;
 constexpr int kMaxOut = 256;  // output columns per tile (coupling prefetch buffer)
-constexpr size_t kSmemBytes =
-    1024 + kRingBytes + kXRows * kXPitch * 4 + 4 * 32 * kStgPitch * 4 + kMaxOut * 4 + 256;
+static_assert(kStagingBytes == kXRows * kXPitch * 4 + 4 * 32 * kStgPitch * 4, "staging size");
+constexpr size_t kSmemBytes = 1024 + kRingRegion + kMaxOut * 4 + 256;
 
 struct Params {
   int M, m_primary, n_out, n_aux, epilogue;
   int kblocks, BN, half, out_per_tile, n_tiles, C, stages, stage_bytes;
+  int staging_in_ring;  // 1: the epilogue staging starts at the ring's base (see kRingRegion)
   int tpb;            // tiles per batch entry: tile t is (batch t / tpb, column tile t % tpb)
   int64_t ystride_b;  // output batch stride (elements)
   int batched;        // X / W tensor maps are 3-D (batch > 1); 2-D otherwise
@@ -323,9 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* xbuf = reinterpret_cast<float*>(smem + kRingBytes);      // [64][33]
+  float* xbuf = reinterpret_cast<float*>(smem + (p.staging_in_ring ? 0 : kRingBytes));  // [64][33]
   float* stg_all = xbuf + kXRows * kXPitch;                        // 4 x [32][36]
-  float* cpl_s = stg_all + 4 * 32 * kStgPitch;                     // [256] coupling of a tile
+  float* cpl_s = reinterpret_cast<float*>(smem + kRingRegion);     // [256] coupling of a tile
   uint64_t* full = reinterpret_cast<uint64_t*>(cpl_s + kMaxOut);
   uint64_t* empty = full + kMaxStages;
   uint64_t* acc_full = empty + kMaxStages;
@@ -721,6 +728,7 @@ const ClusterCaps* caps_for_device() {
 struct Plan {
   bool ok;
   int BN, C, n_tiles, ctas, stages, stage_bytes;
+  bool staging_in_ring;
   double est_us;
   int tpb;  // tiles per batch entry (n_tiles = batch * tpb)
 };
@@ -745,6 +753,8 @@ Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_
     int stages = kRingBytes / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 3) continue;
+    int stages_region = kRingRegion / stage_bytes;  // one tile, no cluster partner
+    if (stages_region > kMaxStages) stages_region = kMaxStages;
     for (int C = 1; C <= kMaxCluster && C <= KB; ++C) {
       int ctas, tpc;
       if (C == 1) {
@@ -768,7 +778,9 @@ Plan make_plan(int M, int N, int K, int epilogue, const ClusterCaps* caps, size_
       if (tot / 77e3 > t) t = tot / 77e3;
       t += (C > 1 ? 2.5 : 0.0) + tpc * 1.5 + 2.5;
       if (t < best.est_us) {
-        best = Plan{true, BN, C, n_tiles, ctas, stages, stage_bytes, t, tpb};
+        const bool in_ring = C == 1 && tpc == 1;
+        best = Plan{true, BN, C, n_tiles, ctas, in_ring ? stages_region : stages, stage_bytes,
+                    in_ring, t, tpb};
       }
     }
   }
@@ -827,6 +839,7 @@ int launch_if_better(const Request& r) {
   p.C = pl.C;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
+  p.staging_in_ring = pl.staging_in_ring ? 1 : 0;
   p.idesc = make_idesc(kBM, pl.BN);
   p.F = r.N / 2;
   p.y = static_cast<__nv_bfloat16*>(r.y);
