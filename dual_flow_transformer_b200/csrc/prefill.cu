@@ -14,10 +14,9 @@
 //  1. append_kernel: token t of sequence b goes to cache position
 //     ctx_lens[b] + (t - cu_seqlens[b]) (one CTA per token, 16-byte copies);
 //  2. causal flash attention of the chunk's primary queries over the cache
-//     (prefix + chunk): tc::pair_kernel or tc::solo_kernel on the tcgen05
-//     tensor cores (D = 128, at least 128 token rows, 16-byte aligned output
-//     rows; described at the kernels), otherwise attn_kernel: one CTA per
-//     (query head, 64-row tile,
+//     (prefix + chunk): tc::pair_kernel on the tcgen05 tensor cores (D = 128,
+//     at least 128 token rows, 16-byte aligned output rows; described at the
+//     kernel), otherwise attn_kernel: one CTA per (query head, 64-row tile,
 //     sequence), heads fastest so that the CTAs sharing a KV head run side by
 //     side and meet its pages in L2; tiles of one sequence are issued longest
 //     first. 4 consumer warps own 16 query rows each; 1 producer warp streams
@@ -144,6 +143,7 @@ struct AttnParams {
   int T, Hkv, G, num_blocks, max_q_len, max_seqlen, tiles;
   float scale_log2;  // softmax scale * log2(e)
   int32_t* err;
+  int pair_rows;     // two-tile kernel: pair row tiles of one head (1) or heads (0)
 };
 
 // Byte address of 16-byte chunk `ch` of token row `tok` in a TMA-written
@@ -440,10 +440,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 // The same computation on the 5th-generation tensor cores, for D = 128, over
 // key blocks of 128 tokens (two cache pages): S = Q K^T (M 128, N 128) into
 // TMEM, the softmax warps write P as bf16 into TMEM, and O += P V takes P
-// from TMEM as its A operand. Two kernels: pair_kernel (two query heads of a
-// KV group per CTA, the tensor core alternating between their tiles) when the
-// group has an even number of heads, solo_kernel (one head per CTA, S and P
-// double-buffered) otherwise; both are described at their definitions. The
+// from TMEM as its A operand. pair_kernel (described at its definition) holds
+// two 128-row tiles per CTA, the tensor core alternating between them: two
+// query heads of a KV group over one row tile when the group has an even
+// number of heads, else two consecutive row tiles of one head. The
 // reference max m of a row changes (and O is rescaled in TMEM) only when the
 // row's max exceeds it by more than 2^8, so P stays <= 256 and O is rarely
 // touched. After the last block: O / l from TMEM to bf16 rows.
@@ -483,11 +483,15 @@ __device__ __forceinline__ float exp2_sfu(float x) {
 }
 
 // ------------------------------------------------------------------ two tiles per CTA
-// The same computation for two query heads h0 = 2x, h1 = 2x + 1 of one KV
-// group and one 128-row tile, over key blocks of 128 tokens (two cache pages).
-// Both tiles read the same K/V blocks (one load serves 256 query rows), and
-// the tensor core alternates between them: it computes one tile's P V and
-// next S while the other tile's softmax warps work.
+// The same computation for two 128-row query tiles of one KV group, over key
+// blocks of 128 tokens (two cache pages): either two query heads h0 = 2x,
+// h1 = 2x + 1 over one row tile (pair_rows = 0, the group has an even number
+// of heads) or one head over row tiles 2y and 2y + 1 (pair_rows = 1). Both
+// tiles read the same K/V blocks (one load serves 256 query rows), and the
+// tensor core alternates between them: it computes one tile's P V and next S
+// while the other tile's softmax warps work. With row pairs the two tiles see
+// different causal ends; the CTA loads K/V up to the later one, tile 0 stops
+// at its own end, and a tile past the chunk (an odd tile count) does nothing.
 //  * S_t = Q_t K_j^T: M 128, N 128 (both pages of block j), K 128, both
 //    operands in shared memory, into tile t's 128-column TMEM region;
 //  * P_t, bf16 with two keys per 32-bit column, overwrites the first 64
@@ -686,23 +690,41 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* mma_done = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
-  const int h0 = 2 * static_cast<int>(blockIdx.x);
-  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
+  // The CTA's two tiles: two heads of one KV group over the same row tile
+  // (p.pair_rows = 0), or two consecutive row tiles of one head (1), which
+  // share every key block of the first; longest work first.
+  int hd[2], i0s[2];
+  if (p.pair_rows) {
+    const int pr = (p.tiles + 1) / 2 - 1 - static_cast<int>(blockIdx.y);
+    hd[0] = hd[1] = static_cast<int>(blockIdx.x);
+    i0s[0] = 2 * pr * kRows;
+    i0s[1] = i0s[0] + kRows;
+  } else {
+    hd[0] = 2 * static_cast<int>(blockIdx.x);
+    hd[1] = hd[0] + 1;
+    i0s[0] = i0s[1] = (p.tiles - 1 - static_cast<int>(blockIdx.y)) * kRows;
+  }
   const int b = blockIdx.z;
-  const int g = h0 / p.G;
+  const int g = hd[0] / p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
 
   const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
   if (!c.ok) {
-    if (h0 == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
+    if (hd[0] == 0 && i0s[0] == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
     return;
   }
-  const int i0 = tile * kRows;
-  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
-  const int rows = min(kRows, c.n - i0);
-  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
+  if (i0s[0] >= c.n) return;  // before any barrier or TMEM allocation
+  // per tile: rows, keys [0, kend) it attends to, its key blocks (0 = no tile)
+  int rows_t[2], kend_t[2], nb_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    rows_t[t] = i0s[t] < c.n ? min(kRows, c.n - i0s[t]) : 0;
+    kend_t[t] = c.ctx + i0s[t] + rows_t[t];
+    nb_t[t] = rows_t[t] > 0 ? ((kend_t[t] + kPage - 1) / kPage + 1) / 2 : 0;
+  }
+  const int kend = max(kend_t[0], rows_t[1] > 0 ? kend_t[1] : 0);  // keys of the CTA
   const int npages = (kend + kPage - 1) / kPage;
   const int nblk = (npages + 1) / 2;
 
@@ -742,13 +764,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * Lay::kQBytes);
+      mbar_arrive_expect_tx(q_full, (rows_t[1] > 0 ? 2 : 1) * Lay::kQBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
+        if (rows_t[t] > 0) {
 #pragma unroll
-        for (int hf = 0; hf < H; ++hf)
-          tma_load_2d(smem + t * Lay::kQBytes + hf * (kRows * 128), &tmQ, q_full,
-                      (h0 + t) * D + hf * 64, c.t0 + i0);
+          for (int hf = 0; hf < H; ++hf)
+            tma_load_2d(smem + t * Lay::kQBytes + hf * (kRows * 128), &tmQ, q_full,
+                        hd[t] * D + hf * 64, c.t0 + i0s[t]);
+        }
       const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
       // One block = pages 2j and (if the key range reaches it) 2j + 1; a
       // missing second page leaves its rows stale: their keys are masked and
@@ -802,10 +826,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t dq0 = umma::smem_desc(smem_u32(smem));
       const uint64_t dk0 = umma::smem_desc(smem_u32(smem + Lay::kOffK));
       const uint64_t dv0 = smem_desc_mn(smem_u32(smem + Lay::kOffV), Lay::kHalf);
-      // S_j of tile t into its TMEM region (tile 0 first waits for the block)
+      // S_j of tile t into its TMEM region (the block's first user waits for it)
       auto issue_s = [&](int t, int j) -> bool {
         const int st = j % kKStages;
-        if (t == 0 && !mbar_wait(&k_full[st], (j / kKStages) & 1)) return false;
+        if ((t == 0 || j >= nb_t[0]) && !mbar_wait(&k_full[st], (j / kKStages) & 1)) return false;
         umma::tc_fence_after();
         const uint64_t dq = dq0 + static_cast<uint64_t>((t * Lay::kQBytes) >> 4);
         const uint64_t dk = dk0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
@@ -817,14 +841,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                           dk + ((hf * Lay::kHalf + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
         }
         umma::umma_commit(&s_full[t]);
-        if (t == 1) umma::umma_commit(&k_empty[st]);  // block j's K read by both tiles
         return true;
       };
       // O_t += P_j V_j once tile t's softmax has written P_j
       auto issue_pv = [&](int t, int j) -> bool {
         const int st = j % kVStages;
         if (!mbar_wait(&p_full[t], j & 1)) return false;
-        if (t == 0 && !mbar_wait(&v_full[st], (j / kVStages) & 1)) return false;
+        if ((t == 0 || j >= nb_t[0]) && !mbar_wait(&v_full[st], (j / kVStages) & 1)) return false;
         umma::tc_fence_after();
         const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
         const uint32_t a_tmem = tmem + t * kBlk;
@@ -834,15 +857,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           umma_bf16_ts(d_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdPV,
                        (j > 0 || kk > 0) ? 1u : 0u);
         umma::umma_commit(&pv_done[t]);
-        if (t == 1) umma::umma_commit(&v_empty[st]);  // block j's V read by both tiles
         return true;
       };
-      if (ok) ok = issue_s(0, 0) && issue_s(1, 0);
+      // a block's K (V) stage is released after the S (P V) of every tile
+      // that reads it
+      if (ok) ok = issue_s(0, 0) && (nb_t[1] == 0 || issue_s(1, 0));
+      if (ok) umma::umma_commit(&k_empty[0]);
       for (int j = 0; ok && j < nblk; ++j) {
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (ok && !issue_pv(t, j)) ok = false;
-          if (ok && j + 1 < nblk && !issue_s(t, j + 1)) ok = false;
+          if (ok && j < nb_t[t] && !issue_pv(t, j)) ok = false;
+          if (ok && j + 1 < nb_t[t] && !issue_s(t, j + 1)) ok = false;
+        }
+        if (ok) {
+          umma::umma_commit(&v_empty[j % kVStages]);
+          if (j + 1 < nblk) umma::umma_commit(&k_empty[(j + 1) % kKStages]);
         }
       }
       if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
@@ -854,13 +883,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int t = warp >= 6 ? 1 : 0;  // the tile this warp serves
     const int quarter = warp & 3;     // this warp may access TMEM lanes 32 quarter .. + 31
     const int r = quarter * 32 + lane;
+    const int i0 = i0s[t], rows = rows_t[t], tnb = nb_t[t];
     const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t t_s = t_lane + t * kBlk;             // S / P of this tile
     const uint32_t t_o = t_lane + kPairOCol + t * D;    // O of this tile
     float m_ref = kNegInf, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
+    for (int j = 0; j < tnb; ++j) {
       const int kbase = j * kBlk;
       // S_j landed; every earlier MMA of this CTA (P_{j-1} V_{j-1} included)
       // has completed with it.
@@ -957,11 +987,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       tmem_wait_st();
       l = fmaf(l, alpha, sum[0] + sum[1]);
 
-      // Keys at or past kend in the last block hold other tokens' bytes (or
-      // stale rows where the block has one page): their weights are 0, and
-      // their V rows are zeroed, as 0 * NaN would still be NaN in the
-      // accumulator. Both tiles' warps clear the same rows (the same zero
-      // bytes), each before its own P is published.
+      // Keys at or past the CTA's kend in its last block hold other tokens'
+      // bytes (or stale rows where the block has one page): their weights
+      // are 0, and their V rows are zeroed, as 0 * NaN would still be NaN in
+      // the accumulator. Every tile that reads that block clears the same
+      // rows (the same zero bytes) before its own P is published. (Keys a
+      // first row tile masks inside the CTA's range are its partner's
+      // tokens: zero weights on finite values.)
       if (kbase + kBlk > kend) {
         const int sv = j % kVStages;
         if (!mbar_wait_warp(&v_full[sv], (j / kVStages) & 1)) {  // the block has landed
@@ -982,11 +1014,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok) ok = mbar_wait_warp(&pv_done[t], (nblk - 1) & 1);
-    if (ok) {
+    if (ok && tnb > 0) ok = mbar_wait_warp(&pv_done[t], (tnb - 1) & 1);
+    if (tnb == 0) {
+      // no tile here (a last row tile past the chunk): nothing to store
+    } else if (ok) {
       umma::tc_fence_after();
       __nv_bfloat16* orow = p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t +
-                            (h0 + t) * D;
+                            hd[t] * D;
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         float o[32];
@@ -1006,398 +1040,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kPairTmemCols)
-                 : "memory");
-  }
-}
-
-// ------------------------------------------------------------------ one tile per CTA
-// One query head and one 128-row tile per CTA (any number of query heads per
-// KV head), over key blocks of 128 tokens. S and P are double-buffered in
-// TMEM, so S of block j + 1 is computed while the softmax warps work on
-// block j; P_j (bf16 pairs) is the A operand of O += P_j V_j. Each query row
-// is shared by two softmax warps, one per 64-key half of the block (eight
-// softmax warps, two per SM sub-partition, so that one hides the other's
-// latencies): both read the whole S row for its maximum (the same bits, so
-// the same decisions), each writes the weights of its half, keeps its own
-// row sum, and owns half of O's columns for a rescale and the division.
-// Warp 0: TMA producer (Q once; K and V blocks through 3-stage rings);
-// warp 1: MMA issuer (S_0, S_1, then per block j: P_j V_j and S_{j+2} into
-// the S buffer block j used -- MMAs of one thread run in order, and the
-// softmax warps have read S_j before publishing P_j);
-// warps 2-9: softmax, half h = (warp - 2) / 4, TMEM lane quarter warp % 4.
-// TMEM: S buffers at columns [0, 128) and [128, 256), O at [256, 384), P
-// buffers at [384, 448) and [448, 512).
-
-constexpr int kSoloThreads = 320;
-constexpr uint32_t kSoloTmemCols = 512;
-constexpr int kSoloStages = 3;          // K and V block rings
-constexpr uint32_t kSoloOCol = 256;
-constexpr uint32_t kSoloPCol = 384;
-
-template <int D>
-struct SoloLayout {
-  static constexpr int kQBytes = kRows * D * 2;
-  static constexpr int kBlkBytes = kBlk * D * 2;
-  static constexpr int kHalf = kBlk * 128;
-  static constexpr int kOffK = kQBytes;
-  static constexpr int kOffV = kOffK + kSoloStages * kBlkBytes;
-  static constexpr int kOffX = kOffV + kSoloStages * kBlkBytes;  // [2 halves][128] row sums
-  static constexpr int kOffBar = kOffX + 2 * kRows * 4;
-  static constexpr int kNumBars = 1 + 4 * kSoloStages + 3 * 2 + 2;
-  static constexpr size_t kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kSoloThreads, 1)
-    solo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using Lay = SoloLayout<D>;
-  constexpr int H = D / 64;
-  constexpr float kNegInf = -INFINITY;
-  static_assert(D == 128, "the one-tile prefill kernel is built for head_dim 128");
-  static_assert(SoloLayout<D>::kSmem <= 227 * 1024, "shared memory budget");
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  float* xl = reinterpret_cast<float*>(smem + Lay::kOffX);  // [half][row] row sums
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + 1;
-  uint64_t* k_empty = k_full + kSoloStages;
-  uint64_t* v_full = k_empty + kSoloStages;
-  uint64_t* v_empty = v_full + kSoloStages;
-  uint64_t* s_full = v_empty + kSoloStages;  // [buffer] S_j landed (and every earlier S / P V)
-  uint64_t* p_full = s_full + 2;             // [buffer] P_j written (8 softmax warps)
-  uint64_t* pv_done = p_full + 2;            // [buffer] O += P_j V_j completed
-  uint64_t* mma_done = pv_done + 2;
-  uint64_t* l_ready = mma_done + 1;          // both halves' row sums written (8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_ready + 1);
-
-  const int h = blockIdx.x;
-  const int tile = p.tiles - 1 - static_cast<int>(blockIdx.y);  // longest tiles first
-  const int b = blockIdx.z;
-  const int g = h / p.G;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();
-  pdl_trigger();
-
-  const Chunk c = load_chunk(p.cu_seqlens, p.ctx_lens, b, p.T, p.max_q_len, p.max_seqlen);
-  if (!c.ok) {
-    if (h == 0 && tile == 0 && threadIdx.x == 0) set_err(p.err, DF_DEVERR_SEQLEN);
-    return;
-  }
-  const int i0 = tile * kRows;
-  if (i0 >= c.n) return;  // before any barrier or TMEM allocation
-  const int rows = min(kRows, c.n - i0);
-  const int kend = c.ctx + i0 + rows;  // keys [0, kend) serve this tile
-  const int npages = (kend + kPage - 1) / kPage;
-  const int nblk = (npages + 1) / 2;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < kSoloStages; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);
-      mbar_init(&pv_done[i], 1);
-    }
-    mbar_init(mma_done, 1);
-    mbar_init(l_ready, 8);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kSoloTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  umma::tc_fence_before();
-  __syncthreads();
-  umma::tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, Lay::kQBytes);
-#pragma unroll
-      for (int hf = 0; hf < H; ++hf)
-        tma_load_2d(smem + hf * (kRows * 128), &tmQ, q_full, h * D + hf * 64, c.t0 + i0);
-      const int32_t* tbl = p.block_table + static_cast<int64_t>(b) * p.max_blocks_per_seq;
-      // one block = pages 2j and (if the key range reaches it) 2j + 1; a
-      // missing second page leaves stale rows: masked keys, cleared V rows
-      auto load_block = [&](const CUtensorMap* tm, uint64_t* bar, uint8_t* dst, int j) {
-        const int np = min(2, npages - 2 * j);
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(np * H * kPage * 128));
-        for (int q = 0; q < np; ++q) {
-          int page = tbl[2 * j + q];
-          if (page < 0 || page >= p.num_blocks) {  // flagged; page 0 stands in (outputs invalid)
-            set_err(p.err, DF_DEVERR_BLOCK);
-            page = 0;
-          }
-          const int row = (page * p.Hkv + g) * kPage;
-#pragma unroll
-          for (int hf = 0; hf < H; ++hf)
-            tma_load_2d(dst + hf * Lay::kHalf + q * (kPage * 128), tm, bar, hf * 64, row);
-        }
-      };
-      int issued = 0;
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j % kSoloStages;
-        if (j >= kSoloStages && !mbar_wait(&k_empty[st], ((j / kSoloStages) - 1) & 1)) {
-          set_err(p.err, DF_DEVERR_TIMEOUT);
-          break;
-        }
-        load_block(&tmK, &k_full[st], smem + Lay::kOffK + st * Lay::kBlkBytes, j);
-        if (j >= kSoloStages && !mbar_wait(&v_empty[st], ((j / kSoloStages) - 1) & 1)) {
-          set_err(p.err, DF_DEVERR_TIMEOUT);
-          mbar_wait(&k_full[st], (j / kSoloStages) & 1);  // the K block issued above
-          break;
-        }
-        load_block(&tmV, &v_full[st], smem + Lay::kOffV + st * Lay::kBlkBytes, j);
-        ++issued;
-      }
-      // Leave no copy in flight (bounded waits).
-      mbar_wait(q_full, 0);
-      for (int j = issued > kSoloStages ? issued - kSoloStages : 0; j < issued; ++j) {
-        mbar_wait(&k_full[j % kSoloStages], (j / kSoloStages) & 1);
-        mbar_wait(&v_full[j % kSoloStages], (j / kSoloStages) & 1);
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = umma::make_idesc(kRows, kBlk);
-      constexpr uint32_t kIdPV = umma::make_idesc(kRows, D) | (1u << 16);  // V MN-major
-      bool ok = mbar_wait(q_full, 0);
-      const uint64_t dq = umma::smem_desc(smem_u32(smem));
-      const uint64_t dk0 = umma::smem_desc(smem_u32(smem + Lay::kOffK));
-      const uint64_t dv0 = smem_desc_mn(smem_u32(smem + Lay::kOffV), Lay::kHalf);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kSoloStages;
-        if (!mbar_wait(&k_full[st], (j / kSoloStages) & 1)) return false;
-        umma::tc_fence_after();
-        const uint64_t dk = dk0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
-        const uint32_t d_tmem = tmem + (j & 1) * kBlk;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int hf = kk >> 2, kq = kk & 3;
-          umma::umma_bf16(d_tmem, dq + ((hf * (kRows * 128) + kq * 32) >> 4),
-                          dk + ((hf * Lay::kHalf + kq * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
-        }
-        umma::umma_commit(&s_full[j & 1]);
-        umma::umma_commit(&k_empty[st]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && nblk > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int st = j % kSoloStages, bb = j & 1;
-        if (!mbar_wait(&p_full[bb], (j >> 1) & 1) ||
-            !mbar_wait(&v_full[st], (j / kSoloStages) & 1)) {
-          ok = false;
-          break;
-        }
-        umma::tc_fence_after();
-        const uint64_t dv = dv0 + static_cast<uint64_t>((st * Lay::kBlkBytes) >> 4);
-        const uint32_t a_tmem = tmem + kSoloPCol + bb * (kBlk / 2);
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          umma_bf16_ts(tmem + kSoloOCol, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdPV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-        umma::umma_commit(&pv_done[bb]);
-        umma::umma_commit(&v_empty[st]);
-        if (j + 2 < nblk && !issue_s(j + 2)) ok = false;
-      }
-      if (!ok) set_err(p.err, DF_DEVERR_TIMEOUT);
-      umma::umma_commit(mma_done);  // completes when every MMA issued above has
-      mbar_wait(mma_done, 0);
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax warps
-    const int hh = (warp - 2) >> 2;   // key half of each block this warp serves
-    const int quarter = warp & 3;     // TMEM lanes 32 quarter .. + 31
-    const int r = quarter * 32 + lane;
-    const int pos = c.ctx + min(i0 + r, c.n - 1);  // a padding row repeats the last real row
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t t_o = t_lane + kSoloOCol + hh * 64;  // this half's 64 columns of O
-    float m_ref = kNegInf, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      const int bb = j & 1;
-      const int kbase = j * kBlk + hh * 64;
-      if (!mbar_wait_warp(&s_full[bb], (j >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      umma::tc_fence_after();
-      const uint32_t t_s = t_lane + bb * kBlk;                       // S_j, both halves
-      const uint32_t t_p = t_lane + kSoloPCol + bb * (kBlk / 2) + hh * 32;  // this half's P
-      // the other half first, for the row maximum only
-      float omax;
-      {
-        uint32_t rr[64];
-        tmem_ld64_wait(t_s + (hh ^ 1) * 64, rr);
-        const int obase = j * kBlk + (hh ^ 1) * 64;
-        float mo[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mo[q] = obase + q > pos ? kNegInf : __uint_as_float(rr[q]);
-#pragma unroll
-        for (int k = 8; k < 64; k += 16) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float x0 = obase + k + q > pos ? kNegInf : __uint_as_float(rr[k + q]);
-            const float x1 = obase + k + 8 + q > pos ? kNegInf : __uint_as_float(rr[k + 8 + q]);
-            mo[q] = max3f(mo[q], x0, x1);
-          }
-        }
-        omax = fmaxf(max3f(mo[0], mo[1], mo[2]), max3f(max3f(mo[3], mo[4], mo[5]), mo[6], mo[7]));
-      }
-      float s[64];
-      {
-        uint32_t rr[64];
-        tmem_ld64_wait(t_s + hh * 64, rr);
-#pragma unroll
-        for (int k = 0; k < 64; ++k) s[k] = __uint_as_float(rr[k]);
-      }
-      if (kbase + 63 > pos) {  // causal mask (and keys past the chunk end)
-#pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (kbase + k > pos) s[k] = kNegInf;
-      }
-      float mx[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mx[q] = s[q];
-#pragma unroll
-      for (int k = 8; k < 64; k += 16) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx[q] = max3f(mx[q], s[k + q], s[k + 8 + q]);
-      }
-      // the row's maximum over both halves: the same value in both warps
-      const float m_cand =
-          max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), max3f(mx[6], mx[7], omax)) *
-          p.scale_log2;
-      const bool rescale = (m_ref != kNegInf) && (m_cand > m_ref + kRescaleLog2);
-      float alpha = 1.f;
-      if (m_ref == kNegInf) {
-        m_ref = m_cand;  // first block: O holds nothing yet
-      } else if (rescale) {
-        alpha = exp2f(m_ref - m_cand);
-        m_ref = m_cand;
-      }
-      const float mu = (m_ref == kNegInf) ? 0.f : m_ref;
-
-      const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-      const uint64_t nmu2 = f2_pack(-mu, -mu);
-      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t w[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint64_t x2 = f2_fma(f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2, nmu2);
-          uint64_t e2;
-          if (poly_pair(k)) {
-            e2 = exp2_poly2(x2);
-          } else {
-            float xa, xb;
-            f2_unpack(x2, xa, xb);
-            e2 = f2_pack(exp2_sfu(xa), exp2_sfu(xb));
-          }
-          sum2[k & 3] = f2_add(sum2[k & 3], e2);
-          float a, a2;
-          f2_unpack(e2, a, a2);
-          w[k] = pack_f32_bf16x2(a, a2);
-        }
-        tmem_st16(t_p + 16 * q, w);
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled in place
-        if (!mbar_wait_warp(&pv_done[bb ^ 1], ((j - 1) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        umma::tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < 64; cc += 32) {
-          float o[32];
-          umma::tmem_ld<32>(t_o + cc, o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= alpha;
-          tmem_st32(t_o + cc, o);
-        }
-      }
-      tmem_wait_st();
-      {
-        float e[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) f2_unpack(sum2[i], e[2 * i], e[2 * i + 1]);
-        l = fmaf(l, alpha, ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7])));
-      }
-      // Keys at or past kend in the last block: zero weights, and their V
-      // rows cleared (0 * NaN would still be NaN); every softmax thread
-      // clears its share before the block's P is published.
-      if (j * kBlk + kBlk > kend) {
-        const int st = j % kSoloStages;
-        if (!mbar_wait_warp(&v_full[st], (j / kSoloStages) & 1)) {
-          ok = false;
-          break;
-        }
-        const int kend_rel = kend - j * kBlk;
-        uint8_t* sV = smem + Lay::kOffV + st * Lay::kBlkBytes;
-        const int nvec = (kBlk - kend_rel) * H * 8;
-        for (int v = hh * kRows + r; v < nvec; v += 2 * kRows) {
-          const int row = kend_rel + v / (H * 8), hf = (v / 8) % H, ch = v % 8;
-          *reinterpret_cast<uint4*>(sV + hf * Lay::kHalf + row * 128 + ch * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-      umma::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[bb]);
-    }
-    if (ok) ok = mbar_wait_warp(&pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1);
-    // the row sum over both halves (every warp publishes its own, even after
-    // a failed wait, so that its partner's bounded wait ends)
-    xl[hh * kRows + r] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(l_ready);
-    if (ok) ok = mbar_wait_warp(l_ready, 0);
-    if (ok) {
-      l += xl[(hh ^ 1) * kRows + r];
-      umma::tc_fence_after();
-      __nv_bfloat16* orow =
-          p.o1 + static_cast<int64_t>(c.t0 + i0 + min(r, rows - 1)) * p.o_stride_t + h * D + hh * 64;
-#pragma unroll
-      for (int cc = 0; cc < 64; cc += 32) {
-        float o[32];
-        umma::tmem_ld<32>(t_o + cc, o);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) o[k] = o[k] / l;
-        if (r < rows) umma::store_bf16<32>(orow + cc, o);
-      }
-    } else if (lane == 0) {
-      set_err(p.err, DF_DEVERR_TIMEOUT);
-    }
-  }
-
-  umma::tc_fence_before();
-  __syncthreads();
-  umma::tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kSoloTmemCols)
                  : "memory");
   }
 }
@@ -1451,21 +1093,17 @@ cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* t
 
 // Two query heads of one KV group per CTA when the group has an even number
 // of heads (both tiles then read the same pages), else one head per CTA.
-cudaError_t launch_attn_tc(const AttnParams& p, int Hq, int B, const CUtensorMap* tmQ,
+cudaError_t launch_attn_tc(AttnParams p, int Hq, int B, const CUtensorMap* tmQ,
                            const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
-  if (p.G % 2 == 0) {
-    constexpr size_t smem2 = tc::PairLayout<128>::kSmem;
-    cudaError_t e2 =
-        ensure_dynamic_smem(reinterpret_cast<const void*>(tc::pair_kernel<128>), smem2);
-    if (e2 != cudaSuccess) return e2;
-    return launch_pdl(tc::pair_kernel<128>, dim3(Hq / 2, p.tiles, B), dim3(tc::kPairThreads),
-                      smem2, stream, *tmQ, *tmK, *tmV, p);
-  }
-  constexpr size_t smem = tc::SoloLayout<128>::kSmem;
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::solo_kernel<128>), smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(tc::solo_kernel<128>, dim3(Hq, p.tiles, B), dim3(tc::kSoloThreads), smem, stream,
-                    *tmQ, *tmK, *tmV, p);
+  constexpr size_t smem2 = tc::PairLayout<128>::kSmem;
+  cudaError_t e2 = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::pair_kernel<128>), smem2);
+  if (e2 != cudaSuccess) return e2;
+  // two query heads of a KV group per CTA when the group has an even number
+  // of heads, else two consecutive row tiles of one head
+  p.pair_rows = p.G % 2 == 0 ? 0 : 1;
+  const dim3 grid = p.pair_rows ? dim3(Hq, (p.tiles + 1) / 2, B) : dim3(Hq / 2, p.tiles, B);
+  return launch_pdl(tc::pair_kernel<128>, grid, dim3(tc::kPairThreads), smem2, stream, *tmQ, *tmK,
+                    *tmV, p);
 }
 
 // Workspace of the auxiliary step: the decode workspace (its arrival counters
@@ -1590,7 +1228,7 @@ extern "C" df_status dualflow_prefill_ex(
   if (!encode_tmap_bf16_2d(&tmK, k_cache, rows, D, D * 2, kPage, 64) ||
       !encode_tmap_bf16_2d(&tmV, v_cache, rows, D, D * 2, kPage, 64))
     return DF_ERR_CUDA;
-  AttnParams p;
+  AttnParams p{};
   p.q1 = static_cast<const __nv_bfloat16*>(q1);
   p.q_stride_t = qs;
   p.block_table = block_table;
