@@ -74,6 +74,11 @@ KERNELS = ["mma_sync", "tcgen05"]
     (4, 4, 128, (256, 129), (0, 0)),                   # MHA, fresh prompts
     (6, 2, 128, (64, 128, 191), (1, 63, 0)),           # G = 3
     (8, 2, 128, (127, 128, 129, 300), (0, 5, 200, 64)),  # 128-row tile edges
+    # odd groups: the tcgen05 kernel pairs row tiles 2y, 2y + 1 of one head
+    # (different causal ends; 3 tiles leave the second tile of the last pair
+    # empty)
+    (2, 2, 128, (300, 129, 384), (70, 0, 5)),          # MHA, 3 row tiles, prefixes
+    (3, 1, 128, (200, 260, 385), (0, 130, 0)),         # G = 3, 4 row tiles (last: 1 row)
 ])
 def test_prefill_matches_oracle(cuda_device, Hq, Hkv, D, lengths, ctx, kernel):
     if kernel == "tcgen05" and D != 128:
@@ -219,17 +224,20 @@ def test_launch_count():
 
 
 @pytest.mark.slow
-def test_full_size_prefill_sampled_rows(cuda_device):
-    """The timed workload (16 prompts of 4096 tokens, 32/8 heads, D 128):
-    every row of the cache written bit-exactly is checked on sampled tokens,
-    and sampled output rows against the oracle's attention of that row."""
-    inp = synth.make_prefill_inputs(W)
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (32, 32), (24, 8)])
+def test_full_size_prefill_sampled_rows(cuda_device, Hq, Hkv):
+    """The timed workload (16 prompts of 4096 tokens, D 128; 32/8 heads, and
+    the odd groups of MHA and G = 3 that pair row tiles): every row of the
+    cache written bit-exactly is checked on sampled tokens, and sampled
+    output rows against the oracle's attention of that row."""
+    w = _w(Hq=Hq, Hkv=Hkv)
+    inp = synth.make_prefill_inputs(w)
     d = _dev(inp, cuda_device)
     o1, o2 = _run(d)   # automatic choice: the tcgen05 kernel at these sizes
     kc, vc = d["k_cache"].cpu(), d["v_cache"].cpu()
     tbl, cu = inp["block_table"], inp["cu_seqlens"].tolist()
-    G = W.Hq // W.Hkv
-    scale = 1.0 / math.sqrt(W.D)
+    G = w.Hq // w.Hkv
+    scale = 1.0 / math.sqrt(w.D)
     rng = np.random.default_rng(0)
     for b in (0, 7, 15):
         t0, n = cu[b], cu[b + 1] - cu[b]
@@ -238,7 +246,7 @@ def test_full_size_prefill_sampled_rows(cuda_device):
             page, slot = int(tbl[b, i // 64]), i % 64
             assert torch.equal(kc[page, :, slot], inp["k_new"][t])
             assert torch.equal(vc[page, :, slot], inp["v_new"][t])
-            for h in (0, 13, 31):
+            for h in (0, 13, w.Hq - 1):
                 g = h // G
                 K = f32(inp["k_new"][t0:t + 1, g])
                 V = f32(inp["v_new"][t0:t + 1, g])
@@ -247,7 +255,7 @@ def test_full_size_prefill_sampled_rows(cuda_device):
         last = t0 + n - 1
         q2 = oracle.couple_query(f32(inp["q1"][last])[None], f32(inp["q2raw"][b])[None],
                                  f32(inp["a"]))[0]
-        for h in (0, 31):
+        for h in (0, w.Hq - 1):
             g = h // G
             K = f32(inp["k_new"][t0:last + 1, g])
             V = f32(inp["v_new"][t0:last + 1, g])
