@@ -257,6 +257,55 @@ def rank_seed(base, rank):
     return base + 1000 * rank
 
 
+def workload_config(name, w, host, world=1):
+    """The workload as both arms name it in their JSON lines: its sizes and
+    whether its inputs exceed L2, from the workload and its host inputs alone
+    (no device, no library). How this build runs it goes under "path"."""
+    if name == "layer":
+        L = w.cache_len + 1
+        kv = w.B * L * w.Hkv * w.D * 2 * 2
+        cfg = {"workload": "dual-flow decoder layer step: d_model %d, %d/%d heads, head_dim %d, "
+                           "SwiGLU %d, batch %d per flow (M=%d), cache %d+1"
+                           % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
+               "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
+               "attended": L,
+               "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
+                     % (kv / 1e9, 436207616 / 1e9)}
+    elif name == "mixture":
+        B, V, d = w.B, w.V, w.d_model
+        cfg = {"workload": "dual-flow mixture head: LM-head projection of both flows (batch %d "
+                           "per flow, M=%d, d_model %d, vocabulary %d, bf16 weights %.1f MB) + "
+                           "mixed next-token distribution (fp32)"
+                           % (B, 2 * B, d, V, V * d * 2 / 1e6),
+               "l2": "inputs larger than L2 (%.0f MB of weights per step)" % (V * d * 2 / 1e6)}
+    elif name == "moe":
+        B, d, F, E = w.B, w.d_model, w.F, w.E
+        cfg = {"workload": "dual-flow MoE MLP block with router replay: %d tokens per flow, "
+                           "d_model %d, %d SwiGLU experts of width %d, primary top-%d, auxiliary "
+                           "fan-out %d (%.1f MB of expert weights)"
+                           % (B, d, E, F, w.k, w.k_aux, E * 3 * F * d * 2 / 1e6),
+               "l2": "inputs larger than L2 (%.0f MB of expert weights per step)"
+                     % (E * 3 * F * d * 2 / 1e6)}
+    elif name == "prefill":
+        cfg = {"workload": "dual-flow primary prefill: %d fresh prompts of %d..%d tokens, %d/%d "
+                           "heads, head_dim %d, bf16, 64-token pages in a random block table, "
+                           "auxiliary query at each last position"
+                           % (host["B"], w.len_lo, w.len_hi, w.Hq, w.Hkv, w.D),
+               "l2": "inputs larger than L2 (%.0f MB of queries, %.0f MB of new K/V)"
+                     % (host["q1"].numel() * 2 / 1e6, 2 * host["k_new"].numel() * 2 / 1e6)}
+    else:
+        esize = 4 if w.dtype == "fp32" else 2
+        kv = int(host["seqlens"].sum()) * w.Hkv * w.D * 2 * esize
+        cfg = {"workload": "dual-flow decode attention '%s': batch %d, %d/%d heads, head_dim %d, "
+                           "%s, lengths %d..%d%s" % (
+                               name, w.B, w.Hq, w.Hkv, w.D, w.dtype, w.len_lo, w.len_hi,
+                               ", random block table" if w.random_table else ""),
+               "l2": "inputs larger than L2" if kv > 126e6
+                     else "inputs smaller than L2 (not flushed)"}
+    cfg["parallelism"] = "replicas" if world > 1 else "single GPU"
+    return cfg
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -307,18 +356,13 @@ class LayerRun:
         self.kv_bytes = w.B * L * w.Hkv * w.D * 2 * 2
         self.units = w.B * w.Hkv * L  # (sequence, KV head, token) units per attention launch
         self.bytes_per_unit = w.D * 2 * 2
-        self.config = {"workload": "dual-flow decoder layer step: d_model %d, %d/%d heads, "
-                                   "head_dim %d, SwiGLU %d, batch %d per flow (M=%d), cache %d+1"
-                                   % (w.d_model, w.Hq, w.Hkv, w.D, w.F, w.B, 2 * w.B, w.cache_len),
-                       "batch_per_flow": w.B, "rows": 2 * w.B, "cache_len": w.cache_len,
-                       "attended": L, "attn_launches": self.layer.attn_launches,
-                       "pre_attention": ("one launch, reduced in the attention launch"
-                                         if self.layer.split_pre else "one launch")
-                                        if self.layer.fused_pre else "three launches",
-                       "post_attention": "one persistent launch" if self.layer.fused_post
-                                         else "four launches",
-                       "l2": "inputs larger than L2 (KV %.2f GB + weights %.2f GB read per step)"
-                             % (self.kv_bytes / 1e9, 436207616 / 1e9)}
+        self.config = workload_config("layer", w, self.host)
+        self.path = {"attn_launches": self.layer.attn_launches,
+                     "pre_attention": ("one launch, reduced in the attention launch"
+                                       if self.layer.split_pre else "one launch")
+                                      if self.layer.fused_pre else "three launches",
+                     "post_attention": "one persistent launch" if self.layer.fused_post
+                                       else "four launches"}
         self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"
 
     def step(self, timers=None):
@@ -387,13 +431,8 @@ class AttnRun:
         self.kv_bytes = tot * w.Hkv * w.D * 2 * esize
         self.units = tot * w.Hkv
         self.bytes_per_unit = w.D * 2 * esize
-        self.config = {"workload": "dual-flow decode attention '%s': batch %d, %d/%d heads, "
-                                   "head_dim %d, %s, lengths %d..%d%s" % (
-                                       name, w.B, w.Hq, w.Hkv, w.D, w.dtype, w.len_lo, w.len_hi,
-                                       ", random block table" if w.random_table else ""),
-                       "attn_launches": n_attn,
-                       "l2": "inputs larger than L2" if self.kv_bytes > 126e6
-                             else "inputs smaller than L2 (not flushed)"}
+        self.config = workload_config(name, w, self.host)
+        self.path = {"attn_launches": n_attn}
         self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"
         # CUDA graphs: [append] and [attention], replayed every step
         self._append()
@@ -498,12 +537,8 @@ class MixtureRun:
         self.dom_bytes = V * d * 2 + 2 * B * d * 2 + 2 * B * V * 2
         # mixture kernel: logits read once, p_mix and alpha written once
         self.mix_bytes = 2 * B * V * 2 + B * V * 4 + B * 4
-        self.config = {"workload": "dual-flow mixture head: LM-head projection of both flows "
-                                   "(batch %d per flow, M=%d, d_model %d, vocabulary %d, bf16 "
-                                   "weights %.1f MB) + mixed next-token distribution (fp32)"
-                                   % (B, 2 * B, d, V, V * d * 2 / 1e6),
-                       "l2": "inputs larger than L2 (%.0f MB of weights per step)"
-                             % (V * d * 2 / 1e6)}
+        self.config = workload_config("mixture", w, self.host)
+        self.path = {}
         self.dominant = "dualflow_grouped_proj (LM head, tcgen05)"
         self._proj()
         self._mix()
@@ -578,12 +613,8 @@ class MoERun:
         self.bytes_per_unit = 3 * F * d * 2
         rows = 2 * api.MOE_ROWS
         self.dom_bytes = E * (self.bytes_per_unit + rows * d * 2 + rows * F * 2 * 2 + rows * d * 2)
-        self.config = {"workload": "dual-flow MoE MLP block with router replay: %d tokens per "
-                                   "flow, d_model %d, %d SwiGLU experts of width %d, primary "
-                                   "top-%d, auxiliary fan-out %d (%.1f MB of expert weights)"
-                                   % (B, d, E, F, w.k, w.k_aux, E * 3 * F * d * 2 / 1e6),
-                       "l2": "inputs larger than L2 (%.0f MB of expert weights per step)"
-                             % (E * 3 * F * d * 2 / 1e6)}
+        self.config = workload_config("moe", w, self.host)
+        self.path = {}
         self.dominant = "dualflow_grouped_proj (expert SwiGLU projections, tcgen05)"
         self._all()
         torch.cuda.synchronize()
@@ -676,17 +707,12 @@ class PrefillRun:
         self.units = w.Hq * pairs                  # (query row, visible key) pairs, all heads
         self.flops_per_unit = 4 * w.D              # q.k and p*v, multiply-add each
         self.dom_flops = self.units * self.flops_per_unit
-        self.config = {"workload": "dual-flow primary prefill: %d fresh prompts of %d..%d tokens, "
-                                   "%d/%d heads, head_dim %d, bf16, 64-token pages in a random "
-                                   "block table, auxiliary query at each last position"
-                                   % (h["B"], w.len_lo, w.len_hi, w.Hq, w.Hkv, w.D),
-                       "l2": "inputs larger than L2 (%.0f MB of queries, %.0f MB of new K/V)"
-                             % (h["q1"].numel() * 2 / 1e6, 2 * h["k_new"].numel() * 2 / 1e6)}
+        self.config = workload_config("prefill", w, h)
         kern = api.prefill_kernel(w.D, h["T"], self.o1, w.Hq)
         self.dominant = ("dualflow_prefill attention kernel (%s)"
                          % ("tcgen05, TMEM accumulators" if kern == "tcgen05"
                             else "mma.sync, TMA page ring"))
-        self.config["attn_kernel"] = kern
+        self.path = {"attn_kernel": kern}
         self._full()
         torch.cuda.synchronize()
         self.g_full, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
@@ -964,13 +990,13 @@ def run_reference(args):
     if args.workload in ("mixture", "moe", "prefill"):
         h.w = synth.WORKLOADS[args.workload]
         if args.workload == "mixture":
-            h.host = synth.make_mixture_inputs(h.w)
+            h.host = synth.make_mixture_inputs(h.w, seed=synth_seed(args.workload))
             v, sample, el, steps = time_oracle_mixture(h.host, 20.0)
         elif args.workload == "prefill":
-            h.host = synth.make_prefill_inputs(h.w)
+            h.host = synth.make_prefill_inputs(h.w, seed=synth_seed(args.workload))
             v, sample, el, steps = time_oracle_prefill(h.host, 20.0)
         else:
-            h.host = synth.make_moe_inputs(h.w)
+            h.host = synth.make_moe_inputs(h.w, seed=synth_seed(args.workload))
             v, sample, el, steps = time_oracle_moe(h.host, 20.0)
         line = {"impl": "reference",
                 "metric": PREFILL_METRIC if args.workload == "prefill" else METRIC,
@@ -978,7 +1004,7 @@ def run_reference(args):
                 "n_gpus": world, "steps": steps, "steps_requested": args.steps,
                 "warmup": args.warmup, "ms_per_step": el / steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": args.workload},
+                "config": workload_config(args.workload, h.w, h.host, world),
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads_used(),
                                  "kind": "oracle", "sample": sample},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -987,10 +1013,10 @@ def run_reference(args):
         return 0
     if args.workload == "layer":
         h.w = synth.WORKLOADS["layer"]
-        h.host = synth.make_layer_inputs(h.w)
+        h.host = synth.make_layer_inputs(h.w, seed=synth_seed(args.workload))
     else:
         h.w = synth.WORKLOADS[args.workload]
-        h.host = synth.make_attn_inputs(h.w)
+        h.host = synth.make_attn_inputs(h.w, seed=synth_seed(args.workload))
     import oracle
     budget = 150.0
     if args.workload == "layer":
@@ -1028,7 +1054,7 @@ def run_reference(args):
             "n_gpus": world, "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
             "ms_per_step": el / steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload},
+            "config": workload_config(args.workload, h.w, h.host, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -1189,6 +1215,7 @@ def main(argv=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations/cache, N(0,0.02) weights, N(0,0.1) couplings)",
         "config": dict(run.config, parallelism="replicas" if world > 1 else "single GPU"),
+        "path": run.path,
         "dominant_ms_per_launch": attn_ms,
         "kernel_timing": "second pass of the same %d steps, the timed kernels' graphs bracketed "
                          "by CUDA events on the launching stream (value uses the single-graph "

@@ -56,3 +56,21 @@ def test_clock_record_without_samples_says_so():
 def test_clock_record_maps_slowdown_bits():
     rec = _sampler(["1.0 1500 104"], 0.0, 2.0).stop()  # 0x40 | 0x20 | 0x8
     assert rec["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_reference_arm_names_the_same_workload_config(capsys, monkeypatch):
+    """Both arms print the same `config` object: the reference arm builds it
+    with the same function, from the same seeded host inputs, that the
+    CUDA arm uses (sizes and the L2 note only; no device needed)."""
+    import json
+    from dual_flow_transformer_b200 import synth
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.delenv("RANK", raising=False)
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "2",
+                             "--warmup", "3"])
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    w = synth.WORKLOADS["tiny"]
+    host = synth.make_attn_inputs(w, seed=bench.synth_seed("tiny"))
+    assert line["config"] == bench.workload_config("tiny", w, host)
+    assert line["impl"] == "reference" and line["config"]["parallelism"] == "single GPU"
