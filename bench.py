@@ -66,6 +66,10 @@ def parse_args(argv=None):
                     help="layer workload, with the one-launch pre-attention half: 1 = it "
                          "stores fp32 partial products that the attention launch reduces, "
                          "0 = it reduces them itself (default: the layer's own default)")
+    ap.add_argument("--layer-stack", action="store_true",
+                    help="layer workload: time the layer-stack form (the post-attention launch "
+                         "also computes the next step's QKV partial products; each step's input "
+                         "is the previous step's output)")
     ap.add_argument("--fused-post", type=int, choices=[0, 1], default=None,
                     help="layer workload: 1 = the post-attention half as one persistent launch, "
                          "0 = four launches (default: the layer's own default)")
@@ -341,6 +345,8 @@ class LayerRun:
             kw["fused_pre"] = bool(args.fused_pre)
         if args.split_pre is not None:
             kw["split_pre"] = bool(args.split_pre)
+        if args.layer_stack:
+            kw["layer_stack"] = True
         self.layer = DualFlowLayer(W, w.Hq, w.Hkv, w.D, w.F, w.B, w.cache_len + 1, device=dev,
                                    num_splits=args.num_splits, **kw)
         self.X = torch.cat([d["x1"], d["x2"]]).contiguous()
@@ -363,6 +369,10 @@ class LayerRun:
                                       if self.layer.fused_pre else "three launches",
                      "post_attention": "one persistent launch" if self.layer.fused_post
                                        else "four launches"}
+        if self.layer.layer_stack:
+            self.path["pre_attention"] = ("inside the previous step's post-attention launch "
+                                          "(layer-stack form: each step's input is the previous "
+                                          "step's output; e2e runs the three-launch step)")
         self.dominant = "dualflow_decode_attn (split kernel, combine inside it)"
 
     def step(self, timers=None):

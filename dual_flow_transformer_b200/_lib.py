@@ -121,6 +121,14 @@ SIGNATURES = {
         _c_float,                           # eps
         _vp, _vp, _vp,                      # x_mid, h, x_out
         _vp, _c_size, _vp, _vp]),           # workspace, bytes, err_flag, stream
+    "dualflow_layer_post_attention_qkv": (_c_int, [
+        _vp, _vp, _vp, _vp, _vp, _vp, _vp,  # attn, x, w_o, w_gu, w_down, b, c
+        _c_int, _c_int, _c_int, _c_int,     # m_primary, d_model, q_dim, F
+        _c_float,                           # eps
+        _vp, _vp, _vp,                      # x_mid, h, x_out
+        _vp, _c_size,                       # workspace, bytes
+        _vp, _c_int, _c_int, _c_int,        # w_qkv_next, Hq, Hkv, D
+        _vp, _vp, _vp, _vp]),               # part, ss_part, err_flag, stream
 }
 
 _lib = None

@@ -527,14 +527,20 @@ def new_post_attention_workspace(m_primary, d_model, q_dim, F, device="cuda"):
 
 
 def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=None, h=None,
-                         x_out=None, workspace=None, err_flag=None, stream=None):
+                         x_out=None, workspace=None, err_flag=None, stream=None,
+                         qkv_next=None):
     """x_mid = x + attn W_o^T; r = RMSNorm row scale of x_mid; h = SiLU(r
     x_mid W_gate^T) * (r x_mid W_up^T) (+ b coupling); x_out = x_mid + h
     W_down^T (+ c coupling), in one launch.
 
     attn: bf16 [2m, q_dim]; x: bf16 [2m, d_model] (primary rows first); w_o
     [d_model, q_dim], w_gu [2F, d_model], w_down [d_model, F]; b [F], c
-    [d_model] or None. Returns (x_out, x_mid, h)."""
+    [d_model] or None. Returns (x_out, x_mid, h).
+
+    qkv_next = (w_qkv, Hq, Hkv, D, part, ss_part): the same launch also
+    computes the next layer's QKV partial products of x_out into part fp32
+    [4, 2m, (Hq + 2 Hkv) D] and ss_part fp32 [4, 2m], as layer_qkv_partials
+    (x_out, w_qkv, ...) would (part bit for bit)."""
     M, q_dim = attn.shape
     d_model = x.shape[1]
     F = w_down.shape[1]
@@ -555,9 +561,27 @@ def layer_post_attention(attn, x, w_o, w_gu, w_down, b, c, *, eps=1e-5, x_mid=No
             raise ValueError("outputs must be contiguous")
     if workspace is None:
         workspace = new_post_attention_workspace(mp, d_model, q_dim, F, dev)
-    st = _lib().dualflow_layer_post_attention(
+    wbytes = workspace.numel() * workspace.element_size()
+    if qkv_next is None:
+        st = _lib().dualflow_layer_post_attention(
+            _ptr(attn), _ptr(x), _ptr(w_o), _ptr(w_gu), _ptr(w_down), _ptr(b), _ptr(c), mp,
+            d_model, q_dim, F, float(eps), _ptr(x_mid), _ptr(h), _ptr(x_out), _ptr(workspace),
+            wbytes, _ptr(err_flag), _stream(stream))
+        L.check("dualflow_layer_post_attention", st)
+        return x_out, x_mid, h
+    w_qkv, Hq, Hkv, D, part, ss_part = qkv_next
+    nout = (Hq + 2 * Hkv) * D
+    if not w_qkv.is_contiguous() or w_qkv.dtype != torch.bfloat16 or \
+            tuple(w_qkv.shape) != (nout, d_model):
+        raise ValueError("w_qkv must be bf16 [(Hq + 2 Hkv) D, d_model], contiguous")
+    if tuple(part.shape) != (4, M, nout) or tuple(ss_part.shape) != (4, M) or \
+            part.dtype != torch.float32 or ss_part.dtype != torch.float32 or \
+            not part.is_contiguous() or not ss_part.is_contiguous():
+        raise ValueError("part must be fp32 [4, 2m, N] and ss_part fp32 [4, 2m], contiguous")
+    st = _lib().dualflow_layer_post_attention_qkv(
         _ptr(attn), _ptr(x), _ptr(w_o), _ptr(w_gu), _ptr(w_down), _ptr(b), _ptr(c), mp, d_model,
-        q_dim, F, float(eps), _ptr(x_mid), _ptr(h), _ptr(x_out), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream))
-    L.check("dualflow_layer_post_attention", st)
+        q_dim, F, float(eps), _ptr(x_mid), _ptr(h), _ptr(x_out), _ptr(workspace), wbytes,
+        _ptr(w_qkv), int(Hq), int(Hkv), int(D), _ptr(part), _ptr(ss_part), _ptr(err_flag),
+        _stream(stream))
+    L.check("dualflow_layer_post_attention_qkv", st)
     return x_out, x_mid, h

@@ -114,12 +114,15 @@ static_assert(kRingLow % 1024 == 0 && kRingBytes % 1024 == 0 && kXBytes % 1024 =
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // grid counters: CTAs past P0 (x_mid and the sums of squares stored), past
-// P1 (h stored), done
-enum { kCntA2 = 0, kCntC = 1, kCntExit = 2 };
+// P1 (h stored), done, past P2 (x_out and its sums of squares stored; P3 only)
+enum { kCntA2 = 0, kCntC = 1, kCntExit = 2, kCntD = 3 };
 
 // Weight stages filled before counter A2 (gate/up) and C (W_down) is seen.
 constexpr int kEarlyGateUpStages = 4;
 constexpr int kEarlyDownStages = 7;
+// Weight stages of P3 filled before counter D is seen (the ones below the
+// receive buffer, which P2's reduction still uses).
+constexpr int kEarlyQkvStages = 4;
 
 struct Gemm {
   int units;    // P0 / P2: column tiles (one per cluster); P1: SwiGLU tiles
@@ -135,7 +138,7 @@ struct Gemm {
 struct Params {
   int M, mp, d, qd, F;
   float eps;
-  Gemm g[3];
+  Gemm g[4];  // P0 W_o, P1 W_gate / W_up, P2 W_down, P3 the next layer's W_qkv
   const __nv_bfloat16* x;
   const __nv_bfloat16* b;
   const __nv_bfloat16* c;
@@ -145,7 +148,13 @@ struct Params {
   float* ss_part;  // [d / 32 slices][128 rows] sums of squares of stored x_mid values
   int* cnt;        // [kCounters]
   int32_t* err;
-  int early[3];    // weight stages of phase q filled before its grid counter is complete
+  int early[4];    // weight stages of phase q filled before its grid counter is complete
+  // P3 (part != nullptr): rank r's fp32 partial product of x_out W_qkv^T over
+  // its K quarter, part[r][row][column] (nout columns), and ss_out[r][row],
+  // the sum of squares of the stored x_out row over that quarter
+  float* part;
+  float* ss_out;
+  int nout;
 };
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -389,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     post_kernel(const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
                 const __grid_constant__ CUtensorMap tmXg, const __grid_constant__ CUtensorMap tmWg,
                 const __grid_constant__ CUtensorMap tmXd, const __grid_constant__ CUtensorMap tmWd,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmXq, const __grid_constant__ CUtensorMap tmWq,
+                const __grid_constant__ CUtensorMap tmP, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -406,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* wfills = reinterpret_cast<int*>(recv_free + 1);  // [kMaxStages] fills per slot: weights
   int* xfills = wfills + kMaxStages;                     // [kMaxStages] activation tiles
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfills + kMaxStages);
-  // [0] abort, [1] epilogue broadcast, [2] / [3] counter A2 / C seen by the
-  // activation producer
+  // [0] abort, [1] epilogue broadcast, [2] / [3] / [4] counter A2 / C / D
+  // seen by the activation producer
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -433,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     flags[1] = 0;
     flags[2] = 0;
     flags[3] = 0;
+    flags[4] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -455,175 +466,197 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producers
     // warp 0: weights (may run ahead of the kernel launched before this one:
     // the weights are constants); warp 2: activation tiles.
-    if (lane == 0) {
-      const bool wrole = warp == 0;
-      if (wrole) {
-        prefetch_tensormap(&tmWo);
-        prefetch_tensormap(&tmWg);
-        prefetch_tensormap(&tmWd);
-      } else {
-        prefetch_tensormap(&tmXo);
-        prefetch_tensormap(&tmXg);
-        prefetch_tensormap(&tmXd);
-      }
-      const uint64_t pol = wrole ? l2_policy_evict_first() : l2_policy_evict_last();
-      int* fills = wrole ? wfills : xfills;
-      uint32_t par = 0;  // bit i: parity of this producer's fills of slot i
-      bool recv_ok = false;
-      bool ok = true;
-      for (int q = 0; q < 3 && ok; ++q) {
-        const Gemm& g = p.g[q];
-        const CUtensorMap* tm = wrole ? (q == 0 ? &tmWo : (q == 1 ? &tmWg : &tmWd))
-                                      : (q == 0 ? &tmXo : (q == 1 ? &tmXg : &tmXd));
-        // The ring changes its stage size at a phase boundary: every earlier
-        // fill of every slot must have been consumed first.
-        if (q > 0) {
-          for (int i = 0; i < kMaxStages && ok; ++i) {
-            if (!mbar_wait(&empty[i], ((par >> i) & 1u) ^ 1u)) {
-              set_err(p.err, DF_DEVERR_TIMEOUT);
-              flags[0] = 1;
-              ok = false;
-            }
+    const bool wrole = warp == 0;
+    const uint64_t pol = wrole ? l2_policy_evict_first() : l2_policy_evict_last();
+    int* fills = wrole ? wfills : xfills;
+    uint32_t par = 0;  // bit i: parity of this producer's fills of slot i
+    bool recv_ok = false;
+    bool ok = true;
+    const bool qkv = p.part != nullptr;  // phase P3: the next layer's QKV partials
+    // one phase's fills (lane 0)
+    auto fill_phase = [&](int q) {
+      const Gemm& g = p.g[q];
+      const CUtensorMap* tm =
+          wrole ? (q == 0 ? &tmWo : (q == 1 ? &tmWg : (q == 2 ? &tmWd : &tmWq)))
+                : (q == 0 ? &tmXo : (q == 1 ? &tmXg : (q == 2 ? &tmXd : &tmXq)));
+      // The ring changes its stage size at a phase boundary: every earlier
+      // fill of every slot must have been consumed first.
+      if (q > 0) {
+        for (int i = 0; i < kMaxStages && ok; ++i) {
+          if (!mbar_wait(&empty[i], ((par >> i) & 1u) ^ 1u)) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            flags[0] = 1;
+            ok = false;
           }
         }
-        int s = 0;
-        int fills_q = 0;  // this producer's fills in this phase
-        const Units us = units_of(g, q, cta, cid, G);
-        for (int u = us.first; u < g.units && ok; u += us.step) {
-          int k0, k1;
-          k_range(g, q, static_cast<int>(rank), k0, k1);
-          if (!wrole && q > 0 && k1 > k0) {
-            // P1 reads x_mid (counter A2), P2 every column of h (counter C)
-            if (!wait_count(p.cnt + (q == 1 ? kCntA2 : kCntC), G)) {
-              set_err(p.err, DF_DEVERR_TIMEOUT);
-              flags[0] = 1;
-              ok = false;
-              break;
-            }
-            fence_proxy_async_global();
-            flags[1 + q] = 1;  // counter A2 / C seen (see the weight producer)
+      }
+      int s = 0;
+      int fills_q = 0;  // this producer's fills in this phase
+      const Units us = units_of(g, q, cta, cid, G);
+      for (int u = us.first; u < g.units && ok; u += us.step) {
+        int k0, k1;
+        k_range(g, q, static_cast<int>(rank), k0, k1);
+        if (!wrole && q > 0 && k1 > k0) {
+          // P1 reads x_mid (counter A2), P2 every column of h (counter C),
+          // P3 x_out (counter D)
+          if (!wait_count(p.cnt + (q == 1 ? kCntA2 : (q == 2 ? kCntC : kCntD)), G)) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            flags[0] = 1;
+            ok = false;
+            break;
           }
-          for (int kb = k0; kb < k1 && ok; ++kb) {
-            if (wrole && q > 0 && fills_q == p.early[q]) {
-              // Weight traffic in flight delays the grid counter the phase's
-              // activations wait for: beyond p.early[q] stages, wait until
-              // the activation producer has seen it (counter A2 / C).
-              const long long t0 = clock64();
-              while (flags[1 + q] == 0 && !flags[0]) {
-                if (clock64() - t0 > kWaitLimitCycles) {
-                  set_err(p.err, DF_DEVERR_TIMEOUT);
-                  flags[0] = 1;
-                }
-                __nanosleep(64);
-              }
-              if (flags[0]) {
-                ok = false;
-                break;
-              }
-            }
-            if (!recv_ok && static_cast<size_t>(s + 1) * g.stage > kRingLow) {
-              // this slot reaches into the receive buffer: wait until this
-              // CTA's epilogue has consumed P0's received slices
-              if (!mbar_wait(recv_free, 0)) {
+          fence_proxy_async_global();
+          flags[1 + q] = 1;  // counter A2 / C / D seen (see the weight producer)
+        }
+        for (int kb = k0; kb < k1 && ok; ++kb) {
+          if (wrole && q > 0 && fills_q == p.early[q]) {
+            // Weight traffic in flight delays the grid counter the phase's
+            // activations wait for: beyond p.early[q] stages, wait until
+            // the activation producer has seen it (counter A2 / C / D).
+            const long long t0 = clock64();
+            while (flags[1 + q] == 0 && !flags[0]) {
+              if (clock64() - t0 > kWaitLimitCycles) {
                 set_err(p.err, DF_DEVERR_TIMEOUT);
                 flags[0] = 1;
-                ok = false;
-                break;
               }
-              recv_ok = true;
-            }
-            if (!mbar_wait(&empty[s], ((par >> s) & 1u) ^ 1u)) {
-              set_err(p.err, DF_DEVERR_TIMEOUT);
-              flags[0] = 1;
-              ok = false;
-              break;
+              __nanosleep(64);
             }
             if (flags[0]) {
               ok = false;
               break;
             }
-            uint8_t* st = smem + static_cast<size_t>(s) * g.stage;
-            if (wrole) {
-              mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(g.w_bytes));
-              if (q == 1) {
-                tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * g.half, pol);
-                tma_load_2d_hint(st + kXBytes + g.half * 128, tm, &full[s], kb * kBK,
-                                 p.F + u * g.half, pol);
-              } else {
-                tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * kTileN, pol);
-              }
-            } else {
-              mbar_arrive_expect_tx(&full[s], kXBytes);
-              tma_load_3d_hint(st, tm, &full[s], kb * kBK, 0, 0, pol);
-            }
-            ++fills[s];
-            ++fills_q;
-            par ^= 1u << s;
-            if (++s == g.nst) s = 0;
           }
+          if (!recv_ok && static_cast<size_t>(s + 1) * g.stage > kRingLow) {
+            // this slot reaches into the receive buffer: wait until this
+            // CTA's epilogue has consumed the received slices (P0's before
+            // P1, P2's before P3)
+            if (!mbar_wait(recv_free, q == 3 ? 1u : 0u)) {
+              set_err(p.err, DF_DEVERR_TIMEOUT);
+              flags[0] = 1;
+              ok = false;
+              break;
+            }
+            recv_ok = true;
+          }
+          if (!mbar_wait(&empty[s], ((par >> s) & 1u) ^ 1u)) {
+            set_err(p.err, DF_DEVERR_TIMEOUT);
+            flags[0] = 1;
+            ok = false;
+            break;
+          }
+          if (flags[0]) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + static_cast<size_t>(s) * g.stage;
+          if (wrole) {
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(g.w_bytes));
+            if (q == 1) {
+              tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * g.half, pol);
+              tma_load_2d_hint(st + kXBytes + g.half * 128, tm, &full[s], kb * kBK,
+                               p.F + u * g.half, pol);
+            } else {
+              tma_load_2d_hint(st + kXBytes, tm, &full[s], kb * kBK, u * g.BN, pol);
+            }
+          } else {
+            mbar_arrive_expect_tx(&full[s], kXBytes);
+            tma_load_3d_hint(st, tm, &full[s], kb * kBK, 0, 0, pol);
+          }
+          ++fills[s];
+          ++fills_q;
+          par ^= 1u << s;
+          if (++s == g.nst) s = 0;
         }
       }
-      if (wrole) pdl_trigger();
+        };
+    if (lane == 0) {
+      if (wrole) {
+        prefetch_tensormap(&tmWo);
+        prefetch_tensormap(&tmWg);
+        prefetch_tensormap(&tmWd);
+        if (qkv) prefetch_tensormap(&tmWq);
+      } else {
+        prefetch_tensormap(&tmXo);
+        prefetch_tensormap(&tmXg);
+        prefetch_tensormap(&tmXd);
+        if (qkv) prefetch_tensormap(&tmXq);
+      }
+      for (int q = 0; q < 3 && ok; ++q) fill_phase(q);
+      if (wrole && !qkv) pdl_trigger();
     }
     // P2's reduction may write into this CTA's ring once every role of every
     // rank is done with it (the epilogue meets this barrier after P2's MMAs)
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
+    if (lane == 0 && qkv) {
+      // P3: the low stages are free (every P2 MMA has completed); a stage
+      // that reaches into the receive buffer waits for P2's reduction
+      recv_ok = false;
+      if (ok) fill_phase(3);
+      if (wrole) pdl_trigger();
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t par = 0;  // bit i: parity of the next phase of full[i] to wait for
-      int seg = 0;
-      bool ok = true;
-      for (int q = 0; q < 3 && ok; ++q) {
-        const Gemm& g = p.g[q];
-        int s = 0;  // the producers restart the ring at every phase
-        const Units us = units_of(g, q, cta, cid, G);
-        for (int u = us.first; u < g.units && ok; u += us.step, ++seg) {
-          int k0, k1;
-          k_range(g, q, static_cast<int>(rank), k0, k1);
-          const int acc = seg & 1;
-          if (seg >= 2 &&
-              !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
+    uint32_t par = 0;  // bit i: parity of the next phase of full[i] to wait for
+    int seg = 0;
+    bool ok = true;
+    auto mma_phase = [&](int q) {
+      const Gemm& g = p.g[q];
+      int s = 0;  // the producers restart the ring at every phase
+      const Units us = units_of(g, q, cta, cid, G);
+      for (int u = us.first; u < g.units && ok; u += us.step, ++seg) {
+        int k0, k1;
+        k_range(g, q, static_cast<int>(rank), k0, k1);
+        const int acc = seg & 1;
+        if (seg >= 2 &&
+            !mbar_wait(&acc_empty[acc], static_cast<uint32_t>(((seg >> 1) - 1) & 1))) {
+          set_err(p.err, DF_DEVERR_TIMEOUT);
+          flags[0] = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = k0; kb < k1; ++kb) {
+          if (!mbar_wait(&full[s], (par >> s) & 1u) || flags[0]) {
             set_err(p.err, DF_DEVERR_TIMEOUT);
             flags[0] = 1;
             ok = false;
             break;
           }
+          par ^= 1u << s;
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-          for (int kb = k0; kb < k1; ++kb) {
-            if (!mbar_wait(&full[s], (par >> s) & 1u) || flags[0]) {
-              set_err(p.err, DF_DEVERR_TIMEOUT);
-              flags[0] = 1;
-              ok = false;
-              break;
-            }
-            par ^= 1u << s;
-            tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * g.stage);
-            const uint32_t b_addr = a_addr + kXBytes;
+          const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * g.stage);
+          const uint32_t b_addr = a_addr + kXBytes;
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              umma_bf16(d_tmem, smem_desc(a_addr + kk * 32), smem_desc(b_addr + kk * 32), g.idesc,
-                        (kb > k0 || kk > 0) ? 1u : 0u);
-            umma_commit(&empty[s]);
-            if (++s == g.nst) s = 0;
-          }
-          if (!ok) break;
-          // (a unit without k-blocks commits at once: its partial is zero)
-          umma_commit(&acc_full[acc]);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16(d_tmem, smem_desc(a_addr + kk * 32), smem_desc(b_addr + kk * 32), g.idesc,
+                      (kb > k0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+          if (++s == g.nst) s = 0;
         }
+        if (!ok) break;
+        // (a unit without k-blocks commits at once: its partial is zero)
+        umma_commit(&acc_full[acc]);
       }
+    };
+    if (lane == 0) {
+      for (int q = 0; q < 3 && ok; ++q) mma_phase(q);
       // no tensor-core operation may still be reading shared memory or TMEM
-      // when the CTA leaves (this commit completes after every MMA above)
+      // when the ring retires or the CTA leaves (this commit completes after
+      // every MMA above)
       umma_commit(mma_done);
       mbar_wait(mma_done, 0);
     }
     tc_fence_before();
     cluster_sync();  // the ring retires (see the producers)
     tc_fence_after();
+    if (lane == 0 && p.part != nullptr) {
+      if (ok) mma_phase(3);
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 1);
+    }
   } else {
     // ------------------------------------------------------------ epilogue warps
     // Two warps per TMEM lane quarter (warps q + 3 and q + 7 take quarter
@@ -793,10 +826,91 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < kHalfN; ++i) sum[i] += res[i];
+          if (p.part != nullptr) {
+            // P3 reads x_out and needs its rows' sums of squares: per
+            // 32-column slice, over the stored (bf16) values, as for x_mid
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < kHalfN; ++i) {
+              sum[i] = __bfloat162float(__float2bfloat16_rn(sum[i]));
+              ss = fmaf(sum[i], sum[i], ss);
+            }
+            if (half == 1) red[tl] = ss;
+            epi_bar<kEpiThreads>();
+            if (half == 0 && live)
+              p.ss_part[static_cast<size_t>(cid * kCluster + static_cast<int>(rank)) * kBM + row] =
+                  ss + red[tl];
+          }
           if (live) store_bf16<kHalfN>(p.x_out + static_cast<size_t>(row) * p.d + col0, sum);
         }
       }
       ++seg;
+    }
+    if (p.part != nullptr) {
+      // P3: the next layer's QKV partial products over x_out (the rows'
+      // sums of squares of each K quarter from the slices above)
+      ok = epi_bar_and<kEpiThreads>(ok);
+      if (et == 0) mbar_arrive(recv_free);  // P2's received slices are consumed
+      arrive_count(p.cnt + kCntD, et);
+      if (ok && cid < p.g[3].units) {
+        const int acc = seg & 1;
+        int k0, k1;
+        k_range(p.g[3], 3, static_cast<int>(rank), k0, k1);
+        float ssq = 0.f;
+        if (cid == 0) {
+          // cluster 0 stores ss_out: this half's slices of the quarter in
+          // slice order, then the two halves added in a fixed order
+          if (!grid_wait(kCntD)) {
+            ok = false;
+          } else {
+            const int per = p.d / kSliceN / kCluster;  // slices per K quarter
+            const int k_first = static_cast<int>(rank) * per + half * (per / 2);
+            if (live)
+              for (int k = 0; k < per / 2; ++k)
+                ssq += __ldcg(p.ss_part + static_cast<size_t>(k_first + k) * kBM + row);
+            if (half == 1) red[tl] = ssq;
+            epi_bar<kEpiThreads>();
+            if (half == 0) ssq += red[tl];
+          }
+        }
+        if (ok && !take_acc(acc, seg)) fail();
+        if (ok) {
+          tc_fence_after();
+          // this thread's half of the tile, in boxes of 32 columns (128-byte
+          // swizzle), staged in the retired ring at the output row: every
+          // MMA of this CTA has completed, and no other rank writes here
+          const int nbox = p.g[3].BN / 32;
+          for (int j = half * (nbox / 2); j < (half + 1) * (nbox / 2); ++j) {
+            float v[32];
+            if (k1 == k0) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            } else {
+              tmem_ld<32>(acc_addr(acc) + 32 * j, v);
+            }
+            if (live) {
+              uint8_t* box = smem + static_cast<size_t>(j) * (kBM * 128) + row * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<float4*>(box + ((c ^ (row & 7)) * 16)) =
+                    make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+          }
+          give_acc(acc);
+          if (cid == 0 && half == 0 && live)
+            p.ss_out[static_cast<size_t>(rank) * p.M + row] = ssq;
+          fence_proxy_async_smem();  // the generic writes above -> the TMA stores' reads
+          epi_bar<kEpiThreads>();
+          if (et == 0) {
+            for (int j = 0; j < nbox; ++j)
+              tma_store_3d(&tmP, smem + static_cast<size_t>(j) * (kBM * 128),
+                           cid * p.g[3].BN + 32 * j, 0, static_cast<int>(rank));
+            bulk_commit_group();
+            bulk_wait_all();
+          }
+        }
+        ++seg;
+      }
     }
   }
 
@@ -918,22 +1032,27 @@ size_t ws_bytes(int d) {
   return kCounterBytes + static_cast<size_t>(d / kSliceN) * kBM * 4;
 }
 
-}  // namespace post
-}  // namespace df
-
-extern "C" size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model,
-                                                               int q_dim, int F) {
-  const df::post::Plan pl = df::post::make_plan(2 * m_primary, m_primary, d_model, q_dim, F);
-  return pl.ok ? df::post::ws_bytes(d_model) : 0;
+// P3's column tile: the narrowest multiple of 64 (at most 256) that divides
+// nout with at most one tile per cluster (0: none fits).
+int qkv_tile(int nout, int d, int clusters) {
+  if (d % (kSliceN * kCluster * 2) != 0) return 0;  // whole slices per half quarter
+  for (int tn = 64; tn <= 256; tn += 64)
+    if (nout % tn == 0 && nout / tn <= clusters) return tn;
+  return 0;
 }
 
-extern "C" df_status dualflow_layer_post_attention(
-    const void* attn, const void* x, const void* w_o, const void* w_gu, const void* w_down,
-    const void* b, const void* c, int m_primary, int d_model, int q_dim, int F, float eps,
-    void* x_mid, void* h, void* x_out, void* workspace, size_t workspace_bytes,
-    int32_t* err_flag, void* stream) {
-  using namespace df;
-  using namespace df::post;
+struct QkvNext {  // P3's operands (w == nullptr: no P3)
+  const void* w;
+  int nout;
+  void* part;
+  void* ss_out;
+};
+
+df_status launch_post(const void* attn, const void* x, const void* w_o, const void* w_gu,
+                      const void* w_down, const void* b, const void* c, int m_primary,
+                      int d_model, int q_dim, int F, float eps, void* x_mid, void* h,
+                      void* x_out, void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                      const QkvNext& nx, void* stream) {
   if (!attn || !x || !w_o || !w_gu || !w_down || !x_mid || !h || !x_out)
     return DF_ERR_NULL;
   if (m_primary < 1 || d_model < 1 || q_dim < 1 || F < 1 || !(eps >= 0.f)) return DF_ERR_SHAPE;
@@ -946,6 +1065,14 @@ extern "C" df_status dualflow_layer_post_attention(
   if ((b && !aligned(b, 16)) || (c && !aligned(c, 16))) return DF_ERR_ALIGN;
   if (!workspace || workspace_bytes < ws_bytes(d_model) || !aligned(workspace, 256))
     return DF_ERR_WORKSPACE;
+  int tn3 = 0;
+  if (nx.w != nullptr) {
+    if (!nx.part || !nx.ss_out) return DF_ERR_NULL;
+    if (!aligned(nx.w, 16) || !aligned(nx.part, 16) || !aligned(nx.ss_out, 16))
+      return DF_ERR_ALIGN;
+    tn3 = qkv_tile(nx.nout, d_model, pl.G / kCluster);
+    if (tn3 == 0) return DF_ERR_UNSUPPORTED;
+  }
 
   Params p{};
   p.M = M;
@@ -970,6 +1097,13 @@ extern "C" df_status dualflow_layer_post_attention(
   p.early[0] = 0;                    // (P0 waits for no counter)
   p.early[1] = kEarlyGateUpStages;
   p.early[2] = kEarlyDownStages;
+  if (tn3 > 0) {
+    p.g[3] = ring_gemm(nx.nout / tn3, d_model / kBK, tn3, 0, kRingBytes);
+    p.early[3] = kEarlyQkvStages;
+    p.part = static_cast<float*>(nx.part);
+    p.ss_out = static_cast<float*>(nx.ss_out);
+    p.nout = nx.nout;
+  }
 
   CUtensorMap tmXo, tmWo, tmXg, tmWg, tmXd, tmWd;
   const uint64_t du = static_cast<uint64_t>(d_model),
@@ -991,6 +1125,19 @@ extern "C" df_status dualflow_layer_post_attention(
       !x_map(&tmXd, h, Fu) ||
       !encode_tmap_bf16_2d(&tmWd, w_down, du, Fu, Fu * 2, kTileN, kBK))
     return DF_ERR_CUDA;
+  CUtensorMap tmXq = tmXo, tmWq = tmWo, tmP = tmXo;  // (unused without P3)
+  if (tn3 > 0) {
+    // P3: x_out interleaved like the other activations; the partials
+    // [rank][row][column] fp32 stored in boxes of 32 columns x 128 rows
+    const uint64_t nout = static_cast<uint64_t>(nx.nout), Mu = static_cast<uint64_t>(M);
+    const uint64_t dims[3] = {nout, Mu, kCluster};
+    const uint64_t strides[2] = {nout * 4, Mu * nout * 4};
+    const uint32_t box[3] = {32, kBM, 1};
+    if (!x_map(&tmXq, x_out, du) ||
+        !encode_tmap_bf16_2d(&tmWq, nx.w, nout, du, du * 2, static_cast<uint32_t>(tn3), kBK) ||
+        !encode_tmap_f32_3d_box(&tmP, nx.part, dims, strides, box))
+      return DF_ERR_CUDA;
+  }
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.G);
@@ -1006,7 +1153,42 @@ extern "C" df_status dualflow_layer_post_attention(
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, post_kernel, tmXo, tmWo, tmXg, tmWg, tmXd, tmWd, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, post_kernel, tmXo, tmWo, tmXg, tmWg, tmXd, tmWd, tmXq, tmWq, tmP,
+                         p) != cudaSuccess)
     return DF_ERR_CUDA;
   return DF_OK;
+}
+
+}  // namespace post
+}  // namespace df
+
+extern "C" size_t dualflow_layer_post_attention_workspace_size(int m_primary, int d_model,
+                                                               int q_dim, int F) {
+  const df::post::Plan pl = df::post::make_plan(2 * m_primary, m_primary, d_model, q_dim, F);
+  return pl.ok ? df::post::ws_bytes(d_model) : 0;
+}
+
+extern "C" df_status dualflow_layer_post_attention(
+    const void* attn, const void* x, const void* w_o, const void* w_gu, const void* w_down,
+    const void* b, const void* c, int m_primary, int d_model, int q_dim, int F, float eps,
+    void* x_mid, void* h, void* x_out, void* workspace, size_t workspace_bytes,
+    int32_t* err_flag, void* stream) {
+  const df::post::QkvNext none{nullptr, 0, nullptr, nullptr};
+  return df::post::launch_post(attn, x, w_o, w_gu, w_down, b, c, m_primary, d_model, q_dim, F,
+                               eps, x_mid, h, x_out, workspace, workspace_bytes, err_flag, none,
+                               stream);
+}
+
+extern "C" df_status dualflow_layer_post_attention_qkv(
+    const void* attn, const void* x, const void* w_o, const void* w_gu, const void* w_down,
+    const void* b, const void* c, int m_primary, int d_model, int q_dim, int F, float eps,
+    void* x_mid, void* h, void* x_out, void* workspace, size_t workspace_bytes,
+    const void* w_qkv_next, int Hq, int Hkv, int D, void* part, void* ss_part,
+    int32_t* err_flag, void* stream) {
+  if (!w_qkv_next) return DF_ERR_NULL;
+  if (Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv != 0 || q_dim != Hq * D) return DF_ERR_SHAPE;
+  const df::post::QkvNext nx{w_qkv_next, (Hq + 2 * Hkv) * D, part, ss_part};
+  return df::post::launch_post(attn, x, w_o, w_gu, w_down, b, c, m_primary, d_model, q_dim, F,
+                               eps, x_mid, h, x_out, workspace, workspace_bytes, err_flag, nx,
+                               stream);
 }

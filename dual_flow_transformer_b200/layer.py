@@ -53,7 +53,8 @@ from . import api
 
 class DualFlowLayer:
     def __init__(self, weights, Hq, Hkv, D, F, B, max_seqlen, device="cuda", eps=1e-5,
-                 num_splits=0, fused_pre=True, fused_post=True, split_pre=True):
+                 num_splits=0, fused_pre=True, fused_post=True, split_pre=True,
+                 layer_stack=False):
         self.w = weights  # dict of device tensors: w_qkv, w_o, w_gu, w_down, a, b, c
         self.Hq, self.Hkv, self.D, self.F, self.B = Hq, Hkv, D, F, B
         self.d_model = weights["w_o"].shape[0]
@@ -102,6 +103,18 @@ class DualFlowLayer:
         pre_launches = 1 if self.fused_pre else \
             2 + api.grouped_proj_num_launches(M, *weights["w_qkv"].shape, "none")
         self._launches = pre_launches + self.attn_launches + post_launches
+        # Layer-stack form of the captured step: the post-attention launch
+        # also computes the NEXT step's QKV partial products from x_out, as
+        # in a stack of layers where each output is the next one's input;
+        # captured steps then alternate between two buffers (x_in -> x_alt
+        # -> x_in ...), one launch fewer per step.
+        self.layer_stack = bool(layer_stack)
+        if self.layer_stack:
+            if not (self.split_pre and self.fused_post):
+                raise ValueError("the layer-stack form needs the split pre-attention and the "
+                                 "fused post-attention launches")
+            self.x_alt = torch.empty(M, self.d_model, dtype=bf, device=dev)
+            self._launches = self.attn_launches + 1
 
     @property
     def launches_per_step(self) -> int:
@@ -134,11 +147,65 @@ class DualFlowLayer:
                 self._step_part(part, *args)
             self.graphs.append(g)
         torch.cuda.synchronize()
+        if self.layer_stack:
+            # the partials of X, then one eager step each way; two graphs
+            # (X -> x_alt, x_alt -> X), and for the timers the attention and
+            # the post-attention launch X -> x_alt
+            w = self.w
+            x_save = X.clone()
+            api.layer_qkv_partials(X, w["w_qkv"], self.Hq, self.Hkv, self.D, part=self.qkv_part,
+                                   ss_part=self.ss_part, err_flag=self.err)
+            self._stack_step(X, self.x_alt, args)
+            self._stack_step(self.x_alt, X, args)
+            torch.cuda.synchronize()
+            self.stack_graphs = []
+            for src, dst in ((X, self.x_alt), (self.x_alt, X)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    self._stack_step(src, dst, args)
+                self.stack_graphs.append(g)
+            self.stack_post = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.stack_post):
+                self._stack_post(X, self.x_alt)
+            # back to X and its partials: the first replay is the step on X
+            X.copy_(x_save)
+            api.layer_qkv_partials(X, w["w_qkv"], self.Hq, self.Hkv, self.D, part=self.qkv_part,
+                                   ss_part=self.ss_part, err_flag=self.err)
+            self._stack_next = 0
+            torch.cuda.synchronize()
+
+    def _stack_post(self, X, x_out, stream=None):
+        w = self.w
+        api.layer_post_attention(self.attn, X, w["w_o"], w["w_gu"], w["w_down"], w["b"], w["c"],
+                                 eps=self.eps, x_mid=self.x_mid, h=self.h, x_out=x_out,
+                                 workspace=self.post_ws, err_flag=self.err, stream=stream,
+                                 qkv_next=(w["w_qkv"], self.Hq, self.Hkv, self.D,
+                                           self.qkv_part, self.ss_part))
+
+    def _stack_step(self, X, x_out, args, stream=None):
+        """Layer-stack step: attention over the partials the previous step
+        left, then the post-attention launch X -> x_out with the next QKV."""
+        self._step_part("attn", *args, stream=stream)
+        self._stack_post(X, x_out, stream=stream)
 
     def replay(self, timers=None):
         """One captured step on the current stream: the single-graph step, or
         with timers ({"attn": (start_event, end_event)}) the three-graph step
-        with the events recorded around the attention."""
+        with the events recorded around the attention. In the layer-stack form
+        the steps alternate X -> x_alt -> X ... (each step's input is the
+        previous output; returns the buffer just written); with timers, the
+        attention and the post-attention launch X -> x_alt."""
+        if self.layer_stack:
+            if timers is None:
+                i = self._stack_next
+                self.stack_graphs[i].replay()
+                self._stack_next = 1 - i
+                return self.x_alt if i == 0 else self._graph_args[0]
+            timers["attn"][0].record()
+            self.graphs[1].replay()
+            timers["attn"][1].record()
+            self.stack_post.replay()
+            return self.x_alt
         if timers is None:
             self.graph_full.replay()
             return self.x_out
@@ -225,7 +292,10 @@ class DualFlowLayer:
         step and copies the layer output back, all queued on the stream."""
         self.x_in.copy_(x_host, non_blocking=True)
         if getattr(self, "graphs", None) and self._graph_args[0] is self.x_in:
-            out = self.replay()
+            # (a new input has no partials from a previous step: the whole
+            # three-launch step, also in the layer-stack form)
+            self.graph_full.replay()
+            out = self.x_out
         else:
             out = self.step(self.x_in, k_cache, v_cache, block_table, positions, seqlens,
                             stream=stream)

@@ -536,6 +536,41 @@ df_status dualflow_layer_post_attention(const void* attn, const void* x, const v
                                         int32_t* err_flag, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* The same launch followed by the NEXT layer's grouped QKV projection of    */
+/* x_out, left as partial products (the layer-stack form).                   */
+/*                                                                           */
+/* Pages "Sintesi Tecnica" ("Architettura Core", "Costi di Inferenza"): in a */
+/* stack of layers the next layer's first step reads this layer's output;    */
+/* computing it inside this launch lets its weight stream follow W_down's    */
+/* through the same pipeline instead of waiting for a new launch. Outputs    */
+/* x_mid, h, x_out exactly as dualflow_layer_post_attention (bit for bit),   */
+/* and, as dualflow_layer_qkv_partials(x_out, w_qkv_next, ...) would:        */
+/*   part[r][row][col] = sum over k in K quarter r of x_out[row][k]           */
+/*                       w_qkv_next[col][k]    (fp32, the same MMA order, so  */
+/*                       bit for bit equal to that call's)                    */
+/*   ss_part[r][row]   = sum over the same k of x_out[row][k]^2 (fp32; other  */
+/*                       summation order: equal within fp32 rounding)         */
+/* for r = 0..3, all M rows (auxiliary rows' K / V columns included, unused), */
+/* col < (Hq + 2 Hkv) D. These feed dualflow_decode_attn_qkv_partials (parts */
+/* = 4) of the next layer, which applies that layer's RMSNorm.                */
+/* w_qkv_next: bf16 [(Hq + 2 Hkv) D][d_model]; part: fp32 [4][M][(Hq + 2 Hkv)*/
+/* D]; ss_part: fp32 [4][M]; all 16-byte aligned, written by the launch and   */
+/* read by the next launch on the stream. w_qkv_next is read before the wait  */
+/* for the kernel launched ahead (like the other weights).                    */
+/* Errors: NULL w_qkv_next / part / ss_part: DF_ERR_NULL; q_dim != Hq * D or */
+/* Hq % Hkv != 0: DF_ERR_SHAPE; (Hq + 2 Hkv) D without a divisor among 64,   */
+/* 128, 192, 256 giving at most one column tile per 4-CTA cluster, or        */
+/* d_model % 256 != 0: DF_ERR_UNSUPPORTED; else as above. One kernel launch; */
+/* the same workspace.                                                        */
+/* ------------------------------------------------------------------------ */
+df_status dualflow_layer_post_attention_qkv(
+    const void* attn, const void* x, const void* w_o, const void* w_gu, const void* w_down,
+    const void* b, const void* c, int m_primary, int d_model, int q_dim, int F, float eps,
+    void* x_mid, void* h, void* x_out, void* workspace, size_t workspace_bytes,
+    const void* w_qkv_next, int Hq, int Hkv, int D, void* part, void* ss_part,
+    int32_t* err_flag, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* MoE MLP block with router replay.                                         */
 /*                                                                           */
 /* Page "Sintesi Tecnica: Dual-Flow Transformers", section "Meccanismi        */

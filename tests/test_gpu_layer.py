@@ -115,3 +115,38 @@ def test_layer_step_full_size_sampled(cuda_device, mode):
     got = torch.cat([out[rows], out[[B + r for r in rows]]])
     assert_close(got, ref["x_out"], "bf16",
                  "full layer x_out (17 seq, %s)" % mode)
+
+
+def test_layer_stack_steps_chain_like_standard_steps(cuda_device):
+    """Layer-stack form (the post-attention launch also computes the next
+    step's QKV partial products from x_out): two replays from X equal two
+    standard steps chained through their output, the first bit for bit (the
+    same partials), the second within the bf16 tolerance (the partial
+    products are equal bit for bit, the RMSNorm sums of squares are added in
+    another order)."""
+    inp = synth.make_layer_inputs(SMALL)
+    d_std, d_st = to_dev(inp, cuda_device), to_dev(inp, cuda_device)
+    w = {k: d_std[k] for k in ("w_qkv", "w_o", "w_gu", "w_down", "a", "b", "c")}
+    B, L = inp["B"], int(inp["positions"].max()) + 1
+    X0 = torch.cat([d_std["x1"], d_std["x2"]]).contiguous()
+    seqlens = (d_std["positions"] + 1).to(torch.int32)
+
+    std = DualFlowLayer(w, inp["Hq"], inp["Hkv"], inp["D"], inp["F"], B, L, device=cuda_device)
+    a = (d_std["k_cache"], d_std["v_cache"], d_std["block_table"], d_std["positions"], seqlens)
+    out1 = std.step(X0.clone(), *a).clone()
+    out2 = std.step(out1.clone(), *a).clone()
+
+    st = DualFlowLayer(w, inp["Hq"], inp["Hkv"], inp["D"], inp["F"], B, L, device=cuda_device,
+                       layer_stack=True)
+    assert st.launches_per_step == st.attn_launches + 1
+    st.x_in.copy_(X0)
+    b = (d_st["k_cache"], d_st["v_cache"], d_st["block_table"], d_st["positions"], seqlens)
+    st.capture(st.x_in, *b)
+    assert torch.equal(st.x_in, X0)
+    got1 = st.replay().clone()
+    got2 = st.replay().clone()
+    torch.cuda.synchronize()
+    assert int(st.err.item()) == 0 and int(std.err.item()) == 0
+    assert torch.equal(got1, out1)
+    assert_close(got2.float().cpu().numpy(), out2.float().cpu().numpy(), "bf16",
+                 "layer-stack second step")
