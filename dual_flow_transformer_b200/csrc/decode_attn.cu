@@ -152,10 +152,13 @@ __device__ __forceinline__ float max_nan(float a, float b) { return (a != a || a
 // Normalise; an empty row (no attended token) gives 0, a NaN row stays NaN.
 __device__ __forceinline__ float safe_div(float o, float l) { return (l == 0.f) ? 0.f : o / l; }
 
-__device__ __forceinline__ int attended_len(const Params& p, int b) {
-  const int L = p.seqlens[b];
+__device__ __forceinline__ int clamp_len(const Params& p, int L) {
   if (L < 1) return 0;
   return L < p.max_seqlen ? L : p.max_seqlen;
+}
+
+__device__ __forceinline__ int attended_len(const Params& p, int b) {
+  return clamp_len(p, p.seqlens[b]);
 }
 
 __device__ __forceinline__ void flag_len(const Params& p, int b) {
@@ -224,10 +227,39 @@ __global__ void __launch_bounds__(kThreads, 2)
   __nv_bfloat16* q1s = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * kStageBytes + 128);
   __nv_bfloat16* q2s = q1s + 4 * D;  // partials mode: this KV head's Q1 / Q2raw rows
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
+
+  // Longest sequences first: with one CTA per (sequence, KV head) and ragged
+  // lengths, the CTAs are issued roughly in blockIdx order, so a long
+  // sequence that comes late sets the tail. Grid row z takes the sequence
+  // of rank z by descending length (ties in index order: a uniform batch
+  // keeps its order), ranked by every CTA from the lengths in shared memory
+  // (the one load of them replaces the load of its own length).
+  int b = blockIdx.z;
+  int len_b = -1;  // seqlens[b], when already loaded
+  if (p.qpart == nullptr && gridDim.x == 1 && p.B > 1 && p.B <= kThreads) {
+    __shared__ int s_len[kThreads];
+    __shared__ int s_b;
+    const int t = threadIdx.x;
+    if (t < p.B) s_len[t] = p.seqlens[t];
+    __syncthreads();
+    if (t < p.B) {
+      const int Lt = s_len[t];
+      int rank = 0;
+#pragma unroll 8
+      for (int j = 0; j < p.B; ++j) {
+        const int Lj = s_len[j];
+        rank += (Lj > Lt || (Lj == Lt && j < t)) ? 1 : 0;
+      }
+      if (rank == static_cast<int>(blockIdx.z)) s_b = t;
+    }
+    __syncthreads();
+    b = s_b;
+    len_b = s_len[b];
+  }
 
   // Partials mode: the query rows' partial products and row sums of squares
   // are loaded first (one L2 round trip, overlapping the set-up below);
@@ -250,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   if (split == 0 && g == 0 && threadIdx.x == 0) flag_len(p, b);
-  const int L = attended_len(p, b);
+  const int L = len_b >= 0 ? clamp_len(p, len_b) : attended_len(p, b);
   const int npages = (L + kPage - 1) / kPage;
   const int pg0 = split * p.chunk_pages;
   const int pg1 = min(npages, pg0 + p.chunk_pages);
