@@ -244,20 +244,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ int s_len[kThreads];
     __shared__ int s_b;
     const int t = threadIdx.x;
-    if (t < p.B) s_len[t] = p.seqlens[t];
-    __syncthreads();
-    if (t < p.B) {
-      const int Lt = s_len[t];
-      int rank = 0;
+    const int Lt = t < p.B ? p.seqlens[t] : 0;
+    const int L0 = p.seqlens[0];
+    if (t < p.B) s_len[t] = Lt;
+    // (a uniform batch keeps its order: no ranking)
+    if (!__syncthreads_and(t >= p.B || Lt == L0)) {
+      if (t < p.B) {
+        int rank = 0;
 #pragma unroll 8
-      for (int j = 0; j < p.B; ++j) {
-        const int Lj = s_len[j];
-        rank += (Lj > Lt || (Lj == Lt && j < t)) ? 1 : 0;
+        for (int j = 0; j < p.B; ++j) {
+          const int Lj = s_len[j];
+          rank += (Lj > Lt || (Lj == Lt && j < t)) ? 1 : 0;
+        }
+        if (rank == static_cast<int>(blockIdx.z)) s_b = t;
       }
-      if (rank == static_cast<int>(blockIdx.z)) s_b = t;
+      __syncthreads();
+      b = s_b;
     }
-    __syncthreads();
-    b = s_b;
     len_b = s_len[b];
   }
 

@@ -286,3 +286,26 @@ def test_tiny_workload_reported(cuda_device):
                                 inp["block_table"].numpy(), inp["seqlens"].numpy())
     assert_attn_close(o1, r1, "fp32", "full tiny O1")
     assert_attn_close(o2, r2, "fp32", "full tiny O2")
+
+
+@pytest.mark.parametrize("num_splits", [0, 1])
+def test_permuting_the_batch_permutes_the_outputs(cuda_device, num_splits):
+    """Every sequence's outputs depend on that sequence alone, whatever order
+    the grid takes the sequences in (unsplit plans take them longest first,
+    ties in index order): the batch reversed gives the outputs reversed, bit
+    for bit. Ragged lengths with ties; 40 sequences x 8 KV heads = 320 units,
+    one CTA each in the automatic plan."""
+    w = _small("gqa", B=40, Hq=16, Hkv=8, len_lo=64, len_hi=700, seed=31)
+    lengths = [300, 64, 700, 300, 65, 700, 128, 1, 511, 300] * 4
+    inp = synth.make_attn_inputs(w, lengths=lengths)
+    perm = torch.arange(len(lengths) - 1, -1, -1)
+    rev = dict(inp)
+    for k in ("q1", "q2raw", "block_table", "seqlens"):
+        rev[k] = inp[k][perm].contiguous()
+    o1, o2 = _run(inp, cuda_device, num_splits=num_splits)
+    r1, r2 = _run(rev, cuda_device, num_splits=num_splits)
+    dev_perm = perm.to(cuda_device)
+    assert torch.equal(r1, o1[dev_perm]) and torch.equal(r2, o2[dev_perm])
+    r1o, r2o = oracle_attn(inp)
+    assert_attn_close(o1, r1o, "bf16", "permuted batch o1")
+    assert_attn_close(o2, r2o, "bf16", "permuted batch o2")
