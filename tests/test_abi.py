@@ -303,3 +303,21 @@ def test_selftest_and_split_pre_entries_reject_invalid_arguments(lib):
     assert attn(m=0) == L.DF_ERR_SHAPE
     assert attn(eps=-1.0) == L.DF_ERR_SHAPE
     assert attn(part=buf + 4) == L.DF_ERR_ALIGN
+
+
+def test_post_attention_qkv_entry_rejects_invalid_arguments(lib):
+    """The layer-stack entry's own checks (before the post-attention launch's
+    and before any CUDA call): the next layer's W_qkv is required, and the
+    head layout must match the attention width."""
+    buf = 4096
+
+    def call(w_qkv=buf, Hq=4, Hkv=2, D=128, q_dim=512):
+        return lib.dualflow_layer_post_attention_qkv(
+            buf, buf, buf, buf, buf, None, None, 8, 512, q_dim, 1024, 1e-5, buf, buf, buf, buf,
+            1 << 20, w_qkv, Hq, Hkv, D, buf, buf, None, None)
+
+    assert call(w_qkv=None) == L.DF_ERR_NULL
+    assert call(Hq=0) == L.DF_ERR_SHAPE
+    assert call(Hkv=3) == L.DF_ERR_SHAPE        # Hq % Hkv != 0
+    assert call(q_dim=256) == L.DF_ERR_SHAPE    # q_dim != Hq * D
+    assert call(D=0) == L.DF_ERR_SHAPE
