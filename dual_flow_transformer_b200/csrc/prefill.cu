@@ -14,8 +14,8 @@
 //  1. append_kernel: token t of sequence b goes to cache position
 //     ctx_lens[b] + (t - cu_seqlens[b]) (one CTA per token, 16-byte copies);
 //  2. causal flash attention of the chunk's primary queries over the cache
-//     (prefix + chunk): tc::pair_kernel on the tcgen05 tensor cores (D = 128,
-//     at least 128 token rows, 16-byte aligned output rows; described at the
+//     (prefix + chunk): tc::pair_kernel on the tcgen05 tensor cores (D = 64
+//     or 128, at least 128 token rows, 16-byte aligned output rows; described at the
 //     kernel), otherwise attn_kernel: one CTA per (query head, 64-row tile,
 //     sequence), heads fastest so that the CTAs sharing a KV head run side by
 //     side and meet its pages in L2; tiles of one sequence are issued longest
@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ------------------------------------------------------------------ 2'. attention, tcgen05
 //
-// The same computation on the 5th-generation tensor cores, for D = 128, over
+// The same computation on the 5th-generation tensor cores, for D = 64 or 128, over
 // key blocks of 128 tokens (two cache pages): S = Q K^T (M 128, N 128) into
 // TMEM, the softmax warps write P as bf16 into TMEM, and O += P V takes P
 // from TMEM as its A operand. pair_kernel (described at its definition) holds
@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   using Lay = PairLayout<D>;
   constexpr int H = D / 64;
   constexpr float kNegInf = -INFINITY;
-  static_assert(D == 128, "the two-tile prefill kernel is built for head_dim 128");
+  static_assert(D == 64 || D == 128, "the two-tile prefill kernel is built for head_dim 64 / 128");
   static_assert(PairLayout<D>::kSmem <= 227 * 1024, "shared memory budget");
 
   extern __shared__ uint8_t smem_raw[];
@@ -1093,17 +1093,24 @@ cudaError_t launch_attn(const AttnParams& p, int Hq, int B, const CUtensorMap* t
 
 // Two query heads of one KV group per CTA when the group has an even number
 // of heads (both tiles then read the same pages), else one head per CTA.
-cudaError_t launch_attn_tc(AttnParams p, int Hq, int B, const CUtensorMap* tmQ,
-                           const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
-  constexpr size_t smem2 = tc::PairLayout<128>::kSmem;
-  cudaError_t e2 = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::pair_kernel<128>), smem2);
+template <int D>
+cudaError_t launch_pair(AttnParams p, int Hq, int B, const CUtensorMap* tmQ,
+                        const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
+  constexpr size_t smem2 = tc::PairLayout<D>::kSmem;
+  cudaError_t e2 = ensure_dynamic_smem(reinterpret_cast<const void*>(tc::pair_kernel<D>), smem2);
   if (e2 != cudaSuccess) return e2;
   // two query heads of a KV group per CTA when the group has an even number
   // of heads, else two consecutive row tiles of one head
   p.pair_rows = p.G % 2 == 0 ? 0 : 1;
   const dim3 grid = p.pair_rows ? dim3(Hq, (p.tiles + 1) / 2, B) : dim3(Hq / 2, p.tiles, B);
-  return launch_pdl(tc::pair_kernel<128>, grid, dim3(tc::kPairThreads), smem2, stream, *tmQ, *tmK,
+  return launch_pdl(tc::pair_kernel<D>, grid, dim3(tc::kPairThreads), smem2, stream, *tmQ, *tmK,
                     *tmV, p);
+}
+
+cudaError_t launch_attn_tc(AttnParams p, int Hq, int B, int D, const CUtensorMap* tmQ,
+                           const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
+  return D == 64 ? launch_pair<64>(p, Hq, B, tmQ, tmK, tmV, stream)
+                 : launch_pair<128>(p, Hq, B, tmQ, tmK, tmV, stream);
 }
 
 // Workspace of the auxiliary step: the decode workspace (its arrival counters
@@ -1135,11 +1142,12 @@ extern "C" int dualflow_prefill_num_launches(int with_append, int with_aux) {
   return (with_append ? 1 : 0) + 1 + (with_aux ? 2 : 0);
 }
 
-// The tcgen05 attention kernel serves D = 128 with at least one full tile of
-// token rows and 16-byte aligned output rows; anything else takes the
+// The tcgen05 attention kernel serves D = 64 and 128 with at least one full
+// tile of token rows and 16-byte aligned output rows; anything else takes the
 // mma.sync kernel.
 static bool tc_kernel_fits(int D, int T, const void* o1, int64_t o_stride_t) {
-  return D == 128 && T >= df::prefill::tc::kRows && df::aligned(o1, 16) && o_stride_t % 8 == 0;
+  return (D == 64 || D == 128) && T >= df::prefill::tc::kRows && df::aligned(o1, 16) &&
+         o_stride_t % 8 == 0;
 }
 
 extern "C" int dualflow_prefill_kernel(int D, int T, const void* o1, int64_t o_stride_t, int Hq) {
@@ -1253,7 +1261,7 @@ extern "C" df_status dualflow_prefill_ex(
     if (!encode_tmap_bf16_2d(&tmQ, q1, static_cast<uint64_t>(T), static_cast<uint64_t>(Hq) * D,
                              static_cast<uint64_t>(qs) * 2, tc::kRows, 64))
       return DF_ERR_CUDA;
-    e = launch_attn_tc(p, Hq, B, &tmQ, &tmK, &tmV, st);
+    e = launch_attn_tc(p, Hq, B, D, &tmQ, &tmK, &tmV, st);
   } else {
     e = (D == 64) ? launch_attn<64>(p, Hq, B, &tmK, &tmV, st)
                   : launch_attn<128>(p, Hq, B, &tmK, &tmV, st);

@@ -264,7 +264,7 @@ size_t dualflow_prefill_workspace_size(int B, int Hq, int Hkv, int D, int max_se
                                        int block_size);
 /* Attention kernel of a prefill call. DF_PREFILL_KERNEL_TCGEN05: tensor    */
 /* cores with TMEM accumulators, 128-row tiles; used (automatically) when    */
-/* D = 128, T >= 128, o1 is 16-byte aligned and o_stride_t % 8 == 0.          */
+/* D = 64 or 128, T >= 128, o1 is 16-byte aligned and o_stride_t % 8 == 0.   */
 /* DF_PREFILL_KERNEL_MMA_SYNC: warp-level mma.sync, 64-row tiles, any        */
 /* supported shape. Both compute the same result within the tolerance; the   */
 /* cache write and the auxiliary step are the same code.                     */

@@ -71,6 +71,7 @@ KERNELS = ["mma_sync", "tcgen05"]
 @pytest.mark.parametrize("Hq,Hkv,D,lengths,ctx", [
     (8, 2, 128, (1, 63, 65, 200), (0, 37, 64, 130)),   # ragged chunks, prefixes, tile edges
     (16, 4, 64, (130, 7), (0, 0)),                     # D 64, 4 query heads per KV head
+    (8, 2, 64, (300, 129, 1), (40, 0, 7)),             # D 64: row tiles, prefixes, one token
     (4, 4, 128, (256, 129), (0, 0)),                   # MHA, fresh prompts
     (6, 2, 128, (64, 128, 191), (1, 63, 0)),           # G = 3
     (8, 2, 128, (127, 128, 129, 300), (0, 5, 200, 64)),  # 128-row tile edges
@@ -81,8 +82,6 @@ KERNELS = ["mma_sync", "tcgen05"]
     (3, 1, 128, (200, 260, 385), (0, 130, 0)),         # G = 3, 4 row tiles (last: 1 row)
 ])
 def test_prefill_matches_oracle(cuda_device, Hq, Hkv, D, lengths, ctx, kernel):
-    if kernel == "tcgen05" and D != 128:
-        pytest.skip("the tcgen05 prefill kernel is built for head_dim 128")
     inp = synth.make_prefill_inputs(_w(Hq=Hq, Hkv=Hkv, D=D), lengths=lengths, ctx=ctx)
     d = _dev(inp, cuda_device)
     o1, o2 = _run(d, kernel=kernel)
@@ -92,7 +91,9 @@ def test_prefill_matches_oracle(cuda_device, Hq, Hkv, D, lengths, ctx, kernel):
 def test_automatic_kernel_choice(cuda_device):
     o1 = torch.empty((256, 8, 128), dtype=torch.bfloat16, device=cuda_device)
     assert api.prefill_kernel(128, 256, o1, 8) == "tcgen05"
-    assert api.prefill_kernel(64, 256, o1[:, :, :64], 8) == "mma_sync"
+    assert api.prefill_kernel(64, 256, o1[:, :, :64], 8) == "tcgen05"
+    assert api.prefill_kernel(64, 100, o1[:100, :, :64], 8) == "mma_sync"
+    assert api.prefill_kernel(96, 256, o1[:, :, :96], 8) == "mma_sync"
     assert api.prefill_kernel(128, 100, o1[:100], 8) == "mma_sync"
 
 
