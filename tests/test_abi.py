@@ -271,12 +271,13 @@ def test_prefill_kernel_choice_is_checked(lib):
                                        FAKE, None, 256, 400, o1, 0, None, 2, T, 8, 2, D, 64, 16,
                                        0.0, L.DF_BF16, kernel, None, 0, None, None)
     assert ex(7) == L.DF_ERR_SHAPE
-    assert ex(L.DF_PREFILL_KERNEL_TCGEN05, D=64) == L.DF_ERR_UNSUPPORTED
     assert ex(L.DF_PREFILL_KERNEL_TCGEN05, T=100, o1=FAKE) == L.DF_ERR_SHAPE  # max_q_len > T
     assert ex(L.DF_PREFILL_KERNEL_TCGEN05, o1=FAKE + 4) == L.DF_ERR_UNSUPPORTED
     assert lib.dualflow_prefill_kernel(128, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_TCGEN05
     assert lib.dualflow_prefill_kernel(128, 100, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
-    assert lib.dualflow_prefill_kernel(64, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
+    assert lib.dualflow_prefill_kernel(64, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_TCGEN05
+    assert lib.dualflow_prefill_kernel(64, 100, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
+    assert lib.dualflow_prefill_kernel(96, 300, FAKE, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
     assert lib.dualflow_prefill_kernel(128, 300, FAKE + 4, 0, 8) == L.DF_PREFILL_KERNEL_MMA_SYNC
 
 
