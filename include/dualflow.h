@@ -235,7 +235,10 @@ df_status dualflow_kv_append(const void* k_new, const void* v_new, int64_t new_s
 /*  3. if q2raw and o2 are given: O2[b,h] = the decode step's auxiliary      */
 /*     output for the last position P = ctx_lens[b] + n_b - 1, i.e. Q2 =     */
 /*     q2raw[b] + a (.) q1[last row of b] over positions j <= P (computed by */
-/*     the decode attention kernel in auxiliary-only mode).                  */
+/*     the decode attention kernel in auxiliary-only mode, with its own     */
+/*     split plan; when ctx_lens is NULL and T = B max_q_len, i.e. every     */
+/*     chunk has max_q_len tokens, with the split count that fills one wave  */
+/*     of 2 CTAs per SM, capped by that plan).                               */
 /*                                                                           */
 /* q1        : bf16 [T][Hq][D], token row t at q1 + t*q_stride_t elements    */
 /*             (0 = Hq*D); 16-byte aligned, q_stride_t % 8 == 0.              */

@@ -124,6 +124,40 @@ def test_aux_output_is_the_decode_step_of_the_last_position(cuda_device):
     assert_attn_close(o1[last.to(cuda_device)], r1[last.numpy()], "bf16", "prefill O1 last rows")
 
 
+def test_uniform_batch_aux_step_takes_one_wave_of_splits(cuda_device):
+    """Fresh prompts of one length without ctx_lens: the auxiliary step runs
+    the decode kernel with the split count that fills one wave (2 CTAs per
+    SM, capped by the decode plan), so it equals that decode call bit for
+    bit, and the oracle's decode step within the tolerance. 16 prompts x 8
+    KV heads = 128 units of 2600 tokens: the plan's 5 splits against 2."""
+    B, Hkv, n = 16, 8, 2600
+    inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=Hkv, D=64), lengths=(n,) * B, ctx=(0,) * B)
+    d = _dev(inp, cuda_device)
+    o1, o2 = api.prefill(d["q1"], d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
+                         d["block_table"], d["cu_seqlens"], inp["max_q_len"], inp["max_seqlen"],
+                         q2raw=d["q2raw"], a=d["a"])
+    plan = api.decode_attn_num_splits(B, Hkv, inp["max_seqlen"])
+    splits = min(plan, 296 // (B * Hkv))
+    assert plan > splits >= 1
+    last = (inp["cu_seqlens"][1:] - 1).long()
+    seqlens = torch.full((B,), n, dtype=torch.int32, device=cuda_device)
+    q_last = d["q1"][last.to(cuda_device)].contiguous()
+    _, d2 = api.decode_attn(q_last, d["q2raw"], d["a"], d["k_cache"], d["v_cache"],
+                            d["block_table"], seqlens, inp["max_seqlen"], num_splits=splits)
+    torch.cuda.synchronize()
+    assert torch.equal(d2, o2)
+    cu = inp["cu_seqlens"].tolist()
+    scale = 1.0 / math.sqrt(64)
+    for b in (0, 7, 15):
+        q2 = oracle.couple_query(f32(inp["q1"][cu[b + 1] - 1])[None], f32(inp["q2raw"][b])[None],
+                                 f32(inp["a"]))[0]
+        for h in (0, 5):
+            K = f32(inp["k_new"][cu[b]:cu[b + 1], h])
+            V = f32(inp["v_new"][cu[b]:cu[b + 1], h])
+            ref = oracle.attn_weights(q2[h][None], K, scale) @ V
+            assert_attn_close(o2[b, h][None], ref, "bf16", "uniform batch O2 b=%d h=%d" % (b, h))
+
+
 def test_primary_output_ignores_aux_inputs_even_nan(cuda_device):
     inp = synth.make_prefill_inputs(_w(Hq=8, Hkv=2), lengths=(100, 33), ctx=(5, 0))
     d = _dev(inp, cuda_device)
