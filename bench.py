@@ -711,6 +711,9 @@ class PrefillRun:
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         lens = (h["cu_seqlens"][1:] - h["cu_seqlens"][:-1]).tolist()
         ctx = h["ctx_lens"].tolist()
+        # fresh prompts (no cached prefix) are passed as the API's "no
+        # prefix" (ctx_lens = None), as a caller of a fresh prefill would
+        self.fresh = all(c == 0 for c in ctx)
         pairs = sum(n * c + n * (n + 1) // 2 for n, c in zip(lens, ctx))
         self.tokens_per_step = h["T"]
         self.launches_per_step = api.prefill_num_launches(True, True)
@@ -736,7 +739,8 @@ class PrefillRun:
         d = self.d
         self.api.prefill(d["q1"], d["k_new"] if append else None, d["v_new"] if append else None,
                          d["k_cache"], d["v_cache"], d["block_table"], d["cu_seqlens"],
-                         d["max_q_len"], d["max_seqlen"], ctx_lens=d["ctx_lens"],
+                         d["max_q_len"], d["max_seqlen"],
+                         ctx_lens=None if self.fresh else d["ctx_lens"],
                          q2raw=d["q2raw"] if aux else None, a=d["a"] if aux else None,
                          o1=self.o1, o2=self.o2 if aux else None, workspace=self.ws,
                          err_flag=self.err)
